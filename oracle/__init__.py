@@ -1,0 +1,195 @@
+"""CPU oracle for selection-driven block-sparse causal attention (fp64).
+
+TEST INFRASTRUCTURE ONLY. Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this package. It shares no code with
+the CUDA path and never imports it; the CUDA path never imports this.
+
+The arithmetic lives in ``spa_oracle.c`` (plain C loops, fp64, OpenMP over
+independent units); this module only compiles it with gcc and marshals numpy
+arrays. Each function cites the passage it follows in its C counterpart.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "spa_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle_spa.so")
+_lib = None
+_lock = threading.Lock()
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_D = ctypes.c_double
+_I64 = ctypes.c_int64
+
+
+def build(force: bool = False) -> str:
+    """Compile ``spa_oracle.c`` into ``liboracle_spa.so`` (gcc, fp64, no fast-math)."""
+    if (not force and os.path.exists(_LIB_PATH)
+            and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC)):
+        return _LIB_PATH
+    tmp = _LIB_PATH + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", "-ffp-contract=off",
+           "-fno-fast-math", "-Wall", "-Wextra", _SRC, "-o", tmp, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _bind(path: str):
+    lib = ctypes.CDLL(path)
+    lib.oracle_num_threads.restype = _I
+    lib.oracle_block_stats.argtypes = [_P, _I, _I, _I, _I, _I, _I, _P, _P]
+    lib.oracle_scores.argtypes = [_P, _I, _P, _P, _I, _I, _I, _I, _I, _I, _I, _D, _P]
+    lib.oracle_select_from_scores.argtypes = [_P, _I, _I, _I, _I, _I, _D, _I, _I, _I,
+                                              _P, _I, _P]
+    lib.oracle_attention.argtypes = [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I,
+                                     _P, _I, _P, _D, _P, _I64, _P, _P]
+    for f in ("oracle_block_stats", "oracle_scores", "oracle_select_from_scores",
+              "oracle_attention"):
+        getattr(lib, f).restype = _I
+    return lib
+
+
+def use_library(path: str | None):
+    """Point this module at another build of the oracle (``None``: the default).
+
+    Used by the mutation tests, which compile deliberately broken copies of the
+    oracle source to show that the pins catch them.
+    """
+    global _lib
+    with _lock:
+        _lib = _bind(path) if path else None
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            _lib = _bind(build())
+    return _lib
+
+
+def num_threads() -> int:
+    """Threads the oracle's parallel loops use (OpenMP's default team size)."""
+    return int(_load().oracle_num_threads())
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _inp(x: np.ndarray, dtype: str) -> tuple[np.ndarray, int]:
+    if dtype == "bf16":
+        return np.ascontiguousarray(x, dtype=np.uint16), 1
+    if dtype == "f32":
+        return np.ascontiguousarray(x, dtype=np.float32), 0
+    raise ValueError(dtype)
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise RuntimeError(f"oracle {what} failed with code {rc}")
+
+
+def block_stats(k: np.ndarray, dtype: str, block: int):
+    """Per-block key mean and population variance (fp64). k: [B,Hkv,T,d]."""
+    k, isb = _inp(k, dtype)
+    B, Hkv, T, d = k.shape
+    nb = -(-T // block)
+    mean = np.empty((B, Hkv, nb, d), np.float64)
+    var = np.empty_like(mean)
+    _check(_load().oracle_block_stats(_ptr(k), isb, B, Hkv, T, d, block, _ptr(mean), _ptr(var)),
+           "block_stats")
+    return mean, var
+
+
+def scores(q: np.ndarray, dtype: str, mean: np.ndarray, var: np.ndarray, T: int, block: int,
+           scale: float) -> np.ndarray:
+    """Log Taylor block scores [B,Hq,nq,nb] (fp64); -inf beyond the causal limit."""
+    q, isb = _inp(q, dtype)
+    B, Hq, Lq, d = q.shape
+    Hkv = mean.shape[1]
+    nb = -(-T // block)
+    nq = -(-Lq // block)
+    mean = np.ascontiguousarray(mean, np.float64)
+    var = np.ascontiguousarray(var, np.float64)
+    l = np.empty((B, Hq, nq, nb), np.float64)
+    _check(_load().oracle_scores(_ptr(q), isb, _ptr(mean), _ptr(var), B, Hq, Hkv, Lq, T, d,
+                                 block, float(scale), _ptr(l)), "scores")
+    return l
+
+
+def select_from_scores(l: np.ndarray, Lq: int, T: int, block: int, top_p: float, n_sink: int = 1,
+                       n_local: int = 1, k_min: int = 0, cap: int | None = None):
+    """Dual top-p cut over given log scores. Returns (idx [B,Hq,nq,cap] int32, count int32)."""
+    l = np.ascontiguousarray(l, np.float64)
+    B, Hq, nq, nb = l.shape
+    cap = nb if cap is None else cap
+    idx = np.empty((B, Hq, nq, cap), np.int32)
+    count = np.empty((B, Hq, nq), np.int32)
+    _check(_load().oracle_select_from_scores(_ptr(l), B, Hq, Lq, T, block, float(top_p), n_sink,
+                                             n_local, k_min, _ptr(idx), cap, _ptr(count)),
+           "select")
+    return idx, count
+
+
+def select(q, k, dtype: str, block: int, scale: float, top_p: float, n_sink: int = 1,
+           n_local: int = 1, k_min: int = 0, cap: int | None = None):
+    """Stats -> pooled scores -> cut. Returns dict(mean, var, scores, idx, count)."""
+    mean, var = block_stats(k, dtype, block)
+    T = k.shape[2]
+    l = scores(q, dtype, mean, var, T, block, scale)
+    idx, count = select_from_scores(l, q.shape[2], T, block, top_p, n_sink, n_local, k_min, cap)
+    return {"mean": mean, "var": var, "scores": l, "idx": idx, "count": count}
+
+
+def attention(q, k, v, dtype: str, block: int, idx: np.ndarray, count: np.ndarray, scale: float,
+              rows: np.ndarray | None = None):
+    """Masked dense softmax attention (fp64), all rows or the flat row ids ``rows``.
+
+    Returns (out, lse): out [B,Hq,Lq,d] (or [len(rows), d]), lse likewise without d.
+    """
+    q, isb = _inp(q, dtype)
+    k, _ = _inp(k, dtype)
+    v, _ = _inp(v, dtype)
+    B, Hq, Lq, d = q.shape
+    Hkv, T = k.shape[1], k.shape[2]
+    idx = np.ascontiguousarray(idx, np.int32)
+    count = np.ascontiguousarray(count, np.int32)
+    cap = idx.shape[-1]
+    if rows is None:
+        n = B * Hq * Lq
+        out = np.empty((B, Hq, Lq, d), np.float64)
+        lse = np.empty((B, Hq, Lq), np.float64)
+        rp = None
+    else:
+        rows = np.ascontiguousarray(rows, np.int64)
+        n = rows.size
+        out = np.empty((n, d), np.float64)
+        lse = np.empty((n,), np.float64)
+        rp = _ptr(rows)
+    _check(_load().oracle_attention(_ptr(q), _ptr(k), _ptr(v), isb, B, Hq, Hkv, Lq, T, d, block,
+                                    _ptr(idx), cap, _ptr(count), float(scale), rp, n, _ptr(out),
+                                    _ptr(lse)), "attention")
+    return out, lse
+
+
+def full_lists(B: int, Hq: int, Lq: int, T: int, block: int):
+    """Kept lists that keep every causal block (dense causal attention)."""
+    nb = -(-T // block)
+    nq = -(-Lq // block)
+    idx = np.full((B, Hq, nq, nb), -1, np.int32)
+    count = np.empty((B, Hq, nq), np.int32)
+    for i in range(nq):
+        last_row = min((i + 1) * block, Lq)
+        jmax = (T - Lq + last_row - 1) // block
+        idx[:, :, i, :jmax + 1] = np.arange(jmax + 1, dtype=np.int32)
+        count[:, :, i] = jmax + 1
+    return idx, count

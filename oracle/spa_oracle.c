@@ -1,0 +1,371 @@
+/*
+ * CPU oracle for selection-driven block-sparse causal attention.
+ *
+ * TEST INFRASTRUCTURE ONLY. This file is the plain, slow, fp64 statement of what
+ * the CUDA path computes. Only the tests, the smoke check and the benchmark's CPU
+ * baseline leg may load it; the library path never does. It shares no code with
+ * the CUDA sources and includes none of their headers.
+ *
+ * Sources (the pages are web summaries of five papers on block-sparse attention):
+ *   - "SPLA - Block Sparse Plus Linear Attention for Long Context Modeling",
+ *     section 2.1: block relevance = integrated attention mass of the block's
+ *     tokens, approximated by a second-order Taylor expansion about the block
+ *     mean: exp(q.kbar) * (1 + 1/2 q^T Cov(k) q), with Cov(k) taken diagonal.
+ *   - "SpotAttention", section 3 (dual top-p rule): a sink prefix and a recency
+ *     suffix are always kept; nucleus (top-p) selection runs over the residual
+ *     blocks and stops once the cumulative mass reaches p; K_min is a floor.
+ *   - "Sparsere Blok-Sparse Attention via Tokenpermutatie" (PBS-Attn), sections
+ *     3-4: block importance from mean-pooled queries.
+ *   - "S2O", section 3: exact attention over the selected key tiles with the
+ *     online-softmax state (m, l, acc). The oracle does not use online softmax: it
+ *     builds the token mask and evaluates the textbook masked softmax per row.
+ *
+ * Readings where the pages are silent (each applies to one function below):
+ *   - the Taylor score is expanded with the attention's own scale s, i.e.
+ *     exp(s q.kbar)(1 + s^2/2 q^T diag(var) q), times the token count n_j of the
+ *     block (the block mass is a sum over its tokens);
+ *   - the variance is the population variance (divide by n_j);
+ *   - one pooled query per query block: the mean of the block's query rows;
+ *   - top-p is normalised over the residual (non-reserved) candidates only; a block
+ *     is kept while the mass accumulated before it is below p, so the block that
+ *     crosses p is kept; p >= 1 keeps the whole residual; equal scores order by
+ *     the smaller block index;
+ *   - the cut is decided on fp32 scores (the kernel's precision): the fp64 score is
+ *     rounded to fp32 first; masses and their prefix sums are fp64.
+ *
+ * Inputs are fp32 arrays or bf16 bit patterns (uint16); bf16 widens to fp32
+ * exactly, and all arithmetic below is fp64.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORACLE_OK 0
+#define ORACLE_EINVAL 1
+#define ORACLE_ENOMEM 2
+
+static double elem(const void *x, int is_bf16, size_t i)
+{
+    if (is_bf16) {
+        uint32_t u = (uint32_t)((const uint16_t *)x)[i] << 16;
+        float f;
+        memcpy(&f, &u, sizeof f);
+        return (double)f;
+    }
+    return (double)((const float *)x)[i];
+}
+
+static int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/*
+ * Block statistics (SPLA, section 2.1): for every (b, kv-head g, block j)
+ *   kbar_j[c] = (1/n_j) sum_{t in block j} k_t[c]
+ *   var_j[c]  = (1/n_j) sum_{t in block j} (k_t[c] - kbar_j[c])^2
+ * two passes over the block; n_j = block, except a shorter last block.
+ * k: [B, Hkv, T, d]; mean, var: [B, Hkv, nb, d].
+ */
+int oracle_block_stats(const void *k, int k_bf16, int B, int Hkv, int T, int d, int block,
+                       double *mean, double *var)
+{
+    if (B <= 0 || Hkv <= 0 || T <= 0 || d <= 0 || block <= 0) return ORACLE_EINVAL;
+    const int nb = ceil_div(T, block);
+    const long units = (long)B * Hkv * nb;
+#pragma omp parallel for schedule(static)
+    for (long u = 0; u < units; ++u) {
+        const long bg = u / nb;
+        const int j = (int)(u % nb);
+        const int t0 = j * block;
+        const int n = (T - t0 < block) ? (T - t0) : block;
+        const size_t base = ((size_t)bg * T + t0) * d;
+        double *mu = mean + (size_t)u * d;
+        double *vr = var + (size_t)u * d;
+        for (int c = 0; c < d; ++c) {
+            double s = 0.0;
+            for (int t = 0; t < n; ++t) s += elem(k, k_bf16, base + (size_t)t * d + c);
+            mu[c] = s / n;
+        }
+        for (int c = 0; c < d; ++c) {
+            double s = 0.0;
+            for (int t = 0; t < n; ++t) {
+                double x = elem(k, k_bf16, base + (size_t)t * d + c) - mu[c];
+                s += x * x;
+            }
+            vr[c] = s / n;
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* Last key block a query block may see: queries occupy the last Lq positions. */
+static int last_candidate(int i, int Lq, int T, int block)
+{
+    int last_row = (i + 1) * block < Lq ? (i + 1) * block : Lq;   /* exclusive */
+    int last_pos = T - Lq + last_row - 1;
+    return last_pos / block;
+}
+
+/*
+ * Log block scores (SPLA, section 2.1, with the pooled query of PBS-Attn):
+ *   qbar_i = mean of the query rows of query block i
+ *   l[b,h,i,j] = s qbar_i . kbar_j + log(1 + s^2/2 sum_c qbar_i[c]^2 var_j[c]) + log n_j
+ * which is the log of n_j exp(s qbar.kbar)(1 + s^2/2 qbar^T diag(var) qbar).
+ * Query head h reads kv-head h / (Hq/Hkv). Candidates j > jmax(i) get -inf.
+ * q: [B, Hq, Lq, d] with Lq == T (prefill) or Lq == 1 (decode: the query at T-1).
+ * l: [B, Hq, nq, nb].
+ */
+int oracle_scores(const void *q, int q_bf16, const double *mean, const double *var,
+                  int B, int Hq, int Hkv, int Lq, int T, int d, int block, double scale,
+                  double *l)
+{
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || T <= 0 || d <= 0 || block <= 0)
+        return ORACLE_EINVAL;
+    if (!(Lq == T || Lq == 1)) return ORACLE_EINVAL;
+    const int nb = ceil_div(T, block), nq = ceil_div(Lq, block), G = Hq / Hkv;
+    const long units = (long)B * Hq * nq;
+    int err = 0;
+#pragma omp parallel
+    {
+        double *qbar = (double *)malloc(sizeof(double) * d);
+        if (!qbar) {
+#pragma omp atomic write
+            err = 1;
+        }
+#pragma omp for schedule(dynamic, 16)
+        for (long u = 0; u < units; ++u) {
+            if (!qbar) continue;
+            const long bh = u / nq;
+            const int i = (int)(u % nq);
+            const int b = (int)(bh / Hq), h = (int)(bh % Hq), g = h / G;
+            const int r0 = i * block;
+            const int nr = (Lq - r0 < block) ? (Lq - r0) : block;
+            for (int c = 0; c < d; ++c) {
+                double s = 0.0;
+                for (int r = 0; r < nr; ++r) s += elem(q, q_bf16, ((size_t)bh * Lq + r0 + r) * d + c);
+                qbar[c] = s / nr;
+            }
+            const int jmax = last_candidate(i, Lq, T, block);
+            double *lrow = l + (size_t)u * nb;
+            for (int j = 0; j < nb; ++j) {
+                if (j > jmax) { lrow[j] = -INFINITY; continue; }
+                const double *mu = mean + (((size_t)b * Hkv + g) * nb + j) * d;
+                const double *vr = var + (((size_t)b * Hkv + g) * nb + j) * d;
+                double dot = 0.0, quad = 0.0;
+                for (int c = 0; c < d; ++c) {
+                    dot += qbar[c] * mu[c];
+                    quad += qbar[c] * qbar[c] * vr[c];
+                }
+                const int nj = (T - j * block < block) ? (T - j * block) : block;
+                lrow[j] = scale * dot + log1p(0.5 * scale * scale * quad) + log((double)nj);
+            }
+        }
+        free(qbar);
+    }
+    return err ? ORACLE_ENOMEM : ORACLE_OK;
+}
+
+typedef struct { float key; int j; } cand_t;
+
+/* Descending key; equal keys: smaller block index first. */
+static int cand_cmp(const void *a, const void *b)
+{
+    const cand_t *x = (const cand_t *)a, *y = (const cand_t *)b;
+    if (x->key > y->key) return -1;
+    if (x->key < y->key) return 1;
+    return (x->j > y->j) - (x->j < y->j);
+}
+
+/*
+ * Dual top-p cut (SpotAttention, section 3) on one score row.
+ *   reserved = {0 .. n_sink-1} U {jmax-n_local+1 .. jmax}, within [0, jmax]
+ *   residual R = [0, jmax] minus reserved
+ *   masses over R: w_j = exp(l_j - max_R l) / sum_R exp(l - max_R l)
+ *   R sorted by score, descending; a block is kept while the mass accumulated
+ *   before it is below p (p >= 1 keeps all of R); then at least min(k_min, |R|)
+ *   blocks are kept. Output: reserved U kept, ascending; returns the count.
+ * The decision uses fp32 keys (the fp64 score rounded to fp32); masses are fp64.
+ * Returns -1 on allocation failure or when cap is too small.
+ */
+static int cut_row(const double *lrow, int jmax, double top_p, int n_sink, int n_local,
+                   int k_min, int32_t *out, int cap, cand_t *cand, unsigned char *keep)
+{
+    int nr = 0;
+    for (int j = 0; j <= jmax; ++j) {
+        int rsv = (j < n_sink) || (j > jmax - n_local);
+        keep[j] = (unsigned char)rsv;
+        if (!rsv) {
+            cand[nr].key = (float)lrow[j];
+            cand[nr].j = j;
+            ++nr;
+        }
+    }
+    if (nr > 0) {
+        qsort(cand, (size_t)nr, sizeof(cand_t), cand_cmp);
+        int nk;
+        if (top_p >= 1.0) {
+            nk = nr;
+        } else {
+            const double mx = (double)cand[0].key;
+            double total = 0.0;
+            for (int k = 0; k < nr; ++k) total += exp((double)cand[k].key - mx);
+            double cum = 0.0;
+            nk = 0;
+            for (int k = 0; k < nr; ++k) {
+                if (!(cum / total < top_p)) break;
+                cum += exp((double)cand[k].key - mx);
+                ++nk;
+            }
+        }
+        int floor_k = k_min < nr ? k_min : nr;
+        if (nk < floor_k) nk = floor_k;
+        for (int k = 0; k < nk; ++k) keep[cand[k].j] = 1;
+    }
+    int cnt = 0;
+    for (int j = 0; j <= jmax; ++j) {
+        if (!keep[j]) continue;
+        if (cnt >= cap) return -1;
+        out[cnt++] = j;
+    }
+    return cnt;
+}
+
+/*
+ * Selection from given log scores l: [B, Hq, nq, nb] -> idx [B, Hq, nq, cap]
+ * (ascending, unused tail set to -1) and count [B, Hq, nq].
+ */
+int oracle_select_from_scores(const double *l, int B, int Hq, int Lq, int T, int block,
+                              double top_p, int n_sink, int n_local, int k_min,
+                              int32_t *idx, int cap, int32_t *count)
+{
+    if (B <= 0 || Hq <= 0 || T <= 0 || block <= 0 || !(Lq == T || Lq == 1)) return ORACLE_EINVAL;
+    if (!(top_p > 0.0) || n_sink < 0 || n_local < 0 || k_min < 0) return ORACLE_EINVAL;
+    const int nb = ceil_div(T, block), nq = ceil_div(Lq, block);
+    if (cap < nb) return ORACLE_EINVAL;
+    const long units = (long)B * Hq * nq;
+    int err = 0;
+#pragma omp parallel
+    {
+        cand_t *cand = (cand_t *)malloc(sizeof(cand_t) * nb);
+        unsigned char *keep = (unsigned char *)malloc((size_t)nb);
+        if (!cand || !keep) {
+#pragma omp atomic write
+            err = ORACLE_ENOMEM;
+        }
+#pragma omp for schedule(dynamic, 16)
+        for (long u = 0; u < units; ++u) {
+            if (!cand || !keep) continue;
+            const int i = (int)(u % nq);
+            int32_t *out = idx + (size_t)u * cap;
+            for (int c = 0; c < cap; ++c) out[c] = -1;
+            int cnt = cut_row(l + (size_t)u * nb, last_candidate(i, Lq, T, block), top_p,
+                              n_sink, n_local, k_min, out, cap, cand, keep);
+            if (cnt < 0) {
+#pragma omp atomic write
+                err = ORACLE_EINVAL;
+                cnt = 0;
+            }
+            count[u] = cnt;
+        }
+        free(cand);
+        free(keep);
+    }
+    return err;
+}
+
+/*
+ * Masked dense softmax attention, row by row (the textbook form; no online
+ * softmax). For query row t of (b, h) at position pos = T - Lq + t, in query block
+ * i = t / block, the allowed keys are
+ *   M[t, u] = (u <= pos) and (block(u) is in the kept list of (b, h, i));
+ *   z_u = s q_t . k_u on allowed keys, -inf elsewhere;
+ *   o_t = sum_u softmax(z)_u v_u,  lse_t = log sum_u exp(z_u).
+ * A row with no allowed key gets o = 0 and lse = -inf.
+ * rows: flat row ids r = (b*Hq + h)*Lq + t, or NULL for every row in order.
+ * out: [nrows, d]; lse: [nrows] (may be NULL).
+ */
+int oracle_attention(const void *q, const void *k, const void *v, int is_bf16,
+                     int B, int Hq, int Hkv, int Lq, int T, int d, int block,
+                     const int32_t *idx, int cap, const int32_t *count, double scale,
+                     const int64_t *rows, int64_t nrows, double *out, double *lse)
+{
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || T <= 0 || d <= 0 || block <= 0)
+        return ORACLE_EINVAL;
+    if (!(Lq == T || Lq == 1)) return ORACLE_EINVAL;
+    const int nb = ceil_div(T, block), nq = ceil_div(Lq, block), G = Hq / Hkv;
+    if (cap < 1) return ORACLE_EINVAL;
+    if (!rows) nrows = (int64_t)B * Hq * Lq;
+    int err = 0;
+#pragma omp parallel
+    {
+        unsigned char *kept = (unsigned char *)malloc((size_t)nb);
+        double *z = (double *)malloc(sizeof(double) * T);
+        if (!kept || !z) {
+#pragma omp atomic write
+            err = ORACLE_ENOMEM;
+        }
+#pragma omp for schedule(dynamic, 4)
+        for (int64_t n = 0; n < nrows; ++n) {
+            if (!kept || !z) continue;
+            const int64_t r = rows ? rows[n] : n;
+            const int64_t bh = r / Lq;
+            const int t = (int)(r % Lq);
+            const int b = (int)(bh / Hq), h = (int)(bh % Hq), g = h / G;
+            const int pos = T - Lq + t;
+            const int i = t / block;
+            const size_t u_list = ((size_t)bh * nq + i);
+            memset(kept, 0, (size_t)nb);
+            int cnt = count[u_list];
+            int bad = cnt < 0 || cnt > cap;
+            for (int c = 0; c < cnt && !bad; ++c) {
+                int j = idx[u_list * cap + c];
+                if (j < 0 || j >= nb) bad = 1; else kept[j] = 1;
+            }
+            if (bad) {
+#pragma omp atomic write
+                err = ORACLE_EINVAL;
+                continue;
+            }
+            const size_t qoff = (size_t)r * d;
+            const size_t kvbase = ((size_t)b * Hkv + g) * T;
+            double m = -INFINITY;
+            for (int u = 0; u < T; ++u) {
+                if (!(u <= pos && kept[u / block])) { z[u] = -INFINITY; continue; }
+                double s = 0.0;
+                for (int c = 0; c < d; ++c)
+                    s += elem(q, is_bf16, qoff + c) * elem(k, is_bf16, (kvbase + u) * d + c);
+                z[u] = scale * s;
+                if (z[u] > m) m = z[u];
+            }
+            double *o = out + (size_t)n * d;
+            for (int c = 0; c < d; ++c) o[c] = 0.0;
+            if (m == -INFINITY) {
+                if (lse) lse[n] = -INFINITY;
+                continue;
+            }
+            double den = 0.0;
+            for (int u = 0; u < T; ++u) {
+                if (z[u] == -INFINITY) continue;
+                double p = exp(z[u] - m);
+                den += p;
+                for (int c = 0; c < d; ++c) o[c] += p * elem(v, is_bf16, (kvbase + u) * d + c);
+            }
+            for (int c = 0; c < d; ++c) o[c] /= den;
+            if (lse) lse[n] = m + log(den);
+        }
+        free(kept);
+        free(z);
+    }
+    return err;
+}

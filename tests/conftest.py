@@ -1,0 +1,16 @@
+"""Pytest configuration: registers the ``gpu`` marker and shared fixtures."""
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+
+def pytest_configure(config):
+    config.addinivalue_line(
+        "markers", "gpu: needs a CUDA device (B200, sm_100a); runs the CUDA path through the C-ABI")
+    config.addinivalue_line(
+        "markers", "slow: full-size workload; generation and oracle take tens of seconds")

@@ -1,0 +1,82 @@
+"""The pins catch plausible mistakes: each case plants one mistake in a temporary
+copy of the oracle's C source (on the CPU), builds it, points the oracle module at
+it and checks that the named pin tests now fail. CPU only.
+"""
+import os
+import subprocess
+
+import pytest
+
+import oracle
+from tests import test_oracle_pins as pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "spa_oracle.c")
+
+
+def dense_causal_at_p_one():
+    pins.test_top_p_one_equals_dense_causal_attention(70, 16)
+
+# (name, text to replace, replacement, pins that must fail)
+MUTATIONS = [
+    ("dropped_half_in_variance_term", "log1p(0.5 * scale * scale * quad)",
+     "log1p(scale * scale * quad)",
+     [pins.test_score_hand_worked_examples, pins.test_score_error_is_third_order_in_query_norm]),
+    ("dropped_scale_squared", "log1p(0.5 * scale * scale * quad)", "log1p(0.5 * quad)",
+     [pins.test_score_error_is_third_order_in_query_norm]),
+    ("std_instead_of_variance", "lrow[j] = scale * dot", "quad = sqrt(quad); lrow[j] = scale * dot",
+     [pins.test_score_error_is_third_order_in_query_norm]),
+    ("dropped_block_count", " + log((double)nj);", ";",
+     [pins.test_score_exact_when_block_keys_identical, pins.test_score_hand_worked_examples]),
+    ("sample_variance", "vr[c] = s / n;", "vr[c] = s / (n > 1 ? n - 1 : 1);",
+     [pins.test_stats_match_numpy_mean_and_population_variance, pins.test_stats_two_key_closed_form]),
+    ("mean_divides_by_block", "mu[c] = s / n;", "mu[c] = s / block;",
+     [pins.test_stats_match_numpy_mean_and_population_variance]),
+    ("sum_pooled_query", "qbar[c] = s / nr;", "qbar[c] = s;",
+     [pins.test_score_hand_worked_examples]),
+    ("wrong_gqa_group_in_scores", "g = h / G;\n            const int r0", "g = h % Hkv;\n            const int r0",
+     [pins.test_score_gqa_head_reads_its_group]),
+    ("strict_causal_mask", "if (!(u <= pos && kept[u / block]))", "if (!(u < pos && kept[u / block]))",
+     [pins.test_attention_hand_worked_example, pins.test_attention_constant_keys_average_allowed_values]),
+    ("dropped_softmax_scale", "z[u] = scale * s;", "z[u] = s;",
+     [dense_causal_at_p_one]),
+    ("ties_prefer_larger_index", "return (x->j > y->j) - (x->j < y->j);",
+     "return (x->j < y->j) - (x->j > y->j);",
+     [pins.test_top_p_hand_worked_examples, pins.test_top_p_equal_scores_prefer_smaller_index]),
+    ("crossing_block_dropped", "cum += exp((double)cand[k].key - mx);\n                ++nk;",
+     "cum += exp((double)cand[k].key - mx);\n                if (cum / total < top_p) ++nk;",
+     [pins.test_top_p_hand_worked_examples]),
+    ("local_window_too_wide", "(j > jmax - n_local)", "(j >= jmax - n_local)",
+     [pins.test_top_p_hand_worked_examples]),
+    ("ascending_sort", "if (x->key > y->key) return -1;\n    if (x->key < y->key) return 1;",
+     "if (x->key < y->key) return -1;\n    if (x->key > y->key) return 1;",
+     [pins.test_top_p_hand_worked_examples, pins.test_top_p_tiny_p_keeps_top_one]),
+]
+
+
+@pytest.fixture(scope="module")
+def workdir(tmp_path_factory):
+    return tmp_path_factory.mktemp("oracle_mutants")
+
+
+@pytest.mark.parametrize("name,old,new,must_fail", MUTATIONS, ids=[m[0] for m in MUTATIONS])
+def test_pins_catch_planted_mistake(name, old, new, must_fail, workdir):
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation anchor for {name} not unique"
+    mutant_c = os.path.join(workdir, f"{name}.c")
+    mutant_so = os.path.join(workdir, f"{name}.so")
+    with open(mutant_c, "w") as f:
+        f.write(src.replace(old, new))
+    subprocess.run(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", "-ffp-contract=off",
+                    "-w", mutant_c, "-o", mutant_so, "-lm"], check=True)
+    oracle.use_library(mutant_so)
+    try:
+        caught = []
+        for test in must_fail:
+            try:
+                test()
+            except (AssertionError, RuntimeError):
+                caught.append(test.__name__)
+        assert caught, f"no pin caught mutation {name}"
+        assert len(caught) == len(must_fail), f"{name}: only {caught} failed"
+    finally:
+        oracle.use_library(None)

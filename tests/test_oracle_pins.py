@@ -1,0 +1,481 @@
+"""Pins for the CPU oracle: closed forms, hand-worked examples, brute force,
+invariants and special cases, none of which re-types the oracle's own formulas.
+
+Each test names the passage it pins. CPU only.
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "worked_examples.json")
+
+
+def _golden():
+    with open(GOLDEN) as f:
+        return json.load(f)
+
+
+def _rand(shape, seed, scale=1.0):
+    return (np.random.default_rng(seed).standard_normal(shape) * scale).astype(np.float32)
+
+
+# ---------------------------------------------------------------- block statistics
+# SPLA, section 2.1: first- and second-order block statistics (mean, diagonal variance).
+
+def test_stats_match_numpy_mean_and_population_variance():
+    k = _rand((2, 3, 37, 8), 1)            # 37 = 4 full blocks of 8 + a partial block of 5
+    mean, var = oracle.block_stats(k, "f32", 8)
+    assert mean.shape == (2, 3, 5, 8)
+    for j in range(5):
+        blk = k[:, :, 8 * j:8 * (j + 1), :].astype(np.float64)
+        np.testing.assert_allclose(mean[:, :, j], blk.mean(axis=2), rtol=1e-13, atol=1e-14)
+        np.testing.assert_allclose(var[:, :, j], blk.var(axis=2, ddof=0), rtol=1e-12, atol=1e-14)
+
+
+def test_stats_two_key_closed_form():
+    a, b = np.float32(1.5), np.float32(-0.25)
+    k = np.array([[[[a, 0.0], [b, 2.0]]]], np.float32)
+    mean, var = oracle.block_stats(k, "f32", 2)
+    assert mean[0, 0, 0, 0] == (a + b) / 2 and mean[0, 0, 0, 1] == 1.0
+    assert var[0, 0, 0, 0] == pytest.approx(((a - b) / 2) ** 2, rel=1e-15)
+    assert var[0, 0, 0, 1] == pytest.approx(1.0, rel=1e-15)
+
+
+def test_stats_invariant_under_permutation_within_block():
+    k = _rand((1, 2, 64, 16), 2)
+    perm = np.concatenate([np.random.default_rng(3).permutation(16) + 16 * j for j in range(4)])
+    m0, v0 = oracle.block_stats(k, "f32", 16)
+    m1, v1 = oracle.block_stats(k[:, :, perm], "f32", 16)
+    np.testing.assert_allclose(m1, m0, rtol=1e-13, atol=1e-15)
+    np.testing.assert_allclose(v1, v0, rtol=1e-12, atol=1e-15)
+
+
+def test_stats_read_bf16_bit_patterns():
+    from workloads import bf16_bits, widen
+    k32 = _rand((1, 1, 20, 8), 4)
+    bits = bf16_bits(k32)
+    m_b, v_b = oracle.block_stats(bits, "bf16", 8)
+    m_f, v_f = oracle.block_stats(widen(bits, "bf16"), "f32", 8)
+    assert np.array_equal(m_b, m_f) and np.array_equal(v_b, v_f)
+
+
+# ---------------------------------------------------------------- Taylor score
+# SPLA, section 2.1: the score approximates the block's integrated attention mass
+# sum_u exp(s qbar . k_u) by a second-order expansion about the block mean.
+
+def test_score_hand_worked_examples():
+    g = _golden()["taylor_score"]
+    for case in g["cases"]:
+        k = np.array(case["k"], np.float32)[None, None]
+        q = np.array(case["q"], np.float32)[None, None]
+        mean, var = oracle.block_stats(k, "f32", case["block"])
+        l = oracle.scores(q, "f32", mean, var, case["T"], case["block"], case["scale"])
+        np.testing.assert_allclose(l[0, 0, -1, :len(case["expected_l"])], case["expected_l"],
+                                   rtol=1e-15, atol=1e-15, err_msg=case["name"])
+
+
+def _exact_log_mass(qbar, keys, s):
+    z = s * keys.astype(np.float64) @ qbar
+    m = z.max()
+    return m + math.log(np.exp(z - m).sum())
+
+
+def test_score_exact_when_block_keys_identical():
+    # var = 0 => no approximation is left: l_j == log sum_u exp(s qbar.k_u) exactly.
+    rng = np.random.default_rng(5)
+    T, blk, d = 96, 16, 8
+    keys = np.repeat(rng.standard_normal((T // blk, d)).astype(np.float32), blk, axis=0)
+    q = rng.standard_normal((1, 1, 1, d)).astype(np.float32)
+    mean, var = oracle.block_stats(keys[None, None], "f32", blk)
+    assert np.all(var == 0)
+    s = 0.3
+    l = oracle.scores(q, "f32", mean, var, T, blk, s)[0, 0, 0]
+    for j in range(T // blk):
+        ref = _exact_log_mass(q[0, 0, 0].astype(np.float64), keys[j * blk:(j + 1) * blk], s)
+        assert l[j] == pytest.approx(ref, rel=1e-13, abs=1e-13)
+
+
+def test_score_exact_for_unit_blocks_and_pooled_prefill_query():
+    rng = np.random.default_rng(6)
+    T, d = 9, 4
+    k = rng.standard_normal((1, 1, T, d)).astype(np.float32)
+    q = rng.standard_normal((1, 1, T, d)).astype(np.float32)
+    mean, var = oracle.block_stats(k, "f32", 1)
+    l = oracle.scores(q, "f32", mean, var, T, 1, 0.7)
+    for i in range(T):
+        for j in range(T):
+            if j > i:
+                assert l[0, 0, i, j] == -np.inf
+            else:
+                ref = 0.7 * float(q[0, 0, i].astype(np.float64) @ k[0, 0, j].astype(np.float64))
+                assert l[0, 0, i, j] == pytest.approx(ref, rel=1e-13, abs=1e-14)
+
+
+def _diag_cov_block(d, rng):
+    """3d keys whose deviations from the mean lie on single axes: the sample
+    covariance is exactly diagonal and the third moment is non-zero."""
+    mu = rng.standard_normal(d)
+    a = 0.5 + rng.random(d)
+    rows = []
+    for c in range(d):
+        e = np.zeros(d)
+        e[c] = a[c]
+        rows += [mu + 2 * e, mu - e, mu - e]
+    return np.array(rows, np.float64).astype(np.float32)
+
+
+def test_score_error_is_third_order_in_query_norm():
+    # With a diagonal covariance, exact log mass - l = O(|q|^3) (second-order
+    # expansion). A dropped 1/2, a dropped s^2, a wrong sign or a std in place of a
+    # variance leaves an O(|q|^2) error; a wrong mean term leaves O(|q|).
+    rng = np.random.default_rng(7)
+    d = 6
+    keys = _diag_cov_block(d, rng)
+    blk = keys.shape[0]
+    mean, var = oracle.block_stats(keys[None, None], "f32", blk)
+    direction = rng.standard_normal(d)
+    s = 1 / math.sqrt(d)
+    errs = []
+    for eps in [0.2, 0.1, 0.05, 0.025]:
+        qv = (eps * direction).astype(np.float32)
+        l = oracle.scores(qv[None, None, None], "f32", mean, var, blk, blk, s)[0, 0, 0, 0]
+        errs.append(abs(_exact_log_mass(qv.astype(np.float64), keys, s) - l))
+    ratios = [errs[n] / errs[n + 1] for n in range(3)]
+    assert all(6.5 < r < 9.5 for r in ratios), (errs, ratios)
+
+
+def test_score_gqa_head_reads_its_group():
+    rng = np.random.default_rng(8)
+    B, Hq, Hkv, T, d, blk = 2, 4, 2, 40, 8, 8
+    q = rng.standard_normal((B, Hq, T, d)).astype(np.float32)
+    k = rng.standard_normal((B, Hkv, T, d)).astype(np.float32)
+    mean, var = oracle.block_stats(k, "f32", blk)
+    l = oracle.scores(q, "f32", mean, var, T, blk, 0.35)
+    for b in range(B):
+        for h in range(Hq):
+            g = h // (Hq // Hkv)
+            one = oracle.scores(q[b:b + 1, h:h + 1], "f32", mean[b:b + 1, g:g + 1],
+                                var[b:b + 1, g:g + 1], T, blk, 0.35)
+            np.testing.assert_array_equal(l[b, h], one[0, 0])
+
+
+# ---------------------------------------------------------------- dual top-p cut
+# SpotAttention, section 3: reserved sink/recency blocks, nucleus over the residual,
+# K_min floor.
+
+def test_top_p_hand_worked_examples():
+    g = _golden()["top_p"]
+    l = np.array(g["scores"], np.float64)[None, None, None]
+    T = 6 * 4
+    for case in g["cases"]:
+        idx, cnt = oracle.select_from_scores(l, 1, T, 4, case["top_p"], 1, 1, case["k_min"])
+        got = list(idx[0, 0, 0, :cnt[0, 0, 0]])
+        assert got == case["expected"], (case, got)
+        assert np.all(idx[0, 0, 0, cnt[0, 0, 0]:] == -1)
+
+
+def _brute_force_keep(scores32, p, k_min):
+    """Smallest subset of the residual whose normalised mass reaches p (the
+    heaviest such subset), then padded to the K_min heaviest."""
+    n = len(scores32)
+    w = np.exp(scores32.astype(np.float64) - scores32.max())
+    w /= w.sum()
+    order = sorted(range(n), key=lambda j: (-scores32[j], j))
+    best = None
+    if p >= 1:
+        best = set(range(n))
+    else:
+        for c in range(1, n + 1):
+            cands = [S for S in itertools.combinations(range(n), c) if w[list(S)].sum() >= p]
+            if cands:
+                top = max(w[list(S)].sum() for S in cands)
+                best = set(min(S for S in cands if w[list(S)].sum() == top))
+                break
+    floor = min(k_min, n)
+    if len(best) < floor:
+        best = set(order[:floor])
+    return best
+
+
+@pytest.mark.parametrize("seed", range(40))
+def test_top_p_matches_brute_force(seed):
+    rng = np.random.default_rng(100 + seed)
+    jmax = int(rng.integers(0, 14))
+    n_sink, n_local = int(rng.integers(0, 3)), int(rng.integers(0, 3))
+    k_min = int(rng.choice([0, 0, 1, 3]))
+    p = float(rng.choice([rng.random(), 1.0, rng.random() * 0.3]))
+    p = max(p, 1e-6)
+    blk = 4
+    T = (jmax + 1) * blk
+    l = rng.standard_normal(jmax + 1) * 2.0
+    idx, cnt = oracle.select_from_scores(l[None, None, None], 1, T, blk, p, n_sink, n_local, k_min)
+    got = set(idx[0, 0, 0, :cnt[0, 0, 0]].tolist())
+    rsv = {j for j in range(jmax + 1) if j < n_sink or j > jmax - n_local}
+    resid = [j for j in range(jmax + 1) if j not in rsv]
+    exp = set(rsv)
+    if resid:
+        s32 = l[resid].astype(np.float32)
+        # skip cases whose decision sits within rounding of p
+        w = np.exp(s32.astype(np.float64) - s32.max())
+        w /= w.sum()
+        cum = np.cumsum(np.sort(w)[::-1])
+        if p < 1 and np.any(np.abs(cum - p) < 1e-9):
+            pytest.skip("boundary case")
+        exp |= {resid[j] for j in _brute_force_keep(s32, p, k_min)}
+    assert got == exp
+    assert list(idx[0, 0, 0, :cnt[0, 0, 0]]) == sorted(exp)
+
+
+def test_top_p_tiny_p_keeps_top_one():
+    l = np.array([0.0, 0.5, 3.0, -1.0, 2.9, 0.0])[None, None, None]
+    idx, cnt = oracle.select_from_scores(l, 1, 6, 1, 1e-9, 1, 1)
+    assert list(idx[0, 0, 0, :cnt[0, 0, 0]]) == [0, 2, 5]
+
+
+def test_top_p_equal_scores_prefer_smaller_index():
+    l = np.zeros((1, 1, 1, 6))
+    idx, cnt = oracle.select_from_scores(l, 1, 6, 1, 0.5, 1, 1)   # residual 1..4, 1/4 each
+    assert list(idx[0, 0, 0, :cnt[0, 0, 0]]) == [0, 1, 2, 5]
+
+
+def test_top_p_prefill_reserved_blocks_and_causal_limit():
+    rng = np.random.default_rng(9)
+    nq = 7
+    l = rng.standard_normal((1, 2, nq, nq))
+    l[..., np.triu_indices(nq, 1)[0], np.triu_indices(nq, 1)[1]] = -np.inf
+    idx, cnt = oracle.select_from_scores(l, nq * 8, nq * 8, 8, 0.3, 1, 1)
+    for h in range(2):
+        for i in range(nq):
+            lst = idx[0, h, i, :cnt[0, h, i]].tolist()
+            assert lst == sorted(set(lst))
+            assert 0 in lst and i in lst and max(lst) == i
+    assert cnt[0, 0, 0] == 1 and cnt[0, 0, 1] == 2
+
+
+# ---------------------------------------------------------------- attention
+# S2O, section 3: exact softmax attention over the selected blocks.
+
+def test_attention_hand_worked_example():
+    g = _golden()["attention"]
+    T, d, blk = g["T"], g["d"], g["block"]
+    q = np.array(g["q"], np.float32).reshape(1, 1, T, d)
+    k = np.array(g["k"], np.float32).reshape(1, 1, T, d)
+    v = np.array(g["v"], np.float32).reshape(1, 1, T, d)
+    idx, cnt = oracle.full_lists(1, 1, T, T, blk)
+    out, lse = oracle.attention(q, k, v, "f32", blk, idx, cnt, g["scale"])
+    np.testing.assert_allclose(out[0, 0, :, 0], g["expected_prefill_out"], rtol=1e-14)
+    np.testing.assert_allclose(lse[0, 0], g["expected_prefill_lse"], rtol=1e-14, atol=1e-15)
+
+
+def _random_lists(B, Hq, T, blk, seed):
+    rng = np.random.default_rng(seed)
+    nb = -(-T // blk)
+    idx = np.full((B, Hq, nb, nb), -1, np.int32)
+    cnt = np.zeros((B, Hq, nb), np.int32)
+    for b in range(B):
+        for h in range(Hq):
+            for i in range(nb):
+                keep = sorted({0, i} | {j for j in range(i + 1) if rng.random() < 0.5})
+                idx[b, h, i, :len(keep)] = keep
+                cnt[b, h, i] = len(keep)
+    return idx, cnt
+
+
+def test_attention_constant_keys_average_allowed_values():
+    # Equal logits => the output is the plain mean of the allowed values
+    # (u <= t and block(u) kept): pins the mask and the normalisation.
+    rng = np.random.default_rng(10)
+    B, Hq, Hkv, T, d, blk = 1, 2, 1, 45, 4, 8
+    q = rng.standard_normal((B, Hq, T, d)).astype(np.float32)
+    k = np.tile(rng.standard_normal(d).astype(np.float32), (B, Hkv, T, 1))
+    v = rng.standard_normal((B, Hkv, T, d)).astype(np.float32)
+    idx, cnt = _random_lists(B, Hq, T, blk, 11)
+    out, _ = oracle.attention(q, k, v, "f32", blk, idx, cnt, 0.5)
+    for h in range(Hq):
+        for t in range(T):
+            kept = set(idx[0, h, t // blk, :cnt[0, h, t // blk]].tolist())
+            allowed = [u for u in range(t + 1) if u // blk in kept]
+            np.testing.assert_allclose(out[0, h, t], v[0, 0, allowed].astype(np.float64).mean(0),
+                                       rtol=1e-12, atol=1e-13)
+
+
+def test_attention_constant_values_and_dominant_key():
+    rng = np.random.default_rng(12)
+    T, d, blk = 30, 4, 8
+    q = rng.standard_normal((1, 1, T, d)).astype(np.float32)
+    k = rng.standard_normal((1, 1, T, d)).astype(np.float32)
+    c = rng.standard_normal(d).astype(np.float32)
+    v = np.tile(c, (1, 1, T, 1))
+    idx, cnt = _random_lists(1, 1, T, blk, 13)
+    out, _ = oracle.attention(q, k, v, "f32", blk, idx, cnt, 0.4)
+    np.testing.assert_allclose(out[0, 0], np.tile(c.astype(np.float64), (T, 1)), rtol=1e-12)
+    # one key with a huge logit for every query that can see it
+    k2 = k.copy()
+    k2[0, 0, 3] = 0
+    q2 = q.copy()
+    q2[0, 0, :, 0] = 1
+    k2[0, 0, 3, 0] = 200.0
+    v2 = rng.standard_normal((1, 1, T, d)).astype(np.float32)
+    full_i, full_c = oracle.full_lists(1, 1, T, T, blk)
+    out2, _ = oracle.attention(q2, k2, v2, "f32", blk, full_i, full_c, 1.0)
+    np.testing.assert_allclose(out2[0, 0, 3:], np.tile(v2[0, 0, 3].astype(np.float64), (T - 3, 1)),
+                               rtol=1e-12, atol=1e-12)
+
+
+def _dense_causal_numpy(q, k, v, s):
+    B, Hq, L, d = q.shape
+    G = Hq // k.shape[1]
+    out = np.empty(q.shape, np.float64)
+    mask = np.tril(np.ones((L, L), bool))
+    for b in range(B):
+        for h in range(Hq):
+            z = s * q[b, h].astype(np.float64) @ k[b, h // G].astype(np.float64).T
+            z = np.where(mask, z, -np.inf)
+            z -= z.max(axis=1, keepdims=True)
+            p = np.exp(z)
+            p /= p.sum(axis=1, keepdims=True)
+            out[b, h] = p @ v[b, h // G].astype(np.float64)
+    return out
+
+
+@pytest.mark.parametrize("T,blk", [(64, 16), (70, 16), (33, 64)])
+def test_top_p_one_equals_dense_causal_attention(T, blk):
+    rng = np.random.default_rng(14 + T)
+    B, Hq, Hkv, d = 2, 4, 2, 8
+    q = rng.standard_normal((B, Hq, T, d)).astype(np.float32)
+    k = rng.standard_normal((B, Hkv, T, d)).astype(np.float32)
+    v = rng.standard_normal((B, Hkv, T, d)).astype(np.float32)
+    s = 1 / math.sqrt(d)
+    sel = oracle.select(q, k, "f32", blk, s, 1.0)
+    nq = -(-T // blk)
+    for i in range(nq):
+        assert np.all(sel["count"][:, :, i] == i + 1)
+    out, _ = oracle.attention(q, k, v, "f32", blk, sel["idx"], sel["count"], s)
+    np.testing.assert_allclose(out, _dense_causal_numpy(q, k, v, s), rtol=1e-11, atol=1e-12)
+
+
+def test_single_block_sequence_is_dense_causal_at_any_p():
+    rng = np.random.default_rng(15)
+    for T in (16, 11):
+        q = rng.standard_normal((1, 2, T, 8)).astype(np.float32)
+        k = rng.standard_normal((1, 1, T, 8)).astype(np.float32)
+        v = rng.standard_normal((1, 1, T, 8)).astype(np.float32)
+        sel = oracle.select(q, k, "f32", 16, 0.3, 0.1)
+        out, _ = oracle.attention(q, k, v, "f32", 16, sel["idx"], sel["count"], 0.3)
+        np.testing.assert_allclose(out, _dense_causal_numpy(q, k, v, 0.3), rtol=1e-11, atol=1e-12)
+
+
+def test_kv_permutation_within_earlier_blocks_changes_nothing():
+    # Sparsere Blok-Sparse Attention via Tokenpermutatie, section 1: attention is
+    # invariant under a joint permutation of (k, v) pairs; within a block that lies
+    # wholly before the query block the stats (up to rounding), the selection and
+    # the output of the last query block are unchanged.
+    rng = np.random.default_rng(16)
+    B, Hq, Hkv, T, d, blk = 1, 4, 2, 96, 8, 16
+    q = rng.standard_normal((B, Hq, T, d)).astype(np.float32)
+    k = rng.standard_normal((B, Hkv, T, d)).astype(np.float32)
+    v = rng.standard_normal((B, Hkv, T, d)).astype(np.float32)
+    perm = np.arange(T)
+    for j in range(T // blk - 1):
+        perm[j * blk:(j + 1) * blk] = j * blk + rng.permutation(blk)
+    s = 1 / math.sqrt(d)
+    a = oracle.select(q, k, "f32", blk, s, 0.7)
+    b = oracle.select(q, k[:, :, perm], "f32", blk, s, 0.7)
+    np.testing.assert_allclose(b["mean"], a["mean"], rtol=1e-13, atol=1e-15)
+    np.testing.assert_allclose(b["var"], a["var"], rtol=1e-12, atol=1e-15)
+    assert np.array_equal(a["idx"], b["idx"]) and np.array_equal(a["count"], b["count"])
+    rows = np.array([(h * T + t) for h in range(Hq) for t in range(T - blk, T)])
+    oa, _ = oracle.attention(q, k, v, "f32", blk, a["idx"], a["count"], s, rows=rows)
+    ob, _ = oracle.attention(q, k[:, :, perm], v[:, :, perm], "f32", blk, b["idx"], b["count"], s,
+                             rows=rows)
+    np.testing.assert_allclose(ob, oa, rtol=1e-12, atol=1e-13)
+
+
+def test_segmented_permutation_keeps_later_segments_at_p_one():
+    # Same page, section 2: permuting within a segment of size S keeps every query
+    # of a later segment unchanged (all of the segment lies in its causal past).
+    rng = np.random.default_rng(17)
+    T, d, blk, S = 64, 8, 8, 16
+    q = rng.standard_normal((1, 2, T, d)).astype(np.float32)
+    k = rng.standard_normal((1, 1, T, d)).astype(np.float32)
+    v = rng.standard_normal((1, 1, T, d)).astype(np.float32)
+    perm = np.concatenate([seg * S + rng.permutation(S) for seg in range(T // S)])
+    fi, fc = oracle.full_lists(1, 2, T, T, blk)
+    oa, _ = oracle.attention(q, k, v, "f32", blk, fi, fc, 0.3)
+    for seg in range(T // S):
+        p = np.arange(T)
+        p[seg * S:(seg + 1) * S] = perm[seg * S:(seg + 1) * S]
+        ob, _ = oracle.attention(q, k[:, :, p], v[:, :, p], "f32", blk, fi, fc, 0.3)
+        later = slice((seg + 1) * S, T)
+        np.testing.assert_allclose(ob[:, :, later], oa[:, :, later], rtol=1e-12, atol=1e-13)
+        if seg < T // S - 1:
+            assert not np.allclose(ob[:, :, seg * S:(seg + 1) * S], oa[:, :, seg * S:(seg + 1) * S])
+
+
+def test_decode_equals_prefill_last_row():
+    rng = np.random.default_rng(18)
+    B, Hq, Hkv, T, d, blk = 2, 4, 2, 77, 8, 16
+    q = rng.standard_normal((B, Hq, T, d)).astype(np.float32)
+    k = rng.standard_normal((B, Hkv, T, d)).astype(np.float32)
+    v = rng.standard_normal((B, Hkv, T, d)).astype(np.float32)
+    s = 0.33
+    qd = q[:, :, T - 1:T].copy()
+    dec = oracle.select(qd, k, "f32", blk, s, 0.6)
+    od, lse_d = oracle.attention(qd, k, v, "f32", blk, dec["idx"], dec["count"], s)
+    # prefill lists: every query block keeps everything, except the last one, which
+    # takes the decode list
+    nq = -(-T // blk)
+    pi, pc = oracle.full_lists(B, Hq, T, T, blk)
+    pi[:, :, nq - 1] = dec["idx"][:, :, 0]
+    pc[:, :, nq - 1] = dec["count"][:, :, 0]
+    op, lse_p = oracle.attention(q, k, v, "f32", blk, pi, pc, s)
+    np.testing.assert_allclose(od[:, :, 0], op[:, :, T - 1], rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(lse_d[:, :, 0], lse_p[:, :, T - 1], rtol=1e-13)
+    # decode at p = 1 is dense attention of one query over the whole cache
+    full = oracle.select(qd, k, "f32", blk, s, 1.0)
+    of, _ = oracle.attention(qd, k, v, "f32", blk, full["idx"], full["count"], s)
+    ref = _dense_causal_numpy(q, k, v, s)[:, :, T - 1]
+    np.testing.assert_allclose(of[:, :, 0], ref, rtol=1e-11, atol=1e-12)
+
+
+def test_attention_rows_subset_matches_full():
+    rng = np.random.default_rng(19)
+    B, Hq, Hkv, T, d, blk = 1, 4, 2, 50, 8, 8
+    q = rng.standard_normal((B, Hq, T, d)).astype(np.float32)
+    k = rng.standard_normal((B, Hkv, T, d)).astype(np.float32)
+    v = rng.standard_normal((B, Hkv, T, d)).astype(np.float32)
+    idx, cnt = _random_lists(B, Hq, T, blk, 20)
+    full, lse = oracle.attention(q, k, v, "f32", blk, idx, cnt, 0.3)
+    rows = np.array([0, 5, 49, 50, 123, 199])
+    part, lse_p = oracle.attention(q, k, v, "f32", blk, idx, cnt, 0.3, rows=rows)
+    np.testing.assert_array_equal(part, full.reshape(-1, d)[rows])
+    np.testing.assert_array_equal(lse_p, lse.reshape(-1)[rows])
+
+
+def test_attention_gqa_head_reads_its_group():
+    rng = np.random.default_rng(21)
+    B, Hq, Hkv, T, d, blk = 1, 6, 3, 40, 4, 8
+    q = rng.standard_normal((B, Hq, T, d)).astype(np.float32)
+    k = rng.standard_normal((B, Hkv, T, d)).astype(np.float32)
+    v = rng.standard_normal((B, Hkv, T, d)).astype(np.float32)
+    idx, cnt = _random_lists(B, Hq, T, blk, 22)
+    out, _ = oracle.attention(q, k, v, "f32", blk, idx, cnt, 0.5)
+    for h in range(Hq):
+        g = h // 2
+        one, _ = oracle.attention(q[:, h:h + 1], k[:, g:g + 1], v[:, g:g + 1], "f32", blk,
+                                  idx[:, h:h + 1], cnt[:, h:h + 1], 0.5)
+        np.testing.assert_array_equal(out[:, h], one[:, 0])
+
+
+def test_oracle_rejects_bad_lists():
+    q = np.zeros((1, 1, 8, 4), np.float32)
+    idx = np.array([[[[0, 5]]]], np.int32)            # block 5 does not exist
+    cnt = np.array([[[2]]], np.int32)
+    with pytest.raises(RuntimeError):
+        oracle.attention(q, q, q, "f32", 8, idx, cnt, 1.0)
