@@ -1,0 +1,427 @@
+#!/usr/bin/env python
+"""Benchmark of the block-sparse attention path on B200.
+
+One step = the whole prefill path over one batch of the 32K workload: block
+statistics -> Taylor-score top-p selection -> block-sparse causal attention
+(three kernels through the C-ABI). Printed as one JSON line by rank 0:
+
+  value     prefill tokens/s over all ranks (device time, CUDA events on the
+            launching stream, inputs resident in HBM, L2 flushed between steps)
+  roofline  the attention kernel's kept-block TFLOP/s against the measured bf16
+            tensor peak
+  decode    decode kept-KV GB/s of the decode workload against measured HBM peak
+  e2e       the same prefill metric with host buffers: pinned host -> device
+            copies of Q, K, V and the device -> host copy of O inside the timed
+            region
+  cpu_baseline  the CPU oracle on a bounded sample (rank 0, one GPU only)
+
+`--impl reference` times the CPU oracle on the same workload instead (the
+reference arm of this comparison) and prints the same line with "impl":
+"reference".
+
+Multi-GPU: one process per GPU (torchrun); every rank runs its own replica of the
+workload (the units are independent, so the path needs no collective); the time
+is the max over ranks and the value counts the tokens of all ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from workloads import WORKLOADS, generate, n_threads  # noqa: E402
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+METRIC = "prefill tokens/s & kept-FLOP TFLOP/s at 32K; decode KV GB/s vs HBM peak"
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+# ---------------------------------------------------------------- algorithmic work
+
+def kept_flops(count: np.ndarray, idx: np.ndarray, L: int, block: int, d: int) -> float:
+    """4 d x (unmasked query-key pairs) over every kept (head, query block, block) tile."""
+    nq = count.shape[-1]
+    n_i = np.minimum(block, L - np.arange(nq) * block).astype(np.float64)       # rows per q-block
+    last = np.take_along_axis(idx, np.maximum(count - 1, 0)[..., None], axis=-1)[..., 0]
+    diag = (last == np.arange(nq)).astype(np.float64)
+    pairs = (count - diag) * n_i * block + diag * n_i * (n_i + 1) / 2
+    return float(4.0 * d * pairs.sum())
+
+
+def kept_kv_bytes(count: np.ndarray, idx: np.ndarray, G: int, T: int, block: int, d: int) -> float:
+    """K and V bytes of the union of the kept blocks of each (b, kv-head)."""
+    B, Hq = count.shape[:2]
+    nb = -(-T // block)
+    tokens = np.minimum(block, T - np.arange(nb) * block)
+    total = 0
+    for b in range(B):
+        for g in range(Hq // G):
+            kept = np.zeros(nb, bool)
+            for h in range(g * G, (g + 1) * G):
+                kept[idx[b, h, 0, :count[b, h, 0]]] = True
+            total += int(tokens[kept].sum())
+    return float(total * d * 2 * 2)
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.15)
+        self.proc.terminate()
+        self.proc.wait()
+        rows = [l.split(",") for l in open(self.path).read().strip().splitlines() if l.strip()]
+        os.unlink(self.path)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            r = [c.strip() for c in r]
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+            except (ValueError, IndexError):
+                continue
+            for n, v in zip(names, r[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- CPU oracle
+
+def time_oracle(w, x, n_tokens: int, seed: int):
+    """Oracle on a bounded sample: stats + selection on the whole workload, masked
+    attention on n_tokens uniformly drawn query positions (all heads). Returns
+    (tokens/s estimate, detail)."""
+    import oracle
+    t0 = time.perf_counter()
+    sel = oracle.select(x["q"], x["k"], w.dtype, w.block, w.scale, w.top_p, w.n_sink, w.n_local,
+                        w.k_min)
+    t_sel = time.perf_counter() - t0
+    rng = np.random.default_rng(seed)
+    pos = rng.choice(w.B * w.Lq, size=n_tokens, replace=False)
+    b, t = pos // w.Lq, pos % w.Lq
+    rows = ((b[:, None] * w.Hq + np.arange(w.Hq)[None, :]) * w.Lq + t[:, None]).reshape(-1)
+    t0 = time.perf_counter()
+    oracle.attention(x["q"], x["k"], x["v"], w.dtype, w.block, sel["idx"], sel["count"], w.scale,
+                     rows=rows)
+    t_att = time.perf_counter() - t0
+    total_tokens = w.B * w.Lq
+    t_est = t_att + t_sel * n_tokens / total_tokens
+    return n_tokens / t_est, {"t_select_s": t_sel, "t_attention_sample_s": t_att,
+                              "threads": oracle.num_threads()}
+
+
+# ---------------------------------------------------------------- reference arm
+
+def run_reference(args, rank: int):
+    if rank != 0:
+        return
+    w = WORKLOADS[args.workload]
+    x = generate(w)
+    per_step = []
+    n_tok = args.ref_tokens
+    for s in range(args.warmup + args.steps):
+        v, det = time_oracle(w, x, n_tok, 1000 + s)
+        if s >= args.warmup:
+            per_step.append(v)
+    value = statistics.median(per_step)
+    cores = det["threads"]
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": w.B * w.Lq / value * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "L": w.T, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d,
+                   "block": w.block, "top_p": w.top_p, "l2": "n/a (CPU)"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"per step: stats + selection on the whole {w.name} workload, "
+                                   f"masked fp64 attention on {n_tok} random query positions x "
+                                   f"{w.Hq} heads; tokens/s = sampled tokens / (their attention "
+                                   f"time + stats/selection time pro-rated per token)"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- CUDA arm
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=40)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["spa", "reference"], default="spa")
+    ap.add_argument("--workload", type=int, default=3)
+    ap.add_argument("--decode-workload", type=int, default=5)
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--cpu-tokens", type=int, default=192)
+    ap.add_argument("--ref-tokens", type=int, default=48)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+
+    import torch
+    import torch.distributed as dist
+    import block_sparse_long_stats_b200 as spa
+
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    peaks, peak_src = load_peaks()
+    w = WORKLOADS[args.workload]
+    x = generate(w)
+
+    def dev(a):
+        if w.dtype == "bf16":
+            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda().view(torch.bfloat16)
+        return torch.from_numpy(a).cuda()
+
+    q, k, v = dev(x["q"]), dev(x["k"]), dev(x["v"])
+    B, Hq, L, d = q.shape
+    Hkv = k.shape[1]
+    nb = -(-L // w.block)
+    mean = torch.empty((B, Hkv, nb, d), device="cuda", dtype=torch.float32)
+    var = torch.empty_like(mean)
+    idx = torch.empty((B, Hq, nb, nb), device="cuda", dtype=torch.int32)
+    cnt = torch.empty((B, Hq, nb), device="cuda", dtype=torch.int32)
+    out = torch.empty_like(q)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        spa.spa_block_stats(k, w.block, mean=mean, var=var)
+        if ev:
+            ev[1].record(stream)
+        spa.spa_select(q, mean, var, L, w.block, w.scale, w.top_p, w.n_sink, w.n_local, w.k_min,
+                       idx=idx, count=cnt)
+        if ev:
+            ev[2].record(stream)
+        spa.spa_sparse_attn_prefill(q, k, v, w.block, idx, cnt, w.scale, out=out)
+        if ev:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    assert spa.spa_get_device_error() == 0
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier()
+    torch.cuda.synchronize()
+    for s in range(args.steps):
+        flush.zero_()          # L2 flush between timed steps (outside the events)
+        step(evs[s])
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    t_stats = [e[0].elapsed_time(e[1]) for e in evs]
+    t_sel = [e[1].elapsed_time(e[2]) for e in evs]
+    t_att = [e[2].elapsed_time(e[3]) for e in evs]
+    t_step = [e[0].elapsed_time(e[3]) for e in evs]
+    total_ms = max_over_ranks(sum(t_step))
+    ms_per_step = total_ms / args.steps
+    value = world * B * L * args.steps / (total_ms / 1e3)
+
+    count_h = cnt.cpu().numpy()
+    idx_h = idx.cpu().numpy()
+    F = kept_flops(count_h, idx_h, L, w.block, d)
+    att_ms = statistics.mean(t_att)
+    achieved = F / (att_ms / 1e3) / 1e12
+    peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    dense_tiles = B * Hq * nb * (nb + 1) / 2
+    kept_frac = float(count_h.sum()) / dense_tiles
+    stats_bytes = B * Hkv * L * d * 2 + 2 * B * Hkv * nb * d * 4
+    per_kernel = {
+        "block_stats": {"ms": statistics.mean(t_stats),
+                        "GB/s": stats_bytes / (statistics.mean(t_stats) / 1e3) / 1e9},
+        "select": {"ms": statistics.mean(t_sel)},
+        "sparse_attn_prefill": {"ms": att_ms, "TFLOP/s": achieved},
+    }
+
+    # ---- end to end through host buffers
+    qh = torch.from_numpy(np.ascontiguousarray(x["q"]).view(np.int16)).pin_memory()
+    kh = torch.from_numpy(np.ascontiguousarray(x["k"]).view(np.int16)).pin_memory()
+    vh = torch.from_numpy(np.ascontiguousarray(x["v"]).view(np.int16)).pin_memory()
+    oh = torch.empty(out.shape, dtype=torch.int16).pin_memory()
+    qd, kd, vd = (torch.empty(t.shape, dtype=torch.int16, device="cuda") for t in (qh, kh, vh))
+    e_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+             for _ in range(args.e2e_steps)]
+    barrier()
+    torch.cuda.synchronize()
+    for s in range(args.e2e_steps):
+        e_evs[s][0].record(stream)
+        qd.copy_(qh, non_blocking=True)
+        kd.copy_(kh, non_blocking=True)
+        vd.copy_(vh, non_blocking=True)
+        qq, kk, vv = qd.view(torch.bfloat16), kd.view(torch.bfloat16), vd.view(torch.bfloat16)
+        spa.spa_block_stats(kk, w.block, mean=mean, var=var)
+        spa.spa_select(qq, mean, var, L, w.block, w.scale, w.top_p, w.n_sink, w.n_local, w.k_min,
+                       idx=idx, count=cnt)
+        spa.spa_sparse_attn_prefill(qq, kk, vv, w.block, idx, cnt, w.scale, out=out)
+        oh.copy_(out.view(torch.int16), non_blocking=True)
+        e_evs[s][1].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e_evs)) / args.e2e_steps
+    e2e = {"value": world * B * L / (e2e_ms / 1e3), "unit": "tokens/s",
+           "h2d_bytes_per_step": int(qh.numel() * 2 + kh.numel() * 2 + vh.numel() * 2),
+           "d2h_bytes_per_step": int(oh.numel() * 2), "ms_per_step": e2e_ms}
+    del qh, kh, vh, oh, qd, kd, vd
+
+    # ---- decode leg
+    decode = None
+    if not args.no_decode:
+        wd = WORKLOADS[args.decode_workload]
+        xd = generate(wd)
+        qd_ = torch.from_numpy(np.ascontiguousarray(xd["q"]).view(np.int16)).cuda().view(torch.bfloat16)
+        kc = torch.from_numpy(np.ascontiguousarray(xd["k"]).view(np.int16)).cuda().view(torch.bfloat16)
+        vc = torch.from_numpy(np.ascontiguousarray(xd["v"]).view(np.int16)).cuda().view(torch.bfloat16)
+        del xd
+        dm, dv = spa.spa_block_stats(kc, wd.block)
+        didx = torch.empty((wd.B, wd.Hq, 1, wd.nb), device="cuda", dtype=torch.int32)
+        dcnt = torch.empty((wd.B, wd.Hq, 1), device="cuda", dtype=torch.int32)
+        ws = torch.empty(spa.spa_decode_workspace_bytes(wd.B, wd.Hq, wd.Hkv, wd.T, wd.d, wd.block),
+                         dtype=torch.uint8, device="cuda")
+        dout = torch.empty_like(qd_)
+        for _ in range(3):
+            spa.spa_select(qd_, dm, dv, wd.T, wd.block, wd.scale, wd.top_p, idx=didx, count=dcnt)
+            spa.spa_sparse_attn_decode(qd_, kc, vc, wd.block, didx, dcnt, wd.scale, workspace=ws,
+                                       out=dout)
+        torch.cuda.synchronize()
+        assert spa.spa_get_device_error() == 0
+        n_dec = max(10, args.steps // 2)
+        d_evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_dec)]
+        barrier()
+        torch.cuda.synchronize()
+        for s in range(n_dec):
+            flush.zero_()
+            d_evs[s][0].record(stream)
+            spa.spa_select(qd_, dm, dv, wd.T, wd.block, wd.scale, wd.top_p, idx=didx, count=dcnt)
+            d_evs[s][1].record(stream)
+            spa.spa_sparse_attn_decode(qd_, kc, vc, wd.block, didx, dcnt, wd.scale, workspace=ws,
+                                       out=dout)
+            d_evs[s][2].record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        t_dsel = statistics.mean(e[0].elapsed_time(e[1]) for e in d_evs)
+        t_dec = statistics.mean(e[1].elapsed_time(e[2]) for e in d_evs)
+        dbytes = kept_kv_bytes(dcnt.cpu().numpy(), didx.cpu().numpy(), wd.G, wd.T, wd.block, wd.d)
+        gbs = dbytes / (t_dec / 1e3) / 1e9
+        decode = {"workload": wd.name, "kept_kv_bytes": dbytes, "attn_ms": t_dec,
+                  "select_ms": t_dsel, "GB/s": gbs, "peak_GB/s": peaks["hbm_gbs"],
+                  "frac": gbs / peaks["hbm_gbs"], "peak_source": peak_src,
+                  "tokens/s": world * wd.B / ((t_dsel + t_dec) / 1e3),
+                  "kept_fraction": float(dcnt.float().mean().item()) / wd.nb}
+        del kc, vc
+
+    # ---- CPU oracle baseline (rank 0, one GPU)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        v_cpu, det = time_oracle(w, x, args.cpu_tokens, 7)
+        cpu = {"value": v_cpu, "unit": "tokens/s", "cores": det["threads"], "kind": "oracle",
+               "sample": f"stats + selection on the whole workload ({det['t_select_s']:.2f} s), "
+                         f"masked fp64 attention on {args.cpu_tokens} random query positions x "
+                         f"{Hq} heads ({det['t_attention_sample_s']:.2f} s); tokens/s = sampled "
+                         f"tokens / (their attention time + stats/selection pro-rated per token)"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": w.name, "B": B, "L": L, "Hq": Hq, "Hkv": Hkv, "d": d,
+                       "block": w.block, "top_p": w.top_p, "kept_fraction": kept_frac,
+                       "parallelism": f"replicas x{world}",
+                       "l2": "flushed (256 MiB memset) between timed steps"},
+            "roofline": {"bound": "tensor", "kernel": "sparse_attn_prefill", "achieved": achieved,
+                         "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                         "peak_source": f"{peak_src} bf16_tflops_sustained",
+                         "kept_flops_per_launch": F, "traffic": None},
+            "kernels": per_kernel,
+            "decode": decode,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+            "clocks": clk,
+            "gpu_launches": 3 * args.steps,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

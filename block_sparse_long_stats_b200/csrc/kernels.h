@@ -1,0 +1,48 @@
+// Launchers of the sm_100a kernels (one translation unit each). Host-side
+// argument validation happens in spa_api.cu before any of these is called.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace spa {
+
+cudaError_t launch_block_stats(const void *k, bool bf16, int B, int Hkv, int T, int d, int block,
+                               int blk_begin, int blk_end, float *mean, float *var,
+                               cudaStream_t s);
+
+cudaError_t launch_select(const void *q, bool bf16, const float *mean, const float *var, int B,
+                          int Hq, int Hkv, int Lq, int T, int d, int block, float scale,
+                          float top_p, int n_sink, int n_local, int k_min, int32_t *idx, int cap,
+                          int32_t *count, int *err, cudaStream_t s);
+
+cudaError_t launch_prefill_f32(const float *q, const float *k, const float *v, int B, int Hq,
+                               int Hkv, int L, int d, int block, const int32_t *idx, int cap,
+                               const int32_t *count, float scale, float *out, float *lse,
+                               int *err, cudaStream_t s);
+
+// bf16, d = 128, block 64 or 128: TMA + tcgen05/TMEM. Returns cudaErrorNotSupported
+// when the tensor maps cannot be built.
+cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, int B, int Hq, int Hkv,
+                              int L, int block, const int32_t *idx, int cap,
+                              const int32_t *count, float scale, void *out, float *lse, int *err,
+                              cudaStream_t s);
+
+int decode_splits(int B, int Hkv, int T, int block);
+size_t decode_workspace_bytes(int B, int Hq, int Hkv, int T, int d, int block);
+cudaError_t launch_decode(const void *q, const void *kc, const void *vc, int B, int Hq, int Hkv,
+                          int T, int d, int block, const int32_t *idx, int cap,
+                          const int32_t *count, float scale, void *workspace, void *out, int *err,
+                          cudaStream_t s);
+
+// Driver entry point for cuTensorMapEncodeTiled (resolved once through the runtime).
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_tiled_fn();
+
+}  // namespace spa

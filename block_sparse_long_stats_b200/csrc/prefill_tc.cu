@@ -1,0 +1,414 @@
+// bf16 block-sparse causal prefill attention on the sm_100a tensor cores.
+//
+// Follows "S2O", sections 1 and 3: the kept key/value tiles are gathered by index
+// (coordinate-scheduled loading, no physical permutation) and folded into an
+// online-softmax state (m, l, acc) per query row; attention over the kept tiles
+// is exact.
+//
+// One CTA per tile of 128 query rows: one query block of one head (block 128), or
+// the same query block of two heads of one kv-group stacked (block 64; the pair
+// walks the union of its two kept lists, and a row masks the blocks its own head
+// did not keep). Warp roles:
+//   warps 0-3 : softmax; thread r owns query row r = TMEM lane r
+//   warp 4    : TMA producer (Q once; K_j and V_j per kept block into a ring)
+//   warp 5    : TMEM allocator and single-thread tcgen05.mma issuer
+// TMEM: S = Q K_j^T in columns [0, 128), O in columns [128, 256), fp32.
+// Per kept block n the issuer runs S(n) = Q K^T (8 MMAs, K = 16 each, over
+// d = 128) as soon as the softmax has read S(n-1), then O += P(n-1) V(n-1) once P
+// is in shared memory. The softmax scales by s*log2(e), takes exp2, keeps the
+// running max m lazily (O is rescaled only when the max grows by more than 8, in
+// log2 units), and writes P as bf16 in the 128-byte-swizzled K-major layout the
+// MMA reads. Epilogue: O / l from TMEM to bf16 rows, lse = (m + log2 l) ln 2.
+#include <math.h>
+
+#include "kernels.h"
+
+namespace spa {
+namespace {
+
+constexpr int kD = 128;
+constexpr int kThreads = 192;
+constexpr int kStages = 2;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kRescaleThreshold = 8.0f;   // log2 units
+
+template <int BLK>
+struct Cfg {
+    static constexpr int HPT = 128 / BLK;               // heads stacked in the M = 128 tile
+    static constexpr int Q_BYTES = 128 * kD * 2;        // 32 KB: two 64-column halves
+    static constexpr int KV_BYTES = BLK * kD * 2;       // one K or V tile
+    static constexpr int KV_HALF = BLK * 128;           // one 64-column half of it
+    static constexpr int P_BYTES = 128 * BLK * 2;
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_K = OFF_Q + Q_BYTES;
+    static constexpr int OFF_V = OFF_K + kStages * KV_BYTES;
+    static constexpr int OFF_P = OFF_V + kStages * KV_BYTES;
+    static constexpr int SMEM = OFF_P + P_BYTES;
+    static constexpr uint32_t IDESC_S = idesc_bf16(128, BLK, false);
+    static constexpr uint32_t IDESC_O = idesc_bf16(128, kD, true);
+};
+
+struct PrefillArgs {
+    const int32_t *idx;
+    const int32_t *count;
+    __nv_bfloat16 *out;
+    float *lse;
+    int B, Hq, Hkv, L, G, nq, cap, npairs;
+    float scale_log2;
+    int *err;
+};
+
+// Walks the ascending kept lists of the HPT heads of a tile in merged order. All
+// roles run identical cursors, so they agree on the block sequence; entries that
+// are out of range or not ascending are skipped (and reported by one role).
+template <int HPT>
+struct Cursor {
+    const int32_t *lst[HPT];
+    int cnt[HPT], pos[HPT], last[HPT];
+    int jmax;
+
+    __device__ void init(const PrefillArgs &a, int b, int h0, int i, bool report) {
+        jmax = i;
+#pragma unroll
+        for (int r = 0; r < HPT; ++r) {
+            const size_t unit = ((size_t)b * a.Hq + h0 + r) * a.nq + i;
+            int c = __ldg(a.count + unit);
+            if (c < 0 || c > a.cap) {
+                if (report) set_error(a.err, SPA_DEVERR_BAD_COUNT);
+                c = c < 0 ? 0 : a.cap;
+            }
+            lst[r] = a.idx + unit * a.cap;
+            cnt[r] = c;
+            pos[r] = 0;
+            last[r] = -1;
+        }
+    }
+    __device__ bool next(int &j, uint32_t &mask, int *err, bool report) {
+        int cand[HPT];
+        j = 0x7fffffff;
+#pragma unroll
+        for (int r = 0; r < HPT; ++r) {
+            cand[r] = 0x7fffffff;
+            while (pos[r] < cnt[r]) {
+                const int x = __ldg(lst[r] + pos[r]);
+                if (x > last[r] && x <= jmax) {
+                    cand[r] = x;
+                    break;
+                }
+                if (report) set_error(err, SPA_DEVERR_BAD_INDEX);
+                ++pos[r];
+            }
+            j = min(j, cand[r]);
+        }
+        if (j == 0x7fffffff) return false;
+        mask = 0;
+#pragma unroll
+        for (int r = 0; r < HPT; ++r) {
+            if (cand[r] == j) {
+                mask |= 1u << r;
+                last[r] = j;
+                ++pos[r];
+            }
+        }
+        return true;
+    }
+};
+
+template <int BLK>
+__global__ void __launch_bounds__(kThreads, 1)
+    prefill_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                      const __grid_constant__ CUtensorMap tv, PrefillArgs a) {
+    using C = Cfg<BLK>;
+    constexpr int HPT = C::HPT;
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char *smem = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    __shared__ uint64_t bar_q, full_k[kStages], full_v[kStages], empty_k[kStages],
+        empty_v[kStages], s_full, s_free, p_ready, o_done;
+    __shared__ uint32_t tmem_slot;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    // Heaviest tiles first: query block index descending.
+    const int per_i = a.B * a.Hkv * a.npairs;
+    const int i = a.nq - 1 - (int)(blockIdx.x / per_i);
+    const int rest = (int)(blockIdx.x % per_i);
+    const int b = rest / (a.Hkv * a.npairs);
+    const int g = (rest / a.npairs) % a.Hkv;
+    const int hp = rest % a.npairs;
+    const int h0 = g * a.G + hp * HPT;
+
+    if (tid == 0) {
+        mbar_init(&bar_q, 1);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full_k[s], 1);
+            mbar_init(&full_v[s], 1);
+            mbar_init(&empty_k[s], 1);
+            mbar_init(&empty_v[s], 1);
+        }
+        mbar_init(&s_full, 1);
+        mbar_init(&s_free, 128);
+        mbar_init(&p_ready, 128);
+        mbar_init(&o_done, 1);
+        fence_mbar_init();
+    }
+    if (warp == 5) tmem_alloc(&tmem_slot, 256);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_slot;
+    const uint32_t t_s = tmem, t_o = tmem + 128;
+
+    Cursor<HPT> cur;
+    if (warp == 4) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            prefetch_tmap(&tq);
+            prefetch_tmap(&tk);
+            prefetch_tmap(&tv);
+            mbar_arrive_expect_tx(&bar_q, C::Q_BYTES);
+#pragma unroll
+            for (int r = 0; r < HPT; ++r) {
+                const int row = ((b * a.Hq + h0 + r) * a.L) + i * BLK;
+                tma_load_2d(smem + C::OFF_Q + r * BLK * 128, &tq, &bar_q, 0, row);
+                tma_load_2d(smem + C::OFF_Q + 16384 + r * BLK * 128, &tq, &bar_q, 64, row);
+            }
+            cur.init(a, b, h0, i, true);
+            const int kv_row0 = (b * a.Hkv + g) * a.L;
+            int j;
+            uint32_t mask;
+            for (int n = 0; cur.next(j, mask, a.err, true); ++n) {
+                const int s = n % kStages;
+                const uint32_t ph = (n / kStages) & 1;
+                unsigned char *kt = smem + C::OFF_K + s * C::KV_BYTES;
+                unsigned char *vt = smem + C::OFF_V + s * C::KV_BYTES;
+                if (!mbar_wait(&empty_k[s], ph ^ 1, a.err)) break;
+                mbar_arrive_expect_tx(&full_k[s], C::KV_BYTES);
+                tma_load_2d(kt, &tk, &full_k[s], 0, kv_row0 + j * BLK);
+                tma_load_2d(kt + C::KV_HALF, &tk, &full_k[s], 64, kv_row0 + j * BLK);
+                if (!mbar_wait(&empty_v[s], ph ^ 1, a.err)) break;
+                mbar_arrive_expect_tx(&full_v[s], C::KV_BYTES);
+                tma_load_2d(vt, &tv, &full_v[s], 0, kv_row0 + j * BLK);
+                tma_load_2d(vt + C::KV_HALF, &tv, &full_v[s], 64, kv_row0 + j * BLK);
+            }
+        }
+    } else if (warp == 5) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            cur.init(a, b, h0, i, false);
+            const uint32_t q_base = smem_u32(smem + C::OFF_Q);
+            const uint32_t p_base = smem_u32(smem + C::OFF_P);
+            bool ok = mbar_wait(&bar_q, 0, a.err);
+            int n = 0, j;
+            uint32_t mask;
+            auto issue_pv = [&](int m) -> bool {
+                const int s = m % kStages;
+                if (!mbar_wait(&p_ready, m & 1, a.err)) return false;
+                if (!mbar_wait(&full_v[s], (m / kStages) & 1, a.err)) return false;
+                tc_fence_after();
+                const uint32_t v_base = smem_u32(smem + C::OFF_V + s * C::KV_BYTES);
+#pragma unroll
+                for (int kk = 0; kk < BLK / 16; ++kk) {
+                    const uint64_t ad = sw128_desc(p_base + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+                    const uint64_t bd = sw128_desc(v_base + kk * 2048, C::KV_HALF, 1024);
+                    tc_mma_ss(t_o, ad, bd, C::IDESC_O, (m > 0 || kk > 0) ? 1u : 0u);
+                }
+                tc_commit(&o_done);
+                tc_commit(&empty_v[s]);
+                return true;
+            };
+            while (ok && cur.next(j, mask, a.err, false)) {
+                const int s = n % kStages;
+                if (!mbar_wait(&full_k[s], (n / kStages) & 1, a.err)) break;
+                if (n > 0 && !mbar_wait(&s_free, (n - 1) & 1, a.err)) break;
+                tc_fence_after();
+                const uint32_t k_base = smem_u32(smem + C::OFF_K + s * C::KV_BYTES);
+#pragma unroll
+                for (int kk = 0; kk < kD / 16; ++kk) {
+                    const uint64_t ad = sw128_desc(q_base + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+                    const uint64_t bd = sw128_desc(k_base + (kk >> 2) * C::KV_HALF + (kk & 3) * 32, 16, 1024);
+                    tc_mma_ss(t_s, ad, bd, C::IDESC_S, kk > 0 ? 1u : 0u);
+                }
+                tc_commit(&s_full);
+                tc_commit(&empty_k[s]);
+                if (n > 0 && !issue_pv(n - 1)) { ok = false; break; }
+                ++n;
+            }
+            if (ok && n > 0) issue_pv(n - 1);
+        }
+    } else {
+        // ------------------------------------------------------------ softmax (rows)
+        const int r = tid;                       // TMEM lane
+        const int rg = r / BLK, rr = r % BLK;    // stacked head, row inside the block
+        const int h = h0 + rg;
+        const int t = i * BLK + rr;
+        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        cur.init(a, b, h0, i, false);
+        float m_used = -INFINITY, l = 0.f;
+        unsigned char *prow = smem + C::OFF_P + r * 128;
+        int n = 0, j;
+        uint32_t mask;
+        bool ok = true;
+        while (cur.next(j, mask, a.err, false)) {
+            if (!mbar_wait(&s_full, n & 1, a.err)) { ok = false; break; }
+            tc_fence_after();
+            float x[BLK];
+#pragma unroll
+            for (int c = 0; c < BLK / 32; ++c) {
+                uint32_t v[32];
+                tmem_ld32(t_s + lane_off + c * 32, v);
+                tc_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) x[c * 32 + e] = __uint_as_float(v[e]);
+            }
+            tc_fence_before();
+            mbar_arrive(&s_free);
+
+            const bool keep = (mask >> rg) & 1u;
+            const int lim = (j == i) ? rr : BLK - 1;          // causal limit inside the block
+            const int lim_t = min(lim, a.L - 1 - j * BLK);    // short last block
+            float mx = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < BLK; ++c) {
+                x[c] = (keep && c <= lim_t) ? x[c] * a.scale_log2 : -INFINITY;
+                mx = fmaxf(mx, x[c]);
+            }
+            float alpha = 1.f;
+            bool rescale = false;
+            if (mx > m_used + kRescaleThreshold) {
+                alpha = fast_exp2(m_used - mx);               // 0 when m_used = -inf
+                rescale = l > 0.f;
+                m_used = mx;
+            }
+            const float base = m_used == -INFINITY ? 0.f : m_used;
+            float rs = 0.f;
+#pragma unroll
+            for (int c = 0; c < BLK; ++c) {
+                x[c] = fast_exp2(x[c] - base);
+                rs += x[c];
+            }
+            l = l * alpha + rs;
+
+            if (n > 0) {
+                if (!mbar_wait(&o_done, (n - 1) & 1, a.err)) { ok = false; break; }
+                tc_fence_after();
+                if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+                    for (int c = 0; c < kD / 32; ++c) {
+                        uint32_t v[32];
+                        tmem_ld32(t_o + lane_off + c * 32, v);
+                        tc_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
+                        tmem_st32(t_o + lane_off + c * 32, v);
+                    }
+                    tc_wait_st();
+                }
+            }
+            // P row -> shared memory, bf16, K-major 128-byte swizzle (64 keys per half)
+#pragma unroll
+            for (int q8 = 0; q8 < BLK / 8; ++q8) {
+                uint4 w;
+                w.x = pack_bf16x2(x[q8 * 8 + 0], x[q8 * 8 + 1]);
+                w.y = pack_bf16x2(x[q8 * 8 + 2], x[q8 * 8 + 3]);
+                w.z = pack_bf16x2(x[q8 * 8 + 4], x[q8 * 8 + 5]);
+                w.w = pack_bf16x2(x[q8 * 8 + 6], x[q8 * 8 + 7]);
+                const int half = q8 >> 3, cq = q8 & 7;
+                *reinterpret_cast<uint4 *>(prow + half * 16384 + ((cq ^ (r & 7)) << 4)) = w;
+            }
+            fence_async_shared();
+            tc_fence_before();
+            mbar_arrive(&p_ready);
+            ++n;
+        }
+        // ------------------------------------------------------------ epilogue
+        if (ok && n > 0) ok = mbar_wait(&o_done, (n - 1) & 1, a.err);
+        tc_fence_after();
+        const bool store = t < a.L;
+        const float inv = (l > 0.f) ? 1.f / l : 0.f;
+        __nv_bfloat16 *orow = a.out + (((size_t)b * a.Hq + h) * a.L + t) * kD;
+#pragma unroll
+        for (int c = 0; c < kD / 32; ++c) {
+            uint32_t v[32];
+            if (ok && n > 0) {
+                tmem_ld32(t_o + lane_off + c * 32, v);
+                tc_wait_ld();
+            } else {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) v[e] = 0u;
+            }
+            if (store) {
+#pragma unroll
+                for (int e = 0; e < 32; e += 8) {
+                    uint4 w;
+                    w.x = pack_bf16x2(__uint_as_float(v[e + 0]) * inv, __uint_as_float(v[e + 1]) * inv);
+                    w.y = pack_bf16x2(__uint_as_float(v[e + 2]) * inv, __uint_as_float(v[e + 3]) * inv);
+                    w.z = pack_bf16x2(__uint_as_float(v[e + 4]) * inv, __uint_as_float(v[e + 5]) * inv);
+                    w.w = pack_bf16x2(__uint_as_float(v[e + 6]) * inv, __uint_as_float(v[e + 7]) * inv);
+                    *reinterpret_cast<uint4 *>(orow + c * 32 + e) = w;
+                }
+            }
+        }
+        if (store && a.lse)
+            a.lse[((size_t)b * a.Hq + h) * a.L + t] = l > 0.f ? (m_used + __log2f(l)) * kLn2 : -INFINITY;
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 5) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
+    }
+}
+
+bool make_map(CUtensorMap *map, const void *base, uint64_t rows, int box_rows) {
+    EncodeTiledFn enc = encode_tiled_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)kD, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)kD * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
+               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int BLK>
+cudaError_t launch_blk(const void *q, const void *k, const void *v, const PrefillArgs &a,
+                       cudaStream_t s) {
+    using C = Cfg<BLK>;
+    CUtensorMap mq, mk, mv;
+    if (!make_map(&mq, q, (uint64_t)a.B * a.Hq * a.L, BLK) ||
+        !make_map(&mk, k, (uint64_t)a.B * a.Hkv * a.L, BLK) ||
+        !make_map(&mv, v, (uint64_t)a.B * a.Hkv * a.L, BLK))
+        return cudaErrorNotSupported;
+    const size_t smem = C::SMEM + 1024;
+    auto kern = prefill_tc_kernel<BLK>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const unsigned grid = (unsigned)((size_t)a.nq * a.B * a.Hkv * a.npairs);
+    kern<<<grid, kThreads, smem, s>>>(mq, mk, mv, a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, int B, int Hq, int Hkv,
+                              int L, int block, const int32_t *idx, int cap,
+                              const int32_t *count, float scale, void *out, float *lse, int *err,
+                              cudaStream_t s) {
+    PrefillArgs a;
+    a.idx = idx;
+    a.count = count;
+    a.out = reinterpret_cast<__nv_bfloat16 *>(out);
+    a.lse = lse;
+    a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.L = L;
+    a.G = Hq / Hkv;
+    a.nq = (L + block - 1) / block;
+    a.cap = cap;
+    a.npairs = a.G / (128 / block);
+    a.scale_log2 = scale * kLog2e;
+    a.err = err;
+    return block == 64 ? launch_blk<64>(q, k, v, a, s) : launch_blk<128>(q, k, v, a, s);
+}
+
+}  // namespace spa

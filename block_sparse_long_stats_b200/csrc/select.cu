@@ -1,0 +1,290 @@
+// Block selection: pooled query, second-order Taylor block score, dual top-p cut.
+//
+//  - score: "SPLA - Block Sparse Plus Linear Attention for Long Context
+//    Modeling", section 2.1 (exp(q.kbar)(1 + 1/2 q^T diag(var) q), expanded with
+//    the attention scale s, times the block's token count), in the log domain;
+//  - pooled query: mean of the query block's rows ("Sparsere Blok-Sparse Attention
+//    via Tokenpermutatie", section 4, mean pooling);
+//  - cut: "SpotAttention", section 3 (sink and recency blocks reserved, nucleus
+//    over the residual, K_min floor).
+//
+// One CTA (256 threads) per (b, query head, query block). The residual candidates
+// are the contiguous range [r_lo, r_hi) of block indices between the sink prefix
+// and the local suffix, so only those are scored. Scores are fp32 (warp per
+// candidate, 128-bit loads of the block statistics, shuffle reductions). They are
+// packed with the block index into 64-bit keys that sort ascending in the order
+// (score descending, index ascending) and sorted with a shared-memory bitonic
+// network. Masses and their exclusive prefix sums are fp64, so the cut is decided
+// on fp32 scores with no further rounding in the masses. The kept set is written
+// as an ascending list by a prefix scan over per-block flags.
+#include <float.h>
+
+#include "kernels.h"
+
+namespace spa {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+
+__device__ __forceinline__ uint32_t order_desc(float f) {
+    uint32_t b = __float_as_uint(f);
+    uint32_t ord = (b & 0x80000000u) ? ~b : (b | 0x80000000u);   // ascending with f
+    return ~ord;                                                  // descending with f
+}
+__device__ __forceinline__ float key_score(uint64_t key) {
+    uint32_t ord = ~(uint32_t)(key >> 32);
+    uint32_t b = (ord & 0x80000000u) ? (ord ^ 0x80000000u) : ~ord;
+    return __uint_as_float(b);
+}
+
+// Block-wide exclusive scan (sum) of one value per thread; returns the exclusive
+// prefix, writes the block total to *total.
+template <typename V>
+__device__ V block_exclusive_scan(V x, V *warp_tot, V *total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    V inc = x;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        V y = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += y;
+    }
+    if (lane == 31) warp_tot[warp] = inc;
+    __syncthreads();
+    if (warp == 0) {
+        V t = lane < kWarps ? warp_tot[lane] : V(0);
+        V ti = t;
+#pragma unroll
+        for (int o = 1; o < kWarps; o <<= 1) {
+            V y = __shfl_up_sync(0xffffffffu, ti, o);
+            if (lane >= o) ti += y;
+        }
+        if (lane < kWarps) warp_tot[lane] = ti - t;   // exclusive warp offsets
+        if (lane == kWarps - 1) *total = ti;
+    }
+    __syncthreads();
+    V r = warp_tot[warp] + inc - x;
+    __syncthreads();
+    return r;
+}
+
+struct SelectArgs {
+    const void *q;
+    const float *mean;
+    const float *var;
+    int B, Hq, Hkv, Lq, T, d, block, nb, nq, G;
+    float scale;
+    float top_p;
+    int n_sink, n_local, k_min;
+    int32_t *idx;
+    int cap;
+    int32_t *count;
+    int *err;
+    int sort_cap;   // power of two >= the largest residual of any unit
+};
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kThreads) select_kernel(SelectArgs a) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    uint64_t *keys = reinterpret_cast<uint64_t *>(smem_raw);               // [sort_cap]
+    float *red = reinterpret_cast<float *>(keys + a.sort_cap);             // [kThreads * 8]
+    unsigned char *flag = reinterpret_cast<unsigned char *>(red + kThreads * 8); // [nb]
+    __shared__ double dtot[kWarps];
+    __shared__ double dsum;
+    __shared__ int itot[kWarps];
+    __shared__ int isum;
+    __shared__ float qbar_s[D];
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    // Heaviest units first: query block index descending.
+    const int i = a.nq - 1 - (int)(blockIdx.x % a.nq);
+    const int bh = (int)(blockIdx.x / a.nq);
+    const int b = bh / a.Hq, h = bh % a.Hq, g = h / a.G;
+    const size_t unit = (size_t)bh * a.nq + i;
+
+    // ---- pooled query: mean of the rows of query block i
+    {
+        constexpr int V = 16 / sizeof(T);
+        constexpr int CPR = D / V;             // 16-byte chunks per row
+        constexpr int RG = kThreads / CPR;     // row groups
+        const int r0 = i * a.block;
+        const int nr = min(a.block, a.Lq - r0);
+        const int c = tid % CPR, rg = tid / CPR;
+        float acc[V];
+#pragma unroll
+        for (int v = 0; v < V; ++v) acc[v] = 0.f;
+        const T *qrow = reinterpret_cast<const T *>(a.q) + ((size_t)bh * a.Lq + r0) * D + c * V;
+        for (int r = rg; r < nr; r += RG) {
+            uint4 u = __ldg(reinterpret_cast<const uint4 *>(qrow + (size_t)r * D));
+            if constexpr (sizeof(T) == 2) {
+                acc[0] += bf16lo(u.x); acc[1] += bf16hi(u.x); acc[2] += bf16lo(u.y);
+                acc[3] += bf16hi(u.y); acc[4] += bf16lo(u.z); acc[5] += bf16hi(u.z);
+                acc[6] += bf16lo(u.w); acc[7] += bf16hi(u.w);
+            } else {
+                acc[0] += __uint_as_float(u.x); acc[1] += __uint_as_float(u.y);
+                acc[2] += __uint_as_float(u.z); acc[3] += __uint_as_float(u.w);
+            }
+        }
+#pragma unroll
+        for (int v = 0; v < V; ++v) red[rg * D + c * V + v] = acc[v];
+        __syncthreads();
+        if (tid < D) {
+            float s = 0.f;
+            for (int r = 0; r < RG; ++r) s += red[r * D + tid];
+            qbar_s[tid] = s / (float)nr;
+        }
+        __syncthreads();
+    }
+
+    // ---- candidates
+    const int last_row = min((i + 1) * a.block, a.Lq);
+    const int jmax = (a.T - a.Lq + last_row - 1) / a.block;
+    const int r_lo = min(a.n_sink, jmax + 1);
+    const int r_hi = max(r_lo, jmax - a.n_local + 1);
+    const int nres = r_hi - r_lo;
+    int N = 1;
+    while (N < nres) N <<= 1;
+
+    // ---- fp32 scores of the residual candidates, one warp per candidate
+    {
+        constexpr int PL = D / 32;   // components per lane
+        float qv[PL], q2[PL];
+#pragma unroll
+        for (int c = 0; c < PL; ++c) {
+            qv[c] = qbar_s[lane * PL + c];
+            q2[c] = qv[c] * qv[c];
+        }
+        const float hs2 = 0.5f * a.scale * a.scale;
+        const float *mb = a.mean + ((size_t)b * a.Hkv + g) * a.nb * D + lane * PL;
+        const float *vb = a.var + ((size_t)b * a.Hkv + g) * a.nb * D + lane * PL;
+        for (int r = warp; r < nres; r += kWarps) {
+            const int j = r_lo + r;
+            float mu[PL], vr[PL];
+            if constexpr (PL == 4) {
+                float4 m4 = __ldg(reinterpret_cast<const float4 *>(mb + (size_t)j * D));
+                float4 v4 = __ldg(reinterpret_cast<const float4 *>(vb + (size_t)j * D));
+                mu[0] = m4.x; mu[1] = m4.y; mu[2] = m4.z; mu[3] = m4.w;
+                vr[0] = v4.x; vr[1] = v4.y; vr[2] = v4.z; vr[3] = v4.w;
+            } else {
+                float2 m2 = __ldg(reinterpret_cast<const float2 *>(mb + (size_t)j * D));
+                float2 v2 = __ldg(reinterpret_cast<const float2 *>(vb + (size_t)j * D));
+                mu[0] = m2.x; mu[1] = m2.y;
+                vr[0] = v2.x; vr[1] = v2.y;
+            }
+            float dot = 0.f, quad = 0.f;
+#pragma unroll
+            for (int c = 0; c < PL; ++c) {
+                dot = fmaf(qv[c], mu[c], dot);
+                quad = fmaf(q2[c], vr[c], quad);
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                dot += __shfl_xor_sync(0xffffffffu, dot, o);
+                quad += __shfl_xor_sync(0xffffffffu, quad, o);
+            }
+            if (lane == 0) {
+                const int nj = min(a.block, a.T - j * a.block);
+                const float l = a.scale * dot + log1pf(hs2 * quad) + logf((float)nj);
+                keys[r] = ((uint64_t)order_desc(l) << 32) | (uint32_t)j;
+            }
+        }
+        for (int r = nres + tid; r < N; r += kThreads) keys[r] = ~0ull;
+        for (int j = tid; j <= jmax; j += kThreads)
+            flag[j] = (j < r_lo || j >= r_hi) ? 1 : 0;     // reserved blocks
+        __syncthreads();
+    }
+
+    // ---- bitonic sort, ascending keys = descending score, ascending index
+    for (int kk = 2; kk <= N; kk <<= 1) {
+        for (int jj = kk >> 1; jj > 0; jj >>= 1) {
+            for (int x = tid; x < N; x += kThreads) {
+                const int y = x ^ jj;
+                if (y > x) {
+                    const uint64_t kx = keys[x], ky = keys[y];
+                    const bool up = (x & kk) == 0;
+                    if ((kx > ky) == up) {
+                        keys[x] = ky;
+                        keys[y] = kx;
+                    }
+                }
+            }
+            __syncthreads();
+        }
+    }
+
+    // ---- cut: keep while the mass accumulated before a block is below top_p
+    int nk = nres;
+    if (nres > 0 && a.top_p < 1.0f) {
+        const int per = (nres + kThreads - 1) / kThreads;      // contiguous segment per thread
+        const int s0 = min(tid * per, nres), s1 = min(s0 + per, nres);
+        const double mx = (double)key_score(keys[0]);
+        double local = 0.0;
+        for (int x = s0; x < s1; ++x) local += exp((double)key_score(keys[x]) - mx);
+        const double before = block_exclusive_scan<double>(local, dtot, &dsum);
+        const double total = dsum;
+        const double p = (double)a.top_p;
+        int kept_here = 0;
+        double cum = before;
+        for (int x = s0; x < s1; ++x) {
+            if (cum / total < p) ++kept_here;
+            cum += exp((double)key_score(keys[x]) - mx);
+        }
+        block_exclusive_scan<int>(kept_here, itot, &isum);
+        nk = isum;
+    }
+    nk = max(nk, min(a.k_min, nres));
+    for (int x = tid; x < nk; x += kThreads) flag[(int)(uint32_t)keys[x]] = 1;
+    __syncthreads();
+
+    // ---- ascending list of the kept blocks
+    {
+        const int n = jmax + 1;
+        const int per = (n + kThreads - 1) / kThreads;
+        const int s0 = min(tid * per, n), s1 = min(s0 + per, n);
+        int c = 0;
+        for (int j = s0; j < s1; ++j) c += flag[j];
+        int pos = block_exclusive_scan<int>(c, itot, &isum);
+        int32_t *out = a.idx + unit * a.cap;
+        for (int j = s0; j < s1; ++j)
+            if (flag[j]) out[pos++] = j;
+        if (tid == 0) a.count[unit] = isum;
+    }
+}
+
+template <typename T, int D>
+cudaError_t launch_t(const SelectArgs &a, cudaStream_t s) {
+    const size_t smem = (size_t)a.sort_cap * 8 + kThreads * 8 * sizeof(float) + (size_t)a.nb + 16;
+    auto kern = select_kernel<T, D>;
+    if (smem > 48 * 1024) {
+        cudaError_t e =
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    const unsigned grid = (unsigned)((size_t)a.B * a.Hq * a.nq);
+    kern<<<grid, kThreads, smem, s>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_select(const void *q, bool bf16, const float *mean, const float *var, int B,
+                          int Hq, int Hkv, int Lq, int T, int d, int block, float scale,
+                          float top_p, int n_sink, int n_local, int k_min, int32_t *idx, int cap,
+                          int32_t *count, int *err, cudaStream_t s) {
+    SelectArgs a;
+    a.q = q; a.mean = mean; a.var = var;
+    a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.Lq = Lq; a.T = T; a.d = d; a.block = block;
+    a.nb = (T + block - 1) / block;
+    a.nq = (Lq + block - 1) / block;
+    a.G = Hq / Hkv;
+    a.scale = scale; a.top_p = top_p;
+    a.n_sink = n_sink; a.n_local = n_local; a.k_min = k_min;
+    a.idx = idx; a.cap = cap; a.count = count; a.err = err;
+    int n = 1;
+    while (n < a.nb) n <<= 1;
+    a.sort_cap = n;
+    if (bf16) return d == 128 ? launch_t<__nv_bfloat16, 128>(a, s) : launch_t<__nv_bfloat16, 64>(a, s);
+    return d == 128 ? launch_t<float, 128>(a, s) : launch_t<float, 64>(a, s);
+}
+
+}  // namespace spa

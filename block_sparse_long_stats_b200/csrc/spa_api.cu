@@ -1,0 +1,222 @@
+// C-ABI entry points of libspa.so (declared in include/spa.h): host-side argument
+// validation, the per-device error word, and dispatch to the kernels.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+#include <string>
+
+#include "kernels.h"
+
+#define SPA_API extern "C" __attribute__((visibility("default")))
+
+namespace spa {
+namespace {
+
+__device__ int g_device_error = 0;
+
+constexpr int kMaxDevices = 64;
+int *g_err_ptr[kMaxDevices] = {nullptr};
+std::mutex g_err_mu;
+
+thread_local std::string t_last_error;
+
+spa_status fail(spa_status st, const std::string &msg) {
+    t_last_error = msg;
+    return st;
+}
+
+spa_status cuda_fail(cudaError_t e, const char *what) {
+    return fail(SPA_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+}
+
+// Device address of the error word of the current device (looked up once per
+// device; the symbol's host-side name is not a device address).
+int *device_error_ptr() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(g_err_mu);
+    if (!g_err_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+        g_err_ptr[dev] = static_cast<int *>(p);
+    }
+    return g_err_ptr[dev];
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+}  // namespace
+
+EncodeTiledFn encode_tiled_fn() {
+    static EncodeTiledFn fn = []() -> EncodeTiledFn {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        return reinterpret_cast<EncodeTiledFn>(p);
+    }();
+    return fn;
+}
+
+}  // namespace spa
+
+using namespace spa;
+
+SPA_API const char *spa_status_string(spa_status s) {
+    switch (s) {
+        case SPA_OK: return "ok";
+        case SPA_ERR_INVALID: return "invalid argument";
+        case SPA_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+        case SPA_ERR_CUDA: return "CUDA error";
+        case SPA_ERR_DEVICE: return "device-side error recorded";
+    }
+    return "unknown status";
+}
+
+SPA_API const char *spa_last_error(void) { return t_last_error.c_str(); }
+
+SPA_API spa_status spa_block_stats(const void *k, spa_dtype dt, int B, int Hkv, int T, int d,
+                                   int block, int blk_begin, int blk_end, float *mean, float *var,
+                                   spa_stream stream) {
+    t_last_error.clear();
+    if (!k || !mean || !var) return fail(SPA_ERR_INVALID, "null pointer");
+    if (B <= 0 || Hkv <= 0 || T <= 0 || d <= 0 || block <= 0)
+        return fail(SPA_ERR_INVALID, "sizes must be positive");
+    if (dt != SPA_F32 && dt != SPA_BF16) return fail(SPA_ERR_INVALID, "unknown dtype");
+    const int nb = ceil_div(T, block);
+    if (blk_begin < 0 || blk_end > nb || blk_begin > blk_end)
+        return fail(SPA_ERR_INVALID, "block range outside [0, nb]");
+    if (!aligned16(k) || !aligned16(mean) || !aligned16(var))
+        return fail(SPA_ERR_INVALID, "tensors must be 16-byte aligned");
+    if (d != 64 && d != 128) return fail(SPA_ERR_UNSUPPORTED, "d must be 64 or 128");
+    if (block != 16 && block != 32 && block != 64 && block != 128)
+        return fail(SPA_ERR_UNSUPPORTED, "block must be 16, 32, 64 or 128");
+    cudaError_t e = launch_block_stats(k, dt == SPA_BF16, B, Hkv, T, d, block, blk_begin, blk_end,
+                                       mean, var, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? SPA_OK : cuda_fail(e, "block_stats launch");
+}
+
+SPA_API spa_status spa_select(const void *q, spa_dtype dt, const float *mean, const float *var,
+                              int B, int Hq, int Hkv, int Lq, int T, int d, int block, float scale,
+                              float top_p, int n_sink, int n_local, int k_min, int32_t *idx,
+                              int cap, int32_t *count, spa_stream stream) {
+    t_last_error.clear();
+    if (!q || !mean || !var || !idx || !count) return fail(SPA_ERR_INVALID, "null pointer");
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Lq <= 0 || T <= 0 || d <= 0 || block <= 0)
+        return fail(SPA_ERR_INVALID, "sizes must be positive");
+    if (Hq % Hkv) return fail(SPA_ERR_INVALID, "Hq must be a multiple of Hkv");
+    if (Lq != T && Lq != 1) return fail(SPA_ERR_INVALID, "Lq must equal T (prefill) or 1 (decode)");
+    if (dt != SPA_F32 && dt != SPA_BF16) return fail(SPA_ERR_INVALID, "unknown dtype");
+    if (!(scale > 0.f) || !(top_p > 0.f)) return fail(SPA_ERR_INVALID, "scale and top_p must be > 0");
+    if (n_sink < 0 || n_local < 0 || k_min < 0)
+        return fail(SPA_ERR_INVALID, "n_sink, n_local and k_min must be >= 0");
+    const int nb = ceil_div(T, block);
+    if (cap < nb) return fail(SPA_ERR_INVALID, "cap must be >= nb");
+    if (!aligned16(q) || !aligned16(mean) || !aligned16(var))
+        return fail(SPA_ERR_INVALID, "tensors must be 16-byte aligned");
+    if (d != 64 && d != 128) return fail(SPA_ERR_UNSUPPORTED, "d must be 64 or 128");
+    if (block < 1 || block > 1024) return fail(SPA_ERR_UNSUPPORTED, "block must be in [1, 1024]");
+    if (nb > 16384) return fail(SPA_ERR_UNSUPPORTED, "more than 16384 key blocks");
+    int *err = device_error_ptr();
+    if (!err) return fail(SPA_ERR_CUDA, "device error word unavailable");
+    cudaError_t e = launch_select(q, dt == SPA_BF16, mean, var, B, Hq, Hkv, Lq, T, d, block, scale,
+                                  top_p, n_sink, n_local, k_min, idx, cap, count, err,
+                                  static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? SPA_OK : cuda_fail(e, "select launch");
+}
+
+SPA_API spa_status spa_sparse_attn_prefill(const void *q, const void *k, const void *v,
+                                           spa_dtype dt, int B, int Hq, int Hkv, int L, int d,
+                                           int block, const int32_t *idx, int cap,
+                                           const int32_t *count, float scale, void *out,
+                                           float *lse, spa_stream stream) {
+    t_last_error.clear();
+    if (!q || !k || !v || !idx || !count || !out) return fail(SPA_ERR_INVALID, "null pointer");
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || L <= 0 || d <= 0 || block <= 0)
+        return fail(SPA_ERR_INVALID, "sizes must be positive");
+    if (Hq % Hkv) return fail(SPA_ERR_INVALID, "Hq must be a multiple of Hkv");
+    if (dt != SPA_F32 && dt != SPA_BF16) return fail(SPA_ERR_INVALID, "unknown dtype");
+    if (!(scale > 0.f)) return fail(SPA_ERR_INVALID, "scale must be > 0");
+    if (cap < ceil_div(L, block)) return fail(SPA_ERR_INVALID, "cap must be >= nb");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+        return fail(SPA_ERR_INVALID, "tensors must be 16-byte aligned");
+    if (dt == SPA_BF16) {
+        if (d != 128) return fail(SPA_ERR_UNSUPPORTED, "bf16 prefill needs d = 128");
+        if (block != 64 && block != 128)
+            return fail(SPA_ERR_UNSUPPORTED, "bf16 prefill needs block 64 or 128");
+        if ((Hq / Hkv) % (128 / block))
+            return fail(SPA_ERR_UNSUPPORTED, "block 64 needs an even number of query heads per kv-head");
+    } else {
+        if (d != 64 && d != 128) return fail(SPA_ERR_UNSUPPORTED, "fp32 prefill needs d = 64 or 128");
+        if (block != 32 && block != 64 && block != 128)
+            return fail(SPA_ERR_UNSUPPORTED, "fp32 prefill needs block 32, 64 or 128");
+    }
+    int *err = device_error_ptr();
+    if (!err) return fail(SPA_ERR_CUDA, "device error word unavailable");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    if (dt == SPA_BF16) {
+        e = launch_prefill_tc(q, k, v, B, Hq, Hkv, L, block, idx, cap, count, scale, out, lse, err, s);
+        if (e == cudaErrorNotSupported)
+            return fail(SPA_ERR_UNSUPPORTED, "tensor map encoding unavailable");
+    } else {
+        e = launch_prefill_f32(static_cast<const float *>(q), static_cast<const float *>(k),
+                               static_cast<const float *>(v), B, Hq, Hkv, L, d, block, idx, cap,
+                               count, scale, static_cast<float *>(out), lse, err, s);
+    }
+    return e == cudaSuccess ? SPA_OK : cuda_fail(e, "prefill launch");
+}
+
+SPA_API size_t spa_decode_workspace_bytes(int B, int Hq, int Hkv, int T, int d, int block) {
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || T <= 0 || d <= 0 || block <= 0) return 0;
+    return decode_workspace_bytes(B, Hq, Hkv, T, d, block);
+}
+
+SPA_API spa_status spa_sparse_attn_decode(const void *q, const void *kc, const void *vc,
+                                          spa_dtype dt, int B, int Hq, int Hkv, int T, int d,
+                                          int block, const int32_t *idx, int cap,
+                                          const int32_t *count, float scale, void *workspace,
+                                          void *out, spa_stream stream) {
+    t_last_error.clear();
+    if (!q || !kc || !vc || !idx || !count || !workspace || !out)
+        return fail(SPA_ERR_INVALID, "null pointer");
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || T <= 0 || d <= 0 || block <= 0)
+        return fail(SPA_ERR_INVALID, "sizes must be positive");
+    if (Hq % Hkv) return fail(SPA_ERR_INVALID, "Hq must be a multiple of Hkv");
+    if (!(scale > 0.f)) return fail(SPA_ERR_INVALID, "scale must be > 0");
+    if (cap < ceil_div(T, block)) return fail(SPA_ERR_INVALID, "cap must be >= nb");
+    if (!aligned16(q) || !aligned16(kc) || !aligned16(vc) || !aligned16(workspace) ||
+        !aligned16(out))
+        return fail(SPA_ERR_INVALID, "tensors must be 16-byte aligned");
+    if (dt != SPA_BF16) return fail(SPA_ERR_UNSUPPORTED, "decode is bf16 only");
+    if (d != 128) return fail(SPA_ERR_UNSUPPORTED, "decode needs d = 128");
+    if (block != 16 && block != 32 && block != 64 && block != 128)
+        return fail(SPA_ERR_UNSUPPORTED, "decode needs block 16, 32, 64 or 128");
+    if (Hq / Hkv > 16) return fail(SPA_ERR_UNSUPPORTED, "decode supports up to 16 query heads per kv-head");
+    int *err = device_error_ptr();
+    if (!err) return fail(SPA_ERR_CUDA, "device error word unavailable");
+    cudaError_t e = launch_decode(q, kc, vc, B, Hq, Hkv, T, d, block, idx, cap, count, scale,
+                                  workspace, out, err, static_cast<cudaStream_t>(stream));
+    if (e == cudaErrorNotSupported) return fail(SPA_ERR_UNSUPPORTED, "tensor map encoding unavailable");
+    return e == cudaSuccess ? SPA_OK : cuda_fail(e, "decode launch");
+}
+
+SPA_API spa_status spa_get_device_error(int *code) {
+    t_last_error.clear();
+    if (!code) return fail(SPA_ERR_INVALID, "null pointer");
+    int *p = device_error_ptr();
+    if (!p) return fail(SPA_ERR_CUDA, "device error word unavailable");
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e, "synchronize");
+    int v = 0;
+    e = cudaMemcpy(&v, p, sizeof v, cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "read error word");
+    const int zero = 0;
+    e = cudaMemcpy(p, &zero, sizeof zero, cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return cuda_fail(e, "clear error word");
+    *code = v;
+    return v ? SPA_ERR_DEVICE : SPA_OK;
+}

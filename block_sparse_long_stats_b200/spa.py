@@ -1,0 +1,221 @@
+"""Thin ctypes binding of libspa.so (include/spa.h), with the same names.
+
+Argument marshalling only: every step runs in the CUDA kernels behind the C-ABI.
+PyTorch is used for device memory and the current stream. There is no CPU path:
+importing this module without a built libspa.so raises, and every call needs CUDA
+tensors.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+__all__ = ["SpaError", "lib", "spa_block_stats", "spa_select", "spa_sparse_attn_prefill",
+           "spa_decode_workspace_bytes", "spa_sparse_attn_decode", "spa_get_device_error",
+           "spa_status_string", "spa_last_error", "prefill", "decode", "LIB_PATH"]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libspa.so")
+
+SPA_F32, SPA_BF16 = 0, 1
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_F = ctypes.c_float
+
+_lib = None
+
+
+class SpaError(RuntimeError):
+    """A libspa call returned a non-zero spa_status."""
+
+    def __init__(self, fn: str, status: int, detail: str):
+        self.status = status
+        super().__init__(f"{fn}: {_status_name(status)} (status {status}): {detail}")
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libspa.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libspa.so not found at {LIB_PATH}; build it with "
+                              "`python -m block_sparse_long_stats_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        L.spa_block_stats.argtypes = [_P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P]
+        L.spa_select.argtypes = [_P, _I, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _F, _I, _I, _I,
+                                 _P, _I, _P, _P]
+        L.spa_sparse_attn_prefill.argtypes = [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _I, _P,
+                                              _F, _P, _P, _P]
+        L.spa_decode_workspace_bytes.argtypes = [_I, _I, _I, _I, _I, _I]
+        L.spa_decode_workspace_bytes.restype = ctypes.c_size_t
+        L.spa_sparse_attn_decode.argtypes = [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _I, _P,
+                                             _F, _P, _P, _P]
+        L.spa_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_int)]
+        L.spa_status_string.argtypes = [_I]
+        L.spa_status_string.restype = ctypes.c_char_p
+        L.spa_last_error.restype = ctypes.c_char_p
+        for f in ("spa_block_stats", "spa_select", "spa_sparse_attn_prefill",
+                  "spa_sparse_attn_decode", "spa_get_device_error"):
+            getattr(L, f).restype = _I
+        _lib = L
+    return _lib
+
+
+def _status_name(st: int) -> str:
+    return lib().spa_status_string(st).decode()
+
+
+def spa_status_string(status: int) -> str:
+    return _status_name(status)
+
+
+def spa_last_error() -> str:
+    return lib().spa_last_error().decode()
+
+
+def _check(fn: str, st: int):
+    if st != 0:
+        raise SpaError(fn, st, spa_last_error())
+
+
+def _ptr(t: torch.Tensor | None):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("libspa works on CUDA tensors only")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return SPA_BF16
+    if t.dtype == torch.float32:
+        return SPA_F32
+    raise ValueError(f"unsupported dtype {t.dtype}")
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def spa_block_stats(k: torch.Tensor, block: int, blk_begin: int = 0, blk_end: int | None = None,
+                    mean: torch.Tensor | None = None, var: torch.Tensor | None = None,
+                    stream=None):
+    """Per-block key mean and variance: k [B,Hkv,T,d] -> mean, var [B,Hkv,nb,d] fp32."""
+    B, Hkv, T, d = k.shape
+    nb = -(-T // block)
+    blk_end = nb if blk_end is None else blk_end
+    if mean is None:
+        mean = torch.empty((B, Hkv, nb, d), device=k.device, dtype=torch.float32)
+    if var is None:
+        var = torch.empty((B, Hkv, nb, d), device=k.device, dtype=torch.float32)
+    _check("spa_block_stats", lib().spa_block_stats(_ptr(k), _dt(k), B, Hkv, T, d, block,
+                                                    blk_begin, blk_end, _ptr(mean), _ptr(var),
+                                                    _stream(stream)))
+    return mean, var
+
+
+def spa_select(q: torch.Tensor, mean: torch.Tensor, var: torch.Tensor, T: int, block: int,
+               scale: float, top_p: float, n_sink: int = 1, n_local: int = 1, k_min: int = 0,
+               idx: torch.Tensor | None = None, count: torch.Tensor | None = None,
+               cap: int | None = None, stream=None):
+    """Kept-block lists: q [B,Hq,Lq,d] (Lq = T or 1) -> idx [B,Hq,nq,cap], count [B,Hq,nq]."""
+    B, Hq, Lq, d = q.shape
+    Hkv = mean.shape[1]
+    nb = -(-T // block)
+    nq = -(-Lq // block)
+    if idx is None:
+        cap = nb if cap is None else cap
+        idx = torch.empty((B, Hq, nq, cap), device=q.device, dtype=torch.int32)
+    cap = idx.shape[-1]
+    if count is None:
+        count = torch.empty((B, Hq, nq), device=q.device, dtype=torch.int32)
+    _check("spa_select", lib().spa_select(_ptr(q), _dt(q), _ptr(mean), _ptr(var), B, Hq, Hkv, Lq, T,
+                                          d, block, scale, top_p, n_sink, n_local, k_min,
+                                          _ptr(idx), cap, _ptr(count), _stream(stream)))
+    return idx, count
+
+
+def spa_sparse_attn_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block: int,
+                            idx: torch.Tensor, count: torch.Tensor, scale: float,
+                            out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
+                            want_lse: bool = False, stream=None):
+    """Block-sparse causal attention over the kept blocks. Returns (out, lse or None)."""
+    B, Hq, L, d = q.shape
+    Hkv = k.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq, L), device=q.device, dtype=torch.float32)
+    _check("spa_sparse_attn_prefill",
+           lib().spa_sparse_attn_prefill(_ptr(q), _ptr(k), _ptr(v), _dt(q), B, Hq, Hkv, L, d,
+                                         block, _ptr(idx), idx.shape[-1], _ptr(count), scale,
+                                         _ptr(out), _ptr(lse), _stream(stream)))
+    return out, lse
+
+
+def spa_decode_workspace_bytes(B: int, Hq: int, Hkv: int, T: int, d: int, block: int) -> int:
+    return int(lib().spa_decode_workspace_bytes(B, Hq, Hkv, T, d, block))
+
+
+def spa_sparse_attn_decode(q: torch.Tensor, kc: torch.Tensor, vc: torch.Tensor, block: int,
+                           idx: torch.Tensor, count: torch.Tensor, scale: float,
+                           workspace: torch.Tensor | None = None,
+                           out: torch.Tensor | None = None, stream=None):
+    """Decode attention for one query per sequence: q [B,Hq,1,d] -> out [B,Hq,1,d]."""
+    B, Hq, _, d = q.shape
+    Hkv, T = kc.shape[1], kc.shape[2]
+    if workspace is None:
+        n = spa_decode_workspace_bytes(B, Hq, Hkv, T, d, block)
+        workspace = torch.empty((max(n, 16),), device=q.device, dtype=torch.uint8)
+    if out is None:
+        out = torch.empty_like(q)
+    _check("spa_sparse_attn_decode",
+           lib().spa_sparse_attn_decode(_ptr(q), _ptr(kc), _ptr(vc), _dt(q), B, Hq, Hkv, T, d,
+                                        block, _ptr(idx), idx.shape[-1], _ptr(count), scale,
+                                        _ptr(workspace), _ptr(out), _stream(stream)))
+    return out
+
+
+def spa_get_device_error() -> int:
+    """Reads and clears the device error word (synchronises); 0 means no error."""
+    code = ctypes.c_int(0)
+    st = lib().spa_get_device_error(ctypes.byref(code))
+    if st not in (0, 4):
+        _check("spa_get_device_error", st)
+    return code.value
+
+
+def prefill(q, k, v, block: int, top_p: float, scale: float | None = None, n_sink: int = 1,
+            n_local: int = 1, k_min: int = 0, want_lse: bool = False, stream=None):
+    """The whole prefill path: block stats -> selection -> sparse attention.
+
+    Returns dict(out, lse, idx, count, mean, var).
+    """
+    T = k.shape[2]
+    scale = 1.0 / math.sqrt(q.shape[-1]) if scale is None else scale
+    mean, var = spa_block_stats(k, block, stream=stream)
+    idx, count = spa_select(q, mean, var, T, block, scale, top_p, n_sink, n_local, k_min,
+                            stream=stream)
+    out, lse = spa_sparse_attn_prefill(q, k, v, block, idx, count, scale, want_lse=want_lse,
+                                       stream=stream)
+    return {"out": out, "lse": lse, "idx": idx, "count": count, "mean": mean, "var": var}
+
+
+def decode(q, kc, vc, block: int, top_p: float, mean=None, var=None, scale: float | None = None,
+           n_sink: int = 1, n_local: int = 1, k_min: int = 0, workspace=None, stream=None):
+    """One decode step: (stats, if not given) -> selection -> sparse decode attention."""
+    T = kc.shape[2]
+    scale = 1.0 / math.sqrt(q.shape[-1]) if scale is None else scale
+    if mean is None or var is None:
+        mean, var = spa_block_stats(kc, block, stream=stream)
+    idx, count = spa_select(q, mean, var, T, block, scale, top_p, n_sink, n_local, k_min,
+                            stream=stream)
+    out = spa_sparse_attn_decode(q, kc, vc, block, idx, count, scale, workspace=workspace,
+                                 stream=stream)
+    return {"out": out, "idx": idx, "count": count, "mean": mean, "var": var}

@@ -1,0 +1,169 @@
+/*
+ * spa.h - C-ABI of libspa.so: selection-driven block-sparse causal attention on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The pipeline, per attention layer:
+ *   spa_block_stats  -> per-KV-block key mean and diagonal variance
+ *   spa_select       -> per (batch, query head, query block) kept-block list
+ *   spa_sparse_attn_prefill / spa_sparse_attn_decode -> exact attention over the
+ *                       kept blocks only
+ *
+ * Conventions shared by every call
+ *   - All tensors are dense, contiguous, row-major, in DEVICE memory, allocated and
+ *     owned by the caller. The library allocates nothing and keeps no per-call
+ *     state; it never frees or retains caller pointers.
+ *   - Layouts: Q [B, Hq, Lq, d]; K, V [B, Hkv, T, d]; block statistics
+ *     [B, Hkv, nb, d]; kept lists [B, Hq, nq, cap] (int32) with counts
+ *     [B, Hq, nq] (int32), where nb = ceil(T / block), nq = ceil(Lq / block).
+ *   - Query head h reads kv-head h / (Hq / Hkv) (grouped-query attention).
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy default
+ *     stream) and return as soon as the work is enqueued.
+ *   - Errors found on the host return before any launch: SPA_ERR_INVALID for null
+ *     pointers, non-positive sizes, Hq % Hkv != 0, cap < nb, top_p <= 0,
+ *     scale <= 0, or tensor bases not 16-byte aligned; SPA_ERR_UNSUPPORTED for
+ *     shapes this build has no kernel for. A failed launch returns SPA_ERR_CUDA.
+ *     Faults the kernels detect themselves (a kept-list entry out of range or not
+ *     ascending, a count outside [0, cap], a bounded wait that ran out) are
+ *     recorded in a device error word, read with spa_get_device_error; the kernel
+ *     skips the bad entry instead of touching memory out of bounds.
+ *   - No C++ exception crosses this interface.
+ */
+#ifndef SPA_H
+#define SPA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SPA_OK = 0,
+    SPA_ERR_INVALID = 1,      /* bad argument (host check) */
+    SPA_ERR_UNSUPPORTED = 2,  /* valid, but no kernel for this shape/dtype */
+    SPA_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed */
+    SPA_ERR_DEVICE = 4        /* a kernel recorded a device-side error */
+} spa_status;
+
+typedef enum { SPA_F32 = 0, SPA_BF16 = 1 } spa_dtype;
+
+/* Device-side error codes reported by spa_get_device_error. */
+#define SPA_DEVERR_NONE 0
+#define SPA_DEVERR_BAD_INDEX 1   /* kept-list entry out of range or not ascending: skipped */
+#define SPA_DEVERR_BAD_COUNT 2   /* count < 0 or > cap: clamped */
+#define SPA_DEVERR_TIMEOUT 3     /* a bounded wait on an mbarrier ran out: the kernel quit */
+
+typedef void *spa_stream; /* cudaStream_t */
+
+/*
+ * Block statistics. Follows "SPLA - Block Sparse Plus Linear Attention for Long
+ * Context Modeling", section 2.1: the first- and second-order statistics of the keys
+ * of each block, with the covariance taken diagonal:
+ *   mean[b,g,j,c] = (1/n_j) sum_{t in block j} k[b,g,t,c]
+ *   var [b,g,j,c] = (1/n_j) sum_{t in block j} (k[b,g,t,c] - mean[b,g,j,c])^2
+ * (population variance; n_j = block, or T - j*block for a shorter last block).
+ *   k      : [B, Hkv, T, d], dt = SPA_BF16 or SPA_F32
+ *   block  : 16, 32, 64 or 128;  d: 64 or 128
+ *   blk_begin, blk_end : only blocks j in [blk_begin, blk_end) are computed and
+ *            written (0 and nb for all; a decode step that appended tokens to the
+ *            last block passes nb-1 and nb). Other entries are left untouched.
+ *   mean, var : [B, Hkv, nb, d] fp32 outputs.
+ * Reads each key once; fp32 accumulation, two passes over the block in registers.
+ */
+spa_status spa_block_stats(const void *k, spa_dtype dt, int B, int Hkv, int T, int d, int block,
+                           int blk_begin, int blk_end, float *mean, float *var, spa_stream stream);
+
+/*
+ * Block selection. Follows "SPLA ...", section 2.1 (second-order Taylor block
+ * score), with the mean-pooled query block of "Sparsere Blok-Sparse Attention via
+ * Tokenpermutatie", section 4, and the dual top-p rule of "SpotAttention",
+ * section 3:
+ *   qbar_i   = mean of the query rows of query block i (decode: the one query)
+ *   l_{i,j}  = s qbar_i.mean_j + log(1 + s^2/2 sum_c qbar_i[c]^2 var_j[c]) + log n_j
+ *              for the candidate blocks j <= jmax(i) (prefill: jmax = i; decode:
+ *              jmax = nb - 1)
+ *   reserved = {0 .. n_sink-1} U {jmax-n_local+1 .. jmax}
+ *   residual = candidates minus reserved, sorted by l descending (equal l: smaller
+ *              j first); masses w_j = exp(l_j - max l) / sum; a block is kept while
+ *              the mass accumulated before it is below top_p (top_p >= 1 keeps all);
+ *              then at least min(k_min, |residual|) residual blocks are kept.
+ *   Output: reserved U kept, ASCENDING, in idx[b,h,i,0:count[b,h,i]]; entries
+ *   idx[b,h,i,count:cap] are left unspecified.
+ * Scores are fp32; masses and their prefix sums are fp64.
+ *   q      : [B, Hq, Lq, d], dt; Lq == T (prefill) or Lq == 1 (decode: the query
+ *            sits at position T-1 of a cache of length T)
+ *   mean, var : the outputs of spa_block_stats for the same K (fp32)
+ *   scale  : the softmax scale s (> 0), normally 1/sqrt(d)
+ *   idx    : [B, Hq, nq, cap] int32 output, cap >= nb;  count: [B, Hq, nq] int32
+ */
+spa_status spa_select(const void *q, spa_dtype dt, const float *mean, const float *var, int B,
+                      int Hq, int Hkv, int Lq, int T, int d, int block, float scale, float top_p,
+                      int n_sink, int n_local, int k_min, int32_t *idx, int cap, int32_t *count,
+                      spa_stream stream);
+
+/*
+ * Block-sparse causal prefill attention. Follows "S2O", sections 1 and 3 (index-
+ * driven loading of the selected key/value tiles; online-softmax state m, l, acc):
+ *   out[b,h,t,:] = sum_u softmax_u(s q_t.k_u) v_u over the keys u <= t whose block
+ *                  is in idx[b,h,t/block,0:count]
+ *   lse[b,h,t]   = log sum_u exp(s q_t.k_u) over the same keys (natural log)
+ * A row whose list keeps no visible key gets out = 0 and lse = -inf.
+ *   q, k, v : [B,Hq,L,d], [B,Hkv,L,d], [B,Hkv,L,d] (dt; L = T)
+ *   bf16: d = 128 and block 64 or 128 (TMA-staged tiles, tcgen05 MMAs with TMEM
+ *         accumulators, fp32 softmax, P rounded to bf16 for the PV product);
+ *   fp32: d 64 or 128, block 16..128 (fp32 FFMA throughout).
+ *   out    : [B,Hq,L,d], same dtype as q;  lse: [B,Hq,L] fp32 or NULL.
+ */
+spa_status spa_sparse_attn_prefill(const void *q, const void *k, const void *v, spa_dtype dt,
+                                   int B, int Hq, int Hkv, int L, int d, int block,
+                                   const int32_t *idx, int cap, const int32_t *count, float scale,
+                                   void *out, float *lse, spa_stream stream);
+
+/*
+ * Bytes of device workspace spa_sparse_attn_decode needs for these sizes (the
+ * split-KV partial states). The caller allocates it once and may reuse it for
+ * every step with the same sizes.
+ */
+size_t spa_decode_workspace_bytes(int B, int Hq, int Hkv, int T, int d, int block);
+
+/*
+ * Block-sparse decode attention: one new query per sequence against a KV cache of
+ * length T that already holds the new token (the query sits at position T-1). The
+ * pages describe decode as bound by re-reading the cache ("SpotAttention", problem
+ * statement and results); only the kept blocks are read.
+ *   out[b,h,:] = sum_u softmax_u(s q.k_u) v_u over u < T with block(u) in
+ *                idx[b,h,0,0:count[b,h,0]]
+ * Split-KV: every (b, kv-head) is cut into ranges of blocks; each range reads the
+ * union of the kept blocks of the group's query heads once and keeps one
+ * (m, l, acc) state per head; a combine kernel merges the ranges.
+ *   q      : [B, Hq, 1, d] bf16;  kc, vc: [B, Hkv, T, d] bf16;  d = 128
+ *   block  : 16, 32, 64 or 128
+ *   idx, count : from spa_select with Lq = 1 ([B,Hq,1,cap], [B,Hq,1])
+ *   workspace : >= spa_decode_workspace_bytes(...) bytes of device memory, 16-byte
+ *               aligned; overwritten
+ *   out    : [B, Hq, 1, d] bf16
+ */
+spa_status spa_sparse_attn_decode(const void *q, const void *kc, const void *vc, spa_dtype dt,
+                                  int B, int Hq, int Hkv, int T, int d, int block,
+                                  const int32_t *idx, int cap, const int32_t *count, float scale,
+                                  void *workspace, void *out, spa_stream stream);
+
+/*
+ * Reads and clears the device error word of the current device (one of
+ * SPA_DEVERR_*). Synchronises the device. Returns SPA_ERR_DEVICE when the word was
+ * non-zero, SPA_OK otherwise.
+ */
+spa_status spa_get_device_error(int *code);
+
+/* Static description of a status code. */
+const char *spa_status_string(spa_status status);
+
+/* Detail of the last error returned on the calling thread ("" if none). */
+const char *spa_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPA_H */

@@ -1,0 +1,128 @@
+"""The C-ABI library loads and exports every call include/spa.h declares, and the
+host-side checks reject bad arguments before any launch. CPU only: nothing here
+reaches a kernel or needs a device."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from block_sparse_long_stats_b200 import build as spa_build
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "spa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    path = spa_build.build()
+    return ctypes.CDLL(path)
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(spa_[a-z_]+)\s*\(", src)))
+
+
+def test_header_declares_the_pipeline_calls():
+    names = declared_functions()
+    for n in ("spa_block_stats", "spa_select", "spa_sparse_attn_prefill",
+              "spa_sparse_attn_decode", "spa_decode_workspace_bytes", "spa_get_device_error"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for n in declared_functions():
+        assert hasattr(lib, n), f"{n} declared in spa.h but not exported"
+
+
+def test_only_the_abi_is_exported():
+    out = subprocess.run(["nm", "-D", "--defined-only", spa_build.LIB], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {l.split()[-1] for l in out.splitlines() if " T " in l}
+    ours = {s for s in exported if s.startswith("spa_")}
+    assert ours == set(declared_functions())
+
+
+def test_status_strings(lib):
+    lib.spa_status_string.restype = ctypes.c_char_p
+    assert lib.spa_status_string(0) == b"ok"
+    assert lib.spa_status_string(1) == b"invalid argument"
+    assert lib.spa_status_string(2) == b"unsupported shape or dtype"
+
+
+P = ctypes.c_void_p
+FAKE = P(0x10000)   # aligned, never dereferenced: every call below fails a host check first
+
+
+def _last(lib):
+    lib.spa_last_error.restype = ctypes.c_char_p
+    return lib.spa_last_error().decode()
+
+
+def test_block_stats_host_checks(lib):
+    f = lib.spa_block_stats
+    f.argtypes = [P] + [ctypes.c_int] * 8 + [P, P, P]
+    assert f(None, 1, 1, 1, 64, 128, 64, 0, 1, FAKE, FAKE, None) == 1
+    assert f(FAKE, 1, 0, 1, 64, 128, 64, 0, 1, FAKE, FAKE, None) == 1
+    assert f(FAKE, 1, 1, 1, 64, 128, 64, 0, 2, FAKE, FAKE, None) == 1      # range beyond nb
+    assert "range" in _last(lib)
+    assert f(FAKE, 1, 1, 1, 64, 96, 64, 0, 1, FAKE, FAKE, None) == 2       # d = 96
+    assert f(FAKE, 1, 1, 1, 64, 128, 48, 0, 1, FAKE, FAKE, None) == 2      # block 48
+    assert f(P(0x10008), 1, 1, 1, 64, 128, 64, 0, 1, FAKE, FAKE, None) == 1  # misaligned
+
+
+def test_select_host_checks(lib):
+    f = lib.spa_select
+    I, F = ctypes.c_int, ctypes.c_float
+    f.argtypes = [P, I, P, P, I, I, I, I, I, I, I, F, F, I, I, I, P, I, P, P]
+    ok = dict(B=1, Hq=4, Hkv=2, Lq=256, T=256, d=128, block=64, scale=0.1, top_p=0.9, n_sink=1,
+              n_local=1, k_min=0, cap=4)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return f(FAKE, 1, FAKE, FAKE, a["B"], a["Hq"], a["Hkv"], a["Lq"], a["T"], a["d"],
+                 a["block"], a["scale"], a["top_p"], a["n_sink"], a["n_local"], a["k_min"], FAKE,
+                 a["cap"], FAKE, None)
+
+    assert call(Hq=3) == 1
+    assert call(Lq=100) == 1
+    assert call(top_p=0.0) == 1
+    assert call(scale=-1.0) == 1
+    assert call(cap=3) == 1
+    assert call(n_sink=-1) == 1
+    assert call(d=96) == 2
+
+
+def test_prefill_and_decode_host_checks(lib):
+    I, F = ctypes.c_int, ctypes.c_float
+    f = lib.spa_sparse_attn_prefill
+    f.argtypes = [P, P, P, I, I, I, I, I, I, I, P, I, P, F, P, P, P]
+    assert f(FAKE, FAKE, FAKE, 1, 1, 4, 2, 256, 96, 64, FAKE, 4, FAKE, 0.1, FAKE, None, None) == 2
+    assert f(FAKE, FAKE, FAKE, 1, 1, 4, 2, 256, 128, 32, FAKE, 8, FAKE, 0.1, FAKE, None, None) == 2
+    assert f(FAKE, FAKE, FAKE, 1, 1, 2, 2, 256, 128, 64, FAKE, 4, FAKE, 0.1, FAKE, None, None) == 2
+    assert f(FAKE, FAKE, FAKE, 1, 1, 4, 2, 256, 128, 64, FAKE, 3, FAKE, 0.1, FAKE, None, None) == 1
+    assert f(FAKE, FAKE, None, 1, 1, 4, 2, 256, 128, 64, FAKE, 4, FAKE, 0.1, FAKE, None, None) == 1
+    g = lib.spa_sparse_attn_decode
+    g.argtypes = [P, P, P, I, I, I, I, I, I, I, P, I, P, F, P, P, P]
+    assert g(FAKE, FAKE, FAKE, 0, 1, 4, 2, 256, 128, 16, FAKE, 16, FAKE, 0.1, FAKE, FAKE, None) == 2
+    assert g(FAKE, FAKE, FAKE, 1, 1, 4, 2, 256, 128, 16, FAKE, 15, FAKE, 0.1, FAKE, FAKE, None) == 1
+    assert g(FAKE, FAKE, FAKE, 1, 1, 4, 2, 256, 128, 16, FAKE, 16, FAKE, 0.1, None, FAKE, None) == 1
+
+
+def test_decode_workspace_size(lib):
+    f = lib.spa_decode_workspace_bytes
+    f.restype = ctypes.c_size_t
+    f.argtypes = [ctypes.c_int] * 6
+    n = f(16, 32, 8, 131072, 128, 16)
+    assert n > 0 and n % (16 * 32 * 130 * 4) == 0
+    assert f(0, 32, 8, 131072, 128, 16) == 0
+
+
+def test_binding_fails_loudly_without_cuda_tensors():
+    import torch
+    import block_sparse_long_stats_b200 as spa
+    k = torch.zeros((1, 1, 64, 128), dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        spa.spa_block_stats(k, 64)

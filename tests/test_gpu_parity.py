@@ -1,0 +1,297 @@
+"""Parity of the CUDA path (through the C-ABI) with the CPU oracle.
+
+Tolerances: kept lists bit-exact except excused near ties (counted); attention
+outputs max-abs 2e-2 for bf16 and 1e-4 for fp32; block statistics relative 1e-5.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import block_sparse_long_stats_b200 as spa
+from tests._parity import compare_lists, sample_rows, to_dev, to_host
+from workloads import PARITY_WORKLOADS, WORKLOADS, generate, widen
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"bf16": 2e-2, "f32": 1e-4}
+LSE_TOL = {"bf16": 2e-3, "f32": 1e-4}
+PREFILL = [k for k, w in PARITY_WORKLOADS.items() if w.mode == "prefill"]
+DECODE = [k for k, w in PARITY_WORKLOADS.items() if w.mode == "decode"]
+
+_cache = {}
+
+
+def inputs(w):
+    key = (w.name, w.T, w.B, w.block)
+    if key not in _cache:
+        x = generate(w)
+        _cache.clear()
+        _cache[key] = (x, {n: to_dev(a, w.dtype) for n, a in x.items()})
+    return _cache[key]
+
+
+def oracle_select(w, x):
+    return oracle.select(x["q"], x["k"], w.dtype, w.block, w.scale, w.top_p, w.n_sink,
+                         w.n_local, w.k_min)
+
+
+def assert_no_device_error():
+    assert spa.spa_get_device_error() == 0
+
+
+def check_lists(w, g_idx, g_cnt, sel, Lq):
+    r = compare_lists(g_idx.cpu().numpy(), g_cnt.cpu().numpy(), sel["idx"], sel["count"],
+                      sel["scores"], w.top_p, w.n_sink, w.n_local, Lq, w.T, w.block)
+    print(f"\n{w.name}: {r['units']} lists, {r['equal']} equal, {r['excused']} excused near ties")
+    assert not r["unexcused"], r["unexcused"][:3]
+    return r
+
+
+# ------------------------------------------------------------------ block statistics
+
+@pytest.mark.parametrize("key", list(PARITY_WORKLOADS))
+def test_block_stats_match_oracle(key):
+    w = PARITY_WORKLOADS[key]
+    x, dev = inputs(w)
+    mean, var = spa.spa_block_stats(dev["k"], w.block)
+    torch.cuda.synchronize()
+    om, ov = oracle.block_stats(x["k"], w.dtype, w.block)
+    np.testing.assert_allclose(mean.cpu().numpy(), om, rtol=1e-5, atol=1e-6)
+    np.testing.assert_allclose(var.cpu().numpy(), ov, rtol=1e-5, atol=1e-6)
+    assert_no_device_error()
+
+
+def test_block_stats_incremental_range_touches_only_its_blocks():
+    w = PARITY_WORKLOADS["d_bf16_blk16"]
+    x, dev = inputs(w)
+    full_m, full_v = spa.spa_block_stats(dev["k"], w.block)
+    m = torch.full_like(full_m, 7.0)
+    v = torch.full_like(full_v, 7.0)
+    nb = w.nb
+    spa.spa_block_stats(dev["k"], w.block, nb - 3, nb, mean=m, var=v)
+    torch.cuda.synchronize()
+    assert torch.equal(m[:, :, nb - 3:], full_m[:, :, nb - 3:])
+    assert torch.equal(v[:, :, nb - 3:], full_v[:, :, nb - 3:])
+    assert torch.all(m[:, :, :nb - 3] == 7.0) and torch.all(v[:, :, :nb - 3] == 7.0)
+
+
+# ------------------------------------------------------------------ selection
+
+@pytest.mark.parametrize("key", list(PARITY_WORKLOADS))
+def test_select_matches_oracle(key):
+    w = PARITY_WORKLOADS[key]
+    x, dev = inputs(w)
+    mean, var = spa.spa_block_stats(dev["k"], w.block)
+    idx, cnt = spa.spa_select(dev["q"], mean, var, w.T, w.block, w.scale, w.top_p, w.n_sink,
+                              w.n_local, w.k_min)
+    torch.cuda.synchronize()
+    check_lists(w, idx, cnt, oracle_select(w, x), w.Lq)
+    assert_no_device_error()
+
+
+@pytest.mark.parametrize("p,k_min,n_sink,n_local", [(1.0, 0, 1, 1), (1e-4, 0, 1, 1),
+                                                   (0.5, 3, 2, 2), (0.7, 0, 0, 0)])
+def test_select_rule_variants(p, k_min, n_sink, n_local):
+    w = PARITY_WORKLOADS["p_bf16_blk64"].with_(top_p=p, k_min=k_min, n_sink=n_sink,
+                                                 n_local=n_local)
+    x, dev = inputs(w)
+    mean, var = spa.spa_block_stats(dev["k"], w.block)
+    idx, cnt = spa.spa_select(dev["q"], mean, var, w.T, w.block, w.scale, p, n_sink, n_local,
+                              k_min)
+    torch.cuda.synchronize()
+    check_lists(w, idx, cnt, oracle_select(w, x), w.Lq)
+
+
+# ------------------------------------------------------------------ attention
+
+@pytest.mark.parametrize("key", PREFILL)
+def test_prefill_matches_oracle_on_oracle_lists(key):
+    w = PARITY_WORKLOADS[key]
+    x, dev = inputs(w)
+    sel = oracle_select(w, x)
+    idx = torch.from_numpy(sel["idx"]).cuda()
+    cnt = torch.from_numpy(sel["count"]).cuda()
+    out, lse = spa.spa_sparse_attn_prefill(dev["q"], dev["k"], dev["v"], w.block, idx, cnt,
+                                           w.scale, want_lse=True)
+    torch.cuda.synchronize()
+    o_out, o_lse = oracle.attention(x["q"], x["k"], x["v"], w.dtype, w.block, sel["idx"],
+                                    sel["count"], w.scale)
+    err = np.abs(to_host(out) - o_out).max()
+    print(f"\n{w.name}: max-abs {err:.3e}")
+    assert err <= TOL[w.dtype]
+    np.testing.assert_allclose(lse.cpu().numpy(), o_lse, rtol=0, atol=LSE_TOL[w.dtype])
+    assert_no_device_error()
+
+
+@pytest.mark.parametrize("key", PREFILL)
+def test_prefill_pipeline_matches_oracle(key):
+    w = PARITY_WORKLOADS[key]
+    x, dev = inputs(w)
+    r = spa.prefill(dev["q"], dev["k"], dev["v"], w.block, w.top_p, w.scale, w.n_sink, w.n_local,
+                    w.k_min)
+    torch.cuda.synchronize()
+    sel = oracle_select(w, x)
+    check_lists(w, r["idx"], r["count"], sel, w.Lq)
+    o_out, _ = oracle.attention(x["q"], x["k"], x["v"], w.dtype, w.block, sel["idx"],
+                                sel["count"], w.scale)
+    g_cnt = r["count"].cpu().numpy()
+    g_idx = r["idx"].cpu().numpy()
+    out = to_host(r["out"])
+    for b in range(w.B):
+        for h in range(w.Hq):
+            for i in range(w.nq):
+                c = g_cnt[b, h, i]
+                if c == sel["count"][b, h, i] and np.array_equal(g_idx[b, h, i, :c],
+                                                                  sel["idx"][b, h, i, :c]):
+                    rows = slice(i * w.block, min(w.T, (i + 1) * w.block))
+                    assert np.abs(out[b, h, rows] - o_out[b, h, rows]).max() <= TOL[w.dtype]
+
+
+def test_prefill_top_p_one_is_dense_causal_attention():
+    w = PARITY_WORKLOADS["p_bf16_blk128"]
+    x, dev = inputs(w)
+    r = spa.prefill(dev["q"], dev["k"], dev["v"], w.block, 1.0, w.scale)
+    torch.cuda.synchronize()
+    fi, fc = oracle.full_lists(w.B, w.Hq, w.T, w.T, w.block)
+    assert np.array_equal(r["count"].cpu().numpy(), fc)
+    dense, _ = oracle.attention(x["q"], x["k"], x["v"], w.dtype, w.block, fi, fc, w.scale)
+    assert np.abs(to_host(r["out"]) - dense).max() <= TOL[w.dtype]
+
+
+@pytest.mark.parametrize("L,block", [(64, 128), (128, 128), (130, 128), (200, 64), (64, 64),
+                                     (40, 64)])
+def test_prefill_short_and_ragged_sequences(L, block):
+    w = PARITY_WORKLOADS["p_bf16_blk128"].with_(T=L, block=block, B=1)
+    x, dev = inputs(w)
+    r = spa.prefill(dev["q"], dev["k"], dev["v"], w.block, w.top_p, w.scale)
+    torch.cuda.synchronize()
+    sel = oracle_select(w, x)
+    check_lists(w, r["idx"], r["count"], sel, w.Lq)
+    idx = torch.from_numpy(sel["idx"]).cuda()
+    cnt = torch.from_numpy(sel["count"]).cuda()
+    out, _ = spa.spa_sparse_attn_prefill(dev["q"], dev["k"], dev["v"], w.block, idx, cnt, w.scale)
+    torch.cuda.synchronize()
+    o_out, _ = oracle.attention(x["q"], x["k"], x["v"], w.dtype, w.block, sel["idx"],
+                                sel["count"], w.scale)
+    assert np.abs(to_host(out) - o_out).max() <= TOL[w.dtype]
+
+
+@pytest.mark.parametrize("key", DECODE)
+def test_decode_matches_oracle(key):
+    w = PARITY_WORKLOADS[key]
+    x, dev = inputs(w)
+    sel = oracle_select(w, x)
+    idx = torch.from_numpy(sel["idx"]).cuda()
+    cnt = torch.from_numpy(sel["count"]).cuda()
+    out = spa.spa_sparse_attn_decode(dev["q"], dev["k"], dev["v"], w.block, idx, cnt, w.scale)
+    torch.cuda.synchronize()
+    o_out, _ = oracle.attention(x["q"], x["k"], x["v"], w.dtype, w.block, sel["idx"],
+                                sel["count"], w.scale)
+    err = np.abs(to_host(out) - o_out).max()
+    print(f"\n{w.name}: max-abs {err:.3e}")
+    assert err <= TOL[w.dtype]
+    # the whole decode step through the binding
+    r = spa.decode(dev["q"], dev["k"], dev["v"], w.block, w.top_p, scale=w.scale)
+    torch.cuda.synchronize()
+    check_lists(w, r["idx"], r["count"], sel, 1)
+    assert_no_device_error()
+
+
+def test_corrupt_lists_are_reported_and_skipped():
+    w = PARITY_WORKLOADS["p_bf16_blk128"]
+    x, dev = inputs(w)
+    sel = oracle_select(w, x)
+    idx = sel["idx"].copy()
+    cnt = sel["count"].copy()
+    idx[0, 0, 5, 1] = 7          # beyond the causal limit of query block 5: skipped
+    idx[0, 1, 6, 2] = 0          # not ascending: skipped
+    ref_idx, ref_cnt = sel["idx"].copy(), sel["count"].copy()
+    for (b, h, i, p) in [(0, 0, 5, 1), (0, 1, 6, 2)]:
+        keep = [j for j in ref_idx[b, h, i, :ref_cnt[b, h, i]].tolist()
+                if j != sel["idx"][b, h, i, p]]
+        ref_idx[b, h, i, :len(keep)] = keep
+        ref_cnt[b, h, i] = len(keep)
+    out, _ = spa.spa_sparse_attn_prefill(dev["q"], dev["k"], dev["v"], w.block,
+                                         torch.from_numpy(idx).cuda(),
+                                         torch.from_numpy(cnt).cuda(), w.scale)
+    assert spa.spa_get_device_error() == 1      # SPA_DEVERR_BAD_INDEX
+    o_out, _ = oracle.attention(x["q"], x["k"], x["v"], w.dtype, w.block, ref_idx, ref_cnt,
+                                w.scale)
+    assert np.abs(to_host(out) - o_out).max() <= TOL[w.dtype]
+    cnt2 = sel["count"].copy()
+    cnt2[1, 3, 2] = w.nb + 5     # count beyond cap: clamped
+    spa.spa_sparse_attn_prefill(dev["q"], dev["k"], dev["v"], w.block,
+                                torch.from_numpy(sel["idx"]).cuda(),
+                                torch.from_numpy(cnt2).cuda(), w.scale)
+    assert spa.spa_get_device_error() == 2      # SPA_DEVERR_BAD_COUNT
+    assert spa.spa_get_device_error() == 0      # reading clears it
+
+
+# ------------------------------------------------------------------ headline workloads
+
+@pytest.mark.slow
+def test_tiny_fp32_workload_full():
+    w = WORKLOADS[1]
+    x = generate(w)
+    dev = {n: to_dev(a, w.dtype) for n, a in x.items()}
+    r = spa.prefill(dev["q"], dev["k"], dev["v"], w.block, w.top_p, w.scale, want_lse=True)
+    torch.cuda.synchronize()
+    sel = oracle_select(w, x)
+    check_lists(w, r["idx"], r["count"], sel, w.Lq)
+    o_out, o_lse = oracle.attention(x["q"], x["k"], x["v"], w.dtype, w.block, sel["idx"],
+                                    sel["count"], w.scale)
+    assert np.abs(to_host(r["out"]) - o_out).max() <= TOL["f32"]
+    assert np.abs(r["lse"].cpu().numpy() - o_lse).max() <= LSE_TOL["f32"]
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("cid", [2, 3, 4])
+def test_prefill_workload_full_size(cid):
+    w = WORKLOADS[cid]
+    x = generate(w)
+    dev = {n: to_dev(a, w.dtype) for n, a in x.items()}
+    r = spa.prefill(dev["q"], dev["k"], dev["v"], w.block, w.top_p, w.scale)
+    torch.cuda.synchronize()
+    sel = oracle_select(w, x)
+    res = check_lists(w, r["idx"], r["count"], sel, w.Lq)
+    kept = sel["count"].sum() / (w.B * w.Hq * w.nq * (w.nq + 1) / 2)
+    print(f"kept fraction of causal blocks: {kept:.3f}; excused {res['excused']}")
+    # outputs on sampled rows, both through the kernel on the oracle's lists and
+    # through the full pipeline where the lists agree
+    idx = torch.from_numpy(sel["idx"]).cuda()
+    cnt = torch.from_numpy(sel["count"]).cuda()
+    out, _ = spa.spa_sparse_attn_prefill(dev["q"], dev["k"], dev["v"], w.block, idx, cnt, w.scale)
+    torch.cuda.synchronize()
+    rows = sample_rows(w.B, w.Hq, w.T, w.block, 96, cid)
+    o_rows, _ = oracle.attention(x["q"], x["k"], x["v"], w.dtype, w.block, sel["idx"],
+                                 sel["count"], w.scale, rows=rows)
+    g_rows = to_host(out.reshape(-1, w.d)[torch.from_numpy(rows).cuda()])
+    err = np.abs(g_rows - o_rows).max()
+    print(f"{w.name}: sampled max-abs {err:.3e}")
+    assert err <= TOL[w.dtype]
+    assert_no_device_error()
+
+
+@pytest.mark.slow
+def test_decode_workload_full_size():
+    w = WORKLOADS[5]
+    x = generate(w)
+    dev = {n: to_dev(a, w.dtype) for n, a in x.items()}
+    r = spa.decode(dev["q"], dev["k"], dev["v"], w.block, w.top_p, scale=w.scale)
+    torch.cuda.synchronize()
+    sel = oracle_select(w, x)
+    res = check_lists(w, r["idx"], r["count"], sel, 1)
+    print(f"kept fraction {sel['count'].mean() / w.nb:.3f}; excused {res['excused']}")
+    idx = torch.from_numpy(sel["idx"]).cuda()
+    cnt = torch.from_numpy(sel["count"]).cuda()
+    out = spa.spa_sparse_attn_decode(dev["q"], dev["k"], dev["v"], w.block, idx, cnt, w.scale)
+    torch.cuda.synchronize()
+    o_out, _ = oracle.attention(x["q"], x["k"], x["v"], w.dtype, w.block, sel["idx"],
+                                sel["count"], w.scale)
+    err = np.abs(to_host(out) - o_out).max()
+    print(f"{w.name}: max-abs {err:.3e}")
+    assert err <= TOL[w.dtype]
+    assert_no_device_error()
