@@ -112,7 +112,7 @@ spa_status spa_select(const void *q, spa_dtype dt, const float *mean, const floa
  *   q, k, v : [B,Hq,L,d], [B,Hkv,L,d], [B,Hkv,L,d] (dt; L = T)
  *   bf16: d = 128 and block 64 or 128 (TMA-staged tiles, tcgen05 MMAs with TMEM
  *         accumulators, fp32 softmax, P rounded to bf16 for the PV product);
- *   fp32: d 64 or 128, block 16..128 (fp32 FFMA throughout).
+ *   fp32: d 64 or 128, block 32, 64 or 128 (fp32 FFMA throughout).
  *   out    : [B,Hq,L,d], same dtype as q;  lse: [B,Hq,L] fp32 or NULL.
  */
 spa_status spa_sparse_attn_prefill(const void *q, const void *k, const void *v, spa_dtype dt,
