@@ -428,3 +428,107 @@ cudaError_t launch_decode(const void *q, const void *kc, const void *vc, int B, 
 }
 
 }  // namespace spa
+
+// ---------------------------------------------------------------------------
+// Decode without caller-provided workspace.
+//
+// Some callers cannot allocate device memory for this call: a plugin or custom-op
+// interface that hands the op only its input and output buffers, or a serving loop
+// that must not call cudaMalloc on its hot path (cudaMalloc can synchronise the
+// device and stall other streams, and a caching allocator may already hold all the
+// free memory). For them spa_sparse_attn_decode_noalloc keeps the split-KV partial
+// states in the file-scope device array below instead of a caller workspace.
+//
+// The array's size is fixed at build time (kNoallocScratchBytes); every GPU that
+// loads the library holds that much device memory until the process exits. In host
+// code `g_decode_scratch` names a host-side stand-in, not a device address, so its
+// device address is looked up once per device with cudaGetSymbolAddress (with that
+// device current) on the first call made on the device; that first call should
+// therefore come before any stream capture. All calls on a device share the one
+// array: two calls whose kernels overlap on the GPU (different streams, no ordering
+// between them) race on it. Each call overwrites every partial state it later reads,
+// so nothing needs clearing between calls.
+// ---------------------------------------------------------------------------
+#include <stdio.h>
+
+#include <mutex>
+
+namespace spa {
+namespace {
+
+constexpr size_t kNoallocScratchBytes = 8u << 20;   // 8 MiB per device
+static __device__ __align__(256) unsigned char g_decode_scratch[kNoallocScratchBytes];
+
+constexpr int kNoallocMaxDevices = 64;
+void *g_scratch_addr[kNoallocMaxDevices] = {nullptr};
+std::mutex g_scratch_mu;
+
+spa_status noalloc_fail(spa_status st, const char *msg) {
+    record_last_error(msg);
+    return st;
+}
+
+}  // namespace
+}  // namespace spa
+
+extern "C" __attribute__((visibility("default"))) spa_status spa_sparse_attn_decode_noalloc(
+    const void *q, const void *kc, const void *vc, spa_dtype dt, int B, int Hq, int Hkv, int T,
+    int d, int block, const int32_t *idx, int cap, const int32_t *count, float scale, void *out,
+    spa_stream stream) {
+    using namespace spa;
+    record_last_error("");
+    if (!q || !kc || !vc || !idx || !count || !out) return noalloc_fail(SPA_ERR_INVALID, "null pointer");
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || T <= 0 || d <= 0 || block <= 0)
+        return noalloc_fail(SPA_ERR_INVALID, "sizes must be positive");
+    if (Hq % Hkv) return noalloc_fail(SPA_ERR_INVALID, "Hq must be a multiple of Hkv");
+    if (!(scale > 0.f)) return noalloc_fail(SPA_ERR_INVALID, "scale must be > 0");
+    if (cap < (T + block - 1) / block) return noalloc_fail(SPA_ERR_INVALID, "cap must be >= nb");
+    const uintptr_t mis = (reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(kc) |
+                           reinterpret_cast<uintptr_t>(vc) | reinterpret_cast<uintptr_t>(out)) & 15u;
+    if (mis) return noalloc_fail(SPA_ERR_INVALID, "tensors must be 16-byte aligned");
+    if (dt != SPA_BF16) return noalloc_fail(SPA_ERR_UNSUPPORTED, "decode is bf16 only");
+    if (d != 128) return noalloc_fail(SPA_ERR_UNSUPPORTED, "decode needs d = 128");
+    if (block != 16 && block != 32 && block != 64 && block != 128)
+        return noalloc_fail(SPA_ERR_UNSUPPORTED, "decode needs block 16, 32, 64 or 128");
+    if (Hq / Hkv > 16)
+        return noalloc_fail(SPA_ERR_UNSUPPORTED, "decode supports up to 16 query heads per kv-head");
+    const size_t need = decode_workspace_bytes(B, Hq, Hkv, T, d, block);
+    if (need > kNoallocScratchBytes) {
+        char msg[200];
+        snprintf(msg, sizeof msg,
+                 "these sizes need %zu bytes of scratch; the built-in maximum is %zu bytes "
+                 "(use spa_sparse_attn_decode with a caller workspace)",
+                 need, kNoallocScratchBytes);
+        return noalloc_fail(SPA_ERR_UNSUPPORTED, msg);
+    }
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoallocMaxDevices)
+        return noalloc_fail(SPA_ERR_CUDA, "no current CUDA device");
+    void *scratch = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_scratch_mu);
+        if (!g_scratch_addr[dev]) {
+            void *p = nullptr;
+            const cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
+            if (e != cudaSuccess || !p) {
+                char msg[200];
+                snprintf(msg, sizeof msg, "cudaGetSymbolAddress: %s", cudaGetErrorString(e));
+                return noalloc_fail(SPA_ERR_CUDA, msg);
+            }
+            g_scratch_addr[dev] = p;
+        }
+        scratch = g_scratch_addr[dev];
+    }
+    int *err = device_error_word();
+    if (!err) return noalloc_fail(SPA_ERR_CUDA, "device error word unavailable");
+    const cudaError_t e = launch_decode(q, kc, vc, B, Hq, Hkv, T, d, block, idx, cap, count, scale,
+                                        scratch, out, err, static_cast<cudaStream_t>(stream));
+    if (e == cudaErrorNotSupported)
+        return noalloc_fail(SPA_ERR_UNSUPPORTED, "tensor map encoding unavailable");
+    if (e != cudaSuccess) {
+        char msg[200];
+        snprintf(msg, sizeof msg, "decode launch: %s", cudaGetErrorString(e));
+        return noalloc_fail(SPA_ERR_CUDA, msg);
+    }
+    return SPA_OK;
+}

@@ -38,6 +38,11 @@ cudaError_t launch_decode(const void *q, const void *kc, const void *vc, int B, 
                           const int32_t *count, float scale, void *workspace, void *out, int *err,
                           cudaStream_t s);
 
+// Device address of the current device's error word (looked up once per device),
+// and the per-thread detail string spa_last_error returns; both live in spa_api.cu.
+int *device_error_word();
+void record_last_error(const char *msg);
+
 // Driver entry point for cuTensorMapEncodeTiled (resolved once through the runtime).
 using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
                                    const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,

@@ -48,6 +48,9 @@ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
 }  // namespace
 
+int *device_error_word() { return device_error_ptr(); }
+void record_last_error(const char *msg) { t_last_error = msg; }
+
 EncodeTiledFn encode_tiled_fn() {
     static EncodeTiledFn fn = []() -> EncodeTiledFn {
         void *p = nullptr;

@@ -150,6 +150,32 @@ spa_status spa_sparse_attn_decode(const void *q, const void *kc, const void *vc,
                                   void *workspace, void *out, spa_stream stream);
 
 /*
+ * spa_sparse_attn_decode without a caller workspace. The pages have no counterpart
+ * to this call: it exists for callers that cannot allocate device memory for it,
+ * such as a plugin or custom-op interface that passes the op only its input and
+ * output buffers, or a serving loop that must not call cudaMalloc on its hot path
+ * (cudaMalloc can synchronise the device and stall other streams, and a caching
+ * allocator may already hold all free memory).
+ *   Arguments, layouts and results are those of spa_sparse_attn_decode, minus the
+ *   workspace. The split-KV partial states live instead in a device array of
+ *   8 MiB compiled into the library; every GPU that loads the library holds it
+ *   until the process exits. Sizes whose spa_decode_workspace_bytes exceeds
+ *   8 MiB (8388608 bytes) are rejected with SPA_ERR_UNSUPPORTED and a message in
+ *   spa_last_error. The call allocates nothing.
+ *   The first call on a device looks up the array's device address (once per
+ *   device, with that device current); make that first call before any stream
+ *   capture. All calls on a device share the one array: calls whose kernels may
+ *   overlap on the GPU (different streams with no ordering between them) race on
+ *   it. Every call overwrites all the partial states it reads, so nothing carries
+ *   over from one call to the next.
+ */
+spa_status spa_sparse_attn_decode_noalloc(const void *q, const void *kc, const void *vc,
+                                          spa_dtype dt, int B, int Hq, int Hkv, int T, int d,
+                                          int block, const int32_t *idx, int cap,
+                                          const int32_t *count, float scale, void *out,
+                                          spa_stream stream);
+
+/*
  * Reads and clears the device error word of the current device (one of
  * SPA_DEVERR_*). Synchronises the device. Returns SPA_ERR_DEVICE when the word was
  * non-zero, SPA_OK otherwise.
