@@ -252,27 +252,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         while (cur.next(j, mask, a.err, false)) {
             if (!mbar_wait(&s_full, n & 1, a.err)) { ok = false; break; }
             tc_fence_after();
+            // All column loads in flight, then one wait.
             float x[BLK];
 #pragma unroll
-            for (int c = 0; c < BLK / 32; ++c) {
-                uint32_t v[32];
-                tmem_ld32(t_s + lane_off + c * 32, v);
-                tc_wait_ld();
-#pragma unroll
-                for (int e = 0; e < 32; ++e) x[c * 32 + e] = __uint_as_float(v[e]);
-            }
+            for (int c = 0; c < BLK / 32; ++c) tmem_ld32f(t_s + lane_off + c * 32, x + c * 32);
+            tc_wait_ld();
             tc_fence_before();
             mbar_arrive(&s_free);
 
+            // Masking only where it can apply (warp-uniform: a warp's rows share a head).
             const bool keep = (mask >> rg) & 1u;
-            const int lim = (j == i) ? rr : BLK - 1;          // causal limit inside the block
-            const int lim_t = min(lim, a.L - 1 - j * BLK);    // short last block
-            float mx = -INFINITY;
+            const bool whole = keep && j != i && (j + 1) * BLK <= a.L;
+            if (!whole) {
+                const int lim = (j == i) ? rr : BLK - 1;          // causal limit inside the block
+                const int lim_t = min(lim, a.L - 1 - j * BLK);    // short last block
 #pragma unroll
-            for (int c = 0; c < BLK; ++c) {
-                x[c] = (keep && c <= lim_t) ? x[c] * a.scale_log2 : -INFINITY;
-                mx = fmaxf(mx, x[c]);
+                for (int c = 0; c < BLK; ++c) x[c] = (keep && c <= lim_t) ? x[c] : -INFINITY;
             }
+            // Row max of the raw scores with 8 independent chains.
+            float mp[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) mp[e] = x[e];
+#pragma unroll
+            for (int c = 8; c < BLK; ++c) mp[c & 7] = fmaxf(mp[c & 7], x[c]);
+            const float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
+                                   fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7]))) *
+                             a.scale_log2;                 // log2 units
             float alpha = 1.f;
             bool rescale = false;
             if (mx > m_used + kRescaleThreshold) {
@@ -281,26 +286,34 @@ __global__ void __launch_bounds__(kThreads, 1)
                 m_used = mx;
             }
             const float base = m_used == -INFINITY ? 0.f : m_used;
-            float rs = 0.f;
+            // p = 2^(s * scale * log2 e - m): one FFMA and one MUFU op per score;
+            // the row sum with 8 independent chains.
+            float sp[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) sp[e] = 0.f;
 #pragma unroll
             for (int c = 0; c < BLK; ++c) {
-                x[c] = fast_exp2(x[c] - base);
-                rs += x[c];
+                x[c] = fast_exp2(fmaf(x[c], a.scale_log2, -base));
+                sp[c & 7] += x[c];
             }
+            const float rs = ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
+            uint32_t pk[BLK / 2];   // P as bf16 pairs (frees the fp32 scores before the rescale)
+#pragma unroll
+            for (int c = 0; c < BLK / 2; ++c) pk[c] = pack_bf16x2(x[2 * c], x[2 * c + 1]);
             l = l * alpha + rs;
 
             if (n > 0) {
                 if (!mbar_wait(&o_done, (n - 1) & 1, a.err)) { ok = false; break; }
                 tc_fence_after();
-                if (__any_sync(0xffffffffu, rescale)) {
-#pragma unroll
+                if (__any_sync(0xffffffffu, rescale)) {   // rare: the max grew by > 8
+#pragma unroll 1
                     for (int c = 0; c < kD / 32; ++c) {
-                        uint32_t v[32];
-                        tmem_ld32(t_o + lane_off + c * 32, v);
+                        uint32_t o0[32];
+                        tmem_ld32(t_o + lane_off + c * 32, o0);
                         tc_wait_ld();
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
-                        tmem_st32(t_o + lane_off + c * 32, v);
+                        for (int e = 0; e < 32; ++e) o0[e] = __float_as_uint(__uint_as_float(o0[e]) * alpha);
+                        tmem_st32(t_o + lane_off + c * 32, o0);
                     }
                     tc_wait_st();
                 }
@@ -308,11 +321,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // P row -> shared memory, bf16, K-major 128-byte swizzle (64 keys per half)
 #pragma unroll
             for (int q8 = 0; q8 < BLK / 8; ++q8) {
-                uint4 w;
-                w.x = pack_bf16x2(x[q8 * 8 + 0], x[q8 * 8 + 1]);
-                w.y = pack_bf16x2(x[q8 * 8 + 2], x[q8 * 8 + 3]);
-                w.z = pack_bf16x2(x[q8 * 8 + 4], x[q8 * 8 + 5]);
-                w.w = pack_bf16x2(x[q8 * 8 + 6], x[q8 * 8 + 7]);
+                const uint4 w = make_uint4(pk[4 * q8], pk[4 * q8 + 1], pk[4 * q8 + 2], pk[4 * q8 + 3]);
                 const int half = q8 >> 3, cq = q8 & 7;
                 *reinterpret_cast<uint4 *>(prow + half * 16384 + ((cq ^ (r & 7)) << 4)) = w;
             }
