@@ -12,13 +12,19 @@
 //   warps 0-3 : softmax; thread r owns query row r = TMEM lane r
 //   warp 4    : TMA producer (Q once; K_j and V_j per kept block into a ring)
 //   warp 5    : TMEM allocator and single-thread tcgen05.mma issuer
-// TMEM: S = Q K_j^T in columns [0, 128), O in columns [128, 256), fp32.
-// Per kept block n the issuer runs S(n) = Q K^T (8 MMAs, K = 16 each, over
-// d = 128) as soon as the softmax has read S(n-1), then O += P(n-1) V(n-1) once P
-// is in shared memory. The softmax scales by s*log2(e), takes exp2, keeps the
-// running max m lazily (O is rescaled only when the max grows by more than 8, in
-// log2 units), and writes P as bf16 in the 128-byte-swizzled K-major layout the
-// MMA reads. Epilogue: O / l from TMEM to bf16 rows, lse = (m + log2 l) ln 2.
+// TMEM (fp32 columns): S_lo [0,128), S_hi [128,256), P [256,256+BLK/2) as bf16
+// pairs, O [384,512).
+//
+// The MMA forms follow measured tcgen05 rates on B200: a chain of MMAs into one
+// accumulator pays a fixed latency per instruction, so S = Q K^T is split over the
+// two halves of d into two accumulators whose MMAs are issued interleaved (the
+// softmax adds them); and P V reads P from tensor memory (A operand in TMEM, V
+// from its TMA layout as an MN-major B), the fastest form for that product.
+// Per kept block n the issuer runs S(n) as soon as the softmax has read S(n-1),
+// then P(n-1) V once P(n-1) is in TMEM. The softmax scales by s*log2(e), takes
+// exp2, keeps the running max lazily (O is rescaled only when the max grows by
+// more than 8, in log2 units) and writes P once the previous P V has finished.
+// Epilogue: O / l from TMEM to bf16 rows, lse = (m + log2 l) ln 2.
 #include <math.h>
 
 #include "kernels.h"
@@ -28,7 +34,6 @@ namespace {
 
 constexpr int kD = 128;
 constexpr int kThreads = 192;
-constexpr int kStages = 2;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
@@ -36,15 +41,15 @@ constexpr float kRescaleThreshold = 8.0f;   // log2 units
 template <int BLK>
 struct Cfg {
     static constexpr int HPT = 128 / BLK;               // heads stacked in the M = 128 tile
+    static constexpr int STAGES = BLK == 128 ? 3 : 4;   // K/V ring depth
     static constexpr int Q_BYTES = 128 * kD * 2;        // 32 KB: two 64-column halves
     static constexpr int KV_BYTES = BLK * kD * 2;       // one K or V tile
     static constexpr int KV_HALF = BLK * 128;           // one 64-column half of it
-    static constexpr int P_BYTES = 128 * BLK * 2;
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_K = OFF_Q + Q_BYTES;
-    static constexpr int OFF_V = OFF_K + kStages * KV_BYTES;
-    static constexpr int OFF_P = OFF_V + kStages * KV_BYTES;
-    static constexpr int SMEM = OFF_P + P_BYTES;
+    static constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
+    static constexpr int SMEM = OFF_V + STAGES * KV_BYTES;
+    static constexpr uint32_t T_SLO = 0, T_SHI = 128, T_P = 256, T_O = 384;
     static constexpr uint32_t IDESC_S = idesc_bf16(128, BLK, false);
     static constexpr uint32_t IDESC_O = idesc_bf16(128, kD, true);
 };
@@ -65,7 +70,7 @@ struct PrefillArgs {
 template <int HPT>
 struct Cursor {
     const int32_t *lst[HPT];
-    int cnt[HPT], pos[HPT], last[HPT];
+    int cnt[HPT], pos[HPT], last[HPT], pre[HPT];   // pre: the entry at pos, loaded ahead
     int jmax;
 
     __device__ void init(const PrefillArgs &a, int b, int h0, int i, bool report) {
@@ -82,7 +87,12 @@ struct Cursor {
             cnt[r] = c;
             pos[r] = 0;
             last[r] = -1;
+            pre[r] = c > 0 ? __ldg(lst[r]) : 0;
         }
+    }
+    __device__ void advance(int r) {
+        ++pos[r];
+        pre[r] = pos[r] < cnt[r] ? __ldg(lst[r] + pos[r]) : 0;
     }
     __device__ bool next(int &j, uint32_t &mask, int *err, bool report) {
         int cand[HPT];
@@ -91,13 +101,13 @@ struct Cursor {
         for (int r = 0; r < HPT; ++r) {
             cand[r] = 0x7fffffff;
             while (pos[r] < cnt[r]) {
-                const int x = __ldg(lst[r] + pos[r]);
+                const int x = pre[r];
                 if (x > last[r] && x <= jmax) {
                     cand[r] = x;
                     break;
                 }
                 if (report) set_error(err, SPA_DEVERR_BAD_INDEX);
-                ++pos[r];
+                advance(r);
             }
             j = min(j, cand[r]);
         }
@@ -108,7 +118,7 @@ struct Cursor {
             if (cand[r] == j) {
                 mask |= 1u << r;
                 last[r] = j;
-                ++pos[r];
+                advance(r);
             }
         }
         return true;
@@ -121,11 +131,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                       const __grid_constant__ CUtensorMap tv, PrefillArgs a) {
     using C = Cfg<BLK>;
     constexpr int HPT = C::HPT;
+    constexpr int ST = C::STAGES;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char *smem = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    __shared__ uint64_t bar_q, full_k[kStages], full_v[kStages], empty_k[kStages],
-        empty_v[kStages], s_full, s_free, p_ready, o_done;
+    __shared__ uint64_t bar_q, full_k[ST], full_v[ST], empty_k[ST], empty_v[ST], s_full, s_free,
+        p_ready, o_done;
     __shared__ uint32_t tmem_slot;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -140,7 +151,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (tid == 0) {
         mbar_init(&bar_q, 1);
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < ST; ++s) {
             mbar_init(&full_k[s], 1);
             mbar_init(&full_v[s], 1);
             mbar_init(&empty_k[s], 1);
@@ -152,12 +163,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&o_done, 1);
         fence_mbar_init();
     }
-    if (warp == 5) tmem_alloc(&tmem_slot, 256);
+    if (warp == 5) tmem_alloc(&tmem_slot, 512);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tmem_slot;
-    const uint32_t t_s = tmem, t_o = tmem + 128;
 
     Cursor<HPT> cur;
     if (warp == 4) {
@@ -178,8 +188,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             int j;
             uint32_t mask;
             for (int n = 0; cur.next(j, mask, a.err, true); ++n) {
-                const int s = n % kStages;
-                const uint32_t ph = (n / kStages) & 1;
+                const int s = n % ST;
+                const uint32_t ph = (n / ST) & 1;
                 unsigned char *kt = smem + C::OFF_K + s * C::KV_BYTES;
                 unsigned char *vt = smem + C::OFF_V + s * C::KV_BYTES;
                 if (!mbar_wait(&empty_k[s], ph ^ 1, a.err)) break;
@@ -197,37 +207,40 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             cur.init(a, b, h0, i, false);
             const uint32_t q_base = smem_u32(smem + C::OFF_Q);
-            const uint32_t p_base = smem_u32(smem + C::OFF_P);
             bool ok = mbar_wait(&bar_q, 0, a.err);
             int n = 0, j;
             uint32_t mask;
             auto issue_pv = [&](int m) -> bool {
-                const int s = m % kStages;
+                const int s = m % ST;
                 if (!mbar_wait(&p_ready, m & 1, a.err)) return false;
-                if (!mbar_wait(&full_v[s], (m / kStages) & 1, a.err)) return false;
+                if (!mbar_wait(&full_v[s], (m / ST) & 1, a.err)) return false;
                 tc_fence_after();
                 const uint32_t v_base = smem_u32(smem + C::OFF_V + s * C::KV_BYTES);
 #pragma unroll
                 for (int kk = 0; kk < BLK / 16; ++kk) {
-                    const uint64_t ad = sw128_desc(p_base + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
                     const uint64_t bd = sw128_desc(v_base + kk * 2048, C::KV_HALF, 1024);
-                    tc_mma_ss(t_o, ad, bd, C::IDESC_O, (m > 0 || kk > 0) ? 1u : 0u);
+                    tc_mma_ts(tmem + C::T_O, tmem + C::T_P + kk * 8, bd, C::IDESC_O,
+                              (m > 0 || kk > 0) ? 1u : 0u);
                 }
                 tc_commit(&o_done);
                 tc_commit(&empty_v[s]);
                 return true;
             };
             while (ok && cur.next(j, mask, a.err, false)) {
-                const int s = n % kStages;
-                if (!mbar_wait(&full_k[s], (n / kStages) & 1, a.err)) break;
+                const int s = n % ST;
+                if (!mbar_wait(&full_k[s], (n / ST) & 1, a.err)) break;
                 if (n > 0 && !mbar_wait(&s_free, (n - 1) & 1, a.err)) break;
                 tc_fence_after();
                 const uint32_t k_base = smem_u32(smem + C::OFF_K + s * C::KV_BYTES);
+                // d = 0..63 into S_lo and d = 64..127 into S_hi, interleaved.
 #pragma unroll
-                for (int kk = 0; kk < kD / 16; ++kk) {
-                    const uint64_t ad = sw128_desc(q_base + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-                    const uint64_t bd = sw128_desc(k_base + (kk >> 2) * C::KV_HALF + (kk & 3) * 32, 16, 1024);
-                    tc_mma_ss(t_s, ad, bd, C::IDESC_S, kk > 0 ? 1u : 0u);
+                for (int kk = 0; kk < 4; ++kk) {
+                    const uint64_t a0 = sw128_desc(q_base + kk * 32, 16, 1024);
+                    const uint64_t b0 = sw128_desc(k_base + kk * 32, 16, 1024);
+                    const uint64_t a1 = sw128_desc(q_base + 16384 + kk * 32, 16, 1024);
+                    const uint64_t b1 = sw128_desc(k_base + C::KV_HALF + kk * 32, 16, 1024);
+                    tc_mma_ss(tmem + C::T_SLO, a0, b0, C::IDESC_S, kk > 0 ? 1u : 0u);
+                    tc_mma_ss(tmem + C::T_SHI, a1, b1, C::IDESC_S, kk > 0 ? 1u : 0u);
                 }
                 tc_commit(&s_full);
                 tc_commit(&empty_k[s]);
@@ -243,20 +256,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int h = h0 + rg;
         const int t = i * BLK + rr;
         const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        const uint32_t t_slo = tmem + C::T_SLO + lane_off, t_shi = tmem + C::T_SHI + lane_off;
+        const uint32_t t_p = tmem + C::T_P + lane_off, t_o = tmem + C::T_O + lane_off;
         cur.init(a, b, h0, i, false);
         float m_used = -INFINITY, l = 0.f;
-        unsigned char *prow = smem + C::OFF_P + r * 128;
         int n = 0, j;
         uint32_t mask;
         bool ok = true;
         while (cur.next(j, mask, a.err, false)) {
             if (!mbar_wait(&s_full, n & 1, a.err)) { ok = false; break; }
             tc_fence_after();
-            // All column loads in flight, then one wait.
+            // S = S_lo + S_hi, half the columns per TMEM round trip.
             float x[BLK];
 #pragma unroll
-            for (int c = 0; c < BLK / 32; ++c) tmem_ld32f(t_s + lane_off + c * 32, x + c * 32);
-            tc_wait_ld();
+            for (int hh = 0; hh < 2; ++hh) {
+                float y[BLK / 2];
+#pragma unroll
+                for (int c = 0; c < BLK / 64; ++c) {
+                    tmem_ld32f(t_slo + hh * (BLK / 2) + c * 32, x + hh * (BLK / 2) + c * 32);
+                    tmem_ld32f(t_shi + hh * (BLK / 2) + c * 32, y + c * 32);
+                }
+                tc_wait_ld();
+#pragma unroll
+                for (int e = 0; e < BLK / 2; ++e) x[hh * (BLK / 2) + e] += y[e];
+            }
             tc_fence_before();
             mbar_arrive(&s_free);
 
@@ -287,21 +310,23 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             const float base = m_used == -INFINITY ? 0.f : m_used;
             // p = 2^(s * scale * log2 e - m): one FFMA and one MUFU op per score;
-            // the row sum with 8 independent chains.
+            // the row sum with 8 independent chains; P packed to bf16 pairs.
             float sp[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) sp[e] = 0.f;
+            uint32_t pk[BLK / 2];
 #pragma unroll
-            for (int c = 0; c < BLK; ++c) {
-                x[c] = fast_exp2(fmaf(x[c], a.scale_log2, -base));
-                sp[c & 7] += x[c];
+            for (int c = 0; c < BLK / 2; ++c) {
+                const float p0 = fast_exp2(fmaf(x[2 * c], a.scale_log2, -base));
+                const float p1 = fast_exp2(fmaf(x[2 * c + 1], a.scale_log2, -base));
+                sp[(2 * c) & 7] += p0;
+                sp[(2 * c + 1) & 7] += p1;
+                pk[c] = pack_bf16x2(p0, p1);
             }
             const float rs = ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
-            uint32_t pk[BLK / 2];   // P as bf16 pairs (frees the fp32 scores before the rescale)
-#pragma unroll
-            for (int c = 0; c < BLK / 2; ++c) pk[c] = pack_bf16x2(x[2 * c], x[2 * c + 1]);
             l = l * alpha + rs;
 
+            // The previous P V has read P and updated O before either is touched.
             if (n > 0) {
                 if (!mbar_wait(&o_done, (n - 1) & 1, a.err)) { ok = false; break; }
                 tc_fence_after();
@@ -309,23 +334,22 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
                     for (int c = 0; c < kD / 32; ++c) {
                         uint32_t o0[32];
-                        tmem_ld32(t_o + lane_off + c * 32, o0);
+                        tmem_ld32(t_o + c * 32, o0);
                         tc_wait_ld();
 #pragma unroll
                         for (int e = 0; e < 32; ++e) o0[e] = __float_as_uint(__uint_as_float(o0[e]) * alpha);
-                        tmem_st32(t_o + lane_off + c * 32, o0);
+                        tmem_st32(t_o + c * 32, o0);
                     }
-                    tc_wait_st();
                 }
             }
-            // P row -> shared memory, bf16, K-major 128-byte swizzle (64 keys per half)
 #pragma unroll
-            for (int q8 = 0; q8 < BLK / 8; ++q8) {
-                const uint4 w = make_uint4(pk[4 * q8], pk[4 * q8 + 1], pk[4 * q8 + 2], pk[4 * q8 + 3]);
-                const int half = q8 >> 3, cq = q8 & 7;
-                *reinterpret_cast<uint4 *>(prow + half * 16384 + ((cq ^ (r & 7)) << 4)) = w;
+            for (int c = 0; c < BLK / 32; ++c) {
+                uint32_t w[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) w[e] = pk[c * 16 + e];
+                tmem_st16(t_p + c * 16, w);
             }
-            fence_async_shared();
+            tc_wait_st();
             tc_fence_before();
             mbar_arrive(&p_ready);
             ++n;
@@ -340,7 +364,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < kD / 32; ++c) {
             uint32_t v[32];
             if (ok && n > 0) {
-                tmem_ld32(t_o + lane_off + c * 32, v);
+                tmem_ld32(t_o + c * 32, v);
                 tc_wait_ld();
             } else {
 #pragma unroll
@@ -365,7 +389,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     if (warp == 5) {
         tc_fence_after();
-        tmem_dealloc(tmem, 256);
+        tmem_dealloc(tmem, 512);
     }
 }
 

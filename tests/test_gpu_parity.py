@@ -25,7 +25,7 @@ _cache = {}
 
 
 def inputs(w):
-    key = (w.name, w.T, w.B, w.block)
+    key = (w.name, w.T, w.B, w.block, w.Hq, w.Hkv)
     if key not in _cache:
         x = generate(w)
         _cache.clear()
@@ -294,4 +294,24 @@ def test_decode_workload_full_size():
     err = np.abs(to_host(out) - o_out).max()
     print(f"{w.name}: max-abs {err:.3e}")
     assert err <= TOL[w.dtype]
+    assert_no_device_error()
+
+
+@pytest.mark.parametrize("Hq,Hkv,block", [(4, 4, 128), (4, 2, 128), (8, 2, 128), (2, 1, 64),
+                                          (4, 1, 64), (8, 2, 64)])
+def test_prefill_head_groupings(Hq, Hkv, block):
+    # One, two or four query heads per kv-head: exercises the two-tile kernel (two
+    # tiles of the same kv-group fit) and the single-tile kernel (they do not).
+    w = PARITY_WORKLOADS["p_bf16_blk128"].with_(Hq=Hq, Hkv=Hkv, block=block, B=1, T=777)
+    x, dev = inputs(w)
+    sel = oracle_select(w, x)
+    idx = torch.from_numpy(sel["idx"]).cuda()
+    cnt = torch.from_numpy(sel["count"]).cuda()
+    out, lse = spa.spa_sparse_attn_prefill(dev["q"], dev["k"], dev["v"], w.block, idx, cnt,
+                                           w.scale, want_lse=True)
+    torch.cuda.synchronize()
+    o_out, o_lse = oracle.attention(x["q"], x["k"], x["v"], w.dtype, w.block, sel["idx"],
+                                    sel["count"], w.scale)
+    assert np.abs(to_host(out) - o_out).max() <= TOL[w.dtype]
+    np.testing.assert_allclose(lse.cpu().numpy(), o_lse, rtol=0, atol=LSE_TOL[w.dtype])
     assert_no_device_error()
