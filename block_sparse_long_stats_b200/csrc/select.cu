@@ -68,6 +68,47 @@ __device__ V block_exclusive_scan(V x, V *warp_tot, V *total) {
     return r;
 }
 
+// Log Taylor score of one candidate from one lane's PL components of the pooled
+// query (qv, its squares q2) and of the block's mean and variance: per-lane fused
+// multiply-adds, then an xor-shuffle tree across the warp. Both selection paths
+// use this exact order, so their scores agree to the bit.
+template <int PL>
+__device__ __forceinline__ void lane_partials(const float (&qv)[PL], const float (&q2)[PL],
+                                              const float (&mu)[PL], const float (&vr)[PL],
+                                              float &dot, float &quad) {
+    dot = 0.f;
+    quad = 0.f;
+#pragma unroll
+    for (int c = 0; c < PL; ++c) {
+        dot = fmaf(qv[c], mu[c], dot);
+        quad = fmaf(q2[c], vr[c], quad);
+    }
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+__device__ __forceinline__ float log_score(float dot, float quad, float scale, float hs2, int nj) {
+    return scale * dot + log1pf(hs2 * quad) + logf((float)nj);
+}
+
+template <int PL>
+__device__ __forceinline__ void load_stats(const float *mb, const float *vb, float (&mu)[PL],
+                                           float (&vr)[PL]) {
+    if constexpr (PL == 4) {
+        const float4 m4 = __ldg(reinterpret_cast<const float4 *>(mb));
+        const float4 v4 = __ldg(reinterpret_cast<const float4 *>(vb));
+        mu[0] = m4.x; mu[1] = m4.y; mu[2] = m4.z; mu[3] = m4.w;
+        vr[0] = v4.x; vr[1] = v4.y; vr[2] = v4.z; vr[3] = v4.w;
+    } else {
+        const float2 m2 = __ldg(reinterpret_cast<const float2 *>(mb));
+        const float2 v2 = __ldg(reinterpret_cast<const float2 *>(vb));
+        mu[0] = m2.x; mu[1] = m2.y;
+        vr[0] = v2.x; vr[1] = v2.y;
+    }
+}
+
 struct SelectArgs {
     const void *q;
     const float *mean;
@@ -81,6 +122,7 @@ struct SelectArgs {
     int32_t *count;
     int *err;
     int sort_cap;   // power of two >= the largest residual of any unit
+    bool prescored; // decode: the fp32 scores are already in the unit's row of idx
 };
 
 template <typename T, int D>
@@ -103,7 +145,7 @@ __global__ void __launch_bounds__(kThreads) select_kernel(SelectArgs a) {
     const size_t unit = (size_t)bh * a.nq + i;
 
     // ---- pooled query: mean of the rows of query block i
-    {
+    if (!a.prescored) {
         constexpr int V = 16 / sizeof(T);
         constexpr int CPR = D / V;             // 16-byte chunks per row
         constexpr int RG = kThreads / CPR;     // row groups
@@ -146,7 +188,13 @@ __global__ void __launch_bounds__(kThreads) select_kernel(SelectArgs a) {
     while (N < nres) N <<= 1;
 
     // ---- fp32 scores of the residual candidates, one warp per candidate
-    {
+    if (a.prescored) {
+        const float *sc = reinterpret_cast<const float *>(a.idx + unit * a.cap);
+        for (int r = tid; r < nres; r += kThreads) {
+            const int j = r_lo + r;
+            keys[r] = ((uint64_t)order_desc(sc[j]) << 32) | (uint32_t)j;
+        }
+    } else {
         constexpr int PL = D / 32;   // components per lane
         float qv[PL], q2[PL];
 #pragma unroll
@@ -159,40 +207,21 @@ __global__ void __launch_bounds__(kThreads) select_kernel(SelectArgs a) {
         const float *vb = a.var + ((size_t)b * a.Hkv + g) * a.nb * D + lane * PL;
         for (int r = warp; r < nres; r += kWarps) {
             const int j = r_lo + r;
-            float mu[PL], vr[PL];
-            if constexpr (PL == 4) {
-                float4 m4 = __ldg(reinterpret_cast<const float4 *>(mb + (size_t)j * D));
-                float4 v4 = __ldg(reinterpret_cast<const float4 *>(vb + (size_t)j * D));
-                mu[0] = m4.x; mu[1] = m4.y; mu[2] = m4.z; mu[3] = m4.w;
-                vr[0] = v4.x; vr[1] = v4.y; vr[2] = v4.z; vr[3] = v4.w;
-            } else {
-                float2 m2 = __ldg(reinterpret_cast<const float2 *>(mb + (size_t)j * D));
-                float2 v2 = __ldg(reinterpret_cast<const float2 *>(vb + (size_t)j * D));
-                mu[0] = m2.x; mu[1] = m2.y;
-                vr[0] = v2.x; vr[1] = v2.y;
-            }
-            float dot = 0.f, quad = 0.f;
-#pragma unroll
-            for (int c = 0; c < PL; ++c) {
-                dot = fmaf(qv[c], mu[c], dot);
-                quad = fmaf(q2[c], vr[c], quad);
-            }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                dot += __shfl_xor_sync(0xffffffffu, dot, o);
-                quad += __shfl_xor_sync(0xffffffffu, quad, o);
-            }
+            float mu[PL], vr[PL], dot, quad;
+            load_stats<PL>(mb + (size_t)j * D, vb + (size_t)j * D, mu, vr);
+            lane_partials<PL>(qv, q2, mu, vr, dot, quad);
+            dot = warp_sum(dot);
+            quad = warp_sum(quad);
             if (lane == 0) {
-                const int nj = min(a.block, a.T - j * a.block);
-                const float l = a.scale * dot + log1pf(hs2 * quad) + logf((float)nj);
+                const float l = log_score(dot, quad, a.scale, hs2, min(a.block, a.T - j * a.block));
                 keys[r] = ((uint64_t)order_desc(l) << 32) | (uint32_t)j;
             }
         }
-        for (int r = nres + tid; r < N; r += kThreads) keys[r] = ~0ull;
-        for (int j = tid; j <= jmax; j += kThreads)
-            flag[j] = (j < r_lo || j >= r_hi) ? 1 : 0;     // reserved blocks
-        __syncthreads();
     }
+    for (int r = nres + tid; r < N; r += kThreads) keys[r] = ~0ull;
+    for (int j = tid; j <= jmax; j += kThreads)
+        flag[j] = (j < r_lo || j >= r_hi) ? 1 : 0;     // reserved blocks
+    __syncthreads();   // (prescored: every score is read before the list overwrites them)
 
     // ---- bitonic sort, ascending keys = descending score, ascending index
     for (int kk = 2; kk <= N; kk <<= 1) {
@@ -251,6 +280,79 @@ __global__ void __launch_bounds__(kThreads) select_kernel(SelectArgs a) {
     }
 }
 
+// Decode scoring: CTA (tile, b*Hkv + g) scores kDecTile candidate blocks for all
+// G query heads of kv-head g, so each block's statistics are read once per group
+// (the step reads the statistics exactly once: HBM-bound). Warp per candidate,
+// lanes over d, four candidates in flight per warp; lane h writes head h's fp32
+// score into that head's row of idx, used as scratch (decode rows hold exactly
+// cap >= nb entries) until the cut kernel replaces it with the kept list.
+constexpr int kDecTile = 256;
+
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(kThreads) decode_score_kernel(SelectArgs a) {
+    constexpr int PL = D / 32;
+    constexpr int U = 4;
+    __shared__ float qs[G][D];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int bg = blockIdx.y, b = bg / a.Hkv, g = bg % a.Hkv;
+    for (int x = tid; x < G * D; x += kThreads) {
+        const int hh = x / D, c = x % D;
+        const T *qrow = reinterpret_cast<const T *>(a.q) + ((size_t)b * a.Hq + g * G + hh) * D;
+        if constexpr (sizeof(T) == 2)
+            qs[hh][c] = __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(qrow)[c]);
+        else
+            qs[hh][c] = reinterpret_cast<const float *>(qrow)[c];
+    }
+    __syncthreads();
+    float qv[G][PL], q2[G][PL];
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh)
+#pragma unroll
+        for (int c = 0; c < PL; ++c) {
+            qv[hh][c] = qs[hh][lane * PL + c];
+            q2[hh][c] = qv[hh][c] * qv[hh][c];
+        }
+    const float hs2 = 0.5f * a.scale * a.scale;
+    const float *mb = a.mean + (size_t)bg * a.nb * D + lane * PL;
+    const float *vb = a.var + (size_t)bg * a.nb * D + lane * PL;
+    float *rows = reinterpret_cast<float *>(a.idx) + ((size_t)b * a.Hq + g * G) * a.cap;
+    const int j0 = blockIdx.x * kDecTile;
+    for (int r = warp * U; r < kDecTile; r += kWarps * U) {
+        float mu[U][PL], vr[U][PL];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int j = min(j0 + r + u, a.nb - 1);
+            load_stats<PL>(mb + (size_t)j * D, vb + (size_t)j * D, mu[u], vr[u]);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int j = j0 + r + u;
+            float lsc = 0.f;
+#pragma unroll
+            for (int hh = 0; hh < G; ++hh) {
+                float dot, quad;
+                lane_partials<PL>(qv[hh], q2[hh], mu[u], vr[u], dot, quad);
+                dot = warp_sum(dot);
+                quad = warp_sum(quad);
+                if (lane == hh) lsc = log_score(dot, quad, a.scale, hs2, min(a.block, a.T - j * a.block));
+            }
+            if (lane < G && j < a.nb) rows[(size_t)lane * a.cap + j] = lsc;
+        }
+    }
+}
+
+template <typename T, int D>
+cudaError_t launch_decode_scores(const SelectArgs &a, cudaStream_t s) {
+    dim3 grid((unsigned)((a.nb + kDecTile - 1) / kDecTile), (unsigned)(a.B * a.Hkv));
+    switch (a.G) {
+        case 1: decode_score_kernel<T, D, 1><<<grid, kThreads, 0, s>>>(a); break;
+        case 2: decode_score_kernel<T, D, 2><<<grid, kThreads, 0, s>>>(a); break;
+        case 4: decode_score_kernel<T, D, 4><<<grid, kThreads, 0, s>>>(a); break;
+        default: decode_score_kernel<T, D, 8><<<grid, kThreads, 0, s>>>(a); break;
+    }
+    return cudaGetLastError();
+}
+
 template <typename T, int D>
 cudaError_t launch_t(const SelectArgs &a, cudaStream_t s) {
     const size_t smem = (size_t)a.sort_cap * 8 + kThreads * 8 * sizeof(float) + (size_t)a.nb + 16;
@@ -258,6 +360,10 @@ cudaError_t launch_t(const SelectArgs &a, cudaStream_t s) {
     if (smem > 48 * 1024) {
         cudaError_t e =
             cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    if (a.prescored) {
+        cudaError_t e = launch_decode_scores<T, D>(a, s);
         if (e != cudaSuccess) return e;
     }
     const unsigned grid = (unsigned)((size_t)a.B * a.Hq * a.nq);
@@ -283,6 +389,7 @@ cudaError_t launch_select(const void *q, bool bf16, const float *mean, const flo
     int n = 1;
     while (n < a.nb) n <<= 1;
     a.sort_cap = n;
+    a.prescored = Lq == 1 && (a.G == 1 || a.G == 2 || a.G == 4 || a.G == 8);
     if (bf16) return d == 128 ? launch_t<__nv_bfloat16, 128>(a, s) : launch_t<__nv_bfloat16, 64>(a, s);
     return d == 128 ? launch_t<float, 128>(a, s) : launch_t<float, 64>(a, s);
 }
