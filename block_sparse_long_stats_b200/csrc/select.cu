@@ -109,6 +109,36 @@ __device__ __forceinline__ void load_stats(const float *mb, const float *vb, flo
     }
 }
 
+__host__ __device__ constexpr int ilog2(int x) { return x <= 1 ? 0 : 1 + ilog2(x / 2); }
+
+// Reduces K values (K a power of two, 2 <= K <= 32) across the 32 lanes of a warp
+// with K - 1 + (5 - log2 K) shuffles; lane L ends with the total of value
+// (L >> (5 - log2 K)). Offsets run 16, 8, ... like the per-value xor butterfly,
+// and each addition is own + partner, so every total equals the butterfly's.
+template <int K>
+__device__ __forceinline__ float reduce_transpose(float (&v)[K], int lane) {
+    constexpr int LK = ilog2(K);
+    float w[K];
+#pragma unroll
+    for (int k = 0; k < K; ++k) w[k] = v[k];
+#pragma unroll
+    for (int st = 0; st < LK; ++st) {
+        const int off = 16 >> st;
+        const int half = K >> (st + 1);
+        const bool upper = (lane & off) != 0;
+#pragma unroll
+        for (int k = 0; k < half; ++k) {
+            const float send = upper ? w[k] : w[k + half];
+            const float keep = upper ? w[k + half] : w[k];
+            w[k] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+        }
+    }
+    float t = w[0];
+#pragma unroll
+    for (int off = 16 >> LK; off > 0; off >>= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
+    return t;
+}
+
 struct SelectArgs {
     const void *q;
     const float *mean;
@@ -129,8 +159,9 @@ template <typename T, int D>
 __global__ void __launch_bounds__(kThreads) select_kernel(SelectArgs a) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     uint64_t *keys = reinterpret_cast<uint64_t *>(smem_raw);               // [sort_cap]
-    float *red = reinterpret_cast<float *>(keys + a.sort_cap);             // [kThreads * 8]
-    unsigned char *flag = reinterpret_cast<unsigned char *>(red + kThreads * 8); // [nb]
+    // [kThreads * 8] pooling buffer, absent when the scores come precomputed
+    float *red = reinterpret_cast<float *>(keys + a.sort_cap);
+    unsigned char *flag = reinterpret_cast<unsigned char *>(red + (a.prescored ? 0 : kThreads * 8)); // [nb]
     __shared__ double dtot[kWarps];
     __shared__ double dsum;
     __shared__ int itot[kWarps];
@@ -223,17 +254,35 @@ __global__ void __launch_bounds__(kThreads) select_kernel(SelectArgs a) {
         flag[j] = (j < r_lo || j >= r_hi) ? 1 : 0;     // reserved blocks
     __syncthreads();   // (prescored: every score is read before the list overwrites them)
 
-    // ---- bitonic sort, ascending keys = descending score, ascending index
+    // ---- bitonic sort, ascending keys = descending score, ascending index.
+    // Pair p of a stage compares x = (p / jj) * 2jj + p % jj with x + jj (shifts:
+    // jj is a power of two); every
+    // thread works on N/2/kThreads pairs, four loads in flight at a time.
     for (int kk = 2; kk <= N; kk <<= 1) {
         for (int jj = kk >> 1; jj > 0; jj >>= 1) {
-            for (int x = tid; x < N; x += kThreads) {
-                const int y = x ^ jj;
-                if (y > x) {
-                    const uint64_t kx = keys[x], ky = keys[y];
-                    const bool up = (x & kk) == 0;
-                    if ((kx > ky) == up) {
-                        keys[x] = ky;
-                        keys[y] = kx;
+            const int npair = N >> 1;
+            const int lj = __ffs(jj) - 1;      // jj is a power of two
+            for (int p0 = tid; p0 < npair; p0 += 4 * kThreads) {
+                uint64_t kx[4], ky[4];
+                int xs[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int p = p0 + u * kThreads;
+                    xs[u] = ((p >> lj) << (lj + 1)) | (p & (jj - 1));
+                    if (p < npair) {
+                        kx[u] = keys[xs[u]];
+                        ky[u] = keys[xs[u] + jj];
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int p = p0 + u * kThreads;
+                    if (p < npair) {
+                        const bool up = (xs[u] & kk) == 0;
+                        if ((kx[u] > ky[u]) == up) {
+                            keys[xs[u]] = ky[u];
+                            keys[xs[u] + jj] = kx[u];
+                        }
                     }
                 }
             }
@@ -327,16 +376,21 @@ __global__ void __launch_bounds__(kThreads) decode_score_kernel(SelectArgs a) {
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const int j = j0 + r + u;
-            float lsc = 0.f;
+            // 2G per-lane partials: dot of head h at [h], quad of head h at [G + h].
+            float v[2 * G];
 #pragma unroll
-            for (int hh = 0; hh < G; ++hh) {
-                float dot, quad;
-                lane_partials<PL>(qv[hh], q2[hh], mu[u], vr[u], dot, quad);
-                dot = warp_sum(dot);
-                quad = warp_sum(quad);
-                if (lane == hh) lsc = log_score(dot, quad, a.scale, hs2, min(a.block, a.T - j * a.block));
-            }
-            if (lane < G && j < a.nb) rows[(size_t)lane * a.cap + j] = lsc;
+            for (int hh = 0; hh < G; ++hh) lane_partials<PL>(qv[hh], q2[hh], mu[u], vr[u], v[hh], v[G + hh]);
+            // Transposing halving reduction: at each xor offset every lane keeps half
+            // of its values and adds its partner's copy of them, the same pairwise
+            // sums the per-value butterfly forms. Afterwards the lanes of group k
+            // (lane >> (5 - log2(2G))) hold the warp total of value k.
+            const float tot = reduce_transpose<2 * G>(v, lane);
+            constexpr int LB = 5 - ilog2(2 * G);            // lanes per value = 2^LB
+            const float quad = __shfl_sync(0xffffffffu, tot, (lane + (G << LB)) & 31);
+            const int hh = lane >> LB;                      // value index of this lane's group
+            if (hh < G && (lane & ((1 << LB) - 1)) == 0 && j < a.nb)
+                rows[(size_t)hh * a.cap + j] =
+                    log_score(tot, quad, a.scale, hs2, min(a.block, a.T - j * a.block));
         }
     }
 }
@@ -355,7 +409,8 @@ cudaError_t launch_decode_scores(const SelectArgs &a, cudaStream_t s) {
 
 template <typename T, int D>
 cudaError_t launch_t(const SelectArgs &a, cudaStream_t s) {
-    const size_t smem = (size_t)a.sort_cap * 8 + kThreads * 8 * sizeof(float) + (size_t)a.nb + 16;
+    const size_t smem = (size_t)a.sort_cap * 8 + (a.prescored ? 0 : kThreads * 8 * sizeof(float)) +
+                        (size_t)a.nb + 16;
     auto kern = select_kernel<T, D>;
     if (smem > 48 * 1024) {
         cudaError_t e =
