@@ -351,6 +351,19 @@ def main():
         vc = torch.from_numpy(np.ascontiguousarray(xd["v"]).view(np.int16)).cuda().view(torch.bfloat16)
         del xd
         dm, dv = spa.spa_block_stats(kc, wd.block)
+        st_ms = []
+        for _ in range(5):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            spa.spa_block_stats(kc, wd.block, mean=dm, var=dv)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            st_ms.append(e0.elapsed_time(e1))
+        st_bytes = kc.numel() * 2 + 2 * dm.numel() * 4
+        stats_full = {"ms": statistics.median(st_ms[1:]),
+                      "GB/s": st_bytes / (statistics.median(st_ms[1:]) / 1e3) / 1e9,
+                      "bytes": st_bytes}
         didx = torch.empty((wd.B, wd.Hq, 1, wd.nb), device="cuda", dtype=torch.int32)
         dcnt = torch.empty((wd.B, wd.Hq, 1), device="cuda", dtype=torch.int32)
         ws = torch.empty(spa.spa_decode_workspace_bytes(wd.B, wd.Hq, wd.Hkv, wd.T, wd.d, wd.block),
@@ -384,7 +397,8 @@ def main():
                   "select_ms": t_dsel, "GB/s": gbs, "peak_GB/s": peaks["hbm_gbs"],
                   "frac": gbs / peaks["hbm_gbs"], "peak_source": peak_src,
                   "tokens/s": world * wd.B / ((t_dsel + t_dec) / 1e3),
-                  "kept_fraction": float(dcnt.float().mean().item()) / wd.nb}
+                  "kept_fraction": float(dcnt.float().mean().item()) / wd.nb,
+                  "block_stats_full_cache": stats_full}
         del kc, vc
 
     # ---- CPU oracle baseline (rank 0, one GPU)

@@ -33,6 +33,33 @@ struct Elem<float> {
     }
 };
 
+// Sums K values (K a power of two <= 16) over the 16 lanes of a half-warp by
+// halving: at each xor offset (8, 4, ...) a lane keeps half of its values and adds
+// its partner's copy of them. Lane rg ends with the total of value rg >> (4 - log2 K).
+template <int K>
+__device__ __forceinline__ float halfwarp_reduce_transpose(float (&v)[K], int rg) {
+    constexpr int LK = K >= 16 ? 4 : K >= 8 ? 3 : K >= 4 ? 2 : K >= 2 ? 1 : 0;
+    float w[K];
+#pragma unroll
+    for (int k = 0; k < K; ++k) w[k] = v[k];
+#pragma unroll
+    for (int st = 0; st < LK; ++st) {
+        const int off = 8 >> st;
+        const int half = K >> (st + 1);
+        const bool upper = (rg & off) != 0;
+#pragma unroll
+        for (int k = 0; k < half; ++k) {
+            const float send = upper ? w[k] : w[k + half];
+            const float keep = upper ? w[k + half] : w[k];
+            w[k] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+        }
+    }
+    float t = w[0];
+#pragma unroll
+    for (int off = 8 >> LK; off > 0; off >>= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
+    return t;
+}
+
 constexpr int kTileRows = 128;
 constexpr int kRowGroups = 16;
 constexpr int kRowsPerLane = kTileRows / kRowGroups;  // 8
@@ -85,15 +112,15 @@ __global__ void __launch_bounds__(512) block_stats_kernel(const T *__restrict__ 
 #pragma unroll
             for (int v = 0; v < V; ++v) s[v] += x[v];
         }
-#pragma unroll
-        for (int v = 0; v < V; ++v) {
-#pragma unroll
-            for (int o = 1; o < 16; o <<= 1) s[v] += __shfl_xor_sync(0xffffffffu, s[v], o);
-        }
+        // Column totals (lane rg holds column rg / (16 / V)), then every lane gets
+        // all V means back.
+        constexpr int LPV = 16 / V;                      // lanes per value
         const float inv_n = 1.0f / (float)n;
+        const float mean_own = halfwarp_reduce_transpose<V>(s, rg) * inv_n;
+        const int hbase = lane & 16;                     // this half-warp's first lane
         float mu[V];
 #pragma unroll
-        for (int v = 0; v < V; ++v) mu[v] = s[v] * inv_n;
+        for (int v = 0; v < V; ++v) mu[v] = __shfl_sync(0xffffffffu, mean_own, hbase + v * LPV);
 #pragma unroll
         for (int v = 0; v < V; ++v) s[v] = 0.f;
 #pragma unroll
@@ -109,23 +136,11 @@ __global__ void __launch_bounds__(512) block_stats_kernel(const T *__restrict__ 
                 }
             }
         }
-#pragma unroll
-        for (int v = 0; v < V; ++v) {
-#pragma unroll
-            for (int o = 1; o < 16; o <<= 1) s[v] += __shfl_xor_sync(0xffffffffu, s[v], o);
-        }
-        if (rg < V) {
-            float m_out = 0.f, v_out = 0.f;
-#pragma unroll
-            for (int v = 0; v < V; ++v) {
-                if (v == rg) {
-                    m_out = mu[v];
-                    v_out = s[v] * inv_n;
-                }
-            }
-            const size_t o = ((size_t)bg * nb + j) * d + (size_t)chunk * V + rg;
-            mean[o] = m_out;
-            var[o] = v_out;
+        const float var_own = halfwarp_reduce_transpose<V>(s, rg) * inv_n;
+        if ((rg & (LPV - 1)) == 0) {
+            const size_t o = ((size_t)bg * nb + j) * d + (size_t)chunk * V + rg / LPV;
+            mean[o] = mean_own;
+            var[o] = var_own;
         }
     }
 }
