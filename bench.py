@@ -83,6 +83,25 @@ def kept_kv_bytes(count: np.ndarray, idx: np.ndarray, G: int, T: int, block: int
     return float(total * d * 2 * 2)
 
 
+# ---------------------------------------------------------------- ranks
+
+def max_over_ranks(v: float, world: int, device) -> float:
+    """Max of a per-rank device time over all ranks (all_reduce MAX; no-op on one rank)."""
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank: int, world: int, steps: int, total_ms: float) -> float:
+    """Whole-job units/s: every rank processes its own replica (weak scaling), and the
+    slowest rank's time counts."""
+    return world * units_per_rank * steps / (total_ms / 1e3)
+
+
 # ---------------------------------------------------------------- clocks
 
 class ClockSampler:
@@ -228,12 +247,8 @@ def main():
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        t = torch.tensor([v], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    def rank_max(v: float) -> float:
+        return max_over_ranks(v, world, "cuda")
 
     peaks, peak_src = load_peaks()
     w = WORKLOADS[args.workload]
@@ -291,9 +306,9 @@ def main():
     t_sel = [e[1].elapsed_time(e[2]) for e in evs]
     t_att = [e[2].elapsed_time(e[3]) for e in evs]
     t_step = [e[0].elapsed_time(e[3]) for e in evs]
-    total_ms = max_over_ranks(sum(t_step))
+    total_ms = rank_max(sum(t_step))
     ms_per_step = total_ms / args.steps
-    value = world * B * L * args.steps / (total_ms / 1e3)
+    value = job_throughput(B * L, world, args.steps, total_ms)
 
     count_h = cnt.cpu().numpy()
     idx_h = idx.cpu().numpy()
@@ -335,8 +350,8 @@ def main():
         e_evs[s][1].record(stream)
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e_evs)) / args.e2e_steps
-    e2e = {"value": world * B * L / (e2e_ms / 1e3), "unit": "tokens/s",
+    e2e_ms = rank_max(sum(a.elapsed_time(b) for a, b in e_evs)) / args.e2e_steps
+    e2e = {"value": job_throughput(B * L, world, 1, e2e_ms), "unit": "tokens/s",
            "h2d_bytes_per_step": int(qh.numel() * 2 + kh.numel() * 2 + vh.numel() * 2),
            "d2h_bytes_per_step": int(oh.numel() * 2), "ms_per_step": e2e_ms}
     del qh, kh, vh, oh, qd, kd, vd
@@ -389,8 +404,8 @@ def main():
             d_evs[s][2].record(stream)
         torch.cuda.synchronize()
         barrier()
-        t_dsel = statistics.mean(e[0].elapsed_time(e[1]) for e in d_evs)
-        t_dec = statistics.mean(e[1].elapsed_time(e[2]) for e in d_evs)
+        t_dsel = rank_max(statistics.mean(e[0].elapsed_time(e[1]) for e in d_evs))
+        t_dec = rank_max(statistics.mean(e[1].elapsed_time(e[2]) for e in d_evs))
         dbytes = kept_kv_bytes(dcnt.cpu().numpy(), didx.cpu().numpy(), wd.G, wd.T, wd.block, wd.d)
         gbs = dbytes / (t_dec / 1e3) / 1e9
         decode = {"workload": wd.name, "kept_kv_bytes": dbytes, "attn_ms": t_dec,
