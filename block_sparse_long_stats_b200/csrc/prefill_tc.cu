@@ -10,21 +10,19 @@
 // walks the union of its two kept lists, and a row masks the blocks its own head
 // did not keep). Warp roles:
 //   warps 0-3 : softmax; thread r owns query row r = TMEM lane r
-//   warp 4    : TMA producer (Q once; K_j and V_j per kept block into a ring)
+//   warp 4    : TMA producer (Q once; K_j and V_j per kept block)
 //   warp 5    : TMEM allocator and single-thread tcgen05.mma issuer
-// TMEM (fp32 columns): S_lo [0,128), S_hi [128,256), P [256,256+BLK/2) as bf16
-// pairs, O [384,512).
-//
-// The MMA forms follow measured tcgen05 rates on B200: a chain of MMAs into one
-// accumulator pays a fixed latency per instruction, so S = Q K^T is split over the
-// two halves of d into two accumulators whose MMAs are issued interleaved (the
-// softmax adds them); and P V reads P from tensor memory (A operand in TMEM, V
-// from its TMA layout as an MN-major B), the fastest form for that product.
-// Per kept block n the issuer runs S(n) as soon as the softmax has read S(n-1),
-// then P(n-1) V once P(n-1) is in TMEM. The softmax scales by s*log2(e), takes
-// exp2, keeps the running max lazily (O is rescaled only when the max grows by
-// more than 8, in log2 units) and writes P once the previous P V has finished.
-// Epilogue: O / l from TMEM to bf16 rows, lse = (m + log2 l) ln 2.
+// Per kept block n: S = Q K_j^T (8 MMAs, both operands K-major in shared memory,
+// fp32 accumulator in TMEM); the softmax scales by s*log2(e), takes exp2, keeps the
+// running max lazily (O is rescaled only when the max grows by more than 8, in
+// log2 units) and writes P as bf16 over the first BLK/2 columns of S; then
+// O += P V_j reads P from tensor memory (A operand in TMEM, V in its TMA layout as
+// an MN-major B), the fastest measured form for that product.
+// Each CTA's chain is serial (S(n+1) overwrites P(n), so it is issued after
+// P(n) V; MMAs of one thread run in issue order). The kernel is sized for two CTAs
+// per SM (256 TMEM columns and 96 KB of shared memory each), and the SM interleaves
+// one CTA's softmax with the other's MMAs. Epilogue: O / l from TMEM to bf16 rows,
+// lse = (m + log2 l) ln 2.
 #include <math.h>
 
 #include "kernels.h"
@@ -37,22 +35,6 @@ constexpr int kThreads = 192;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
-
-template <int BLK>
-struct Cfg {
-    static constexpr int HPT = 128 / BLK;               // heads stacked in the M = 128 tile
-    static constexpr int STAGES = BLK == 128 ? 3 : 4;   // K/V ring depth
-    static constexpr int Q_BYTES = 128 * kD * 2;        // 32 KB: two 64-column halves
-    static constexpr int KV_BYTES = BLK * kD * 2;       // one K or V tile
-    static constexpr int KV_HALF = BLK * 128;           // one 64-column half of it
-    static constexpr int OFF_Q = 0;
-    static constexpr int OFF_K = OFF_Q + Q_BYTES;
-    static constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
-    static constexpr int SMEM = OFF_V + STAGES * KV_BYTES;
-    static constexpr uint32_t T_SLO = 0, T_SHI = 128, T_P = 256, T_O = 384;
-    static constexpr uint32_t IDESC_S = idesc_bf16(128, BLK, false);
-    static constexpr uint32_t IDESC_O = idesc_bf16(128, kD, true);
-};
 
 struct PrefillArgs {
     const int32_t *idx;
@@ -125,22 +107,39 @@ struct Cursor {
     }
 };
 
+// TMEM: S [0,128) with P written over its first BLK/2 columns, O [128,256).
+// Shared memory: Q, one K and one V buffer (block 128) or two of each (block 64).
 template <int BLK>
-__global__ void __launch_bounds__(kThreads, 1)
+struct Cfg {
+    static constexpr int HPT = 128 / BLK;
+    static constexpr int STAGES = BLK == 128 ? 1 : 2;
+    static constexpr int Q_BYTES = 128 * kD * 2;
+    static constexpr int KV_BYTES = BLK * kD * 2;
+    static constexpr int KV_HALF = BLK * 128;
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_K = OFF_Q + Q_BYTES;
+    static constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
+    static constexpr int SMEM = OFF_V + STAGES * KV_BYTES;
+    static constexpr uint32_t T_S = 0, T_O = 128;
+    static constexpr uint32_t IDESC_S = idesc_bf16(128, BLK, false);
+    static constexpr uint32_t IDESC_O = idesc_bf16(128, kD, true);
+};
+
+template <int BLK>
+__global__ void __launch_bounds__(kThreads, 2)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-                      const __grid_constant__ CUtensorMap tv, PrefillArgs a) {
+                       const __grid_constant__ CUtensorMap tv, PrefillArgs a) {
     using C = Cfg<BLK>;
     constexpr int HPT = C::HPT;
     constexpr int ST = C::STAGES;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char *smem = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    __shared__ uint64_t bar_q, full_k[ST], full_v[ST], empty_k[ST], empty_v[ST], s_full, s_free,
-        p_ready, o_done;
+    __shared__ uint64_t bar_q, full_k[ST], full_v[ST], empty_k[ST], empty_v[ST], s_full, p_ready,
+        o_done;
     __shared__ uint32_t tmem_slot;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    // Heaviest tiles first: query block index descending.
     const int per_i = a.B * a.Hkv * a.npairs;
     const int i = a.nq - 1 - (int)(blockIdx.x / per_i);
     const int rest = (int)(blockIdx.x % per_i);
@@ -158,12 +157,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&empty_v[s], 1);
         }
         mbar_init(&s_full, 1);
-        mbar_init(&s_free, 128);
         mbar_init(&p_ready, 128);
         mbar_init(&o_done, 1);
         fence_mbar_init();
     }
-    if (warp == 5) tmem_alloc(&tmem_slot, 512);
+    if (warp == 5) tmem_alloc(&tmem_slot, 256);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -171,7 +169,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     Cursor<HPT> cur;
     if (warp == 4) {
-        // ------------------------------------------------------------ producer
         if (lane == 0) {
             prefetch_tmap(&tq);
             prefetch_tmap(&tk);
@@ -203,7 +200,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     } else if (warp == 5) {
-        // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             cur.init(a, b, h0, i, false);
             const uint32_t q_base = smem_u32(smem + C::OFF_Q);
@@ -219,45 +215,37 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int kk = 0; kk < BLK / 16; ++kk) {
                     const uint64_t bd = sw128_desc(v_base + kk * 2048, C::KV_HALF, 1024);
-                    tc_mma_ts(tmem + C::T_O, tmem + C::T_P + kk * 8, bd, C::IDESC_O,
+                    tc_mma_ts(tmem + C::T_O, tmem + C::T_S + kk * 8, bd, C::IDESC_O,
                               (m > 0 || kk > 0) ? 1u : 0u);
                 }
-                tc_commit(&o_done);
                 tc_commit(&empty_v[s]);
                 return true;
             };
             while (ok && cur.next(j, mask, a.err, false)) {
+                if (n > 0 && !issue_pv(n - 1)) { ok = false; break; }
                 const int s = n % ST;
                 if (!mbar_wait(&full_k[s], (n / ST) & 1, a.err)) break;
-                if (n > 0 && !mbar_wait(&s_free, (n - 1) & 1, a.err)) break;
                 tc_fence_after();
                 const uint32_t k_base = smem_u32(smem + C::OFF_K + s * C::KV_BYTES);
-                // d = 0..63 into S_lo and d = 64..127 into S_hi, interleaved.
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t a0 = sw128_desc(q_base + kk * 32, 16, 1024);
-                    const uint64_t b0 = sw128_desc(k_base + kk * 32, 16, 1024);
-                    const uint64_t a1 = sw128_desc(q_base + 16384 + kk * 32, 16, 1024);
-                    const uint64_t b1 = sw128_desc(k_base + C::KV_HALF + kk * 32, 16, 1024);
-                    tc_mma_ss(tmem + C::T_SLO, a0, b0, C::IDESC_S, kk > 0 ? 1u : 0u);
-                    tc_mma_ss(tmem + C::T_SHI, a1, b1, C::IDESC_S, kk > 0 ? 1u : 0u);
+                for (int kk = 0; kk < kD / 16; ++kk) {
+                    const uint64_t ad = sw128_desc(q_base + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+                    const uint64_t bd = sw128_desc(k_base + (kk >> 2) * C::KV_HALF + (kk & 3) * 32, 16, 1024);
+                    tc_mma_ss(tmem + C::T_S, ad, bd, C::IDESC_S, kk > 0 ? 1u : 0u);
                 }
                 tc_commit(&s_full);
                 tc_commit(&empty_k[s]);
-                if (n > 0 && !issue_pv(n - 1)) { ok = false; break; }
                 ++n;
             }
-            if (ok && n > 0) issue_pv(n - 1);
+            if (ok && n > 0 && issue_pv(n - 1)) tc_commit(&o_done);
         }
     } else {
-        // ------------------------------------------------------------ softmax (rows)
-        const int r = tid;                       // TMEM lane
-        const int rg = r / BLK, rr = r % BLK;    // stacked head, row inside the block
+        const int r = tid;
+        const int rg = r / BLK, rr = r % BLK;
         const int h = h0 + rg;
         const int t = i * BLK + rr;
         const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-        const uint32_t t_slo = tmem + C::T_SLO + lane_off, t_shi = tmem + C::T_SHI + lane_off;
-        const uint32_t t_p = tmem + C::T_P + lane_off, t_o = tmem + C::T_O + lane_off;
+        const uint32_t t_s = tmem + C::T_S + lane_off, t_o = tmem + C::T_O + lane_off;
         cur.init(a, b, h0, i, false);
         float m_used = -INFINITY, l = 0.f;
         int n = 0, j;
@@ -266,33 +254,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         while (cur.next(j, mask, a.err, false)) {
             if (!mbar_wait(&s_full, n & 1, a.err)) { ok = false; break; }
             tc_fence_after();
-            // S = S_lo + S_hi, half the columns per TMEM round trip.
             float x[BLK];
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                float y[BLK / 2];
-#pragma unroll
-                for (int c = 0; c < BLK / 64; ++c) {
-                    tmem_ld32f(t_slo + hh * (BLK / 2) + c * 32, x + hh * (BLK / 2) + c * 32);
-                    tmem_ld32f(t_shi + hh * (BLK / 2) + c * 32, y + c * 32);
-                }
-                tc_wait_ld();
-#pragma unroll
-                for (int e = 0; e < BLK / 2; ++e) x[hh * (BLK / 2) + e] += y[e];
-            }
-            tc_fence_before();
-            mbar_arrive(&s_free);
-
-            // Masking only where it can apply (warp-uniform: a warp's rows share a head).
+            for (int c = 0; c < BLK / 32; ++c) tmem_ld32f(t_s + c * 32, x + c * 32);
+            tc_wait_ld();
             const bool keep = (mask >> rg) & 1u;
             const bool whole = keep && j != i && (j + 1) * BLK <= a.L;
             if (!whole) {
-                const int lim = (j == i) ? rr : BLK - 1;          // causal limit inside the block
-                const int lim_t = min(lim, a.L - 1 - j * BLK);    // short last block
+                const int lim = (j == i) ? rr : BLK - 1;
+                const int lim_t = min(lim, a.L - 1 - j * BLK);
 #pragma unroll
                 for (int c = 0; c < BLK; ++c) x[c] = (keep && c <= lim_t) ? x[c] : -INFINITY;
             }
-            // Row max of the raw scores with 8 independent chains.
             float mp[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) mp[e] = x[e];
@@ -300,62 +273,51 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int c = 8; c < BLK; ++c) mp[c & 7] = fmaxf(mp[c & 7], x[c]);
             const float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
                                    fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7]))) *
-                             a.scale_log2;                 // log2 units
+                             a.scale_log2;
             float alpha = 1.f;
             bool rescale = false;
             if (mx > m_used + kRescaleThreshold) {
-                alpha = fast_exp2(m_used - mx);               // 0 when m_used = -inf
+                alpha = fast_exp2(m_used - mx);
                 rescale = l > 0.f;
                 m_used = mx;
             }
             const float base = m_used == -INFINITY ? 0.f : m_used;
-            // p = 2^(s * scale * log2 e - m): one FFMA and one MUFU op per score;
-            // the row sum with 8 independent chains; P packed to bf16 pairs.
             float sp[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) sp[e] = 0.f;
-            uint32_t pk[BLK / 2];
-#pragma unroll
-            for (int c = 0; c < BLK / 2; ++c) {
-                const float p0 = fast_exp2(fmaf(x[2 * c], a.scale_log2, -base));
-                const float p1 = fast_exp2(fmaf(x[2 * c + 1], a.scale_log2, -base));
-                sp[(2 * c) & 7] += p0;
-                sp[(2 * c + 1) & 7] += p1;
-                pk[c] = pack_bf16x2(p0, p1);
-            }
-            const float rs = ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
-            l = l * alpha + rs;
-
-            // The previous P V has read P and updated O before either is touched.
-            if (n > 0) {
-                if (!mbar_wait(&o_done, (n - 1) & 1, a.err)) { ok = false; break; }
-                tc_fence_after();
-                if (__any_sync(0xffffffffu, rescale)) {   // rare: the max grew by > 8
+            // O is stable: the previous P V completed before S(n) did.
+            if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll 1
-                    for (int c = 0; c < kD / 32; ++c) {
-                        uint32_t o0[32];
-                        tmem_ld32(t_o + c * 32, o0);
-                        tc_wait_ld();
+                for (int c = 0; c < kD / 32; ++c) {
+                    uint32_t o0[32];
+                    tmem_ld32(t_o + c * 32, o0);
+                    tc_wait_ld();
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) o0[e] = __float_as_uint(__uint_as_float(o0[e]) * alpha);
-                        tmem_st32(t_o + c * 32, o0);
-                    }
+                    for (int e = 0; e < 32; ++e) o0[e] = __float_as_uint(__uint_as_float(o0[e]) * alpha);
+                    tmem_st32(t_o + c * 32, o0);
                 }
             }
 #pragma unroll
             for (int c = 0; c < BLK / 32; ++c) {
                 uint32_t w[16];
 #pragma unroll
-                for (int e = 0; e < 16; ++e) w[e] = pk[c * 16 + e];
-                tmem_st16(t_p + c * 16, w);
+                for (int e = 0; e < 16; ++e) {
+                    const float p0 = fast_exp2(fmaf(x[c * 32 + 2 * e], a.scale_log2, -base));
+                    const float p1 = fast_exp2(fmaf(x[c * 32 + 2 * e + 1], a.scale_log2, -base));
+                    sp[(2 * e) & 7] += p0;
+                    sp[(2 * e + 1) & 7] += p1;
+                    w[e] = pack_bf16x2(p0, p1);
+                }
+                tmem_st16(t_s + c * 16, w);
             }
+            const float rs = ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
+            l = l * alpha + rs;
             tc_wait_st();
             tc_fence_before();
             mbar_arrive(&p_ready);
             ++n;
         }
-        // ------------------------------------------------------------ epilogue
-        if (ok && n > 0) ok = mbar_wait(&o_done, (n - 1) & 1, a.err);
+        if (ok && n > 0) ok = mbar_wait(&o_done, 0, a.err);
         tc_fence_after();
         const bool store = t < a.L;
         const float inv = (l > 0.f) ? 1.f / l : 0.f;
@@ -373,12 +335,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (store) {
 #pragma unroll
                 for (int e = 0; e < 32; e += 8) {
-                    uint4 w;
-                    w.x = pack_bf16x2(__uint_as_float(v[e + 0]) * inv, __uint_as_float(v[e + 1]) * inv);
-                    w.y = pack_bf16x2(__uint_as_float(v[e + 2]) * inv, __uint_as_float(v[e + 3]) * inv);
-                    w.z = pack_bf16x2(__uint_as_float(v[e + 4]) * inv, __uint_as_float(v[e + 5]) * inv);
-                    w.w = pack_bf16x2(__uint_as_float(v[e + 6]) * inv, __uint_as_float(v[e + 7]) * inv);
-                    *reinterpret_cast<uint4 *>(orow + c * 32 + e) = w;
+                    uint4 w4;
+                    w4.x = pack_bf16x2(__uint_as_float(v[e + 0]) * inv, __uint_as_float(v[e + 1]) * inv);
+                    w4.y = pack_bf16x2(__uint_as_float(v[e + 2]) * inv, __uint_as_float(v[e + 3]) * inv);
+                    w4.z = pack_bf16x2(__uint_as_float(v[e + 4]) * inv, __uint_as_float(v[e + 5]) * inv);
+                    w4.w = pack_bf16x2(__uint_as_float(v[e + 6]) * inv, __uint_as_float(v[e + 7]) * inv);
+                    *reinterpret_cast<uint4 *>(orow + c * 32 + e) = w4;
                 }
             }
         }
@@ -389,7 +351,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     if (warp == 5) {
         tc_fence_after();
-        tmem_dealloc(tmem, 512);
+        tmem_dealloc(tmem, 256);
     }
 }
 
