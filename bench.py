@@ -56,6 +56,22 @@ def load_peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
+def captured_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu capture of `kernel`, or None when
+    the kernel's source changed since the capture (or none was taken)."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            rec = json.load(f)[kernel]
+        with open(os.path.join(ROOT, "block_sparse_long_stats_b200", "csrc", "prefill_tc.cu"), "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()
+    except (OSError, KeyError, ValueError):
+        return None
+    if rec.get("source_sha256") != sha or rec.get("workload") != workload:
+        return None
+    return float(rec["dram_bytes_per_launch"])
+
+
 # ---------------------------------------------------------------- algorithmic work
 
 def kept_flops(count: np.ndarray, idx: np.ndarray, L: int, block: int, d: int) -> float:
@@ -220,6 +236,8 @@ def main():
     ap.add_argument("--workload", type=int, default=3)
     ap.add_argument("--decode-workload", type=int, default=5)
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--decode-batch", type=int, default=None,
+                    help="override the decode workload's batch (smaller captures for profiling)")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-tokens", type=int, default=192)
@@ -360,6 +378,8 @@ def main():
     decode = None
     if not args.no_decode:
         wd = WORKLOADS[args.decode_workload]
+        if args.decode_batch:
+            wd = wd.with_(B=args.decode_batch)
         xd = generate(wd)
         qd_ = torch.from_numpy(np.ascontiguousarray(xd["q"]).view(np.int16)).cuda().view(torch.bfloat16)
         kc = torch.from_numpy(np.ascontiguousarray(xd["k"]).view(np.int16)).cuda().view(torch.bfloat16)
@@ -439,7 +459,10 @@ def main():
             "roofline": {"bound": "tensor", "kernel": "sparse_attn_prefill", "achieved": achieved,
                          "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                          "peak_source": f"{peak_src} bf16_tflops_sustained",
-                         "kept_flops_per_launch": F, "traffic": None},
+                         "kept_flops_per_launch": F,
+                         "traffic": captured_traffic("prefill_tc_kernel<128>", w.name),
+                         "traffic_unit": "bytes per launch (ncu dram read + write)",
+                         "algorithmic_bytes": float(2 * q.numel() * 2 + 2 * k.numel() * 2)},
             "kernels": per_kernel,
             "decode": decode,
             "e2e": e2e,
