@@ -25,7 +25,7 @@ _cache = {}
 
 
 def inputs(w):
-    key = (w.name, w.T, w.B, w.block, w.Hq, w.Hkv)
+    key = (w.name, w.T, w.B, w.block, w.Hq, w.Hkv)  # the data depend on these only
     if key not in _cache:
         x = generate(w)
         _cache.clear()
@@ -314,4 +314,22 @@ def test_prefill_head_groupings(Hq, Hkv, block):
                                     sel["count"], w.scale)
     assert np.abs(to_host(out) - o_out).max() <= TOL[w.dtype]
     np.testing.assert_allclose(lse.cpu().numpy(), o_lse, rtol=0, atol=LSE_TOL[w.dtype])
+    assert_no_device_error()
+
+
+@pytest.mark.parametrize("p,k_min", [(0.9, 0), (1e-4, 0), (0.3, 200), (1.0, 0), (0.999, 0)])
+def test_decode_select_long_residual_rule_variants(p, k_min):
+    # 1250 candidate blocks per head: the selection's wide (register-held) cut.
+    w = PARITY_WORKLOADS["d_bf16_blk16"].with_(T=20000, B=2, top_p=p, k_min=k_min)
+    x, dev = inputs(w)
+    r = spa.decode(dev["q"], dev["k"], dev["v"], w.block, p, scale=w.scale, k_min=k_min)
+    torch.cuda.synchronize()
+    sel = oracle_select(w, x)
+    check_lists(w, r["idx"], r["count"], sel, 1)
+    o_out, _ = oracle.attention(x["q"], x["k"], x["v"], w.dtype, w.block, sel["idx"], sel["count"],
+                                w.scale)
+    same = all(np.array_equal(r["idx"].cpu().numpy()[b, h, 0, :c], sel["idx"][b, h, 0, :c])
+               for b in range(w.B) for h in range(w.Hq) for c in [sel["count"][b, h, 0]])
+    if same:
+        assert np.abs(to_host(r["out"]) - o_out).max() <= TOL[w.dtype]
     assert_no_device_error()
