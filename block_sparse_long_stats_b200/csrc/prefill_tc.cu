@@ -15,7 +15,8 @@
 // Per kept block n: S = Q K_j^T (8 MMAs, both operands K-major in shared memory,
 // fp32 accumulator in TMEM); the softmax scales by s*log2(e), takes exp2, keeps the
 // running max lazily (O is rescaled only when the max grows by more than 8, in
-// log2 units) and writes P as bf16 over the first BLK/2 columns of S; then
+// log2 units) and writes P as bf16 over the first BLK/2 columns of S (scaling and
+// row sums in packed f32x2 pairs, row maxima with three-operand max); then
 // O += P V_j reads P from tensor memory (A operand in TMEM, V in its TMA layout as
 // an MN-major B), the fastest measured form for that product.
 // Each CTA's chain is serial (S(n+1) overwrites P(n), so it is issued after
@@ -266,13 +267,16 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
                 for (int c = 0; c < BLK; ++c) x[c] = (keep && c <= lim_t) ? x[c] : -INFINITY;
             }
+            // Row maximum: eight independent chains of three-operand maxima.
             float mp[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) mp[e] = x[e];
+            for (int e = 0; e < 8; ++e) mp[e] = fmaxf(x[e], x[e + 8]);
 #pragma unroll
-            for (int c = 8; c < BLK; ++c) mp[c & 7] = fmaxf(mp[c & 7], x[c]);
-            const float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
-                                   fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7]))) *
+            for (int c = 16; c < BLK; c += 16)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) mp[e] = fmax3(mp[e], x[c + e], x[c + 8 + e]);
+            const float mx = fmax3(fmax3(mp[0], mp[1], mp[2]), fmax3(mp[3], mp[4], mp[5]),
+                                   fmaxf(mp[6], mp[7])) *
                              a.scale_log2;
             float alpha = 1.f;
             bool rescale = false;
@@ -282,9 +286,12 @@ __global__ void __launch_bounds__(kThreads, 2)
                 m_used = mx;
             }
             const float base = m_used == -INFINITY ? 0.f : m_used;
-            float sp[8];
+            // Exponent arguments and row sums in packed pairs.
+            uint64_t sp[4];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) sp[e] = 0.f;
+            for (int e = 0; e < 4; ++e) sp[e] = 0ull;
+            const uint64_t scale2 = f32x2(a.scale_log2, a.scale_log2);
+            const uint64_t nbase2 = f32x2(-base, -base);
             // O is stable: the previous P V completed before S(n) did.
             if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll 1
@@ -302,15 +309,19 @@ __global__ void __launch_bounds__(kThreads, 2)
                 uint32_t w[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
-                    const float p0 = fast_exp2(fmaf(x[c * 32 + 2 * e], a.scale_log2, -base));
-                    const float p1 = fast_exp2(fmaf(x[c * 32 + 2 * e + 1], a.scale_log2, -base));
-                    sp[(2 * e) & 7] += p0;
-                    sp[(2 * e + 1) & 7] += p1;
+                    float y0, y1;
+                    f32x2_split(fma_f32x2(f32x2(x[c * 32 + 2 * e], x[c * 32 + 2 * e + 1]), scale2,
+                                          nbase2),
+                                y0, y1);
+                    const float p0 = fast_exp2(y0), p1 = fast_exp2(y1);
+                    sp[e & 3] = add_f32x2(sp[e & 3], f32x2(p0, p1));
                     w[e] = pack_bf16x2(p0, p1);
                 }
                 tmem_st16(t_s + c * 16, w);
             }
-            const float rs = ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
+            float rs0, rs1;
+            f32x2_split(add_f32x2(add_f32x2(sp[0], sp[1]), add_f32x2(sp[2], sp[3])), rs0, rs1);
+            const float rs = rs0 + rs1;
             l = l * alpha + rs;
             tc_wait_st();
             tc_fence_before();
