@@ -51,8 +51,11 @@ def _bind(path: str):
                                               _P, _I, _P]
     lib.oracle_attention.argtypes = [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I,
                                      _P, _I, _P, _D, _P, _I64, _P, _P]
+    lib.oracle_rla.argtypes = [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I,
+                               _P, _I, _P, _P, _I64, _P, _P]
+    lib.oracle_rla_block_states.argtypes = [_P, _P, _I, _I, _I, _I, _I, _I, _P]
     for f in ("oracle_block_stats", "oracle_scores", "oracle_select_from_scores",
-              "oracle_attention"):
+              "oracle_attention", "oracle_rla", "oracle_rla_block_states"):
         getattr(lib, f).restype = _I
     return lib
 
@@ -179,6 +182,50 @@ def attention(q, k, v, dtype: str, block: int, idx: np.ndarray, count: np.ndarra
                                     _ptr(idx), cap, _ptr(count), float(scale), rp, n, _ptr(out),
                                     _ptr(lse)), "attention")
     return out, lse
+
+
+def rla(q, k, v, dtype: str, block: int, idx: np.ndarray, count: np.ndarray,
+        rows: np.ndarray | None = None):
+    """Residual Linear Attention (fp64): for each query row, the linear attention
+    with phi = exp over the causal tokens of the blocks its kept list leaves out.
+
+    Returns (out, mag): out [B,Hq,Lq,d] (or [len(rows), d]); mag is the same sum
+    with |v| in place of v (the magnitude that rounding errors scale with).
+    """
+    q, isb = _inp(q, dtype)
+    k, _ = _inp(k, dtype)
+    v, _ = _inp(v, dtype)
+    B, Hq, Lq, d = q.shape
+    Hkv, T = k.shape[1], k.shape[2]
+    idx = np.ascontiguousarray(idx, np.int32)
+    count = np.ascontiguousarray(count, np.int32)
+    cap = idx.shape[-1]
+    if rows is None:
+        n = B * Hq * Lq
+        out = np.empty((B, Hq, Lq, d), np.float64)
+        rp = None
+    else:
+        rows = np.ascontiguousarray(rows, np.int64)
+        n = rows.size
+        out = np.empty((n, d), np.float64)
+        rp = _ptr(rows)
+    mag = np.empty_like(out)
+    _check(_load().oracle_rla(_ptr(q), _ptr(k), _ptr(v), isb, B, Hq, Hkv, Lq, T, d, block,
+                              _ptr(idx), cap, _ptr(count), rp, n, _ptr(out), _ptr(mag)), "rla")
+    return out, mag
+
+
+def rla_block_states(k, v, dtype: str, block: int) -> np.ndarray:
+    """Per-block states W_j[e][c] = sum_{u in block j} v_u,e exp(k_u,c), fp64
+    [B, Hkv, nb, d, d]."""
+    k, isb = _inp(k, dtype)
+    v, _ = _inp(v, dtype)
+    B, Hkv, T, d = k.shape
+    nb = -(-T // block)
+    out = np.empty((B, Hkv, nb, d, d), np.float64)
+    _check(_load().oracle_rla_block_states(_ptr(k), _ptr(v), isb, B, Hkv, T, d, block, _ptr(out)),
+           "rla_block_states")
+    return out
 
 
 def full_lists(B: int, Hq: int, Lq: int, T: int, block: int):

@@ -19,6 +19,12 @@
  *   - "S2O", section 3: exact attention over the selected key tiles with the
  *     online-softmax state (m, l, acc). The oracle does not use online softmax: it
  *     builds the token mask and evaluates the textbook masked softmax per row.
+ *   - "SPLA - Block Sparse Plus Linear Attention for Long Context Modeling",
+ *     sections 2.2-2.3 (Residual Linear Attention): the tokens of the blocks the
+ *     selection did not keep enter a linear-attention branch with the
+ *     parameter-free exponential feature map; its output is the global linear
+ *     attention minus the linear attention over the kept blocks, i.e. the linear
+ *     attention over the unkept (residual) tokens alone.
  *
  * Readings where the pages are silent (each applies to one function below):
  *   - the Taylor score is expanded with the attention's own scale s, i.e.
@@ -31,7 +37,12 @@
  *     crosses p is kept; p >= 1 keeps the whole residual; equal scores order by
  *     the smaller block index;
  *   - the cut is decided on fp32 scores (the kernel's precision): the fp64 score is
- *     rounded to fp32 first; masses and their prefix sums are fp64.
+ *     rounded to fp32 first; masses and their prefix sums are fp64;
+ *   - Residual Linear Attention: the feature map is phi(x) = exp(x) per component,
+ *     applied to q and k as given (no softmax scale), and the branch output is the
+ *     unnormalised sum  o_t = sum_u (phi(q_t) . phi(k_u)) v_u  over the causal
+ *     residual tokens u; the gate and the RMS-norm scale that follow it on the
+ *     page are trained parameters and are not part of the oracle.
  *
  * Inputs are fp32 arrays or bf16 bit patterns (uint16); bf16 widens to fp32
  * exactly, and all arithmetic below is fp64.
@@ -368,4 +379,121 @@ int oracle_attention(const void *q, const void *k, const void *v, int is_bf16,
         free(z);
     }
     return err;
+}
+
+/*
+ * Residual Linear Attention ("SPLA", sections 2.2-2.3), row by row. For query row
+ * t of (b, h) at position pos = T - Lq + t, in query block i = t / block, the
+ * residual tokens are
+ *   U(t) = { u <= pos : block(u) is NOT in the kept list of (b, h, i) },
+ * the complement of the exact branch's token set among the causal tokens. With
+ * phi(x) = exp(x) per component,
+ *   a_u   = phi(q_t) . phi(k_u) = sum_c exp(q_t,c) exp(k_u,c),
+ *   o_t   = sum_{u in U(t)} a_u v_u,
+ *   mag_t = sum_{u in U(t)} a_u |v_u|   (per component; the scale that rounding
+ *                                        errors of any evaluation order act on).
+ * rows: flat row ids r = (b*Hq + h)*Lq + t, or NULL for every row in order.
+ * out, mag: [nrows, d] (mag may be NULL).
+ */
+int oracle_rla(const void *q, const void *k, const void *v, int is_bf16,
+               int B, int Hq, int Hkv, int Lq, int T, int d, int block,
+               const int32_t *idx, int cap, const int32_t *count,
+               const int64_t *rows, int64_t nrows, double *out, double *mag)
+{
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || T <= 0 || d <= 0 || block <= 0)
+        return ORACLE_EINVAL;
+    if (!(Lq == T || Lq == 1)) return ORACLE_EINVAL;
+    const int nb = ceil_div(T, block), nq = ceil_div(Lq, block), G = Hq / Hkv;
+    if (cap < 1) return ORACLE_EINVAL;
+    if (!rows) nrows = (int64_t)B * Hq * Lq;
+    int err = 0;
+#pragma omp parallel
+    {
+        unsigned char *kept = (unsigned char *)malloc((size_t)nb);
+        double *phq = (double *)malloc(sizeof(double) * d);
+        if (!kept || !phq) {
+#pragma omp atomic write
+            err = ORACLE_ENOMEM;
+        }
+#pragma omp for schedule(dynamic, 4)
+        for (int64_t n = 0; n < nrows; ++n) {
+            if (!kept || !phq) continue;
+            const int64_t r = rows ? rows[n] : n;
+            const int64_t bh = r / Lq;
+            const int t = (int)(r % Lq);
+            const int b = (int)(bh / Hq), h = (int)(bh % Hq), g = h / G;
+            const int pos = T - Lq + t;
+            const int i = t / block;
+            const size_t u_list = ((size_t)bh * nq + i);
+            memset(kept, 0, (size_t)nb);
+            int cnt = count[u_list];
+            int bad = cnt < 0 || cnt > cap;
+            for (int c = 0; c < cnt && !bad; ++c) {
+                int j = idx[u_list * cap + c];
+                if (j < 0 || j >= nb) bad = 1; else kept[j] = 1;
+            }
+            if (bad) {
+#pragma omp atomic write
+                err = ORACLE_EINVAL;
+                continue;
+            }
+            const size_t qoff = (size_t)r * d;
+            const size_t kvbase = ((size_t)b * Hkv + g) * T;
+            for (int c = 0; c < d; ++c) phq[c] = exp(elem(q, is_bf16, qoff + c));
+            double *o = out + (size_t)n * d;
+            double *m = mag ? mag + (size_t)n * d : NULL;
+            for (int c = 0; c < d; ++c) {
+                o[c] = 0.0;
+                if (m) m[c] = 0.0;
+            }
+            for (int u = 0; u <= pos; ++u) {
+                if (kept[u / block]) continue;
+                double a = 0.0;
+                for (int c = 0; c < d; ++c)
+                    a += phq[c] * exp(elem(k, is_bf16, (kvbase + u) * d + c));
+                for (int c = 0; c < d; ++c) {
+                    const double vu = elem(v, is_bf16, (kvbase + u) * d + c);
+                    o[c] += a * vu;
+                    if (m) m[c] += a * fabs(vu);
+                }
+            }
+        }
+        free(kept);
+        free(phq);
+    }
+    return err;
+}
+
+/*
+ * Per-block linear-attention state of the exponential feature map ("SPLA",
+ * section 2.2: the recurrent state that unselected blocks are folded into):
+ *   W_j[e][c] = sum_{u in block j, u < T} v_u,e exp(k_u,c),
+ * i.e. the transpose of phi(K_j)^T V_j, for each (b, g, j). The branch output
+ * of a row is then phi(q_t) contracted with the sum of W_j over its residual
+ * blocks (plus the causal part of a residual diagonal block).
+ * out: [B, Hkv, nb, d, d] fp64, out[..., e, c] = W_j[e][c].
+ */
+int oracle_rla_block_states(const void *k, const void *v, int is_bf16, int B, int Hkv, int T,
+                            int d, int block, double *out)
+{
+    if (B <= 0 || Hkv <= 0 || T <= 0 || d <= 0 || block <= 0) return ORACLE_EINVAL;
+    const int nb = ceil_div(T, block);
+    const int64_t units = (int64_t)B * Hkv * nb;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t n = 0; n < units; ++n) {
+        const int64_t bg = n / nb;
+        const int j = (int)(n % nb);
+        double *w = out + (size_t)n * d * d;
+        for (size_t x = 0; x < (size_t)d * d; ++x) w[x] = 0.0;
+        const int u_end = (j + 1) * block < T ? (j + 1) * block : T;
+        for (int u = j * block; u < u_end; ++u) {
+            const size_t row = ((size_t)bg * T + u) * d;
+            for (int e = 0; e < d; ++e) {
+                const double ve = elem(v, is_bf16, row + e);
+                for (int c = 0; c < d; ++c)
+                    w[(size_t)e * d + c] += ve * exp(elem(k, is_bf16, row + c));
+            }
+        }
+    }
+    return ORACLE_OK;
 }

@@ -47,6 +47,20 @@ MUTATIONS = [
      [pins.test_top_p_hand_worked_examples]),
     ("local_window_too_wide", "(j > jmax - n_local)", "(j >= jmax - n_local)",
      [pins.test_top_p_hand_worked_examples]),
+    ("rla_sums_kept_blocks", "if (kept[u / block]) continue;", "if (!kept[u / block]) continue;",
+     [pins.test_rla_hand_worked_examples, pins.test_rla_is_zero_when_every_causal_block_is_kept,
+      pins.test_rla_global_minus_kept_equals_residual]),
+    ("rla_strict_causal", "for (int u = 0; u <= pos; ++u) {\n                if (kept",
+     "for (int u = 0; u < pos; ++u) {\n                if (kept",
+     [pins.test_rla_hand_worked_examples, pins.test_rla_global_minus_kept_equals_residual]),
+    ("rla_linear_kernel_feature_map", "a += phq[c] * exp(elem(k, is_bf16, (kvbase + u) * d + c));",
+     "a += log(phq[c]) * elem(k, is_bf16, (kvbase + u) * d + c);",
+     [pins.test_rla_hand_worked_examples, pins.test_rla_query_shift_scales_output,
+      pins.test_rla_unit_features_sum_residual_values]),
+    ("rla_states_transposed", "w[(size_t)e * d + c] += ve * exp(", "w[(size_t)c * d + e] += ve * exp(",
+     [pins.test_rla_block_states_contract_to_residual_output]),
+    ("rla_magnitude_without_abs", "m[c] += a * fabs(vu);", "m[c] += a * vu;",
+     [pins.test_rla_hand_worked_examples]),
     ("ascending_sort", "if (x->key > y->key) return -1;\n    if (x->key < y->key) return 1;",
      "if (x->key < y->key) return -1;\n    if (x->key > y->key) return 1;",
      [pins.test_top_p_hand_worked_examples, pins.test_top_p_tiny_p_keeps_top_one]),

@@ -479,3 +479,181 @@ def test_oracle_rejects_bad_lists():
     cnt = np.array([[[2]]], np.int32)
     with pytest.raises(RuntimeError):
         oracle.attention(q, q, q, "f32", 8, idx, cnt, 1.0)
+
+
+# ---------------------------------------------------------------- residual linear attention
+# SPLA, sections 2.2-2.3: the unkept blocks enter a linear-attention branch with the
+# feature map phi = exp; its output is the global linear attention minus the linear
+# attention over the kept blocks.
+
+def _rla_golden_inputs(g):
+    q = np.array(g["q"], np.float32)[None, None]
+    k = np.array(g["k"], np.float32)[None, None]
+    v = np.array(g["v"], np.float32)[None, None]
+    return q, k, v
+
+
+def test_rla_hand_worked_examples():
+    g = _golden()["rla"]
+    q, k, v = _rla_golden_inputs(g)
+    for tag in ("A", "B"):
+        lists = g["lists_" + tag]
+        idx = np.array(lists["idx"], np.int32)[None, None]
+        cnt = np.array(lists["count"], np.int32)[None, None]
+        out, mag = oracle.rla(q, k, v, "f32", g["block"], idx, cnt)
+        np.testing.assert_allclose(out[0, 0], np.array(g["expected_" + tag]), rtol=1e-14, atol=1e-14)
+        if tag == "B":
+            np.testing.assert_allclose(mag[0, 0, 3], g["expected_B_mag_row3"], rtol=1e-14)
+    dl = g["decode_list"]
+    out, _ = oracle.rla(q[:, :, 3:4], k, v, "f32", g["block"],
+                        np.array(dl["idx"], np.int32).reshape(1, 1, 1, 2),
+                        np.array([dl["count"]], np.int32).reshape(1, 1, 1))
+    np.testing.assert_allclose(out[0, 0, 0], g["expected_decode"], rtol=1e-14)
+
+
+def test_rla_is_zero_when_every_causal_block_is_kept():
+    q, k, v = _rand((1, 4, 70, 8), 41, 0.5), _rand((1, 2, 70, 8), 42, 0.5), _rand((1, 2, 70, 8), 43)
+    idx, cnt = oracle.full_lists(1, 4, 70, 70, 16)
+    out, mag = oracle.rla(q, k, v, "f32", 16, idx, cnt)
+    assert np.all(out == 0.0) and np.all(mag == 0.0)
+
+
+def _residual_token_mask(idx, cnt, Lq, T, block, b, h, t):
+    i = t // block
+    kept = set(int(j) for j in idx[b, h, i, :cnt[b, h, i]])
+    pos = T - Lq + t
+    return np.array([(u <= pos) and (u // block not in kept) for u in range(T)])
+
+
+def test_rla_unit_features_sum_residual_values():
+    # q = k = 0: phi = 1, every weight is d, so the output is d times the plain sum of
+    # the residual tokens' values.
+    B, Hq, Hkv, T, d, blk = 1, 2, 1, 40, 4, 8
+    q = np.zeros((B, Hq, T, d), np.float32)
+    k = np.zeros((B, Hkv, T, d), np.float32)
+    v = _rand((B, Hkv, T, d), 44)
+    idx, cnt = _random_lists(B, Hq, T, blk, 45)
+    out, _ = oracle.rla(q, k, v, "f32", blk, idx, cnt)
+    for h in range(Hq):
+        for t in range(T):
+            m = _residual_token_mask(idx, cnt, T, T, blk, 0, h, t)
+            np.testing.assert_allclose(out[0, h, t], d * v[0, 0][m].astype(np.float64).sum(axis=0),
+                                       rtol=1e-13, atol=1e-13)
+
+
+def test_rla_global_minus_kept_equals_residual():
+    # The subtraction form: linear attention over every causal token (global),
+    # minus that over the kept blocks, is the residual branch. Global and kept parts
+    # are evaluated here as masked matrix products.
+    B, Hq, Hkv, T, d, blk = 1, 2, 2, 48, 6, 8
+    q, k, v = _rand((B, Hq, T, d), 46, 0.4), _rand((B, Hkv, T, d), 47, 0.4), _rand((B, Hkv, T, d), 48)
+    # lists that may leave out the sink and the query's own (diagonal) block
+    rng = np.random.default_rng(49)
+    nb = T // blk
+    idx = np.full((B, Hq, nb, nb), -1, np.int32)
+    cnt = np.zeros((B, Hq, nb), np.int32)
+    for h in range(Hq):
+        for i in range(nb):
+            keep = [j for j in range(i + 1) if rng.random() < 0.5]
+            idx[0, h, i, :len(keep)] = keep
+            cnt[0, h, i] = len(keep)
+    assert any(cnt[0, h, i] == 0 or idx[0, h, i, cnt[0, h, i] - 1] != i
+               for h in range(Hq) for i in range(nb))
+    out, _ = oracle.rla(q, k, v, "f32", blk, idx, cnt)
+    for h in range(Hq):
+        A = np.exp(q[0, h].astype(np.float64)) @ np.exp(k[0, h].astype(np.float64)).T
+        causal = np.tril(np.ones((T, T)))
+        kept = np.zeros((T, T))
+        for t in range(T):
+            i = t // blk
+            for j in idx[0, h, i, :cnt[0, h, i]]:
+                kept[t, j * blk:(j + 1) * blk] = 1
+        kept *= causal
+        o_global = (A * causal) @ v[0, h].astype(np.float64)
+        o_kept = (A * kept) @ v[0, h].astype(np.float64)
+        np.testing.assert_allclose(out[0, h], o_global - o_kept, rtol=1e-10, atol=1e-10)
+
+
+def test_rla_block_states_contract_to_residual_output():
+    # The chunked form: W_j = (phi(K_j)^T V_j)^T per block; a row whose own block is
+    # kept gets phi(q_t) contracted with the sum of W_j over its residual blocks.
+    B, Hq, Hkv, T, d, blk = 1, 4, 2, 64, 8, 16
+    q, k, v = _rand((B, Hq, T, d), 50, 0.4), _rand((B, Hkv, T, d), 51, 0.4), _rand((B, Hkv, T, d), 52)
+    W = oracle.rla_block_states(k, v, "f32", blk)
+    nb = T // blk
+    for g in range(Hkv):
+        for j in range(nb):
+            Kj = np.exp(k[0, g, j * blk:(j + 1) * blk].astype(np.float64))
+            Vj = v[0, g, j * blk:(j + 1) * blk].astype(np.float64)
+            np.testing.assert_allclose(W[0, g, j], (Kj.T @ Vj).T, rtol=1e-12)
+    idx, cnt = oracle.full_lists(B, Hq, T, T, blk)
+    rng = np.random.default_rng(53)
+    for h in range(Hq):
+        for i in range(nb):
+            keep = [j for j in range(i) if rng.random() < 0.5] + [i]
+            idx[0, h, i, :] = -1
+            idx[0, h, i, :len(keep)] = keep
+            cnt[0, h, i] = len(keep)
+    out, _ = oracle.rla(q, k, v, "f32", blk, idx, cnt)
+    for h in range(Hq):
+        g = h // (Hq // Hkv)
+        for i in range(nb):
+            res = [j for j in range(i) if j not in set(idx[0, h, i, :cnt[0, h, i]])]
+            S = sum((W[0, g, j] for j in res), np.zeros((d, d)))
+            rows = np.exp(q[0, h, i * blk:(i + 1) * blk].astype(np.float64))
+            np.testing.assert_allclose(out[0, h, i * blk:(i + 1) * blk], rows @ S.T, rtol=1e-11,
+                                       atol=1e-11)
+
+
+def test_rla_query_shift_scales_output():
+    # phi(q + c) = e^c phi(q) component-wise, so a uniform shift of the query scales
+    # the branch output by e^c (a dot-product feature map would not do this).
+    B, Hq, Hkv, T, d, blk = 1, 1, 1, 32, 4, 8
+    q, k, v = _rand((B, Hq, T, d), 54, 0.5), _rand((B, Hkv, T, d), 55, 0.5), _rand((B, Hkv, T, d), 56)
+    idx, cnt = _random_lists(B, Hq, T, blk, 57)
+    o0, _ = oracle.rla(q, k, v, "f32", blk, idx, cnt)
+    o1, _ = oracle.rla(q + np.float32(0.75), k, v, "f32", blk, idx, cnt)
+    np.testing.assert_allclose(o1, o0 * math.exp(0.75), rtol=1e-6)
+
+
+def test_rla_ignores_future_tokens_and_kept_blocks():
+    B, Hq, Hkv, T, d, blk = 1, 2, 1, 48, 4, 8
+    q, k, v = _rand((B, Hq, T, d), 58, 0.5), _rand((B, Hkv, T, d), 59, 0.5), _rand((B, Hkv, T, d), 60)
+    idx, cnt = _random_lists(B, Hq, T, blk, 61)
+    out, _ = oracle.rla(q, k, v, "f32", blk, idx, cnt)
+    t = 27                               # row in query block 3
+    k2, v2 = k.copy(), v.copy()
+    k2[:, :, t + 1:] += 3.0              # future tokens
+    v2[:, :, t + 1:] -= 5.0
+    for h in range(Hq):
+        for j in idx[0, h, 3, :cnt[0, h, 3]]:
+            if h == 0:                   # blocks head 0 keeps for this query block
+                k2[:, :, j * blk:min((j + 1) * blk, t + 1)] *= 2.0
+    out2, _ = oracle.rla(q, k2, v2, "f32", blk, idx, cnt)
+    np.testing.assert_allclose(out2[0, 0, t], out[0, 0, t], rtol=1e-13, atol=1e-13)
+
+
+def test_rla_decode_equals_prefill_last_row():
+    B, Hq, Hkv, T, d, blk = 2, 4, 2, 45, 4, 8
+    q, k, v = _rand((B, Hq, T, d), 62, 0.5), _rand((B, Hkv, T, d), 63, 0.5), _rand((B, Hkv, T, d), 64)
+    idx, cnt = _random_lists(B, Hq, T, blk, 65)
+    out, _ = oracle.rla(q, k, v, "f32", blk, idx, cnt)
+    i = (T - 1) // blk
+    od, _ = oracle.rla(q[:, :, T - 1:T], k, v, "f32", blk, idx[:, :, i:i + 1], cnt[:, :, i:i + 1])
+    np.testing.assert_allclose(od[:, :, 0], out[:, :, T - 1], rtol=1e-13, atol=1e-13)
+
+
+def test_rla_gqa_head_reads_its_group():
+    B, Hq, Hkv, T, d, blk = 1, 4, 2, 32, 4, 8
+    q = np.repeat(_rand((B, 1, T, d), 66, 0.5), Hq, axis=1)
+    k, v = _rand((B, Hkv, T, d), 67, 0.5), _rand((B, Hkv, T, d), 68)
+    idx, cnt = oracle.full_lists(B, Hq, T, T, blk)
+    idx[:, :, 3, :] = -1
+    idx[:, :, 3, 0] = 3
+    cnt[:, :, 3] = 1
+    out, _ = oracle.rla(q, k, v, "f32", blk, idx, cnt)
+    np.testing.assert_array_equal(out[0, 0], out[0, 1])
+    np.testing.assert_array_equal(out[0, 2], out[0, 3])
+    assert np.abs(out[0, 0, 31] - out[0, 2, 31]).max() > 1e-3
+    ref, _ = oracle.rla(q[:, 2:3], k[:, 1:2], v[:, 1:2], "f32", blk, idx[:, 2:3], cnt[:, 2:3])
+    np.testing.assert_array_equal(out[0, 2], ref[0, 0])
