@@ -238,6 +238,8 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--decode-batch", type=int, default=None,
                     help="override the decode workload's batch (smaller captures for profiling)")
+    ap.add_argument("--no-rla", action="store_true",
+                    help="skip the Residual Linear Attention leg")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-tokens", type=int, default=192)
@@ -374,6 +376,44 @@ def main():
            "d2h_bytes_per_step": int(oh.numel() * 2), "ms_per_step": e2e_ms}
     del qh, kh, vh, oh, qd, kd, vd
 
+    # ---- Residual Linear Attention leg (the branch over the blocks the lists leave out)
+    rla = None
+    if not args.no_rla:
+        states = torch.empty((B, Hkv, nb, d, d), device="cuda", dtype=torch.bfloat16)
+        rout = torch.empty((B, Hq, L, d), device="cuda", dtype=torch.float32)
+        for _ in range(3):
+            spa.spa_rla_block_states(k, v, w.block, states=states)
+            spa.spa_rla_prefill(q, k, v, states, w.block, idx, cnt, out=rout)
+        torch.cuda.synchronize()
+        assert spa.spa_get_device_error() == 0
+        n_rla = max(10, args.steps // 2)
+        r_evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_rla)]
+        barrier()
+        torch.cuda.synchronize()
+        for s in range(n_rla):
+            flush.zero_()
+            r_evs[s][0].record(stream)
+            spa.spa_rla_block_states(k, v, w.block, states=states)
+            r_evs[s][1].record(stream)
+            spa.spa_rla_prefill(q, k, v, states, w.block, idx, cnt, out=rout)
+            r_evs[s][2].record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        t_st = rank_max(statistics.mean(e[0].elapsed_time(e[1]) for e in r_evs))
+        t_rla = rank_max(statistics.mean(e[1].elapsed_time(e[2]) for e in r_evs))
+        # residual blocks before each query block (its own block is always kept here)
+        n_res = float(sum(i for i in range(nb)) * B * Hq - (count_h.sum() - B * Hq * nb))
+        st_bytes = 2 * k.numel() * 2 + states.numel() * 2
+        rla_flops = n_res * 2 * 128 * d * d
+        rla = {"states_ms": t_st, "states_GB/s": st_bytes / (t_st / 1e3) / 1e9,
+               "states_bytes": st_bytes, "branch_ms": t_rla,
+               "residual_blocks": n_res, "branch_flops": rla_flops,
+               "branch_TFLOP/s": rla_flops / (t_rla / 1e3) / 1e12,
+               "branch_state_bytes_read": n_res * d * d * 2,
+               "tokens/s_with_branch": job_throughput(B * L, world, 1,
+                                                      ms_per_step + t_st + t_rla)}
+        del states, rout
+
     # ---- decode leg
     decode = None
     if not args.no_decode:
@@ -464,6 +504,7 @@ def main():
                          "traffic_unit": "bytes per launch (ncu dram read + write)",
                          "algorithmic_bytes": float(2 * q.numel() * 2 + 2 * k.numel() * 2)},
             "kernels": per_kernel,
+            "rla": rla,
             "decode": decode,
             "e2e": e2e,
             "cpu_baseline": cpu,

@@ -31,6 +31,15 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, int B
                               const int32_t *count, float scale, void *out, float *lse, int *err,
                               cudaStream_t s);
 
+// Residual Linear Attention (bf16, d = 128, block 64 or 128): per-block states
+// W_j [B, Hkv, nb, d, d] bf16, and the prefill branch output [B, Hq, L, d] fp32.
+cudaError_t launch_rla_block_states(const void *k, const void *v, int B, int Hkv, int T, int block,
+                                    int blk_begin, int blk_end, void *states, int *err,
+                                    cudaStream_t s);
+cudaError_t launch_rla_prefill(const void *q, const void *k, const void *v, const void *states,
+                               int B, int Hq, int Hkv, int L, int block, const int32_t *idx, int cap,
+                               const int32_t *count, float *out, int *err, cudaStream_t s);
+
 int decode_splits(int B, int Hkv, int T, int block);
 size_t decode_workspace_bytes(int B, int Hq, int Hkv, int T, int d, int block);
 cudaError_t launch_decode(const void *q, const void *kc, const void *vc, int B, int Hq, int Hkv,

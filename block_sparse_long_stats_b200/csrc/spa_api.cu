@@ -173,6 +173,54 @@ SPA_API spa_status spa_sparse_attn_prefill(const void *q, const void *k, const v
     return e == cudaSuccess ? SPA_OK : cuda_fail(e, "prefill launch");
 }
 
+SPA_API spa_status spa_rla_block_states(const void *k, const void *v, spa_dtype dt, int B, int Hkv,
+                                        int T, int d, int block, int blk_begin, int blk_end,
+                                        void *states, spa_stream stream) {
+    t_last_error.clear();
+    if (!k || !v || !states) return fail(SPA_ERR_INVALID, "null pointer");
+    if (B <= 0 || Hkv <= 0 || T <= 0 || d <= 0 || block <= 0)
+        return fail(SPA_ERR_INVALID, "sizes must be positive");
+    if (dt != SPA_F32 && dt != SPA_BF16) return fail(SPA_ERR_INVALID, "unknown dtype");
+    const int nb = ceil_div(T, block);
+    if (blk_begin < 0 || blk_end > nb || blk_begin > blk_end)
+        return fail(SPA_ERR_INVALID, "need 0 <= blk_begin <= blk_end <= nb");
+    if (!aligned16(k) || !aligned16(v) || !aligned16(states))
+        return fail(SPA_ERR_INVALID, "tensors must be 16-byte aligned");
+    if (dt != SPA_BF16 || d != 128) return fail(SPA_ERR_UNSUPPORTED, "block states need bf16, d = 128");
+    if (block != 64 && block != 128) return fail(SPA_ERR_UNSUPPORTED, "block states need block 64 or 128");
+    int *err = device_error_ptr();
+    if (!err) return fail(SPA_ERR_CUDA, "device error word unavailable");
+    cudaError_t e = launch_rla_block_states(k, v, B, Hkv, T, block, blk_begin, blk_end, states, err,
+                                            static_cast<cudaStream_t>(stream));
+    if (e == cudaErrorNotSupported) return fail(SPA_ERR_UNSUPPORTED, "tensor map encoding unavailable");
+    return e == cudaSuccess ? SPA_OK : cuda_fail(e, "block states launch");
+}
+
+SPA_API spa_status spa_rla_prefill(const void *q, const void *k, const void *v, const void *states,
+                                   spa_dtype dt, int B, int Hq, int Hkv, int L, int d, int block,
+                                   const int32_t *idx, int cap, const int32_t *count, float *out,
+                                   spa_stream stream) {
+    t_last_error.clear();
+    if (!q || !k || !v || !states || !idx || !count || !out) return fail(SPA_ERR_INVALID, "null pointer");
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || L <= 0 || d <= 0 || block <= 0)
+        return fail(SPA_ERR_INVALID, "sizes must be positive");
+    if (Hq % Hkv) return fail(SPA_ERR_INVALID, "Hq must be a multiple of Hkv");
+    if (dt != SPA_F32 && dt != SPA_BF16) return fail(SPA_ERR_INVALID, "unknown dtype");
+    if (cap < ceil_div(L, block)) return fail(SPA_ERR_INVALID, "cap must be >= nb");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(states) || !aligned16(out))
+        return fail(SPA_ERR_INVALID, "tensors must be 16-byte aligned");
+    if (dt != SPA_BF16 || d != 128) return fail(SPA_ERR_UNSUPPORTED, "residual branch needs bf16, d = 128");
+    if (block != 64 && block != 128)
+        return fail(SPA_ERR_UNSUPPORTED, "residual branch needs block 64 or 128");
+    if (ceil_div(L, block) > 65536) return fail(SPA_ERR_UNSUPPORTED, "more than 65536 blocks");
+    int *err = device_error_ptr();
+    if (!err) return fail(SPA_ERR_CUDA, "device error word unavailable");
+    cudaError_t e = launch_rla_prefill(q, k, v, states, B, Hq, Hkv, L, block, idx, cap, count, out,
+                                       err, static_cast<cudaStream_t>(stream));
+    if (e == cudaErrorNotSupported) return fail(SPA_ERR_UNSUPPORTED, "tensor map encoding unavailable");
+    return e == cudaSuccess ? SPA_OK : cuda_fail(e, "residual branch launch");
+}
+
 SPA_API size_t spa_decode_workspace_bytes(int B, int Hq, int Hkv, int T, int d, int block) {
     if (B <= 0 || Hq <= 0 || Hkv <= 0 || T <= 0 || d <= 0 || block <= 0) return 0;
     return decode_workspace_bytes(B, Hq, Hkv, T, d, block);

@@ -52,12 +52,16 @@ def lib() -> ctypes.CDLL:
         L.spa_decode_workspace_bytes.restype = ctypes.c_size_t
         L.spa_sparse_attn_decode.argtypes = [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _I, _P,
                                              _F, _P, _P, _P]
+        L.spa_rla_block_states.argtypes = [_P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P]
+        L.spa_rla_prefill.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _I, _P, _P,
+                                      _P]
         L.spa_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_int)]
         L.spa_status_string.argtypes = [_I]
         L.spa_status_string.restype = ctypes.c_char_p
         L.spa_last_error.restype = ctypes.c_char_p
         for f in ("spa_block_stats", "spa_select", "spa_sparse_attn_prefill",
-                  "spa_sparse_attn_decode", "spa_get_device_error"):
+                  "spa_sparse_attn_decode", "spa_get_device_error", "spa_rla_block_states",
+                  "spa_rla_prefill"):
             getattr(L, f).restype = _I
         _lib = L
     return _lib
@@ -157,6 +161,38 @@ def spa_sparse_attn_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, b
                                          block, _ptr(idx), idx.shape[-1], _ptr(count), scale,
                                          _ptr(out), _ptr(lse), _stream(stream)))
     return out, lse
+
+
+def spa_rla_block_states(k: torch.Tensor, v: torch.Tensor, block: int, blk_begin: int = 0,
+                         blk_end: int | None = None, states: torch.Tensor | None = None,
+                         stream=None) -> torch.Tensor:
+    """Per-block linear-attention states W_j[e][c] = sum_u v_u[e] exp(k_u[c]):
+    [B, Hkv, nb, d, d] bf16."""
+    B, Hkv, T, d = k.shape
+    nb = -(-T // block)
+    if blk_end is None:
+        blk_end = nb
+    if states is None:
+        states = torch.empty((B, Hkv, nb, d, d), device=k.device, dtype=torch.bfloat16)
+    _check("spa_rla_block_states",
+           lib().spa_rla_block_states(_ptr(k), _ptr(v), _dt(k), B, Hkv, T, d, block, blk_begin,
+                                      blk_end, _ptr(states), _stream(stream)))
+    return states
+
+
+def spa_rla_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, states: torch.Tensor,
+                    block: int, idx: torch.Tensor, count: torch.Tensor,
+                    out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Residual Linear Attention branch of prefill: [B, Hq, L, d] fp32."""
+    B, Hq, L, d = q.shape
+    Hkv = k.shape[1]
+    if out is None:
+        out = torch.empty((B, Hq, L, d), device=q.device, dtype=torch.float32)
+    _check("spa_rla_prefill",
+           lib().spa_rla_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(states), _dt(q), B, Hq, Hkv, L, d,
+                                 block, _ptr(idx), idx.shape[-1], _ptr(count), _ptr(out),
+                                 _stream(stream)))
+    return out
 
 
 def spa_decode_workspace_bytes(B: int, Hq: int, Hkv: int, T: int, d: int, block: int) -> int:

@@ -7,6 +7,8 @@
  *   spa_select       -> per (batch, query head, query block) kept-block list
  *   spa_sparse_attn_prefill / spa_sparse_attn_decode -> exact attention over the
  *                       kept blocks only
+ *   spa_rla_block_states / spa_rla_prefill -> (optional) linear attention with an
+ *                       exponential feature map over the blocks left out
  *
  * Conventions shared by every call
  *   - All tensors are dense, contiguous, row-major, in DEVICE memory, allocated and
@@ -174,6 +176,50 @@ spa_status spa_sparse_attn_decode_noalloc(const void *q, const void *kc, const v
                                           int block, const int32_t *idx, int cap,
                                           const int32_t *count, float scale, void *out,
                                           spa_stream stream);
+
+/*
+ * Residual Linear Attention, block states. Follows "SPLA - Block Sparse Plus Linear
+ * Attention for Long Context Modeling", section 2.2: the tokens of blocks that a
+ * kept list leaves out are folded into a linear-attention state with the feature
+ * map phi(x) = exp(x) (per component, on k as given). Per (b, g, block j):
+ *   states[b,g,j,e,c] = sum_{t in block j, t < T} v[b,g,t,e] * exp(k[b,g,t,c])
+ * i.e. the transpose of phi(K_j)^T V_j, rounded to bf16.
+ *   k, v   : [B, Hkv, T, d], dt = SPA_BF16, d = 128, block 64 or 128
+ *   blk_begin, blk_end : blocks [blk_begin, blk_end) are computed (0, nb for all);
+ *            others are left untouched
+ *   states : [B, Hkv, nb, d, d] bf16 output, 16-byte aligned
+ * exp is evaluated in fp32 and rounded to bf16 before the product (fp32
+ * accumulation); keys above about 88 overflow to inf.
+ */
+spa_status spa_rla_block_states(const void *k, const void *v, spa_dtype dt, int B, int Hkv, int T,
+                                int d, int block, int blk_begin, int blk_end, void *states,
+                                spa_stream stream);
+
+/*
+ * Residual Linear Attention, prefill branch output. Follows "SPLA ...", sections
+ * 2.2-2.3: alongside the exact attention over the kept blocks, each query row gets
+ * the linear attention over the causal tokens of the blocks its kept list leaves
+ * out (the residual):
+ *   out[b,h,t,:] = sum over u <= t with block(u) not kept by (b, h, t / block) of
+ *                  (sum_c exp(q[b,h,t,c]) exp(k[b,g,u,c])) v[b,g,u,:]
+ * (unnormalised; the page follows it with a trained gate and RMS-norm scale, which
+ * are the caller's). The residual blocks before the query's own block are
+ * contracted through `states`; the own block, when the list leaves it out, is
+ * evaluated token by token with the causal mask. The kept lists are read with the
+ * attention kernels' rule (entries outside [0, i] or not ascending are skipped and
+ * reported as SPA_DEVERR_BAD_INDEX; counts are clamped to [0, cap]).
+ *   q      : [B, Hq, L, d]; k, v : [B, Hkv, L, d]; dt = SPA_BF16, d = 128,
+ *            block 64 or 128, ceil(L / block) <= 65536
+ *   states : spa_rla_block_states of the same k, v, block (all blocks)
+ *   idx, count : kept lists as for spa_sparse_attn_prefill
+ *   out    : [B, Hq, L, d] fp32
+ * exp(q) and the masked scores of the own block are rounded to bf16 before their
+ * products (fp32 accumulation).
+ */
+spa_status spa_rla_prefill(const void *q, const void *k, const void *v, const void *states,
+                           spa_dtype dt, int B, int Hq, int Hkv, int L, int d, int block,
+                           const int32_t *idx, int cap, const int32_t *count, float *out,
+                           spa_stream stream);
 
 /*
  * Reads and clears the device error word of the current device (one of

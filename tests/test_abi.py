@@ -111,6 +111,25 @@ def test_prefill_and_decode_host_checks(lib):
     assert g(FAKE, FAKE, FAKE, 1, 1, 4, 2, 256, 128, 16, FAKE, 16, FAKE, 0.1, None, FAKE, None) == 1
 
 
+def test_rla_host_checks(lib):
+    I = ctypes.c_int
+    f = lib.spa_rla_block_states
+    f.argtypes = [P, P, I, I, I, I, I, I, I, I, P, P]
+    assert f(FAKE, FAKE, 0, 1, 2, 256, 128, 128, 0, 2, FAKE, None) == 2     # fp32
+    assert f(FAKE, FAKE, 1, 1, 2, 256, 64, 128, 0, 2, FAKE, None) == 2      # d = 64
+    assert f(FAKE, FAKE, 1, 1, 2, 256, 128, 16, 0, 16, FAKE, None) == 2     # block 16
+    assert f(FAKE, FAKE, 1, 1, 2, 256, 128, 128, 0, 3, FAKE, None) == 1     # blk_end > nb
+    assert f(FAKE, FAKE, 1, 1, 2, 256, 128, 128, 2, 1, FAKE, None) == 1     # begin > end
+    assert f(FAKE, None, 1, 1, 2, 256, 128, 128, 0, 2, FAKE, None) == 1
+    g = lib.spa_rla_prefill
+    g.argtypes = [P, P, P, P, I, I, I, I, I, I, I, P, I, P, P, P]
+    assert g(FAKE, FAKE, FAKE, FAKE, 0, 1, 4, 2, 256, 128, 128, FAKE, 2, FAKE, FAKE, None) == 2
+    assert g(FAKE, FAKE, FAKE, FAKE, 1, 1, 4, 2, 256, 128, 32, FAKE, 8, FAKE, FAKE, None) == 2
+    assert g(FAKE, FAKE, FAKE, FAKE, 1, 1, 4, 2, 256, 128, 128, FAKE, 1, FAKE, FAKE, None) == 1
+    assert g(FAKE, FAKE, FAKE, FAKE, 1, 1, 4, 3, 256, 128, 128, FAKE, 2, FAKE, FAKE, None) == 1
+    assert g(FAKE, FAKE, FAKE, None, 1, 1, 4, 2, 256, 128, 128, FAKE, 2, FAKE, FAKE, None) == 1
+
+
 def test_decode_workspace_size(lib):
     f = lib.spa_decode_workspace_bytes
     f.restype = ctypes.c_size_t
