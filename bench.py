@@ -468,12 +468,54 @@ def main():
         t_dec = rank_max(statistics.mean(e[1].elapsed_time(e[2]) for e in d_evs))
         dbytes = kept_kv_bytes(dcnt.cpu().numpy(), didx.cpu().numpy(), wd.G, wd.T, wd.block, wd.d)
         gbs = dbytes / (t_dec / 1e3) / 1e9
+        drla = None
+        if not args.no_rla:
+            dstate = torch.zeros((wd.B, wd.Hkv, wd.d, wd.d), device="cuda", dtype=torch.float32)
+            ws_r = torch.empty(spa.spa_rla_decode_workspace_bytes(wd.B, wd.Hq, wd.Hkv, wd.T, wd.d,
+                                                                  wd.block),
+                               dtype=torch.uint8, device="cuda")
+            orla = torch.empty(qd_.shape, device="cuda", dtype=torch.float32)
+            sb_ms = []
+            for _ in range(4):
+                flush.zero_()
+                dstate.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                spa.spa_rla_decode_state(kc, vc, state=dstate)
+                e1.record(stream)
+                torch.cuda.synchronize()
+                sb_ms.append(e0.elapsed_time(e1))
+            for _ in range(3):
+                spa.spa_sparse_attn_decode_rla(qd_, kc, vc, dstate, wd.block, didx, dcnt, wd.scale,
+                                               workspace=ws_r, out=dout, out_rla=orla)
+            torch.cuda.synchronize()
+            assert spa.spa_get_device_error() == 0
+            r_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                     for _ in range(n_dec)]
+            barrier()
+            torch.cuda.synchronize()
+            for s in range(n_dec):
+                flush.zero_()
+                r_evs[s][0].record(stream)
+                spa.spa_sparse_attn_decode_rla(qd_, kc, vc, dstate, wd.block, didx, dcnt, wd.scale,
+                                               workspace=ws_r, out=dout, out_rla=orla)
+                r_evs[s][1].record(stream)
+            torch.cuda.synchronize()
+            barrier()
+            t_drla = rank_max(statistics.mean(a_.elapsed_time(b_) for a_, b_ in r_evs))
+            sb = statistics.median(sb_ms[1:])
+            drla = {"state_build_ms": sb,
+                    "state_build_GB/s": 2 * kc.numel() * 2 / (sb / 1e3) / 1e9,
+                    "attn_with_branch_ms": t_drla,
+                    "GB/s": (dbytes + dstate.numel() * 4) / (t_drla / 1e3) / 1e9,
+                    "tokens/s": world * wd.B / ((t_dsel + t_drla) / 1e3)}
+            del dstate, ws_r, orla
         decode = {"workload": wd.name, "kept_kv_bytes": dbytes, "attn_ms": t_dec,
                   "select_ms": t_dsel, "GB/s": gbs, "peak_GB/s": peaks["hbm_gbs"],
                   "frac": gbs / peaks["hbm_gbs"], "peak_source": peak_src,
                   "tokens/s": world * wd.B / ((t_dsel + t_dec) / 1e3),
                   "kept_fraction": float(dcnt.float().mean().item()) / wd.nb,
-                  "block_stats_full_cache": stats_full}
+                  "block_stats_full_cache": stats_full, "rla": drla}
         del kc, vc
 
     # ---- CPU oracle baseline (rank 0, one GPU)

@@ -59,6 +59,14 @@ __device__ __forceinline__ float fast_exp2(float x) {
     return y;
 }
 
+// exp of two bf16 values (a packed pair), rounded back to bf16: the exponential
+// feature map of the linear-attention branch. Every kernel that applies it uses this
+// one function, so the same key gets the same rounded feature everywhere.
+__device__ __forceinline__ uint32_t exp_bf16x2(uint32_t w) {
+    constexpr float kLog2eF = 1.4426950408889634f;
+    return pack_bf16x2(fast_exp2(bf16lo(w) * kLog2eF), fast_exp2(bf16hi(w) * kLog2eF));
+}
+
 // ------------------------------------------------------------------ shared memory
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));

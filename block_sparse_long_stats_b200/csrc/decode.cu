@@ -39,6 +39,13 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t &r0, uint32_t 
                  : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
                  : "r"(addr));
 }
+// Transpose of an 8x8 bf16 matrix held one 32-bit pair per lane (row lane / 4,
+// columns 2 (lane % 4) and +1), returned in the same distribution.
+__device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
+    uint32_t y;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+    return y;
+}
 __device__ __forceinline__ void mma_bf16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                          uint32_t a3, uint32_t b0, uint32_t b1) {
     asm volatile(
@@ -60,6 +67,7 @@ struct DecodeArgs {
     const int32_t *idx;
     const int32_t *count;
     float *ws;        // [B*Hq][splits][D + 2]
+    float *ws_rla;    // [B*Hq][splits][D]: kept-token linear branch (RLA variant only)
     int Hq, Hkv, T, nb, G, cap, splits, R;
     float scale_log2;
     int *err;
@@ -67,7 +75,17 @@ struct DecodeArgs {
 
 // Each stage of the ring is always consumed by the same warp (stage % CONS), so a
 // warp never waits on a stage two phases ahead (the mbarrier parity would alias).
-template <int BLOCK, int STAGES, int CONS>
+//
+// RLA variant ("SPLA", sections 2.2-2.3, subtraction form): the warps also take the
+// linear attention with feature map exp over the kept tokens of every head,
+//   ot[head][e] = sum_{u kept} (exp(q_head) . exp(k_u)) v_u[e],
+// from the tiles already in shared memory; the combine subtracts it from the
+// global state's exp(q) . P. Per 16 keys: A'[key][head] = exp(K) exp(q)^T with keys
+// on the MMA rows (the group's heads, at most 8, are the columns), split into bf16
+// hi + lo parts so the kept sum is not rounded as a whole (it cancels against the
+// global state), transposed in registers (movmatrix) and applied as
+// ot^T += V^T A'^T.
+template <int BLOCK, int STAGES, int CONS, bool RLA>
 __global__ void __launch_bounds__((CONS + 1) * 32) decode_kernel(const __grid_constant__ CUtensorMap tk,
                                                           const __grid_constant__ CUtensorMap tv,
                                                           DecodeArgs a) {
@@ -190,6 +208,19 @@ __global__ void __launch_bounds__((CONS + 1) * 32) decode_kernel(const __grid_co
         float o[16][4];
 #pragma unroll
         for (int nt = 0; nt < 16; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
+        // RLA: exp(q) as the B operand (k = d, n = head gq) and the kept-token branch
+        // ot^T [d][head] (rows mt*16 + gq and + 8, heads 2 tq and 2 tq + 1).
+        uint32_t fq[RLA ? 8 : 1][2];
+        float ot[RLA ? 8 : 1][4];
+        if constexpr (RLA) {
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                fq[ks][0] = gq < a.G ? exp_bf16x2(qa[ks][0]) : 0u;
+                fq[ks][1] = gq < a.G ? exp_bf16x2(qa[ks][2]) : 0u;
+            }
+#pragma unroll
+            for (int mt = 0; mt < 8; ++mt) ot[mt][0] = ot[mt][1] = ot[mt][2] = ot[mt][3] = 0.f;
+        }
         float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;   // rows gq, gq + 8
 
         // ldmatrix lane geometry
@@ -272,6 +303,40 @@ __global__ void __launch_bounds__((CONS + 1) * 32) decode_kernel(const __grid_co
                     mma_bf16(o[dt + 1], a0, a1, a2, a3, v2, v3);
                 }
             }
+            if constexpr (RLA) {
+                const bool hk0 = (msk >> (2 * tq)) & 1u, hk1 = (msk >> (2 * tq + 1)) & 1u;
+#pragma unroll
+                for (int kt16 = 0; kt16 < BLOCK / 16; ++kt16) {
+                    float sa[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks) {
+                        uint32_t k0, k1, k2, k3;
+                        ldsm_x4(kt + swz<BLOCK>(kt16 * 16 + (lm & 1) * 8 + lr, ks * 2 + (lm >> 1)),
+                                k0, k1, k2, k3);
+                        mma_bf16(sa, exp_bf16x2(k0), exp_bf16x2(k1), exp_bf16x2(k2),
+                                 exp_bf16x2(k3), fq[ks][0], fq[ks][1]);
+                    }
+                    // keep keys inside the cache and heads that kept this block
+                    const int key0 = j * BLOCK + kt16 * 16 + gq, key1 = key0 + 8;
+                    const float a0 = (key0 < a.T && hk0) ? sa[0] : 0.f;
+                    const float a1 = (key0 < a.T && hk1) ? sa[1] : 0.f;
+                    const float a2 = (key1 < a.T && hk0) ? sa[2] : 0.f;
+                    const float a3 = (key1 < a.T && hk1) ? sa[3] : 0.f;
+                    const uint32_t h01 = pack_bf16x2(a0, a1), h23 = pack_bf16x2(a2, a3);
+                    const uint32_t l01 = pack_bf16x2(a0 - bf16lo(h01), a1 - bf16hi(h01));
+                    const uint32_t l23 = pack_bf16x2(a2 - bf16lo(h23), a3 - bf16hi(h23));
+                    const uint32_t bh0 = movmatrix_t(h01), bh1 = movmatrix_t(h23);
+                    const uint32_t bl0 = movmatrix_t(l01), bl1 = movmatrix_t(l23);
+#pragma unroll
+                    for (int mt = 0; mt < 8; ++mt) {
+                        uint32_t v0, v1, v2, v3;
+                        ldsm_x4_t(vt + swz<BLOCK>(kt16 * 16 + (lm >> 1) * 8 + lr, mt * 2 + (lm & 1)),
+                                  v0, v1, v2, v3);
+                        mma_bf16(ot[mt], v0, v1, v2, v3, bh0, bh1);
+                        mma_bf16(ot[mt], v0, v1, v2, v3, bl0, bl1);
+                    }
+                }
+            }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[s]);
         }
@@ -319,13 +384,45 @@ __global__ void __launch_bounds__((CONS + 1) * 32) decode_kernel(const __grid_co
                 dst[kD + 1] = L;
             }
         }
+        if constexpr (RLA) {
+            // sum the warps' kept-token branch (plain sums: no softmax scaling)
+            asm volatile("bar.sync 1, %0;" ::"n"(kConsumers * 32) : "memory");
+#pragma unroll
+            for (int mt = 0; mt < 8; ++mt) {
+                const int e = mt * 16 + gq;
+                if (2 * tq < a.G) {
+                    xo[(warp * a.G + 2 * tq) * kD + e] = ot[mt][0];
+                    xo[(warp * a.G + 2 * tq) * kD + e + 8] = ot[mt][2];
+                }
+                if (2 * tq + 1 < a.G) {
+                    xo[(warp * a.G + 2 * tq + 1) * kD + e] = ot[mt][1];
+                    xo[(warp * a.G + 2 * tq + 1) * kD + e + 8] = ot[mt][3];
+                }
+            }
+            asm volatile("bar.sync 1, %0;" ::"n"(kConsumers * 32) : "memory");
+            for (int x = tid; x < a.G * kD; x += kConsumers * 32) {
+                const int row = x / kD, c = x % kD;
+                float O = 0.f;
+#pragma unroll
+                for (int w = 0; w < kConsumers; ++w) O += xo[(w * a.G + row) * kD + c];
+                a.ws_rla[(((size_t)b * a.Hq + g * a.G + row) * a.splits + split) * kD + c] = O;
+            }
+        }
     }
 }
 
 // Merge the split partials of one (b, h): o = sum_s acc_s 2^(m_s - M) / sum_s l_s 2^(m_s - M).
+// RLA variant: also out_rla = exp(q) . P[b, g] - sum_s ot_s, with exp(q) rounded to
+// bf16 exactly as the decode kernel's fragments, so the kept tokens cancel.
+template <bool RLA>
 __global__ void __launch_bounds__(kD) decode_combine_kernel(const float *__restrict__ ws,
                                                             int splits,
-                                                            __nv_bfloat16 *__restrict__ out) {
+                                                            __nv_bfloat16 *__restrict__ out,
+                                                            const float *__restrict__ ws_rla,
+                                                            const __nv_bfloat16 *__restrict__ q,
+                                                            const float *__restrict__ state,
+                                                            int Hq, int G,
+                                                            float *__restrict__ out_rla) {
     const int bh = blockIdx.x, c = threadIdx.x;
     const float *p = ws + (size_t)bh * splits * (kD + 2);
     float M = -INFINITY;
@@ -338,6 +435,25 @@ __global__ void __launch_bounds__(kD) decode_combine_kernel(const float *__restr
         O += p[s * (kD + 2) + c] * f;
     }
     out[(size_t)bh * kD + c] = __float2bfloat16_rn(L > 0.f ? O / L : 0.f);
+    if constexpr (RLA) {
+        __shared__ float fq[kD];
+        const uint32_t e2 = exp_bf16x2(reinterpret_cast<const uint32_t *>(q + (size_t)bh * kD)[c >> 1]);
+        fq[c] = (c & 1) ? bf16hi(e2) : bf16lo(e2);
+        __syncthreads();
+        const int b = bh / Hq, g = (bh % Hq) / G;
+        const float *prow = state + (((size_t)b * (Hq / G) + g) * kD + c) * kD;   // row e = c
+        float ob = 0.f;
+        for (int x = 0; x < kD; x += 4) {
+            const float4 p4 = *reinterpret_cast<const float4 *>(prow + x);
+            ob = fmaf(fq[x], p4.x, ob);
+            ob = fmaf(fq[x + 1], p4.y, ob);
+            ob = fmaf(fq[x + 2], p4.z, ob);
+            ob = fmaf(fq[x + 3], p4.w, ob);
+        }
+        float ot = 0.f;
+        for (int s = 0; s < splits; ++s) ot += ws_rla[((size_t)bh * splits + s) * kD + c];
+        out_rla[(size_t)bh * kD + c] = ob - ot;
+    }
 }
 
 bool make_map(CUtensorMap *map, const void *base, uint64_t rows, int box_rows) {
@@ -359,14 +475,14 @@ constexpr int stages_for() {   // up to 128 KB of K/V in flight per CTA, 2..8 st
     return n < 2 ? 2 : (n > 8 ? 8 : n);
 }
 
-template <int BLOCK>
+template <int BLOCK, bool RLA>
 cudaError_t launch_b(const CUtensorMap &tk, const CUtensorMap &tv, const DecodeArgs &a, int B,
                      cudaStream_t s) {
     constexpr int STAGES = stages_for<BLOCK>();
     constexpr int CONS = STAGES < 4 ? STAGES : 4;
     const size_t smem = 1024 + (size_t)STAGES * 2 * BLOCK * kD * 2 + (size_t)a.R * 4 +
                         (size_t)CONS * a.G * kD * 4;
-    auto kern = decode_kernel<BLOCK, STAGES, CONS>;
+    auto kern = decode_kernel<BLOCK, STAGES, CONS, RLA>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)a.splits, (unsigned)(B * a.Hkv));
@@ -392,11 +508,17 @@ size_t decode_workspace_bytes(int B, int Hq, int Hkv, int T, int d, int block) {
     return (size_t)B * Hq * decode_splits(B, Hkv, T, block) * (d + 2) * sizeof(float);
 }
 
+// The RLA variant appends the kept-token branch partials, 256-byte aligned.
+size_t decode_rla_workspace_bytes(int B, int Hq, int Hkv, int T, int d, int block) {
+    const size_t base = (decode_workspace_bytes(B, Hq, Hkv, T, d, block) + 255) & ~size_t(255);
+    return base + (size_t)B * Hq * decode_splits(B, Hkv, T, block) * d * sizeof(float);
+}
+
 cudaError_t launch_decode(const void *q, const void *kc, const void *vc, int B, int Hq, int Hkv,
                           int T, int d, int block, const int32_t *idx, int cap,
                           const int32_t *count, float scale, void *workspace, void *out, int *err,
-                          cudaStream_t s) {
-    (void)d;
+                          cudaStream_t s, const float *rla_state, float *out_rla) {
+    const bool rla = out_rla != nullptr;
     CUtensorMap tk, tv;
     const uint64_t rows = (uint64_t)B * Hkv * T;
     if (!make_map(&tk, kc, rows, block) || !make_map(&tv, vc, rows, block))
@@ -406,6 +528,10 @@ cudaError_t launch_decode(const void *q, const void *kc, const void *vc, int B, 
     a.idx = idx;
     a.count = count;
     a.ws = reinterpret_cast<float *>(workspace);
+    a.ws_rla = rla ? reinterpret_cast<float *>(
+                         reinterpret_cast<unsigned char *>(workspace) +
+                         ((decode_workspace_bytes(B, Hq, Hkv, T, d, block) + 255) & ~size_t(255)))
+                   : nullptr;
     a.Hq = Hq; a.Hkv = Hkv; a.T = T;
     a.nb = (T + block - 1) / block;
     a.G = Hq / Hkv;
@@ -415,15 +541,29 @@ cudaError_t launch_decode(const void *q, const void *kc, const void *vc, int B, 
     a.scale_log2 = scale * kLog2e;
     a.err = err;
     cudaError_t e;
-    switch (block) {
-        case 16: e = launch_b<16>(tk, tv, a, B, s); break;
-        case 32: e = launch_b<32>(tk, tv, a, B, s); break;
-        case 64: e = launch_b<64>(tk, tv, a, B, s); break;
-        default: e = launch_b<128>(tk, tv, a, B, s); break;
+    if (rla) {
+        switch (block) {
+            case 16: e = launch_b<16, true>(tk, tv, a, B, s); break;
+            case 32: e = launch_b<32, true>(tk, tv, a, B, s); break;
+            default: e = launch_b<64, true>(tk, tv, a, B, s); break;
+        }
+    } else {
+        switch (block) {
+            case 16: e = launch_b<16, false>(tk, tv, a, B, s); break;
+            case 32: e = launch_b<32, false>(tk, tv, a, B, s); break;
+            case 64: e = launch_b<64, false>(tk, tv, a, B, s); break;
+            default: e = launch_b<128, false>(tk, tv, a, B, s); break;
+        }
     }
     if (e != cudaSuccess) return e;
-    decode_combine_kernel<<<(unsigned)(B * Hq), kD, 0, s>>>(a.ws, a.splits,
-                                                           reinterpret_cast<__nv_bfloat16 *>(out));
+    if (rla)
+        decode_combine_kernel<true><<<(unsigned)(B * Hq), kD, 0, s>>>(
+            a.ws, a.splits, reinterpret_cast<__nv_bfloat16 *>(out), a.ws_rla, a.q, rla_state, Hq,
+            a.G, out_rla);
+    else
+        decode_combine_kernel<false><<<(unsigned)(B * Hq), kD, 0, s>>>(
+            a.ws, a.splits, reinterpret_cast<__nv_bfloat16 *>(out), nullptr, nullptr, nullptr, Hq,
+            a.G, nullptr);
     return cudaGetLastError();
 }
 

@@ -42,10 +42,21 @@ cudaError_t launch_rla_prefill(const void *q, const void *k, const void *v, cons
 
 int decode_splits(int B, int Hkv, int T, int block);
 size_t decode_workspace_bytes(int B, int Hq, int Hkv, int T, int d, int block);
+size_t decode_rla_workspace_bytes(int B, int Hq, int Hkv, int T, int d, int block);
+// With out_rla set (block 16, 32 or 64; at most 8 query heads per kv-head) the
+// kernel also takes the kept-token linear branch and writes
+// out_rla = exp(q) . rla_state - (that branch); the workspace then needs
+// decode_rla_workspace_bytes.
 cudaError_t launch_decode(const void *q, const void *kc, const void *vc, int B, int Hq, int Hkv,
                           int T, int d, int block, const int32_t *idx, int cap,
                           const int32_t *count, float scale, void *workspace, void *out, int *err,
-                          cudaStream_t s);
+                          cudaStream_t s, const float *rla_state = nullptr,
+                          float *out_rla = nullptr);
+// Global linear-attention state of tokens [tok_begin, tok_end) added into
+// state [B, Hkv, d, d] fp32 (state[e][c] += sum_u v_u[e] exp(k_u[c])).
+cudaError_t launch_rla_decode_state(const void *k, const void *v, int B, int Hkv, int T,
+                                    int tok_begin, int tok_end, float *state, int *err,
+                                    cudaStream_t s);
 
 // Device address of the current device's error word (looked up once per device),
 // and the per-thread detail string spa_last_error returns; both live in spa_api.cu.

@@ -34,15 +34,9 @@ constexpr int kD = 128;
 constexpr int kThreads = 192;            // warps 0-3: exp / epilogue, 4: TMA, 5: MMA
 constexpr int kProducerWarp = 4;
 constexpr int kMmaWarp = 5;
-constexpr float kLog2e = 1.4426950408889634f;
-
 // exp(x) of 8 bf16 values held in a 16-byte chunk, rounded back to bf16.
 __device__ __forceinline__ uint4 exp_bf16x8(uint4 u) {
-    uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e)
-        w[e] = pack_bf16x2(fast_exp2(bf16lo(w[e]) * kLog2e), fast_exp2(bf16hi(w[e]) * kLog2e));
-    return make_uint4(w[0], w[1], w[2], w[3]);
+    return make_uint4(exp_bf16x2(u.x), exp_bf16x2(u.y), exp_bf16x2(u.z), exp_bf16x2(u.w));
 }
 
 // Applies exp to rows [0, nvalid) of a 128-column bf16 tile of `rows` rows stored as
@@ -542,6 +536,121 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
 }
 
+// ------------------------------------------------------------------ decode global state
+
+// state[b,g][e][c] += sum_{u in [tok_begin, tok_end)} v_u[e] exp(k_u[c]): the global
+// linear-attention state that decode's branch contracts with exp(q) (the pages'
+// "global context estimate"). CTA (split, b*Hkv + g) sums 128-token chunks
+// [c0, c1) of its range in one TMEM accumulator (same MMA as the block states)
+// and adds the result into `state` with fp32 atomics.
+struct RangeArgs {
+    float *state;                // [B, Hkv, d, d]
+    int T, tok_begin, tok_end, per_cta;
+    int *err;
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+    rla_range_state_kernel(const __grid_constant__ CUtensorMap tk,
+                           const __grid_constant__ CUtensorMap tv, RangeArgs a) {
+    using C = StCfg<128>;
+    constexpr int ST = C::STAGES;
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char *smem = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    __shared__ uint64_t full[ST], empty[ST], phi_ready[ST], acc_full;
+    __shared__ uint32_t tmem_slot;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int bg = blockIdx.y;
+    const int nch = (a.tok_end - a.tok_begin + 127) / 128;
+    const int c0 = blockIdx.x * a.per_cta;
+    const int nblk = min(nch, c0 + a.per_cta) - c0;
+
+    if (tid == 0) {
+        for (int s = 0; s < ST; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+            mbar_init(&phi_ready[s], 128);
+        }
+        mbar_init(&acc_full, 1);
+        fence_mbar_init();
+    }
+    if (warp == kMmaWarp) tmem_alloc(&tmem_slot, 128);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_slot;
+
+    if (warp == kProducerWarp) {
+        if (lane == 0) {
+            prefetch_tmap(&tk);
+            prefetch_tmap(&tv);
+            for (int n = 0; n < nblk; ++n) {
+                const int s = n % ST;
+                if (!mbar_wait(&empty[s], ((n / ST) & 1) ^ 1, a.err)) break;
+                const int row = bg * a.T + a.tok_begin + (c0 + n) * 128;
+                unsigned char *kt = smem + C::OFF_K + s * C::TILE;
+                unsigned char *vt = smem + C::OFF_V + s * C::TILE;
+                mbar_arrive_expect_tx(&full[s], 2 * C::TILE);
+                tma_load_2d(kt, &tk, &full[s], 0, row);
+                tma_load_2d(kt + C::HALF, &tk, &full[s], 64, row);
+                tma_load_2d(vt, &tv, &full[s], 0, row);
+                tma_load_2d(vt + C::HALF, &tv, &full[s], 64, row);
+            }
+        }
+    } else if (warp == kMmaWarp) {
+        if (lane == 0) {
+            bool ok = true;
+            for (int n = 0; n < nblk; ++n) {
+                const int s = n % ST;
+                if (!mbar_wait(&phi_ready[s], (n / ST) & 1, a.err)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t kb = smem_u32(smem + C::OFF_K + s * C::TILE);
+                const uint32_t vb = smem_u32(smem + C::OFF_V + s * C::TILE);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint64_t ad = sw128_desc(vb + kk * 2048, C::HALF, 1024);
+                    const uint64_t bd = sw128_desc(kb + kk * 2048, C::HALF, 1024);
+                    tc_mma_ss(tmem, ad, bd, C::IDESC, (n > 0 || kk > 0) ? 1u : 0u);
+                }
+                tc_commit(&empty[s]);
+            }
+            if (ok) tc_commit(&acc_full);
+        }
+    } else {
+        bool ok = true;
+        for (int n = 0; n < nblk; ++n) {
+            const int s = n % ST;
+            if (!mbar_wait(&full[s], (n / ST) & 1, a.err)) { ok = false; break; }
+            const int nvalid = min(128, a.tok_end - a.tok_begin - (c0 + n) * 128);
+            exp_tile(smem + C::OFF_K + s * C::TILE, 128, nvalid, tid, false);
+            if (nvalid < 128) exp_tile(smem + C::OFF_V + s * C::TILE, 128, nvalid, tid, true);
+            fence_async_shared();
+            mbar_arrive(&phi_ready[s]);
+        }
+        ok = __all_sync(0xffffffffu, ok && nblk > 0 && mbar_wait(&acc_full, 0, a.err));
+        if (ok) {
+            tc_fence_after();
+            const int e = warp * 32 + lane;
+            float *row = a.state + ((size_t)bg * kD + e) * kD;
+#pragma unroll 1
+            for (int c = 0; c < kD / 32; ++c) {
+                uint32_t v[32];
+                tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + c * 32, v);
+                tc_wait_ld();
+#pragma unroll
+                for (int x = 0; x < 32; ++x) atomicAdd(row + c * 32 + x, __uint_as_float(v[x]));
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 128);
+    }
+}
+
 bool make_map(CUtensorMap *map, const void *base, uint64_t rows, int box_rows) {
     EncodeTiledFn enc = encode_tiled_fn();
     if (!enc) return false;
@@ -600,6 +709,32 @@ cudaError_t launch_rla_blk(const void *q, const void *k, const void *v, const vo
 }
 
 }  // namespace
+
+cudaError_t launch_rla_decode_state(const void *k, const void *v, int B, int Hkv, int T,
+                                    int tok_begin, int tok_end, float *state, int *err,
+                                    cudaStream_t s) {
+    if (tok_end <= tok_begin) return cudaSuccess;
+    CUtensorMap mk, mv;
+    if (!make_map(&mk, k, (uint64_t)B * Hkv * T, 128) || !make_map(&mv, v, (uint64_t)B * Hkv * T, 128))
+        return cudaErrorNotSupported;
+    RangeArgs a;
+    a.state = state;
+    a.T = T;
+    a.tok_begin = tok_begin;
+    a.tok_end = tok_end;
+    a.err = err;
+    const int nch = (tok_end - tok_begin + 127) / 128;
+    // about two waves of one CTA per SM
+    const int splits = std::max(1, std::min(nch, (296 + B * Hkv - 1) / (B * Hkv)));
+    a.per_cta = (nch + splits - 1) / splits;
+    const size_t smem = StCfg<128>::SMEM + 1024;
+    cudaError_t e = cudaFuncSetAttribute(rla_range_state_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid((unsigned)((nch + a.per_cta - 1) / a.per_cta), (unsigned)(B * Hkv));
+    rla_range_state_kernel<<<grid, kThreads, smem, s>>>(mk, mv, a);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_rla_block_states(const void *k, const void *v, int B, int Hkv, int T, int block,
                                     int blk_begin, int blk_end, void *states, int *err,

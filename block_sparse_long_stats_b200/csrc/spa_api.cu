@@ -255,6 +255,63 @@ SPA_API spa_status spa_sparse_attn_decode(const void *q, const void *kc, const v
     return e == cudaSuccess ? SPA_OK : cuda_fail(e, "decode launch");
 }
 
+SPA_API spa_status spa_rla_decode_state(const void *kc, const void *vc, spa_dtype dt, int B,
+                                        int Hkv, int T, int d, int tok_begin, int tok_end,
+                                        float *state, spa_stream stream) {
+    t_last_error.clear();
+    if (!kc || !vc || !state) return fail(SPA_ERR_INVALID, "null pointer");
+    if (B <= 0 || Hkv <= 0 || T <= 0 || d <= 0) return fail(SPA_ERR_INVALID, "sizes must be positive");
+    if (dt != SPA_F32 && dt != SPA_BF16) return fail(SPA_ERR_INVALID, "unknown dtype");
+    if (tok_begin < 0 || tok_end > T || tok_begin > tok_end)
+        return fail(SPA_ERR_INVALID, "need 0 <= tok_begin <= tok_end <= T");
+    if (!aligned16(kc) || !aligned16(vc) || !aligned16(state))
+        return fail(SPA_ERR_INVALID, "tensors must be 16-byte aligned");
+    if (dt != SPA_BF16 || d != 128) return fail(SPA_ERR_UNSUPPORTED, "decode state needs bf16, d = 128");
+    int *err = device_error_ptr();
+    if (!err) return fail(SPA_ERR_CUDA, "device error word unavailable");
+    cudaError_t e = launch_rla_decode_state(kc, vc, B, Hkv, T, tok_begin, tok_end, state, err,
+                                            static_cast<cudaStream_t>(stream));
+    if (e == cudaErrorNotSupported) return fail(SPA_ERR_UNSUPPORTED, "tensor map encoding unavailable");
+    return e == cudaSuccess ? SPA_OK : cuda_fail(e, "decode state launch");
+}
+
+SPA_API size_t spa_rla_decode_workspace_bytes(int B, int Hq, int Hkv, int T, int d, int block) {
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || T <= 0 || d <= 0 || block <= 0) return 0;
+    return decode_rla_workspace_bytes(B, Hq, Hkv, T, d, block);
+}
+
+SPA_API spa_status spa_sparse_attn_decode_rla(const void *q, const void *kc, const void *vc,
+                                              const float *state, spa_dtype dt, int B, int Hq,
+                                              int Hkv, int T, int d, int block, const int32_t *idx,
+                                              int cap, const int32_t *count, float scale,
+                                              void *workspace, void *out, float *out_rla,
+                                              spa_stream stream) {
+    t_last_error.clear();
+    if (!q || !kc || !vc || !state || !idx || !count || !workspace || !out || !out_rla)
+        return fail(SPA_ERR_INVALID, "null pointer");
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || T <= 0 || d <= 0 || block <= 0)
+        return fail(SPA_ERR_INVALID, "sizes must be positive");
+    if (Hq % Hkv) return fail(SPA_ERR_INVALID, "Hq must be a multiple of Hkv");
+    if (!(scale > 0.f)) return fail(SPA_ERR_INVALID, "scale must be > 0");
+    if (cap < ceil_div(T, block)) return fail(SPA_ERR_INVALID, "cap must be >= nb");
+    if (!aligned16(q) || !aligned16(kc) || !aligned16(vc) || !aligned16(state) ||
+        !aligned16(workspace) || !aligned16(out) || !aligned16(out_rla))
+        return fail(SPA_ERR_INVALID, "tensors must be 16-byte aligned");
+    if (dt != SPA_BF16) return fail(SPA_ERR_UNSUPPORTED, "decode is bf16 only");
+    if (d != 128) return fail(SPA_ERR_UNSUPPORTED, "decode needs d = 128");
+    if (block != 16 && block != 32 && block != 64)
+        return fail(SPA_ERR_UNSUPPORTED, "decode with the linear branch needs block 16, 32 or 64");
+    if (Hq / Hkv > 8)
+        return fail(SPA_ERR_UNSUPPORTED, "the linear branch supports up to 8 query heads per kv-head");
+    int *err = device_error_ptr();
+    if (!err) return fail(SPA_ERR_CUDA, "device error word unavailable");
+    cudaError_t e = launch_decode(q, kc, vc, B, Hq, Hkv, T, d, block, idx, cap, count, scale,
+                                  workspace, out, err, static_cast<cudaStream_t>(stream), state,
+                                  out_rla);
+    if (e == cudaErrorNotSupported) return fail(SPA_ERR_UNSUPPORTED, "tensor map encoding unavailable");
+    return e == cudaSuccess ? SPA_OK : cuda_fail(e, "decode launch");
+}
+
 SPA_API spa_status spa_get_device_error(int *code) {
     t_last_error.clear();
     if (!code) return fail(SPA_ERR_INVALID, "null pointer");

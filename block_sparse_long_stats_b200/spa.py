@@ -55,13 +55,18 @@ def lib() -> ctypes.CDLL:
         L.spa_rla_block_states.argtypes = [_P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P]
         L.spa_rla_prefill.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _I, _P, _P,
                                       _P]
+        L.spa_rla_decode_state.argtypes = [_P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P]
+        L.spa_rla_decode_workspace_bytes.argtypes = [_I, _I, _I, _I, _I, _I]
+        L.spa_rla_decode_workspace_bytes.restype = ctypes.c_size_t
+        L.spa_sparse_attn_decode_rla.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P,
+                                                 _I, _P, _F, _P, _P, _P, _P]
         L.spa_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_int)]
         L.spa_status_string.argtypes = [_I]
         L.spa_status_string.restype = ctypes.c_char_p
         L.spa_last_error.restype = ctypes.c_char_p
         for f in ("spa_block_stats", "spa_select", "spa_sparse_attn_prefill",
                   "spa_sparse_attn_decode", "spa_get_device_error", "spa_rla_block_states",
-                  "spa_rla_prefill"):
+                  "spa_rla_prefill", "spa_rla_decode_state", "spa_sparse_attn_decode_rla"):
             getattr(L, f).restype = _I
         _lib = L
     return _lib
@@ -193,6 +198,51 @@ def spa_rla_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, states: t
                                  block, _ptr(idx), idx.shape[-1], _ptr(count), _ptr(out),
                                  _stream(stream)))
     return out
+
+
+def spa_rla_decode_state(kc: torch.Tensor, vc: torch.Tensor, tok_begin: int = 0,
+                         tok_end: int | None = None, state: torch.Tensor | None = None,
+                         stream=None) -> torch.Tensor:
+    """Adds sum_{t in [tok_begin, tok_end)} v_t exp(k_t)^T into state [B, Hkv, d, d]
+    fp32 (a zeroed state is made when none is given)."""
+    B, Hkv, T, d = kc.shape
+    if tok_end is None:
+        tok_end = T
+    if state is None:
+        state = torch.zeros((B, Hkv, d, d), device=kc.device, dtype=torch.float32)
+    _check("spa_rla_decode_state",
+           lib().spa_rla_decode_state(_ptr(kc), _ptr(vc), _dt(kc), B, Hkv, T, d, tok_begin,
+                                      tok_end, _ptr(state), _stream(stream)))
+    return state
+
+
+def spa_rla_decode_workspace_bytes(B: int, Hq: int, Hkv: int, T: int, d: int, block: int) -> int:
+    return int(lib().spa_rla_decode_workspace_bytes(B, Hq, Hkv, T, d, block))
+
+
+def spa_sparse_attn_decode_rla(q: torch.Tensor, kc: torch.Tensor, vc: torch.Tensor,
+                               state: torch.Tensor, block: int, idx: torch.Tensor,
+                               count: torch.Tensor, scale: float,
+                               workspace: torch.Tensor | None = None,
+                               out: torch.Tensor | None = None,
+                               out_rla: torch.Tensor | None = None, stream=None):
+    """Decode attention plus the linear branch over the unkept blocks.
+    Returns (out [B,Hq,1,d] bf16, out_rla [B,Hq,1,d] fp32)."""
+    B, Hq, _, d = q.shape
+    Hkv, T = kc.shape[1], kc.shape[2]
+    if workspace is None:
+        n = spa_rla_decode_workspace_bytes(B, Hq, Hkv, T, d, block)
+        workspace = torch.empty((max(n, 16),), device=q.device, dtype=torch.uint8)
+    if out is None:
+        out = torch.empty_like(q)
+    if out_rla is None:
+        out_rla = torch.empty(q.shape, device=q.device, dtype=torch.float32)
+    _check("spa_sparse_attn_decode_rla",
+           lib().spa_sparse_attn_decode_rla(_ptr(q), _ptr(kc), _ptr(vc), _ptr(state), _dt(q), B,
+                                            Hq, Hkv, T, d, block, _ptr(idx), idx.shape[-1],
+                                            _ptr(count), scale, _ptr(workspace), _ptr(out),
+                                            _ptr(out_rla), _stream(stream)))
+    return out, out_rla
 
 
 def spa_decode_workspace_bytes(B: int, Hq: int, Hkv: int, T: int, d: int, block: int) -> int:

@@ -7,7 +7,8 @@
  *   spa_select       -> per (batch, query head, query block) kept-block list
  *   spa_sparse_attn_prefill / spa_sparse_attn_decode -> exact attention over the
  *                       kept blocks only
- *   spa_rla_block_states / spa_rla_prefill -> (optional) linear attention with an
+ *   spa_rla_block_states / spa_rla_prefill, spa_rla_decode_state /
+ *   spa_sparse_attn_decode_rla -> (optional) linear attention with an
  *                       exponential feature map over the blocks left out
  *
  * Conventions shared by every call
@@ -220,6 +221,49 @@ spa_status spa_rla_prefill(const void *q, const void *k, const void *v, const vo
                            spa_dtype dt, int B, int Hq, int Hkv, int L, int d, int block,
                            const int32_t *idx, int cap, const int32_t *count, float *out,
                            spa_stream stream);
+
+/*
+ * Residual Linear Attention for decode, global state. Follows "SPLA ...", section
+ * 2.2: the global context estimate is linear attention over every cached token,
+ * kept as one state per (b, g):
+ *   state[b,g,e,c] += sum_{tok_begin <= t < tok_end} v[b,g,t,e] * exp(k[b,g,t,c])
+ * The call ADDS into state: zero it and pass [0, T) to build it, or pass the new
+ * tokens' range after appending them to the cache.
+ *   kc, vc : [B, Hkv, T, d] caches, dt = SPA_BF16, d = 128
+ *   state  : [B, Hkv, d, d] fp32, 16-byte aligned
+ * exp(k) is rounded to bf16 exactly as spa_sparse_attn_decode_rla rounds it;
+ * products are accumulated in fp32. Contributions of one call are added with fp32
+ * atomics, so the last bits can differ from call to call.
+ */
+spa_status spa_rla_decode_state(const void *kc, const void *vc, spa_dtype dt, int B, int Hkv,
+                                int T, int d, int tok_begin, int tok_end, float *state,
+                                spa_stream stream);
+
+/* Workspace bytes for spa_sparse_attn_decode_rla with these sizes (0 if invalid). */
+size_t spa_rla_decode_workspace_bytes(int B, int Hq, int Hkv, int T, int d, int block);
+
+/*
+ * spa_sparse_attn_decode plus the Residual Linear Attention branch. Follows
+ * "SPLA ...", sections 2.2-2.3, in the pages' subtraction form: the branch output
+ * is the global estimate minus the linear attention over the kept blocks, which
+ * the kernel evaluates from the K/V tiles it already loads for exact attention,
+ * so the blocks left out are never read:
+ *   out_rla[b,h,:] = sum_c exp(q[b,h,c]) state[b,g,:,c]
+ *                    - sum over kept tokens u of (sum_c exp(q[b,h,c]) exp(k[b,g,u,c])) v[b,g,u,:]
+ * (unnormalised; the gate and RMS-norm scale that follow it are the caller's).
+ *   state  : spa_rla_decode_state of the whole cache [0, T)
+ *   block  : 16, 32 or 64; at most 8 query heads per kv-head
+ *   workspace : >= spa_rla_decode_workspace_bytes(...) bytes, 16-byte aligned
+ *   out    : [B, Hq, 1, d] bf16 (as spa_sparse_attn_decode); out_rla: [B, Hq, 1, d] fp32
+ * exp(q) and exp(k) are rounded to bf16; each kept token's weight is applied as a
+ * bf16 pair (hi + lo), so the kept part cancels against the state to about 2^-16
+ * of its size.
+ */
+spa_status spa_sparse_attn_decode_rla(const void *q, const void *kc, const void *vc,
+                                      const float *state, spa_dtype dt, int B, int Hq, int Hkv,
+                                      int T, int d, int block, const int32_t *idx, int cap,
+                                      const int32_t *count, float scale, void *workspace,
+                                      void *out, float *out_rla, spa_stream stream);
 
 /*
  * Reads and clears the device error word of the current device (one of

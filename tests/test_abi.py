@@ -130,6 +130,32 @@ def test_rla_host_checks(lib):
     assert g(FAKE, FAKE, FAKE, None, 1, 1, 4, 2, 256, 128, 128, FAKE, 2, FAKE, FAKE, None) == 1
 
 
+def test_rla_decode_host_checks(lib):
+    I, F = ctypes.c_int, ctypes.c_float
+    f = lib.spa_rla_decode_state
+    f.argtypes = [P, P, I, I, I, I, I, I, I, P, P]
+    assert f(FAKE, FAKE, 0, 1, 2, 256, 128, 0, 256, FAKE, None) == 2       # fp32
+    assert f(FAKE, FAKE, 1, 1, 2, 256, 128, 0, 257, FAKE, None) == 1       # beyond T
+    assert f(FAKE, FAKE, 1, 1, 2, 256, 128, 9, 8, FAKE, None) == 1         # begin > end
+    assert f(FAKE, FAKE, 1, 1, 2, 256, 128, 0, 256, None, None) == 1
+    g = lib.spa_sparse_attn_decode_rla
+    g.argtypes = [P, P, P, P, I, I, I, I, I, I, I, P, I, P, F, P, P, P, P]
+    assert g(FAKE, FAKE, FAKE, FAKE, 1, 1, 4, 2, 256, 128, 128, FAKE, 2, FAKE, 0.1, FAKE, FAKE,
+             FAKE, None) == 2                                               # block 128
+    assert g(FAKE, FAKE, FAKE, FAKE, 1, 1, 32, 2, 256, 128, 16, FAKE, 16, FAKE, 0.1, FAKE, FAKE,
+             FAKE, None) == 2                                               # 16 heads per group
+    assert g(FAKE, FAKE, FAKE, FAKE, 1, 1, 4, 2, 256, 128, 16, FAKE, 16, FAKE, 0.1, FAKE, FAKE,
+             None, None) == 1                                               # no out_rla
+    h = lib.spa_rla_decode_workspace_bytes
+    h.restype = ctypes.c_size_t
+    h.argtypes = [I] * 6
+    d = lib.spa_decode_workspace_bytes
+    d.restype = ctypes.c_size_t
+    d.argtypes = [I] * 6
+    assert h(16, 32, 8, 131072, 128, 16) > d(16, 32, 8, 131072, 128, 16)
+    assert h(0, 32, 8, 131072, 128, 16) == 0
+
+
 def test_decode_workspace_size(lib):
     f = lib.spa_decode_workspace_bytes
     f.restype = ctypes.c_size_t

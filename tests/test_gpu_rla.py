@@ -183,3 +183,79 @@ def test_rla_prefill_full_size_sampled_rows():
                       r["count"].cpu().numpy(), rows=rows)
     print(f"\n{w.name}: worst |err| / mag = {within(g, o, m, w.name):.3e}")
     assert spa.spa_get_device_error() == 0
+
+
+# ------------------------------------------------------------------ decode (subtraction form)
+
+DECODE = [k for k, w in PARITY_WORKLOADS.items() if w.mode == "decode"]
+# The kept part cancels against the global state: besides the rounding of exp(q) and
+# exp(k) (two roundings on the residual), the fp32 sums of the state and of the kept
+# tokens differ by accumulation error relative to the whole cache's magnitude.
+GLOBAL_REL = 2.0 ** -12
+
+
+def test_decode_state_matches_oracle_and_adds_up():
+    w = PARITY_WORKLOADS["d_bf16_blk64"]
+    x, dev = inputs(w)
+    st = spa.spa_rla_decode_state(dev["k"], dev["v"])
+    torch.cuda.synchronize()
+    o = oracle.rla_block_states(x["k"], x["v"], "bf16", w.T)[:, :, 0]
+    m = oracle.rla_block_states(x["k"], abs_v(x)["v"], "bf16", w.T)[:, :, 0]
+    within(st.cpu().numpy().astype(np.float64), o, m, "decode state", 1)
+    st2 = spa.spa_rla_decode_state(dev["k"], dev["v"], 0, w.T - 5)
+    spa.spa_rla_decode_state(dev["k"], dev["v"], w.T - 5, w.T, state=st2)
+    torch.cuda.synchronize()
+    within(st2.cpu().numpy().astype(np.float64), o, m, "decode state in two calls", 1)
+    assert spa.spa_get_device_error() == 0
+
+
+def decode_rla_check(w, x, dev, idx, cnt, what):
+    st = spa.spa_rla_decode_state(dev["k"], dev["v"])
+    out, orla = spa.spa_sparse_attn_decode_rla(dev["q"], dev["k"], dev["v"], st, w.block,
+                                               torch.from_numpy(idx).cuda(),
+                                               torch.from_numpy(cnt).cuda(), w.scale)
+    torch.cuda.synchronize()
+    g = orla.cpu().numpy().astype(np.float64)
+    o, m = oracle.rla(x["q"], x["k"], x["v"], "bf16", w.block, idx, cnt)
+    _, m_all = oracle.rla(x["q"], x["k"], x["v"], "bf16", w.block, idx, np.zeros_like(cnt))
+    err = np.abs(g - o)
+    bound = (2 + 0.2) * U_BF16 * m + GLOBAL_REL * m_all.max(axis=-1, keepdims=True)
+    assert (err <= bound).all(), (what, float((err / bound).max()))
+    # the exact branch is unchanged by the linear one
+    ref = spa.spa_sparse_attn_decode(dev["q"], dev["k"], dev["v"], w.block,
+                                     torch.from_numpy(idx).cuda(), torch.from_numpy(cnt).cuda(),
+                                     w.scale)
+    assert torch.equal(out, ref)
+    print(f"\n{what}: worst err / bound = {float((err / bound).max()):.3e}, "
+          f"residual share of magnitude {float(m.sum() / m_all.sum()):.3f}")
+    assert spa.spa_get_device_error() == 0
+
+
+@pytest.mark.parametrize("top_p", [None, 0.3])
+@pytest.mark.parametrize("key", DECODE)
+def test_decode_rla_on_oracle_lists(key, top_p):
+    w = PARITY_WORKLOADS[key]
+    x, dev = inputs(w)
+    if top_p is not None:
+        w = w.with_(top_p=top_p)
+    sel = oracle.select(x["q"], x["k"], w.dtype, w.block, w.scale, w.top_p, w.n_sink, w.n_local,
+                        w.k_min)
+    decode_rla_check(w, x, dev, sel["idx"], sel["count"], f"{w.name} p={w.top_p}")
+
+
+def test_decode_rla_random_lists_and_edges():
+    w = PARITY_WORKLOADS["d_bf16_blk16"]
+    x, dev = inputs(w)
+    rng = np.random.default_rng(5)
+    idx = np.full((w.B, w.Hq, 1, w.nb), -1, np.int32)
+    cnt = np.zeros((w.B, w.Hq, 1), np.int32)
+    for b in range(w.B):
+        for h in range(w.Hq):
+            keep = [j for j in range(w.nb) if rng.random() < 0.5]
+            if h == 1:
+                keep = []                          # nothing kept: global linear attention
+            if h == 2:
+                keep = list(range(w.nb))           # everything kept: the branch is ~0
+            idx[b, h, 0, :len(keep)] = keep
+            cnt[b, h, 0] = len(keep)
+    decode_rla_check(w, x, dev, idx, cnt, "random lists")
