@@ -54,8 +54,11 @@ def _bind(path: str):
     lib.oracle_rla.argtypes = [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I,
                                _P, _I, _P, _P, _I64, _P, _P]
     lib.oracle_rla_block_states.argtypes = [_P, _P, _I, _I, _I, _I, _I, _I, _P]
+    lib.oracle_quantize_stats.argtypes = [_P, _P, _I, _I, _I, _I, _P, _P, _P, _P]
+    lib.oracle_dequantize_stats.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _P, _P]
     for f in ("oracle_block_stats", "oracle_scores", "oracle_select_from_scores",
-              "oracle_attention", "oracle_rla", "oracle_rla_block_states"):
+              "oracle_attention", "oracle_rla", "oracle_rla_block_states",
+              "oracle_quantize_stats", "oracle_dequantize_stats"):
         getattr(lib, f).restype = _I
     return lib
 
@@ -226,6 +229,49 @@ def rla_block_states(k, v, dtype: str, block: int) -> np.ndarray:
     _check(_load().oracle_rla_block_states(_ptr(k), _ptr(v), isb, B, Hkv, T, d, block, _ptr(out)),
            "rla_block_states")
     return out
+
+
+def quantize_stats(mean: np.ndarray, var: np.ndarray) -> dict:
+    """INT4 microscale block statistics (SpotAttention, section 4; the format is
+    documented at oracle_quantize_stats). Returns codes cm (int8), cv (uint8) shaped
+    like mean, and per-32-feature exponents km, kv (int8) [B, Hkv, nb, d / 32]."""
+    mean = np.ascontiguousarray(mean, np.float64)
+    var = np.ascontiguousarray(var, np.float64)
+    B, Hkv, nb, d = mean.shape
+    cm = np.empty(mean.shape, np.int8)
+    cv = np.empty(mean.shape, np.uint8)
+    km = np.empty((B, Hkv, nb, d // 32), np.int8)
+    kv = np.empty_like(km)
+    _check(_load().oracle_quantize_stats(_ptr(mean), _ptr(var), B, Hkv, nb, d, _ptr(cm), _ptr(cv),
+                                         _ptr(km), _ptr(kv)), "quantize_stats")
+    return {"cm": cm, "cv": cv, "km": km, "kv": kv}
+
+
+def dequantize_stats(qs: dict):
+    """(mean, var) fp64 from quantize_stats' codes: code * 2^k."""
+    cm = np.ascontiguousarray(qs["cm"], np.int8)
+    cv = np.ascontiguousarray(qs["cv"], np.uint8)
+    km = np.ascontiguousarray(qs["km"], np.int8)
+    kv = np.ascontiguousarray(qs["kv"], np.int8)
+    B, Hkv, nb, d = cm.shape
+    mean = np.empty(cm.shape, np.float64)
+    var = np.empty(cm.shape, np.float64)
+    _check(_load().oracle_dequantize_stats(_ptr(cm), _ptr(cv), _ptr(km), _ptr(kv), B, Hkv, nb, d,
+                                           _ptr(mean), _ptr(var)), "dequantize_stats")
+    return mean, var
+
+
+def select_quantized(q, k, dtype: str, block: int, scale: float, top_p: float, n_sink: int = 1,
+                     n_local: int = 1, k_min: int = 0):
+    """The selection of `select` on quantised statistics: stats -> quantize ->
+    dequantize -> scores -> cut."""
+    mean, var = block_stats(k, dtype, block)
+    qs = quantize_stats(mean, var)
+    dm, dv = dequantize_stats(qs)
+    Lq, T = q.shape[2], k.shape[2]
+    l = scores(q, dtype, dm, dv, T, block, scale)
+    idx, count = select_from_scores(l, Lq, T, block, top_p, n_sink, n_local, k_min)
+    return {"mean": mean, "var": var, "q": qs, "scores": l, "idx": idx, "count": count}
 
 
 def full_lists(B: int, Hq: int, Lq: int, T: int, block: int):

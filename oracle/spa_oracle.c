@@ -497,3 +497,77 @@ int oracle_rla_block_states(const void *k, const void *v, int is_bf16, int B, in
     }
     return ORACLE_OK;
 }
+
+/*
+ * Quantised block statistics ("SpotAttention", section 4: the selector's cache
+ * in INT4 microscale). Reading of the format: per (b, g, block j) and per group of
+ * 32 consecutive features c, one power-of-two scale 2^k and 4-bit codes,
+ *   mean: signed codes in [-7, 7],  k = the smallest k with max|mean| <= 7 * 2^k,
+ *   var : unsigned codes in [0, 15], k = the smallest k with max var <= 15 * 2^k,
+ *   code = round-half-even(x / 2^k),  dequantised value = code * 2^k,
+ * with k clamped to [-126, 126] (a group of zeros gets k = -126 and zero codes).
+ * The decision is taken on the statistics rounded to fp32 (the kernels' precision);
+ * with a power-of-two scale, x / 2^k and the rounding are then exact in any
+ * precision.
+ * mean, var: fp64 [B, Hkv, nb, d]; cm, cv: codes [B, Hkv, nb, d] (int8, uint8);
+ * km, kv: exponents [B, Hkv, nb, d / 32] (int8). d must be a multiple of 32.
+ */
+static int qexp(double amax, double top)
+{
+    if (!(amax > 0.0)) return -126;
+    int e;
+    (void)frexp(amax, &e);             /* amax = m 2^e, m in [0.5, 1) */
+    int k = e - 4;                     /* smallest k with amax <= top 2^k, top in {7, 15} */
+    while (amax > top * ldexp(1.0, k)) ++k;
+    while (k > -126 && amax <= top * ldexp(1.0, k - 1)) --k;
+    if (k < -126) k = -126;
+    if (k > 126) k = 126;
+    return k;
+}
+
+int oracle_quantize_stats(const double *mean, const double *var, int B, int Hkv, int nb, int d,
+                          int8_t *cm, uint8_t *cv, int8_t *km, int8_t *kv)
+{
+    if (B <= 0 || Hkv <= 0 || nb <= 0 || d <= 0 || d % 32) return ORACLE_EINVAL;
+    const int64_t groups = (int64_t)B * Hkv * nb * (d / 32);
+#pragma omp parallel for schedule(static)
+    for (int64_t gi = 0; gi < groups; ++gi) {
+        const size_t base = (size_t)gi * 32;
+        double am = 0.0, av = 0.0;
+        double xm[32], xv[32];
+        for (int c = 0; c < 32; ++c) {
+            xm[c] = (double)(float)mean[base + c];     /* the fp32 statistic */
+            xv[c] = (double)(float)var[base + c];
+            if (fabs(xm[c]) > am) am = fabs(xm[c]);
+            if (xv[c] > av) av = xv[c];
+        }
+        const int k1 = qexp(am, 7.0), k2 = qexp(av, 15.0);
+        km[gi] = (int8_t)k1;
+        kv[gi] = (int8_t)k2;
+        for (int c = 0; c < 32; ++c) {
+            double q1 = nearbyint(ldexp(xm[c], -k1));  /* default rounding: half to even */
+            double q2 = nearbyint(ldexp(xv[c], -k2));
+            if (q1 > 7) q1 = 7;
+            if (q1 < -7) q1 = -7;
+            if (q2 > 15) q2 = 15;
+            if (q2 < 0) q2 = 0;
+            cm[base + c] = (int8_t)q1;
+            cv[base + c] = (uint8_t)q2;
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* Dequantised statistics: code * 2^k, exact. Layouts as oracle_quantize_stats. */
+int oracle_dequantize_stats(const int8_t *cm, const uint8_t *cv, const int8_t *km,
+                            const int8_t *kv, int B, int Hkv, int nb, int d, double *mean,
+                            double *var)
+{
+    if (B <= 0 || Hkv <= 0 || nb <= 0 || d <= 0 || d % 32) return ORACLE_EINVAL;
+    const int64_t n = (int64_t)B * Hkv * nb * d;
+    for (int64_t x = 0; x < n; ++x) {
+        mean[x] = ldexp((double)cm[x], km[x / 32]);
+        var[x] = ldexp((double)cv[x], kv[x / 32]);
+    }
+    return ORACLE_OK;
+}

@@ -61,6 +61,15 @@ MUTATIONS = [
      [pins.test_rla_block_states_contract_to_residual_output]),
     ("rla_magnitude_without_abs", "m[c] += a * fabs(vu);", "m[c] += a * vu;",
      [pins.test_rla_hand_worked_examples]),
+    ("quant_round_half_away", "double q1 = nearbyint(ldexp(xm[c], -k1));",
+     "double q1 = round(ldexp(xm[c], -k1));",
+     [pins.test_quantized_stats_hand_worked_group]),
+    ("quant_scale_one_step_coarse", "const int k1 = qexp(am, 7.0), k2 = qexp(av, 15.0);",
+     "const int k1 = qexp(am, 7.0) + 1, k2 = qexp(av, 15.0);",
+     [pins.test_quantized_stats_hand_worked_group, pins.test_quantized_stats_error_and_scale_bounds,
+      pins.test_quantized_stats_on_the_grid_round_trip_exactly]),
+    ("quant_variance_signed_range", "qexp(av, 15.0)", "qexp(av, 7.0)",
+     [pins.test_quantized_stats_hand_worked_group, pins.test_quantized_stats_error_and_scale_bounds]),
     ("ascending_sort", "if (x->key > y->key) return -1;\n    if (x->key < y->key) return 1;",
      "if (x->key < y->key) return -1;\n    if (x->key > y->key) return 1;",
      [pins.test_top_p_hand_worked_examples, pins.test_top_p_tiny_p_keeps_top_one]),

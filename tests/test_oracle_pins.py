@@ -657,3 +657,90 @@ def test_rla_gqa_head_reads_its_group():
     assert np.abs(out[0, 0, 31] - out[0, 2, 31]).max() > 1e-3
     ref, _ = oracle.rla(q[:, 2:3], k[:, 1:2], v[:, 1:2], "f32", blk, idx[:, 2:3], cnt[:, 2:3])
     np.testing.assert_array_equal(out[0, 2], ref[0, 0])
+
+
+# ---------------------------------------------------------------- quantised statistics
+# SpotAttention, section 4: the selector's cache in INT4 microscale (format as read:
+# power-of-two scale per 32 features, round half to even).
+
+def test_quantized_stats_hand_worked_group():
+    g = _golden()["quantized_stats"]
+    mean = np.array(g["mean_group"], np.float64).reshape(1, 1, 1, 32)
+    var = np.array(g["var_group"], np.float64).reshape(1, 1, 1, 32)
+    qs = oracle.quantize_stats(mean, var)
+    assert int(qs["km"][0, 0, 0, 0]) == g["expected_km"]
+    assert int(qs["kv"][0, 0, 0, 0]) == g["expected_kv"]
+    assert qs["cm"].reshape(-1).tolist() == g["expected_cm"]
+    assert qs["cv"].reshape(-1).tolist() == g["expected_cv"]
+
+
+def _quant_inputs(seed):
+    rng = np.random.default_rng(seed)
+    mean = rng.standard_normal((2, 2, 5, 64)) * np.exp(rng.uniform(-6, 6, (2, 2, 5, 2)))[..., None].repeat(32, -1).reshape(2, 2, 5, 64)
+    var = rng.exponential(1.0, (2, 2, 5, 64)) * 10.0 ** rng.integers(-3, 3, (2, 2, 5, 1))
+    mean[0, 0, 1, :32] = 0.0                   # an all-zero group
+    var[1, 1, 2, 32:] = 0.0
+    return mean, var
+
+
+def test_quantized_stats_error_and_scale_bounds():
+    mean, var = _quant_inputs(70)
+    qs = oracle.quantize_stats(mean, var)
+    dm, dv = oracle.dequantize_stats(qs)
+    m32, v32 = mean.astype(np.float32).astype(np.float64), var.astype(np.float32).astype(np.float64)
+    step_m = np.ldexp(1.0, qs["km"].astype(np.int64)).repeat(32, axis=-1)
+    step_v = np.ldexp(1.0, qs["kv"].astype(np.int64)).repeat(32, axis=-1)
+    assert np.all(np.abs(dm - m32) <= step_m / 2) and np.all(np.abs(dv - v32) <= step_v / 2)
+    assert qs["cm"].min() >= -7 and qs["cm"].max() <= 7 and qs["cv"].max() <= 15
+    gm = np.abs(m32).reshape(2, 2, 5, 2, 32).max(-1)
+    gv = v32.reshape(2, 2, 5, 2, 32).max(-1)
+    km, kv = qs["km"].astype(np.int64), qs["kv"].astype(np.int64)
+    nz = gm > 0
+    # the scale is the smallest power of two that covers the group maximum
+    assert np.all(gm[nz] <= 7 * np.ldexp(1.0, km[nz])) and np.all(gm[nz] > 7 * np.ldexp(1.0, km[nz] - 1))
+    nzv = gv > 0
+    assert np.all(gv[nzv] <= 15 * np.ldexp(1.0, kv[nzv])) and np.all(gv[nzv] > 15 * np.ldexp(1.0, kv[nzv] - 1))
+    assert np.all(dm[0, 0, 1, :32] == 0) and np.all(dv[1, 1, 2, 32:] == 0)
+
+
+def test_quantized_stats_power_of_two_scaling_shifts_only_the_exponent():
+    mean, var = _quant_inputs(71)
+    q0 = oracle.quantize_stats(mean, var)
+    q1 = oracle.quantize_stats(mean * 2.0 ** 5, var * 2.0 ** -3)
+    assert np.array_equal(q0["cm"], q1["cm"]) and np.array_equal(q0["cv"], q1["cv"])
+    nzm = np.abs(mean).reshape(2, 2, 5, 2, 32).max(-1) > 0
+    nzv = var.reshape(2, 2, 5, 2, 32).max(-1) > 0
+    assert np.all(q1["km"][nzm].astype(int) == q0["km"][nzm].astype(int) + 5)
+    assert np.all(q1["kv"][nzv].astype(int) == q0["kv"][nzv].astype(int) - 3)
+
+
+def test_quantized_stats_on_the_grid_round_trip_exactly():
+    rng = np.random.default_rng(72)
+    codes_m = rng.integers(-7, 8, (1, 2, 3, 64))
+    codes_m[..., 0] = 7                         # every group reaches the top code
+    codes_m[..., 32] = -7
+    codes_v = rng.integers(0, 16, (1, 2, 3, 64))
+    codes_v[..., 0] = 15
+    codes_v[..., 32] = 15
+    mean = codes_m * 2.0 ** -4
+    var = codes_v * 2.0 ** 3
+    qs = oracle.quantize_stats(mean, var)
+    dm, dv = oracle.dequantize_stats(qs)
+    assert np.array_equal(dm, mean) and np.array_equal(dv, var)
+    assert np.all(qs["km"] == -4) and np.all(qs["kv"] == 3)
+
+
+def test_quantized_selection_equals_plain_selection_on_grid_statistics():
+    # keys constant within a block and on a coarse grid: mean exactly on the grid,
+    # variance 0, so quantisation changes nothing and neither does the selection
+    rng = np.random.default_rng(73)
+    B, Hq, Hkv, T, d, blk = 1, 4, 2, 256, 64, 32
+    vals = rng.integers(-7, 8, (B, Hkv, T // blk, d)).astype(np.float32) * np.float32(0.125)
+    vals[..., 0] = 7 * 0.125
+    vals[..., 32] = -7 * 0.125
+    k = np.repeat(vals, blk, axis=2)
+    q = _rand((B, Hq, T, d), 74)
+    a = oracle.select(q, k, "f32", blk, 0.125, 0.6)
+    b = oracle.select_quantized(q, k, "f32", blk, 0.125, 0.6)
+    assert np.array_equal(a["count"], b["count"]) and np.array_equal(a["idx"], b["idx"])
+    assert np.array_equal(a["scores"], b["scores"])
