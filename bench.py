@@ -240,6 +240,8 @@ def main():
                     help="override the decode workload's batch (smaller captures for profiling)")
     ap.add_argument("--no-rla", action="store_true",
                     help="skip the Residual Linear Attention leg")
+    ap.add_argument("--no-quant", action="store_true",
+                    help="skip the selection on quantised statistics in the decode leg")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-tokens", type=int, default=192)
@@ -510,12 +512,51 @@ def main():
                     "GB/s": (dbytes + dstate.numel() * 4) / (t_drla / 1e3) / 1e9,
                     "tokens/s": world * wd.B / ((t_dsel + t_drla) / 1e3)}
             del dstate, ws_r, orla
+        # selection on INT4 microscale statistics (SpotAttention, section 4)
+        dq = None
+        if not args.no_quant:
+            qrec = spa.spa_quantize_block_stats(dm, dv, wd.T, wd.block)
+            qi = torch.empty_like(didx)
+            qc = torch.empty_like(dcnt)
+            q_ms = []
+            for _ in range(4):
+                flush.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                spa.spa_quantize_block_stats(dm, dv, wd.T, wd.block, qstats=qrec)
+                e1.record(stream)
+                torch.cuda.synchronize()
+                q_ms.append(e0.elapsed_time(e1))
+            for _ in range(3):
+                spa.spa_select_quantized(qd_, qrec, wd.T, wd.block, wd.scale, wd.top_p, idx=qi,
+                                         count=qc)
+            torch.cuda.synchronize()
+            assert spa.spa_get_device_error() == 0
+            qs_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                      for _ in range(n_dec)]
+            barrier()
+            torch.cuda.synchronize()
+            for s in range(n_dec):
+                flush.zero_()
+                qs_evs[s][0].record(stream)
+                spa.spa_select_quantized(qd_, qrec, wd.T, wd.block, wd.scale, wd.top_p, idx=qi,
+                                         count=qc)
+                qs_evs[s][1].record(stream)
+            torch.cuda.synchronize()
+            barrier()
+            t_qsel = rank_max(statistics.mean(a_.elapsed_time(b_) for a_, b_ in qs_evs))
+            dq = {"stats_bytes_fp32": 2 * dm.numel() * 4, "stats_bytes_int4": qrec.numel(),
+                  "quantize_full_cache_ms": statistics.median(q_ms[1:]),
+                  "select_ms": t_qsel,
+                  "kept_fraction": float(qc.float().mean().item()) / wd.nb,
+                  "tokens/s": world * wd.B / ((t_qsel + t_dec) / 1e3)}
+            del qrec, qi, qc
         decode = {"workload": wd.name, "kept_kv_bytes": dbytes, "attn_ms": t_dec,
                   "select_ms": t_dsel, "GB/s": gbs, "peak_GB/s": peaks["hbm_gbs"],
                   "frac": gbs / peaks["hbm_gbs"], "peak_source": peak_src,
                   "tokens/s": world * wd.B / ((t_dsel + t_dec) / 1e3),
                   "kept_fraction": float(dcnt.float().mean().item()) / wd.nb,
-                  "block_stats_full_cache": stats_full, "rla": drla}
+                  "block_stats_full_cache": stats_full, "rla": drla, "quantized_stats": dq}
         del kc, vc
 
     # ---- CPU oracle baseline (rank 0, one GPU)

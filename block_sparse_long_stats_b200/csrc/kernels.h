@@ -17,7 +17,14 @@ cudaError_t launch_block_stats(const void *k, bool bf16, int B, int Hkv, int T, 
 cudaError_t launch_select(const void *q, bool bf16, const float *mean, const float *var, int B,
                           int Hq, int Hkv, int Lq, int T, int d, int block, float scale,
                           float top_p, int n_sink, int n_local, int k_min, int32_t *idx, int cap,
-                          int32_t *count, int *err, cudaStream_t s);
+                          int32_t *count, int *err, cudaStream_t s, const void *qstats = nullptr);
+
+// Quantised block statistics (INT4 microscale records of d + d/16 bytes per block;
+// format in qstats.cu). launch_select reads them instead of mean/var when qstats is set.
+size_t quantized_stats_bytes(int B, int Hkv, int T, int d, int block);
+cudaError_t launch_quantize_stats(const float *mean, const float *var, int B, int Hkv, int T, int d,
+                                  int block, int blk_begin, int blk_end, void *qstats,
+                                  cudaStream_t s);
 
 cudaError_t launch_prefill_f32(const float *q, const float *k, const float *v, int B, int Hq,
                                int Hkv, int L, int d, int block, const int32_t *idx, int cap,

@@ -1,0 +1,114 @@
+// Quantised block statistics: INT4 microscale ("SpotAttention", section 4: the
+// selector's cache quantised to INT4 / FP4 microscale, about 3.5x smaller than
+// bf16, without touching the backbone's KV cache).
+//
+// Format (one record of d + d/16 bytes per (b, kv-head, block)):
+//   [0, d/2)          mean codes, two per byte (feature 2c in the low nibble),
+//                     signed 4-bit in [-7, 7]
+//   [d/2, d)          variance codes, unsigned 4-bit in [0, 15]
+//   [d, d + d/32)     mean scale exponents k (int8), one per 32 features
+//   [d + d/32, ...)   variance scale exponents
+// A group's scale is 2^k with k the smallest integer such that the group's largest
+// |mean| <= 7 * 2^k (variance: largest var <= 15 * 2^k), clamped to [-126, 126];
+// code = round-half-even(x / 2^k). Dequantised: code * 2^k, exactly. The decision is
+// taken on the fp32 statistics; with a power-of-two scale the division and the
+// rounding are exact.
+//
+// HBM-bound and tiny: one warp per record reads 2 d fp32 values and writes
+// d + d/16 bytes.
+#include "kernels.h"
+
+namespace spa {
+namespace {
+
+__device__ __forceinline__ int group_exponent(float amax, float top) {
+    if (!(amax > 0.f)) return -126;
+    int e;
+    (void)frexpf(amax, &e);
+    int k = e - 4;
+    while (amax > top * ldexpf(1.f, k)) ++k;
+    while (k > -126 && amax <= top * ldexpf(1.f, k - 1)) --k;
+    return max(-126, min(126, k));
+}
+
+template <int D>
+__global__ void __launch_bounds__(256) quantize_stats_kernel(const float *__restrict__ mean,
+                                                             const float *__restrict__ var, int nb,
+                                                             int blk_begin, int nblk, int units,
+                                                             uint8_t *__restrict__ qs) {
+    constexpr int PL = D / 32;            // features per lane
+    constexpr int LPG = 32 / PL;          // lanes per 32-feature group
+    constexpr int RB = D + D / 16;        // record bytes
+    const int lane = threadIdx.x & 31;
+    const int u = blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (u >= units) return;               // warp-uniform
+    const int bg = u / nblk, j = blk_begin + u % nblk;
+    const size_t row = ((size_t)bg * nb + j) * D + lane * PL;
+    float m[PL], v[PL];
+    if constexpr (PL == 4) {
+        const float4 a = *reinterpret_cast<const float4 *>(mean + row);
+        const float4 b = *reinterpret_cast<const float4 *>(var + row);
+        m[0] = a.x; m[1] = a.y; m[2] = a.z; m[3] = a.w;
+        v[0] = b.x; v[1] = b.y; v[2] = b.z; v[3] = b.w;
+    } else {
+        const float2 a = *reinterpret_cast<const float2 *>(mean + row);
+        const float2 b = *reinterpret_cast<const float2 *>(var + row);
+        m[0] = a.x; m[1] = a.y;
+        v[0] = b.x; v[1] = b.y;
+    }
+    float am = 0.f, av = 0.f;
+#pragma unroll
+    for (int c = 0; c < PL; ++c) {
+        am = fmaxf(am, fabsf(m[c]));
+        av = fmaxf(av, v[c]);
+    }
+#pragma unroll
+    for (int o = LPG / 2; o > 0; o >>= 1) {
+        am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+        av = fmaxf(av, __shfl_xor_sync(0xffffffffu, av, o));
+    }
+    const int km = group_exponent(am, 7.f), kv = group_exponent(av, 15.f);
+    uint32_t pm = 0, pv = 0;
+#pragma unroll
+    for (int c = 0; c < PL; ++c) {
+        const int qm = max(-7, min(7, (int)rintf(ldexpf(m[c], -km))));
+        const int qv = max(0, min(15, (int)rintf(ldexpf(v[c], -kv))));
+        pm |= (uint32_t)(qm & 15) << (4 * c);
+        pv |= (uint32_t)qv << (4 * c);
+    }
+    uint8_t *rec = qs + ((size_t)bg * nb + j) * RB;
+    if constexpr (PL == 4) {
+        reinterpret_cast<uint16_t *>(rec)[lane] = (uint16_t)pm;
+        reinterpret_cast<uint16_t *>(rec + D / 2)[lane] = (uint16_t)pv;
+    } else {
+        rec[lane] = (uint8_t)pm;
+        rec[D / 2 + lane] = (uint8_t)pv;
+    }
+    if (lane % LPG == 0) {
+        rec[D + lane / LPG] = (uint8_t)(int8_t)km;
+        rec[D + D / 32 + lane / LPG] = (uint8_t)(int8_t)kv;
+    }
+}
+
+}  // namespace
+
+size_t quantized_stats_bytes(int B, int Hkv, int T, int d, int block) {
+    return (size_t)B * Hkv * ((T + block - 1) / block) * (d + d / 16);
+}
+
+cudaError_t launch_quantize_stats(const float *mean, const float *var, int B, int Hkv, int T, int d,
+                                  int block, int blk_begin, int blk_end, void *qstats,
+                                  cudaStream_t s) {
+    if (blk_end <= blk_begin) return cudaSuccess;
+    const int nb = (T + block - 1) / block, nblk = blk_end - blk_begin;
+    const int units = B * Hkv * nblk;
+    const unsigned grid = (unsigned)((units + 7) / 8);
+    uint8_t *q = reinterpret_cast<uint8_t *>(qstats);
+    if (d == 128)
+        quantize_stats_kernel<128><<<grid, 256, 0, s>>>(mean, var, nb, blk_begin, nblk, units, q);
+    else
+        quantize_stats_kernel<64><<<grid, 256, 0, s>>>(mean, var, nb, blk_begin, nblk, units, q);
+    return cudaGetLastError();
+}
+
+}  // namespace spa

@@ -109,6 +109,30 @@ __device__ __forceinline__ void load_stats(const float *mb, const float *vb, flo
     }
 }
 
+// The same PL components from a quantised record (INT4 codes, a power-of-two scale
+// per 32 features; layout in qstats.cu), dequantised exactly: code * 2^k.
+template <int D>
+__device__ __forceinline__ void load_stats_q(const uint8_t *rec, int lane, float (&mu)[D / 32],
+                                             float (&vr)[D / 32]) {
+    constexpr int PL = D / 32, LPG = 32 / PL;
+    uint32_t cm, cv;
+    if constexpr (PL == 4) {
+        cm = __ldg(reinterpret_cast<const unsigned short *>(rec) + lane);
+        cv = __ldg(reinterpret_cast<const unsigned short *>(rec + D / 2) + lane);
+    } else {
+        cm = __ldg(rec + lane);
+        cv = __ldg(rec + D / 2 + lane);
+    }
+    const int km = (int8_t)__ldg(rec + D + lane / LPG);
+    const int kv = (int8_t)__ldg(rec + D + D / 32 + lane / LPG);
+    const float sm = __int_as_float((km + 127) << 23), sv = __int_as_float((kv + 127) << 23);
+#pragma unroll
+    for (int c = 0; c < PL; ++c) {
+        mu[c] = (float)((int)(cm << (28 - 4 * c)) >> 28) * sm;   // sign-extended nibble
+        vr[c] = (float)((cv >> (4 * c)) & 15u) * sv;
+    }
+}
+
 __host__ __device__ constexpr int ilog2(int x) { return x <= 1 ? 0 : 1 + ilog2(x / 2); }
 
 // Reduces K values (K a power of two, 2 <= K <= 32) across the 32 lanes of a warp
@@ -153,9 +177,10 @@ struct SelectArgs {
     int *err;
     int sort_cap;   // power of two >= the largest residual of any unit
     bool prescored; // decode: the fp32 scores are already in the unit's row of idx
+    const uint8_t *qstats;  // quantised statistics (records of d + d/16 bytes) or null
 };
 
-template <typename T, int D>
+template <typename T, int D, bool QS>
 __global__ void __launch_bounds__(kThreads) select_kernel(SelectArgs a) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     uint64_t *keys = reinterpret_cast<uint64_t *>(smem_raw);               // [sort_cap]
@@ -234,12 +259,17 @@ __global__ void __launch_bounds__(kThreads) select_kernel(SelectArgs a) {
             q2[c] = qv[c] * qv[c];
         }
         const float hs2 = 0.5f * a.scale * a.scale;
-        const float *mb = a.mean + ((size_t)b * a.Hkv + g) * a.nb * D + lane * PL;
-        const float *vb = a.var + ((size_t)b * a.Hkv + g) * a.nb * D + lane * PL;
+        const size_t bgo = ((size_t)b * a.Hkv + g) * a.nb;
+        const float *mb = QS ? nullptr : a.mean + bgo * D + lane * PL;
+        const float *vb = QS ? nullptr : a.var + bgo * D + lane * PL;
+        const uint8_t *qb = QS ? a.qstats + bgo * (D + D / 16) : nullptr;
         for (int r = warp; r < nres; r += kWarps) {
             const int j = r_lo + r;
             float mu[PL], vr[PL], dot, quad;
-            load_stats<PL>(mb + (size_t)j * D, vb + (size_t)j * D, mu, vr);
+            if constexpr (QS)
+                load_stats_q<D>(qb + (size_t)j * (D + D / 16), lane, mu, vr);
+            else
+                load_stats<PL>(mb + (size_t)j * D, vb + (size_t)j * D, mu, vr);
             lane_partials<PL>(qv, q2, mu, vr, dot, quad);
             dot = warp_sum(dot);
             quad = warp_sum(quad);
@@ -337,10 +367,14 @@ __global__ void __launch_bounds__(kThreads) select_kernel(SelectArgs a) {
 // cap >= nb entries) until the cut kernel replaces it with the kept list.
 constexpr int kDecTile = 256;
 
-template <typename T, int D, int G>
+template <typename T, int D, int G, bool QS>
 __global__ void __launch_bounds__(kThreads) decode_score_kernel(SelectArgs a) {
     constexpr int PL = D / 32;
-    constexpr int U = 4;
+    // U candidates per warp step, so that the 2G partial sums of all of them fill
+    // one transposing reduction of up to 32 values: 16 (candidate, head) scores
+    // then come out on 16 lanes at once instead of G lanes per candidate.
+    constexpr int U = G >= 8 ? 2 : (G == 4 ? 4 : 8);
+    constexpr int NV = 2 * G * U;                   // values per reduction (<= 32)
     __shared__ float qs[G][D];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int bg = blockIdx.y, b = bg / a.Hkv, g = bg % a.Hkv;
@@ -362,68 +396,237 @@ __global__ void __launch_bounds__(kThreads) decode_score_kernel(SelectArgs a) {
             q2[hh][c] = qv[hh][c] * qv[hh][c];
         }
     const float hs2 = 0.5f * a.scale * a.scale;
-    const float *mb = a.mean + (size_t)bg * a.nb * D + lane * PL;
-    const float *vb = a.var + (size_t)bg * a.nb * D + lane * PL;
+    const float *mb = QS ? nullptr : a.mean + (size_t)bg * a.nb * D + lane * PL;
+    const float *vb = QS ? nullptr : a.var + (size_t)bg * a.nb * D + lane * PL;
+    const uint8_t *qb = QS ? a.qstats + (size_t)bg * a.nb * (D + D / 16) : nullptr;
     float *rows = reinterpret_cast<float *>(a.idx) + ((size_t)b * a.Hq + g * G) * a.cap;
     const int j0 = blockIdx.x * kDecTile;
+    constexpr int LB = 5 - ilog2(NV);               // lanes per value = 2^LB
+    const int vi = lane >> LB;                      // value this lane's group ends with
+    const int uu = vi / (2 * G), kk = vi % (2 * G); // its candidate, and dot (< G) or quad
     for (int r = warp * U; r < kDecTile; r += kWarps * U) {
         float mu[U][PL], vr[U][PL];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const int j = min(j0 + r + u, a.nb - 1);
-            load_stats<PL>(mb + (size_t)j * D, vb + (size_t)j * D, mu[u], vr[u]);
+            if constexpr (QS)
+                load_stats_q<D>(qb + (size_t)j * (D + D / 16), lane, mu[u], vr[u]);
+            else
+                load_stats<PL>(mb + (size_t)j * D, vb + (size_t)j * D, mu[u], vr[u]);
         }
+        // per-lane partials: value u*2G + h is the dot of head h with candidate u,
+        // value u*2G + G + h its variance term
+        float v[NV];
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int j = j0 + r + u;
-            // 2G per-lane partials: dot of head h at [h], quad of head h at [G + h].
-            float v[2 * G];
+        for (int u = 0; u < U; ++u)
 #pragma unroll
-            for (int hh = 0; hh < G; ++hh) lane_partials<PL>(qv[hh], q2[hh], mu[u], vr[u], v[hh], v[G + hh]);
-            // Transposing halving reduction: at each xor offset every lane keeps half
-            // of its values and adds its partner's copy of them, the same pairwise
-            // sums the per-value butterfly forms. Afterwards the lanes of group k
-            // (lane >> (5 - log2(2G))) hold the warp total of value k.
-            const float tot = reduce_transpose<2 * G>(v, lane);
-            constexpr int LB = 5 - ilog2(2 * G);            // lanes per value = 2^LB
-            const float quad = __shfl_sync(0xffffffffu, tot, (lane + (G << LB)) & 31);
-            const int hh = lane >> LB;                      // value index of this lane's group
-            if (hh < G && (lane & ((1 << LB) - 1)) == 0 && j < a.nb)
-                rows[(size_t)hh * a.cap + j] =
-                    log_score(tot, quad, a.scale, hs2, min(a.block, a.T - j * a.block));
-        }
+            for (int hh = 0; hh < G; ++hh)
+                lane_partials<PL>(qv[hh], q2[hh], mu[u], vr[u], v[u * 2 * G + hh],
+                                  v[u * 2 * G + G + hh]);
+        // Transposing halving reduction: at each xor offset every lane keeps half of
+        // its values and adds its partner's copy of them, the same pairwise sums the
+        // per-value butterfly forms.
+        const float tot = reduce_transpose<NV>(v, lane);
+        const float quad = __shfl_sync(0xffffffffu, tot, (lane + (G << LB)) & 31);
+        const int j = j0 + r + uu;
+        if (kk < G && (lane & ((1 << LB) - 1)) == 0 && j < a.nb)
+            rows[(size_t)kk * a.cap + j] =
+                log_score(tot, quad, a.scale, hs2, min(a.block, a.T - j * a.block));
     }
 }
 
-template <typename T, int D>
+template <typename T, int D, bool QS>
 cudaError_t launch_decode_scores(const SelectArgs &a, cudaStream_t s) {
     dim3 grid((unsigned)((a.nb + kDecTile - 1) / kDecTile), (unsigned)(a.B * a.Hkv));
     switch (a.G) {
-        case 1: decode_score_kernel<T, D, 1><<<grid, kThreads, 0, s>>>(a); break;
-        case 2: decode_score_kernel<T, D, 2><<<grid, kThreads, 0, s>>>(a); break;
-        case 4: decode_score_kernel<T, D, 4><<<grid, kThreads, 0, s>>>(a); break;
-        default: decode_score_kernel<T, D, 8><<<grid, kThreads, 0, s>>>(a); break;
+        case 1: decode_score_kernel<T, D, 1, QS><<<grid, kThreads, 0, s>>>(a); break;
+        case 2: decode_score_kernel<T, D, 2, QS><<<grid, kThreads, 0, s>>>(a); break;
+        case 4: decode_score_kernel<T, D, 4, QS><<<grid, kThreads, 0, s>>>(a); break;
+        default: decode_score_kernel<T, D, 8, QS><<<grid, kThreads, 0, s>>>(a); break;
     }
     return cudaGetLastError();
 }
 
-template <typename T, int D>
-cudaError_t launch_t(const SelectArgs &a, cudaStream_t s) {
+// The fp32 score a key's high word encodes.
+__device__ __forceinline__ float score_of(uint32_t o) { return key_score((uint64_t)o << 32); }
+
+// Block-wide sum, the same value in every thread; the warp partials go through a
+// double buffer indexed by the caller's step parity, so one barrier per call suffices.
+template <typename V>
+__device__ __forceinline__ V block_sum(V x, V (*buf)[kWarps], int &parity) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    if (lane == 0) buf[parity][warp] = x;
+    __syncthreads();
+    V t = V(0);
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) t += buf[parity][w];
+    parity ^= 1;
+    return t;
+}
+
+// Decode cut: the same rule as select_kernel's (residual blocks ranked by score
+// descending, index ascending; a block is kept while the mass ranked before it is
+// below top_p; then at least min(k_min, |residual|) blocks), found without sorting.
+// With keys kappa = (order_desc(score) << 32 | j) ascending in rank, the mass
+// ranked before a key, F(kappa), is monotone in kappa, so the kept blocks are
+// exactly the keys <= kappa*, the largest kappa with F(kappa) / total < top_p.
+// kappa* is found by bisection: 32 steps over the score word, then up to 14 over
+// the index; each step is one block-wide fp64 sum of the masses below the probe.
+// The K_min floor is the same bisection on counts. One CTA per (b, head); the
+// scores come from the unit's idx row (decode_score_kernel) and the row is then
+// overwritten with the ascending list.
+__global__ void __launch_bounds__(kThreads) decode_cut_kernel(SelectArgs a) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    const int tid = threadIdx.x;
+    const int unit = blockIdx.x;                     // (b, h); one query
+    const int jmax = a.nb - 1;
+    const int r_lo = min(a.n_sink, jmax + 1);
+    const int r_hi = max(r_lo, jmax - a.n_local + 1);
+    const int nres = r_hi - r_lo;
+    double *ms = reinterpret_cast<double *>(smem_raw);                 // [nb]
+    uint32_t *ord = reinterpret_cast<uint32_t *>(ms + a.nb);           // [nb]
+    unsigned char *flag = reinterpret_cast<unsigned char *>(ord + a.nb);   // [nb]
+    __shared__ double dbuf[2][kWarps];
+    __shared__ float fbuf[kWarps];
+    __shared__ int ibuf[2][kWarps];
+    __shared__ int itot[kWarps];
+    __shared__ int isum;
+    int dpar = 0, ipar = 0;
+
+    const float *row = reinterpret_cast<const float *>(a.idx + (size_t)unit * a.cap);
+    float lmax = -FLT_MAX;
+    for (int r = tid; r < nres; r += kThreads) {
+        const float sc = row[r_lo + r];
+        ord[r] = order_desc(sc);
+        lmax = fmaxf(lmax, sc);
+    }
+    for (int j = tid; j <= jmax; j += kThreads) flag[j] = (j < r_lo || j >= r_hi) ? 1 : 0;
+    // block maximum of the scores (every score is read before the row is rewritten)
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) lmax = fmaxf(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
+    if ((tid & 31) == 0) fbuf[tid >> 5] = lmax;
+    __syncthreads();
+    float mxf = -FLT_MAX;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) mxf = fmaxf(mxf, fbuf[w]);
+    const double mx = (double)mxf;
+    double local = 0.0;
+    for (int r = tid; r < nres; r += kThreads) {
+        const double m = exp((double)score_of(ord[r]) - mx);
+        ms[r] = m;
+        local += m;
+    }
+    const double total = block_sum<double>(local, dbuf, dpar);   // also publishes ms[]
+
+    // kept <=> (ord < s_star) or (ord == s_star and j <= j_star)
+    uint32_t s_star = 0xFFFFFFFFu;
+    int j_star = a.nb;
+    if (nres > 0 && a.top_p < 1.0f) {
+        const double p = (double)a.top_p;
+        auto mass_below = [&](uint32_t s, int jj) -> double {   // F((s << 32) | jj)
+            double acc = 0.0;
+            for (int r = tid; r < nres; r += kThreads) {
+                const uint32_t o = ord[r];
+                if (o < s || (o == s && r_lo + r < jj)) acc += ms[r];
+            }
+            return block_sum<double>(acc, dbuf, dpar);
+        };
+        uint32_t lo = 0, hi = 0xFFFFFFFFu;       // F(0) = 0 < p: the predicate holds at lo
+        while (lo < hi) {
+            const uint32_t mid = (uint32_t)(lo + ((uint64_t)hi - lo + 1) / 2);
+            if (mass_below(mid, 0) / total < p) lo = mid; else hi = mid - 1;
+        }
+        s_star = lo;
+        int jl = 0, jh = a.nb;
+        while (jl < jh) {
+            const int mid = jl + (jh - jl + 1) / 2;
+            if (mass_below(s_star, mid) / total < p) jl = mid; else jh = mid - 1;
+        }
+        j_star = jl;
+    }
+    auto kept_count = [&](uint32_t s, int jj) -> int {              // keys <= (s << 32) | jj
+        int c = 0;
+        for (int r = tid; r < nres; r += kThreads) {
+            const uint32_t o = ord[r];
+            c += (o < s || (o == s && r_lo + r <= jj)) ? 1 : 0;
+        }
+        return block_sum<int>(c, ibuf, ipar);
+    };
+    const int kfloor = min(a.k_min, nres);
+    if (kfloor > 0 && kept_count(s_star, j_star) < kfloor) {
+        // the kfloor smallest keys: the largest key with fewer than kfloor keys below it
+        auto below = [&](uint32_t s, int jj) -> int {               // keys < (s << 32) | jj
+            int c = 0;
+            for (int r = tid; r < nres; r += kThreads) {
+                const uint32_t o = ord[r];
+                c += (o < s || (o == s && r_lo + r < jj)) ? 1 : 0;
+            }
+            return block_sum<int>(c, ibuf, ipar);
+        };
+        uint32_t lo = 0, hi = 0xFFFFFFFFu;
+        while (lo < hi) {
+            const uint32_t mid = (uint32_t)(lo + ((uint64_t)hi - lo + 1) / 2);
+            if (below(mid, 0) < kfloor) lo = mid; else hi = mid - 1;
+        }
+        int jl = 0, jh = a.nb;
+        while (jl < jh) {
+            const int mid = jl + (jh - jl + 1) / 2;
+            if (below(lo, mid) < kfloor) jl = mid; else jh = mid - 1;
+        }
+        s_star = lo;
+        j_star = jl;
+    }
+    for (int r = tid; r < nres; r += kThreads) {
+        const uint32_t o = ord[r];
+        if (o < s_star || (o == s_star && r_lo + r <= j_star)) flag[r_lo + r] = 1;
+    }
+    __syncthreads();
+
+    // ascending list of the kept blocks
+    const int n = jmax + 1;
+    const int per = (n + kThreads - 1) / kThreads;
+    const int s0 = min(tid * per, n), s1 = min(s0 + per, n);
+    int c = 0;
+    for (int j = s0; j < s1; ++j) c += flag[j];
+    int pos = block_exclusive_scan<int>(c, itot, &isum);
+    int32_t *out = a.idx + (size_t)unit * a.cap;
+    for (int j = s0; j < s1; ++j)
+        if (flag[j]) out[pos++] = j;
+    if (tid == 0) a.count[unit] = isum;
+}
+
+template <typename T, int D, bool QS>
+cudaError_t launch_tq(const SelectArgs &a, cudaStream_t s) {
     const size_t smem = (size_t)a.sort_cap * 8 + (a.prescored ? 0 : kThreads * 8 * sizeof(float)) +
                         (size_t)a.nb + 16;
-    auto kern = select_kernel<T, D>;
+    auto kern = select_kernel<T, D, QS>;
     if (smem > 48 * 1024) {
         cudaError_t e =
             cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
     }
     if (a.prescored) {
-        cudaError_t e = launch_decode_scores<T, D>(a, s);
+        cudaError_t e = launch_decode_scores<T, D, QS>(a, s);
         if (e != cudaSuccess) return e;
+        const size_t csmem = (size_t)a.nb * 13 + 16;
+        if (csmem > 48 * 1024) {
+            e = cudaFuncSetAttribute(decode_cut_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)csmem);
+            if (e != cudaSuccess) return e;
+        }
+        decode_cut_kernel<<<(unsigned)(a.B * a.Hq), kThreads, csmem, s>>>(a);
+        return cudaGetLastError();
     }
     const unsigned grid = (unsigned)((size_t)a.B * a.Hq * a.nq);
     kern<<<grid, kThreads, smem, s>>>(a);
     return cudaGetLastError();
+}
+
+template <typename T, int D>
+cudaError_t launch_t(const SelectArgs &a, cudaStream_t s) {
+    return a.qstats ? launch_tq<T, D, true>(a, s) : launch_tq<T, D, false>(a, s);
 }
 
 }  // namespace
@@ -431,9 +634,10 @@ cudaError_t launch_t(const SelectArgs &a, cudaStream_t s) {
 cudaError_t launch_select(const void *q, bool bf16, const float *mean, const float *var, int B,
                           int Hq, int Hkv, int Lq, int T, int d, int block, float scale,
                           float top_p, int n_sink, int n_local, int k_min, int32_t *idx, int cap,
-                          int32_t *count, int *err, cudaStream_t s) {
+                          int32_t *count, int *err, cudaStream_t s, const void *qstats) {
     SelectArgs a;
     a.q = q; a.mean = mean; a.var = var;
+    a.qstats = reinterpret_cast<const uint8_t *>(qstats);
     a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.Lq = Lq; a.T = T; a.d = d; a.block = block;
     a.nb = (T + block - 1) / block;
     a.nq = (Lq + block - 1) / block;

@@ -131,6 +131,58 @@ SPA_API spa_status spa_select(const void *q, spa_dtype dt, const float *mean, co
     return e == cudaSuccess ? SPA_OK : cuda_fail(e, "select launch");
 }
 
+SPA_API size_t spa_quantized_stats_bytes(int B, int Hkv, int T, int d, int block) {
+    if (B <= 0 || Hkv <= 0 || T <= 0 || block <= 0 || (d != 64 && d != 128)) return 0;
+    return quantized_stats_bytes(B, Hkv, T, d, block);
+}
+
+SPA_API spa_status spa_quantize_block_stats(const float *mean, const float *var, int B, int Hkv,
+                                            int T, int d, int block, int blk_begin, int blk_end,
+                                            void *qstats, spa_stream stream) {
+    t_last_error.clear();
+    if (!mean || !var || !qstats) return fail(SPA_ERR_INVALID, "null pointer");
+    if (B <= 0 || Hkv <= 0 || T <= 0 || d <= 0 || block <= 0)
+        return fail(SPA_ERR_INVALID, "sizes must be positive");
+    const int nb = ceil_div(T, block);
+    if (blk_begin < 0 || blk_end > nb || blk_begin > blk_end)
+        return fail(SPA_ERR_INVALID, "need 0 <= blk_begin <= blk_end <= nb");
+    if (!aligned16(mean) || !aligned16(var) || !aligned16(qstats))
+        return fail(SPA_ERR_INVALID, "tensors must be 16-byte aligned");
+    if (d != 64 && d != 128) return fail(SPA_ERR_UNSUPPORTED, "d must be 64 or 128");
+    cudaError_t e = launch_quantize_stats(mean, var, B, Hkv, T, d, block, blk_begin, blk_end, qstats,
+                                          static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? SPA_OK : cuda_fail(e, "quantize launch");
+}
+
+SPA_API spa_status spa_select_quantized(const void *q, spa_dtype dt, const void *qstats, int B,
+                                        int Hq, int Hkv, int Lq, int T, int d, int block,
+                                        float scale, float top_p, int n_sink, int n_local,
+                                        int k_min, int32_t *idx, int cap, int32_t *count,
+                                        spa_stream stream) {
+    t_last_error.clear();
+    if (!q || !qstats || !idx || !count) return fail(SPA_ERR_INVALID, "null pointer");
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Lq <= 0 || T <= 0 || d <= 0 || block <= 0)
+        return fail(SPA_ERR_INVALID, "sizes must be positive");
+    if (Hq % Hkv) return fail(SPA_ERR_INVALID, "Hq must be a multiple of Hkv");
+    if (Lq != T && Lq != 1) return fail(SPA_ERR_INVALID, "Lq must equal T (prefill) or 1 (decode)");
+    if (dt != SPA_F32 && dt != SPA_BF16) return fail(SPA_ERR_INVALID, "unknown dtype");
+    if (!(scale > 0.f) || !(top_p > 0.f)) return fail(SPA_ERR_INVALID, "scale and top_p must be > 0");
+    if (n_sink < 0 || n_local < 0 || k_min < 0)
+        return fail(SPA_ERR_INVALID, "n_sink, n_local and k_min must be >= 0");
+    const int nb = ceil_div(T, block);
+    if (cap < nb) return fail(SPA_ERR_INVALID, "cap must be >= nb");
+    if (!aligned16(q) || !aligned16(qstats)) return fail(SPA_ERR_INVALID, "tensors must be 16-byte aligned");
+    if (d != 64 && d != 128) return fail(SPA_ERR_UNSUPPORTED, "d must be 64 or 128");
+    if (block < 1 || block > 1024) return fail(SPA_ERR_UNSUPPORTED, "block must be in [1, 1024]");
+    if (nb > 16384) return fail(SPA_ERR_UNSUPPORTED, "more than 16384 key blocks");
+    int *err = device_error_ptr();
+    if (!err) return fail(SPA_ERR_CUDA, "device error word unavailable");
+    cudaError_t e = launch_select(q, dt == SPA_BF16, nullptr, nullptr, B, Hq, Hkv, Lq, T, d, block,
+                                  scale, top_p, n_sink, n_local, k_min, idx, cap, count, err,
+                                  static_cast<cudaStream_t>(stream), qstats);
+    return e == cudaSuccess ? SPA_OK : cuda_fail(e, "select launch");
+}
+
 SPA_API spa_status spa_sparse_attn_prefill(const void *q, const void *k, const void *v,
                                            spa_dtype dt, int B, int Hq, int Hkv, int L, int d,
                                            int block, const int32_t *idx, int cap,

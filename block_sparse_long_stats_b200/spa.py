@@ -60,13 +60,19 @@ def lib() -> ctypes.CDLL:
         L.spa_rla_decode_workspace_bytes.restype = ctypes.c_size_t
         L.spa_sparse_attn_decode_rla.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P,
                                                  _I, _P, _F, _P, _P, _P, _P]
+        L.spa_quantized_stats_bytes.argtypes = [_I, _I, _I, _I, _I]
+        L.spa_quantized_stats_bytes.restype = ctypes.c_size_t
+        L.spa_quantize_block_stats.argtypes = [_P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P]
+        L.spa_select_quantized.argtypes = [_P, _I, _P, _I, _I, _I, _I, _I, _I, _I, _F, _F, _I, _I,
+                                           _I, _P, _I, _P, _P]
         L.spa_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_int)]
         L.spa_status_string.argtypes = [_I]
         L.spa_status_string.restype = ctypes.c_char_p
         L.spa_last_error.restype = ctypes.c_char_p
         for f in ("spa_block_stats", "spa_select", "spa_sparse_attn_prefill",
                   "spa_sparse_attn_decode", "spa_get_device_error", "spa_rla_block_states",
-                  "spa_rla_prefill", "spa_rla_decode_state", "spa_sparse_attn_decode_rla"):
+                  "spa_rla_prefill", "spa_rla_decode_state", "spa_sparse_attn_decode_rla",
+                  "spa_quantize_block_stats", "spa_select_quantized"):
             getattr(L, f).restype = _I
         _lib = L
     return _lib
@@ -147,6 +153,45 @@ def spa_select(q: torch.Tensor, mean: torch.Tensor, var: torch.Tensor, T: int, b
     _check("spa_select", lib().spa_select(_ptr(q), _dt(q), _ptr(mean), _ptr(var), B, Hq, Hkv, Lq, T,
                                           d, block, scale, top_p, n_sink, n_local, k_min,
                                           _ptr(idx), cap, _ptr(count), _stream(stream)))
+    return idx, count
+
+
+def spa_quantized_stats_bytes(B: int, Hkv: int, T: int, d: int, block: int) -> int:
+    return int(lib().spa_quantized_stats_bytes(B, Hkv, T, d, block))
+
+
+def spa_quantize_block_stats(mean: torch.Tensor, var: torch.Tensor, T: int, block: int,
+                             blk_begin: int = 0, blk_end: int | None = None,
+                             qstats: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """INT4 microscale records [B, Hkv, nb, d + d/16] uint8 from fp32 block statistics."""
+    B, Hkv, nb, d = mean.shape
+    if blk_end is None:
+        blk_end = nb
+    if qstats is None:
+        qstats = torch.empty((B, Hkv, nb, d + d // 16), device=mean.device, dtype=torch.uint8)
+    _check("spa_quantize_block_stats",
+           lib().spa_quantize_block_stats(_ptr(mean), _ptr(var), B, Hkv, T, d, block, blk_begin,
+                                          blk_end, _ptr(qstats), _stream(stream)))
+    return qstats
+
+
+def spa_select_quantized(q: torch.Tensor, qstats: torch.Tensor, T: int, block: int, scale: float,
+                         top_p: float, n_sink: int = 1, n_local: int = 1, k_min: int = 0,
+                         idx: torch.Tensor | None = None, count: torch.Tensor | None = None,
+                         stream=None):
+    """spa_select on quantised statistics. Returns (idx, count)."""
+    B, Hq, Lq, d = q.shape
+    Hkv = qstats.shape[1]
+    nb = -(-T // block)
+    nq = -(-Lq // block)
+    if idx is None:
+        idx = torch.empty((B, Hq, nq, nb), device=q.device, dtype=torch.int32)
+    if count is None:
+        count = torch.empty((B, Hq, nq), device=q.device, dtype=torch.int32)
+    _check("spa_select_quantized",
+           lib().spa_select_quantized(_ptr(q), _dt(q), _ptr(qstats), B, Hq, Hkv, Lq, T, d, block,
+                                      scale, top_p, n_sink, n_local, k_min, _ptr(idx),
+                                      idx.shape[-1], _ptr(count), _stream(stream)))
     return idx, count
 
 

@@ -106,6 +106,41 @@ spa_status spa_select(const void *q, spa_dtype dt, const float *mean, const floa
                       spa_stream stream);
 
 /*
+ * Quantised block statistics. Follows "SpotAttention", section 4: the selector's
+ * cache may be held in INT4 / FP4 microscale (about 3.5x smaller than bf16) without
+ * touching the backbone's KV cache. Here the selector's cache is the block
+ * statistics; the format read from that passage: per (b, g, block) one record of
+ * d + d/16 bytes,
+ *   [0, d/2)        mean codes, two per byte (feature 2c in the low nibble),
+ *                   signed 4-bit in [-7, 7]
+ *   [d/2, d)        variance codes, unsigned 4-bit in [0, 15]
+ *   [d, d + d/32)   mean scale exponents k, int8, one per 32 features
+ *   [d + d/32, d + d/16)  variance scale exponents
+ * where 2^k is the smallest power of two with max |mean| <= 7 * 2^k over the 32
+ * features (variance: max var <= 15 * 2^k), k clamped to [-126, 126], and
+ * code = round-half-even(x / 2^k); the value read back is code * 2^k, exactly.
+ * 136 bytes per block at d = 128, against 1024 in fp32.
+ *   mean, var : spa_block_stats output [B, Hkv, nb, d] fp32; d = 64 or 128
+ *   blk_begin, blk_end : records [blk_begin, blk_end) are written (others untouched)
+ *   qstats : [B, Hkv, nb] records, spa_quantized_stats_bytes(...) bytes, 16-byte aligned
+ *            (that call returns 0 for sizes it does not support)
+ */
+size_t spa_quantized_stats_bytes(int B, int Hkv, int T, int d, int block);
+spa_status spa_quantize_block_stats(const float *mean, const float *var, int B, int Hkv, int T,
+                                    int d, int block, int blk_begin, int blk_end, void *qstats,
+                                    spa_stream stream);
+
+/*
+ * spa_select on quantised statistics: the same score, cut and output, with each
+ * block's mean and variance read back from its record (code * 2^k) instead of
+ * from fp32 arrays. Arguments as spa_select, with qstats in place of mean, var.
+ */
+spa_status spa_select_quantized(const void *q, spa_dtype dt, const void *qstats, int B, int Hq,
+                                int Hkv, int Lq, int T, int d, int block, float scale,
+                                float top_p, int n_sink, int n_local, int k_min, int32_t *idx,
+                                int cap, int32_t *count, spa_stream stream);
+
+/*
  * Block-sparse causal prefill attention. Follows "S2O", sections 1 and 3 (index-
  * driven loading of the selected key/value tiles; online-softmax state m, l, acc):
  *   out[b,h,t,:] = sum_u softmax_u(s q_t.k_u) v_u over the keys u <= t whose block

@@ -85,3 +85,54 @@ def sample_rows(B, Hq, L, block, n, seed):
     while len(rows) < n:
         rows.add(int(rng.integers(0, B * Hq)) * L + int(rng.integers(0, L)))
     return np.array(sorted(rows), np.int64)
+
+
+# ------------------------------------------------------------------ quantised statistics records
+# Record layout of spa_quantize_block_stats (include/spa.h): d/2 bytes of mean codes
+# (two per byte, even feature in the low nibble, signed), d/2 bytes of variance
+# codes (unsigned), d/32 int8 mean exponents, d/32 int8 variance exponents.
+
+def pack_qstats(qs: dict) -> np.ndarray:
+    cm = qs["cm"].astype(np.int16) & 15
+    cv = qs["cv"].astype(np.int16) & 15
+    B, Hkv, nb, d = cm.shape
+    rec = np.empty((B, Hkv, nb, d + d // 16), np.uint8)
+    rec[..., :d // 2] = (cm[..., 0::2] | (cm[..., 1::2] << 4)).astype(np.uint8)
+    rec[..., d // 2:d] = (cv[..., 0::2] | (cv[..., 1::2] << 4)).astype(np.uint8)
+    rec[..., d:d + d // 32] = qs["km"].view(np.uint8)
+    rec[..., d + d // 32:] = qs["kv"].view(np.uint8)
+    return rec
+
+
+def unpack_qstats(rec: np.ndarray, d: int) -> dict:
+    rec = np.asarray(rec, np.uint8)
+    lo_m, hi_m = rec[..., :d // 2] & 15, rec[..., :d // 2] >> 4
+    lo_v, hi_v = rec[..., d // 2:d] & 15, rec[..., d // 2:d] >> 4
+    cm = np.empty(rec.shape[:-1] + (d,), np.int16)
+    cm[..., 0::2], cm[..., 1::2] = lo_m, hi_m
+    cm = np.where(cm >= 8, cm - 16, cm).astype(np.int8)
+    cv = np.empty(rec.shape[:-1] + (d,), np.uint8)
+    cv[..., 0::2], cv[..., 1::2] = lo_v, hi_v
+    return {"cm": cm, "cv": cv, "km": rec[..., d:d + d // 32].view(np.int8),
+            "kv": rec[..., d + d // 32:].view(np.int8)}
+
+
+def quant_ambiguous(mean: np.ndarray, var: np.ndarray, qs: dict, rel: float = 1e-5) -> np.ndarray:
+    """Per 32-feature group: True where the oracle's quantisation decision is a near
+    tie for fp32 statistics that differ in rounding order: a value within `rel` of a
+    rounding boundary (a half step), or the group maximum within `rel` of a scale
+    boundary. [B, Hkv, nb, d / 32], for mean or variance."""
+    out = []
+    for x, k, top in ((np.abs(mean.astype(np.float32).astype(np.float64)), qs["km"], 7.0),
+                      (var.astype(np.float32).astype(np.float64), qs["kv"], 15.0)):
+        B, Hkv, nb, d = x.shape
+        step = np.ldexp(1.0, k.astype(np.int64)).repeat(32, axis=-1)
+        t = x / step
+        frac = np.abs(t - np.floor(t) - 0.5)
+        near_code = (frac <= rel * np.maximum(1.0, t)).reshape(B, Hkv, nb, d // 32, 32).any(-1)
+        amax = x.reshape(B, Hkv, nb, d // 32, 32).max(-1)
+        kk = k.astype(np.int64)
+        near_scale = ((np.abs(amax / (top * np.ldexp(1.0, kk)) - 1) <= rel) |
+                      (np.abs(amax / (top * np.ldexp(1.0, kk - 1)) - 1) <= rel))
+        out.append(near_code | near_scale)
+    return out[0] | out[1]

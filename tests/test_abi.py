@@ -156,6 +156,25 @@ def test_rla_decode_host_checks(lib):
     assert h(0, 32, 8, 131072, 128, 16) == 0
 
 
+def test_quantized_stats_host_checks(lib):
+    I, F = ctypes.c_int, ctypes.c_float
+    n = lib.spa_quantized_stats_bytes
+    n.restype = ctypes.c_size_t
+    n.argtypes = [I] * 5
+    assert n(16, 8, 131072, 128, 16) == 16 * 8 * 8192 * 136
+    assert n(1, 1, 100, 96, 16) == 0                                     # d % 32
+    f = lib.spa_quantize_block_stats
+    f.argtypes = [P, P, I, I, I, I, I, I, I, P, P]
+    assert f(FAKE, FAKE, 1, 2, 256, 96, 16, 0, 16, FAKE, None) == 2       # d = 96
+    assert f(FAKE, FAKE, 1, 2, 256, 128, 16, 0, 17, FAKE, None) == 1      # beyond nb
+    assert f(FAKE, None, 1, 2, 256, 128, 16, 0, 16, FAKE, None) == 1
+    g = lib.spa_select_quantized
+    g.argtypes = [P, I, P, I, I, I, I, I, I, I, F, F, I, I, I, P, I, P, P]
+    assert g(FAKE, 1, FAKE, 1, 4, 2, 1, 256, 128, 16, 0.1, 0.9, 1, 1, 0, FAKE, 15, FAKE, None) == 1
+    assert g(FAKE, 1, FAKE, 1, 4, 2, 1, 256, 96, 16, 0.1, 0.9, 1, 1, 0, FAKE, 16, FAKE, None) == 2
+    assert g(FAKE, 1, None, 1, 4, 2, 1, 256, 128, 16, 0.1, 0.9, 1, 1, 0, FAKE, 16, FAKE, None) == 1
+
+
 def test_decode_workspace_size(lib):
     f = lib.spa_decode_workspace_bytes
     f.restype = ctypes.c_size_t
