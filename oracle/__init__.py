@@ -54,11 +54,13 @@ def _bind(path: str):
     lib.oracle_rla.argtypes = [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I,
                                _P, _I, _P, _P, _I64, _P, _P]
     lib.oracle_rla_block_states.argtypes = [_P, _P, _I, _I, _I, _I, _I, _I, _P]
+    lib.oracle_early_stop.argtypes = [_P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _I, _P, _D, _I,
+                                      _I, _D, _P, _P]
     lib.oracle_quantize_stats.argtypes = [_P, _P, _I, _I, _I, _I, _P, _P, _P, _P]
     lib.oracle_dequantize_stats.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _P, _P]
     for f in ("oracle_block_stats", "oracle_scores", "oracle_select_from_scores",
               "oracle_attention", "oracle_rla", "oracle_rla_block_states",
-              "oracle_quantize_stats", "oracle_dequantize_stats"):
+              "oracle_quantize_stats", "oracle_dequantize_stats", "oracle_early_stop"):
         getattr(lib, f).restype = _I
     return lib
 
@@ -272,6 +274,50 @@ def select_quantized(q, k, dtype: str, block: int, scale: float, top_p: float, n
     l = scores(q, dtype, dm, dv, T, block, scale)
     idx, count = select_from_scores(l, Lq, T, block, top_p, n_sink, n_local, k_min)
     return {"mean": mean, "var": var, "q": qs, "scores": l, "idx": idx, "count": count}
+
+
+def score_order(sel: dict, Lq: int, T: int, block: int, n_sink: int = 1, n_local: int = 1):
+    """The kept lists of `select` in traversal order (S2O, section 2): the local
+    blocks (the own block first, descending), the sink blocks (ascending), then the
+    kept residual blocks by descending fp32 score, equal scores by ascending index.
+    Returns (idx, count) with the same counts."""
+    idx, count, l = sel["idx"], sel["count"], sel["scores"]
+    out = np.full_like(idx, -1)
+    B, Hq, nq, cap = idx.shape
+    for b in range(B):
+        for h in range(Hq):
+            for i in range(nq):
+                c = int(count[b, h, i])
+                lst = [int(j) for j in idx[b, h, i, :c]]
+                last_row = min((i + 1) * block, Lq)
+                jmax = (T - Lq + last_row - 1) // block
+                local = sorted([j for j in lst if j > jmax - n_local], reverse=True)
+                sink = sorted([j for j in lst if j < n_sink and j <= jmax - n_local])
+                res = [j for j in lst if n_sink <= j <= jmax - n_local]
+                res.sort(key=lambda j: (-float(np.float32(l[b, h, i, j])), j))
+                order = local + sink + res
+                out[b, h, i, :c] = order
+    return out, count.copy()
+
+
+def early_stop(q, k, dtype: str, block: int, idx: np.ndarray, count: np.ndarray, scale: float,
+               tau: float, n_sink: int = 1, n_local: int = 1):
+    """S2O's monotone-gain early stop over score-ordered lists (prefill). Returns
+    (processed [B,Hq,nq] int32, ratios [B,Hq,nq,cap] fp64: R_n per position, -1 past
+    the stop)."""
+    q, isb = _inp(q, dtype)
+    k, _ = _inp(k, dtype)
+    B, Hq, Lq, d = q.shape
+    Hkv, T = k.shape[1], k.shape[2]
+    idx = np.ascontiguousarray(idx, np.int32)
+    count = np.ascontiguousarray(count, np.int32)
+    cap = idx.shape[-1]
+    processed = np.empty(count.shape, np.int32)
+    ratios = np.empty(idx.shape, np.float64)
+    _check(_load().oracle_early_stop(_ptr(q), _ptr(k), isb, B, Hq, Hkv, Lq, T, d, block, _ptr(idx),
+                                     cap, _ptr(count), float(scale), n_sink, n_local, float(tau),
+                                     _ptr(processed), _ptr(ratios)), "early_stop")
+    return processed, ratios
 
 
 def full_lists(B: int, Hq: int, Lq: int, T: int, block: int):

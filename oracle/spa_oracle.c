@@ -571,3 +571,113 @@ int oracle_dequantize_stats(const int8_t *cm, const uint8_t *cv, const int8_t *k
     }
     return ORACLE_OK;
 }
+
+/*
+ * Score-ordered traversal with a monotone-gain early stop ("S2O", section 2 and
+ * section 3's second pass). The lists are in traversal order (the local blocks and
+ * the sink first, then the kept residual blocks by descending score). For query
+ * block i of (b, h), with z_u = s q_t . k_u on the causal keys u <= t of a block,
+ *   gain_n(t) = sum_{u in block n, u <= t} exp(z_u),
+ *   acc_n(t)  = gain_1(t) + ... + gain_n(t),
+ *   R_n       = max over the rows t of the block (t < Lq) of gain_n(t) / acc_n(t)
+ *               (0 where acc_n(t) = 0).
+ * Reading: reserved entries (j < n_sink or j > i - n_local) are always processed;
+ * the traversal stops after the first ranked (residual) entry n with R_n < tau,
+ * which is processed. processed[b,h,i] = number of entries processed.
+ * ratios: [B, Hq, nq, cap] fp64, R_n per list position (or NULL); -1 beyond count.
+ * Ratios are invariant to a common shift of z, so each row shifts by its largest
+ * logit over the listed blocks.
+ */
+int oracle_early_stop(const void *q, const void *k, int is_bf16, int B, int Hq, int Hkv, int Lq,
+                      int T, int d, int block, const int32_t *idx, int cap, const int32_t *count,
+                      double scale, int n_sink, int n_local, double tau, int32_t *processed,
+                      double *ratios)
+{
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || T <= 0 || d <= 0 || block <= 0 || cap < 1)
+        return ORACLE_EINVAL;
+    if (Lq != T) return ORACLE_EINVAL;
+    const int nq = ceil_div(Lq, block), nb = ceil_div(T, block), G = Hq / Hkv;
+    const int64_t units = (int64_t)B * Hq * nq;
+    int err = 0;
+#pragma omp parallel
+    {
+        double *z = (double *)malloc(sizeof(double) * (size_t)block * T);
+        double *acc = (double *)malloc(sizeof(double) * block);
+        double *zmax = (double *)malloc(sizeof(double) * block);
+        if (!z || !acc || !zmax) {
+#pragma omp atomic write
+            err = ORACLE_ENOMEM;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t un = 0; un < units; ++un) {
+            if (!z || !acc || !zmax) continue;
+            const int64_t bh = un / nq;
+            const int i = (int)(un % nq);
+            const int b = (int)(bh / Hq), h = (int)(bh % Hq), g = h / G;
+            const int cnt = count[un];
+            const int32_t *lst = idx + un * cap;
+            double *rat = ratios ? ratios + un * cap : NULL;
+            if (cnt < 0 || cnt > cap) {
+#pragma omp atomic write
+                err = ORACLE_EINVAL;
+                continue;
+            }
+            const int t0 = i * block, nr = (t0 + block < Lq ? block : Lq - t0);
+            const size_t kvbase = ((size_t)b * Hkv + g) * T;
+            int bad = 0;
+            /* logits of every row of the block against every listed key */
+            for (int r = 0; r < nr; ++r) {
+                const int t = t0 + r;
+                zmax[r] = -INFINITY;
+                for (int n = 0; n < cnt; ++n) {
+                    const int j = lst[n];
+                    if (j < 0 || j >= nb || j > i) { bad = 1; break; }
+                    for (int u = j * block; u < (j + 1) * block && u < T; ++u) {
+                        double s = 0.0;
+                        if (u <= t)
+                            for (int c = 0; c < d; ++c)
+                                s += elem(q, is_bf16, ((size_t)bh * Lq + t) * d + c) *
+                                     elem(k, is_bf16, (kvbase + u) * d + c);
+                        const double zu = u <= t ? scale * s : -INFINITY;
+                        z[(size_t)r * T + u] = zu;
+                        if (zu > zmax[r]) zmax[r] = zu;
+                    }
+                }
+                acc[r] = 0.0;
+            }
+            if (bad) {
+#pragma omp atomic write
+                err = ORACLE_EINVAL;
+                continue;
+            }
+            int done = cnt;
+            for (int n = 0; n < cnt; ++n) {
+                const int j = lst[n];
+                double R = 0.0;
+                for (int r = 0; r < nr; ++r) {
+                    double gsum = 0.0;
+                    for (int u = j * block; u < (j + 1) * block && u < T; ++u) {
+                        const double zu = z[(size_t)r * T + u];
+                        if (zu != -INFINITY) gsum += exp(zu - zmax[r]);
+                    }
+                    acc[r] += gsum;
+                    const double ratio = acc[r] > 0.0 ? gsum / acc[r] : 0.0;
+                    if (ratio > R) R = ratio;
+                }
+                if (rat) rat[n] = R;
+                const int reserved = j < n_sink || j > i - n_local;
+                if (!reserved && R < tau) {
+                    done = n + 1;
+                    for (int x = n + 1; rat && x < cnt; ++x) rat[x] = -1.0;
+                    break;
+                }
+            }
+            processed[un] = done;
+            for (int x = cnt; rat && x < cap; ++x) rat[x] = -1.0;
+        }
+        free(z);
+        free(acc);
+        free(zmax);
+    }
+    return err;
+}

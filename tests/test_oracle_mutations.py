@@ -70,6 +70,15 @@ MUTATIONS = [
       pins.test_quantized_stats_on_the_grid_round_trip_exactly]),
     ("quant_variance_signed_range", "qexp(av, 15.0)", "qexp(av, 7.0)",
      [pins.test_quantized_stats_hand_worked_group, pins.test_quantized_stats_error_and_scale_bounds]),
+    ("early_stop_on_reserved_blocks", "if (!reserved && R < tau) {", "if (R < tau) {",
+     [pins.test_early_stop_limits_of_tau]),
+    ("early_stop_drops_the_stopping_block", "done = n + 1;", "done = n;",
+     [pins.test_early_stop_constant_keys_closed_form, pins.test_early_stop_limits_of_tau]),
+    ("early_stop_ratio_before_accumulating",
+     "acc[r] += gsum;\n                    const double ratio = acc[r] > 0.0 ? gsum / acc[r] : 0.0;",
+     "const double ratio = acc[r] > 0.0 ? gsum / acc[r] : 0.0;\n                    acc[r] += gsum;",
+     [pins.test_early_stop_ratio_is_gain_over_accumulated_mass,
+      pins.test_early_stop_constant_keys_closed_form]),
     ("ascending_sort", "if (x->key > y->key) return -1;\n    if (x->key < y->key) return 1;",
      "if (x->key < y->key) return -1;\n    if (x->key > y->key) return 1;",
      [pins.test_top_p_hand_worked_examples, pins.test_top_p_tiny_p_keeps_top_one]),

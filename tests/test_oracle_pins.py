@@ -744,3 +744,84 @@ def test_quantized_selection_equals_plain_selection_on_grid_statistics():
     b = oracle.select_quantized(q, k, "f32", blk, 0.125, 0.6)
     assert np.array_equal(a["count"], b["count"]) and np.array_equal(a["idx"], b["idx"])
     assert np.array_equal(a["scores"], b["scores"])
+
+
+# ---------------------------------------------------------------- score-ordered early stop
+# S2O, sections 2-3: blocks in descending estimated importance after the dense pass
+# over the own block; stop once a block's marginal gain in attention mass falls
+# below tau relative to the accumulated mass.
+
+def _ordered_full_lists(B, Hq, T, blk):
+    """Every causal block, in traversal order: own block, sink, then ascending."""
+    nb = -(-T // blk)
+    idx = np.full((B, Hq, nb, nb), -1, np.int32)
+    cnt = np.zeros((B, Hq, nb), np.int32)
+    for i in range(nb):
+        order = [i] + ([0] if i > 0 else []) + list(range(1, i))
+        idx[:, :, i, :len(order)] = order
+        cnt[:, :, i] = len(order)
+    return idx, cnt
+
+
+def test_early_stop_constant_keys_closed_form():
+    # k = 0: every logit is 0, so a block's gain for the row at offset r of query
+    # block i is its number of visible tokens: r + 1 for the own block, blk for the
+    # others. The tightest row is r = 0: after the own block, the sink and m more
+    # blocks, its ratio is blk / (1 + (m + 1) blk). With blk = 4 the ratios of the
+    # ranked blocks m = 1, 2, 3, ... are 4/9, 4/13, 4/17, 4/21: tau = 0.25 stops at
+    # the third ranked block (4/17 < 0.25 <= 4/13), after 5 list entries.
+    B, Hq, T, blk, d = 1, 2, 40, 4, 8
+    q = _rand((B, Hq, T, d), 80)
+    k = np.zeros((B, 1, T, d), np.float32)
+    idx, cnt = _ordered_full_lists(B, Hq, T, blk)
+    done, rat = oracle.early_stop(q, k, "f32", blk, idx, cnt, 0.125, 0.25)
+    for i in range(T // blk):
+        expect = 5 if i >= 5 else cnt[0, 0, i]
+        assert np.all(done[:, :, i] == expect), (i, done[:, :, i], expect)
+    np.testing.assert_allclose(rat[0, 0, 7, 2:5], [4 / 9, 4 / 13, 4 / 17], rtol=1e-14)
+    assert rat[0, 0, 7, 5] == -1.0
+
+
+def test_early_stop_limits_of_tau():
+    B, Hq, Hkv, T, blk, d = 1, 4, 2, 48, 8, 8
+    q, k = _rand((B, Hq, T, d), 81), _rand((B, Hkv, T, d), 82)
+    idx, cnt = _ordered_full_lists(B, Hq, T, blk)
+    done0, _ = oracle.early_stop(q, k, "f32", blk, idx, cnt, 0.3, 0.0)
+    assert np.array_equal(done0, cnt)                  # a ratio is never below 0
+    done1, _ = oracle.early_stop(q, k, "f32", blk, idx, cnt, 0.3, 1.5)
+    reserved = np.minimum(cnt, 2)                      # own block + sink
+    expect = np.where(cnt > reserved, reserved + 1, cnt)   # first ranked block: ratio <= 1
+    assert np.array_equal(done1, expect)
+
+
+def test_early_stop_ratio_is_gain_over_accumulated_mass():
+    # two-block unit written out: own block then one ranked block, one row each
+    B, Hq, T, blk, d = 1, 1, 4, 2, 1
+    q = np.array([[[[0.0], [0.0], [1.0], [1.0]]]], np.float32)
+    k = np.array([[[[0.0], [1.0], [2.0], [0.5]]]], np.float32)
+    idx = np.array([[[[0, -1], [1, 0]]]], np.int32)
+    cnt = np.array([[[1, 2]]], np.int32)
+    _, rat = oracle.early_stop(q, k, "f32", blk, idx, cnt, 1.0, 0.0, n_sink=0, n_local=1)
+    # query block 1, rows t = 2, 3 (q = 1): own block keys 2 (both rows) and 3 (row 3):
+    # row 2: own gain e^2, then block 0 gain e^0 + e^1; row 3: own e^2 + e^0.5, then 1 + e.
+    g_own = np.array([math.exp(2), math.exp(2) + math.exp(0.5)])
+    g0 = np.array([1 + math.e, 1 + math.e])
+    assert rat[0, 0, 1, 0] == pytest.approx(1.0)
+    assert rat[0, 0, 1, 1] == pytest.approx(np.max(g0 / (g_own + g0)), rel=1e-14)
+
+
+def test_score_order_lists_are_the_kept_sets_in_rank_order():
+    B, Hq, Hkv, T, d, blk = 1, 4, 2, 96, 16, 8
+    q, k = _rand((B, Hq, T, d), 83), _rand((B, Hkv, T, d), 84)
+    sel = oracle.select(q, k, "f32", blk, 0.25, 0.6)
+    oidx, ocnt = oracle.score_order(sel, T, T, blk)
+    assert np.array_equal(ocnt, sel["count"])
+    for (b, h, i), c in np.ndenumerate(ocnt):
+        lst = oidx[b, h, i, :c].tolist()
+        assert sorted(lst) == sel["idx"][b, h, i, :c].tolist()
+        assert lst[0] == i                               # the own block first
+        ranked = [j for j in lst if 1 <= j <= i - 1]
+        if i > 0:
+            assert lst[1] == 0                           # then the sink
+        s32 = [float(np.float32(sel["scores"][b, h, i, j])) for j in ranked]
+        assert all((s32[x], -ranked[x]) >= (s32[x + 1], -ranked[x + 1]) for x in range(len(s32) - 1))
