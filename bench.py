@@ -240,6 +240,8 @@ def main():
                     help="override the decode workload's batch (smaller captures for profiling)")
     ap.add_argument("--no-rla", action="store_true",
                     help="skip the Residual Linear Attention leg")
+    ap.add_argument("--tau", type=float, default=0.2,
+                    help="early-stop threshold for the score-ordered traversal leg (0: skip)")
     ap.add_argument("--no-quant", action="store_true",
                     help="skip the selection on quantised statistics in the decode leg")
     ap.add_argument("--no-cpu", action="store_true")
@@ -416,6 +418,57 @@ def main():
                                                       ms_per_step + t_st + t_rla)}
         del states, rout
 
+    # ---- score-ordered traversal with early stop (S2O, sections 2-3), block 128
+    early = None
+    if args.tau > 0 and w.block == 128 and w.dtype == "bf16":
+        oidx = torch.empty_like(idx)
+        ocnt = torch.empty_like(cnt)
+        proc = torch.empty_like(cnt)
+        eout = torch.empty_like(q)
+
+        def early_step():
+            spa.spa_select_score_order(q, mean, var, w.block, w.scale, w.top_p, w.n_sink,
+                                       w.n_local, w.k_min, idx=oidx, count=ocnt)
+            spa.spa_sparse_attn_prefill_early_stop(q, k, v, w.block, oidx, ocnt, w.scale, args.tau,
+                                                   w.n_sink, w.n_local, out=eout,
+                                                   processed=proc)
+        for _ in range(3):
+            early_step()
+        torch.cuda.synchronize()
+        assert spa.spa_get_device_error() == 0
+        n_es = max(5, args.steps // 4)
+        es_evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_es)]
+        barrier()
+        torch.cuda.synchronize()
+        for s_ in range(n_es):
+            flush.zero_()
+            es_evs[s_][0].record(stream)
+            spa.spa_select_score_order(q, mean, var, w.block, w.scale, w.top_p, w.n_sink,
+                                       w.n_local, w.k_min, idx=oidx, count=ocnt)
+            es_evs[s_][1].record(stream)
+            spa.spa_sparse_attn_prefill_early_stop(q, k, v, w.block, oidx, ocnt, w.scale, args.tau,
+                                                   w.n_sink, w.n_local, out=eout,
+                                                   processed=proc)
+            es_evs[s_][2].record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        t_osel = rank_max(statistics.mean(e[0].elapsed_time(e[1]) for e in es_evs))
+        t_es = rank_max(statistics.mean(e[1].elapsed_time(e[2]) for e in es_evs))
+        pr = proc.cpu().numpy()
+        oi = oidx.cpu().numpy()
+        trunc = np.where(np.arange(oi.shape[-1]) < pr[..., None], oi, -1)
+        F_es = kept_flops(pr, np.sort(np.where(trunc < 0, 1 << 30, trunc), axis=-1), L, w.block, d)
+        dev_ = (eout.float() - out.float())
+        early = {"tau": args.tau, "processed_fraction": float(pr.sum()) / float(count_h.sum()),
+                 "vs_kept_attention": {"max_abs": float(dev_.abs().max().item()),
+                                       "rms": float(dev_.pow(2).mean().sqrt().item()),
+                                       "output_rms": float(out.float().pow(2).mean().sqrt().item())},
+                 "select_score_order_ms": t_osel, "attn_ms": t_es,
+                 "processed_flops": F_es, "TFLOP/s": F_es / (t_es / 1e3) / 1e12,
+                 "tokens/s": job_throughput(B * L, world, 1,
+                                            statistics.mean(t_stats) + t_osel + t_es)}
+        del oidx, ocnt, proc, eout
+
     # ---- decode leg
     decode = None
     if not args.no_decode:
@@ -588,6 +641,7 @@ def main():
                          "algorithmic_bytes": float(2 * q.numel() * 2 + 2 * k.numel() * 2)},
             "kernels": per_kernel,
             "rla": rla,
+            "early_stop": early,
             "decode": decode,
             "e2e": e2e,
             "cpu_baseline": cpu,

@@ -17,7 +17,8 @@ cudaError_t launch_block_stats(const void *k, bool bf16, int B, int Hkv, int T, 
 cudaError_t launch_select(const void *q, bool bf16, const float *mean, const float *var, int B,
                           int Hq, int Hkv, int Lq, int T, int d, int block, float scale,
                           float top_p, int n_sink, int n_local, int k_min, int32_t *idx, int cap,
-                          int32_t *count, int *err, cudaStream_t s, const void *qstats = nullptr);
+                          int32_t *count, int *err, cudaStream_t s, const void *qstats = nullptr,
+                          bool score_order = false);
 
 // Quantised block statistics (INT4 microscale records of d + d/16 bytes per block;
 // format in qstats.cu). launch_select reads them instead of mean/var when qstats is set.
@@ -46,6 +47,14 @@ cudaError_t launch_rla_block_states(const void *k, const void *v, int B, int Hkv
 cudaError_t launch_rla_prefill(const void *q, const void *k, const void *v, const void *states,
                                int B, int Hq, int Hkv, int L, int block, const int32_t *idx, int cap,
                                const int32_t *count, float *out, int *err, cudaStream_t s);
+
+// Score-ordered lists (traversal order) with S2O's early stop; bf16, d = 128,
+// block 128; processed [B, Hq, nq] receives the number of list entries used.
+cudaError_t launch_prefill_tc_early_stop(const void *q, const void *k, const void *v, int B, int Hq,
+                                         int Hkv, int L, const int32_t *idx, int cap,
+                                         const int32_t *count, float scale, int n_sink,
+                                         int n_local, float tau, void *out, float *lse,
+                                         int32_t *processed, int *err, cudaStream_t s);
 
 int decode_splits(int B, int Hkv, int T, int block);
 size_t decode_workspace_bytes(int B, int Hq, int Hkv, int T, int d, int block);

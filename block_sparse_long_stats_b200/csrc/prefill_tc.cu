@@ -45,6 +45,11 @@ struct PrefillArgs {
     int B, Hq, Hkv, L, G, nq, cap, npairs;
     float scale_log2;
     int *err;
+    // score-ordered traversal with early stop (block 128 only)
+    int n_sink, n_local;
+    float tau;
+    int32_t *processed;   // [B, Hq, nq]: list entries processed
+    int nwords;           // words of the duplicate bitmap
 };
 
 // Walks the ascending kept lists of the HPT heads of a tile in merged order. All
@@ -126,10 +131,19 @@ struct Cfg {
     static constexpr uint32_t IDESC_O = idesc_bf16(128, kD, true);
 };
 
-template <int BLK>
+// ES: score-ordered traversal with S2O's monotone-gain early stop (sections 2-3).
+// The unit's list (in traversal order) is validated into shared memory first:
+// entries outside [0, i] and repeats are dropped (and reported). After each ranked
+// block the softmax warps take, over the tile's rows, the largest ratio of the
+// block's mass to the accumulated mass (both in the running normalisation); below
+// tau, the tile stops after that block. The MMA thread learns it at p_ready and
+// issues that block's P V as the last product; the producer learns it from
+// decided[] before loading the next V, and waits for the K copy it already started.
+template <int BLK, bool ES>
 __global__ void __launch_bounds__(kThreads, 2)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                        const __grid_constant__ CUtensorMap tv, PrefillArgs a) {
+    static_assert(!ES || BLK == 128, "early stop walks one head's list");
     using C = Cfg<BLK>;
     constexpr int HPT = C::HPT;
     constexpr int ST = C::STAGES;
@@ -139,6 +153,11 @@ __global__ void __launch_bounds__(kThreads, 2)
     __shared__ uint64_t bar_q, full_k[ST], full_v[ST], empty_k[ST], empty_v[ST], s_full, p_ready,
         o_done;
     __shared__ uint32_t tmem_slot;
+    __shared__ uint64_t decided[2];
+    __shared__ int n_list, stop_at;
+    __shared__ float es_max[2][4];
+    int32_t *list_s = reinterpret_cast<int32_t *>(smem + C::SMEM);          // ES: [nq]
+    uint32_t *bits = reinterpret_cast<uint32_t *>(list_s + (ES ? a.nq : 0)); // ES: [nwords]
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int per_i = a.B * a.Hkv * a.npairs;
@@ -160,15 +179,64 @@ __global__ void __launch_bounds__(kThreads, 2)
         mbar_init(&s_full, 1);
         mbar_init(&p_ready, 128);
         mbar_init(&o_done, 1);
+        mbar_init(&decided[0], 1);
+        mbar_init(&decided[1], 1);
+        stop_at = 0x7fffffff;
         fence_mbar_init();
     }
     if (warp == 5) tmem_alloc(&tmem_slot, 256);
+    if constexpr (ES) {
+        if (warp == 0) {
+            for (int w = lane; w < a.nwords; w += 32) bits[w] = 0u;
+            __syncwarp();
+            const size_t unit = ((size_t)b * a.Hq + h0) * a.nq + i;
+            int c = __ldg(a.count + unit);
+            bool bad = false;
+            if (c < 0 || c > a.cap) {
+                if (lane == 0) set_error(a.err, SPA_DEVERR_BAD_COUNT);
+                c = c < 0 ? 0 : a.cap;
+            }
+            const int32_t *lst = a.idx + unit * a.cap;
+            int nl = 0;
+            for (int base = 0; base < c; base += 32) {
+                const int e = base + lane;
+                const int x = e < c ? __ldg(lst + e) : -1;
+                bool ok = e < c && x >= 0 && x <= i;
+                // the first occurrence wins: lowest lane within the chunk, and not
+                // seen in an earlier chunk
+                const unsigned peers = __match_any_sync(0xffffffffu, ok ? x : -1 - lane);
+                ok = ok && (__ffs(peers) - 1 == lane);
+                if (ok) ok = !((bits[x >> 5] >> (x & 31)) & 1u);
+                __syncwarp();
+                if (ok) atomicOr(&bits[x >> 5], 1u << (x & 31));
+                if (e < c && !ok) bad = true;
+                const unsigned bal = __ballot_sync(0xffffffffu, ok);
+                if (ok) list_s[nl + __popc(bal & ((1u << lane) - 1u))] = x;
+                nl += __popc(bal);
+                __syncwarp();
+            }
+            if (bad) set_error(a.err, SPA_DEVERR_BAD_INDEX);
+            if (lane == 0) n_list = nl;
+        }
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tmem_slot;
 
     Cursor<HPT> cur;
+    int lpos = 0;
+    // the next block of the walk: the validated list (ES) or the merged ascending lists
+    auto next = [&](int &j, uint32_t &mask, bool report) -> bool {
+        if constexpr (ES) {
+            if (lpos >= n_list) return false;
+            j = list_s[lpos++];
+            mask = 1u;
+            return true;
+        } else {
+            return cur.next(j, mask, a.err, report);
+        }
+    };
     if (warp == 4) {
         if (lane == 0) {
             prefetch_tmap(&tq);
@@ -185,7 +253,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             const int kv_row0 = (b * a.Hkv + g) * a.L;
             int j;
             uint32_t mask;
-            for (int n = 0; cur.next(j, mask, a.err, true); ++n) {
+            for (int n = 0; next(j, mask, true); ++n) {
                 const int s = n % ST;
                 const uint32_t ph = (n / ST) & 1;
                 unsigned char *kt = smem + C::OFF_K + s * C::KV_BYTES;
@@ -194,6 +262,15 @@ __global__ void __launch_bounds__(kThreads, 2)
                 mbar_arrive_expect_tx(&full_k[s], C::KV_BYTES);
                 tma_load_2d(kt, &tk, &full_k[s], 0, kv_row0 + j * BLK);
                 tma_load_2d(kt + C::KV_HALF, &tk, &full_k[s], 64, kv_row0 + j * BLK);
+                if constexpr (ES) {
+                    if (n > 0) {
+                        if (!mbar_wait(&decided[(n - 1) & 1], ((n - 1) >> 1) & 1, a.err)) break;
+                        if (*reinterpret_cast<volatile int *>(&stop_at) <= n - 1) {
+                            mbar_wait(&full_k[s], ph, a.err);   // the copy already started
+                            break;
+                        }
+                    }
+                }
                 if (!mbar_wait(&empty_v[s], ph ^ 1, a.err)) break;
                 mbar_arrive_expect_tx(&full_v[s], C::KV_BYTES);
                 tma_load_2d(vt, &tv, &full_v[s], 0, kv_row0 + j * BLK);
@@ -222,8 +299,13 @@ __global__ void __launch_bounds__(kThreads, 2)
                 tc_commit(&empty_v[s]);
                 return true;
             };
-            while (ok && cur.next(j, mask, a.err, false)) {
+            bool stopped = false;
+            while (ok && next(j, mask, false)) {
                 if (n > 0 && !issue_pv(n - 1)) { ok = false; break; }
+                if (ES && *reinterpret_cast<volatile int *>(&stop_at) <= n - 1) {
+                    stopped = true;   // P(n - 1) V was the last product
+                    break;
+                }
                 const int s = n % ST;
                 if (!mbar_wait(&full_k[s], (n / ST) & 1, a.err)) break;
                 tc_fence_after();
@@ -238,7 +320,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 tc_commit(&empty_k[s]);
                 ++n;
             }
-            if (ok && n > 0 && issue_pv(n - 1)) tc_commit(&o_done);
+            if (ok && n > 0 && (stopped || issue_pv(n - 1))) tc_commit(&o_done);
         }
     } else {
         const int r = tid;
@@ -252,7 +334,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         int n = 0, j;
         uint32_t mask;
         bool ok = true;
-        while (cur.next(j, mask, a.err, false)) {
+        while (next(j, mask, false)) {
             if (!mbar_wait(&s_full, n & 1, a.err)) { ok = false; break; }
             tc_fence_after();
             float x[BLK];
@@ -323,11 +405,29 @@ __global__ void __launch_bounds__(kThreads, 2)
             f32x2_split(add_f32x2(add_f32x2(sp[0], sp[1]), add_f32x2(sp[2], sp[3])), rs0, rs1);
             const float rs = rs0 + rs1;
             l = l * alpha + rs;
+            bool stop = false;
+            if constexpr (ES) {
+                // largest ratio of this block's mass to the accumulated mass over the
+                // tile's rows; reserved blocks (sink, local) never stop the walk
+                float ratio = (t < a.L && l > 0.f) ? rs / l : 0.f;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) ratio = fmaxf(ratio, __shfl_xor_sync(0xffffffffu, ratio, o));
+                if (lane == 0) es_max[n & 1][warp] = ratio;
+                named_bar_sync(1, 128);
+                const float rmax = fmaxf(fmaxf(es_max[n & 1][0], es_max[n & 1][1]),
+                                         fmaxf(es_max[n & 1][2], es_max[n & 1][3]));
+                const bool ranked = !(j < a.n_sink || j > i - a.n_local);
+                stop = ranked && rmax < a.tau;
+                if (tid == 0 && stop) stop_at = n;
+            }
             tc_wait_st();
             tc_fence_before();
             mbar_arrive(&p_ready);
+            if (ES && tid == 0) mbar_arrive(&decided[n & 1]);
             ++n;
+            if (stop) break;
         }
+        if (ES && tid == 0) a.processed[((size_t)b * a.Hq + h0) * a.nq + i] = n;
         if (ok && n > 0) ok = mbar_wait(&o_done, 0, a.err);
         tc_fence_after();
         const bool store = t < a.L;
@@ -378,7 +478,7 @@ bool make_map(CUtensorMap *map, const void *base, uint64_t rows, int box_rows) {
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BLK>
+template <int BLK, bool ES>
 cudaError_t launch_blk(const void *q, const void *k, const void *v, const PrefillArgs &a,
                        cudaStream_t s) {
     using C = Cfg<BLK>;
@@ -387,8 +487,8 @@ cudaError_t launch_blk(const void *q, const void *k, const void *v, const Prefil
         !make_map(&mk, k, (uint64_t)a.B * a.Hkv * a.L, BLK) ||
         !make_map(&mv, v, (uint64_t)a.B * a.Hkv * a.L, BLK))
         return cudaErrorNotSupported;
-    const size_t smem = C::SMEM + 1024;
-    auto kern = prefill_tc_kernel<BLK>;
+    const size_t smem = C::SMEM + 1024 + (ES ? (size_t)a.nq * 4 + (size_t)a.nwords * 4 : 0);
+    auto kern = prefill_tc_kernel<BLK, ES>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)((size_t)a.nq * a.B * a.Hkv * a.npairs);
@@ -414,7 +514,37 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, int B
     a.npairs = a.G / (128 / block);
     a.scale_log2 = scale * kLog2e;
     a.err = err;
-    return block == 64 ? launch_blk<64>(q, k, v, a, s) : launch_blk<128>(q, k, v, a, s);
+    a.n_sink = 0;
+    a.n_local = 0;
+    a.tau = 0.f;
+    a.processed = nullptr;
+    a.nwords = 0;
+    return block == 64 ? launch_blk<64, false>(q, k, v, a, s) : launch_blk<128, false>(q, k, v, a, s);
+}
+
+cudaError_t launch_prefill_tc_early_stop(const void *q, const void *k, const void *v, int B, int Hq,
+                                         int Hkv, int L, const int32_t *idx, int cap,
+                                         const int32_t *count, float scale, int n_sink,
+                                         int n_local, float tau, void *out, float *lse,
+                                         int32_t *processed, int *err, cudaStream_t s) {
+    PrefillArgs a;
+    a.idx = idx;
+    a.count = count;
+    a.out = reinterpret_cast<__nv_bfloat16 *>(out);
+    a.lse = lse;
+    a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.L = L;
+    a.G = Hq / Hkv;
+    a.nq = (L + 127) / 128;
+    a.cap = cap;
+    a.npairs = a.G;
+    a.scale_log2 = scale * kLog2e;
+    a.err = err;
+    a.n_sink = n_sink;
+    a.n_local = n_local;
+    a.tau = tau;
+    a.processed = processed;
+    a.nwords = (a.nq + 31) / 32;
+    return launch_blk<128, true>(q, k, v, a, s);
 }
 
 }  // namespace spa

@@ -178,6 +178,7 @@ struct SelectArgs {
     int sort_cap;   // power of two >= the largest residual of any unit
     bool prescored; // decode: the fp32 scores are already in the unit's row of idx
     const uint8_t *qstats;  // quantised statistics (records of d + d/16 bytes) or null
+    bool score_order;       // prefill: lists in traversal order instead of ascending
 };
 
 template <typename T, int D, bool QS>
@@ -341,6 +342,17 @@ __global__ void __launch_bounds__(kThreads) select_kernel(SelectArgs a) {
         nk = isum;
     }
     nk = max(nk, min(a.k_min, nres));
+    if (a.score_order) {
+        // traversal order: the local blocks (own block first), the sink blocks, then
+        // the kept residual blocks in rank order (the sorted keys)
+        int32_t *out = a.idx + unit * a.cap;
+        const int nloc = jmax + 1 - r_hi;
+        for (int x = tid; x < nloc; x += kThreads) out[x] = jmax - x;
+        for (int x = tid; x < r_lo; x += kThreads) out[nloc + x] = x;
+        for (int x = tid; x < nk; x += kThreads) out[nloc + r_lo + x] = (int)(uint32_t)keys[x];
+        if (tid == 0) a.count[unit] = nloc + r_lo + nk;
+        return;
+    }
     for (int x = tid; x < nk; x += kThreads) flag[(int)(uint32_t)keys[x]] = 1;
     __syncthreads();
 
@@ -634,8 +646,10 @@ cudaError_t launch_t(const SelectArgs &a, cudaStream_t s) {
 cudaError_t launch_select(const void *q, bool bf16, const float *mean, const float *var, int B,
                           int Hq, int Hkv, int Lq, int T, int d, int block, float scale,
                           float top_p, int n_sink, int n_local, int k_min, int32_t *idx, int cap,
-                          int32_t *count, int *err, cudaStream_t s, const void *qstats) {
+                          int32_t *count, int *err, cudaStream_t s, const void *qstats,
+                          bool score_order) {
     SelectArgs a;
+    a.score_order = score_order;
     a.q = q; a.mean = mean; a.var = var;
     a.qstats = reinterpret_cast<const uint8_t *>(qstats);
     a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.Lq = Lq; a.T = T; a.d = d; a.block = block;

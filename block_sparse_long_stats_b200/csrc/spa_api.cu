@@ -131,6 +131,63 @@ SPA_API spa_status spa_select(const void *q, spa_dtype dt, const float *mean, co
     return e == cudaSuccess ? SPA_OK : cuda_fail(e, "select launch");
 }
 
+SPA_API spa_status spa_select_score_order(const void *q, spa_dtype dt, const float *mean,
+                                          const float *var, int B, int Hq, int Hkv, int L, int d,
+                                          int block, float scale, float top_p, int n_sink,
+                                          int n_local, int k_min, int32_t *idx, int cap,
+                                          int32_t *count, spa_stream stream) {
+    t_last_error.clear();
+    if (!q || !mean || !var || !idx || !count) return fail(SPA_ERR_INVALID, "null pointer");
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || L <= 0 || d <= 0 || block <= 0)
+        return fail(SPA_ERR_INVALID, "sizes must be positive");
+    if (Hq % Hkv) return fail(SPA_ERR_INVALID, "Hq must be a multiple of Hkv");
+    if (dt != SPA_F32 && dt != SPA_BF16) return fail(SPA_ERR_INVALID, "unknown dtype");
+    if (!(scale > 0.f) || !(top_p > 0.f)) return fail(SPA_ERR_INVALID, "scale and top_p must be > 0");
+    if (n_sink < 0 || n_local < 0 || k_min < 0)
+        return fail(SPA_ERR_INVALID, "n_sink, n_local and k_min must be >= 0");
+    const int nb = ceil_div(L, block);
+    if (cap < nb) return fail(SPA_ERR_INVALID, "cap must be >= nb");
+    if (!aligned16(q) || !aligned16(mean) || !aligned16(var))
+        return fail(SPA_ERR_INVALID, "tensors must be 16-byte aligned");
+    if (d != 64 && d != 128) return fail(SPA_ERR_UNSUPPORTED, "d must be 64 or 128");
+    if (block < 1 || block > 1024) return fail(SPA_ERR_UNSUPPORTED, "block must be in [1, 1024]");
+    if (nb > 16384) return fail(SPA_ERR_UNSUPPORTED, "more than 16384 key blocks");
+    int *err = device_error_ptr();
+    if (!err) return fail(SPA_ERR_CUDA, "device error word unavailable");
+    cudaError_t e = launch_select(q, dt == SPA_BF16, mean, var, B, Hq, Hkv, L, L, d, block, scale,
+                                  top_p, n_sink, n_local, k_min, idx, cap, count, err,
+                                  static_cast<cudaStream_t>(stream), nullptr, true);
+    return e == cudaSuccess ? SPA_OK : cuda_fail(e, "select launch");
+}
+
+SPA_API spa_status spa_sparse_attn_prefill_early_stop(
+    const void *q, const void *k, const void *v, spa_dtype dt, int B, int Hq, int Hkv, int L, int d,
+    int block, const int32_t *idx, int cap, const int32_t *count, float scale, int n_sink,
+    int n_local, float tau, void *out, float *lse, int32_t *processed, spa_stream stream) {
+    t_last_error.clear();
+    if (!q || !k || !v || !idx || !count || !out || !processed)
+        return fail(SPA_ERR_INVALID, "null pointer");
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || L <= 0 || d <= 0 || block <= 0)
+        return fail(SPA_ERR_INVALID, "sizes must be positive");
+    if (Hq % Hkv) return fail(SPA_ERR_INVALID, "Hq must be a multiple of Hkv");
+    if (!(scale > 0.f)) return fail(SPA_ERR_INVALID, "scale must be > 0");
+    if (!(tau >= 0.f)) return fail(SPA_ERR_INVALID, "tau must be >= 0");
+    if (n_sink < 0 || n_local < 0) return fail(SPA_ERR_INVALID, "n_sink and n_local must be >= 0");
+    if (cap < ceil_div(L, block)) return fail(SPA_ERR_INVALID, "cap must be >= nb");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+        return fail(SPA_ERR_INVALID, "tensors must be 16-byte aligned");
+    if (dt != SPA_BF16 || d != 128 || block != 128)
+        return fail(SPA_ERR_UNSUPPORTED, "early stop needs bf16, d = 128, block 128");
+    if (ceil_div(L, block) > 4096) return fail(SPA_ERR_UNSUPPORTED, "more than 4096 query blocks");
+    int *err = device_error_ptr();
+    if (!err) return fail(SPA_ERR_CUDA, "device error word unavailable");
+    cudaError_t e = launch_prefill_tc_early_stop(q, k, v, B, Hq, Hkv, L, idx, cap, count, scale,
+                                                 n_sink, n_local, tau, out, lse, processed, err,
+                                                 static_cast<cudaStream_t>(stream));
+    if (e == cudaErrorNotSupported) return fail(SPA_ERR_UNSUPPORTED, "tensor map encoding unavailable");
+    return e == cudaSuccess ? SPA_OK : cuda_fail(e, "prefill launch");
+}
+
 SPA_API size_t spa_quantized_stats_bytes(int B, int Hkv, int T, int d, int block) {
     if (B <= 0 || Hkv <= 0 || T <= 0 || block <= 0 || (d != 64 && d != 128)) return 0;
     return quantized_stats_bytes(B, Hkv, T, d, block);

@@ -65,6 +65,11 @@ def lib() -> ctypes.CDLL:
         L.spa_quantize_block_stats.argtypes = [_P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P]
         L.spa_select_quantized.argtypes = [_P, _I, _P, _I, _I, _I, _I, _I, _I, _I, _F, _F, _I, _I,
                                            _I, _P, _I, _P, _P]
+        L.spa_select_score_order.argtypes = [_P, _I, _P, _P, _I, _I, _I, _I, _I, _I, _F, _F, _I,
+                                             _I, _I, _P, _I, _P, _P]
+        L.spa_sparse_attn_prefill_early_stop.argtypes = [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I,
+                                                         _P, _I, _P, _F, _I, _I, _F, _P, _P, _P,
+                                                         _P]
         L.spa_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_int)]
         L.spa_status_string.argtypes = [_I]
         L.spa_status_string.restype = ctypes.c_char_p
@@ -72,7 +77,8 @@ def lib() -> ctypes.CDLL:
         for f in ("spa_block_stats", "spa_select", "spa_sparse_attn_prefill",
                   "spa_sparse_attn_decode", "spa_get_device_error", "spa_rla_block_states",
                   "spa_rla_prefill", "spa_rla_decode_state", "spa_sparse_attn_decode_rla",
-                  "spa_quantize_block_stats", "spa_select_quantized"):
+                  "spa_quantize_block_stats", "spa_select_quantized", "spa_select_score_order",
+                  "spa_sparse_attn_prefill_early_stop"):
             getattr(L, f).restype = _I
         _lib = L
     return _lib
@@ -193,6 +199,50 @@ def spa_select_quantized(q: torch.Tensor, qstats: torch.Tensor, T: int, block: i
                                       scale, top_p, n_sink, n_local, k_min, _ptr(idx),
                                       idx.shape[-1], _ptr(count), _stream(stream)))
     return idx, count
+
+
+def spa_select_score_order(q: torch.Tensor, mean: torch.Tensor, var: torch.Tensor, block: int,
+                           scale: float, top_p: float, n_sink: int = 1, n_local: int = 1,
+                           k_min: int = 0, idx: torch.Tensor | None = None,
+                           count: torch.Tensor | None = None, stream=None):
+    """Prefill selection with the kept lists in traversal order. Returns (idx, count)."""
+    B, Hq, L, d = q.shape
+    Hkv = mean.shape[1]
+    nb = -(-L // block)
+    if idx is None:
+        idx = torch.empty((B, Hq, nb, nb), device=q.device, dtype=torch.int32)
+    if count is None:
+        count = torch.empty((B, Hq, nb), device=q.device, dtype=torch.int32)
+    _check("spa_select_score_order",
+           lib().spa_select_score_order(_ptr(q), _dt(q), _ptr(mean), _ptr(var), B, Hq, Hkv, L, d,
+                                        block, scale, top_p, n_sink, n_local, k_min, _ptr(idx),
+                                        idx.shape[-1], _ptr(count), _stream(stream)))
+    return idx, count
+
+
+def spa_sparse_attn_prefill_early_stop(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                                       block: int, idx: torch.Tensor, count: torch.Tensor,
+                                       scale: float, tau: float, n_sink: int = 1, n_local: int = 1,
+                                       out: torch.Tensor | None = None,
+                                       lse: torch.Tensor | None = None, want_lse: bool = False,
+                                       processed: torch.Tensor | None = None, stream=None):
+    """Attention over the prefix of score-ordered lists kept by the early stop.
+    Returns (out, lse or None, processed [B, Hq, nq] int32)."""
+    B, Hq, L, d = q.shape
+    Hkv = k.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq, L), device=q.device, dtype=torch.float32)
+    if processed is None:
+        processed = torch.empty(count.shape, device=q.device, dtype=torch.int32)
+    _check("spa_sparse_attn_prefill_early_stop",
+           lib().spa_sparse_attn_prefill_early_stop(_ptr(q), _ptr(k), _ptr(v), _dt(q), B, Hq, Hkv,
+                                                    L, d, block, _ptr(idx), idx.shape[-1],
+                                                    _ptr(count), scale, n_sink, n_local, tau,
+                                                    _ptr(out), _ptr(lse), _ptr(processed),
+                                                    _stream(stream)))
+    return out, lse, processed
 
 
 def spa_sparse_attn_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block: int,

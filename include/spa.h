@@ -166,6 +166,45 @@ spa_status spa_sparse_attn_prefill(const void *q, const void *k, const void *v, 
 size_t spa_decode_workspace_bytes(int B, int Hq, int Hkv, int T, int d, int block);
 
 /*
+ * Score-ordered traversal with early stop ("S2O", section 2: blocks visited in
+ * descending estimated importance, the walk stopped once a block's marginal gain
+ * in attention mass falls below tau relative to the accumulated mass; section 3:
+ * a dense pass over the own block first).
+ *
+ * spa_select_score_order: spa_select for prefill (Lq = L = T) with the kept lists
+ * written in traversal order instead of ascending: the local blocks (the query's
+ * own block first, descending), the sink blocks (ascending), then the kept residual
+ * blocks in the cut's rank order (score descending, equal scores by ascending
+ * index). Same kept sets and counts as spa_select. Arguments as spa_select.
+ */
+spa_status spa_select_score_order(const void *q, spa_dtype dt, const float *mean, const float *var,
+                                  int B, int Hq, int Hkv, int L, int d, int block, float scale,
+                                  float top_p, int n_sink, int n_local, int k_min, int32_t *idx,
+                                  int cap, int32_t *count, spa_stream stream);
+
+/*
+ * spa_sparse_attn_prefill_early_stop: exact attention over a prefix of each
+ * score-ordered list. After each ranked block (reserved sink and local blocks are
+ * always processed), the query block stops if, for every row t of it (t < L),
+ *   (mass of this block for row t) / (mass of all blocks processed so far for t) < tau,
+ * masses being sums of exp(s q_t . k_u) over the causal keys u <= t, in the
+ * kernel's fp32 online-softmax state; the stopping block is included.
+ *   idx, count : lists in traversal order (spa_select_score_order); entries outside
+ *            [0, i] and repeats are skipped (SPA_DEVERR_BAD_INDEX)
+ *   n_sink, n_local : the reserved blocks, as given to the selection
+ *   tau    : >= 0 (0 never stops)
+ *   out, lse : as spa_sparse_attn_prefill
+ *   processed : [B, Hq, nq] int32 output, the number of list entries processed
+ * bf16, d = 128, block 128, at most 4096 query blocks.
+ */
+spa_status spa_sparse_attn_prefill_early_stop(const void *q, const void *k, const void *v,
+                                              spa_dtype dt, int B, int Hq, int Hkv, int L, int d,
+                                              int block, const int32_t *idx, int cap,
+                                              const int32_t *count, float scale, int n_sink,
+                                              int n_local, float tau, void *out, float *lse,
+                                              int32_t *processed, spa_stream stream);
+
+/*
  * Block-sparse decode attention: one new query per sequence against a KV cache of
  * length T that already holds the new token (the query sits at position T-1). The
  * pages describe decode as bound by re-reading the cache ("SpotAttention", problem

@@ -291,9 +291,13 @@ def score_order(sel: dict, Lq: int, T: int, block: int, n_sink: int = 1, n_local
                 lst = [int(j) for j in idx[b, h, i, :c]]
                 last_row = min((i + 1) * block, Lq)
                 jmax = (T - Lq + last_row - 1) // block
-                local = sorted([j for j in lst if j > jmax - n_local], reverse=True)
-                sink = sorted([j for j in lst if j < n_sink and j <= jmax - n_local])
-                res = [j for j in lst if n_sink <= j <= jmax - n_local]
+                # reserved ranges as the cut defines them: sink [0, r_lo), local
+                # [r_hi, jmax]; where they would overlap the sink takes precedence
+                r_lo = min(n_sink, jmax + 1)
+                r_hi = max(r_lo, jmax - n_local + 1)
+                local = sorted([j for j in lst if j >= r_hi], reverse=True)
+                sink = sorted([j for j in lst if j < r_lo])
+                res = [j for j in lst if r_lo <= j < r_hi]
                 res.sort(key=lambda j: (-float(np.float32(l[b, h, i, j])), j))
                 order = local + sink + res
                 out[b, h, i, :c] = order

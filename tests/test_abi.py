@@ -175,6 +175,23 @@ def test_quantized_stats_host_checks(lib):
     assert g(FAKE, 1, None, 1, 4, 2, 1, 256, 128, 16, 0.1, 0.9, 1, 1, 0, FAKE, 16, FAKE, None) == 1
 
 
+def test_early_stop_host_checks(lib):
+    I, F = ctypes.c_int, ctypes.c_float
+    f = lib.spa_sparse_attn_prefill_early_stop
+    f.argtypes = [P, P, P, I, I, I, I, I, I, I, P, I, P, F, I, I, F, P, P, P, P]
+    args = lambda dt, d, blk, cap, tau, proc: (FAKE, FAKE, FAKE, dt, 1, 4, 2, 512, d, blk, FAKE, cap,
+                                               FAKE, 0.1, 1, 1, tau, FAKE, None, proc, None)
+    assert f(*args(1, 128, 64, 8, 0.1, FAKE)) == 2           # block 64
+    assert f(*args(0, 128, 128, 4, 0.1, FAKE)) == 2          # fp32
+    assert f(*args(1, 128, 128, 3, 0.1, FAKE)) == 1          # cap < nb
+    assert f(*args(1, 128, 128, 4, -1.0, FAKE)) == 1         # tau < 0
+    assert f(*args(1, 128, 128, 4, 0.1, None)) == 1          # no processed output
+    g = lib.spa_select_score_order
+    g.argtypes = [P, I, P, P, I, I, I, I, I, I, F, F, I, I, I, P, I, P, P]
+    assert g(FAKE, 1, FAKE, FAKE, 1, 4, 2, 512, 96, 128, 0.1, 0.9, 1, 1, 0, FAKE, 4, FAKE, None) == 2
+    assert g(FAKE, 1, FAKE, FAKE, 1, 4, 2, 512, 128, 128, 0.1, 0.9, 1, 1, 0, FAKE, 3, FAKE, None) == 1
+
+
 def test_decode_workspace_size(lib):
     f = lib.spa_decode_workspace_bytes
     f.restype = ctypes.c_size_t
