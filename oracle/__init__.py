@@ -56,11 +56,15 @@ def _bind(path: str):
     lib.oracle_rla_block_states.argtypes = [_P, _P, _I, _I, _I, _I, _I, _I, _P]
     lib.oracle_early_stop.argtypes = [_P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _I, _P, _D, _I,
                                       _I, _D, _P, _P]
+    lib.oracle_pbs_permutation.argtypes = [_P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P]
+    lib.oracle_attention_segperm.argtypes = [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P,
+                                             _I, _P, _D, _P, _I64, _P, _P]
     lib.oracle_quantize_stats.argtypes = [_P, _P, _I, _I, _I, _I, _P, _P, _P, _P]
     lib.oracle_dequantize_stats.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _P, _P]
     for f in ("oracle_block_stats", "oracle_scores", "oracle_select_from_scores",
               "oracle_attention", "oracle_rla", "oracle_rla_block_states",
-              "oracle_quantize_stats", "oracle_dequantize_stats", "oracle_early_stop"):
+              "oracle_quantize_stats", "oracle_dequantize_stats", "oracle_early_stop",
+              "oracle_pbs_permutation", "oracle_attention_segperm"):
         getattr(lib, f).restype = _I
     return lib
 
@@ -322,6 +326,78 @@ def early_stop(q, k, dtype: str, block: int, idx: np.ndarray, count: np.ndarray,
                                      cap, _ptr(count), float(scale), n_sink, n_local, float(tau),
                                      _ptr(processed), _ptr(ratios)), "early_stop")
     return processed, ratios
+
+
+def pbs_permutation(q, k, dtype: str, block: int, seg_blocks: int) -> np.ndarray:
+    """Segmented key permutation (PBS, sections 2-3; reading in spa_oracle.c):
+    perm [B, Hkv, L] int32, the original index of the key at each permuted position."""
+    q, isb = _inp(q, dtype)
+    k, _ = _inp(k, dtype)
+    B, Hq, L, d = q.shape
+    Hkv = k.shape[1]
+    perm = np.empty((B, Hkv, L), np.int32)
+    _check(_load().oracle_pbs_permutation(_ptr(q), _ptr(k), isb, B, Hq, Hkv, L, d, block, seg_blocks,
+                                          _ptr(perm)), "pbs_permutation")
+    return perm
+
+
+def permute(x: np.ndarray, perm: np.ndarray) -> np.ndarray:
+    """x [B, Hkv, L, d] in the permuted layout: row p of (b, g) is x[b, g, perm[b, g, p]]."""
+    return np.take_along_axis(x, perm[..., None].astype(np.int64), axis=2)
+
+
+def select_segperm(q, k, dtype: str, block: int, seg_blocks: int, scale: float, top_p: float,
+                   n_sink: int = 1, n_local: int = 1, k_min: int = 0, perm=None):
+    """The selection on the segment-permuted layout: a query block scores the blocks
+    of earlier segments on the permuted keys' statistics and the blocks of its own
+    segment on the original ones; then the same cut."""
+    if perm is None:
+        perm = pbs_permutation(q, k, dtype, block, seg_blocks)
+    kp = permute(np.asarray(k), perm)
+    mean, var = block_stats(k, dtype, block)
+    mp, vp = block_stats(kp, dtype, block)
+    L = q.shape[2]
+    lo = scores(q, dtype, mean, var, L, block, scale)
+    lp = scores(q, dtype, mp, vp, L, block, scale)
+    nq = lo.shape[2]
+    seg0 = (np.arange(nq) // seg_blocks) * seg_blocks          # first block of the own segment
+    use_p = np.arange(lo.shape[3])[None, :] < seg0[:, None]      # [nq, nb]
+    l = np.where(use_p[None, None], lp, lo)
+    idx, count = select_from_scores(l, L, L, block, top_p, n_sink, n_local, k_min)
+    return {"perm": perm, "mean": mean, "var": var, "mean_p": mp, "var_p": vp, "scores": l,
+            "idx": idx, "count": count}
+
+
+def attention_segperm(q, k, v, dtype: str, block: int, seg_blocks: int, perm: np.ndarray,
+                      idx: np.ndarray, count: np.ndarray, scale: float,
+                      rows: np.ndarray | None = None):
+    """Masked softmax attention for lists on the segment-permuted layout (fp64);
+    returns (out, lse) like `attention`."""
+    q, isb = _inp(q, dtype)
+    k, _ = _inp(k, dtype)
+    v, _ = _inp(v, dtype)
+    B, Hq, L, d = q.shape
+    Hkv = k.shape[1]
+    perm = np.ascontiguousarray(perm, np.int32)
+    idx = np.ascontiguousarray(idx, np.int32)
+    count = np.ascontiguousarray(count, np.int32)
+    cap = idx.shape[-1]
+    if rows is None:
+        n = B * Hq * L
+        out = np.empty((B, Hq, L, d), np.float64)
+        lse = np.empty((B, Hq, L), np.float64)
+        rp = None
+    else:
+        rows = np.ascontiguousarray(rows, np.int64)
+        n = rows.size
+        out = np.empty((n, d), np.float64)
+        lse = np.empty((n,), np.float64)
+        rp = _ptr(rows)
+    _check(_load().oracle_attention_segperm(_ptr(q), _ptr(k), _ptr(v), isb, B, Hq, Hkv, L, d, block,
+                                            seg_blocks, _ptr(perm), _ptr(idx), cap, _ptr(count),
+                                            float(scale), rp, n, _ptr(out), _ptr(lse)),
+           "attention_segperm")
+    return out, lse
 
 
 def full_lists(B: int, Hq: int, Lq: int, T: int, block: int):

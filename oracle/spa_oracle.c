@@ -681,3 +681,161 @@ int oracle_early_stop(const void *q, const void *k, int is_bf16, int B, int Hq, 
     }
     return err;
 }
+
+/*
+ * Segmented key permutation ("Sparsere Blok-Sparse Attention via Tokenpermutatie",
+ * sections 2-3). The keys (with their values) are divided into segments of
+ * seg_blocks * block tokens and sorted inside each segment by a global importance
+ * score, descending; segments keep their order, so causality between segments is
+ * untouched. Reading of the score: the mean pooling of the attention scores of the
+ * last query block, taken on the logits: importance(u) = qbar . k_u, with qbar the
+ * mean of the last query block's rows over the query heads of the kv-group (the
+ * positive softmax scale does not change the order). Equal scores keep the smaller
+ * index first. perm[b, g, p] = the original index of the key at permuted position p.
+ */
+typedef struct { double score; int idx; } imp_t;
+
+static int imp_cmp(const void *a, const void *b)
+{
+    const imp_t *x = (const imp_t *)a, *y = (const imp_t *)b;
+    if (x->score > y->score) return -1;
+    if (x->score < y->score) return 1;
+    return (x->idx > y->idx) - (x->idx < y->idx);
+}
+
+int oracle_pbs_permutation(const void *q, const void *k, int is_bf16, int B, int Hq, int Hkv,
+                           int L, int d, int block, int seg_blocks, int32_t *perm)
+{
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || L <= 0 || d <= 0 || block <= 0 ||
+        seg_blocks <= 0)
+        return ORACLE_EINVAL;
+    const int G = Hq / Hkv, nq = ceil_div(L, block), S = seg_blocks * block;
+    const int r0 = (nq - 1) * block, nr = L - r0;
+    int err = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int bg = 0; bg < B * Hkv; ++bg) {
+        const int b = bg / Hkv, g = bg % Hkv;
+        double *qbar = (double *)calloc((size_t)d, sizeof(double));
+        imp_t *imp = (imp_t *)malloc(sizeof(imp_t) * (size_t)L);
+        if (!qbar || !imp) {
+#pragma omp atomic write
+            err = ORACLE_ENOMEM;
+            free(qbar);
+            free(imp);
+            continue;
+        }
+        for (int hh = 0; hh < G; ++hh)
+            for (int r = 0; r < nr; ++r)
+                for (int c = 0; c < d; ++c)
+                    qbar[c] += elem(q, is_bf16, (((size_t)b * Hq + g * G + hh) * L + r0 + r) * d + c);
+        for (int c = 0; c < d; ++c) qbar[c] /= (double)(G * nr);
+        for (int u = 0; u < L; ++u) {
+            double s = 0.0;
+            for (int c = 0; c < d; ++c) s += qbar[c] * elem(k, is_bf16, ((size_t)bg * L + u) * d + c);
+            imp[u].score = s;
+            imp[u].idx = u;
+        }
+        for (int s0 = 0; s0 < L; s0 += S) {
+            const int n = (s0 + S < L ? S : L - s0);
+            qsort(imp + s0, (size_t)n, sizeof(imp_t), imp_cmp);
+        }
+        for (int p = 0; p < L; ++p) perm[(size_t)bg * L + p] = imp[p].idx;
+        free(qbar);
+        free(imp);
+    }
+    return err;
+}
+
+/*
+ * Attention on the segment-permuted layout, as masked softmax over the ORIGINAL
+ * keys. For query row t (prefill, Lq = T) in query block i, segment start
+ * s_i = (i / seg_blocks) * seg_blocks blocks:
+ *   a key u before the segment start (u < s_i * block) is allowed iff the permuted
+ *   block holding it, inv_perm[u] / block, is in the kept list (those blocks are
+ *   entirely in the past: no token mask);
+ *   a key u of the query's own segment is allowed iff u <= t and its original block
+ *   u / block is in the kept list.
+ * Otherwise as oracle_attention (textbook softmax per row). perm as
+ * oracle_pbs_permutation.
+ */
+int oracle_attention_segperm(const void *q, const void *k, const void *v, int is_bf16, int B,
+                             int Hq, int Hkv, int L, int d, int block, int seg_blocks,
+                             const int32_t *perm, const int32_t *idx, int cap,
+                             const int32_t *count, double scale, const int64_t *rows,
+                             int64_t nrows, double *out, double *lse)
+{
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || L <= 0 || d <= 0 || block <= 0 ||
+        seg_blocks <= 0 || cap < 1)
+        return ORACLE_EINVAL;
+    const int nb = ceil_div(L, block), G = Hq / Hkv;
+    if (!rows) nrows = (int64_t)B * Hq * L;
+    int err = 0;
+#pragma omp parallel
+    {
+        unsigned char *kept = (unsigned char *)malloc((size_t)nb);
+        double *z = (double *)malloc(sizeof(double) * L);
+        int32_t *inv = (int32_t *)malloc(sizeof(int32_t) * L);
+        int inv_bg = -1;
+        if (!kept || !z || !inv) {
+#pragma omp atomic write
+            err = ORACLE_ENOMEM;
+        }
+#pragma omp for schedule(dynamic, 4)
+        for (int64_t n = 0; n < nrows; ++n) {
+            if (!kept || !z || !inv) continue;
+            const int64_t r = rows ? rows[n] : n;
+            const int64_t bh = r / L;
+            const int t = (int)(r % L);
+            const int b = (int)(bh / Hq), h = (int)(bh % Hq), g = h / G, bg = b * Hkv + g;
+            const int i = t / block;
+            const int seg0 = (i / seg_blocks) * seg_blocks * block;
+            if (inv_bg != bg) {
+                for (int p = 0; p < L; ++p) inv[perm[(size_t)bg * L + p]] = p;
+                inv_bg = bg;
+            }
+            const size_t u_list = (size_t)bh * nb + i;
+            memset(kept, 0, (size_t)nb);
+            int cnt = count[u_list];
+            int bad = cnt < 0 || cnt > cap;
+            for (int c = 0; c < cnt && !bad; ++c) {
+                const int j = idx[u_list * cap + c];
+                if (j < 0 || j >= nb) bad = 1; else kept[j] = 1;
+            }
+            if (bad) {
+#pragma omp atomic write
+                err = ORACLE_EINVAL;
+                continue;
+            }
+            const size_t qoff = (size_t)r * d, kvbase = (size_t)bg * L;
+            double m = -INFINITY;
+            for (int u = 0; u < L; ++u) {
+                const int allowed = u < seg0 ? kept[inv[u] / block] : (u <= t && kept[u / block]);
+                if (!allowed) { z[u] = -INFINITY; continue; }
+                double s = 0.0;
+                for (int c = 0; c < d; ++c)
+                    s += elem(q, is_bf16, qoff + c) * elem(k, is_bf16, (kvbase + u) * d + c);
+                z[u] = s * scale;
+                if (z[u] > m) m = z[u];
+            }
+            double *o = out + (size_t)n * d;
+            for (int c = 0; c < d; ++c) o[c] = 0.0;
+            if (m == -INFINITY) {
+                if (lse) lse[n] = -INFINITY;
+                continue;
+            }
+            double den = 0.0;
+            for (int u = 0; u < L; ++u) {
+                if (z[u] == -INFINITY) continue;
+                const double p = exp(z[u] - m);
+                den += p;
+                for (int c = 0; c < d; ++c) o[c] += p * elem(v, is_bf16, (kvbase + u) * d + c);
+            }
+            for (int c = 0; c < d; ++c) o[c] /= den;
+            if (lse) lse[n] = m + log(den);
+        }
+        free(kept);
+        free(z);
+        free(inv);
+    }
+    return err;
+}

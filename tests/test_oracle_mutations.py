@@ -79,6 +79,15 @@ MUTATIONS = [
      "const double ratio = acc[r] > 0.0 ? gsum / acc[r] : 0.0;\n                    acc[r] += gsum;",
      [pins.test_early_stop_ratio_is_gain_over_accumulated_mass,
       pins.test_early_stop_constant_keys_closed_form]),
+    ("segperm_ascending_importance", "if (x->score > y->score) return -1;\n    if (x->score < y->score) return 1;",
+     "if (x->score < y->score) return -1;\n    if (x->score > y->score) return 1;",
+     [pins.test_segperm_hand_worked_permutation,
+      pins.test_segperm_sorts_each_segment_by_pooled_query_logit]),
+    ("segperm_pooled_over_the_first_block", "const int r0 = (nq - 1) * block, nr = L - r0;",
+     "const int r0 = 0, nr = block < L ? block : L;",
+     [pins.test_segperm_sorts_each_segment_by_pooled_query_logit]),
+    ("segperm_earlier_keys_by_original_block", "kept[inv[u] / block]", "kept[u / block]",
+     [pins.test_segperm_attention_in_the_permuted_layout]),
     ("ascending_sort", "if (x->key > y->key) return -1;\n    if (x->key < y->key) return 1;",
      "if (x->key < y->key) return -1;\n    if (x->key > y->key) return 1;",
      [pins.test_top_p_hand_worked_examples, pins.test_top_p_tiny_p_keeps_top_one]),

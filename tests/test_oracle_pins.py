@@ -825,3 +825,79 @@ def test_score_order_lists_are_the_kept_sets_in_rank_order():
             assert lst[1] == 0                           # then the sink
         s32 = [float(np.float32(sel["scores"][b, h, i, j])) for j in ranked]
         assert all((s32[x], -ranked[x]) >= (s32[x + 1], -ranked[x + 1]) for x in range(len(s32) - 1))
+
+
+# ---------------------------------------------------------------- segmented key permutation
+# PBS (Sparsere Blok-Sparse Attention via Tokenpermutatie), sections 2-3: keys sorted
+# by global importance inside segments; segments keep their causal order.
+
+def test_segperm_hand_worked_permutation():
+    g = _golden()["segmented_permutation"]
+    q = np.array(g["q"], np.float32).reshape(1, 1, -1, 1)
+    k = np.array(g["k"], np.float32).reshape(1, 1, -1, 1)
+    perm = oracle.pbs_permutation(q, k, "f32", g["block"], g["seg_blocks"])
+    assert perm.reshape(-1).tolist() == g["expected_perm"]
+
+
+def test_segperm_sorts_each_segment_by_pooled_query_logit():
+    B, Hq, Hkv, L, d, blk, seg = 1, 4, 2, 96, 8, 8, 3
+    q, k = _rand((B, Hq, L, d), 90), _rand((B, Hkv, L, d), 91)
+    perm = oracle.pbs_permutation(q, k, "f32", blk, seg)
+    G, S = Hq // Hkv, seg * blk
+    for g in range(Hkv):
+        qbar = q[0, g * G:(g + 1) * G, L - blk:].astype(np.float64).reshape(-1, d).mean(0)
+        imp = k[0, g].astype(np.float64) @ qbar
+        for s0 in range(0, L, S):
+            p = perm[0, g, s0:s0 + S]
+            assert sorted(p.tolist()) == list(range(s0, min(s0 + S, L)))   # within the segment
+            assert all((imp[p[x]], -p[x]) >= (imp[p[x + 1]], -p[x + 1]) for x in range(len(p) - 1))
+
+
+def test_segperm_at_p_one_is_dense_causal_attention():
+    B, Hq, Hkv, L, d, blk = 1, 4, 2, 64, 16, 8
+    q, k, v = _rand((B, Hq, L, d), 92), _rand((B, Hkv, L, d), 93), _rand((B, Hkv, L, d), 94)
+    ref = _dense_causal_numpy(q, k, v, 0.25)
+    for seg in (1, 2, 3):
+        sel = oracle.select_segperm(q, k, "f32", blk, seg, 0.25, 1.0)
+        out, _ = oracle.attention_segperm(q, k, v, "f32", blk, seg, sel["perm"], sel["idx"],
+                                          sel["count"], 0.25)
+        np.testing.assert_allclose(out, ref, rtol=1e-11, atol=1e-12)
+
+
+def test_segperm_with_one_segment_is_the_plain_path():
+    B, Hq, Hkv, L, d, blk = 1, 4, 2, 64, 16, 8
+    q, k, v = _rand((B, Hq, L, d), 95), _rand((B, Hkv, L, d), 96), _rand((B, Hkv, L, d), 97)
+    a = oracle.select(q, k, "f32", blk, 0.25, 0.6)
+    b = oracle.select_segperm(q, k, "f32", blk, 8, 0.25, 0.6)     # 8 blocks: one segment
+    assert np.array_equal(a["idx"], b["idx"]) and np.array_equal(a["count"], b["count"])
+    oa, _ = oracle.attention(q, k, v, "f32", blk, a["idx"], a["count"], 0.25)
+    ob, _ = oracle.attention_segperm(q, k, v, "f32", blk, 8, b["perm"], b["idx"], b["count"], 0.25)
+    np.testing.assert_allclose(ob, oa, rtol=1e-13, atol=1e-14)
+
+
+def test_segperm_attention_in_the_permuted_layout():
+    # The same masked attention evaluated directly on the permuted keys: earlier
+    # segments by permuted block, the own segment in original order and causal.
+    B, Hq, Hkv, L, d, blk, seg = 1, 2, 1, 48, 8, 4, 3
+    q, k, v = _rand((B, Hq, L, d), 98), _rand((B, Hkv, L, d), 99), _rand((B, Hkv, L, d), 100)
+    sel = oracle.select_segperm(q, k, "f32", blk, seg, 0.5, 0.5)
+    perm = sel["perm"]
+    out, _ = oracle.attention_segperm(q, k, v, "f32", blk, seg, perm, sel["idx"], sel["count"], 0.5)
+    kp, vp = oracle.permute(k, perm)[0, 0].astype(np.float64), oracle.permute(v, perm)[0, 0].astype(np.float64)
+    ko, vo = k[0, 0].astype(np.float64), v[0, 0].astype(np.float64)
+    for h in range(Hq):
+        for t in range(L):
+            i = t // blk
+            s0 = (i // seg) * seg * blk
+            kept = set(sel["idx"][0, h, i, :sel["count"][0, h, i]].tolist())
+            keys, vals = [], []
+            for p in range(s0):                      # earlier segments, permuted layout
+                if p // blk in kept:
+                    keys.append(kp[p]); vals.append(vp[p])
+            for u in range(s0, t + 1):               # own segment, original layout
+                if u // blk in kept:
+                    keys.append(ko[u]); vals.append(vo[u])
+            z = 0.5 * np.array(keys) @ q[0, h, t].astype(np.float64)
+            w = np.exp(z - z.max())
+            np.testing.assert_allclose(out[0, h, t], (w / w.sum()) @ np.array(vals), rtol=1e-11,
+                                       atol=1e-12)
