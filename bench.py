@@ -242,6 +242,8 @@ def main():
                     help="skip the Residual Linear Attention leg")
     ap.add_argument("--tau", type=float, default=0.2,
                     help="early-stop threshold for the score-ordered traversal leg (0: skip)")
+    ap.add_argument("--seg-blocks", type=int, default=16,
+                    help="segment length (in blocks) of the segmented-permutation leg (0: skip)")
     ap.add_argument("--no-quant", action="store_true",
                     help="skip the selection on quantised statistics in the decode leg")
     ap.add_argument("--no-cpu", action="store_true")
@@ -469,6 +471,62 @@ def main():
                                             statistics.mean(t_stats) + t_osel + t_es)}
         del oidx, ocnt, proc, eout
 
+    # ---- segmented key permutation (PBS, sections 2-3)
+    pbs = None
+    if args.seg_blocks > 0 and w.dtype == "bf16" and args.seg_blocks * w.block <= 8192:
+        perm = torch.empty((B, Hkv, L), device="cuda", dtype=torch.int32)
+        kp, vp = torch.empty_like(k), torch.empty_like(v)
+        mp, vp_ = torch.empty_like(mean), torch.empty_like(var)
+        pidx, pcnt = torch.empty_like(idx), torch.empty_like(cnt)
+        pout = torch.empty_like(q)
+
+        def pbs_step(ev=None):
+            if ev:
+                ev[0].record(stream)
+            spa.spa_pbs_permutation(q, k, w.block, args.seg_blocks, perm=perm)
+            spa.spa_pbs_gather(k, perm, xp=kp)
+            spa.spa_pbs_gather(v, perm, xp=vp)
+            spa.spa_block_stats(kp, w.block, mean=mp, var=vp_)
+            if ev:
+                ev[1].record(stream)
+            spa.spa_select_segperm(q, mean, var, mp, vp_, w.block, args.seg_blocks, w.scale,
+                                   w.top_p, w.n_sink, w.n_local, w.k_min, idx=pidx, count=pcnt)
+            if ev:
+                ev[2].record(stream)
+            spa.spa_sparse_attn_prefill_segperm(q, k, v, kp, vp, w.block, args.seg_blocks, pidx,
+                                                pcnt, w.scale, out=pout)
+            if ev:
+                ev[3].record(stream)
+        for _ in range(3):
+            spa.spa_block_stats(k, w.block, mean=mean, var=var)
+            pbs_step()
+        torch.cuda.synchronize()
+        assert spa.spa_get_device_error() == 0
+        n_pb = max(5, args.steps // 4)
+        pb_evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n_pb)]
+        barrier()
+        torch.cuda.synchronize()
+        for s_ in range(n_pb):
+            flush.zero_()
+            pbs_step(pb_evs[s_])
+        torch.cuda.synchronize()
+        barrier()
+        t_perm = rank_max(statistics.mean(e[0].elapsed_time(e[1]) for e in pb_evs))
+        t_psel = rank_max(statistics.mean(e[1].elapsed_time(e[2]) for e in pb_evs))
+        t_patt = rank_max(statistics.mean(e[2].elapsed_time(e[3]) for e in pb_evs))
+        pc = pcnt.cpu().numpy()
+        F_p = kept_flops(pc, pidx.cpu().numpy(), L, w.block, d)
+        dev_ = (pout.float() - out.float())
+        pbs = {"seg_blocks": args.seg_blocks,
+               "kept_fraction": float(pc.sum()) / dense_tiles, "kept_fraction_plain": kept_frac,
+               "permute_gather_stats_ms": t_perm, "select_ms": t_psel, "attn_ms": t_patt,
+               "TFLOP/s": F_p / (t_patt / 1e3) / 1e12,
+               "tokens/s": job_throughput(B * L, world, 1, t_perm + t_psel + t_patt +
+                                          statistics.mean(t_stats)),
+               "vs_plain_output": {"max_abs": float(dev_.abs().max().item()),
+                                   "rms": float(dev_.pow(2).mean().sqrt().item())}}
+        del perm, kp, vp, mp, vp_, pidx, pcnt, pout
+
     # ---- decode leg
     decode = None
     if not args.no_decode:
@@ -642,6 +700,7 @@ def main():
             "kernels": per_kernel,
             "rla": rla,
             "early_stop": early,
+            "segmented_permutation": pbs,
             "decode": decode,
             "e2e": e2e,
             "cpu_baseline": cpu,

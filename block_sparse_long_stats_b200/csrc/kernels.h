@@ -18,7 +18,8 @@ cudaError_t launch_select(const void *q, bool bf16, const float *mean, const flo
                           int Hq, int Hkv, int Lq, int T, int d, int block, float scale,
                           float top_p, int n_sink, int n_local, int k_min, int32_t *idx, int cap,
                           int32_t *count, int *err, cudaStream_t s, const void *qstats = nullptr,
-                          bool score_order = false);
+                          bool score_order = false, const float *mean_p = nullptr,
+                          const float *var_p = nullptr, int seg_blocks = 0);
 
 // Quantised block statistics (INT4 microscale records of d + d/16 bytes per block;
 // format in qstats.cu). launch_select reads them instead of mean/var when qstats is set.
@@ -37,7 +38,16 @@ cudaError_t launch_prefill_f32(const float *q, const float *k, const float *v, i
 cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, int B, int Hq, int Hkv,
                               int L, int block, const int32_t *idx, int cap,
                               const int32_t *count, float scale, void *out, float *lse, int *err,
-                              cudaStream_t s);
+                              cudaStream_t s, const void *kp = nullptr, const void *vp = nullptr,
+                              int seg_blocks = 0);
+
+// Segmented key permutation: perm [B, Hkv, L] (original index per permuted
+// position) and the permuted copy of K or V (rows of row_bytes bytes).
+cudaError_t launch_pbs_permutation(const void *q, const void *k, bool bf16, int B, int Hq, int Hkv,
+                                   int L, int d, int block, int seg_blocks, int32_t *perm,
+                                   cudaStream_t s);
+cudaError_t launch_gather_rows(const void *x, int B, int Hkv, int L, int row_bytes,
+                               const int32_t *perm, void *xp, cudaStream_t s);
 
 // Residual Linear Attention (bf16, d = 128, block 64 or 128): per-block states
 // W_j [B, Hkv, nb, d, d] bf16, and the prefill branch output [B, Hq, L, d] fp32.

@@ -1,0 +1,162 @@
+// Segmented key permutation ("Sparsere Blok-Sparse Attention via Tokenpermutatie",
+// sections 2-3): inside each segment of seg_blocks * block tokens the keys are
+// sorted by a global importance score, descending, so that the keys many queries
+// attend to gather in the segment's first blocks; segments keep their order, so
+// causality between segments holds. The importance of key u is qbar . k_u, with
+// qbar the mean of the last query block's rows over the query heads of the
+// kv-group (the mean-pooled logits of the last query block; the positive softmax
+// scale does not change the order). Equal scores keep the smaller index first.
+//
+// pbs_perm_kernel: one CTA per (segment, b * Hkv + g): qbar (fp32), one fp32 score
+// per key (a warp per key, 16-byte loads, shuffle sum), then a bitonic sort of
+// 64-bit keys (order-flipped score | index) in shared memory; writes perm.
+// gather_rows_kernel: the permuted copy of K or V, 16 bytes per thread.
+#include <float.h>
+
+#include <algorithm>
+
+#include "kernels.h"
+
+namespace spa {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+
+__device__ __forceinline__ uint32_t order_desc(float f) {
+    const uint32_t b = __float_as_uint(f);
+    const uint32_t ord = (b & 0x80000000u) ? ~b : (b | 0x80000000u);   // ascending with f
+    return ~ord;                                                        // descending with f
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kThreads) pbs_perm_kernel(const T *__restrict__ q,
+                                                            const T *__restrict__ k, int Hq,
+                                                            int Hkv, int L, int block,
+                                                            int seg_len, int sort_cap,
+                                                            int32_t *__restrict__ perm) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    uint64_t *keys = reinterpret_cast<uint64_t *>(smem_raw);     // [sort_cap]
+    __shared__ float qbar[D];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int bg = blockIdx.y, b = bg / Hkv, g = bg % Hkv, G = Hq / Hkv;
+    const int s0 = blockIdx.x * seg_len, n = min(seg_len, L - s0);
+    const int nq = (L + block - 1) / block, r0 = (nq - 1) * block, nr = L - r0;
+
+    // pooled query of the last query block over the group's heads
+    for (int c = tid; c < D; c += kThreads) {
+        float acc = 0.f;
+        for (int hh = 0; hh < G; ++hh) {
+            const T *qh = q + (((size_t)b * Hq + g * G + hh) * L + r0) * D + c;
+            for (int r = 0; r < nr; ++r) {
+                if constexpr (sizeof(T) == 2)
+                    acc += __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(qh)[(size_t)r * D]);
+                else
+                    acc += reinterpret_cast<const float *>(qh)[(size_t)r * D];
+            }
+        }
+        qbar[c] = acc / (float)(G * nr);
+    }
+    __syncthreads();
+
+    // importance of each key of the segment: a warp per key
+    constexpr int PL = D / 32;
+    float qv[PL];
+#pragma unroll
+    for (int c = 0; c < PL; ++c) qv[c] = qbar[lane * PL + c];
+    for (int x = warp; x < n; x += kWarps) {
+        const T *kr = k + ((size_t)bg * L + s0 + x) * D + lane * PL;
+        float s = 0.f;
+#pragma unroll
+        for (int c = 0; c < PL; ++c) {
+            float kv;
+            if constexpr (sizeof(T) == 2)
+                kv = __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(kr)[c]);
+            else
+                kv = reinterpret_cast<const float *>(kr)[c];
+            s = fmaf(qv[c], kv, s);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        if (lane == 0) keys[x] = ((uint64_t)order_desc(s) << 32) | (uint32_t)x;
+    }
+    for (int x = n + tid; x < sort_cap; x += kThreads) keys[x] = ~0ull;
+    __syncthreads();
+
+    // bitonic sort, ascending keys = descending score, ascending index
+    for (int kk = 2; kk <= sort_cap; kk <<= 1) {
+        for (int jj = kk >> 1; jj > 0; jj >>= 1) {
+            const int lj = __ffs(jj) - 1;
+            for (int p = tid; p < (sort_cap >> 1); p += kThreads) {
+                const int xa = ((p >> lj) << (lj + 1)) | (p & (jj - 1));
+                const uint64_t ka = keys[xa], kb = keys[xa + jj];
+                const bool up = (xa & kk) == 0;
+                if ((ka > kb) == up) {
+                    keys[xa] = kb;
+                    keys[xa + jj] = ka;
+                }
+            }
+            __syncthreads();
+        }
+    }
+    int32_t *out = perm + (size_t)bg * L + s0;
+    for (int x = tid; x < n; x += kThreads) out[x] = s0 + (int)(uint32_t)keys[x];
+}
+
+// xp[row p of (b, g)] = x[row perm[b, g, p] of (b, g)]; rows of row_bytes bytes.
+__global__ void __launch_bounds__(kThreads) gather_rows_kernel(const uint4 *__restrict__ x,
+                                                               const int32_t *__restrict__ perm,
+                                                               int L, int vec_per_row, size_t n_vec,
+                                                               uint4 *__restrict__ xp) {
+    for (size_t e = (size_t)blockIdx.x * kThreads + threadIdx.x; e < n_vec;
+         e += (size_t)gridDim.x * kThreads) {
+        const size_t row = e / vec_per_row;                 // (b, g, p)
+        const int c = (int)(e % vec_per_row);
+        const size_t bg = row / L;
+        const int src = __ldg(perm + row);
+        xp[e] = __ldg(x + (bg * L + src) * vec_per_row + c);
+    }
+}
+
+template <typename T, int D>
+cudaError_t launch_perm_t(const void *q, const void *k, int B, int Hq, int Hkv, int L, int block,
+                          int seg_blocks, int32_t *perm, cudaStream_t s) {
+    const int seg_len = seg_blocks * block;
+    int cap = 1;
+    while (cap < seg_len) cap <<= 1;
+    const size_t smem = (size_t)cap * 8;
+    auto kern = pbs_perm_kernel<T, D>;
+    if (smem > 48 * 1024) {
+        const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    dim3 grid((unsigned)((L + seg_len - 1) / seg_len), (unsigned)(B * Hkv));
+    kern<<<grid, kThreads, smem, s>>>(reinterpret_cast<const T *>(q), reinterpret_cast<const T *>(k),
+                                      Hq, Hkv, L, block, seg_len, cap, perm);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_pbs_permutation(const void *q, const void *k, bool bf16, int B, int Hq, int Hkv,
+                                   int L, int d, int block, int seg_blocks, int32_t *perm,
+                                   cudaStream_t s) {
+    if (bf16)
+        return d == 128 ? launch_perm_t<__nv_bfloat16, 128>(q, k, B, Hq, Hkv, L, block, seg_blocks, perm, s)
+                        : launch_perm_t<__nv_bfloat16, 64>(q, k, B, Hq, Hkv, L, block, seg_blocks, perm, s);
+    return d == 128 ? launch_perm_t<float, 128>(q, k, B, Hq, Hkv, L, block, seg_blocks, perm, s)
+                    : launch_perm_t<float, 64>(q, k, B, Hq, Hkv, L, block, seg_blocks, perm, s);
+}
+
+cudaError_t launch_gather_rows(const void *x, int B, int Hkv, int L, int row_bytes,
+                               const int32_t *perm, void *xp, cudaStream_t s) {
+    const int vpr = row_bytes / 16;
+    const size_t n_vec = (size_t)B * Hkv * L * vpr;
+    const unsigned grid = (unsigned)std::min<size_t>((n_vec + kThreads - 1) / kThreads, 148 * 32);
+    gather_rows_kernel<<<grid, kThreads, 0, s>>>(reinterpret_cast<const uint4 *>(x), perm, L, vpr,
+                                                  n_vec, reinterpret_cast<uint4 *>(xp));
+    return cudaGetLastError();
+}
+
+}  // namespace spa

@@ -50,6 +50,9 @@ struct PrefillArgs {
     float tau;
     int32_t *processed;   // [B, Hq, nq]: list entries processed
     int nwords;           // words of the duplicate bitmap
+    // segment-permuted layout: blocks before the query's own segment come from the
+    // permuted K/V copies (tkp, tvp); 0: off
+    int seg_blocks;
 };
 
 // Walks the ascending kept lists of the HPT heads of a tile in merged order. All
@@ -142,7 +145,8 @@ struct Cfg {
 template <int BLK, bool ES>
 __global__ void __launch_bounds__(kThreads, 2)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-                       const __grid_constant__ CUtensorMap tv, PrefillArgs a) {
+                       const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tkp,
+                       const __grid_constant__ CUtensorMap tvp, PrefillArgs a) {
     static_assert(!ES || BLK == 128, "early stop walks one head's list");
     using C = Cfg<BLK>;
     constexpr int HPT = C::HPT;
@@ -251,6 +255,11 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
             cur.init(a, b, h0, i, true);
             const int kv_row0 = (b * a.Hkv + g) * a.L;
+            const int seg0 = a.seg_blocks > 0 ? (i / a.seg_blocks) * a.seg_blocks : 0;
+            if (a.seg_blocks > 0) {
+                prefetch_tmap(&tkp);
+                prefetch_tmap(&tvp);
+            }
             int j;
             uint32_t mask;
             for (int n = 0; next(j, mask, true); ++n) {
@@ -259,9 +268,12 @@ __global__ void __launch_bounds__(kThreads, 2)
                 unsigned char *kt = smem + C::OFF_K + s * C::KV_BYTES;
                 unsigned char *vt = smem + C::OFF_V + s * C::KV_BYTES;
                 if (!mbar_wait(&empty_k[s], ph ^ 1, a.err)) break;
+                const bool perm_src = j < seg0;        // an earlier segment: permuted copy
+                const CUtensorMap *mk = perm_src ? &tkp : &tk;
+                const CUtensorMap *mv = perm_src ? &tvp : &tv;
                 mbar_arrive_expect_tx(&full_k[s], C::KV_BYTES);
-                tma_load_2d(kt, &tk, &full_k[s], 0, kv_row0 + j * BLK);
-                tma_load_2d(kt + C::KV_HALF, &tk, &full_k[s], 64, kv_row0 + j * BLK);
+                tma_load_2d(kt, mk, &full_k[s], 0, kv_row0 + j * BLK);
+                tma_load_2d(kt + C::KV_HALF, mk, &full_k[s], 64, kv_row0 + j * BLK);
                 if constexpr (ES) {
                     if (n > 0) {
                         if (!mbar_wait(&decided[(n - 1) & 1], ((n - 1) >> 1) & 1, a.err)) break;
@@ -273,8 +285,8 @@ __global__ void __launch_bounds__(kThreads, 2)
                 }
                 if (!mbar_wait(&empty_v[s], ph ^ 1, a.err)) break;
                 mbar_arrive_expect_tx(&full_v[s], C::KV_BYTES);
-                tma_load_2d(vt, &tv, &full_v[s], 0, kv_row0 + j * BLK);
-                tma_load_2d(vt + C::KV_HALF, &tv, &full_v[s], 64, kv_row0 + j * BLK);
+                tma_load_2d(vt, mv, &full_v[s], 0, kv_row0 + j * BLK);
+                tma_load_2d(vt + C::KV_HALF, mv, &full_v[s], 64, kv_row0 + j * BLK);
             }
         }
     } else if (warp == 5) {
@@ -480,19 +492,20 @@ bool make_map(CUtensorMap *map, const void *base, uint64_t rows, int box_rows) {
 
 template <int BLK, bool ES>
 cudaError_t launch_blk(const void *q, const void *k, const void *v, const PrefillArgs &a,
-                       cudaStream_t s) {
+                       cudaStream_t s, const void *kp = nullptr, const void *vp = nullptr) {
     using C = Cfg<BLK>;
-    CUtensorMap mq, mk, mv;
-    if (!make_map(&mq, q, (uint64_t)a.B * a.Hq * a.L, BLK) ||
-        !make_map(&mk, k, (uint64_t)a.B * a.Hkv * a.L, BLK) ||
-        !make_map(&mv, v, (uint64_t)a.B * a.Hkv * a.L, BLK))
+    CUtensorMap mq, mk, mv, mkp, mvp;
+    const uint64_t kv_rows = (uint64_t)a.B * a.Hkv * a.L;
+    if (!make_map(&mq, q, (uint64_t)a.B * a.Hq * a.L, BLK) || !make_map(&mk, k, kv_rows, BLK) ||
+        !make_map(&mv, v, kv_rows, BLK) || !make_map(&mkp, kp ? kp : k, kv_rows, BLK) ||
+        !make_map(&mvp, vp ? vp : v, kv_rows, BLK))
         return cudaErrorNotSupported;
     const size_t smem = C::SMEM + 1024 + (ES ? (size_t)a.nq * 4 + (size_t)a.nwords * 4 : 0);
     auto kern = prefill_tc_kernel<BLK, ES>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)((size_t)a.nq * a.B * a.Hkv * a.npairs);
-    kern<<<grid, kThreads, smem, s>>>(mq, mk, mv, a);
+    kern<<<grid, kThreads, smem, s>>>(mq, mk, mv, mkp, mvp, a);
     return cudaGetLastError();
 }
 
@@ -501,7 +514,7 @@ cudaError_t launch_blk(const void *q, const void *k, const void *v, const Prefil
 cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, int B, int Hq, int Hkv,
                               int L, int block, const int32_t *idx, int cap,
                               const int32_t *count, float scale, void *out, float *lse, int *err,
-                              cudaStream_t s) {
+                              cudaStream_t s, const void *kp, const void *vp, int seg_blocks) {
     PrefillArgs a;
     a.idx = idx;
     a.count = count;
@@ -519,7 +532,9 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, int B
     a.tau = 0.f;
     a.processed = nullptr;
     a.nwords = 0;
-    return block == 64 ? launch_blk<64, false>(q, k, v, a, s) : launch_blk<128, false>(q, k, v, a, s);
+    a.seg_blocks = seg_blocks;
+    return block == 64 ? launch_blk<64, false>(q, k, v, a, s, kp, vp)
+                       : launch_blk<128, false>(q, k, v, a, s, kp, vp);
 }
 
 cudaError_t launch_prefill_tc_early_stop(const void *q, const void *k, const void *v, int B, int Hq,
@@ -544,6 +559,7 @@ cudaError_t launch_prefill_tc_early_stop(const void *q, const void *k, const voi
     a.tau = tau;
     a.processed = processed;
     a.nwords = (a.nq + 31) / 32;
+    a.seg_blocks = 0;
     return launch_blk<128, true>(q, k, v, a, s);
 }
 

@@ -179,6 +179,10 @@ struct SelectArgs {
     bool prescored; // decode: the fp32 scores are already in the unit's row of idx
     const uint8_t *qstats;  // quantised statistics (records of d + d/16 bytes) or null
     bool score_order;       // prefill: lists in traversal order instead of ascending
+    // segment-permuted layout: blocks before the query's own segment are scored on
+    // the permuted keys' statistics (seg_blocks = 0: off)
+    const float *mean_p, *var_p;
+    int seg_blocks;
 };
 
 template <typename T, int D, bool QS>
@@ -264,11 +268,16 @@ __global__ void __launch_bounds__(kThreads) select_kernel(SelectArgs a) {
         const float *mb = QS ? nullptr : a.mean + bgo * D + lane * PL;
         const float *vb = QS ? nullptr : a.var + bgo * D + lane * PL;
         const uint8_t *qb = QS ? a.qstats + bgo * (D + D / 16) : nullptr;
+        const int seg0 = a.seg_blocks > 0 ? (i / a.seg_blocks) * a.seg_blocks : 0;
+        const float *mbp = a.seg_blocks > 0 ? a.mean_p + bgo * D + lane * PL : nullptr;
+        const float *vbp = a.seg_blocks > 0 ? a.var_p + bgo * D + lane * PL : nullptr;
         for (int r = warp; r < nres; r += kWarps) {
             const int j = r_lo + r;
             float mu[PL], vr[PL], dot, quad;
             if constexpr (QS)
                 load_stats_q<D>(qb + (size_t)j * (D + D / 16), lane, mu, vr);
+            else if (j < seg0)
+                load_stats<PL>(mbp + (size_t)j * D, vbp + (size_t)j * D, mu, vr);
             else
                 load_stats<PL>(mb + (size_t)j * D, vb + (size_t)j * D, mu, vr);
             lane_partials<PL>(qv, q2, mu, vr, dot, quad);
@@ -647,9 +656,13 @@ cudaError_t launch_select(const void *q, bool bf16, const float *mean, const flo
                           int Hq, int Hkv, int Lq, int T, int d, int block, float scale,
                           float top_p, int n_sink, int n_local, int k_min, int32_t *idx, int cap,
                           int32_t *count, int *err, cudaStream_t s, const void *qstats,
-                          bool score_order) {
+                          bool score_order, const float *mean_p, const float *var_p,
+                          int seg_blocks) {
     SelectArgs a;
     a.score_order = score_order;
+    a.mean_p = mean_p;
+    a.var_p = var_p;
+    a.seg_blocks = seg_blocks;
     a.q = q; a.mean = mean; a.var = var;
     a.qstats = reinterpret_cast<const uint8_t *>(qstats);
     a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.Lq = Lq; a.T = T; a.d = d; a.block = block;

@@ -188,6 +188,97 @@ SPA_API spa_status spa_sparse_attn_prefill_early_stop(
     return e == cudaSuccess ? SPA_OK : cuda_fail(e, "prefill launch");
 }
 
+SPA_API spa_status spa_pbs_permutation(const void *q, const void *k, spa_dtype dt, int B, int Hq,
+                                       int Hkv, int L, int d, int block, int seg_blocks,
+                                       int32_t *perm, spa_stream stream) {
+    t_last_error.clear();
+    if (!q || !k || !perm) return fail(SPA_ERR_INVALID, "null pointer");
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || L <= 0 || d <= 0 || block <= 0 || seg_blocks <= 0)
+        return fail(SPA_ERR_INVALID, "sizes must be positive");
+    if (Hq % Hkv) return fail(SPA_ERR_INVALID, "Hq must be a multiple of Hkv");
+    if (dt != SPA_F32 && dt != SPA_BF16) return fail(SPA_ERR_INVALID, "unknown dtype");
+    if (!aligned16(q) || !aligned16(k)) return fail(SPA_ERR_INVALID, "tensors must be 16-byte aligned");
+    if (d != 64 && d != 128) return fail(SPA_ERR_UNSUPPORTED, "d must be 64 or 128");
+    if ((long)seg_blocks * block > 8192)
+        return fail(SPA_ERR_UNSUPPORTED, "a segment holds at most 8192 tokens");
+    cudaError_t e = launch_pbs_permutation(q, k, dt == SPA_BF16, B, Hq, Hkv, L, d, block, seg_blocks,
+                                           perm, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? SPA_OK : cuda_fail(e, "permutation launch");
+}
+
+SPA_API spa_status spa_pbs_gather(const void *x, spa_dtype dt, int B, int Hkv, int L, int d,
+                                  const int32_t *perm, void *xp, spa_stream stream) {
+    t_last_error.clear();
+    if (!x || !perm || !xp) return fail(SPA_ERR_INVALID, "null pointer");
+    if (B <= 0 || Hkv <= 0 || L <= 0 || d <= 0) return fail(SPA_ERR_INVALID, "sizes must be positive");
+    if (dt != SPA_F32 && dt != SPA_BF16) return fail(SPA_ERR_INVALID, "unknown dtype");
+    if (!aligned16(x) || !aligned16(xp)) return fail(SPA_ERR_INVALID, "tensors must be 16-byte aligned");
+    const int row_bytes = d * (dt == SPA_BF16 ? 2 : 4);
+    if (row_bytes % 16) return fail(SPA_ERR_UNSUPPORTED, "rows must be a multiple of 16 bytes");
+    cudaError_t e = launch_gather_rows(x, B, Hkv, L, row_bytes, perm, xp,
+                                       static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? SPA_OK : cuda_fail(e, "gather launch");
+}
+
+SPA_API spa_status spa_select_segperm(const void *q, spa_dtype dt, const float *mean,
+                                      const float *var, const float *mean_p, const float *var_p,
+                                      int B, int Hq, int Hkv, int L, int d, int block,
+                                      int seg_blocks, float scale, float top_p, int n_sink,
+                                      int n_local, int k_min, int32_t *idx, int cap,
+                                      int32_t *count, spa_stream stream) {
+    t_last_error.clear();
+    if (!q || !mean || !var || !mean_p || !var_p || !idx || !count)
+        return fail(SPA_ERR_INVALID, "null pointer");
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || L <= 0 || d <= 0 || block <= 0 || seg_blocks <= 0)
+        return fail(SPA_ERR_INVALID, "sizes must be positive");
+    if (Hq % Hkv) return fail(SPA_ERR_INVALID, "Hq must be a multiple of Hkv");
+    if (dt != SPA_F32 && dt != SPA_BF16) return fail(SPA_ERR_INVALID, "unknown dtype");
+    if (!(scale > 0.f) || !(top_p > 0.f)) return fail(SPA_ERR_INVALID, "scale and top_p must be > 0");
+    if (n_sink < 0 || n_local < 0 || k_min < 0)
+        return fail(SPA_ERR_INVALID, "n_sink, n_local and k_min must be >= 0");
+    const int nb = ceil_div(L, block);
+    if (cap < nb) return fail(SPA_ERR_INVALID, "cap must be >= nb");
+    if (!aligned16(q) || !aligned16(mean) || !aligned16(var) || !aligned16(mean_p) || !aligned16(var_p))
+        return fail(SPA_ERR_INVALID, "tensors must be 16-byte aligned");
+    if (d != 64 && d != 128) return fail(SPA_ERR_UNSUPPORTED, "d must be 64 or 128");
+    if (block < 1 || block > 1024) return fail(SPA_ERR_UNSUPPORTED, "block must be in [1, 1024]");
+    if (nb > 16384) return fail(SPA_ERR_UNSUPPORTED, "more than 16384 key blocks");
+    int *err = device_error_ptr();
+    if (!err) return fail(SPA_ERR_CUDA, "device error word unavailable");
+    cudaError_t e = launch_select(q, dt == SPA_BF16, mean, var, B, Hq, Hkv, L, L, d, block, scale,
+                                  top_p, n_sink, n_local, k_min, idx, cap, count, err,
+                                  static_cast<cudaStream_t>(stream), nullptr, false, mean_p, var_p,
+                                  seg_blocks);
+    return e == cudaSuccess ? SPA_OK : cuda_fail(e, "select launch");
+}
+
+SPA_API spa_status spa_sparse_attn_prefill_segperm(
+    const void *q, const void *k, const void *v, const void *kp, const void *vp, spa_dtype dt,
+    int B, int Hq, int Hkv, int L, int d, int block, int seg_blocks, const int32_t *idx, int cap,
+    const int32_t *count, float scale, void *out, float *lse, spa_stream stream) {
+    t_last_error.clear();
+    if (!q || !k || !v || !kp || !vp || !idx || !count || !out)
+        return fail(SPA_ERR_INVALID, "null pointer");
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || L <= 0 || d <= 0 || block <= 0 || seg_blocks <= 0)
+        return fail(SPA_ERR_INVALID, "sizes must be positive");
+    if (Hq % Hkv) return fail(SPA_ERR_INVALID, "Hq must be a multiple of Hkv");
+    if (!(scale > 0.f)) return fail(SPA_ERR_INVALID, "scale must be > 0");
+    if (cap < ceil_div(L, block)) return fail(SPA_ERR_INVALID, "cap must be >= nb");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(kp) || !aligned16(vp) ||
+        !aligned16(out))
+        return fail(SPA_ERR_INVALID, "tensors must be 16-byte aligned");
+    if (dt != SPA_BF16 || d != 128 || (block != 64 && block != 128))
+        return fail(SPA_ERR_UNSUPPORTED, "the permuted layout needs bf16, d = 128, block 64 or 128");
+    if ((Hq / Hkv) % (128 / block))
+        return fail(SPA_ERR_UNSUPPORTED, "block 64 needs an even number of query heads per kv-head");
+    int *err = device_error_ptr();
+    if (!err) return fail(SPA_ERR_CUDA, "device error word unavailable");
+    cudaError_t e = launch_prefill_tc(q, k, v, B, Hq, Hkv, L, block, idx, cap, count, scale, out, lse,
+                                      err, static_cast<cudaStream_t>(stream), kp, vp, seg_blocks);
+    if (e == cudaErrorNotSupported) return fail(SPA_ERR_UNSUPPORTED, "tensor map encoding unavailable");
+    return e == cudaSuccess ? SPA_OK : cuda_fail(e, "prefill launch");
+}
+
 SPA_API size_t spa_quantized_stats_bytes(int B, int Hkv, int T, int d, int block) {
     if (B <= 0 || Hkv <= 0 || T <= 0 || block <= 0 || (d != 64 && d != 128)) return 0;
     return quantized_stats_bytes(B, Hkv, T, d, block);

@@ -70,6 +70,12 @@ def lib() -> ctypes.CDLL:
         L.spa_sparse_attn_prefill_early_stop.argtypes = [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I,
                                                          _P, _I, _P, _F, _I, _I, _F, _P, _P, _P,
                                                          _P]
+        L.spa_pbs_permutation.argtypes = [_P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P]
+        L.spa_pbs_gather.argtypes = [_P, _I, _I, _I, _I, _I, _P, _P, _P]
+        L.spa_select_segperm.argtypes = [_P, _I, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F,
+                                         _F, _I, _I, _I, _P, _I, _P, _P]
+        L.spa_sparse_attn_prefill_segperm.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I,
+                                                      _I, _I, _P, _I, _P, _F, _P, _P, _P]
         L.spa_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_int)]
         L.spa_status_string.argtypes = [_I]
         L.spa_status_string.restype = ctypes.c_char_p
@@ -78,7 +84,8 @@ def lib() -> ctypes.CDLL:
                   "spa_sparse_attn_decode", "spa_get_device_error", "spa_rla_block_states",
                   "spa_rla_prefill", "spa_rla_decode_state", "spa_sparse_attn_decode_rla",
                   "spa_quantize_block_stats", "spa_select_quantized", "spa_select_score_order",
-                  "spa_sparse_attn_prefill_early_stop"):
+                  "spa_sparse_attn_prefill_early_stop", "spa_pbs_permutation", "spa_pbs_gather",
+                  "spa_select_segperm", "spa_sparse_attn_prefill_segperm"):
             getattr(L, f).restype = _I
         _lib = L
     return _lib
@@ -243,6 +250,73 @@ def spa_sparse_attn_prefill_early_stop(q: torch.Tensor, k: torch.Tensor, v: torc
                                                     _ptr(out), _ptr(lse), _ptr(processed),
                                                     _stream(stream)))
     return out, lse, processed
+
+
+def spa_pbs_permutation(q: torch.Tensor, k: torch.Tensor, block: int, seg_blocks: int,
+                        perm: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Segmented key permutation: perm [B, Hkv, L] int32 (original index per position)."""
+    B, Hq, L, d = q.shape
+    Hkv = k.shape[1]
+    if perm is None:
+        perm = torch.empty((B, Hkv, L), device=q.device, dtype=torch.int32)
+    _check("spa_pbs_permutation",
+           lib().spa_pbs_permutation(_ptr(q), _ptr(k), _dt(q), B, Hq, Hkv, L, d, block, seg_blocks,
+                                     _ptr(perm), _stream(stream)))
+    return perm
+
+
+def spa_pbs_gather(x: torch.Tensor, perm: torch.Tensor, xp: torch.Tensor | None = None,
+                   stream=None) -> torch.Tensor:
+    """The permuted copy of K or V: xp[b, g, p] = x[b, g, perm[b, g, p]]."""
+    B, Hkv, L, d = x.shape
+    if xp is None:
+        xp = torch.empty_like(x)
+    _check("spa_pbs_gather",
+           lib().spa_pbs_gather(_ptr(x), _dt(x), B, Hkv, L, d, _ptr(perm), _ptr(xp),
+                                _stream(stream)))
+    return xp
+
+
+def spa_select_segperm(q: torch.Tensor, mean: torch.Tensor, var: torch.Tensor,
+                       mean_p: torch.Tensor, var_p: torch.Tensor, block: int, seg_blocks: int,
+                       scale: float, top_p: float, n_sink: int = 1, n_local: int = 1,
+                       k_min: int = 0, idx: torch.Tensor | None = None,
+                       count: torch.Tensor | None = None, stream=None):
+    """Prefill selection on the segment-permuted layout. Returns (idx, count)."""
+    B, Hq, L, d = q.shape
+    Hkv = mean.shape[1]
+    nb = -(-L // block)
+    if idx is None:
+        idx = torch.empty((B, Hq, nb, nb), device=q.device, dtype=torch.int32)
+    if count is None:
+        count = torch.empty((B, Hq, nb), device=q.device, dtype=torch.int32)
+    _check("spa_select_segperm",
+           lib().spa_select_segperm(_ptr(q), _dt(q), _ptr(mean), _ptr(var), _ptr(mean_p),
+                                    _ptr(var_p), B, Hq, Hkv, L, d, block, seg_blocks, scale, top_p,
+                                    n_sink, n_local, k_min, _ptr(idx), idx.shape[-1], _ptr(count),
+                                    _stream(stream)))
+    return idx, count
+
+
+def spa_sparse_attn_prefill_segperm(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                                    kp: torch.Tensor, vp: torch.Tensor, block: int, seg_blocks: int,
+                                    idx: torch.Tensor, count: torch.Tensor, scale: float,
+                                    out: torch.Tensor | None = None,
+                                    lse: torch.Tensor | None = None, want_lse: bool = False,
+                                    stream=None):
+    """Block-sparse prefill on the segment-permuted layout. Returns (out, lse or None)."""
+    B, Hq, L, d = q.shape
+    Hkv = k.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq, L), device=q.device, dtype=torch.float32)
+    _check("spa_sparse_attn_prefill_segperm",
+           lib().spa_sparse_attn_prefill_segperm(_ptr(q), _ptr(k), _ptr(v), _ptr(kp), _ptr(vp),
+                                                 _dt(q), B, Hq, Hkv, L, d, block, seg_blocks,
+                                                 _ptr(idx), idx.shape[-1], _ptr(count), scale,
+                                                 _ptr(out), _ptr(lse), _stream(stream)))
+    return out, lse
 
 
 def spa_sparse_attn_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block: int,

@@ -205,6 +205,48 @@ spa_status spa_sparse_attn_prefill_early_stop(const void *q, const void *k, cons
                                               int32_t *processed, spa_stream stream);
 
 /*
+ * Segmented key permutation. Follows "Sparsere Blok-Sparse Attention via
+ * Tokenpermutatie", sections 2-3: the sequence is cut into segments of
+ * seg_blocks * block tokens; inside each, keys (with their values) are sorted by a
+ * global importance score, descending, so the keys many queries attend to gather
+ * in the segment's first blocks; segments keep their order (causality between
+ * segments holds); queries keep their order. Importance (the mean-pooled scores
+ * of the last query block, taken on the logits): qbar . k_u, qbar the mean of the
+ * last query block's rows over the query heads of the kv-group; equal scores keep
+ * the smaller index first (fp32 scores).
+ *
+ * spa_pbs_permutation: perm [B, Hkv, L] int32 output, perm[b,g,p] = the original
+ *   index of the key at permuted position p. q [B, Hq, L, d], k [B, Hkv, L, d],
+ *   dt, d = 64 or 128; a segment holds at most 8192 tokens.
+ * spa_pbs_gather: xp[b,g,p,:] = x[b,g,perm[b,g,p],:], for K and for V (rows of
+ *   d elements of dt; the copies the two calls below read).
+ * spa_select_segperm: spa_select for prefill on this layout: query block i scores
+ *   the blocks before its own segment (j < (i / seg_blocks) * seg_blocks) on the
+ *   statistics of the permuted keys (mean_p, var_p: spa_block_stats of kp) and the
+ *   blocks of its own segment on the original ones; same cut and lists.
+ * spa_sparse_attn_prefill_segperm: spa_sparse_attn_prefill where the kept blocks
+ *   before the query's own segment are read from kp, vp (they lie entirely in the
+ *   past: no mask) and those of its own segment from k, v (the diagonal block
+ *   masked token by token). bf16, d = 128, block 64 or 128.
+ */
+spa_status spa_pbs_permutation(const void *q, const void *k, spa_dtype dt, int B, int Hq, int Hkv,
+                               int L, int d, int block, int seg_blocks, int32_t *perm,
+                               spa_stream stream);
+spa_status spa_pbs_gather(const void *x, spa_dtype dt, int B, int Hkv, int L, int d,
+                          const int32_t *perm, void *xp, spa_stream stream);
+spa_status spa_select_segperm(const void *q, spa_dtype dt, const float *mean, const float *var,
+                              const float *mean_p, const float *var_p, int B, int Hq, int Hkv,
+                              int L, int d, int block, int seg_blocks, float scale, float top_p,
+                              int n_sink, int n_local, int k_min, int32_t *idx, int cap,
+                              int32_t *count, spa_stream stream);
+spa_status spa_sparse_attn_prefill_segperm(const void *q, const void *k, const void *v,
+                                           const void *kp, const void *vp, spa_dtype dt, int B,
+                                           int Hq, int Hkv, int L, int d, int block,
+                                           int seg_blocks, const int32_t *idx, int cap,
+                                           const int32_t *count, float scale, void *out,
+                                           float *lse, spa_stream stream);
+
+/*
  * Block-sparse decode attention: one new query per sequence against a KV cache of
  * length T that already holds the new token (the query sits at position T-1). The
  * pages describe decode as bound by re-reading the cache ("SpotAttention", problem
