@@ -8,7 +8,8 @@
 // scale does not change the order). Equal scores keep the smaller index first.
 //
 // pbs_perm_kernel: one CTA per (segment, b * Hkv + g): qbar (fp32), one fp32 score
-// per key (a warp per key, 16-byte loads, shuffle sum), then a bitonic sort of
+// per key (d / 8 lanes per key with 16-byte loads, four in flight, shuffle sums),
+// then a bitonic sort of
 // 64-bit keys (order-flipped score | index) in shared memory; writes perm.
 // gather_rows_kernel: the permuted copy of K or V, 16 bytes per thread.
 #include <float.h>
@@ -37,48 +38,83 @@ __global__ void __launch_bounds__(kThreads) pbs_perm_kernel(const T *__restrict_
                                                             int32_t *__restrict__ perm) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     uint64_t *keys = reinterpret_cast<uint64_t *>(smem_raw);     // [sort_cap]
+    constexpr int V = 16 / sizeof(T);             // elements per 16-byte chunk
+    constexpr int CPR = D / V;                    // chunks per row
+    constexpr int RG = kThreads / CPR;            // row groups
     __shared__ float qbar[D];
+    __shared__ float part[RG][D];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int bg = blockIdx.y, b = bg / Hkv, g = bg % Hkv, G = Hq / Hkv;
     const int s0 = blockIdx.x * seg_len, n = min(seg_len, L - s0);
     const int nq = (L + block - 1) / block, r0 = (nq - 1) * block, nr = L - r0;
 
-    // pooled query of the last query block over the group's heads
-    for (int c = tid; c < D; c += kThreads) {
-        float acc = 0.f;
-        for (int hh = 0; hh < G; ++hh) {
-            const T *qh = q + (((size_t)b * Hq + g * G + hh) * L + r0) * D + c;
-            for (int r = 0; r < nr; ++r) {
-                if constexpr (sizeof(T) == 2)
-                    acc += __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(qh)[(size_t)r * D]);
-                else
-                    acc += reinterpret_cast<const float *>(qh)[(size_t)r * D];
+    // pooled query of the last query block over the group's heads: thread (rg, c)
+    // sums 16-byte chunk c of rows rg, rg + RG, ... of all G heads
+    {
+        const int c = tid % CPR, rg = tid / CPR;
+        float acc[V];
+#pragma unroll
+        for (int e = 0; e < V; ++e) acc[e] = 0.f;
+        for (int x = rg; x < G * nr; x += RG) {
+            const int hh = x / nr, r = x % nr;
+            const uint4 u = __ldg(reinterpret_cast<const uint4 *>(
+                q + (((size_t)b * Hq + g * G + hh) * L + r0 + r) * D) + c);
+            if constexpr (sizeof(T) == 2) {
+                acc[0] += bf16lo(u.x); acc[1] += bf16hi(u.x); acc[2] += bf16lo(u.y);
+                acc[3] += bf16hi(u.y); acc[4] += bf16lo(u.z); acc[5] += bf16hi(u.z);
+                acc[6] += bf16lo(u.w); acc[7] += bf16hi(u.w);
+            } else {
+                acc[0] += __uint_as_float(u.x); acc[1] += __uint_as_float(u.y);
+                acc[2] += __uint_as_float(u.z); acc[3] += __uint_as_float(u.w);
             }
         }
+#pragma unroll
+        for (int e = 0; e < V; ++e) part[rg][c * V + e] = acc[e];
+    }
+    __syncthreads();
+    for (int c = tid; c < D; c += kThreads) {
+        float acc = 0.f;
+        for (int rg = 0; rg < RG; ++rg) acc += part[rg][c];
         qbar[c] = acc / (float)(G * nr);
     }
     __syncthreads();
 
-    // importance of each key of the segment: a warp per key
-    constexpr int PL = D / 32;
-    float qv[PL];
+    // importance of each key of the segment: LPK lanes per key, one 16-byte chunk
+    // each, U loads in flight per lane
+    constexpr int LPK = CPR;                      // lanes per key
+    constexpr int KPW = 32 / LPK;                 // keys per warp load
+    constexpr int U = 4;
+    const int sub = lane / LPK, cl = lane % LPK;
+    float qv[V];
 #pragma unroll
-    for (int c = 0; c < PL; ++c) qv[c] = qbar[lane * PL + c];
-    for (int x = warp; x < n; x += kWarps) {
-        const T *kr = k + ((size_t)bg * L + s0 + x) * D + lane * PL;
-        float s = 0.f;
+    for (int e = 0; e < V; ++e) qv[e] = qbar[cl * V + e];
+    for (int x0 = warp * KPW * U; x0 < n; x0 += kWarps * KPW * U) {
+        uint4 u[U];
 #pragma unroll
-        for (int c = 0; c < PL; ++c) {
-            float kv;
-            if constexpr (sizeof(T) == 2)
-                kv = __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(kr)[c]);
-            else
-                kv = reinterpret_cast<const float *>(kr)[c];
-            s = fmaf(qv[c], kv, s);
+        for (int uu = 0; uu < U; ++uu) {
+            const int x = x0 + uu * KPW + sub;
+            u[uu] = x < n ? __ldg(reinterpret_cast<const uint4 *>(k + ((size_t)bg * L + s0 + x) * D) + cl)
+                          : make_uint4(0, 0, 0, 0);
         }
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-        if (lane == 0) keys[x] = ((uint64_t)order_desc(s) << 32) | (uint32_t)x;
+        for (int uu = 0; uu < U; ++uu) {
+            float kv[V];
+            if constexpr (sizeof(T) == 2) {
+                kv[0] = bf16lo(u[uu].x); kv[1] = bf16hi(u[uu].x); kv[2] = bf16lo(u[uu].y);
+                kv[3] = bf16hi(u[uu].y); kv[4] = bf16lo(u[uu].z); kv[5] = bf16hi(u[uu].z);
+                kv[6] = bf16lo(u[uu].w); kv[7] = bf16hi(u[uu].w);
+            } else {
+                kv[0] = __uint_as_float(u[uu].x); kv[1] = __uint_as_float(u[uu].y);
+                kv[2] = __uint_as_float(u[uu].z); kv[3] = __uint_as_float(u[uu].w);
+            }
+            float sdot = 0.f;
+#pragma unroll
+            for (int e = 0; e < V; ++e) sdot = fmaf(qv[e], kv[e], sdot);
+#pragma unroll
+            for (int o = LPK / 2; o > 0; o >>= 1) sdot += __shfl_xor_sync(0xffffffffu, sdot, o);
+            const int x = x0 + uu * KPW + sub;
+            if (cl == 0 && x < n) keys[x] = ((uint64_t)order_desc(sdot) << 32) | (uint32_t)x;
+        }
     }
     for (int x = n + tid; x < sort_cap; x += kThreads) keys[x] = ~0ull;
     __syncthreads();
