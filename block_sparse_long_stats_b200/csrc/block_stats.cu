@@ -3,12 +3,18 @@
 // Modeling", section 2.1: first- and second-order block statistics, covariance
 // approximated as diagonal).
 //
-// HBM-bound: every key is read once with 16-byte loads. A CTA takes a tile of 128
-// key rows (128 / block whole blocks). Warp w owns the 16-byte column chunks 2w and
-// 2w+1; inside a warp, lane = (chunk, row group rg), and a lane holds rows
-// rg, rg+16, ..., rg+112 of the tile in registers. Both passes (sum, then the sum
-// of squared deviations from the block mean) run on those registers and reduce
-// over the 16 row groups with half-warp shuffles: no shared memory.
+// HBM-bound: every key is read once with 16-byte loads. A warp load covers
+// RPL = 512 / row_bytes consecutive rows (lane = (row rp, 16-byte column chunk cl));
+// a chunk of R such loads (16 rows for bf16 d = 128) sits in registers, its mean
+// and sum of squared deviations are taken two-pass there and reduced over the rp
+// lanes with xor shuffles. Chunks are combined by exact moment merging of
+// (n, mean, M2): inside a warp in registers (Chan et al.'s pairwise update), across
+// the warps that share a block through shared memory (total mean first, then
+// M2 = sum of M2_p + n_p (mean_p - mean)^2). CTAs are persistent and walk tiles of 8 warps'
+// worth of chunks; every warp issues the loads of its next chunk before it reduces
+// the current one, so two chunks per warp are in flight.
+#include <algorithm>
+
 #include "kernels.h"
 
 namespace spa {
@@ -33,139 +39,205 @@ struct Elem<float> {
     }
 };
 
-// Sums K values (K a power of two <= 16) over the 16 lanes of a half-warp by
-// halving: at each xor offset (8, 4, ...) a lane keeps half of its values and adds
-// its partner's copy of them. Lane rg ends with the total of value rg >> (4 - log2 K).
-template <int K>
-__device__ __forceinline__ float halfwarp_reduce_transpose(float (&v)[K], int rg) {
-    constexpr int LK = K >= 16 ? 4 : K >= 8 ? 3 : K >= 4 ? 2 : K >= 2 ? 1 : 0;
-    float w[K];
+constexpr int kThreads = 256;
+constexpr int kCtasPerSm = 2;
+
+template <typename T, int D, int BLOCK>
+struct StatsShape {
+    static constexpr int V = Elem<T>::kPerChunk;           // values per 16-byte chunk
+    static constexpr int LPR = D / V;                      // lanes per row
+    static constexpr int RPL = 32 / LPR;                   // rows per warp load
+    static constexpr int R = BLOCK / RPL < 8 ? BLOCK / RPL : 8;   // loads per lane per chunk
+    static constexpr int CR = R * RPL;                     // rows per chunk
+    static constexpr int NC = BLOCK / CR;                  // chunks per block
+    static_assert(LPR >= 1 && LPR <= 32 && CR * NC == BLOCK, "unsupported shape");
+};
+
+// (n_a, mu_a, m2_a) <- merge with (n_b, mu_b, m2_b); exact when n_a = 0
+template <int V>
+__device__ __forceinline__ void chan_merge(float &n_a, float (&mu_a)[V], float (&m2_a)[V], float n_b,
+                                           const float (&mu_b)[V], const float (&m2_b)[V]) {
+    if (!(n_b > 0.f)) return;
+    const float n = n_a + n_b, f = n_b / n, g = n_a * f;
 #pragma unroll
-    for (int k = 0; k < K; ++k) w[k] = v[k];
-#pragma unroll
-    for (int st = 0; st < LK; ++st) {
-        const int off = 8 >> st;
-        const int half = K >> (st + 1);
-        const bool upper = (rg & off) != 0;
-#pragma unroll
-        for (int k = 0; k < half; ++k) {
-            const float send = upper ? w[k] : w[k + half];
-            const float keep = upper ? w[k + half] : w[k];
-            w[k] = keep + __shfl_xor_sync(0xffffffffu, send, off);
-        }
+    for (int v = 0; v < V; ++v) {
+        const float delta = mu_b[v] - mu_a[v];
+        mu_a[v] = fmaf(delta, f, mu_a[v]);
+        m2_a[v] = m2_a[v] + m2_b[v] + delta * delta * g;
     }
-    float t = w[0];
-#pragma unroll
-    for (int off = 8 >> LK; off > 0; off >>= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
-    return t;
+    n_a = n;
 }
 
-constexpr int kTileRows = 128;
-constexpr int kRowGroups = 16;
-constexpr int kRowsPerLane = kTileRows / kRowGroups;  // 8
+template <typename T, int D, int BLOCK>
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+block_stats_kernel(const T *__restrict__ k, int T_len, int nb, int blk_begin, int nblk, int units,
+                   float *__restrict__ mean, float *__restrict__ var) {
+    using S = StatsShape<T, D, BLOCK>;
+    constexpr int V = S::V, LPR = S::LPR, RPL = S::RPL, R = S::R, CR = S::CR, NC = S::NC;
+    constexpr int kWarps = kThreads / 32;
+    constexpr int SPW = NC > kWarps ? NC / kWarps : 1;    // chunks per warp per tile
+    constexpr int WPB = NC / SPW;                         // warps per block
+    constexpr int BPT = kWarps / WPB;                     // blocks per tile
+    constexpr int PB = WPB > 1 ? 2 : 1;                   // partial buffers (double-buffered)
+    __shared__ float part_mu[PB][kWarps][WPB > 1 ? D : 1];
+    __shared__ float part_m2[PB][kWarps][WPB > 1 ? D : 1];
+    __shared__ float part_n[PB][kWarps];
+    const int lane = threadIdx.x & 31, wi = threadIdx.x >> 5;
+    const int rp = lane / LPR, cl = lane % LPR;
+    const int tiles = (units + BPT - 1) / BPT;
 
-template <typename T, int BLOCK>
-__global__ void __launch_bounds__(512) block_stats_kernel(const T *__restrict__ k, int T_len,
-                                                          int d, int nb, int blk_begin,
-                                                          int blk_end, float *__restrict__ mean,
-                                                          float *__restrict__ var) {
-    constexpr int V = Elem<T>::kPerChunk;
-    constexpr int NBT = kTileRows / BLOCK;          // blocks per tile
-    constexpr int MPB = BLOCK / kRowGroups;         // rows per lane per block
-    const int lane = threadIdx.x & 31;
-    const int warp = threadIdx.x >> 5;
-    const int rg = lane & 15;
-    const int chunk = 2 * warp + (lane >> 4);
-    const int bg = blockIdx.y;
-    const int row0 = blk_begin * BLOCK + blockIdx.x * kTileRows;   // first row of the tile
-    const int row_end = min(T_len, blk_end * BLOCK);
-
-    const size_t row_bytes = (size_t)d * sizeof(T);
-    const char *base = reinterpret_cast<const char *>(k) + (size_t)bg * T_len * row_bytes +
-                       (size_t)chunk * 16;
-
-    uint4 raw[kRowsPerLane];
-    unsigned valid = 0;
+    // block of this warp in tile t, and the first row of its chunk s
+    auto unit_of = [&](int t) { return t * BPT + wi / WPB; };
+    auto first_row = [&](int u, int sc) {
+        return (blk_begin + u % nblk) * BLOCK + ((wi % WPB) * SPW + sc) * CR;
+    };
+    auto load = [&](uint4 (&raw)[R], int u, int sc) {
+        const int first = first_row(u, sc);
+        const uint4 *src =
+            reinterpret_cast<const uint4 *>(k + ((size_t)(u / nblk) * T_len + first) * D) + cl;
 #pragma unroll
-    for (int m = 0; m < kRowsPerLane; ++m) {
-        const int row = row0 + rg + kRowGroups * m;
-        if (row < row_end) {
-            raw[m] = __ldg(reinterpret_cast<const uint4 *>(base + (size_t)row * row_bytes));
-            valid |= 1u << m;
-        } else {
-            raw[m] = make_uint4(0, 0, 0, 0);
+        for (int i = 0; i < R; ++i) {
+            const int r = i * RPL + rp;
+            raw[i] = first + r < T_len ? __ldg(src + (size_t)r * LPR) : make_uint4(0, 0, 0, 0);
         }
-    }
+    };
 
+    int t = blockIdx.x, sc = 0, buf = 0;
+    uint4 raw[R];
+    if (t < tiles && unit_of(t) < units) load(raw, unit_of(t), 0);
+    float n_a = 0.f, mu_a[V], m2_a[V];
 #pragma unroll
-    for (int lb = 0; lb < NBT; ++lb) {
-        const int j = row0 / BLOCK + lb;
-        const int n = min(BLOCK, row_end - j * BLOCK);
-        if (n <= 0 || j >= blk_end) break;      // uniform across the CTA
-        float s[V];
+    for (int v = 0; v < V; ++v) mu_a[v] = m2_a[v] = 0.f;
+
+    while (t < tiles) {                   // uniform across the CTA
+        int nt = t, nsc = sc + 1;
+        if (nsc == SPW) { nt = t + gridDim.x; nsc = 0; }
+        uint4 nraw[R];
+        if (nt < tiles && unit_of(nt) < units) load(nraw, unit_of(nt), nsc);
+
+        const int u = unit_of(t);
+        const int nv = u < units ? max(0, min(CR, T_len - first_row(u, sc))) : 0;
+        if (nv > 0) {
+            float s[V];
 #pragma unroll
-        for (int v = 0; v < V; ++v) s[v] = 0.f;
+            for (int v = 0; v < V; ++v) s[v] = 0.f;
 #pragma unroll
-        for (int mm = 0; mm < MPB; ++mm) {
-            float x[V];
-            Elem<T>::unpack(raw[lb * MPB + mm], x);
+            for (int i = 0; i < R; ++i) {      // rows past the end were loaded as zeros
+                float x[V];
+                Elem<T>::unpack(raw[i], x);
 #pragma unroll
-            for (int v = 0; v < V; ++v) s[v] += x[v];
-        }
-        // Column totals (lane rg holds column rg / (16 / V)), then every lane gets
-        // all V means back.
-        constexpr int LPV = 16 / V;                      // lanes per value
-        const float inv_n = 1.0f / (float)n;
-        const float mean_own = halfwarp_reduce_transpose<V>(s, rg) * inv_n;
-        const int hbase = lane & 16;                     // this half-warp's first lane
-        float mu[V];
+                for (int v = 0; v < V; ++v) s[v] += x[v];
+            }
 #pragma unroll
-        for (int v = 0; v < V; ++v) mu[v] = __shfl_sync(0xffffffffu, mean_own, hbase + v * LPV);
+            for (int o = LPR; o < 32; o <<= 1)
 #pragma unroll
-        for (int v = 0; v < V; ++v) s[v] = 0.f;
+                for (int v = 0; v < V; ++v) s[v] += __shfl_xor_sync(0xffffffffu, s[v], o);
+            const float inv = 1.0f / (float)nv;
+            float mu_b[V], m2_b[V];
 #pragma unroll
-        for (int mm = 0; mm < MPB; ++mm) {
-            const int m = lb * MPB + mm;
-            float x[V];
-            Elem<T>::unpack(raw[m], x);
-            if (valid & (1u << m)) {
+            for (int v = 0; v < V; ++v) { mu_b[v] = s[v] * inv; m2_b[v] = 0.f; }
 #pragma unroll
-                for (int v = 0; v < V; ++v) {
-                    const float dv = x[v] - mu[v];
-                    s[v] = fmaf(dv, dv, s[v]);
+            for (int i = 0; i < R; ++i) {
+                if (i * RPL + rp < nv) {
+                    float x[V];
+                    Elem<T>::unpack(raw[i], x);
+#pragma unroll
+                    for (int v = 0; v < V; ++v) {
+                        const float dv = x[v] - mu_b[v];
+                        m2_b[v] = fmaf(dv, dv, m2_b[v]);
+                    }
                 }
             }
+#pragma unroll
+            for (int o = LPR; o < 32; o <<= 1)
+#pragma unroll
+                for (int v = 0; v < V; ++v) m2_b[v] += __shfl_xor_sync(0xffffffffu, m2_b[v], o);
+            chan_merge<V>(n_a, mu_a, m2_a, (float)nv, mu_b, m2_b);
         }
-        const float var_own = halfwarp_reduce_transpose<V>(s, rg) * inv_n;
-        if ((rg & (LPV - 1)) == 0) {
-            const size_t o = ((size_t)bg * nb + j) * d + (size_t)chunk * V + rg / LPV;
-            mean[o] = mean_own;
-            var[o] = var_own;
+        if (sc == SPW - 1) {
+            const int j = blk_begin + u % nblk;
+            if constexpr (WPB == 1) {
+                if (u < units && rp == 0) {
+                    const size_t o = ((size_t)(u / nblk) * nb + j) * D + (size_t)cl * V;
+                    const float inv_n = 1.0f / n_a;
+#pragma unroll
+                    for (int v = 0; v < V; v += 4) {
+                        *reinterpret_cast<float4 *>(mean + o + v) =
+                            make_float4(mu_a[v], mu_a[v + 1], mu_a[v + 2], mu_a[v + 3]);
+                        *reinterpret_cast<float4 *>(var + o + v) =
+                            make_float4(m2_a[v] * inv_n, m2_a[v + 1] * inv_n,
+                                        m2_a[v + 2] * inv_n, m2_a[v + 3] * inv_n);
+                    }
+                }
+            } else {
+                if (rp == 0) {
+#pragma unroll
+                    for (int v = 0; v < V; ++v) {
+                        part_mu[buf][wi][cl * V + v] = mu_a[v];
+                        part_m2[buf][wi][cl * V + v] = m2_a[v];
+                    }
+                }
+                if (lane == 0) part_n[buf][wi] = n_a;
+                __syncthreads();
+                // all threads merge: (block bt of the tile, column col) per thread;
+                // N = sum n_p, mean = sum n_p mu_p / N, M2 = sum M2_p + n_p (mu_p - mean)^2
+                for (int x = threadIdx.x; x < BPT * D; x += kThreads) {
+                    const int bt = x / D, col = x % D, ub = t * BPT + bt;
+                    if (ub >= units) break;
+                    float nn = 0.f, sm = 0.f;
+#pragma unroll
+                    for (int p = 0; p < WPB; ++p) {
+                        const float np_ = part_n[buf][bt * WPB + p];
+                        nn += np_;
+                        sm = fmaf(np_, part_mu[buf][bt * WPB + p][col], sm);
+                    }
+                    const float inv_n = 1.0f / nn, mu = sm * inv_n;
+                    float m2 = 0.f;
+#pragma unroll
+                    for (int p = 0; p < WPB; ++p) {
+                        const float dm = part_mu[buf][bt * WPB + p][col] - mu;
+                        m2 += fmaf(part_n[buf][bt * WPB + p] * dm, dm, part_m2[buf][bt * WPB + p][col]);
+                    }
+                    const size_t o = ((size_t)(ub / nblk) * nb + blk_begin + ub % nblk) * D + col;
+                    mean[o] = mu;
+                    var[o] = m2 * inv_n;
+                }
+                buf ^= 1;
+            }
+            n_a = 0.f;
+#pragma unroll
+            for (int v = 0; v < V; ++v) mu_a[v] = m2_a[v] = 0.f;
         }
+#pragma unroll
+        for (int i = 0; i < R; ++i) raw[i] = nraw[i];
+        t = nt;
+        sc = nsc;
     }
 }
 
-template <typename T, int BLOCK>
-cudaError_t launch_t(const void *k, int B, int Hkv, int T_len, int d, int blk_begin, int blk_end,
+template <typename T, int D, int BLOCK>
+cudaError_t launch_t(const void *k, int B, int Hkv, int T_len, int blk_begin, int blk_end,
                      float *mean, float *var, cudaStream_t s) {
-    const int nb = (T_len + BLOCK - 1) / BLOCK;
-    const int chunks = d * (int)sizeof(T) / 16;
-    dim3 block(chunks / 2 * 32);
-    dim3 grid((unsigned)(((blk_end - blk_begin) * BLOCK + kTileRows - 1) / kTileRows),
-              (unsigned)(B * Hkv));
-    block_stats_kernel<T, BLOCK><<<grid, block, 0, s>>>(reinterpret_cast<const T *>(k), T_len,
-                                                        d, nb, blk_begin, blk_end, mean, var);
+    const int nb = (T_len + BLOCK - 1) / BLOCK, nblk = blk_end - blk_begin;
+    const int units = B * Hkv * nblk;
+    using S = StatsShape<T, D, BLOCK>;
+    constexpr int SPW = S::NC > kThreads / 32 ? S::NC / (kThreads / 32) : 1;
+    constexpr int BPT = (kThreads / 32) / (S::NC / SPW);   // blocks per tile
+    const int tiles = (units + BPT - 1) / BPT;
+    const unsigned grid = (unsigned)std::min(tiles, 148 * kCtasPerSm);
+    block_stats_kernel<T, D, BLOCK><<<grid, kThreads, 0, s>>>(
+        reinterpret_cast<const T *>(k), T_len, nb, blk_begin, nblk, units, mean, var);
     return cudaGetLastError();
 }
 
-template <typename T>
-cudaError_t launch_block(const void *k, int B, int Hkv, int T_len, int d, int block,
-                         int blk_begin, int blk_end, float *mean, float *var, cudaStream_t s) {
+template <typename T, int D>
+cudaError_t launch_block(const void *k, int B, int Hkv, int T_len, int block, int blk_begin,
+                         int blk_end, float *mean, float *var, cudaStream_t s) {
     switch (block) {
-        case 16: return launch_t<T, 16>(k, B, Hkv, T_len, d, blk_begin, blk_end, mean, var, s);
-        case 32: return launch_t<T, 32>(k, B, Hkv, T_len, d, blk_begin, blk_end, mean, var, s);
-        case 64: return launch_t<T, 64>(k, B, Hkv, T_len, d, blk_begin, blk_end, mean, var, s);
-        default: return launch_t<T, 128>(k, B, Hkv, T_len, d, blk_begin, blk_end, mean, var, s);
+        case 16: return launch_t<T, D, 16>(k, B, Hkv, T_len, blk_begin, blk_end, mean, var, s);
+        case 32: return launch_t<T, D, 32>(k, B, Hkv, T_len, blk_begin, blk_end, mean, var, s);
+        case 64: return launch_t<T, D, 64>(k, B, Hkv, T_len, blk_begin, blk_end, mean, var, s);
+        default: return launch_t<T, D, 128>(k, B, Hkv, T_len, blk_begin, blk_end, mean, var, s);
     }
 }
 
@@ -175,9 +247,11 @@ cudaError_t launch_block_stats(const void *k, bool bf16, int B, int Hkv, int T, 
                                int blk_begin, int blk_end, float *mean, float *var,
                                cudaStream_t s) {
     if (blk_end <= blk_begin) return cudaSuccess;
-    return bf16 ? launch_block<__nv_bfloat16>(k, B, Hkv, T, d, block, blk_begin, blk_end, mean,
-                                              var, s)
-                : launch_block<float>(k, B, Hkv, T, d, block, blk_begin, blk_end, mean, var, s);
+    if (bf16)
+        return d == 128 ? launch_block<__nv_bfloat16, 128>(k, B, Hkv, T, block, blk_begin, blk_end, mean, var, s)
+                        : launch_block<__nv_bfloat16, 64>(k, B, Hkv, T, block, blk_begin, blk_end, mean, var, s);
+    return d == 128 ? launch_block<float, 128>(k, B, Hkv, T, block, blk_begin, blk_end, mean, var, s)
+                    : launch_block<float, 64>(k, B, Hkv, T, block, blk_begin, blk_end, mean, var, s);
 }
 
 }  // namespace spa

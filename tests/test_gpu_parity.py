@@ -12,7 +12,7 @@ import torch
 import oracle
 import block_sparse_long_stats_b200 as spa
 from tests._parity import compare_lists, sample_rows, to_dev, to_host
-from workloads import PARITY_WORKLOADS, WORKLOADS, generate, widen
+from workloads import PARITY_WORKLOADS, WORKLOADS, bf16_bits, generate, widen
 
 pytestmark = pytest.mark.gpu
 
@@ -61,6 +61,25 @@ def test_block_stats_match_oracle(key):
     om, ov = oracle.block_stats(x["k"], w.dtype, w.block)
     np.testing.assert_allclose(mean.cpu().numpy(), om, rtol=1e-5, atol=1e-6)
     np.testing.assert_allclose(var.cpu().numpy(), ov, rtol=1e-5, atol=1e-6)
+    assert_no_device_error()
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("block", [16, 32, 64, 128])
+def test_block_stats_every_shape_ragged_and_offset(dtype, d, block):
+    # every (dtype, d, block) kernel shape; a ragged last block (1 row, and a
+    # partial chunk), and keys 40 units off zero so that a merge of per-chunk
+    # moments that cancelled badly would miss the variance tolerance
+    rng = np.random.default_rng(1000 * block + d + (dtype == "bf16"))
+    for T in (7 * block + 1, 5 * block + block // 2 + 3):
+        k = 40.0 + rng.standard_normal((2, 3, T, d)) * rng.uniform(0.1, 2.0, (1, 3, 1, d))
+        x = bf16_bits(k) if dtype == "bf16" else k.astype(np.float32)
+        mean, var = spa.spa_block_stats(to_dev(x, dtype), block)
+        torch.cuda.synchronize()
+        om, ov = oracle.block_stats(x, dtype, block)
+        np.testing.assert_allclose(mean.cpu().numpy(), om, rtol=1e-5, atol=1e-6)
+        np.testing.assert_allclose(var.cpu().numpy(), ov, rtol=1e-5, atol=1e-6)
     assert_no_device_error()
 
 
