@@ -10,13 +10,16 @@
 //
 // One CTA (256 threads) per (b, query head, query block). The residual candidates
 // are the contiguous range [r_lo, r_hi) of block indices between the sink prefix
-// and the local suffix, so only those are scored. Scores are fp32 (warp per
-// candidate, 128-bit loads of the block statistics, shuffle reductions). They are
+// and the local suffix, so only those are scored. Scores are fp32 (a warp scores
+// four candidates per step from 128-bit loads of the block statistics, their eight
+// partial sums reduced together by one transposing shuffle reduction). They are
 // packed with the block index into 64-bit keys that sort ascending in the order
-// (score descending, index ascending) and sorted with a shared-memory bitonic
-// network. Masses and their exclusive prefix sums are fp64, so the cut is decided
-// on fp32 scores with no further rounding in the masses. The kept set is written
-// as an ascending list by a prefix scan over per-block flags.
+// (score descending, index ascending). Up to 256 keys are sorted by a bitonic
+// network in one warp's registers (strides below the keys per lane in registers,
+// the rest by shuffles), more by a shared-memory bitonic network. Masses and their
+// exclusive prefix sums are fp64, so the cut is decided on fp32 scores with no
+// further rounding in the masses. The kept set is written as an ascending list by
+// a prefix scan over per-block flags.
 #include <float.h>
 
 #include "kernels.h"
@@ -70,8 +73,8 @@ __device__ V block_exclusive_scan(V x, V *warp_tot, V *total) {
 
 // Log Taylor score of one candidate from one lane's PL components of the pooled
 // query (qv, its squares q2) and of the block's mean and variance: per-lane fused
-// multiply-adds, then an xor-shuffle tree across the warp. Both selection paths
-// use this exact order, so their scores agree to the bit.
+// multiply-adds, then the xor-shuffle tree of reduce_transpose across the warp.
+// Prefill and decode scoring use this exact order, so their scores agree to the bit.
 template <int PL>
 __device__ __forceinline__ void lane_partials(const float (&qv)[PL], const float (&q2)[PL],
                                               const float (&mu)[PL], const float (&vr)[PL],
@@ -83,11 +86,6 @@ __device__ __forceinline__ void lane_partials(const float (&qv)[PL], const float
         dot = fmaf(qv[c], mu[c], dot);
         quad = fmaf(q2[c], vr[c], quad);
     }
-}
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    return v;
 }
 __device__ __forceinline__ float log_score(float dot, float quad, float scale, float hs2, int nj) {
     return scale * dot + log1pf(hs2 * quad) + logf((float)nj);
@@ -163,6 +161,43 @@ __device__ __forceinline__ float reduce_transpose(float (&v)[K], int lane) {
     return t;
 }
 
+// Sorts N = 32 KPL 64-bit keys ascending inside one warp, lane-major (lane l holds
+// positions KPL l .. KPL l + KPL - 1): a bitonic network whose strides below KPL
+// are compare-exchanges in registers and whose larger strides are xor shuffles.
+// No shared memory and no barriers.
+template <int KPL>
+__device__ __forceinline__ void warp_bitonic_sort(uint64_t (&k)[KPL], int lane) {
+    constexpr int N = 32 * KPL;
+#pragma unroll
+    for (int kk = 2; kk <= N; kk <<= 1) {
+#pragma unroll
+        for (int jj = kk >> 1; jj > 0; jj >>= 1) {
+            if (jj < KPL) {
+#pragma unroll
+                for (int e = 0; e < KPL; ++e) {
+                    if ((e & jj) == 0) {
+                        const bool up = ((lane * KPL + e) & kk) == 0;
+                        const uint64_t x = k[e], y = k[e | jj];
+                        const bool sw = (x > y) == up;
+                        k[e] = sw ? y : x;
+                        k[e | jj] = sw ? x : y;
+                    }
+                }
+            } else {
+                const int lm = jj / KPL;                  // partner lane = lane ^ lm
+                const bool lower = (lane & lm) == 0;
+#pragma unroll
+                for (int e = 0; e < KPL; ++e) {
+                    const bool up = ((lane * KPL + e) & kk) == 0;
+                    const uint64_t o = __shfl_xor_sync(0xffffffffu, k[e], lm);
+                    const uint64_t mn = k[e] < o ? k[e] : o, mx = k[e] < o ? o : k[e];
+                    k[e] = lower == up ? mn : mx;
+                }
+            }
+        }
+    }
+}
+
 struct SelectArgs {
     const void *q;
     const float *mean;
@@ -185,13 +220,92 @@ struct SelectArgs {
     int seg_blocks;
 };
 
+constexpr int kWarpSortMax = 256;   // residuals up to this many: sort in one warp
+
+// Up to 32 KPL residual keys (keys[0, nres) in shared memory) sorted in one warp's
+// registers, then the cut: a key is kept while the fp64 mass ranked before it,
+// over the total, is below top_p (the masses are exp(score - max score)); then the
+// K_min floor. Writes the kept blocks' flags, or in traversal order the whole list
+// (local blocks from the own one down, sink blocks, kept residual blocks by rank).
+template <int KPL>
+__device__ __forceinline__ void warp_sort_cut(const uint64_t *keys, unsigned char *flag,
+                                           const SelectArgs &a, size_t unit, int nres, int r_lo,
+                                           int r_hi, int jmax, int lane) {
+    uint64_t k[KPL];
+#pragma unroll
+    for (int e = 0; e < KPL; ++e) {
+        const int x = lane * KPL + e;
+        k[e] = x < nres ? keys[x] : ~0ull;
+    }
+    warp_bitonic_sort<KPL>(k, lane);
+    int nk = nres;
+    if (nres > 0 && a.top_p < 1.0f) {
+        const double mx = (double)key_score(__shfl_sync(0xffffffffu, k[0], 0));
+        double m[KPL], local = 0.0;
+#pragma unroll
+        for (int e = 0; e < KPL; ++e) {
+            m[e] = lane * KPL + e < nres ? exp((double)key_score(k[e]) - mx) : 0.0;
+            local += m[e];
+        }
+        double inc = local;            // inclusive scan over lanes
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const double y = __shfl_up_sync(0xffffffffu, inc, o);
+            if (lane >= o) inc += y;
+        }
+        const double total = __shfl_sync(0xffffffffu, inc, 31);
+        const double prev = __shfl_up_sync(0xffffffffu, inc, 1);
+        double cum = lane == 0 ? 0.0 : prev;
+        const double p = (double)a.top_p;
+        int kept = 0;
+#pragma unroll
+        for (int e = 0; e < KPL; ++e) {
+            if (lane * KPL + e < nres && cum / total < p) ++kept;
+            cum += m[e];
+        }
+        nk = (int)__reduce_add_sync(0xffffffffu, (unsigned)kept);
+    }
+    nk = max(nk, min(a.k_min, nres));
+    if (a.score_order) {
+        int32_t *out = a.idx + unit * a.cap;
+        const int nloc = jmax + 1 - r_hi;
+        for (int x = lane; x < nloc; x += 32) out[x] = jmax - x;
+        for (int x = lane; x < r_lo; x += 32) out[nloc + x] = x;
+#pragma unroll
+        for (int e = 0; e < KPL; ++e) {
+            const int x = lane * KPL + e;
+            if (x < nk) out[nloc + r_lo + x] = (int)(uint32_t)k[e];
+        }
+        if (lane == 0) a.count[unit] = nloc + r_lo + nk;
+    } else {
+#pragma unroll
+        for (int e = 0; e < KPL; ++e)
+            if (lane * KPL + e < nk) flag[(int)(uint32_t)k[e]] = 1;
+    }
+}
+
+// The flagged blocks 0..jmax as an ascending list (block-wide scan over flags).
+__device__ __forceinline__ void write_ascending(const unsigned char *flag, const SelectArgs &a,
+                                                size_t unit, int jmax, int *itot, int *isum) {
+    const int tid = threadIdx.x;
+    const int n = jmax + 1;
+    const int per = (n + kThreads - 1) / kThreads;
+    const int s0 = min(tid * per, n), s1 = min(s0 + per, n);
+    int c = 0;
+    for (int j = s0; j < s1; ++j) c += flag[j];
+    int pos = block_exclusive_scan<int>(c, itot, isum);
+    int32_t *out = a.idx + unit * a.cap;
+    for (int j = s0; j < s1; ++j)
+        if (flag[j]) out[pos++] = j;
+    if (tid == 0) a.count[unit] = *isum;
+}
+
 template <typename T, int D, bool QS>
 __global__ void __launch_bounds__(kThreads) select_kernel(SelectArgs a) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     uint64_t *keys = reinterpret_cast<uint64_t *>(smem_raw);               // [sort_cap]
-    // [kThreads * 8] pooling buffer, absent when the scores come precomputed
-    float *red = reinterpret_cast<float *>(keys + a.sort_cap);
-    unsigned char *flag = reinterpret_cast<unsigned char *>(red + (a.prescored ? 0 : kThreads * 8)); // [nb]
+    float *red = reinterpret_cast<float *>(keys + a.sort_cap);              // [kThreads * 8]
+    unsigned char *flag = reinterpret_cast<unsigned char *>(red + kThreads * 8); // [nb]
     __shared__ double dtot[kWarps];
     __shared__ double dsum;
     __shared__ int itot[kWarps];
@@ -206,7 +320,7 @@ __global__ void __launch_bounds__(kThreads) select_kernel(SelectArgs a) {
     const size_t unit = (size_t)bh * a.nq + i;
 
     // ---- pooled query: mean of the rows of query block i
-    if (!a.prescored) {
+    {
         constexpr int V = 16 / sizeof(T);
         constexpr int CPR = D / V;             // 16-byte chunks per row
         constexpr int RG = kThreads / CPR;     // row groups
@@ -248,15 +362,13 @@ __global__ void __launch_bounds__(kThreads) select_kernel(SelectArgs a) {
     int N = 1;
     while (N < nres) N <<= 1;
 
-    // ---- fp32 scores of the residual candidates, one warp per candidate
-    if (a.prescored) {
-        const float *sc = reinterpret_cast<const float *>(a.idx + unit * a.cap);
-        for (int r = tid; r < nres; r += kThreads) {
-            const int j = r_lo + r;
-            keys[r] = ((uint64_t)order_desc(sc[j]) << 32) | (uint32_t)j;
-        }
-    } else {
+    // ---- fp32 scores of the residual candidates: a warp takes U candidates per
+    // step, and the 2U partial sums (dot, variance term) of all of them go through
+    // one transposing reduction, so U scores come out on U lanes at once
+    {
         constexpr int PL = D / 32;   // components per lane
+        constexpr int U = 4, NV = 2 * U;
+        constexpr int LB = 5 - ilog2(NV);           // lanes per value = 2^LB
         float qv[PL], q2[PL];
 #pragma unroll
         for (int c = 0; c < PL; ++c) {
@@ -271,28 +383,52 @@ __global__ void __launch_bounds__(kThreads) select_kernel(SelectArgs a) {
         const int seg0 = a.seg_blocks > 0 ? (i / a.seg_blocks) * a.seg_blocks : 0;
         const float *mbp = a.seg_blocks > 0 ? a.mean_p + bgo * D + lane * PL : nullptr;
         const float *vbp = a.seg_blocks > 0 ? a.var_p + bgo * D + lane * PL : nullptr;
-        for (int r = warp; r < nres; r += kWarps) {
-            const int j = r_lo + r;
-            float mu[PL], vr[PL], dot, quad;
-            if constexpr (QS)
-                load_stats_q<D>(qb + (size_t)j * (D + D / 16), lane, mu, vr);
-            else if (j < seg0)
-                load_stats<PL>(mbp + (size_t)j * D, vbp + (size_t)j * D, mu, vr);
-            else
-                load_stats<PL>(mb + (size_t)j * D, vb + (size_t)j * D, mu, vr);
-            lane_partials<PL>(qv, q2, mu, vr, dot, quad);
-            dot = warp_sum(dot);
-            quad = warp_sum(quad);
-            if (lane == 0) {
-                const float l = log_score(dot, quad, a.scale, hs2, min(a.block, a.T - j * a.block));
+        const int vi = lane >> LB;                  // value this lane's group ends with
+        for (int r0 = warp * U; r0 < nres; r0 += kWarps * U) {
+            float mu[U][PL], vr[U][PL];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int j = r_lo + min(r0 + u, nres - 1);   // past the end: a repeat, unused
+                if constexpr (QS)
+                    load_stats_q<D>(qb + (size_t)j * (D + D / 16), lane, mu[u], vr[u]);
+                else if (j < seg0)
+                    load_stats<PL>(mbp + (size_t)j * D, vbp + (size_t)j * D, mu[u], vr[u]);
+                else
+                    load_stats<PL>(mb + (size_t)j * D, vb + (size_t)j * D, mu[u], vr[u]);
+            }
+            // value 2u is candidate u's dot, value 2u + 1 its variance term
+            float v[NV];
+#pragma unroll
+            for (int u = 0; u < U; ++u) lane_partials<PL>(qv, q2, mu[u], vr[u], v[2 * u], v[2 * u + 1]);
+            const float tot = reduce_transpose<NV>(v, lane);
+            const float quad = __shfl_sync(0xffffffffu, tot, (lane + (1 << LB)) & 31);
+            const int r = r0 + (vi >> 1);
+            if ((vi & 1) == 0 && (lane & ((1 << LB) - 1)) == 0 && r < nres) {
+                const int j = r_lo + r;
+                const float l = log_score(tot, quad, a.scale, hs2, min(a.block, a.T - j * a.block));
                 keys[r] = ((uint64_t)order_desc(l) << 32) | (uint32_t)j;
             }
         }
     }
-    for (int r = nres + tid; r < N; r += kThreads) keys[r] = ~0ull;
+    if (N > kWarpSortMax)
+        for (int r = nres + tid; r < N; r += kThreads) keys[r] = ~0ull;
     for (int j = tid; j <= jmax; j += kThreads)
         flag[j] = (j < r_lo || j >= r_hi) ? 1 : 0;     // reserved blocks
-    __syncthreads();   // (prescored: every score is read before the list overwrites them)
+    __syncthreads();
+
+    if (N <= kWarpSortMax) {
+        // ---- up to 256 candidates: sort and cut in warp 0's registers
+        if (warp == 0) {
+            if (N <= 32) warp_sort_cut<1>(keys, flag, a, unit, nres, r_lo, r_hi, jmax, lane);
+            else if (N <= 64) warp_sort_cut<2>(keys, flag, a, unit, nres, r_lo, r_hi, jmax, lane);
+            else if (N <= 128) warp_sort_cut<4>(keys, flag, a, unit, nres, r_lo, r_hi, jmax, lane);
+            else warp_sort_cut<8>(keys, flag, a, unit, nres, r_lo, r_hi, jmax, lane);
+        }
+        if (a.score_order) return;      // warp 0 wrote the traversal-order list
+        __syncthreads();
+        write_ascending(flag, a, unit, jmax, itot, &isum);
+        return;
+    }
 
     // ---- bitonic sort, ascending keys = descending score, ascending index.
     // Pair p of a stage compares x = (p / jj) * 2jj + p % jj with x + jj (shifts:
@@ -364,19 +500,171 @@ __global__ void __launch_bounds__(kThreads) select_kernel(SelectArgs a) {
     }
     for (int x = tid; x < nk; x += kThreads) flag[(int)(uint32_t)keys[x]] = 1;
     __syncthreads();
+    write_ascending(flag, a, unit, jmax, itot, &isum);
+}
 
-    // ---- ascending list of the kept blocks
+// Grouped prefill selection: one CTA (256 threads) per (b, kv-head g, query block)
+// serves the G query heads of the group, so every candidate's statistics are read
+// once for all of them. Same rule and arithmetic as select_kernel: fp32 pooled
+// queries (each head's rows summed in row groups, the partials added in order),
+// the scores from lane_partials + reduce_transpose (U candidates x G heads per
+// reduction, as in decode scoring), then warp h sorts and cuts head h's keys in
+// registers and writes head h's list, with no block-wide barrier after the scoring.
+template <typename T, int D, int G, bool QS>
+__global__ void __launch_bounds__(kThreads, 3) select_group_kernel(SelectArgs a) {
+    constexpr int PL = D / 32;
+    constexpr int U = G >= 8 ? 2 : (G == 4 ? 4 : 8);
+    constexpr int NV = 2 * G * U;                   // values per reduction (<= 32)
+    constexpr int LB = 5 - ilog2(NV);               // lanes per value = 2^LB
+    constexpr int V = 16 / sizeof(T);
+    constexpr int CPR = D / V;                      // 16-byte chunks per row
+    constexpr int TPH = kThreads / G;               // pooling threads per head
+    constexpr int RG = TPH / CPR;                   // row groups per head
+    static_assert(RG >= 1, "pooling layout");
+    __shared__ float qs[G][D];
+    __shared__ float red[G][RG][D];
+    __shared__ uint64_t keys[G][kWarpSortMax];
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    unsigned char *flags = smem_raw;                // [G][nb]
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int i = a.nq - 1 - (int)blockIdx.x;       // heaviest query blocks first
+    const int bg = blockIdx.y, b = bg / a.Hkv, g = bg % a.Hkv;
+
+    // ---- pooled queries of the G heads (thread (head, row group, chunk))
     {
-        const int n = jmax + 1;
-        const int per = (n + kThreads - 1) / kThreads;
-        const int s0 = min(tid * per, n), s1 = min(s0 + per, n);
-        int c = 0;
-        for (int j = s0; j < s1; ++j) c += flag[j];
-        int pos = block_exclusive_scan<int>(c, itot, &isum);
-        int32_t *out = a.idx + unit * a.cap;
-        for (int j = s0; j < s1; ++j)
-            if (flag[j]) out[pos++] = j;
-        if (tid == 0) a.count[unit] = isum;
+        const int hh = tid / TPH, c = (tid % TPH) % CPR, rg = (tid % TPH) / CPR;
+        const int r0 = i * a.block, nr = min(a.block, a.Lq - r0);
+        float acc[V];
+#pragma unroll
+        for (int v = 0; v < V; ++v) acc[v] = 0.f;
+        const T *qrow = reinterpret_cast<const T *>(a.q) +
+                        ((size_t)(b * a.Hq + g * G + hh) * a.Lq + r0) * D + c * V;
+        constexpr int PF = 8;                       // loads in flight per thread
+        for (int r = rg; r < nr; r += PF * RG) {
+            uint4 u[PF];
+#pragma unroll
+            for (int p = 0; p < PF; ++p)
+                u[p] = r + p * RG < nr
+                           ? __ldg(reinterpret_cast<const uint4 *>(qrow + (size_t)(r + p * RG) * D))
+                           : make_uint4(0, 0, 0, 0);
+#pragma unroll
+            for (int p = 0; p < PF; ++p) {
+                if (r + p * RG >= nr) break;
+                if constexpr (sizeof(T) == 2) {
+                    acc[0] += bf16lo(u[p].x); acc[1] += bf16hi(u[p].x); acc[2] += bf16lo(u[p].y);
+                    acc[3] += bf16hi(u[p].y); acc[4] += bf16lo(u[p].z); acc[5] += bf16hi(u[p].z);
+                    acc[6] += bf16lo(u[p].w); acc[7] += bf16hi(u[p].w);
+                } else {
+                    acc[0] += __uint_as_float(u[p].x); acc[1] += __uint_as_float(u[p].y);
+                    acc[2] += __uint_as_float(u[p].z); acc[3] += __uint_as_float(u[p].w);
+                }
+            }
+        }
+#pragma unroll
+        for (int v = 0; v < V; ++v) red[hh][rg][c * V + v] = acc[v];
+        __syncthreads();
+        const int nrr = nr;
+        for (int x = tid; x < G * D; x += kThreads) {
+            const int h2 = x / D, cc = x % D;
+            float sm = 0.f;
+            for (int r = 0; r < RG; ++r) sm += red[h2][r][cc];
+            qs[h2][cc] = sm / (float)nrr;
+        }
+    }
+
+    // ---- candidates (the same for every head of the group)
+    const int last_row = min((i + 1) * a.block, a.Lq);
+    const int jmax = (a.T - a.Lq + last_row - 1) / a.block;
+    const int r_lo = min(a.n_sink, jmax + 1);
+    const int r_hi = max(r_lo, jmax - a.n_local + 1);
+    const int nres = r_hi - r_lo;
+    for (int x = tid; x < G * (jmax + 1); x += kThreads) {
+        const int j = x % (jmax + 1);
+        flags[(x / (jmax + 1)) * a.nb + j] = (j < r_lo || j >= r_hi) ? 1 : 0;
+    }
+    __syncthreads();
+
+    // ---- scores: U candidates x G heads per warp step
+    {
+        float qv[G][PL], q2[G][PL];
+#pragma unroll
+        for (int hh = 0; hh < G; ++hh)
+#pragma unroll
+            for (int c = 0; c < PL; ++c) {
+                qv[hh][c] = qs[hh][lane * PL + c];
+                q2[hh][c] = qv[hh][c] * qv[hh][c];
+            }
+        const float hs2 = 0.5f * a.scale * a.scale;
+        const size_t bgo = (size_t)bg * a.nb;
+        const float *mb = QS ? nullptr : a.mean + bgo * D + lane * PL;
+        const float *vb = QS ? nullptr : a.var + bgo * D + lane * PL;
+        const uint8_t *qb = QS ? a.qstats + bgo * (D + D / 16) : nullptr;
+        const int seg0 = a.seg_blocks > 0 ? (i / a.seg_blocks) * a.seg_blocks : 0;
+        const float *mbp = a.seg_blocks > 0 ? a.mean_p + bgo * D + lane * PL : nullptr;
+        const float *vbp = a.seg_blocks > 0 ? a.var_p + bgo * D + lane * PL : nullptr;
+        const int vi = lane >> LB;
+        const int uu = vi / (2 * G), kk = vi % (2 * G);   // candidate; dot (< G) or quad
+        for (int r0 = warp * U; r0 < nres; r0 += kWarps * U) {
+            float mu[U][PL], vr[U][PL];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int j = r_lo + min(r0 + u, nres - 1);   // past the end: a repeat, unused
+                if constexpr (QS)
+                    load_stats_q<D>(qb + (size_t)j * (D + D / 16), lane, mu[u], vr[u]);
+                else if (j < seg0)
+                    load_stats<PL>(mbp + (size_t)j * D, vbp + (size_t)j * D, mu[u], vr[u]);
+                else
+                    load_stats<PL>(mb + (size_t)j * D, vb + (size_t)j * D, mu[u], vr[u]);
+            }
+            float v[NV];
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+#pragma unroll
+                for (int hh = 0; hh < G; ++hh)
+                    lane_partials<PL>(qv[hh], q2[hh], mu[u], vr[u], v[u * 2 * G + hh],
+                                      v[u * 2 * G + G + hh]);
+            const float tot = reduce_transpose<NV>(v, lane);
+            const float quad = __shfl_sync(0xffffffffu, tot, (lane + (G << LB)) & 31);
+            const int r = r0 + uu;
+            if (kk < G && (lane & ((1 << LB) - 1)) == 0 && r < nres) {
+                const int j = r_lo + r;
+                const float l = log_score(tot, quad, a.scale, hs2, min(a.block, a.T - j * a.block));
+                keys[kk][r] = ((uint64_t)order_desc(l) << 32) | (uint32_t)j;
+            }
+        }
+    }
+    __syncthreads();
+
+    // ---- warp h: sort, cut and list of head h
+    if (warp < G) {
+        const int h = g * G + warp;
+        const size_t unit = ((size_t)b * a.Hq + h) * a.nq + i;
+        unsigned char *fl = flags + (size_t)warp * a.nb;
+        const int N = nres <= 32 ? 32 : nres <= 64 ? 64 : nres <= 128 ? 128 : 256;
+        if (N == 32) warp_sort_cut<1>(keys[warp], fl, a, unit, nres, r_lo, r_hi, jmax, lane);
+        else if (N == 64) warp_sort_cut<2>(keys[warp], fl, a, unit, nres, r_lo, r_hi, jmax, lane);
+        else if (N == 128) warp_sort_cut<4>(keys[warp], fl, a, unit, nres, r_lo, r_hi, jmax, lane);
+        else warp_sort_cut<8>(keys[warp], fl, a, unit, nres, r_lo, r_hi, jmax, lane);
+        if (!a.score_order) {
+            __syncwarp();
+            // ascending list: lane l takes flags [l per, (l + 1) per), warp scan of counts
+            const int n = jmax + 1, per = (n + 31) / 32;
+            const int s0 = min(lane * per, n), s1 = min(s0 + per, n);
+            int c = 0;
+            for (int j = s0; j < s1; ++j) c += fl[j];
+            int inc = c;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, inc, o);
+                if (lane >= o) inc += y;
+            }
+            int pos = inc - c;
+            int32_t *out = a.idx + unit * a.cap;
+            for (int j = s0; j < s1; ++j)
+                if (fl[j]) out[pos++] = j;
+            if (lane == 31) a.count[unit] = inc;
+        }
     }
 }
 
@@ -618,8 +906,32 @@ __global__ void __launch_bounds__(kThreads) decode_cut_kernel(SelectArgs a) {
     if (tid == 0) a.count[unit] = isum;
 }
 
+template <typename T, int D, int G, bool QS>
+cudaError_t launch_group(const SelectArgs &a, cudaStream_t s) {
+    const size_t smem = (size_t)G * a.nb;
+    auto kern = select_group_kernel<T, D, G, QS>;
+    if (smem > 16 * 1024) {
+        cudaError_t e =
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    kern<<<dim3((unsigned)a.nq, (unsigned)(a.B * a.Hkv)), kThreads, smem, s>>>(a);
+    return cudaGetLastError();
+}
+
 template <typename T, int D, bool QS>
 cudaError_t launch_tq(const SelectArgs &a, cudaStream_t s) {
+    // prefill, up to kWarpSortMax residual candidates, a head grouping the grouped
+    // kernel has: one CTA per kv-head and query block
+    if (!a.prescored && a.sort_cap <= kWarpSortMax) {
+        switch (a.G) {
+            case 1: return launch_group<T, D, 1, QS>(a, s);
+            case 2: return launch_group<T, D, 2, QS>(a, s);
+            case 4: return launch_group<T, D, 4, QS>(a, s);
+            case 8: return launch_group<T, D, 8, QS>(a, s);
+            default: break;
+        }
+    }
     const size_t smem = (size_t)a.sort_cap * 8 + (a.prescored ? 0 : kThreads * 8 * sizeof(float)) +
                         (size_t)a.nb + 16;
     auto kern = select_kernel<T, D, QS>;
