@@ -777,100 +777,211 @@ __device__ __forceinline__ V block_sum(V x, V (*buf)[kWarps], int &parity) {
 
 // Decode cut: the same rule as select_kernel's (residual blocks ranked by score
 // descending, index ascending; a block is kept while the mass ranked before it is
-// below top_p; then at least min(k_min, |residual|) blocks), found without sorting.
-// With keys kappa = (order_desc(score) << 32 | j) ascending in rank, the mass
-// ranked before a key, F(kappa), is monotone in kappa, so the kept blocks are
-// exactly the keys <= kappa*, the largest kappa with F(kappa) / total < top_p.
-// kappa* is found by bisection: 32 steps over the score word, then up to 14 over
-// the index; each step is one block-wide fp64 sum of the masses below the probe.
-// The K_min floor is the same bisection on counts. One CTA per (b, head); the
-// scores come from the unit's idx row (decode_score_kernel) and the row is then
+// below top_p; then at least min(k_min, |residual|) blocks), found without sorting
+// the whole residual. Keys kappa = (order_desc(score) << 32 | j) ascend in rank;
+// F(kappa), the mass ranked before kappa, is monotone, so the kept blocks are the
+// keys <= kappa*, the largest kappa with F(kappa) / total < top_p.
+//
+// Masses exp(score - max) are held as fixed-point integers M = rint(m 2^sh),
+// sh = 62 - ceil(log2 n) (absolute step 2^-sh, about 1e-15 at n = 8190; the sum
+// of n of them fits 63 bits), so every partial sum is exact and independent of
+// the order or the atomics that form it. Candidates are binned by score into
+// kCutBins equal-width bins between the largest and smallest score (bin index
+// monotone in kappa); the bins' mass sums, scanned, give the bin holding kappa*
+// (the last non-empty bin whose preceding mass satisfies the rule); warp 0 sorts
+// that bin's candidates (up to kWarpSortMax) in registers and finds kappa* from the
+// exact prefix. A bin with more candidates falls back to bisection over kappa, one
+// exact block-wide sum per step (32 steps over the score word, up to 14 over the
+// index). The K_min floor is the same bisection on counts. One CTA per (b, head);
+// the scores come from the unit's idx row (decode_score_kernel) and the row is then
 // overwritten with the ascending list.
+constexpr int kCutBins = 1024;
+
 __global__ void __launch_bounds__(kThreads) decode_cut_kernel(SelectArgs a) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    const int tid = threadIdx.x;
+    using u64 = unsigned long long;
+    const int tid = threadIdx.x, lane = tid & 31;
     const int unit = blockIdx.x;                     // (b, h); one query
     const int jmax = a.nb - 1;
     const int r_lo = min(a.n_sink, jmax + 1);
     const int r_hi = max(r_lo, jmax - a.n_local + 1);
     const int nres = r_hi - r_lo;
-    double *ms = reinterpret_cast<double *>(smem_raw);                 // [nb]
-    uint32_t *ord = reinterpret_cast<uint32_t *>(ms + a.nb);           // [nb]
+    uint32_t *ord = reinterpret_cast<uint32_t *>(smem_raw);                // [nb]
     unsigned char *flag = reinterpret_cast<unsigned char *>(ord + a.nb);   // [nb]
-    __shared__ double dbuf[2][kWarps];
-    __shared__ float fbuf[kWarps];
+    __shared__ u64 bins[kCutBins];
+    __shared__ uint64_t gkeys[kWarpSortMax];
+    __shared__ u64 ubuf[2][kWarps];
+    __shared__ u64 utot[kWarps];
+    __shared__ u64 usum;
+    __shared__ float fbuf[2][kWarps];
     __shared__ int ibuf[2][kWarps];
     __shared__ int itot[kWarps];
     __shared__ int isum;
-    int dpar = 0, ipar = 0;
+    __shared__ int gcount;
+    __shared__ u64 pstar;
+    __shared__ uint32_t sstar_s;
+    __shared__ int jstar_s;
+    int upar = 0, ipar = 0;
 
     const float *row = reinterpret_cast<const float *>(a.idx + (size_t)unit * a.cap);
-    float lmax = -FLT_MAX;
+    float lmax = -FLT_MAX, lmin = FLT_MAX;
     for (int r = tid; r < nres; r += kThreads) {
         const float sc = row[r_lo + r];
         ord[r] = order_desc(sc);
         lmax = fmaxf(lmax, sc);
+        lmin = fminf(lmin, sc);
     }
     for (int j = tid; j <= jmax; j += kThreads) flag[j] = (j < r_lo || j >= r_hi) ? 1 : 0;
-    // block maximum of the scores (every score is read before the row is rewritten)
+    for (int x = tid; x < kCutBins; x += kThreads) bins[x] = 0ull;
+    if (tid == 0) gcount = 0;
+    // block maximum and minimum of the scores (every score is read before the row
+    // is rewritten)
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) lmax = fmaxf(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
-    if ((tid & 31) == 0) fbuf[tid >> 5] = lmax;
-    __syncthreads();
-    float mxf = -FLT_MAX;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) mxf = fmaxf(mxf, fbuf[w]);
-    const double mx = (double)mxf;
-    double local = 0.0;
-    for (int r = tid; r < nres; r += kThreads) {
-        const double m = exp((double)score_of(ord[r]) - mx);
-        ms[r] = m;
-        local += m;
+    for (int o = 16; o > 0; o >>= 1) {
+        lmax = fmaxf(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
+        lmin = fminf(lmin, __shfl_xor_sync(0xffffffffu, lmin, o));
     }
-    const double total = block_sum<double>(local, dbuf, dpar);   // also publishes ms[]
+    if (lane == 0) { fbuf[0][tid >> 5] = lmax; fbuf[1][tid >> 5] = lmin; }
+    __syncthreads();
+    float mxf = -FLT_MAX, mnf = FLT_MAX;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) { mxf = fmaxf(mxf, fbuf[0][w]); mnf = fminf(mnf, fbuf[1][w]); }
+    const double mx = (double)mxf;
+    int lg = 0;
+    while ((1 << lg) < max(nres, 1)) ++lg;
+    const double fp_one = ldexp(1.0, 62 - lg);
+    auto mass = [&](uint32_t o) -> u64 {
+        return (u64)llrint(exp((double)score_of(o) - mx) * fp_one);
+    };
+    const float wbin = mxf > mnf ? (float)kCutBins / (mxf - mnf) : 0.f;
+    auto bin_of = [&](uint32_t o) -> int {
+        return min(kCutBins - 1, (int)((mxf - score_of(o)) * wbin));
+    };
 
     // kept <=> (ord < s_star) or (ord == s_star and j <= j_star)
     uint32_t s_star = 0xFFFFFFFFu;
     int j_star = a.nb;
     if (nres > 0 && a.top_p < 1.0f) {
         const double p = (double)a.top_p;
-        auto mass_below = [&](uint32_t s, int jj) -> double {   // F((s << 32) | jj)
-            double acc = 0.0;
-            for (int r = tid; r < nres; r += kThreads) {
-                const uint32_t o = ord[r];
-                if (o < s || (o == s && r_lo + r < jj)) acc += ms[r];
+        for (int r = tid; r < nres; r += kThreads) atomicAdd(&bins[bin_of(ord[r])], mass(ord[r]));
+        __syncthreads();
+        // exclusive scan of the bin masses; thread t owns bins [4t, 4t + 4)
+        constexpr int BPT = kCutBins / kThreads;
+        u64 own[BPT], loc = 0;
+#pragma unroll
+        for (int e = 0; e < BPT; ++e) { own[e] = bins[tid * BPT + e]; loc += own[e]; }
+        u64 pre = block_exclusive_scan<u64>(loc, utot, &usum);
+        const u64 total = usum;
+        int best = -1;
+        u64 best_pre = 0;
+#pragma unroll
+        for (int e = 0; e < BPT; ++e) {
+            if (own[e] > 0 && (double)pre / (double)total < p) { best = tid * BPT + e; best_pre = pre; }
+            pre += own[e];
+        }
+        // the largest such bin: block maximum of best
+        int bmax = best;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) bmax = max(bmax, __shfl_xor_sync(0xffffffffu, bmax, o));
+        if (lane == 0) ibuf[0][tid >> 5] = bmax;
+        __syncthreads();
+        int bs = -1;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) bs = max(bs, ibuf[0][w]);
+        if (best == bs && best >= 0) pstar = best_pre;          // one owner
+        // gather the candidates of bin bs
+        for (int r = tid; r < nres; r += kThreads) {
+            const uint32_t o = ord[r];
+            if (bin_of(o) == bs) {
+                const int pos = atomicAdd(&gcount, 1);
+                if (pos < kWarpSortMax) gkeys[pos] = ((uint64_t)o << 32) | (uint32_t)(r_lo + r);
             }
-            return block_sum<double>(acc, dbuf, dpar);
-        };
-        uint32_t lo = 0, hi = 0xFFFFFFFFu;       // F(0) = 0 < p: the predicate holds at lo
-        while (lo < hi) {
-            const uint32_t mid = (uint32_t)(lo + ((uint64_t)hi - lo + 1) / 2);
-            if (mass_below(mid, 0) / total < p) lo = mid; else hi = mid - 1;
         }
-        s_star = lo;
-        int jl = 0, jh = a.nb;
-        while (jl < jh) {
-            const int mid = jl + (jh - jl + 1) / 2;
-            if (mass_below(s_star, mid) / total < p) jl = mid; else jh = mid - 1;
+        __syncthreads();
+        const int gc = gcount;
+        if (bs < 0) {
+            // no key satisfies the rule (top_p <= 0): the top-p part keeps nothing
+            s_star = 0;
+            j_star = 0;
+        } else if (gc <= kWarpSortMax) {
+            if (tid < 32) {
+                uint64_t k[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int x = lane * 8 + e;
+                    k[e] = x < gc ? gkeys[x] : ~0ull;
+                }
+                warp_bitonic_sort<8>(k, lane);
+                u64 m[8], lsum = 0;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    m[e] = lane * 8 + e < gc ? mass((uint32_t)(k[e] >> 32)) : 0ull;
+                    lsum += m[e];
+                }
+                u64 inc = lsum;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const u64 y = __shfl_up_sync(0xffffffffu, inc, o);
+                    if (lane >= o) inc += y;
+                }
+                const u64 prev = __shfl_up_sync(0xffffffffu, inc, 1);
+                u64 cum = pstar + (lane == 0 ? 0ull : prev);
+                int cnt = 0;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    if (lane * 8 + e < gc && (double)cum / (double)total < p) ++cnt;
+                    cum += m[e];
+                }
+                const int c = (int)__reduce_add_sync(0xffffffffu, (unsigned)cnt);   // >= 1
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    if (lane * 8 + e == c - 1) {
+                        sstar_s = (uint32_t)(k[e] >> 32);
+                        jstar_s = (int)(uint32_t)k[e];
+                    }
+            }
+            __syncthreads();
+            s_star = sstar_s;
+            j_star = jstar_s;
+        } else {
+            auto mass_below = [&](uint32_t sv, int jj) -> u64 {   // F((sv << 32) | jj)
+                u64 acc = 0;
+                for (int r = tid; r < nres; r += kThreads) {
+                    const uint32_t o = ord[r];
+                    if (o < sv || (o == sv && r_lo + r < jj)) acc += mass(o);
+                }
+                return block_sum<u64>(acc, ubuf, upar);
+            };
+            uint32_t lo = 0, hi = 0xFFFFFFFFu;   // F(0) = 0 < p: the predicate holds at lo
+            while (lo < hi) {
+                const uint32_t mid = (uint32_t)(lo + ((uint64_t)hi - lo + 1) / 2);
+                if ((double)mass_below(mid, 0) / (double)total < p) lo = mid; else hi = mid - 1;
+            }
+            s_star = lo;
+            int jl = 0, jh = a.nb;
+            while (jl < jh) {
+                const int mid = jl + (jh - jl + 1) / 2;
+                if ((double)mass_below(s_star, mid) / (double)total < p) jl = mid; else jh = mid - 1;
+            }
+            j_star = jl;
         }
-        j_star = jl;
     }
-    auto kept_count = [&](uint32_t s, int jj) -> int {              // keys <= (s << 32) | jj
+    auto kept_count = [&](uint32_t sv, int jj) -> int {             // keys <= (sv << 32) | jj
         int c = 0;
         for (int r = tid; r < nres; r += kThreads) {
             const uint32_t o = ord[r];
-            c += (o < s || (o == s && r_lo + r <= jj)) ? 1 : 0;
+            c += (o < sv || (o == sv && r_lo + r <= jj)) ? 1 : 0;
         }
         return block_sum<int>(c, ibuf, ipar);
     };
     const int kfloor = min(a.k_min, nres);
     if (kfloor > 0 && kept_count(s_star, j_star) < kfloor) {
         // the kfloor smallest keys: the largest key with fewer than kfloor keys below it
-        auto below = [&](uint32_t s, int jj) -> int {               // keys < (s << 32) | jj
+        auto below = [&](uint32_t sv, int jj) -> int {              // keys < (sv << 32) | jj
             int c = 0;
             for (int r = tid; r < nres; r += kThreads) {
                 const uint32_t o = ord[r];
-                c += (o < s || (o == s && r_lo + r < jj)) ? 1 : 0;
+                c += (o < sv || (o == sv && r_lo + r < jj)) ? 1 : 0;
             }
             return block_sum<int>(c, ibuf, ipar);
         };
@@ -892,29 +1003,26 @@ __global__ void __launch_bounds__(kThreads) decode_cut_kernel(SelectArgs a) {
         if (o < s_star || (o == s_star && r_lo + r <= j_star)) flag[r_lo + r] = 1;
     }
     __syncthreads();
+    write_ascending(flag, a, (size_t)unit, jmax, itot, &isum);
+}
 
-    // ascending list of the kept blocks
-    const int n = jmax + 1;
-    const int per = (n + kThreads - 1) / kThreads;
-    const int s0 = min(tid * per, n), s1 = min(s0 + per, n);
-    int c = 0;
-    for (int j = s0; j < s1; ++j) c += flag[j];
-    int pos = block_exclusive_scan<int>(c, itot, &isum);
-    int32_t *out = a.idx + (size_t)unit * a.cap;
-    for (int j = s0; j < s1; ++j)
-        if (flag[j]) out[pos++] = j;
-    if (tid == 0) a.count[unit] = isum;
+// Opts the kernel in to dyn bytes of dynamic shared memory where its static shared
+// memory plus dyn passes the default 48 KB.
+template <typename K>
+cudaError_t allow_smem(K kern, size_t dyn) {
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, kern);
+    if (e != cudaSuccess) return e;
+    if (fa.sharedSizeBytes + dyn <= 48 * 1024) return cudaSuccess;
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
 }
 
 template <typename T, int D, int G, bool QS>
 cudaError_t launch_group(const SelectArgs &a, cudaStream_t s) {
     const size_t smem = (size_t)G * a.nb;
     auto kern = select_group_kernel<T, D, G, QS>;
-    if (smem > 16 * 1024) {
-        cudaError_t e =
-            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-    }
+    cudaError_t e = allow_smem(kern, smem);
+    if (e != cudaSuccess) return e;
     kern<<<dim3((unsigned)a.nq, (unsigned)(a.B * a.Hkv)), kThreads, smem, s>>>(a);
     return cudaGetLastError();
 }
@@ -932,26 +1040,19 @@ cudaError_t launch_tq(const SelectArgs &a, cudaStream_t s) {
             default: break;
         }
     }
-    const size_t smem = (size_t)a.sort_cap * 8 + (a.prescored ? 0 : kThreads * 8 * sizeof(float)) +
-                        (size_t)a.nb + 16;
-    auto kern = select_kernel<T, D, QS>;
-    if (smem > 48 * 1024) {
-        cudaError_t e =
-            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-    }
     if (a.prescored) {
         cudaError_t e = launch_decode_scores<T, D, QS>(a, s);
         if (e != cudaSuccess) return e;
-        const size_t csmem = (size_t)a.nb * 13 + 16;
-        if (csmem > 48 * 1024) {
-            e = cudaFuncSetAttribute(decode_cut_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)csmem);
-            if (e != cudaSuccess) return e;
-        }
+        const size_t csmem = (size_t)a.nb * 5 + 16;
+        e = allow_smem(decode_cut_kernel, csmem);
+        if (e != cudaSuccess) return e;
         decode_cut_kernel<<<(unsigned)(a.B * a.Hq), kThreads, csmem, s>>>(a);
         return cudaGetLastError();
     }
+    const size_t smem = (size_t)a.sort_cap * 8 + kThreads * 8 * sizeof(float) + (size_t)a.nb + 16;
+    auto kern = select_kernel<T, D, QS>;
+    cudaError_t e = allow_smem(kern, smem);
+    if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)((size_t)a.B * a.Hq * a.nq);
     kern<<<grid, kThreads, smem, s>>>(a);
     return cudaGetLastError();

@@ -336,6 +336,29 @@ def test_prefill_head_groupings(Hq, Hkv, block):
     assert_no_device_error()
 
 
+@pytest.mark.parametrize("outlier", [False, True])
+def test_decode_cut_dense_bin(outlier):
+    # every residual block with the same statistics: equal scores, so the cut falls
+    # in a score bin of ~600 candidates (more than one warp sorts) and the exact
+    # bisection decides; ties are kept in index order on both sides
+    w = PARITY_WORKLOADS["d_bf16_blk16"].with_(T=16 * 600, B=1, top_p=0.9)
+    x = generate(w)
+    k = np.tile(x["k"][:, :, :w.block, :], (1, 1, w.T // w.block, 1))
+    if outlier:   # one block well above the rest, still short of top_p alone
+        q = widen(x["q"], w.dtype)
+        G = w.Hq // w.Hkv
+        for g in range(w.Hkv):
+            k[0, g, 100 * w.block:101 * w.block, :] = bf16_bits(0.2 * q[0, g * G, -1, :])[None, :]
+    x = dict(x, k=np.ascontiguousarray(k))
+    dev = {n: to_dev(a, w.dtype) for n, a in x.items()}
+    r = spa.decode(dev["q"], dev["k"], dev["v"], w.block, w.top_p, scale=w.scale, k_min=w.k_min)
+    torch.cuda.synchronize()
+    sel = oracle_select(w, x)
+    res = check_lists(w, r["idx"], r["count"], sel, 1)
+    assert res["equal"] == res["units"]
+    assert_no_device_error()
+
+
 @pytest.mark.parametrize("p,k_min", [(0.9, 0), (1e-4, 0), (0.3, 200), (1.0, 0), (0.999, 0)])
 def test_decode_select_long_residual_rule_variants(p, k_min):
     # 1250 candidate blocks per head: the selection's wide (register-held) cut.
