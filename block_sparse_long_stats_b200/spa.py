@@ -15,7 +15,8 @@ import torch
 
 __all__ = ["SpaError", "lib", "spa_block_stats", "spa_select", "spa_sparse_attn_prefill",
            "spa_decode_workspace_bytes", "spa_sparse_attn_decode", "spa_get_device_error",
-           "spa_status_string", "spa_last_error", "prefill", "decode", "LIB_PATH"]
+           "spa_status_string", "spa_last_error", "prefill", "decode", "LIB_PATH",
+           "spa_prefill_host", "spa_prefill_host_workspace_bytes"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libspa.so")
 
@@ -76,6 +77,10 @@ def lib() -> ctypes.CDLL:
                                          _F, _I, _I, _I, _P, _I, _P, _P]
         L.spa_sparse_attn_prefill_segperm.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I,
                                                       _I, _I, _P, _I, _P, _F, _P, _P, _P]
+        L.spa_prefill_host_workspace_bytes.argtypes = [_I, _I, _I, _I, _I, _I, _I]
+        L.spa_prefill_host_workspace_bytes.restype = ctypes.c_size_t
+        L.spa_prefill_host.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _F, _I, _I,
+                                       _I, _P, ctypes.c_size_t, _P]
         L.spa_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_int)]
         L.spa_status_string.argtypes = [_I]
         L.spa_status_string.restype = ctypes.c_char_p
@@ -85,7 +90,7 @@ def lib() -> ctypes.CDLL:
                   "spa_rla_prefill", "spa_rla_decode_state", "spa_sparse_attn_decode_rla",
                   "spa_quantize_block_stats", "spa_select_quantized", "spa_select_score_order",
                   "spa_sparse_attn_prefill_early_stop", "spa_pbs_permutation", "spa_pbs_gather",
-                  "spa_select_segperm", "spa_sparse_attn_prefill_segperm"):
+                  "spa_select_segperm", "spa_sparse_attn_prefill_segperm", "spa_prefill_host"):
             getattr(L, f).restype = _I
         _lib = L
     return _lib
@@ -250,6 +255,43 @@ def spa_sparse_attn_prefill_early_stop(q: torch.Tensor, k: torch.Tensor, v: torc
                                                     _ptr(out), _ptr(lse), _ptr(processed),
                                                     _stream(stream)))
     return out, lse, processed
+
+
+def _hptr(t: torch.Tensor):
+    if t.is_cuda:
+        raise ValueError("spa_prefill_host takes host (CPU) tensors")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def spa_prefill_host_workspace_bytes(dtype: torch.dtype, B: int, Hq: int, Hkv: int, L: int,
+                                     d: int, block: int) -> int:
+    """Device workspace bytes spa_prefill_host needs for these sizes."""
+    dt = SPA_BF16 if dtype == torch.bfloat16 else SPA_F32
+    return int(lib().spa_prefill_host_workspace_bytes(dt, B, Hq, Hkv, L, d, block))
+
+
+def spa_prefill_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block: int,
+                     top_p: float, scale: float | None = None, n_sink: int = 1, n_local: int = 1,
+                     k_min: int = 0, out: torch.Tensor | None = None,
+                     workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """The whole prefill path from host tensors (pinned for copy/compute overlap):
+    q [B,Hq,L,d], k, v [B,Hkv,L,d] on the CPU -> out [B,Hq,L,d] on the CPU. Asynchronous
+    on `stream`: synchronise it before reading out."""
+    B, Hq, L, d = q.shape
+    Hkv = k.shape[1]
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    if out is None:
+        out = torch.empty(q.shape, dtype=q.dtype, pin_memory=q.is_pinned())
+    need = spa_prefill_host_workspace_bytes(q.dtype, B, Hq, Hkv, L, d, block)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device="cuda")
+    _check("spa_prefill_host",
+           lib().spa_prefill_host(_hptr(q), _hptr(k), _hptr(v), _hptr(out), _dt(q), B, Hq, Hkv, L,
+                                  d, block, scale, top_p, n_sink, n_local, k_min, _ptr(workspace),
+                                  workspace.numel() * workspace.element_size(), _stream(stream)))
+    return out
 
 
 def spa_pbs_permutation(q: torch.Tensor, k: torch.Tensor, block: int, seg_blocks: int,

@@ -382,6 +382,38 @@ spa_status spa_sparse_attn_decode_rla(const void *q, const void *kc, const void 
                                       void *out, float *out_rla, spa_stream stream);
 
 /*
+ * The whole prefill path (spa_block_stats -> spa_select -> spa_sparse_attn_prefill,
+ * the same kernels and results) from HOST buffers, the copies included. Each
+ * (b, kv-head) is an independent problem, so the work is cut into chunks of
+ * consecutive (b, kv-head) pairs; three internal streams pipeline them: the
+ * host-to-device copies of chunk c+1, the kernels of chunk c and the
+ * device-to-host copy of chunk c-1 run at the same time, so the PCIe transfers
+ * in both directions hide behind the compute. Asynchronous with respect to the
+ * host: the work is ordered after everything already enqueued on `stream`, and
+ * everything enqueued on `stream` afterwards waits for its end.
+ *   q, out : [B,Hq,L,d] host, dt;  k, v: [B,Hkv,L,d] host, dt (L = T)
+ *            Page-locked (pinned) host memory gives the overlap; pageable memory
+ *            is correct but the copies then serialise. The buffers belong to the
+ *            caller and must stay valid until `stream` reaches the end of the call.
+ *   workspace : device, >= spa_prefill_host_workspace_bytes(...) bytes, 256-byte
+ *            aligned, owned by the caller (three slots of chunk buffers: inputs,
+ *            statistics, lists, output); reusable across calls of the same sizes
+ *            once the previous call has completed on `stream`.
+ *   block, scale, top_p, n_sink, n_local, k_min: as spa_select; dtype, d and block
+ *            limits as spa_sparse_attn_prefill.
+ * Errors: SPA_ERR_INVALID / SPA_ERR_UNSUPPORTED from the host checks, before any
+ * copy or launch; SPA_ERR_CUDA if a copy or launch fails to enqueue (the work
+ * enqueued before it stays enqueued: synchronise `stream` before reusing the
+ * buffers).
+ */
+size_t spa_prefill_host_workspace_bytes(spa_dtype dt, int B, int Hq, int Hkv, int L, int d,
+                                        int block);
+spa_status spa_prefill_host(const void *q, const void *k, const void *v, void *out, spa_dtype dt,
+                            int B, int Hq, int Hkv, int L, int d, int block, float scale,
+                            float top_p, int n_sink, int n_local, int k_min, void *workspace,
+                            size_t workspace_bytes, spa_stream stream);
+
+/*
  * Reads and clears the device error word of the current device (one of
  * SPA_DEVERR_*). Synchronises the device. Returns SPA_ERR_DEVICE when the word was
  * non-zero, SPA_OK otherwise.

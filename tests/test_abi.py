@@ -201,6 +201,44 @@ def test_decode_workspace_size(lib):
     assert f(0, 32, 8, 131072, 128, 16) == 0
 
 
+def test_prefill_host_checks_and_workspace(lib):
+    I, F, Z = ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    w = lib.spa_prefill_host_workspace_bytes
+    w.restype = Z
+    w.argtypes = [I] * 7
+    one = w(1, 1, 4, 1, 4096, 128, 128)            # one (b, kv-head) pair: one slot
+    assert one > 0 and one % 256 == 0
+    # per pair: q + out (4 x 4096 x 128 x 2 each), k, v, mean, var, lists, counts
+    G, L, d, nb = 4, 4096, 128, 32
+    per_pair = 2 * G * L * d * 2 + 2 * L * d * 2 + 2 * nb * d * 4 + G * nb * nb * 4 + G * nb * 4
+    assert per_pair <= one < per_pair + 8 * 256
+    assert w(1, 1, 8, 2, 4096, 128, 128) == 2 * one      # two pairs: two chunks, two slots
+    assert w(1, 2, 8, 2, 4096, 128, 128) == 3 * one      # four pairs: four chunks, three slots
+    assert w(1, 1, 32, 8, 4096, 128, 128) == 3 * one     # eight chunks share three slots
+    assert w(1, 8, 32, 8, 4096, 128, 128) >= 3 * 8 * per_pair   # chunks of eight pairs
+    assert w(1, 0, 4, 1, 4096, 128, 128) == 0
+    assert w(1, 1, 3, 2, 4096, 128, 128) == 0            # Hq not a multiple of Hkv
+    f = lib.spa_prefill_host
+    f.argtypes = [P, P, P, P, I, I, I, I, I, I, I, F, F, I, I, I, P, Z, P]
+    ok = dict(dt=1, B=1, Hq=4, Hkv=1, L=4096, d=128, block=128, top_p=0.9, ws=FAKE, nws=one)
+
+    def call(q=FAKE, **kw):
+        a = dict(ok, **kw)
+        return f(q, FAKE, FAKE, FAKE, a["dt"], a["B"], a["Hq"], a["Hkv"], a["L"], a["d"],
+                 a["block"], 0.1, a["top_p"], 1, 1, 0, a["ws"], a["nws"], None)
+
+    assert call(q=None) == 1
+    assert call(Hq=3, Hkv=2) == 1
+    assert call(top_p=0.0) == 1
+    assert call(d=64) == 2                   # bf16 attention needs d = 128
+    assert call(block=32) == 2
+    assert call(dt=0, block=16) == 2
+    assert call(ws=None) == 1
+    assert call(ws=P(0x10010)) == 1          # not 256-byte aligned
+    assert call(nws=one - 1) == 1
+    assert "workspace" in _last(lib)
+
+
 def test_binding_fails_loudly_without_cuda_tensors():
     import torch
     import block_sparse_long_stats_b200 as spa
