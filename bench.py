@@ -14,6 +14,10 @@ statistics -> Taylor-score top-p selection -> block-sparse causal attention
             buffers: the host -> device copies of Q, K, V and the device -> host
             copy of O inside the timed region, pipelined against the kernels over
             chunks of (b, kv-head) pairs
+  diagnostics   per prefill workload (1K fp32, 8K, 32K): kept fraction of the
+            causal blocks (mean, p50, p99), operator MSE against dense causal
+            attention and the attention-mass coverage of the kept set, all from
+            the library's own kernels (dense = the same prefill at top_p = 1)
   cpu_baseline  the CPU oracle on a bounded sample (rank 0, one GPU only)
 
 `--impl reference` times the CPU oracle on the same workload instead (the
@@ -228,6 +232,32 @@ def run_reference(args, rank: int):
 
 # ---------------------------------------------------------------- CUDA arm
 
+def prefill_diagnostics(spa, torch, wl, q, k, v) -> dict:
+    """Diagnostics of the selection on one prefill workload, from the library's own
+    kernels only: the kept fraction of the causal blocks per (b, head, query block)
+    (mean, p50, p99), the operator MSE of the sparse output against dense causal
+    attention (the same prefill at top_p = 1, which keeps every block), and the
+    attention-mass coverage of the kept set per query row, exp(lse_sparse -
+    lse_dense): the share of the dense softmax mass that falls on kept keys."""
+    sp = spa.prefill(q, k, v, wl.block, wl.top_p, wl.scale, wl.n_sink, wl.n_local, wl.k_min,
+                     want_lse=True)
+    de = spa.prefill(q, k, v, wl.block, 1.0, wl.scale, wl.n_sink, wl.n_local, wl.k_min,
+                     want_lse=True)
+    torch.cuda.synchronize()
+    nq = sp["count"].shape[-1]
+    causal = torch.arange(1, nq + 1, device="cuda", dtype=torch.float32)
+    frac = (sp["count"].float() / causal).flatten()
+    os_, od = sp["out"].float(), de["out"].float()
+    mse = float(((os_ - od) ** 2).mean())
+    cov = torch.exp(sp["lse"] - de["lse"]).flatten()
+    qs = torch.tensor([0.01, 0.5, 0.99], device="cuda")
+    fq = torch.quantile(frac, qs).tolist()
+    cq = torch.quantile(cov, qs).tolist()
+    return {"kept_fraction": {"mean": float(frac.mean()), "p50": fq[1], "p99": fq[2]},
+            "mse_vs_dense": mse, "mse_rel": mse / float((od ** 2).mean()),
+            "coverage": {"mean": float(cov.mean()), "p1": cq[0], "p50": cq[1]}}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -247,6 +277,8 @@ def main():
                     help="segment length (in blocks) of the segmented-permutation leg (0: skip)")
     ap.add_argument("--no-quant", action="store_true",
                     help="skip the selection on quantised statistics in the decode leg")
+    ap.add_argument("--no-diagnostics", action="store_true",
+                    help="skip the kept-fraction / MSE-vs-dense / coverage diagnostics")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-tokens", type=int, default=192)
@@ -673,6 +705,28 @@ def main():
                   "block_stats_full_cache": stats_full, "rla": drla, "quantized_stats": dq}
         del kc, vc
 
+    # ---- selection diagnostics on the three prefill workloads (dense comparisons
+    # on the 1K, 8K and 32K workloads only; the 128K one would need 140 TFLOP more)
+    diag = None
+    if rank == 0 and not args.no_diagnostics:
+        diag = {}
+        for cid in (1, 2, args.workload):
+            wl = WORKLOADS[cid]
+            if wl.mode != "prefill":
+                continue
+            if cid == args.workload:
+                dq, dk, dv = q, k, v
+            else:
+                xl = generate(wl)
+                conv = ((lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16))
+                         .cuda().view(torch.bfloat16)) if wl.dtype == "bf16"
+                        else (lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()))
+                dq, dk, dv = conv(xl["q"]), conv(xl["k"]), conv(xl["v"])
+            diag[wl.name] = prefill_diagnostics(spa, torch, wl, dq, dk, dv)
+            del dq, dk, dv
+        torch.cuda.empty_cache()
+        assert spa.spa_get_device_error() == 0
+
     # ---- CPU oracle baseline (rank 0, one GPU)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
@@ -705,6 +759,7 @@ def main():
             "early_stop": early,
             "segmented_permutation": pbs,
             "decode": decode,
+            "diagnostics": diag,
             "e2e": e2e,
             "cpu_baseline": cpu,
             "clocks": clk,
