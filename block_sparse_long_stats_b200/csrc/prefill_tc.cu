@@ -164,12 +164,14 @@ __global__ void __launch_bounds__(kThreads, 2)
     uint32_t *bits = reinterpret_cast<uint32_t *>(list_s + (ES ? a.nq : 0)); // ES: [nwords]
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int per_i = a.B * a.Hkv * a.npairs;
-    const int i = a.nq - 1 - (int)(blockIdx.x / per_i);
-    const int rest = (int)(blockIdx.x % per_i);
-    const int b = rest / (a.Hkv * a.npairs);
-    const int g = (rest / a.npairs) % a.Hkv;
+    // (b, kv-head)-major, query blocks heaviest first inside each: the CTAs resident
+    // at a time share one kv-head's K and V tiles, which then stay in L2
+    const int per_bg = a.nq * a.npairs;
+    const int bg = (int)(blockIdx.x / per_bg);
+    const int rest = (int)(blockIdx.x % per_bg);
+    const int i = a.nq - 1 - rest / a.npairs;
     const int hp = rest % a.npairs;
+    const int b = bg / a.Hkv, g = bg % a.Hkv;
     const int h0 = g * a.G + hp * HPT;
 
     if (tid == 0) {
