@@ -274,12 +274,15 @@ __global__ void __launch_bounds__(kThreads, 2)
     __shared__ int scan_max[4], res_count, diag_res;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    // Units: query block i descending (most residual work first), then b, head; the
-    // heads of one kv-group are adjacent and read the same W_j tiles.
-    const int per_i = a.B * a.Hq;
-    const int i = a.nq - 1 - (int)(blockIdx.x / per_i);
-    const int rest = (int)(blockIdx.x % per_i);
-    const int b = rest / a.Hq, h = rest % a.Hq, g = h / a.G;
+    // Units: (b, kv-group)-major, then query block i descending (most residual work
+    // first), then the group's heads, adjacent: the CTAs resident at a time read one
+    // kv-group's W_j tiles (8 MB at d = 128, nb = 256), which then stay in L2.
+    const int per_bg = a.nq * a.G;
+    const int bg = (int)(blockIdx.x / per_bg);
+    const int rest = (int)(blockIdx.x % per_bg);
+    const int i = a.nq - 1 - rest / a.G;
+    const int Hkv = a.Hq / a.G;
+    const int b = bg / Hkv, g = bg % Hkv, h = g * a.G + rest % a.G;
     const size_t unit = ((size_t)b * a.Hq + h) * a.nq + i;
 
     if (tid == 0) {
