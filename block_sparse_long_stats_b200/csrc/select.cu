@@ -677,7 +677,7 @@ __global__ void __launch_bounds__(kThreads, 3) select_group_kernel(SelectArgs a)
 constexpr int kDecTile = 256;
 
 template <typename T, int D, int G, bool QS>
-__global__ void __launch_bounds__(kThreads) decode_score_kernel(SelectArgs a) {
+__global__ void __launch_bounds__(kThreads, 2) decode_score_kernel(SelectArgs a) {
     constexpr int PL = D / 32;
     // U candidates per warp step, so that the 2G partial sums of all of them fill
     // one transposing reduction of up to 32 values: 16 (candidate, head) scores
@@ -713,16 +713,26 @@ __global__ void __launch_bounds__(kThreads) decode_score_kernel(SelectArgs a) {
     constexpr int LB = 5 - ilog2(NV);               // lanes per value = 2^LB
     const int vi = lane >> LB;                      // value this lane's group ends with
     const int uu = vi / (2 * G), kk = vi % (2 * G); // its candidate, and dot (< G) or quad
-    for (int r = warp * U; r < kDecTile; r += kWarps * U) {
-        float mu[U][PL], vr[U][PL];
+    // A fixed number of steps per warp; each step's statistics are loaded one step
+    // ahead (two register buffers), so a warp always has loads in flight.
+    constexpr int STEPS = kDecTile / (kWarps * U);
+    float mu[2][U][PL], vr[2][U][PL];
+    auto load = [&](float (&m)[U][PL], float (&w)[U][PL], int r) {
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const int j = min(j0 + r + u, a.nb - 1);
             if constexpr (QS)
-                load_stats_q<D>(qb + (size_t)j * (D + D / 16), lane, mu[u], vr[u]);
+                load_stats_q<D>(qb + (size_t)j * (D + D / 16), lane, m[u], w[u]);
             else
-                load_stats<PL>(mb + (size_t)j * D, vb + (size_t)j * D, mu[u], vr[u]);
+                load_stats<PL>(mb + (size_t)j * D, vb + (size_t)j * D, m[u], w[u]);
         }
+    };
+    load(mu[0], vr[0], warp * U);
+#pragma unroll
+    for (int it = 0; it < STEPS; ++it) {
+        const int r = warp * U + it * kWarps * U;
+        const int cb = it & 1;
+        if (it + 1 < STEPS) load(mu[cb ^ 1], vr[cb ^ 1], r + kWarps * U);
         // per-lane partials: value u*2G + h is the dot of head h with candidate u,
         // value u*2G + G + h its variance term
         float v[NV];
@@ -730,7 +740,7 @@ __global__ void __launch_bounds__(kThreads) decode_score_kernel(SelectArgs a) {
         for (int u = 0; u < U; ++u)
 #pragma unroll
             for (int hh = 0; hh < G; ++hh)
-                lane_partials<PL>(qv[hh], q2[hh], mu[u], vr[u], v[u * 2 * G + hh],
+                lane_partials<PL>(qv[hh], q2[hh], mu[cb][u], vr[cb][u], v[u * 2 * G + hh],
                                   v[u * 2 * G + G + hh]);
         // Transposing halving reduction: at each xor offset every lane keeps half of
         // its values and adds its partner's copy of them, the same pairwise sums the
