@@ -108,10 +108,17 @@ __device__ __forceinline__ void load_stats(const float *mb, const float *vb, flo
 }
 
 // The same PL components from a quantised record (INT4 codes, a power-of-two scale
-// per 32 features; layout in qstats.cu), dequantised exactly: code * 2^k.
+// per 32 features; layout in qstats.cu): the codes as floats in mu, vr and the
+// lane's two group scales 2^k in sm, sv (a lane's PL features lie in one group).
+// The callers scale the lane's dot and variance sums by sm, sv instead of each
+// component: scaling by a power of two commutes with every rounding of the FMA
+// chain (in the normal range), so the sums equal those over code * 2^k exactly.
+// A 4-bit code n becomes a float without a conversion instruction: 2^23 + n has n
+// in its low mantissa bits, so subtracting 2^23 (plus the signed codes' bias of 8,
+// n ^ 8 = code + 8 for two's-complement nibbles) is exact.
 template <int D>
 __device__ __forceinline__ void load_stats_q(const uint8_t *rec, int lane, float (&mu)[D / 32],
-                                             float (&vr)[D / 32]) {
+                                             float (&vr)[D / 32], float &sm, float &sv) {
     constexpr int PL = D / 32, LPG = 32 / PL;
     uint32_t cm, cv;
     if constexpr (PL == 4) {
@@ -123,11 +130,12 @@ __device__ __forceinline__ void load_stats_q(const uint8_t *rec, int lane, float
     }
     const int km = (int8_t)__ldg(rec + D + lane / LPG);
     const int kv = (int8_t)__ldg(rec + D + D / 32 + lane / LPG);
-    const float sm = __int_as_float((km + 127) << 23), sv = __int_as_float((kv + 127) << 23);
+    sm = __int_as_float((km + 127) << 23);
+    sv = __int_as_float((kv + 127) << 23);
 #pragma unroll
     for (int c = 0; c < PL; ++c) {
-        mu[c] = (float)((int)(cm << (28 - 4 * c)) >> 28) * sm;   // sign-extended nibble
-        vr[c] = (float)((cv >> (4 * c)) & 15u) * sv;
+        mu[c] = __uint_as_float(0x4B000000u | (((cm >> (4 * c)) & 15u) ^ 8u)) - 8388616.0f;
+        vr[c] = __uint_as_float(0x4B000000u | ((cv >> (4 * c)) & 15u)) - 8388608.0f;
     }
 }
 
@@ -385,12 +393,12 @@ __global__ void __launch_bounds__(kThreads) select_kernel(SelectArgs a) {
         const float *vbp = a.seg_blocks > 0 ? a.var_p + bgo * D + lane * PL : nullptr;
         const int vi = lane >> LB;                  // value this lane's group ends with
         for (int r0 = warp * U; r0 < nres; r0 += kWarps * U) {
-            float mu[U][PL], vr[U][PL];
+            float mu[U][PL], vr[U][PL], sm[U], sv[U];
 #pragma unroll
             for (int u = 0; u < U; ++u) {
                 const int j = r_lo + min(r0 + u, nres - 1);   // past the end: a repeat, unused
                 if constexpr (QS)
-                    load_stats_q<D>(qb + (size_t)j * (D + D / 16), lane, mu[u], vr[u]);
+                    load_stats_q<D>(qb + (size_t)j * (D + D / 16), lane, mu[u], vr[u], sm[u], sv[u]);
                 else if (j < seg0)
                     load_stats<PL>(mbp + (size_t)j * D, vbp + (size_t)j * D, mu[u], vr[u]);
                 else
@@ -399,7 +407,13 @@ __global__ void __launch_bounds__(kThreads) select_kernel(SelectArgs a) {
             // value 2u is candidate u's dot, value 2u + 1 its variance term
             float v[NV];
 #pragma unroll
-            for (int u = 0; u < U; ++u) lane_partials<PL>(qv, q2, mu[u], vr[u], v[2 * u], v[2 * u + 1]);
+            for (int u = 0; u < U; ++u) {
+                lane_partials<PL>(qv, q2, mu[u], vr[u], v[2 * u], v[2 * u + 1]);
+                if constexpr (QS) {
+                    v[2 * u] *= sm[u];
+                    v[2 * u + 1] *= sv[u];
+                }
+            }
             const float tot = reduce_transpose<NV>(v, lane);
             const float quad = __shfl_sync(0xffffffffu, tot, (lane + (1 << LB)) & 31);
             const int r = r0 + (vi >> 1);
@@ -606,12 +620,12 @@ __global__ void __launch_bounds__(kThreads, 3) select_group_kernel(SelectArgs a)
         const int vi = lane >> LB;
         const int uu = vi / (2 * G), kk = vi % (2 * G);   // candidate; dot (< G) or quad
         for (int r0 = warp * U; r0 < nres; r0 += kWarps * U) {
-            float mu[U][PL], vr[U][PL];
+            float mu[U][PL], vr[U][PL], sm[U], sv[U];
 #pragma unroll
             for (int u = 0; u < U; ++u) {
                 const int j = r_lo + min(r0 + u, nres - 1);   // past the end: a repeat, unused
                 if constexpr (QS)
-                    load_stats_q<D>(qb + (size_t)j * (D + D / 16), lane, mu[u], vr[u]);
+                    load_stats_q<D>(qb + (size_t)j * (D + D / 16), lane, mu[u], vr[u], sm[u], sv[u]);
                 else if (j < seg0)
                     load_stats<PL>(mbp + (size_t)j * D, vbp + (size_t)j * D, mu[u], vr[u]);
                 else
@@ -621,9 +635,14 @@ __global__ void __launch_bounds__(kThreads, 3) select_group_kernel(SelectArgs a)
 #pragma unroll
             for (int u = 0; u < U; ++u)
 #pragma unroll
-                for (int hh = 0; hh < G; ++hh)
+                for (int hh = 0; hh < G; ++hh) {
                     lane_partials<PL>(qv[hh], q2[hh], mu[u], vr[u], v[u * 2 * G + hh],
                                       v[u * 2 * G + G + hh]);
+                    if constexpr (QS) {
+                        v[u * 2 * G + hh] *= sm[u];
+                        v[u * 2 * G + G + hh] *= sv[u];
+                    }
+                }
             const float tot = reduce_transpose<NV>(v, lane);
             const float quad = __shfl_sync(0xffffffffu, tot, (lane + (G << LB)) & 31);
             const int r = r0 + uu;
@@ -716,32 +735,37 @@ __global__ void __launch_bounds__(kThreads, 2) decode_score_kernel(SelectArgs a)
     // A fixed number of steps per warp; each step's statistics are loaded one step
     // ahead (two register buffers), so a warp always has loads in flight.
     constexpr int STEPS = kDecTile / (kWarps * U);
-    float mu[2][U][PL], vr[2][U][PL];
-    auto load = [&](float (&m)[U][PL], float (&w)[U][PL], int r) {
+    float mu[2][U][PL], vr[2][U][PL], sm[2][U], sv[2][U];
+    auto load = [&](float (&m)[U][PL], float (&w)[U][PL], float (&cs)[U], float (&ws)[U], int r) {
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const int j = min(j0 + r + u, a.nb - 1);
             if constexpr (QS)
-                load_stats_q<D>(qb + (size_t)j * (D + D / 16), lane, m[u], w[u]);
+                load_stats_q<D>(qb + (size_t)j * (D + D / 16), lane, m[u], w[u], cs[u], ws[u]);
             else
                 load_stats<PL>(mb + (size_t)j * D, vb + (size_t)j * D, m[u], w[u]);
         }
     };
-    load(mu[0], vr[0], warp * U);
+    load(mu[0], vr[0], sm[0], sv[0], warp * U);
 #pragma unroll
     for (int it = 0; it < STEPS; ++it) {
         const int r = warp * U + it * kWarps * U;
         const int cb = it & 1;
-        if (it + 1 < STEPS) load(mu[cb ^ 1], vr[cb ^ 1], r + kWarps * U);
+        if (it + 1 < STEPS) load(mu[cb ^ 1], vr[cb ^ 1], sm[cb ^ 1], sv[cb ^ 1], r + kWarps * U);
         // per-lane partials: value u*2G + h is the dot of head h with candidate u,
         // value u*2G + G + h its variance term
         float v[NV];
 #pragma unroll
         for (int u = 0; u < U; ++u)
 #pragma unroll
-            for (int hh = 0; hh < G; ++hh)
+            for (int hh = 0; hh < G; ++hh) {
                 lane_partials<PL>(qv[hh], q2[hh], mu[cb][u], vr[cb][u], v[u * 2 * G + hh],
                                   v[u * 2 * G + G + hh]);
+                if constexpr (QS) {
+                    v[u * 2 * G + hh] *= sm[cb][u];
+                    v[u * 2 * G + G + hh] *= sv[cb][u];
+                }
+            }
         // Transposing halving reduction: at each xor offset every lane keeps half of
         // its values and adds its partner's copy of them, the same pairwise sums the
         // per-value butterfly forms.
