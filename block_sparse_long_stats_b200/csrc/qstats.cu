@@ -15,20 +15,28 @@
 // rounding are exact.
 //
 // HBM-bound and tiny: one warp per record reads 2 d fp32 values and writes
-// d + d/16 bytes.
+// d + d/16 bytes. Powers of two come from exponent fields (exact), not from
+// frexpf/ldexpf, so the arithmetic stays off the special-function pipe.
 #include "kernels.h"
 
 namespace spa {
 namespace {
 
+// 2^k as a float, built from its exponent field (exact for k in [-126, 127]).
+__device__ __forceinline__ float pow2i(int k) { return __int_as_float((k + 127) << 23); }
+
+// The smallest k in [-126, 126] with amax <= top * 2^k (top = 7 or 15). Starts from
+// the exponent field of amax and steps k until the exact fp32 comparison decides;
+// zero, subnormal or non-finite maxima take the range's end directly.
 __device__ __forceinline__ int group_exponent(float amax, float top) {
     if (!(amax > 0.f)) return -126;
-    int e;
-    (void)frexpf(amax, &e);
-    int k = e - 4;
-    while (amax > top * ldexpf(1.f, k)) ++k;
-    while (k > -126 && amax <= top * ldexpf(1.f, k - 1)) --k;
-    return max(-126, min(126, k));
+    const int eb = (__float_as_int(amax) >> 23) & 255;
+    if (eb == 0) return -126;                  // subnormal: <= top * 2^-126
+    if (eb == 255) return 126;
+    int k = max(-126, eb - 126 - 4);           // amax in [2^(eb-127), 2^(eb-126))
+    while (k < 126 && amax > top * pow2i(k)) ++k;
+    while (k > -126 && amax <= top * pow2i(k - 1)) --k;
+    return k;
 }
 
 template <int D>
@@ -71,8 +79,8 @@ __global__ void __launch_bounds__(256) quantize_stats_kernel(const float *__rest
     uint32_t pm = 0, pv = 0;
 #pragma unroll
     for (int c = 0; c < PL; ++c) {
-        const int qm = max(-7, min(7, (int)rintf(ldexpf(m[c], -km))));
-        const int qv = max(0, min(15, (int)rintf(ldexpf(v[c], -kv))));
+        const int qm = max(-7, min(7, (int)rintf(m[c] * pow2i(-km))));
+        const int qv = max(0, min(15, (int)rintf(v[c] * pow2i(-kv))));
         pm |= (uint32_t)(qm & 15) << (4 * c);
         pv |= (uint32_t)qv << (4 * c);
     }
