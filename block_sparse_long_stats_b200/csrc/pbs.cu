@@ -9,8 +9,9 @@
 //
 // pbs_perm_kernel: one CTA per (segment, b * Hkv + g): qbar (fp32), one fp32 score
 // per key (d / 8 lanes per key with 16-byte loads, four in flight, shuffle sums),
-// then a bitonic sort of
-// 64-bit keys (order-flipped score | index) in shared memory; writes perm.
+// then a bitonic sort of 64-bit keys (order-flipped score | index): segments up to
+// 2048 keys in registers (eight per thread; shuffles for strides up to 128, shared
+// memory for the six larger ones), longer ones in shared memory; writes perm.
 // gather_rows_kernel: the permuted copy of K or V, 16 bytes per thread.
 #include <float.h>
 
@@ -23,6 +24,7 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
+constexpr int kRegSort = 8 * kThreads;   // segments up to this many keys sort in registers
 
 __device__ __forceinline__ uint32_t order_desc(float f) {
     const uint32_t b = __float_as_uint(f);
@@ -116,6 +118,69 @@ __global__ void __launch_bounds__(kThreads) pbs_perm_kernel(const T *__restrict_
             if (cl == 0 && x < n) keys[x] = ((uint64_t)order_desc(sdot) << 32) | (uint32_t)x;
         }
     }
+    if (sort_cap <= kRegSort) {
+        // up to 2048 keys: 8 per thread in registers, position x = 8 tid + e; strides
+        // below 8 in registers, 8..128 by shuffles, 256 and up through shared memory
+        // (two buffers, one barrier per stride)
+        for (int x = n + tid; x < kRegSort; x += kThreads) keys[x] = ~0ull;
+        __syncthreads();
+        uint64_t kr[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) kr[e] = keys[tid * 8 + e];
+        int pb = 1;                            // keys[] was just read: write buffer 1 first
+        constexpr int LOG_N = 11;              // kRegSort = 2^11
+        static_assert((1 << LOG_N) == kRegSort, "register sort size");
+#pragma unroll
+        for (int lk = 1; lk <= LOG_N; ++lk) {
+            const int kk = 1 << lk;
+#pragma unroll
+            for (int lj = lk - 1; lj >= 0; --lj) {
+                const int jj = 1 << lj;
+                if (jj < 8) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        if ((e & jj) == 0) {
+                            const bool up = ((tid * 8 + e) & kk) == 0;
+                            const uint64_t a = kr[e], c = kr[e | jj];
+                            const bool sw = (a > c) == up;
+                            kr[e] = sw ? c : a;
+                            kr[e | jj] = sw ? a : c;
+                        }
+                    }
+                } else if (jj < 256) {
+                    const int lm = jj / 8;       // partner lane
+                    const bool lower = (lane & lm) == 0;
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const bool up = ((tid * 8 + e) & kk) == 0;
+                        const uint64_t o = __shfl_xor_sync(0xffffffffu, kr[e], lm);
+                        const uint64_t mn = kr[e] < o ? kr[e] : o, mx = kr[e] < o ? o : kr[e];
+                        kr[e] = lower == up ? mn : mx;
+                    }
+                } else {
+                    uint64_t *bw = keys + pb * kRegSort;
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) bw[tid * 8 + e] = kr[e];
+                    __syncthreads();
+                    const bool lower = ((tid * 8) & jj) == 0;
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const bool up = ((tid * 8 + e) & kk) == 0;
+                        const uint64_t o = bw[(tid * 8 + e) ^ jj];
+                        const uint64_t mn = kr[e] < o ? kr[e] : o, mx = kr[e] < o ? o : kr[e];
+                        kr[e] = lower == up ? mn : mx;
+                    }
+                    pb ^= 1;
+                }
+            }
+        }
+        int32_t *out = perm + (size_t)bg * L + s0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+            if (tid * 8 + e < n) out[tid * 8 + e] = s0 + (int)(uint32_t)kr[e];
+        return;
+    }
+
     for (int x = n + tid; x < sort_cap; x += kThreads) keys[x] = ~0ull;
     __syncthreads();
 
@@ -160,7 +225,8 @@ cudaError_t launch_perm_t(const void *q, const void *k, int B, int Hq, int Hkv, 
     const int seg_len = seg_blocks * block;
     int cap = 1;
     while (cap < seg_len) cap <<= 1;
-    const size_t smem = (size_t)cap * 8;
+    // the register sort pads to kRegSort keys and exchanges through two buffers
+    const size_t smem = (size_t)(cap <= kRegSort ? 2 * kRegSort : cap) * 8;
     auto kern = pbs_perm_kernel<T, D>;
     if (smem > 48 * 1024) {
         const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -20,7 +20,9 @@ from workloads import PARITY_WORKLOADS, generate, widen
 pytestmark = pytest.mark.gpu
 
 TOL = 2e-2
-CASES = [("p_bf16_blk128", 2), ("p_bf16_blk128", 3), ("p_bf16_blk64", 4)]
+# segments of 256, 384 (ragged last) and 256 keys sort in registers; 24 blocks of
+# 128 (3072 keys, one segment over the whole sequence) take the shared-memory sort
+CASES = [("p_bf16_blk128", 2), ("p_bf16_blk128", 3), ("p_bf16_blk64", 4), ("p_bf16_blk128", 24)]
 
 _cache = {}
 
