@@ -281,7 +281,7 @@ def main():
                     help="skip the kept-fraction / MSE-vs-dense / coverage diagnostics")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
-    ap.add_argument("--cpu-tokens", type=int, default=192)
+    ap.add_argument("--cpu-tokens", type=int, default=1536)
     ap.add_argument("--ref-tokens", type=int, default=48)
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
