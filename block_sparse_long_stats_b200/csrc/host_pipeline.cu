@@ -109,7 +109,19 @@ struct Pipe {
 std::mutex g_pipe_mu;
 Pipe *g_pipe[64];
 
-// This device's streams and events, created on first use (caller holds g_pipe_mu).
+void destroy_pipe(Pipe *p) {
+    for (cudaStream_t st : {p->h2d, p->comp, p->d2h})
+        if (st) cudaStreamDestroy(st);
+    cudaEvent_t *groups[] = {&p->start, p->join, p->in, p->done, p->freed};
+    const int sizes[] = {1, 3, kSlots, kSlots, kSlots};
+    for (int g = 0; g < 5; ++g)
+        for (int i = 0; i < sizes[g]; ++i)
+            if (groups[g][i]) cudaEventDestroy(groups[g][i]);
+    delete p;
+}
+
+// This device's streams and events, created on first use (caller holds g_pipe_mu);
+// on a failure everything created so far is released and nothing is cached.
 cudaError_t get_pipe(Pipe **out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -118,18 +130,20 @@ cudaError_t get_pipe(Pipe **out) {
     if (!g_pipe[dev]) {
         Pipe *p = new Pipe;
         const unsigned sf = cudaStreamNonBlocking, ef = cudaEventDisableTiming;
-        if ((e = cudaStreamCreateWithFlags(&p->h2d, sf)) != cudaSuccess ||
-            (e = cudaStreamCreateWithFlags(&p->comp, sf)) != cudaSuccess ||
-            (e = cudaStreamCreateWithFlags(&p->d2h, sf)) != cudaSuccess ||
-            (e = cudaEventCreateWithFlags(&p->start, ef)) != cudaSuccess)
+        e = cudaStreamCreateWithFlags(&p->h2d, sf);
+        if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&p->comp, sf);
+        if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&p->d2h, sf);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&p->start, ef);
+        for (int i = 0; i < 3 && e == cudaSuccess; ++i) e = cudaEventCreateWithFlags(&p->join[i], ef);
+        for (int s = 0; s < kSlots && e == cudaSuccess; ++s) {
+            e = cudaEventCreateWithFlags(&p->in[s], ef);
+            if (e == cudaSuccess) e = cudaEventCreateWithFlags(&p->done[s], ef);
+            if (e == cudaSuccess) e = cudaEventCreateWithFlags(&p->freed[s], ef);
+        }
+        if (e != cudaSuccess) {
+            destroy_pipe(p);
             return e;
-        for (int i = 0; i < 3; ++i)
-            if ((e = cudaEventCreateWithFlags(&p->join[i], ef)) != cudaSuccess) return e;
-        for (int s = 0; s < kSlots; ++s)
-            if ((e = cudaEventCreateWithFlags(&p->in[s], ef)) != cudaSuccess ||
-                (e = cudaEventCreateWithFlags(&p->done[s], ef)) != cudaSuccess ||
-                (e = cudaEventCreateWithFlags(&p->freed[s], ef)) != cudaSuccess)
-                return e;
+        }
         g_pipe[dev] = p;
     }
     *out = g_pipe[dev];
