@@ -49,10 +49,10 @@ def test_host_pipeline_equals_device_path(key):
 
 
 @pytest.mark.parametrize("B,Hq,Hkv,T", [(5, 4, 2, 700), (1, 2, 1, 1000), (3, 8, 4, 520),
-                                        (9, 4, 1, 300)])
+                                        (9, 4, 1, 300), (1, 8, 1, 700), (2, 8, 2, 520)])
 def test_host_pipeline_chunkings(B, Hq, Hkv, T):
     # pairs 10 (chunks of 2), 1 (one chunk, one slot), 12 (chunks of 2), 9 (chunks
-    # of 2, the last one pair)
+    # of 2, the last one pair); 1 and 4 pairs of 8 and 4 heads (one pair per chunk)
     w = PARITY_WORKLOADS["p_bf16_blk64"].with_(B=B, Hq=Hq, Hkv=Hkv, T=T)
     s = torch.cuda.Stream()
     x, out, r = run_both(w, pin=True, stream=s)
