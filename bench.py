@@ -381,7 +381,11 @@ def main():
     per_kernel = {
         "block_stats": {"ms": statistics.mean(t_stats),
                         "GB/s": stats_bytes / (statistics.mean(t_stats) / 1e3) / 1e9},
-        "select": {"ms": statistics.mean(t_sel)},
+        # bytes: Q read once to pool it, the statistics once (then L2-resident)
+        "select": {"ms": statistics.mean(t_sel),
+                   "GB/s": (q.numel() * q.element_size() + 2 * mean.numel() * 4)
+                   / (statistics.mean(t_sel) / 1e3) / 1e9,
+                   "share_of_step": statistics.mean(t_sel) / (total_ms / args.steps)},
         "sparse_attn_prefill": {"ms": att_ms, "TFLOP/s": achieved},
     }
 
@@ -698,7 +702,10 @@ def main():
                   "tokens/s": world * wd.B / ((t_qsel + t_dec) / 1e3)}
             del qrec, qi, qc
         decode = {"workload": wd.name, "kept_kv_bytes": dbytes, "attn_ms": t_dec,
-                  "select_ms": t_dsel, "GB/s": gbs, "peak_GB/s": peaks["hbm_gbs"],
+                  "select_ms": t_dsel,
+                  "select_GB/s": 2 * dm.numel() * 4 / (t_dsel / 1e3) / 1e9,
+                  "select_share_of_step": t_dsel / (t_dsel + t_dec),
+                  "GB/s": gbs, "peak_GB/s": peaks["hbm_gbs"],
                   "frac": gbs / peaks["hbm_gbs"], "peak_source": peak_src,
                   "tokens/s": world * wd.B / ((t_dsel + t_dec) / 1e3),
                   "kept_fraction": float(dcnt.float().mean().item()) / wd.nb,

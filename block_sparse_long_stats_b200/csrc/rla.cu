@@ -69,7 +69,9 @@ template <int BLK>
 struct StCfg {
     static constexpr int HALF = BLK * 128;               // bytes of one 64-column half
     static constexpr int TILE = 2 * HALF;
-    static constexpr int STAGES = 2;
+    // three K/V chunks in flight per SM (192 KB at 128 rows): the exponentials and
+    // MMAs of one chunk run while the next two load
+    static constexpr int STAGES = 3;
     static constexpr int OFF_K = 0;
     static constexpr int OFF_V = STAGES * TILE;
     static constexpr int SMEM = 2 * STAGES * TILE;
