@@ -316,6 +316,24 @@ def test_decode_workload_full_size():
     assert_no_device_error()
 
 
+@pytest.mark.parametrize("Hq,Hkv,block,dtype", [(4, 4, 128, "bf16"), (4, 2, 128, "bf16"),
+                                                (8, 2, 128, "bf16"), (8, 1, 64, "bf16"),
+                                                (6, 2, 64, "bf16"), (8, 1, 64, "f32")])
+def test_select_head_groupings(Hq, Hkv, block, dtype):
+    # G = 1, 2, 4, 8 query heads per kv-head take the grouped selection kernel (one
+    # CTA per kv-head and query block, a warp per head for the sort and cut); G = 3
+    # takes the per-head kernel; the fp32 case reads fp32 queries
+    base = "p_bf16_blk128" if dtype == "bf16" else "p_f32_d128"
+    w = PARITY_WORKLOADS[base].with_(Hq=Hq, Hkv=Hkv, block=block, B=1, T=777)
+    x, dev = inputs(w)
+    mean, var = spa.spa_block_stats(dev["k"], w.block)
+    idx, cnt = spa.spa_select(dev["q"], mean, var, w.T, w.block, w.scale, w.top_p, w.n_sink,
+                              w.n_local, w.k_min)
+    torch.cuda.synchronize()
+    check_lists(w, idx, cnt, oracle_select(w, x), w.Lq)
+    assert_no_device_error()
+
+
 @pytest.mark.parametrize("Hq,Hkv,block", [(4, 4, 128), (4, 2, 128), (8, 2, 128), (2, 1, 64),
                                           (4, 1, 64), (8, 2, 64)])
 def test_prefill_head_groupings(Hq, Hkv, block):
