@@ -8,14 +8,18 @@
 // One CTA per tile of 128 query rows: one query block of one head (block 128), or
 // the same query block of two heads of one kv-group stacked (block 64; the pair
 // walks the union of its two kept lists, and a row masks the blocks its own head
-// did not keep). Warp roles:
+// did not keep). A key tile is always 128 keys: one kept block at block 128, two
+// consecutive blocks of the walk at block 64 (two 64-row TMA boxes per 128-byte-
+// swizzled half, whose pattern repeats every 8 rows, so the tile is laid out as one
+// 128-row box; the columns of each half masked by their own block's rules), so that
+// S = Q K^T is always the N = 128 product. Warp roles:
 //   warps 0-3 : softmax; thread r owns query row r = TMEM lane r
 //   warp 4    : TMA producer (Q once; K_j and V_j per kept block)
 //   warp 5    : TMEM allocator and single-thread tcgen05.mma issuer
 // Per kept block n: S = Q K_j^T (8 MMAs, both operands K-major in shared memory,
 // fp32 accumulator in TMEM); the softmax scales by s*log2(e), takes exp2, keeps the
 // running max lazily (O is rescaled only when the max grows by more than 8, in
-// log2 units) and writes P as bf16 over the first BLK/2 columns of S (scaling and
+// log2 units) and writes P as bf16 over the first 64 columns of S (scaling and
 // row sums in packed f32x2 pairs, row maxima with three-operand max); then
 // O += P V_j reads P from tensor memory (A operand in TMEM, V in its TMA layout as
 // an MN-major B), the fastest measured form for that product.
@@ -116,21 +120,22 @@ struct Cursor {
     }
 };
 
-// TMEM: S [0,128) with P written over its first BLK/2 columns, O [128,256).
-// Shared memory: Q, one K and one V buffer (block 128) or two of each (block 64).
+// TMEM: S [0,128) with P written over its first 64 columns, O [128,256).
+// Shared memory: Q, one K and one V tile of 128 keys.
 template <int BLK>
 struct Cfg {
     static constexpr int HPT = 128 / BLK;
-    static constexpr int STAGES = BLK == 128 ? 1 : 2;
+    static constexpr int TK = 128;                 // keys per tile
+    static constexpr int STAGES = 1;
     static constexpr int Q_BYTES = 128 * kD * 2;
-    static constexpr int KV_BYTES = BLK * kD * 2;
-    static constexpr int KV_HALF = BLK * 128;
+    static constexpr int KV_BYTES = TK * kD * 2;
+    static constexpr int KV_HALF = TK * 128;
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_K = OFF_Q + Q_BYTES;
     static constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
     static constexpr int SMEM = OFF_V + STAGES * KV_BYTES;
     static constexpr uint32_t T_S = 0, T_O = 128;
-    static constexpr uint32_t IDESC_S = idesc_bf16(128, BLK, false);
+    static constexpr uint32_t IDESC_S = idesc_bf16(128, TK, false);
     static constexpr uint32_t IDESC_O = idesc_bf16(128, kD, true);
 };
 
@@ -243,6 +248,21 @@ __global__ void __launch_bounds__(kThreads, 2)
             return cur.next(j, mask, a.err, report);
         }
     };
+    // the next key tile: one kept block (block 128), or two consecutive blocks of the
+    // walk (block 64; when one is left, jb = ja with no row keeping it, which keeps
+    // the tile's V rows finite for the masked, zero-weight columns)
+    auto next_tile = [&](int &ja, uint32_t &ma, int &jb, uint32_t &mb, bool report) -> bool {
+        if (!next(ja, ma, report)) return false;
+        jb = ja;
+        mb = 0u;
+        if constexpr (BLK == 64) {
+            if (!next(jb, mb, report)) {
+                jb = ja;
+                mb = 0u;
+            }
+        }
+        return true;
+    };
     if (warp == 4) {
         if (lane == 0) {
             prefetch_tmap(&tq);
@@ -262,20 +282,29 @@ __global__ void __launch_bounds__(kThreads, 2)
                 prefetch_tmap(&tkp);
                 prefetch_tmap(&tvp);
             }
-            int j;
-            uint32_t mask;
-            for (int n = 0; next(j, mask, true); ++n) {
+            int j, jb;
+            uint32_t mask, mb;
+            // tile rows [0, BLK) from block j, [BLK, 128) from block jb (block 64);
+            // an earlier segment's block comes from the permuted copy
+            auto load_tile = [&](unsigned char *dst, const CUtensorMap *m, const CUtensorMap *mp,
+                                 uint64_t *bar) {
+                const CUtensorMap *ma_ = j < seg0 ? mp : m;
+                tma_load_2d(dst, ma_, bar, 0, kv_row0 + j * BLK);
+                tma_load_2d(dst + C::KV_HALF, ma_, bar, 64, kv_row0 + j * BLK);
+                if constexpr (BLK == 64) {
+                    const CUtensorMap *mb_ = jb < seg0 ? mp : m;
+                    tma_load_2d(dst + 64 * 128, mb_, bar, 0, kv_row0 + jb * 64);
+                    tma_load_2d(dst + C::KV_HALF + 64 * 128, mb_, bar, 64, kv_row0 + jb * 64);
+                }
+            };
+            for (int n = 0; next_tile(j, mask, jb, mb, true); ++n) {
                 const int s = n % ST;
                 const uint32_t ph = (n / ST) & 1;
                 unsigned char *kt = smem + C::OFF_K + s * C::KV_BYTES;
                 unsigned char *vt = smem + C::OFF_V + s * C::KV_BYTES;
                 if (!mbar_wait(&empty_k[s], ph ^ 1, a.err)) break;
-                const bool perm_src = j < seg0;        // an earlier segment: permuted copy
-                const CUtensorMap *mk = perm_src ? &tkp : &tk;
-                const CUtensorMap *mv = perm_src ? &tvp : &tv;
                 mbar_arrive_expect_tx(&full_k[s], C::KV_BYTES);
-                tma_load_2d(kt, mk, &full_k[s], 0, kv_row0 + j * BLK);
-                tma_load_2d(kt + C::KV_HALF, mk, &full_k[s], 64, kv_row0 + j * BLK);
+                load_tile(kt, &tk, &tkp, &full_k[s]);
                 if constexpr (ES) {
                     if (n > 0) {
                         if (!mbar_wait(&decided[(n - 1) & 1], ((n - 1) >> 1) & 1, a.err)) break;
@@ -287,8 +316,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 }
                 if (!mbar_wait(&empty_v[s], ph ^ 1, a.err)) break;
                 mbar_arrive_expect_tx(&full_v[s], C::KV_BYTES);
-                tma_load_2d(vt, mv, &full_v[s], 0, kv_row0 + j * BLK);
-                tma_load_2d(vt + C::KV_HALF, mv, &full_v[s], 64, kv_row0 + j * BLK);
+                load_tile(vt, &tv, &tvp, &full_v[s]);
             }
         }
     } else if (warp == 5) {
@@ -296,8 +324,8 @@ __global__ void __launch_bounds__(kThreads, 2)
             cur.init(a, b, h0, i, false);
             const uint32_t q_base = smem_u32(smem + C::OFF_Q);
             bool ok = mbar_wait(&bar_q, 0, a.err);
-            int n = 0, j;
-            uint32_t mask;
+            int n = 0, j, jb;
+            uint32_t mask, mb;
             auto issue_pv = [&](int m) -> bool {
                 const int s = m % ST;
                 if (!mbar_wait(&p_ready, m & 1, a.err)) return false;
@@ -305,7 +333,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 tc_fence_after();
                 const uint32_t v_base = smem_u32(smem + C::OFF_V + s * C::KV_BYTES);
 #pragma unroll
-                for (int kk = 0; kk < BLK / 16; ++kk) {
+                for (int kk = 0; kk < C::TK / 16; ++kk) {
                     const uint64_t bd = sw128_desc(v_base + kk * 2048, C::KV_HALF, 1024);
                     tc_mma_ts(tmem + C::T_O, tmem + C::T_S + kk * 8, bd, C::IDESC_O,
                               (m > 0 || kk > 0) ? 1u : 0u);
@@ -314,7 +342,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 return true;
             };
             bool stopped = false;
-            while (ok && next(j, mask, false)) {
+            while (ok && next_tile(j, mask, jb, mb, false)) {
                 if (n > 0 && !issue_pv(n - 1)) { ok = false; break; }
                 if (ES && *reinterpret_cast<volatile int *>(&stop_at) <= n - 1) {
                     stopped = true;   // P(n - 1) V was the last product
@@ -345,30 +373,41 @@ __global__ void __launch_bounds__(kThreads, 2)
         const uint32_t t_s = tmem + C::T_S + lane_off, t_o = tmem + C::T_O + lane_off;
         cur.init(a, b, h0, i, false);
         float m_used = -INFINITY, l = 0.f;
-        int n = 0, j;
-        uint32_t mask;
+        int n = 0, j, jb;
+        uint32_t mask, mb;
         bool ok = true;
-        while (next(j, mask, false)) {
+        constexpr int TK = C::TK;
+        while (next_tile(j, mask, jb, mb, false)) {
             if (!mbar_wait(&s_full, n & 1, a.err)) { ok = false; break; }
             tc_fence_after();
-            float x[BLK];
+            float x[TK];
 #pragma unroll
-            for (int c = 0; c < BLK / 32; ++c) tmem_ld32f(t_s + c * 32, x + c * 32);
+            for (int c = 0; c < TK / 32; ++c) tmem_ld32f(t_s + c * 32, x + c * 32);
             tc_wait_ld();
+            // columns [0, BLK) belong to block j, [BLK, 128) to block jb (block 64):
+            // a column is kept if the row's head kept its block, the key is not
+            // after the row (diagonal block) and lies inside the sequence
             const bool keep = (mask >> rg) & 1u;
-            const bool whole = keep && j != i && (j + 1) * BLK <= a.L;
+            const bool keep_b = BLK == 64 && ((mb >> rg) & 1u);
+            const int jl = BLK == 64 ? jb : j;        // the tile's last block
+            const bool whole = keep && (BLK == 128 || keep_b) && jl != i && (jl + 1) * BLK <= a.L;
             if (!whole) {
-                const int lim = (j == i) ? rr : BLK - 1;
-                const int lim_t = min(lim, a.L - 1 - j * BLK);
+                const int lim_t = min((j == i) ? rr : BLK - 1, a.L - 1 - j * BLK);
 #pragma unroll
                 for (int c = 0; c < BLK; ++c) x[c] = (keep && c <= lim_t) ? x[c] : -INFINITY;
+                if constexpr (BLK == 64) {
+                    const int lim_b = min((jb == i) ? rr : 63, a.L - 1 - jb * 64);
+#pragma unroll
+                    for (int c = 0; c < 64; ++c)
+                        x[64 + c] = (keep_b && c <= lim_b) ? x[64 + c] : -INFINITY;
+                }
             }
             // Row maximum: eight independent chains of three-operand maxima.
             float mp[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) mp[e] = fmaxf(x[e], x[e + 8]);
 #pragma unroll
-            for (int c = 16; c < BLK; c += 16)
+            for (int c = 16; c < TK; c += 16)
 #pragma unroll
                 for (int e = 0; e < 8; ++e) mp[e] = fmax3(mp[e], x[c + e], x[c + 8 + e]);
             const float mx = fmax3(fmax3(mp[0], mp[1], mp[2]), fmax3(mp[3], mp[4], mp[5]),
@@ -401,7 +440,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 }
             }
 #pragma unroll
-            for (int c = 0; c < BLK / 32; ++c) {
+            for (int c = 0; c < TK / 32; ++c) {
                 uint32_t w[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
