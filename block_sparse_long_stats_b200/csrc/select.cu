@@ -778,9 +778,145 @@ __global__ void __launch_bounds__(kThreads, 2) decode_score_kernel(SelectArgs a)
     }
 }
 
+// Decode scoring on INT4 records with the tensor cores (bf16 queries, d = 128).
+// The scores' contractions are exact there: a 4-bit code is a small integer, exact
+// in bf16; a bf16 query times a code is exact in the fp32 accumulator; q^2 has at
+// most 16 significant bits and splits exactly into two bf16 parts (hi + lo). So
+// per 32-feature group one m16n8k16 pair gives sum q * code and two pairs give
+// sum q^2 * code, each multiplied by the group's power-of-two scale (exact) and
+// added up in fp32: the same sums as the CUDA-core form, in another order. A warp
+// takes 16 candidates (the MMA rows) against the group's G <= 8 query heads (the
+// columns): thread (g, t) = (lane / 4, lane % 4) holds candidates g and g + 8 and
+// heads 2t, 2t + 1 of the result. Codes become bf16 pairs without a conversion:
+// 128 + n is bf16 0x4300 | n, and one packed subtraction removes 128 (136 for the
+// signed mean codes, stored as n ^ 8 = code + 8).
+__device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+// Byte t of w: two codes (features 2c, 2c + 1) as exact bf16 values.
+__device__ __forceinline__ uint32_t codes_bf16x2(uint32_t w, int t, bool is_signed) {
+    const uint32_t b = (w >> (8 * t)) & 0xFFu;
+    const uint32_t flip = is_signed ? 0x00080008u : 0u;
+    const uint32_t packed = (0x43004300u | (b & 0xFu) | ((b >> 4) << 16)) ^ flip;
+    const uint32_t bias = is_signed ? 0x43084308u : 0x43004300u;   // 136 or 128
+    uint32_t r;
+    asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(packed), "r"(bias));
+    return r;
+}
+
+template <int G>
+__global__ void __launch_bounds__(kThreads, 2) decode_score_q_mma_kernel(SelectArgs a) {
+    constexpr int D = 128, RB = D + D / 16;   // record bytes
+    static_assert(G >= 1 && G <= 8, "the heads are the 8 MMA columns");
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int gq = lane >> 2, t = lane & 3;
+    const int bg = blockIdx.y, b = bg / a.Hkv, g = bg % a.Hkv;
+    // B fragments of q, q^2 hi and q^2 lo for head gq (zero past the group's heads):
+    // k-step ks covers features 16 ks .. 16 ks + 15; b0 holds 2t, 2t + 1, b1 + 8
+    uint32_t bq[8][2], bh[8][2], bl[8][2];
+    {
+        const __nv_bfloat16 *qrow =
+            reinterpret_cast<const __nv_bfloat16 *>(a.q) + ((size_t)b * a.Hq + g * G + gq) * D;
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                uint32_t w = 0u, wh = 0u, wl = 0u;
+                if (gq < G) {
+                    w = *reinterpret_cast<const uint32_t *>(qrow + 16 * ks + 8 * h + 2 * t);
+                    const float q0 = bf16lo(w), q1 = bf16hi(w);
+                    const float s0 = q0 * q0, s1 = q1 * q1;          // exact in fp32
+                    wh = pack_bf16x2(s0, s1);
+                    wl = pack_bf16x2(s0 - bf16lo(wh), s1 - bf16hi(wh));
+                }
+                bq[ks][h] = w;
+                bh[ks][h] = wh;
+                bl[ks][h] = wl;
+            }
+    }
+    const float hs2 = 0.5f * a.scale * a.scale;
+    const uint8_t *qb = a.qstats + (size_t)bg * a.nb * RB;
+    float *rows = reinterpret_cast<float *>(a.idx) + ((size_t)b * a.Hq + g * G) * a.cap;
+    const int j0 = blockIdx.x * kDecTile;
+#pragma unroll 1
+    for (int it = 0; it < kDecTile / (kWarps * 16); ++it) {
+        const int base = j0 + (it * kWarps + warp) * 16;
+        if (base >= a.nb) break;                                   // warp-uniform
+        const int ca = min(base + gq, a.nb - 1), cb = min(base + gq + 8, a.nb - 1);
+        const uint8_t *ra = qb + (size_t)ca * RB, *rb = qb + (size_t)cb * RB;
+        const uint2 ea = __ldg(reinterpret_cast<const uint2 *>(ra + D));   // 4 + 4 exponents
+        const uint2 eb = __ldg(reinterpret_cast<const uint2 *>(rb + D));
+        float dot[4] = {0.f, 0.f, 0.f, 0.f}, quad[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int gr = 0; gr < 4; ++gr) {
+            // records are 136 bytes apart, so only 8-byte alignment holds: two 8-byte
+            // loads per 16-byte group of codes
+            auto ld16 = [](const uint8_t *p_) {
+                const uint2 lo = __ldg(reinterpret_cast<const uint2 *>(p_));
+                const uint2 hi = __ldg(reinterpret_cast<const uint2 *>(p_) + 1);
+                return make_uint4(lo.x, lo.y, hi.x, hi.y);
+            };
+            const uint4 ma = ld16(ra + 16 * gr), mb = ld16(rb + 16 * gr);
+            const uint4 va = ld16(ra + D / 2 + 16 * gr), vb = ld16(rb + D / 2 + 16 * gr);
+            float pd[4] = {0.f, 0.f, 0.f, 0.f}, pq[4] = {0.f, 0.f, 0.f, 0.f};
+            // k-step 2 gr: features 0..15 of the group (words x, y); 2 gr + 1: 16..31 (z, w)
+            mma16816(pd, codes_bf16x2(ma.x, t, true), codes_bf16x2(mb.x, t, true),
+                     codes_bf16x2(ma.y, t, true), codes_bf16x2(mb.y, t, true), bq[2 * gr][0],
+                     bq[2 * gr][1]);
+            mma16816(pd, codes_bf16x2(ma.z, t, true), codes_bf16x2(mb.z, t, true),
+                     codes_bf16x2(ma.w, t, true), codes_bf16x2(mb.w, t, true), bq[2 * gr + 1][0],
+                     bq[2 * gr + 1][1]);
+            const uint32_t v0 = codes_bf16x2(va.x, t, false), v1 = codes_bf16x2(vb.x, t, false);
+            const uint32_t v2 = codes_bf16x2(va.y, t, false), v3 = codes_bf16x2(vb.y, t, false);
+            const uint32_t v4 = codes_bf16x2(va.z, t, false), v5 = codes_bf16x2(vb.z, t, false);
+            const uint32_t v6 = codes_bf16x2(va.w, t, false), v7 = codes_bf16x2(vb.w, t, false);
+            mma16816(pq, v0, v1, v2, v3, bh[2 * gr][0], bh[2 * gr][1]);
+            mma16816(pq, v0, v1, v2, v3, bl[2 * gr][0], bl[2 * gr][1]);
+            mma16816(pq, v4, v5, v6, v7, bh[2 * gr + 1][0], bh[2 * gr + 1][1]);
+            mma16816(pq, v4, v5, v6, v7, bl[2 * gr + 1][0], bl[2 * gr + 1][1]);
+            // the group's scales 2^k (rows gq: candidate ca, rows gq + 8: cb)
+            const int kma = (int8_t)((ea.x >> (8 * gr)) & 0xFFu), kmb = (int8_t)((eb.x >> (8 * gr)) & 0xFFu);
+            const int kva = (int8_t)((ea.y >> (8 * gr)) & 0xFFu), kvb = (int8_t)((eb.y >> (8 * gr)) & 0xFFu);
+            const float sma = __int_as_float((kma + 127) << 23), smb = __int_as_float((kmb + 127) << 23);
+            const float sva = __int_as_float((kva + 127) << 23), svb = __int_as_float((kvb + 127) << 23);
+            dot[0] = fmaf(pd[0], sma, dot[0]);
+            dot[1] = fmaf(pd[1], sma, dot[1]);
+            dot[2] = fmaf(pd[2], smb, dot[2]);
+            dot[3] = fmaf(pd[3], smb, dot[3]);
+            quad[0] = fmaf(pq[0], sva, quad[0]);
+            quad[1] = fmaf(pq[1], sva, quad[1]);
+            quad[2] = fmaf(pq[2], svb, quad[2]);
+            quad[3] = fmaf(pq[3], svb, quad[3]);
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int hh = 2 * t + (e & 1);
+            const int j = base + gq + (e >> 1) * 8;
+            if (hh < G && j < a.nb)
+                rows[(size_t)hh * a.cap + j] =
+                    log_score(dot[e], quad[e], a.scale, hs2, min(a.block, a.T - j * a.block));
+        }
+    }
+}
+
 template <typename T, int D, bool QS>
 cudaError_t launch_decode_scores(const SelectArgs &a, cudaStream_t s) {
     dim3 grid((unsigned)((a.nb + kDecTile - 1) / kDecTile), (unsigned)(a.B * a.Hkv));
+    if constexpr (QS && D == 128 && sizeof(T) == 2) {
+        // INT4 records with bf16 queries: the tensor-core form
+        switch (a.G) {
+            case 1: decode_score_q_mma_kernel<1><<<grid, kThreads, 0, s>>>(a); break;
+            case 2: decode_score_q_mma_kernel<2><<<grid, kThreads, 0, s>>>(a); break;
+            case 4: decode_score_q_mma_kernel<4><<<grid, kThreads, 0, s>>>(a); break;
+            default: decode_score_q_mma_kernel<8><<<grid, kThreads, 0, s>>>(a); break;
+        }
+        return cudaGetLastError();
+    }
     switch (a.G) {
         case 1: decode_score_kernel<T, D, 1, QS><<<grid, kThreads, 0, s>>>(a); break;
         case 2: decode_score_kernel<T, D, 2, QS><<<grid, kThreads, 0, s>>>(a); break;
