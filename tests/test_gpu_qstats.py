@@ -81,6 +81,26 @@ def test_select_quantized_on_oracle_records(key):
     assert spa.spa_get_device_error() == 0
 
 
+@pytest.mark.parametrize("Hq,Hkv", [(2, 2), (4, 2), (8, 1), (16, 2)])
+def test_select_quantized_decode_head_groupings(Hq, Hkv):
+    # decode scoring on records runs on the tensor cores with the group's heads as
+    # the MMA columns: one, two, eight (all columns) and eight heads per kv-head
+    # (the four-head case is the parity workload above); a ragged candidate tile
+    w = PARITY_WORKLOADS["d_bf16_blk16"].with_(Hq=Hq, Hkv=Hkv, T=16 * 300 + 5)
+    x, dev = inputs(w)
+    sel = oracle.select_quantized(x["q"], x["k"], w.dtype, w.block, w.scale, w.top_p, w.n_sink,
+                                  w.n_local, w.k_min)
+    rec = torch.from_numpy(pack_qstats(sel["q"])).cuda()
+    idx, cnt = spa.spa_select_quantized(dev["q"], rec, w.T, w.block, w.scale, w.top_p, w.n_sink,
+                                        w.n_local, w.k_min)
+    torch.cuda.synchronize()
+    r = compare_lists(idx.cpu().numpy(), cnt.cpu().numpy(), sel["idx"], sel["count"],
+                      sel["scores"], w.top_p, w.n_sink, w.n_local, w.Lq, w.T, w.block)
+    print(f"\nG={Hq // Hkv}: {r['units']} lists, {r['equal']} equal, {r['excused']} excused")
+    assert not r["unexcused"], r["unexcused"][:3]
+    assert spa.spa_get_device_error() == 0
+
+
 def test_select_quantized_rule_variants():
     w = PARITY_WORKLOADS["d_bf16_blk16"]
     x, dev = inputs(w)
