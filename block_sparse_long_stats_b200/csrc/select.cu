@@ -689,10 +689,12 @@ __global__ void __launch_bounds__(kThreads, 3) select_group_kernel(SelectArgs a)
 
 // Decode scoring: CTA (tile, b*Hkv + g) scores kDecTile candidate blocks for all
 // G query heads of kv-head g, so each block's statistics are read once per group
-// (the step reads the statistics exactly once: HBM-bound). Warp per candidate,
-// lanes over d, four candidates in flight per warp; lane h writes head h's fp32
-// score into that head's row of idx, used as scratch (decode rows hold exactly
-// cap >= nb entries) until the cut kernel replaces it with the kept list.
+// (the step reads the statistics exactly once: HBM-bound). Lanes over d; a warp
+// takes U candidates per pass, their U x G (dot, variance term) partial sums
+// reduced together by one transposing reduction, and loads the next pass's
+// statistics before reducing the current one. The fp32 scores go into each head's
+// row of idx, used as scratch (decode rows hold exactly cap >= nb entries) until
+// the cut kernel replaces it with the kept list.
 constexpr int kDecTile = 256;
 
 template <typename T, int D, int G, bool QS>
