@@ -1,7 +1,8 @@
 """CPU oracle for selection-driven block-sparse causal attention (fp64).
 
 TEST INFRASTRUCTURE ONLY. Only ``tests/``, ``__graft_entry__.smoke()`` and the
-CPU-baseline leg of ``bench.py`` may import this package. It shares no code with
+CPU-baseline and reference (oracle-timing) legs of ``bench.py`` may import this
+package. It shares no code with
 the CUDA path and never imports it; the CUDA path never imports this.
 
 The arithmetic lives in ``spa_oracle.c`` (plain C loops, fp64, OpenMP over

@@ -3,7 +3,8 @@
  *
  * TEST INFRASTRUCTURE ONLY. This file is the plain, slow, fp64 statement of what
  * the CUDA path computes. Only the tests, the smoke check and the benchmark's CPU
- * baseline leg may load it; the library path never does. It shares no code with
+ * baseline and reference (oracle-timing) legs may load it; the library path never
+ * does. It shares no code with
  * the CUDA sources and includes none of their headers.
  *
  * Sources (the pages are web summaries of five papers on block-sparse attention):
