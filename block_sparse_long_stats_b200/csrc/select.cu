@@ -517,6 +517,116 @@ __global__ void __launch_bounds__(kThreads) select_kernel(SelectArgs a) {
     write_ascending(flag, a, unit, jmax, itot, &isum);
 }
 
+constexpr int kCtaSortMax = 1024;   // residuals up to this many: sort across the CTA
+
+// Up to kThreads * KPL residual keys of one head sorted across the CTA: thread tid
+// holds positions KPL tid .. KPL tid + KPL - 1; strides below KPL are register
+// compare-exchanges, strides within a warp's span xor shuffles, the larger ones go
+// through two shared-memory buffers (xbuf, 2 kThreads KPL keys) with one barrier
+// each. Then the same cut as warp_sort_cut (fp64 masses, exclusive prefix in rank
+// order over the CTA, K_min floor), writing the kept blocks' flags (fl) or, in
+// traversal order, the whole list. Called by every thread of the CTA.
+template <int KPL>
+__device__ void cta_sort_cut(const uint64_t *keys, uint64_t *xbuf, unsigned char *fl,
+                             const SelectArgs &a, size_t unit, int nres, int r_lo, int r_hi,
+                             int jmax, double *dtot, double *dsum, int *itot, int *isum,
+                             uint64_t *first) {
+    constexpr int N = kThreads * KPL;
+    constexpr int LOGN = ilog2(N);
+    const int tid = threadIdx.x, lane = tid & 31;
+    uint64_t k[KPL];
+#pragma unroll
+    for (int e = 0; e < KPL; ++e) {
+        const int x = tid * KPL + e;
+        k[e] = x < nres ? keys[x] : ~0ull;
+    }
+    int pb = 0;
+#pragma unroll
+    for (int lk = 1; lk <= LOGN; ++lk) {
+        const int kk = 1 << lk;
+#pragma unroll
+        for (int lj = lk - 1; lj >= 0; --lj) {
+            const int jj = 1 << lj;
+            if (jj < KPL) {
+#pragma unroll
+                for (int e = 0; e < KPL; ++e) {
+                    if ((e & jj) == 0) {
+                        const bool up = ((tid * KPL + e) & kk) == 0;
+                        const uint64_t x = k[e], y = k[e | jj];
+                        const bool sw = (x > y) == up;
+                        k[e] = sw ? y : x;
+                        k[e | jj] = sw ? x : y;
+                    }
+                }
+            } else if (jj < 32 * KPL) {
+                const int lm = jj / KPL;
+                const bool lower = (lane & lm) == 0;
+#pragma unroll
+                for (int e = 0; e < KPL; ++e) {
+                    const bool up = ((tid * KPL + e) & kk) == 0;
+                    const uint64_t o = __shfl_xor_sync(0xffffffffu, k[e], lm);
+                    const uint64_t mn = k[e] < o ? k[e] : o, mx = k[e] < o ? o : k[e];
+                    k[e] = lower == up ? mn : mx;
+                }
+            } else {
+                uint64_t *bw = xbuf + pb * N;
+#pragma unroll
+                for (int e = 0; e < KPL; ++e) bw[tid * KPL + e] = k[e];
+                __syncthreads();
+                const bool lower = ((tid * KPL) & jj) == 0;
+#pragma unroll
+                for (int e = 0; e < KPL; ++e) {
+                    const bool up = ((tid * KPL + e) & kk) == 0;
+                    const uint64_t o = bw[(tid * KPL + e) ^ jj];
+                    const uint64_t mn = k[e] < o ? k[e] : o, mx = k[e] < o ? o : k[e];
+                    k[e] = lower == up ? mn : mx;
+                }
+                pb ^= 1;
+            }
+        }
+    }
+    int nk = nres;
+    if (nres > 0 && a.top_p < 1.0f) {
+        if (tid == 0) *first = k[0];                // the largest score
+        __syncthreads();
+        const double mx = (double)key_score(*first);
+        double m[KPL], local = 0.0;
+#pragma unroll
+        for (int e = 0; e < KPL; ++e) {
+            m[e] = tid * KPL + e < nres ? exp((double)key_score(k[e]) - mx) : 0.0;
+            local += m[e];
+        }
+        double cum = block_exclusive_scan<double>(local, dtot, dsum);
+        const double total = *dsum;
+        const double p = (double)a.top_p;
+        int kept = 0;
+#pragma unroll
+        for (int e = 0; e < KPL; ++e) {
+            if (tid * KPL + e < nres && cum / total < p) ++kept;
+            cum += m[e];
+        }
+        block_exclusive_scan<int>(kept, itot, isum);
+        nk = *isum;
+    }
+    nk = max(nk, min(a.k_min, nres));
+    if (a.score_order) {
+        int32_t *out = a.idx + unit * a.cap;
+        const int nloc = jmax + 1 - r_hi;
+        for (int x = tid; x < nloc; x += kThreads) out[x] = jmax - x;
+        for (int x = tid; x < r_lo; x += kThreads) out[nloc + x] = x;
+#pragma unroll
+        for (int e = 0; e < KPL; ++e) {
+            const int x = tid * KPL + e;
+            if (x < nk) out[nloc + r_lo + x] = (int)(uint32_t)k[e];
+        }
+        if (tid == 0) a.count[unit] = nloc + r_lo + nk;
+    } else {
+#pragma unroll
+        for (int e = 0; e < KPL; ++e)
+            if (tid * KPL + e < nk) fl[(int)(uint32_t)k[e]] = 1;
+    }
+}
+
 // Grouped prefill selection: one CTA (256 threads) per (b, kv-head g, query block)
 // serves the G query heads of the group, so every candidate's statistics are read
 // once for all of them. Same rule and arithmetic as select_kernel: fp32 pooled
@@ -537,9 +647,19 @@ __global__ void __launch_bounds__(kThreads, 3) select_group_kernel(SelectArgs a)
     static_assert(RG >= 1, "pooling layout");
     __shared__ float qs[G][D];
     __shared__ float red[G][RG][D];
-    __shared__ uint64_t keys[G][kWarpSortMax];
+    __shared__ double dtot[kWarps];
+    __shared__ double dsum;
+    __shared__ int itot[kWarps];
+    __shared__ int isum;
+    __shared__ uint64_t first_key;
+    // dynamic: keys [G][kcap], then (more than kWarpSortMax residuals) the sort's two
+    // exchange buffers [2][kcap], then flags [G][nb]
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    unsigned char *flags = smem_raw;                // [G][nb]
+    const int kcap = a.sort_cap <= kWarpSortMax ? kWarpSortMax : a.sort_cap;
+    uint64_t *keys = reinterpret_cast<uint64_t *>(smem_raw);
+    uint64_t *xbuf = keys + (size_t)G * kcap;
+    unsigned char *flags = reinterpret_cast<unsigned char *>(
+        xbuf + (a.sort_cap <= kWarpSortMax ? 0 : 2 * (size_t)kcap));
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int i = a.nq - 1 - (int)blockIdx.x;       // heaviest query blocks first
@@ -649,11 +769,29 @@ __global__ void __launch_bounds__(kThreads, 3) select_group_kernel(SelectArgs a)
             if (kk < G && (lane & ((1 << LB) - 1)) == 0 && r < nres) {
                 const int j = r_lo + r;
                 const float l = log_score(tot, quad, a.scale, hs2, min(a.block, a.T - j * a.block));
-                keys[kk][r] = ((uint64_t)order_desc(l) << 32) | (uint32_t)j;
+                keys[(size_t)kk * kcap + r] = ((uint64_t)order_desc(l) << 32) | (uint32_t)j;
             }
         }
     }
     __syncthreads();
+
+    if (kcap > kWarpSortMax) {
+        // ---- more than kWarpSortMax candidates: head by head, sorted across the CTA
+        for (int hh = 0; hh < G; ++hh) {
+            const size_t unit = ((size_t)b * a.Hq + g * G + hh) * a.nq + i;
+            unsigned char *fl = flags + (size_t)hh * a.nb;
+            if (kcap <= 512)
+                cta_sort_cut<2>(keys + (size_t)hh * kcap, xbuf, fl, a, unit, nres, r_lo, r_hi,
+                                jmax, dtot, &dsum, itot, &isum, &first_key);
+            else
+                cta_sort_cut<4>(keys + (size_t)hh * kcap, xbuf, fl, a, unit, nres, r_lo, r_hi,
+                                jmax, dtot, &dsum, itot, &isum, &first_key);
+            __syncthreads();
+            if (!a.score_order) write_ascending(fl, a, unit, jmax, itot, &isum);
+            __syncthreads();
+        }
+        return;
+    }
 
     // ---- warp h: sort, cut and list of head h
     if (warp < G) {
@@ -661,10 +799,11 @@ __global__ void __launch_bounds__(kThreads, 3) select_group_kernel(SelectArgs a)
         const size_t unit = ((size_t)b * a.Hq + h) * a.nq + i;
         unsigned char *fl = flags + (size_t)warp * a.nb;
         const int N = nres <= 32 ? 32 : nres <= 64 ? 64 : nres <= 128 ? 128 : 256;
-        if (N == 32) warp_sort_cut<1>(keys[warp], fl, a, unit, nres, r_lo, r_hi, jmax, lane);
-        else if (N == 64) warp_sort_cut<2>(keys[warp], fl, a, unit, nres, r_lo, r_hi, jmax, lane);
-        else if (N == 128) warp_sort_cut<4>(keys[warp], fl, a, unit, nres, r_lo, r_hi, jmax, lane);
-        else warp_sort_cut<8>(keys[warp], fl, a, unit, nres, r_lo, r_hi, jmax, lane);
+        const uint64_t *kw = keys + (size_t)warp * kcap;
+        if (N == 32) warp_sort_cut<1>(kw, fl, a, unit, nres, r_lo, r_hi, jmax, lane);
+        else if (N == 64) warp_sort_cut<2>(kw, fl, a, unit, nres, r_lo, r_hi, jmax, lane);
+        else if (N == 128) warp_sort_cut<4>(kw, fl, a, unit, nres, r_lo, r_hi, jmax, lane);
+        else warp_sort_cut<8>(kw, fl, a, unit, nres, r_lo, r_hi, jmax, lane);
         if (!a.score_order) {
             __syncwarp();
             // ascending list: lane l takes flags [l per, (l + 1) per), warp scan of counts
@@ -1191,7 +1330,9 @@ cudaError_t allow_smem(K kern, size_t dyn) {
 
 template <typename T, int D, int G, bool QS>
 cudaError_t launch_group(const SelectArgs &a, cudaStream_t s) {
-    const size_t smem = (size_t)G * a.nb;
+    const size_t kcap = a.sort_cap <= kWarpSortMax ? kWarpSortMax : a.sort_cap;
+    const size_t smem = (size_t)G * kcap * 8 + (a.sort_cap <= kWarpSortMax ? 0 : 2 * kcap * 8) +
+                        (size_t)G * a.nb;
     auto kern = select_group_kernel<T, D, G, QS>;
     cudaError_t e = allow_smem(kern, smem);
     if (e != cudaSuccess) return e;
@@ -1201,9 +1342,9 @@ cudaError_t launch_group(const SelectArgs &a, cudaStream_t s) {
 
 template <typename T, int D, bool QS>
 cudaError_t launch_tq(const SelectArgs &a, cudaStream_t s) {
-    // prefill, up to kWarpSortMax residual candidates, a head grouping the grouped
+    // prefill, up to kCtaSortMax residual candidates, a head grouping the grouped
     // kernel has: one CTA per kv-head and query block
-    if (!a.prescored && a.sort_cap <= kWarpSortMax) {
+    if (!a.prescored && a.sort_cap <= kCtaSortMax) {
         switch (a.G) {
             case 1: return launch_group<T, D, 1, QS>(a, s);
             case 2: return launch_group<T, D, 2, QS>(a, s);
