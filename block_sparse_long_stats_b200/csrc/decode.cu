@@ -530,10 +530,15 @@ cudaError_t launch_b(const CUtensorMap &tk, const CUtensorMap &tv, const DecodeA
 
 }  // namespace
 
+constexpr int kDecodeWaves = 9;
+
 int decode_splits(int B, int Hkv, int T, int block) {
     const int nb = (T + block - 1) / block;
     const int groups = B * Hkv;
-    int splits = (148 * 16 + groups - 1) / groups;
+    // resident CTAs (three per SM at block 16, one otherwise); the grid is sized to
+    // end just under a whole number of waves, so the last wave is not a sliver
+    const int slots = 148 * (block == 16 ? 3 : 1);
+    int splits = (slots * kDecodeWaves) / groups;
     const int max_splits = (nb + 15) / 16;          // at least 16 blocks per split
     if (splits > max_splits) splits = max_splits;
     if (splits < 1) splits = 1;
