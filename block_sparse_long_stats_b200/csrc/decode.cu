@@ -531,14 +531,18 @@ cudaError_t launch_b(const CUtensorMap &tk, const CUtensorMap &tv, const DecodeA
 }  // namespace
 
 constexpr int kDecodeWaves = 9;
+constexpr int kMinSplitBlocks = 64;
 
 int decode_splits(int B, int Hkv, int T, int block) {
     const int nb = (T + block - 1) / block;
     const int groups = B * Hkv;
     // resident CTAs (three per SM at block 16, one otherwise); the grid is sized to
-    // end just under a whole number of waves, so the last wave is not a sliver
+    // end just under a whole number of waves, so the last wave is not a sliver, with
+    // at most kDecodeWaves waves and at least kMinSplitBlocks blocks per split
     const int slots = 148 * (block == 16 ? 3 : 1);
-    int splits = (slots * kDecodeWaves) / groups;
+    const long work = (long)groups * nb;
+    const int waves = (int)std::max(1L, std::min<long>(kDecodeWaves, work / ((long)slots * kMinSplitBlocks)));
+    int splits = (slots * waves) / groups;
     const int max_splits = (nb + 15) / 16;          // at least 16 blocks per split
     if (splits > max_splits) splits = max_splits;
     if (splits < 1) splits = 1;
