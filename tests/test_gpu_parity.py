@@ -219,6 +219,44 @@ def test_decode_matches_oracle(key):
     assert_no_device_error()
 
 
+@pytest.mark.parametrize("Hq,Hkv,block,T", [(2, 2, 16, 1000), (8, 1, 32, 777), (16, 1, 128, 1500),
+                                            (6, 2, 64, 3000), (16, 2, 16, 129)])
+def test_decode_random_lists_groupings_and_edges(Hq, Hkv, block, T):
+    # Lists the selection would never write: random subsets, an empty list (the
+    # output is zero, as the oracle's), every block, the sink alone, the last block
+    # alone; G = 1, 3, 8 and 16 query heads per kv-head; ragged and one-token tails.
+    w = PARITY_WORKLOADS["d_bf16_blk16"].with_(Hq=Hq, Hkv=Hkv, block=block, T=T, B=2)
+    x, dev = inputs(w)
+    rng = np.random.default_rng(Hq * 1000 + block)
+    idx = np.full((w.B, w.Hq, 1, w.nb), -1, np.int32)
+    cnt = np.zeros((w.B, w.Hq, 1), np.int32)
+    for b in range(w.B):
+        for h in range(w.Hq):
+            kind = (b * w.Hq + h) % 5
+            if kind == 0:
+                keep = []
+            elif kind == 1:
+                keep = list(range(w.nb))
+            elif kind == 2:
+                keep = [0]
+            elif kind == 3:
+                keep = [w.nb - 1]
+            else:
+                keep = [j for j in range(w.nb) if rng.random() < 0.3]
+            idx[b, h, 0, :len(keep)] = keep
+            cnt[b, h, 0] = len(keep)
+    out = spa.spa_sparse_attn_decode(dev["q"], dev["k"], dev["v"], w.block,
+                                     torch.from_numpy(idx).cuda(), torch.from_numpy(cnt).cuda(),
+                                     w.scale)
+    torch.cuda.synchronize()
+    o_out, _ = oracle.attention(x["q"], x["k"], x["v"], w.dtype, w.block, idx, cnt, w.scale)
+    g = to_host(out)
+    assert np.abs(g - o_out).max() <= TOL[w.dtype]
+    empty = cnt[:, :, 0] == 0
+    assert (g[empty] == 0).all()
+    assert_no_device_error()
+
+
 def test_corrupt_lists_are_reported_and_skipped():
     w = PARITY_WORKLOADS["p_bf16_blk128"]
     x, dev = inputs(w)
