@@ -40,6 +40,7 @@ constexpr int kThreads = 192;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
+constexpr size_t kL2ResidentBytes = size_t(48) << 20;   // about 40 % of the 126 MB L2
 
 struct PrefillArgs {
     const int32_t *idx;
@@ -57,6 +58,10 @@ struct PrefillArgs {
     // segment-permuted layout: blocks before the query's own segment come from the
     // permuted K/V copies (tkp, tvp); 0: off
     int seg_blocks;
+    // CTA order: 1 = (b, kv-head)-major, the query blocks heaviest first inside each
+    // kv-head (one kv-head's K and V resident in L2 at a time); 0 = heaviest query
+    // blocks first across all heads (when every kv-head's K and V fit in L2 together)
+    int kv_major;
 };
 
 // Walks the ascending kept lists of the HPT heads of a tile in merged order. All
@@ -170,12 +175,23 @@ __global__ void __launch_bounds__(kThreads, 2)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     // (b, kv-head)-major, query blocks heaviest first inside each: the CTAs resident
-    // at a time share one kv-head's K and V tiles, which then stay in L2
-    const int per_bg = a.nq * a.npairs;
-    const int bg = (int)(blockIdx.x / per_bg);
-    const int rest = (int)(blockIdx.x % per_bg);
-    const int i = a.nq - 1 - rest / a.npairs;
-    const int hp = rest % a.npairs;
+    // at a time share one kv-head's K and V tiles, which then stay in L2. With all
+    // K and V in L2 at once, heaviest query blocks first across every head instead,
+    // so the last kv-head's long CTAs do not start at the end of the launch.
+    int bg, i, hp;
+    if (a.kv_major) {
+        const int per_bg = a.nq * a.npairs;
+        bg = (int)(blockIdx.x / per_bg);
+        const int rest = (int)(blockIdx.x % per_bg);
+        i = a.nq - 1 - rest / a.npairs;
+        hp = rest % a.npairs;
+    } else {
+        const int per_i = a.B * a.Hkv * a.npairs;
+        i = a.nq - 1 - (int)(blockIdx.x / per_i);
+        const int rest = (int)(blockIdx.x % per_i);
+        bg = rest / a.npairs;
+        hp = rest % a.npairs;
+    }
     const int b = bg / a.Hkv, g = bg % a.Hkv;
     const int h0 = g * a.G + hp * HPT;
 
@@ -546,7 +562,11 @@ cudaError_t launch_blk(const void *q, const void *k, const void *v, const Prefil
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)((size_t)a.nq * a.B * a.Hkv * a.npairs);
-    kern<<<grid, kThreads, smem, s>>>(mq, mk, mv, mkp, mvp, a);
+    // K and V (and their permuted copies) of every kv-head against half the L2
+    PrefillArgs a2 = a;
+    const size_t kv_bytes = (size_t)kv_rows * kD * 2 * 2 * (kp ? 2 : 1);
+    a2.kv_major = kv_bytes > kL2ResidentBytes ? 1 : 0;
+    kern<<<grid, kThreads, smem, s>>>(mq, mk, mv, mkp, mvp, a2);
     return cudaGetLastError();
 }
 
