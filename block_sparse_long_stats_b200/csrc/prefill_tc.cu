@@ -168,6 +168,10 @@ __global__ void __launch_bounds__(kThreads, 2)
         o_done;
     __shared__ uint32_t tmem_slot;
     __shared__ uint64_t decided[2];
+    // the MMA thread publishes each tile's blocks and row masks here for the
+    // softmax warps (two slots; info_full[s] completes once per use of slot s)
+    __shared__ uint64_t info_full[2];
+    __shared__ int4 tinfo[2];
     __shared__ int n_list, stop_at;
     __shared__ float es_max[2][4];
     int32_t *list_s = reinterpret_cast<int32_t *>(smem + C::SMEM);          // ES: [nq]
@@ -208,6 +212,8 @@ __global__ void __launch_bounds__(kThreads, 2)
         mbar_init(&o_done, 1);
         mbar_init(&decided[0], 1);
         mbar_init(&decided[1], 1);
+        mbar_init(&info_full[0], 1);
+        mbar_init(&info_full[1], 1);
         stop_at = 0x7fffffff;
         fence_mbar_init();
     }
@@ -358,7 +364,14 @@ __global__ void __launch_bounds__(kThreads, 2)
                 return true;
             };
             bool stopped = false;
-            while (ok && next_tile(j, mask, jb, mb, false)) {
+            while (ok) {
+                const bool more = next_tile(j, mask, jb, mb, false);
+                if constexpr (!ES) {
+                    // slot n & 1 last held tile n - 2, read before P(n - 2) was ready
+                    tinfo[n & 1] = more ? make_int4(j, (int)mask, jb, (int)mb) : make_int4(-1, 0, 0, 0);
+                    mbar_arrive(&info_full[n & 1]);
+                }
+                if (!more) break;
                 if (n > 0 && !issue_pv(n - 1)) { ok = false; break; }
                 if (ES && *reinterpret_cast<volatile int *>(&stop_at) <= n - 1) {
                     stopped = true;   // P(n - 1) V was the last product
@@ -387,13 +400,23 @@ __global__ void __launch_bounds__(kThreads, 2)
         const int t = i * BLK + rr;
         const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
         const uint32_t t_s = tmem + C::T_S + lane_off, t_o = tmem + C::T_O + lane_off;
-        cur.init(a, b, h0, i, false);
         float m_used = -INFINITY, l = 0.f;
         int n = 0, j, jb;
         uint32_t mask, mb;
         bool ok = true;
         constexpr int TK = C::TK;
-        while (next_tile(j, mask, jb, mb, false)) {
+        for (;;) {
+            if constexpr (ES) {
+                if (!next_tile(j, mask, jb, mb, false)) break;
+            } else {
+                if (!mbar_wait(&info_full[n & 1], (n >> 1) & 1, a.err)) { ok = false; break; }
+                const int4 ti = tinfo[n & 1];
+                if (ti.x < 0) break;
+                j = ti.x;
+                mask = (uint32_t)ti.y;
+                jb = ti.z;
+                mb = (uint32_t)ti.w;
+            }
             if (!mbar_wait(&s_full, n & 1, a.err)) { ok = false; break; }
             tc_fence_after();
             float x[TK];
