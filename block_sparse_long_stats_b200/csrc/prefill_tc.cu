@@ -64,9 +64,10 @@ struct PrefillArgs {
     int kv_major;
 };
 
-// Walks the ascending kept lists of the HPT heads of a tile in merged order. All
-// roles run identical cursors, so they agree on the block sequence; entries that
-// are out of range or not ascending are skipped (and reported by one role).
+// Walks the ascending kept lists of the HPT heads of a tile in merged order. The
+// producer and the MMA thread run identical cursors, so they agree on the block
+// sequence (the MMA thread hands it on to the softmax warps); entries that are out
+// of range or not ascending are skipped (and reported by the producer).
 template <int HPT>
 struct Cursor {
     const int32_t *lst[HPT];
