@@ -200,7 +200,9 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int b = bg / a.Hkv, g = bg % a.Hkv;
     const int h0 = g * a.G + hp * HPT;
 
-    if (tid == 0) {
+    // The producer thread initialises the barriers and starts the Q tile at once, so
+    // its copy overlaps the TMEM allocation and (early stop) the list validation.
+    if (tid == 128) {
         mbar_init(&bar_q, 1);
         for (int s = 0; s < ST; ++s) {
             mbar_init(&full_k[s], 1);
@@ -217,6 +219,17 @@ __global__ void __launch_bounds__(kThreads, 2)
         mbar_init(&info_full[1], 1);
         stop_at = 0x7fffffff;
         fence_mbar_init();
+        fence_async_shared();
+        prefetch_tmap(&tq);
+        prefetch_tmap(&tk);
+        prefetch_tmap(&tv);
+        mbar_arrive_expect_tx(&bar_q, C::Q_BYTES);
+#pragma unroll
+        for (int r = 0; r < HPT; ++r) {
+            const int row = ((b * a.Hq + h0 + r) * a.L) + i * BLK;
+            tma_load_2d(smem + C::OFF_Q + r * BLK * 128, &tq, &bar_q, 0, row);
+            tma_load_2d(smem + C::OFF_Q + 16384 + r * BLK * 128, &tq, &bar_q, 64, row);
+        }
     }
     if (warp == 5) tmem_alloc(&tmem_slot, 256);
     if constexpr (ES) {
@@ -288,16 +301,6 @@ __global__ void __launch_bounds__(kThreads, 2)
     };
     if (warp == 4) {
         if (lane == 0) {
-            prefetch_tmap(&tq);
-            prefetch_tmap(&tk);
-            prefetch_tmap(&tv);
-            mbar_arrive_expect_tx(&bar_q, C::Q_BYTES);
-#pragma unroll
-            for (int r = 0; r < HPT; ++r) {
-                const int row = ((b * a.Hq + h0 + r) * a.L) + i * BLK;
-                tma_load_2d(smem + C::OFF_Q + r * BLK * 128, &tq, &bar_q, 0, row);
-                tma_load_2d(smem + C::OFF_Q + 16384 + r * BLK * 128, &tq, &bar_q, 64, row);
-            }
             cur.init(a, b, h0, i, true);
             const int kv_row0 = (b * a.Hkv + g) * a.L;
             const int seg0 = a.seg_blocks > 0 ? (i / a.seg_blocks) * a.seg_blocks : 0;
