@@ -287,7 +287,9 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int b = bg / Hkv, g = bg % Hkv, h = g * a.G + rest % a.G;
     const size_t unit = ((size_t)b * a.Hq + h) * a.nq + i;
 
-    if (tid == 0) {
+    // The producer thread initialises the barriers and starts the Q tile at once, so
+    // its copy overlaps the kept-bitmap build below.
+    if (tid == kProducerWarp * 32) {
         mbar_init(&bar_q, 1);
         mbar_init(&q_ready, 128);
         for (int s = 0; s < ST; ++s) {
@@ -301,6 +303,13 @@ __global__ void __launch_bounds__(kThreads, 2)
         mbar_init(&p_ready, 128);
         mbar_init(&acc_done, 1);
         fence_mbar_init();
+        fence_async_shared();
+        prefetch_tmap(&tq);
+        prefetch_tmap(&tw);
+        mbar_arrive_expect_tx(&bar_q, 2 * BLK * 128);
+        const int qrow = (b * a.Hq + h) * a.L + i * BLK;
+        tma_load_2d(smem + C::OFF_Q, &tq, &bar_q, 0, qrow);
+        tma_load_2d(smem + C::OFF_Q + 16384, &tq, &bar_q, 64, qrow);
     }
     if (warp < 4)
         for (int w = tid; w < a.nwords; w += 128) bits[w] = 0u;
@@ -372,12 +381,6 @@ __global__ void __launch_bounds__(kThreads, 2)
 
     if (warp == kProducerWarp) {
         if (lane == 0) {
-            prefetch_tmap(&tq);
-            prefetch_tmap(&tw);
-            mbar_arrive_expect_tx(&bar_q, 2 * BLK * 128);
-            const int qrow = (b * a.Hq + h) * a.L + i * BLK;
-            tma_load_2d(smem + C::OFF_Q, &tq, &bar_q, 0, qrow);
-            tma_load_2d(smem + C::OFF_Q + 16384, &tq, &bar_q, 64, qrow);
             ResidualIter it;
             it.init(bits, i);
             const int wblk0 = (b * a.Hkv + g) * a.nq;     // first state block of (b, g)
