@@ -12,9 +12,9 @@
  *                       exponential feature map over the blocks left out
  *
  * Conventions shared by every call
- *   - All tensors are dense, contiguous, row-major, in DEVICE memory, allocated and
- *     owned by the caller. The library allocates nothing and keeps no per-call
- *     state; it never frees or retains caller pointers.
+ *   - All tensors are dense, contiguous, row-major, in DEVICE memory (spa_prefill_host:
+ *     host memory), allocated and owned by the caller. The library allocates no
+ *     memory and keeps no per-call state; it never frees or retains caller pointers.
  *   - Layouts: Q [B, Hq, Lq, d]; K, V [B, Hkv, T, d]; block statistics
  *     [B, Hkv, nb, d]; kept lists [B, Hq, nq, cap] (int32) with counts
  *     [B, Hq, nq] (int32), where nb = ceil(T / block), nq = ceil(Lq / block).
@@ -405,6 +405,9 @@ spa_status spa_sparse_attn_decode_rla(const void *q, const void *kc, const void 
  * copy or launch; SPA_ERR_CUDA if a copy or launch fails to enqueue (the work
  * enqueued before it stays enqueued: synchronise `stream` before reusing the
  * buffers).
+ * State: the three streams and their events are created on the first call on a
+ * device and kept for the process (the one exception to "no state" above); calls
+ * from several host threads are serialised by a lock.
  */
 size_t spa_prefill_host_workspace_bytes(spa_dtype dt, int B, int Hq, int Hkv, int L, int d,
                                         int block);
