@@ -46,6 +46,17 @@ int *device_error_ptr() {
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
+// One warp waits on a barrier that nothing completes: the bounded wait runs out
+// after limit_ns and records SPA_DEVERR_TIMEOUT (the failure path of every kernel).
+__global__ void selftest_wait_kernel(int *err, uint64_t limit_ns) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+        mbar_wait(&bar, 0, err, limit_ns);
+    }
+}
+
 }  // namespace
 
 int *device_error_word() { return device_error_ptr(); }
@@ -510,6 +521,18 @@ SPA_API spa_status spa_sparse_attn_decode_rla(const void *q, const void *kc, con
                                   out_rla);
     if (e == cudaErrorNotSupported) return fail(SPA_ERR_UNSUPPORTED, "tensor map encoding unavailable");
     return e == cudaSuccess ? SPA_OK : cuda_fail(e, "decode launch");
+}
+
+SPA_API spa_status spa_selftest_wait_timeout(int limit_us, spa_stream stream) {
+    t_last_error.clear();
+    if (limit_us < 1 || limit_us > 1000000)
+        return fail(SPA_ERR_INVALID, "limit_us must be in [1, 1000000]");
+    int *err = device_error_ptr();
+    if (!err) return fail(SPA_ERR_CUDA, "device error word unavailable");
+    selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+        err, (uint64_t)limit_us * 1000ull);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? SPA_OK : cuda_fail(e, "self-test launch");
 }
 
 SPA_API spa_status spa_get_device_error(int *code) {

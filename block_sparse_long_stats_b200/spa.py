@@ -16,7 +16,7 @@ import torch
 __all__ = ["SpaError", "lib", "spa_block_stats", "spa_select", "spa_sparse_attn_prefill",
            "spa_decode_workspace_bytes", "spa_sparse_attn_decode", "spa_get_device_error",
            "spa_status_string", "spa_last_error", "prefill", "decode", "LIB_PATH",
-           "spa_prefill_host", "spa_prefill_host_workspace_bytes"]
+           "spa_prefill_host", "spa_prefill_host_workspace_bytes", "spa_selftest_wait_timeout"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libspa.so")
 
@@ -82,6 +82,7 @@ def lib() -> ctypes.CDLL:
         L.spa_prefill_host.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _F, _I, _I,
                                        _I, _P, ctypes.c_size_t, _P]
         L.spa_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_int)]
+        L.spa_selftest_wait_timeout.argtypes = [_I, _P]
         L.spa_status_string.argtypes = [_I]
         L.spa_status_string.restype = ctypes.c_char_p
         L.spa_last_error.restype = ctypes.c_char_p
@@ -90,7 +91,8 @@ def lib() -> ctypes.CDLL:
                   "spa_rla_prefill", "spa_rla_decode_state", "spa_sparse_attn_decode_rla",
                   "spa_quantize_block_stats", "spa_select_quantized", "spa_select_score_order",
                   "spa_sparse_attn_prefill_early_stop", "spa_pbs_permutation", "spa_pbs_gather",
-                  "spa_select_segperm", "spa_sparse_attn_prefill_segperm", "spa_prefill_host"):
+                  "spa_select_segperm", "spa_sparse_attn_prefill_segperm", "spa_prefill_host",
+                  "spa_selftest_wait_timeout"):
             getattr(L, f).restype = _I
         _lib = L
     return _lib
@@ -477,6 +479,12 @@ def spa_sparse_attn_decode(q: torch.Tensor, kc: torch.Tensor, vc: torch.Tensor, 
                                         block, _ptr(idx), idx.shape[-1], _ptr(count), scale,
                                         _ptr(workspace), _ptr(out), _stream(stream)))
     return out
+
+
+def spa_selftest_wait_timeout(limit_us: int, stream=None) -> None:
+    """Enqueues the bounded-wait self-test: a wait that nothing completes runs out
+    after limit_us and records SPA_DEVERR_TIMEOUT (read it with spa_get_device_error)."""
+    _check("spa_selftest_wait_timeout", lib().spa_selftest_wait_timeout(limit_us, _stream(stream)))
 
 
 def spa_get_device_error() -> int:

@@ -423,6 +423,18 @@ spa_status spa_prefill_host(const void *q, const void *k, const void *v, void *o
  */
 spa_status spa_get_device_error(int *code);
 
+/*
+ * Self-test of the failure path that every kernel's waits share: one warp waits on
+ * a shared-memory mbarrier that nothing ever completes, through the same bounded
+ * wait the kernels use, with a limit of limit_us microseconds (1 .. 1,000,000). The
+ * wait runs out, records SPA_DEVERR_TIMEOUT in the device error word, and the
+ * kernel returns, leaving the context usable. Asynchronous on `stream`; read the
+ * outcome with spa_get_device_error.
+ * Errors: SPA_ERR_INVALID for a limit outside that range; SPA_ERR_CUDA if the
+ * launch fails.
+ */
+spa_status spa_selftest_wait_timeout(int limit_us, spa_stream stream);
+
 /* Static description of a status code. */
 const char *spa_status_string(spa_status status);
 

@@ -61,6 +61,15 @@ def _last(lib):
     return lib.spa_last_error().decode()
 
 
+def test_selftest_wait_limit_host_checks(lib):
+    f = lib.spa_selftest_wait_timeout
+    f.argtypes = [ctypes.c_int, P]
+    assert f(0, None) == 1
+    assert f(-5, None) == 1
+    assert f(1000001, None) == 1
+    assert "limit_us" in _last(lib)
+
+
 def test_block_stats_host_checks(lib):
     f = lib.spa_block_stats
     f.argtypes = [P] + [ctypes.c_int] * 8 + [P, P, P]

@@ -257,6 +257,24 @@ def test_decode_random_lists_groupings_and_edges(Hq, Hkv, block, T):
     assert_no_device_error()
 
 
+def test_bounded_wait_runs_out_and_reports_timeout():
+    # The failure path every kernel's waits share: a barrier that nothing completes.
+    # The wait gives up after its limit, records the timeout in the device error
+    # word, and the context stays usable for the next launch.
+    assert spa.spa_get_device_error() == 0
+    spa.spa_selftest_wait_timeout(2000)
+    assert spa.spa_get_device_error() == 3      # SPA_DEVERR_TIMEOUT
+    assert spa.spa_get_device_error() == 0      # reading clears it
+    w = PARITY_WORKLOADS["p_bf16_blk128"]
+    x, dev = inputs(w)
+    mean, var = spa.spa_block_stats(dev["k"], w.block)
+    torch.cuda.synchronize()
+    om, ov = oracle.block_stats(x["k"], w.dtype, w.block)
+    np.testing.assert_allclose(mean.cpu().numpy(), om, rtol=1e-5, atol=1e-6)
+    np.testing.assert_allclose(var.cpu().numpy(), ov, rtol=1e-5, atol=1e-6)
+    assert_no_device_error()
+
+
 def test_corrupt_lists_are_reported_and_skipped():
     w = PARITY_WORKLOADS["p_bf16_blk128"]
     x, dev = inputs(w)
