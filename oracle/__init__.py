@@ -57,7 +57,7 @@ def _bind(path: str):
     lib.oracle_rla_block_states.argtypes = [_P, _P, _I, _I, _I, _I, _I, _I, _P]
     lib.oracle_early_stop.argtypes = [_P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _I, _P, _D, _I,
                                       _I, _D, _P, _P]
-    lib.oracle_pbs_permutation.argtypes = [_P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P]
+    lib.oracle_pbs_permutation.argtypes = [_P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _D, _P, _P]
     lib.oracle_attention_segperm.argtypes = [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P,
                                              _I, _P, _D, _P, _I64, _P, _P]
     lib.oracle_quantize_stats.argtypes = [_P, _P, _I, _I, _I, _I, _P, _P, _P, _P]
@@ -329,17 +329,22 @@ def early_stop(q, k, dtype: str, block: int, idx: np.ndarray, count: np.ndarray,
     return processed, ratios
 
 
-def pbs_permutation(q, k, dtype: str, block: int, seg_blocks: int) -> np.ndarray:
-    """Segmented key permutation (PBS, sections 2-3; reading in spa_oracle.c):
-    perm [B, Hkv, L] int32, the original index of the key at each permuted position."""
+def pbs_permutation(q, k, dtype: str, block: int, seg_blocks: int, scale: float,
+                    return_importance: bool = False):
+    """Segmented key permutation (PBS, sections 2-3; reading in spa_oracle.c): keys
+    sorted inside each segment by the mean-pooled causal softmax weights of the last
+    query block's rows (all query heads of the kv-group).
+    Returns perm [B, Hkv, L] int32, the original index of the key at each permuted
+    position, and with ``return_importance`` also the fp64 importance [B, Hkv, L]."""
     q, isb = _inp(q, dtype)
     k, _ = _inp(k, dtype)
     B, Hq, L, d = q.shape
     Hkv = k.shape[1]
     perm = np.empty((B, Hkv, L), np.int32)
+    imp = np.empty((B, Hkv, L), np.float64)
     _check(_load().oracle_pbs_permutation(_ptr(q), _ptr(k), isb, B, Hq, Hkv, L, d, block, seg_blocks,
-                                          _ptr(perm)), "pbs_permutation")
-    return perm
+                                          float(scale), _ptr(perm), _ptr(imp)), "pbs_permutation")
+    return (perm, imp) if return_importance else perm
 
 
 def permute(x: np.ndarray, perm: np.ndarray) -> np.ndarray:
@@ -353,7 +358,7 @@ def select_segperm(q, k, dtype: str, block: int, seg_blocks: int, scale: float, 
     of earlier segments on the permuted keys' statistics and the blocks of its own
     segment on the original ones; then the same cut."""
     if perm is None:
-        perm = pbs_permutation(q, k, dtype, block, seg_blocks)
+        perm = pbs_permutation(q, k, dtype, block, seg_blocks, scale)
     kp = permute(np.asarray(k), perm)
     mean, var = block_stats(k, dtype, block)
     mp, vp = block_stats(kp, dtype, block)

@@ -688,11 +688,20 @@ int oracle_early_stop(const void *q, const void *k, int is_bf16, int B, int Hq, 
  * sections 2-3). The keys (with their values) are divided into segments of
  * seg_blocks * block tokens and sorted inside each segment by a global importance
  * score, descending; segments keep their order, so causality between segments is
- * untouched. Reading of the score: the mean pooling of the attention scores of the
- * last query block, taken on the logits: importance(u) = qbar . k_u, with qbar the
- * mean of the last query block's rows over the query heads of the kv-group (the
- * positive softmax scale does not change the order). Equal scores keep the smaller
- * index first. perm[b, g, p] = the original index of the key at permuted position p.
+ * untouched.
+ *
+ * The importance (section 3, proxy scoring): the attention scores of the last
+ * query block, mean-pooled. For every query head h of the kv-group and every row t
+ * of the last query block, the causal softmax row
+ *     a_{h,t}(u) = exp(s q_{h,t} . k_u) / sum_{u' <= t} exp(s q_{h,t} . k_u')   (u <= t)
+ * and a_{h,t}(u) = 0 for u > t (a key after the row is masked, as in attention);
+ *     importance(u) = (1 / (G n_r)) sum_h sum_t a_{h,t}(u)
+ * over the G query heads of the group and the n_r rows of the last block. Each row
+ * is evaluated as the textbook softmax (row maximum, exponentials, their sum,
+ * division). The order is decided on the importance rounded to fp32 (the kernel's
+ * precision); equal values keep the smaller index first.
+ * perm[b, g, p] = the original index of the key at permuted position p;
+ * importance (nullable) [B, Hkv, L] receives the fp64 importance.
  */
 typedef struct { double score; int idx; } imp_t;
 
@@ -705,10 +714,11 @@ static int imp_cmp(const void *a, const void *b)
 }
 
 int oracle_pbs_permutation(const void *q, const void *k, int is_bf16, int B, int Hq, int Hkv,
-                           int L, int d, int block, int seg_blocks, int32_t *perm)
+                           int L, int d, int block, int seg_blocks, double scale, int32_t *perm,
+                           double *importance)
 {
     if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || L <= 0 || d <= 0 || block <= 0 ||
-        seg_blocks <= 0)
+        seg_blocks <= 0 || !(scale > 0.0))
         return ORACLE_EINVAL;
     const int G = Hq / Hkv, nq = ceil_div(L, block), S = seg_blocks * block;
     const int r0 = (nq - 1) * block, nr = L - r0;
@@ -716,24 +726,44 @@ int oracle_pbs_permutation(const void *q, const void *k, int is_bf16, int B, int
 #pragma omp parallel for schedule(dynamic, 1)
     for (int bg = 0; bg < B * Hkv; ++bg) {
         const int b = bg / Hkv, g = bg % Hkv;
-        double *qbar = (double *)calloc((size_t)d, sizeof(double));
+        double *acc = (double *)calloc((size_t)L, sizeof(double));
+        double *z = (double *)malloc(sizeof(double) * (size_t)L);
         imp_t *imp = (imp_t *)malloc(sizeof(imp_t) * (size_t)L);
-        if (!qbar || !imp) {
+        if (!acc || !z || !imp) {
 #pragma omp atomic write
             err = ORACLE_ENOMEM;
-            free(qbar);
+            free(acc);
+            free(z);
             free(imp);
             continue;
         }
-        for (int hh = 0; hh < G; ++hh)
-            for (int r = 0; r < nr; ++r)
-                for (int c = 0; c < d; ++c)
-                    qbar[c] += elem(q, is_bf16, (((size_t)b * Hq + g * G + hh) * L + r0 + r) * d + c);
-        for (int c = 0; c < d; ++c) qbar[c] /= (double)(G * nr);
+        /* attention scores of every row of the last query block, one softmax per row */
+        for (int hh = 0; hh < G; ++hh) {
+            for (int r = 0; r < nr; ++r) {
+                const int t = r0 + r;
+                const int n_seen = t + 1;          /* causal: keys 0..t */
+                const size_t qoff = (((size_t)b * Hq + g * G + hh) * L + t) * d;
+                double m = -INFINITY;
+                for (int u = 0; u < n_seen; ++u) {
+                    double s = 0.0;
+                    for (int c = 0; c < d; ++c)
+                        s += elem(q, is_bf16, qoff + c) * elem(k, is_bf16, ((size_t)bg * L + u) * d + c);
+                    z[u] = s * scale;    /* the attention's logit */
+                    if (z[u] > m) m = z[u];
+                }
+                double den = 0.0;
+                for (int u = 0; u < n_seen; ++u) {
+                    z[u] = exp(z[u] - m);
+                    den += z[u];
+                }
+                for (int u = 0; u < n_seen; ++u) acc[u] += z[u] / den;
+            }
+        }
+        /* mean pooling over the G * nr rows */
         for (int u = 0; u < L; ++u) {
-            double s = 0.0;
-            for (int c = 0; c < d; ++c) s += qbar[c] * elem(k, is_bf16, ((size_t)bg * L + u) * d + c);
-            imp[u].score = s;
+            const double mean = acc[u] / (double)(G * nr);
+            if (importance) importance[(size_t)bg * L + u] = mean;
+            imp[u].score = (double)(float)mean;
             imp[u].idx = u;
         }
         for (int s0 = 0; s0 < L; s0 += S) {
@@ -741,7 +771,8 @@ int oracle_pbs_permutation(const void *q, const void *k, int is_bf16, int B, int
             qsort(imp + s0, (size_t)n, sizeof(imp_t), imp_cmp);
         }
         for (int p = 0; p < L; ++p) perm[(size_t)bg * L + p] = imp[p].idx;
-        free(qbar);
+        free(acc);
+        free(z);
         free(imp);
     }
     return err;

@@ -82,10 +82,26 @@ MUTATIONS = [
     ("segperm_ascending_importance", "if (x->score > y->score) return -1;\n    if (x->score < y->score) return 1;",
      "if (x->score < y->score) return -1;\n    if (x->score > y->score) return 1;",
      [pins.test_segperm_hand_worked_permutation,
-      pins.test_segperm_sorts_each_segment_by_pooled_query_logit]),
+      pins.test_segperm_importance_sums_to_one_and_sorts_each_segment]),
     ("segperm_pooled_over_the_first_block", "const int r0 = (nq - 1) * block, nr = L - r0;",
      "const int r0 = 0, nr = block < L ? block : L;",
-     [pins.test_segperm_sorts_each_segment_by_pooled_query_logit]),
+     [pins.test_segperm_hand_worked_permutation,
+      pins.test_segperm_importance_at_vanishing_scale_is_uniform_causal,
+      pins.test_segperm_importance_reads_only_its_groups_last_block]),
+    ("segperm_logit_proxy", "acc[u] += z[u] / den;", "acc[u] += log(z[u]);",
+     [pins.test_segperm_hand_worked_permutation,
+      pins.test_segperm_importance_sums_to_one_and_sorts_each_segment]),
+    ("segperm_unnormalised_rows", "acc[u] += z[u] / den;", "acc[u] += z[u];",
+     [pins.test_segperm_hand_worked_permutation,
+      pins.test_segperm_importance_sums_to_one_and_sorts_each_segment]),
+    ("segperm_rows_see_later_keys", "const int n_seen = t + 1;", "const int n_seen = L;",
+     [pins.test_segperm_hand_worked_permutation,
+      pins.test_segperm_importance_at_vanishing_scale_is_uniform_causal]),
+    ("segperm_dropped_scale", "z[u] = s * scale;    /* the attention's logit */", "z[u] = s;",
+     [pins.test_segperm_importance_at_vanishing_scale_is_uniform_causal]),
+    ("segperm_heads_of_another_group", "(((size_t)b * Hq + g * G + hh) * L + t) * d",
+     "(((size_t)b * Hq + hh) * L + t) * d",
+     [pins.test_segperm_importance_reads_only_its_groups_last_block]),
     ("segperm_earlier_keys_by_original_block", "kept[inv[u] / block]", "kept[u / block]",
      [pins.test_segperm_attention_in_the_permuted_layout]),
     ("ascending_sort", "if (x->key > y->key) return -1;\n    if (x->key < y->key) return 1;",

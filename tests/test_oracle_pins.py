@@ -827,30 +827,110 @@ def test_score_order_lists_are_the_kept_sets_in_rank_order():
         assert all((s32[x], -ranked[x]) >= (s32[x + 1], -ranked[x + 1]) for x in range(len(s32) - 1))
 
 
+def test_score_order_overlapping_sink_and_local_ranges():
+    # S2O, section 2 (the dense local pass first) with SpotAttention's reserved
+    # ranges: where the sink range [0, n_sink) and the local range [i - n_local + 1, i]
+    # overlap, the overlap belongs to the sink, as in the cut. n_sink = n_local = 2,
+    # full lists, worked out by hand: i = 0 -> [0]; i = 1 -> [0, 1] (block 1 lies in
+    # the sink range); i = 2 -> [2, 0, 1]; i = 3 -> [3, 2, 0, 1]; i = 4 -> the local
+    # blocks 4, 3, the sink 0, 1, then the ranked block 2.
+    nq, blk = 5, 4
+    idx, cnt = oracle.full_lists(1, 1, nq * blk, nq * blk, blk)
+    l = np.zeros(idx.shape, np.float64)
+    oi, oc = oracle.score_order({"idx": idx, "count": cnt, "scores": l}, nq * blk, nq * blk, blk,
+                                n_sink=2, n_local=2)
+    assert np.array_equal(oc, cnt)
+    expect = [[0], [0, 1], [2, 0, 1], [3, 2, 0, 1], [4, 3, 0, 1, 2]]
+    for i in range(nq):
+        assert oi[0, 0, i, :cnt[0, 0, i]].tolist() == expect[i]
+
+
 # ---------------------------------------------------------------- segmented key permutation
 # PBS (Sparsere Blok-Sparse Attention via Tokenpermutatie), sections 2-3: keys sorted
 # by global importance inside segments; segments keep their causal order.
 
 def test_segperm_hand_worked_permutation():
+    # Section 3 (proxy scoring): the mean-pooled softmax rows of the last query
+    # block, worked out in closed form; the logit, unnormalised and first-block
+    # readings each give another order on this input (derivation in the golden file).
     g = _golden()["segmented_permutation"]
-    q = np.array(g["q"], np.float32).reshape(1, 1, -1, 1)
-    k = np.array(g["k"], np.float32).reshape(1, 1, -1, 1)
-    perm = oracle.pbs_permutation(q, k, "f32", g["block"], g["seg_blocks"])
+    q = np.array(g["q"], np.float32)[None, None]
+    k = np.array(g["k"], np.float32)[None, None]
+    perm, imp = oracle.pbs_permutation(q, k, "f32", g["block"], g["seg_blocks"], g["scale"],
+                                       return_importance=True)
+    np.testing.assert_allclose(imp.reshape(-1), g["expected_importance"], rtol=1e-12, atol=0)
     assert perm.reshape(-1).tolist() == g["expected_perm"]
 
 
-def test_segperm_sorts_each_segment_by_pooled_query_logit():
-    B, Hq, Hkv, L, d, blk, seg = 1, 4, 2, 96, 8, 8, 3
-    q, k = _rand((B, Hq, L, d), 90), _rand((B, Hkv, L, d), 91)
-    perm = oracle.pbs_permutation(q, k, "f32", blk, seg)
-    G, S = Hq // Hkv, seg * blk
-    for g in range(Hkv):
-        qbar = q[0, g * G:(g + 1) * G, L - blk:].astype(np.float64).reshape(-1, d).mean(0)
-        imp = k[0, g].astype(np.float64) @ qbar
+def _segperm_case(seed, L=90, blk=8, Hq=4, Hkv=2, d=8):
+    # L = 90: the last query block is ragged (2 rows)
+    return _rand((1, Hq, L, d), seed), _rand((1, Hkv, L, d), seed + 1), blk
+
+
+def test_segperm_importance_sums_to_one_and_sorts_each_segment():
+    # Every softmax row sums to 1, so their mean does too; each segment is a
+    # permutation of its own keys, in descending importance (equal values: smaller
+    # index first).
+    q, k, blk = _segperm_case(90)
+    seg = 3
+    perm, imp = oracle.pbs_permutation(q, k, "f32", blk, seg, 0.4, return_importance=True)
+    np.testing.assert_allclose(imp.sum(axis=-1), 1.0, rtol=1e-13)
+    assert (imp >= 0).all()
+    L, S = q.shape[2], seg * blk
+    for g in range(k.shape[1]):
+        i32 = imp[0, g].astype(np.float32)
         for s0 in range(0, L, S):
             p = perm[0, g, s0:s0 + S]
-            assert sorted(p.tolist()) == list(range(s0, min(s0 + S, L)))   # within the segment
-            assert all((imp[p[x]], -p[x]) >= (imp[p[x + 1]], -p[x + 1]) for x in range(len(p) - 1))
+            assert sorted(p.tolist()) == list(range(s0, min(s0 + S, L)))
+            assert all((i32[p[x]], -p[x]) >= (i32[p[x + 1]], -p[x + 1]) for x in range(len(p) - 1))
+
+
+def test_segperm_importance_at_vanishing_scale_is_uniform_causal():
+    # As s -> 0 every causal row is uniform over keys 0..t: importance(u) =
+    # (1 / n_rows) sum over the last block's rows t >= u of 1 / (t + 1), the same for
+    # every head. Pins the causal limit and which rows are pooled.
+    q, k, blk = _segperm_case(92)
+    L = q.shape[2]
+    _, imp = oracle.pbs_permutation(q, k, "f32", blk, 2, 1e-12, return_importance=True)
+    r0 = (-(-L // blk) - 1) * blk
+    rows = np.arange(r0, L)
+    ref = np.array([sum(1.0 / (t + 1) for t in rows if t >= u) for u in range(L)]) / rows.size
+    np.testing.assert_allclose(imp[0, 0], ref, rtol=1e-9, atol=1e-15)
+    np.testing.assert_allclose(imp[0, 1], ref, rtol=1e-9, atol=1e-15)
+
+
+def test_segperm_importance_invariant_to_a_per_row_logit_offset():
+    # A key component shared by every key adds q_t[c] to each logit of row t: the
+    # softmax of the row, and so the importance, does not change.
+    q, k, blk = _segperm_case(94)
+    k[..., -1] = 1.0
+    q2 = q.copy()
+    L = q.shape[2]
+    r0 = (-(-L // blk) - 1) * blk
+    q2[:, :, r0:, -1] += np.float32(3.0) * np.arange(1, q.shape[1] * (L - r0) + 1,
+                                                        dtype=np.float32).reshape(q.shape[1], -1)[None]
+    _, a = oracle.pbs_permutation(q, k, "f32", blk, 2, 0.5, return_importance=True)
+    _, b = oracle.pbs_permutation(q2, k, "f32", blk, 2, 0.5, return_importance=True)
+    np.testing.assert_allclose(b, a, rtol=1e-10, atol=1e-15)
+
+
+def test_segperm_importance_reads_only_its_groups_last_block():
+    # kv-group 0 pools heads 0 and 1 (G = 2), over the rows of the last query block
+    # only: queries of the other group, or of earlier rows, change nothing.
+    q, k, blk = _segperm_case(96)
+    L = q.shape[2]
+    r0 = (-(-L // blk) - 1) * blk
+    _, a = oracle.pbs_permutation(q, k, "f32", blk, 2, 0.5, return_importance=True)
+    q2 = q.copy()
+    q2[:, 2:] = _rand(q2[:, 2:].shape, 97)          # the other group's heads
+    q2[:, :2, :r0] = _rand(q2[:, :2, :r0].shape, 98)  # earlier rows of this group
+    _, b = oracle.pbs_permutation(q2, k, "f32", blk, 2, 0.5, return_importance=True)
+    np.testing.assert_array_equal(b[0, 0], a[0, 0])
+    q3 = q.copy()
+    q3[:, 1, L - 1] += 1.0                          # a last-block row of head 1
+    _, c = oracle.pbs_permutation(q3, k, "f32", blk, 2, 0.5, return_importance=True)
+    assert not np.allclose(c[0, 0], a[0, 0], rtol=1e-6, atol=0)
+    np.testing.assert_array_equal(c[0, 1], a[0, 1])
 
 
 def test_segperm_at_p_one_is_dense_causal_attention():
