@@ -104,6 +104,13 @@ def kept_kv_bytes(count: np.ndarray, idx: np.ndarray, G: int, T: int, block: int
     return float(total * d * 2 * 2)
 
 
+def workload_config(w, n_gpus: int) -> dict:
+    """The `config` of the JSON line, identical for the CUDA arm and the reference arm."""
+    return {"workload": w.name, "B": w.B, "L": w.T, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d,
+            "block": w.block, "top_p": w.top_p, "parallelism": f"replicas x{n_gpus}",
+            "l2": "flushed (256 MiB memset) between timed steps"}
+
+
 # ---------------------------------------------------------------- ranks
 
 def max_over_ranks(v: float, world: int, device) -> float:
@@ -217,9 +224,10 @@ def run_reference(args, rank: int):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": w.B * w.Lq / value * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "L": w.T, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d,
-                   "block": w.block, "top_p": w.top_p, "l2": "n/a (CPU)"},
+        "config": workload_config(w, args.gpus),
+        "extrapolated": True,
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "extrapolated": True,
                          "sample": f"per step: stats + selection on the whole {w.name} workload, "
                                    f"masked fp64 attention on {n_tok} random query positions x "
                                    f"{w.Hq} heads; tokens/s = sampled tokens / (their attention "
@@ -231,6 +239,86 @@ def run_reference(args, rank: int):
 
 
 # ---------------------------------------------------------------- CUDA arm
+
+def measure_prefill_workload(spa, torch, cid: int, steps: int, warmup: int, peaks: dict,
+                             peak_src: str, flush, stream, world: int, rank_max, barrier,
+                             device_index: int) -> dict:
+    """One prefill workload timed like the headline step (stats -> select ->
+    attention, inputs resident, L2 flushed between steps, CUDA events per kernel,
+    clocks sampled during the timed region)."""
+    w = WORKLOADS[cid]
+    x = generate(w)
+    if w.dtype == "bf16":
+        conv = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda().view(torch.bfloat16)
+    else:
+        conv = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    q, k, v = conv(x["q"]), conv(x["k"]), conv(x["v"])
+    del x
+    B, Hq, L, d = q.shape
+    Hkv = k.shape[1]
+    nb = -(-L // w.block)
+    mean = torch.empty((B, Hkv, nb, d), device="cuda", dtype=torch.float32)
+    var = torch.empty_like(mean)
+    idx = torch.empty((B, Hq, nb, nb), device="cuda", dtype=torch.int32)
+    cnt = torch.empty((B, Hq, nb), device="cuda", dtype=torch.int32)
+    out = torch.empty_like(q)
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        spa.spa_block_stats(k, w.block, mean=mean, var=var)
+        if ev:
+            ev[1].record(stream)
+        spa.spa_select(q, mean, var, L, w.block, w.scale, w.top_p, w.n_sink, w.n_local, w.k_min,
+                       idx=idx, count=cnt)
+        if ev:
+            ev[2].record(stream)
+        spa.spa_sparse_attn_prefill(q, k, v, w.block, idx, cnt, w.scale, out=out)
+        if ev:
+            ev[3].record(stream)
+
+    for _ in range(warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    assert spa.spa_get_device_error() == 0
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    clocks = ClockSampler(device_index)
+    clocks.start()
+    barrier()
+    torch.cuda.synchronize()
+    for s_ in range(steps):
+        flush.zero_()
+        step(evs[s_])
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    total_ms = rank_max(sum(e[0].elapsed_time(e[3]) for e in evs))
+    t_att = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+    count_h = cnt.cpu().numpy()
+    F = kept_flops(count_h, idx.cpu().numpy(), L, w.block, d)
+    achieved = F / (t_att / 1e3) / 1e12
+    if w.dtype == "bf16":
+        bound, peak = "tensor", peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+        psrc = f"{peak_src} bf16_tflops (burst)"
+    else:
+        # fp32 FFMA on the CUDA cores: 148 SMs x 128 lanes x 2 FLOP per clock
+        mhz = peaks.get("sm_max_mhz", 1965.0)
+        bound, peak = "alu", 148 * 128 * 2 * mhz * 1e6 / 1e12
+        psrc = f"derived: 148 SMs x 128 FP32 lanes x 2 FLOP x {mhz:.0f} MHz"
+    res = {"workload": w.name, "tokens/s": job_throughput(B * L, world, steps, total_ms),
+           "ms_per_step": total_ms / steps, "steps": steps,
+           "block_stats_ms": statistics.mean(e[0].elapsed_time(e[1]) for e in evs),
+           "select_ms": statistics.mean(e[1].elapsed_time(e[2]) for e in evs),
+           "attn_ms": t_att, "kept_flops_per_launch": F, "TFLOP/s": achieved,
+           "bound": bound, "peak": peak, "peak_source": psrc, "frac": achieved / peak,
+           "kept_fraction": float(count_h.sum()) / (B * Hq * nb * (nb + 1) / 2),
+           "clocks": clk}
+    del q, k, v, mean, var, idx, cnt, out
+    torch.cuda.empty_cache()
+    return res
+
+
 
 def prefill_diagnostics(spa, torch, wl, q, k, v) -> dict:
     """Diagnostics of the selection on one prefill workload, from the library's own
@@ -271,8 +359,9 @@ def main():
                     help="override the decode workload's batch (smaller captures for profiling)")
     ap.add_argument("--no-rla", action="store_true",
                     help="skip the Residual Linear Attention leg")
-    ap.add_argument("--tau", type=float, default=0.2,
-                    help="early-stop threshold for the score-ordered traversal leg (0: skip)")
+    ap.add_argument("--taus", default="0.001,0.002,0.005,0.01,0.02",
+                    help="early-stop thresholds swept in the score-ordered traversal leg "
+                         "('' to skip)")
     ap.add_argument("--seg-blocks", type=int, default=16,
                     help="segment length (in blocks) of the segmented-permutation leg (0: skip)")
     ap.add_argument("--no-quant", action="store_true",
@@ -280,6 +369,8 @@ def main():
     ap.add_argument("--no-diagnostics", action="store_true",
                     help="skip the kept-fraction / MSE-vs-dense / coverage diagnostics")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--configs", default="1,2,4",
+                    help="other prefill workloads timed beside the headline one ('' to skip)")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-tokens", type=int, default=1536)
     ap.add_argument("--ref-tokens", type=int, default=48)
@@ -374,7 +465,10 @@ def main():
     F = kept_flops(count_h, idx_h, L, w.block, d)
     att_ms = statistics.mean(t_att)
     achieved = F / (att_ms / 1e3) / 1e12
-    peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    # the timed region is well under a second of back-to-back launches: the burst
+    # peak is the one to compare with (the sustained one is reported beside it)
+    peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    peak_sus = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
     dense_tiles = B * Hq * nb * (nb + 1) / 2
     kept_frac = float(count_h.sum()) / dense_tiles
     stats_bytes = B * Hkv * L * d * 2 + 2 * B * Hkv * nb * d * 4
@@ -459,61 +553,89 @@ def main():
                                                       ms_per_step + t_st + t_rla)}
         del states, rout
 
-    # ---- score-ordered traversal with early stop (S2O, sections 2-3), block 128
+    # ---- score-ordered traversal with early stop (S2O, sections 2-3), block 128:
+    # a sweep of tau, each with its processed fraction, attention time and operator
+    # MSE against dense causal attention; the headline tau is the largest whose MSE
+    # stays within 1.1 x the MSE of the top-p selection alone (the error budget)
     early = None
-    if args.tau > 0 and w.block == 128 and w.dtype == "bf16":
+    taus = [float(t) for t in args.taus.split(",") if t.strip()]
+    if taus and w.block == 128 and w.dtype == "bf16":
         oidx = torch.empty_like(idx)
         ocnt = torch.empty_like(cnt)
         proc = torch.empty_like(cnt)
         eout = torch.empty_like(q)
-
-        def early_step():
-            spa.spa_select_score_order(q, mean, var, w.block, w.scale, w.top_p, w.n_sink,
-                                       w.n_local, w.k_min, idx=oidx, count=ocnt)
-            spa.spa_sparse_attn_prefill_early_stop(q, k, v, w.block, oidx, ocnt, w.scale, args.tau,
-                                                   w.n_sink, w.n_local, out=eout,
-                                                   processed=proc)
-        for _ in range(3):
-            early_step()
+        dense = spa.prefill(q, k, v, w.block, 1.0, w.scale, w.n_sink, w.n_local, w.k_min)["out"]
         torch.cuda.synchronize()
-        assert spa.spa_get_device_error() == 0
+        dense_f = dense.float()
+        dense_ms = float(dense_f.pow(2).mean())
+        mse_topp = float((out.float() - dense_f).pow(2).mean())
+        del dense
+        spa.spa_select_score_order(q, mean, var, w.block, w.scale, w.top_p, w.n_sink,
+                                   w.n_local, w.k_min, idx=oidx, count=ocnt)
         n_es = max(5, args.steps // 4)
-        es_evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_es)]
-        barrier()
-        torch.cuda.synchronize()
+        sweep = []
+        for tau in taus:
+            for _ in range(3):
+                spa.spa_sparse_attn_prefill_early_stop(q, k, v, w.block, oidx, ocnt, w.scale, tau,
+                                                       w.n_sink, w.n_local, out=eout,
+                                                       processed=proc)
+            torch.cuda.synchronize()
+            assert spa.spa_get_device_error() == 0
+            es_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                      for _ in range(n_es)]
+            barrier()
+            torch.cuda.synchronize()
+            for s_ in range(n_es):
+                flush.zero_()
+                es_evs[s_][0].record(stream)
+                spa.spa_sparse_attn_prefill_early_stop(q, k, v, w.block, oidx, ocnt, w.scale, tau,
+                                                       w.n_sink, w.n_local, out=eout,
+                                                       processed=proc)
+                es_evs[s_][1].record(stream)
+            torch.cuda.synchronize()
+            barrier()
+            t_es = rank_max(statistics.mean(a_.elapsed_time(b_) for a_, b_ in es_evs))
+            pr = proc.cpu().numpy()
+            oi = oidx.cpu().numpy()
+            trunc = np.where(np.arange(oi.shape[-1]) < pr[..., None], oi, -1)
+            F_es = kept_flops(pr, np.sort(np.where(trunc < 0, 1 << 30, trunc), axis=-1), L,
+                              w.block, d)
+            mse = float((eout.float() - dense_f).pow(2).mean())
+            sweep.append({"tau": tau,
+                          "processed_fraction": float(pr.sum()) / float(count_h.sum()),
+                          "attn_ms": t_es, "processed_flops": F_es,
+                          "TFLOP/s": F_es / (t_es / 1e3) / 1e12,
+                          "mse_vs_dense": mse, "mse_rel": mse / dense_ms,
+                          "within_budget": mse <= 1.1 * mse_topp})
+        # the selection in traversal order, timed once more on its own
+        so_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(n_es)]
         for s_ in range(n_es):
             flush.zero_()
-            es_evs[s_][0].record(stream)
+            so_evs[s_][0].record(stream)
             spa.spa_select_score_order(q, mean, var, w.block, w.scale, w.top_p, w.n_sink,
                                        w.n_local, w.k_min, idx=oidx, count=ocnt)
-            es_evs[s_][1].record(stream)
-            spa.spa_sparse_attn_prefill_early_stop(q, k, v, w.block, oidx, ocnt, w.scale, args.tau,
-                                                   w.n_sink, w.n_local, out=eout,
-                                                   processed=proc)
-            es_evs[s_][2].record(stream)
+            so_evs[s_][1].record(stream)
         torch.cuda.synchronize()
-        barrier()
-        t_osel = rank_max(statistics.mean(e[0].elapsed_time(e[1]) for e in es_evs))
-        t_es = rank_max(statistics.mean(e[1].elapsed_time(e[2]) for e in es_evs))
-        pr = proc.cpu().numpy()
-        oi = oidx.cpu().numpy()
-        trunc = np.where(np.arange(oi.shape[-1]) < pr[..., None], oi, -1)
-        F_es = kept_flops(pr, np.sort(np.where(trunc < 0, 1 << 30, trunc), axis=-1), L, w.block, d)
-        dev_ = (eout.float() - out.float())
-        early = {"tau": args.tau, "processed_fraction": float(pr.sum()) / float(count_h.sum()),
-                 "vs_kept_attention": {"max_abs": float(dev_.abs().max().item()),
-                                       "rms": float(dev_.pow(2).mean().sqrt().item()),
-                                       "output_rms": float(out.float().pow(2).mean().sqrt().item())},
-                 "select_score_order_ms": t_osel, "attn_ms": t_es,
-                 "processed_flops": F_es, "TFLOP/s": F_es / (t_es / 1e3) / 1e12,
-                 "tokens/s": job_throughput(B * L, world, 1,
-                                            statistics.mean(t_stats) + t_osel + t_es)}
-        del oidx, ocnt, proc, eout
+        t_osel = rank_max(statistics.mean(a_.elapsed_time(b_) for a_, b_ in so_evs))
+        ok = [r for r in sweep if r["within_budget"]]
+        head = max(ok, key=lambda r: r["tau"]) if ok else None
+        early = {"budget": {"mse_top_p_vs_dense": mse_topp, "mse_rel_top_p": mse_topp / dense_ms,
+                            "rule": "largest tau with mse_vs_dense <= 1.1 x mse_top_p_vs_dense"},
+                 "select_score_order_ms": t_osel, "sweep": sweep,
+                 "headline": None if head is None else {
+                     "tau": head["tau"], "processed_fraction": head["processed_fraction"],
+                     "attn_ms": head["attn_ms"], "TFLOP/s": head["TFLOP/s"],
+                     "tokens/s": job_throughput(B * L, world, 1, statistics.mean(t_stats) +
+                                                t_osel + head["attn_ms"])}}
+        del oidx, ocnt, proc, eout, dense_f
 
     # ---- segmented key permutation (PBS, sections 2-3)
     pbs = None
     if args.seg_blocks > 0 and w.dtype == "bf16" and args.seg_blocks * w.block <= 8192:
         perm = torch.empty((B, Hkv, L), device="cuda", dtype=torch.int32)
+        pws = torch.empty(spa.spa_pbs_workspace_bytes(B, Hq, Hkv, L, w.block), dtype=torch.uint8,
+                          device="cuda")
         kp, vp = torch.empty_like(k), torch.empty_like(v)
         mp, vp_ = torch.empty_like(mean), torch.empty_like(var)
         pidx, pcnt = torch.empty_like(idx), torch.empty_like(cnt)
@@ -522,7 +644,8 @@ def main():
         def pbs_step(ev=None):
             if ev:
                 ev[0].record(stream)
-            spa.spa_pbs_permutation(q, k, w.block, args.seg_blocks, perm=perm)
+            spa.spa_pbs_permutation(q, k, w.block, args.seg_blocks, w.scale, perm=perm,
+                                    workspace=pws)
             spa.spa_pbs_gather(k, perm, xp=kp)
             spa.spa_pbs_gather(v, perm, xp=vp)
             spa.spa_block_stats(kp, w.block, mean=mp, var=vp_)
@@ -564,7 +687,7 @@ def main():
                                           statistics.mean(t_stats)),
                "vs_plain_output": {"max_abs": float(dev_.abs().max().item()),
                                    "rms": float(dev_.pow(2).mean().sqrt().item())}}
-        del perm, kp, vp, mp, vp_, pidx, pcnt, pout
+        del perm, pws, kp, vp, mp, vp_, pidx, pcnt, pout
 
     # ---- decode leg
     decode = None
@@ -709,8 +832,19 @@ def main():
                   "frac": gbs / peaks["hbm_gbs"], "peak_source": peak_src,
                   "tokens/s": world * wd.B / ((t_dsel + t_dec) / 1e3),
                   "kept_fraction": float(dcnt.float().mean().item()) / wd.nb,
+                  "kept_fraction_union": dbytes / float(2 * kc.numel() * kc.element_size()),
                   "block_stats_full_cache": stats_full, "rla": drla, "quantized_stats": dq}
         del kc, vc
+
+    # ---- the other prefill workloads, each timed like the headline step
+    configs = {}
+    for cid in [int(c) for c in args.configs.split(",") if c.strip()]:
+        if cid == args.workload or WORKLOADS[cid].mode != "prefill":
+            continue
+        n_st = {1: max(args.steps, 20), 4: min(args.steps, 8)}.get(cid, args.steps)
+        configs[WORKLOADS[cid].name] = measure_prefill_workload(
+            spa, torch, cid, n_st, 3, peaks, peak_src, flush, stream, world, rank_max, barrier,
+            local)
 
     # ---- selection diagnostics on the three prefill workloads (dense comparisons
     # on the 1K, 8K and 32K workloads only; the 128K one would need 140 TFLOP more)
@@ -739,6 +873,7 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu:
         v_cpu, det = time_oracle(w, x, args.cpu_tokens, 7)
         cpu = {"value": v_cpu, "unit": "tokens/s", "cores": det["threads"], "kind": "oracle",
+               "extrapolated": True,
                "sample": f"stats + selection on the whole workload ({det['t_select_s']:.2f} s), "
                          f"masked fp64 attention on {args.cpu_tokens} random query positions x "
                          f"{Hq} heads ({det['t_attention_sample_s']:.2f} s); tokens/s = sampled "
@@ -750,18 +885,20 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
-            "config": {"workload": w.name, "B": B, "L": L, "Hq": Hq, "Hkv": Hkv, "d": d,
-                       "block": w.block, "top_p": w.top_p, "kept_fraction": kept_frac,
-                       "parallelism": f"replicas x{world}",
-                       "l2": "flushed (256 MiB memset) between timed steps"},
+            "config": workload_config(w, world),
+            "kept_fraction": kept_frac,
             "roofline": {"bound": "tensor", "kernel": "sparse_attn_prefill", "achieved": achieved,
                          "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                         "peak_source": f"{peak_src} bf16_tflops_sustained",
+                         "peak_source": f"{peak_src} bf16_tflops (burst: the timed region "
+                                        f"is {total_ms / 1e3:.2f} s)",
+                         "sm_mhz_median": clk.get("sm_mhz"),
+                         "peak_sustained": peak_sus, "frac_vs_sustained": achieved / peak_sus,
                          "kept_flops_per_launch": F,
                          "traffic": captured_traffic("prefill_tc_kernel<128>", w.name),
                          "traffic_unit": "bytes per launch (ncu dram read + write)",
                          "algorithmic_bytes": float(2 * q.numel() * 2 + 2 * k.numel() * 2)},
             "kernels": per_kernel,
+            "configs": configs,
             "rla": rla,
             "early_stop": early,
             "segmented_permutation": pbs,

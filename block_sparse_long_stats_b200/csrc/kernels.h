@@ -42,10 +42,12 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, int B
                               int seg_blocks = 0);
 
 // Segmented key permutation: perm [B, Hkv, L] (original index per permuted
-// position) and the permuted copy of K or V (rows of row_bytes bytes).
+// position; it holds the importances between the passes) from the workspace of
+// pbs_workspace_bytes, and the permuted copy of K or V (rows of row_bytes bytes).
+size_t pbs_workspace_bytes(int B, int Hq, int Hkv, int L, int block);
 cudaError_t launch_pbs_permutation(const void *q, const void *k, bool bf16, int B, int Hq, int Hkv,
-                                   int L, int d, int block, int seg_blocks, int32_t *perm,
-                                   cudaStream_t s);
+                                   int L, int d, int block, int seg_blocks, float scale,
+                                   void *workspace, int32_t *perm, cudaStream_t s);
 cudaError_t launch_gather_rows(const void *x, int B, int Hkv, int L, int row_bytes,
                                const int32_t *perm, void *xp, cudaStream_t s);
 

@@ -2,16 +2,28 @@
 // sections 2-3): inside each segment of seg_blocks * block tokens the keys are
 // sorted by a global importance score, descending, so that the keys many queries
 // attend to gather in the segment's first blocks; segments keep their order, so
-// causality between segments holds. The importance of key u is qbar . k_u, with
-// qbar the mean of the last query block's rows over the query heads of the
-// kv-group (the mean-pooled logits of the last query block; the positive softmax
-// scale does not change the order). Equal scores keep the smaller index first.
+// causality between segments holds. The importance (section 3, proxy scoring) is
+// the mean pooling of the attention scores of the last query block: for each of
+// the R = G * n_r rows (t, h) of that block over the kv-group's query heads, the
+// causal softmax row a_{h,t}(u) = exp(s q_{h,t} . k_u - lse_{h,t}) for u <= t, and
+// importance(u) = (1 / R) sum_rows a_{h,t}(u). Equal importances keep the smaller
+// index first.
 //
-// pbs_perm_kernel: one CTA per (segment, b * Hkv + g): qbar (fp32), one fp32 score
-// per key (d / 8 lanes per key with 16-byte loads, four in flight, shuffle sums),
-// then a bitonic sort of 64-bit keys (order-flipped score | index): segments up to
-// 2048 keys in registers (eight per thread; shuffles for strides up to 128, shared
-// memory for the six larger ones), longer ones in shared memory; writes perm.
+// Three passes over the keys of each (b, kv-head), in chunks of kChunk keys:
+//   pbs_rowstats: per (chunk, row) the running maximum and sum of exp2 of the
+//     row's logits over the chunk's visible keys (log2 units) -> workspace;
+//   pbs_lse: per row, the chunks' partials merged into lse2 = m + log2(sum);
+//   pbs_importance: per key, sum over the rows of exp2(logit - lse2), / R, written
+//     as fp32 bits into perm (perm doubles as the importance buffer).
+// For bf16 the logits are mma.sync m16n8k16 products (bf16 products are exact in
+// the fp32 accumulator): a warp holds the A fragments of 16 rows and walks the
+// chunk's keys, staged in padded shared memory, eight at a time. fp32 inputs take
+// plain per-thread dot products (the small fp32 workloads only).
+// pbs_sort_kernel: one CTA per (segment, b * Hkv + g) reads its segment's
+// importances, then a bitonic sort of 64-bit keys (order-flipped importance |
+// index): segments up to 2048 keys in registers (eight per thread; shuffles for
+// strides up to 128, shared memory for the six larger ones), longer ones in shared
+// memory; writes perm over the importances it read.
 // gather_rows_kernel: the permuted copy of K or V, 16 bytes per thread.
 #include <float.h>
 
@@ -32,92 +44,236 @@ __device__ __forceinline__ uint32_t order_desc(float f) {
     return ~ord;                                                        // descending with f
 }
 
-template <typename T, int D>
-__global__ void __launch_bounds__(kThreads) pbs_perm_kernel(const T *__restrict__ q,
-                                                            const T *__restrict__ k, int Hq,
-                                                            int Hkv, int L, int block,
-                                                            int seg_len, int sort_cap,
+constexpr int kChunk = 128;              // keys per CTA in the importance passes
+
+__host__ __device__ __forceinline__ int last_block_rows(int L, int block) {
+    const int nq = (L + block - 1) / block;
+    return L - (nq - 1) * block;
+}
+
+// Workspace of one (b, kv-head): partials [nchunks][R] (m2, s) then lse2 [R].
+__host__ __device__ __forceinline__ size_t ws_floats_per_group(int R, int nchunks) {
+    return (size_t)nchunks * R * 2 + R;
+}
+
+__device__ __forceinline__ void mma_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
+                                          uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Merge a (maximum, sum of exp2 relative to it) pair into another.
+__device__ __forceinline__ void merge_ms(float &m, float &s, float m2, float s2) {
+    if (m2 == -INFINITY) return;
+    if (m == -INFINITY) {
+        m = m2;
+        s = s2;
+        return;
+    }
+    const float mn = fmaxf(m, m2);
+    s = s * fast_exp2(m - mn) + s2 * fast_exp2(m2 - mn);
+    m = mn;
+}
+
+// bf16: one CTA per (key chunk, b * Hkv + g). IMP = false: row partials; true:
+// importances (needs lse2). Rows x in [0, R): head x / n_r, position r0 + x % n_r.
+template <int D, bool IMP>
+__global__ void __launch_bounds__(kThreads) pbs_scores_bf16_kernel(
+    const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k, int Hq, int Hkv,
+    int L, int block, float scale_log2, int nchunks, float *__restrict__ ws,
+    int32_t *__restrict__ perm) {
+    constexpr int KW = D / 2 + 4;                 // padded key row in 32-bit words
+    constexpr int NT = kChunk / 8;                // n-tiles of 8 keys
+    __shared__ __align__(16) uint32_t ks[kChunk * KW];
+    __shared__ float colsum[IMP ? kWarps : 1][IMP ? kChunk : 1];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int gid = lane >> 2, tig = lane & 3;
+    const int bg = blockIdx.y, b = bg / Hkv, g = bg % Hkv, G = Hq / Hkv;
+    const int nr = last_block_rows(L, block), r0 = L - nr, R = G * nr;
+    const int u0 = blockIdx.x * kChunk, nk = min(kChunk, L - u0);
+    float *part = ws + (size_t)bg * ws_floats_per_group(R, nchunks);
+    const float *lse2 = part + (size_t)nchunks * R * 2;
+
+    for (int x = tid; x < kChunk * (D / 8); x += kThreads) {
+        const int row = x / (D / 8), c = x % (D / 8);
+        const uint4 v = row < nk ? __ldg(reinterpret_cast<const uint4 *>(k + ((size_t)bg * L + u0 + row) * D) + c)
+                                 : make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4 *>(&ks[row * KW + c * 4]) = v;
+    }
+    __syncthreads();
+
+    float cs[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) cs[nt][0] = cs[nt][1] = 0.f;
+    for (int rg = warp; rg * 16 < R; rg += kWarps) {
+        const int xa = rg * 16 + gid, xb = xa + 8;
+        const bool va = xa < R, vb = xb < R;
+        const int ta = va ? r0 + xa % nr : -1, tb = vb ? r0 + xb % nr : -1;
+        const uint32_t *qa = reinterpret_cast<const uint32_t *>(
+            q + (((size_t)b * Hq + g * G + (va ? xa / nr : 0)) * L + (va ? ta : r0)) * D);
+        const uint32_t *qb = reinterpret_cast<const uint32_t *>(
+            q + (((size_t)b * Hq + g * G + (vb ? xb / nr : 0)) * L + (vb ? tb : r0)) * D);
+        uint32_t af[D / 16][4];
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+            af[kk][0] = __ldg(qa + kk * 8 + tig);
+            af[kk][1] = __ldg(qb + kk * 8 + tig);
+            af[kk][2] = __ldg(qa + kk * 8 + 4 + tig);
+            af[kk][3] = __ldg(qb + kk * 8 + 4 + tig);
+        }
+        float la = 0.f, lb = 0.f;
+        if constexpr (IMP) {
+            la = va ? lse2[xa] : 0.f;
+            lb = vb ? lse2[xb] : 0.f;
+        }
+        float ma = -INFINITY, sa = 0.f, mb = -INFINITY, sb = 0.f;
+#pragma unroll
+        for (int sub = 0; sub < NT / 8; ++sub) {
+            float z[8][4];
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt) {
+                z[nt][0] = z[nt][1] = z[nt][2] = z[nt][3] = 0.f;
+                const uint32_t *kr = &ks[(sub * 64 + nt * 8 + gid) * KW];
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) mma_16816(z[nt], af[kk], kr[kk * 8 + tig], kr[kk * 8 + 4 + tig]);
+            }
+            // key of (nt, e): u0 + sub * 64 + nt * 8 + 2 tig + e; a row sees keys u <= t
+            float mxa = -INFINITY, mxb = -INFINITY;
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int u = u0 + sub * 64 + nt * 8 + 2 * tig + e;
+                    z[nt][e] = u <= ta ? z[nt][e] * scale_log2 : -INFINITY;
+                    z[nt][2 + e] = u <= tb ? z[nt][2 + e] * scale_log2 : -INFINITY;
+                    mxa = fmaxf(mxa, z[nt][e]);
+                    mxb = fmaxf(mxb, z[nt][2 + e]);
+                }
+            if constexpr (IMP) {
+#pragma unroll
+                for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 2; ++e)
+                        cs[sub * 8 + nt][e] += fast_exp2(z[nt][e] - la) + fast_exp2(z[nt][2 + e] - lb);
+            } else {
+                float ta_ = 0.f, tb_ = 0.f;
+                if (mxa != -INFINITY) {
+#pragma unroll
+                    for (int nt = 0; nt < 8; ++nt) ta_ += fast_exp2(z[nt][0] - mxa) + fast_exp2(z[nt][1] - mxa);
+                }
+                if (mxb != -INFINITY) {
+#pragma unroll
+                    for (int nt = 0; nt < 8; ++nt) tb_ += fast_exp2(z[nt][2] - mxb) + fast_exp2(z[nt][3] - mxb);
+                }
+                merge_ms(ma, sa, mxa, ta_);
+                merge_ms(mb, sb, mxb, tb_);
+            }
+        }
+        if constexpr (!IMP) {
+            // the four lanes of a row hold disjoint columns: merge them
+#pragma unroll
+            for (int o = 1; o < 4; o <<= 1) {
+                const float m2a = __shfl_xor_sync(0xffffffffu, ma, o), s2a = __shfl_xor_sync(0xffffffffu, sa, o);
+                const float m2b = __shfl_xor_sync(0xffffffffu, mb, o), s2b = __shfl_xor_sync(0xffffffffu, sb, o);
+                merge_ms(ma, sa, m2a, s2a);
+                merge_ms(mb, sb, m2b, s2b);
+            }
+            if (tig == 0) {
+                float2 *pp = reinterpret_cast<float2 *>(part) + (size_t)blockIdx.x * R;
+                if (va) pp[xa] = make_float2(ma, sa);
+                if (vb) pp[xb] = make_float2(mb, sb);
+            }
+        }
+    }
+    if constexpr (IMP) {
+        // column sums over the warp's rows (lanes of equal tig), then over the warps
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                float v = cs[nt][e];
+                v += __shfl_xor_sync(0xffffffffu, v, 4);
+                v += __shfl_xor_sync(0xffffffffu, v, 8);
+                v += __shfl_xor_sync(0xffffffffu, v, 16);
+                if (gid == 0) colsum[warp][nt * 8 + 2 * tig + e] = v;
+            }
+        __syncthreads();
+        for (int x = tid; x < nk; x += kThreads) {
+            float v = 0.f;
+#pragma unroll
+            for (int w = 0; w < kWarps; ++w) v += colsum[w][x];
+            perm[(size_t)bg * L + u0 + x] = __float_as_int(v / (float)R);
+        }
+    }
+}
+
+// fp32 inputs: the same two passes with plain dot products (thread per row for the
+// partials, thread per key for the importances).
+template <int D, bool IMP>
+__global__ void __launch_bounds__(kThreads) pbs_scores_f32_kernel(
+    const float *__restrict__ q, const float *__restrict__ k, int Hq, int Hkv, int L, int block,
+    float scale_log2, int nchunks, float *__restrict__ ws, int32_t *__restrict__ perm) {
+    const int tid = threadIdx.x;
+    const int bg = blockIdx.y, b = bg / Hkv, g = bg % Hkv, G = Hq / Hkv;
+    const int nr = last_block_rows(L, block), r0 = L - nr, R = G * nr;
+    const int u0 = blockIdx.x * kChunk, nk = min(kChunk, L - u0);
+    float *part = ws + (size_t)bg * ws_floats_per_group(R, nchunks);
+    const float *lse2 = part + (size_t)nchunks * R * 2;
+    auto logit = [&](int x, int u) {
+        const float *qr = q + (((size_t)b * Hq + g * G + x / nr) * L + r0 + x % nr) * D;
+        const float *kr = k + ((size_t)bg * L + u) * D;
+        float s = 0.f;
+#pragma unroll 8
+        for (int c = 0; c < D; ++c) s = fmaf(__ldg(qr + c), __ldg(kr + c), s);
+        return s * scale_log2;
+    };
+    if constexpr (!IMP) {
+        for (int x = tid; x < R; x += kThreads) {
+            const int t = r0 + x % nr;
+            float m = -INFINITY, s = 0.f;
+            for (int u = u0; u < u0 + nk && u <= t; ++u) merge_ms(m, s, logit(x, u), 1.f);
+            reinterpret_cast<float2 *>(part)[(size_t)blockIdx.x * R + x] = make_float2(m, s);
+        }
+    } else {
+        for (int y = tid; y < nk; y += kThreads) {
+            const int u = u0 + y;
+            float v = 0.f;
+            for (int x = 0; x < R; ++x)
+                if (u <= r0 + x % nr) v += fast_exp2(logit(x, u) - lse2[x]);
+            perm[(size_t)bg * L + u] = __float_as_int(v / (float)R);
+        }
+    }
+}
+
+// lse2 of every row: the chunks' partials merged in chunk order.
+__global__ void __launch_bounds__(kThreads) pbs_lse_kernel(int R, int nchunks, float *__restrict__ ws) {
+    float *part = ws + (size_t)blockIdx.x * ws_floats_per_group(R, nchunks);
+    float *lse2 = part + (size_t)nchunks * R * 2;
+    const float2 *pp = reinterpret_cast<const float2 *>(part);
+    for (int x = threadIdx.x; x < R; x += kThreads) {
+        float m = -INFINITY, s = 0.f;
+        for (int c = 0; c < nchunks; ++c) {
+            const float2 v = pp[(size_t)c * R + x];
+            merge_ms(m, s, v.x, v.y);
+        }
+        lse2[x] = m + __log2f(s);
+    }
+}
+
+// One CTA per (segment, b * Hkv + g): the segment's importances (fp32 bits in
+// perm) sorted descending, equal values by ascending index; perm overwritten.
+__global__ void __launch_bounds__(kThreads) pbs_sort_kernel(int L, int seg_len, int sort_cap,
                                                             int32_t *__restrict__ perm) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     uint64_t *keys = reinterpret_cast<uint64_t *>(smem_raw);     // [sort_cap]
-    constexpr int V = 16 / sizeof(T);             // elements per 16-byte chunk
-    constexpr int CPR = D / V;                    // chunks per row
-    constexpr int RG = kThreads / CPR;            // row groups
-    __shared__ float qbar[D];
-    __shared__ float part[RG][D];
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int bg = blockIdx.y, b = bg / Hkv, g = bg % Hkv, G = Hq / Hkv;
+    const int tid = threadIdx.x, lane = tid & 31;
+    const int bg = blockIdx.y;
     const int s0 = blockIdx.x * seg_len, n = min(seg_len, L - s0);
-    const int nq = (L + block - 1) / block, r0 = (nq - 1) * block, nr = L - r0;
-
-    // pooled query of the last query block over the group's heads: thread (rg, c)
-    // sums 16-byte chunk c of rows rg, rg + RG, ... of all G heads
-    {
-        const int c = tid % CPR, rg = tid / CPR;
-        float acc[V];
-#pragma unroll
-        for (int e = 0; e < V; ++e) acc[e] = 0.f;
-        for (int x = rg; x < G * nr; x += RG) {
-            const int hh = x / nr, r = x % nr;
-            const uint4 u = __ldg(reinterpret_cast<const uint4 *>(
-                q + (((size_t)b * Hq + g * G + hh) * L + r0 + r) * D) + c);
-            if constexpr (sizeof(T) == 2) {
-                acc[0] += bf16lo(u.x); acc[1] += bf16hi(u.x); acc[2] += bf16lo(u.y);
-                acc[3] += bf16hi(u.y); acc[4] += bf16lo(u.z); acc[5] += bf16hi(u.z);
-                acc[6] += bf16lo(u.w); acc[7] += bf16hi(u.w);
-            } else {
-                acc[0] += __uint_as_float(u.x); acc[1] += __uint_as_float(u.y);
-                acc[2] += __uint_as_float(u.z); acc[3] += __uint_as_float(u.w);
-            }
-        }
-#pragma unroll
-        for (int e = 0; e < V; ++e) part[rg][c * V + e] = acc[e];
-    }
-    __syncthreads();
-    for (int c = tid; c < D; c += kThreads) {
-        float acc = 0.f;
-        for (int rg = 0; rg < RG; ++rg) acc += part[rg][c];
-        qbar[c] = acc / (float)(G * nr);
-    }
-    __syncthreads();
-
-    // importance of each key of the segment: LPK lanes per key, one 16-byte chunk
-    // each, U loads in flight per lane
-    constexpr int LPK = CPR;                      // lanes per key
-    constexpr int KPW = 32 / LPK;                 // keys per warp load
-    constexpr int U = 4;
-    const int sub = lane / LPK, cl = lane % LPK;
-    float qv[V];
-#pragma unroll
-    for (int e = 0; e < V; ++e) qv[e] = qbar[cl * V + e];
-    for (int x0 = warp * KPW * U; x0 < n; x0 += kWarps * KPW * U) {
-        uint4 u[U];
-#pragma unroll
-        for (int uu = 0; uu < U; ++uu) {
-            const int x = x0 + uu * KPW + sub;
-            u[uu] = x < n ? __ldg(reinterpret_cast<const uint4 *>(k + ((size_t)bg * L + s0 + x) * D) + cl)
-                          : make_uint4(0, 0, 0, 0);
-        }
-#pragma unroll
-        for (int uu = 0; uu < U; ++uu) {
-            float kv[V];
-            if constexpr (sizeof(T) == 2) {
-                kv[0] = bf16lo(u[uu].x); kv[1] = bf16hi(u[uu].x); kv[2] = bf16lo(u[uu].y);
-                kv[3] = bf16hi(u[uu].y); kv[4] = bf16lo(u[uu].z); kv[5] = bf16hi(u[uu].z);
-                kv[6] = bf16lo(u[uu].w); kv[7] = bf16hi(u[uu].w);
-            } else {
-                kv[0] = __uint_as_float(u[uu].x); kv[1] = __uint_as_float(u[uu].y);
-                kv[2] = __uint_as_float(u[uu].z); kv[3] = __uint_as_float(u[uu].w);
-            }
-            float sdot = 0.f;
-#pragma unroll
-            for (int e = 0; e < V; ++e) sdot = fmaf(qv[e], kv[e], sdot);
-#pragma unroll
-            for (int o = LPK / 2; o > 0; o >>= 1) sdot += __shfl_xor_sync(0xffffffffu, sdot, o);
-            const int x = x0 + uu * KPW + sub;
-            if (cl == 0 && x < n) keys[x] = ((uint64_t)order_desc(sdot) << 32) | (uint32_t)x;
-        }
-    }
+    for (int x = tid; x < n; x += kThreads)
+        keys[x] = ((uint64_t)order_desc(__int_as_float(perm[(size_t)bg * L + s0 + x])) << 32) | (uint32_t)x;
     if (sort_cap <= kRegSort) {
         // up to 2048 keys: 8 per thread in registers, position x = 8 tid + e; strides
         // below 8 in registers, 8..128 by shuffles, 256 and up through shared memory
@@ -219,36 +375,57 @@ __global__ void __launch_bounds__(kThreads) gather_rows_kernel(const uint4 *__re
     }
 }
 
-template <typename T, int D>
-cudaError_t launch_perm_t(const void *q, const void *k, int B, int Hq, int Hkv, int L, int block,
-                          int seg_blocks, int32_t *perm, cudaStream_t s) {
+template <int D>
+cudaError_t launch_perm_d(const void *q, const void *k, bool bf16, int B, int Hq, int Hkv, int L,
+                          int block, int seg_blocks, float scale, void *ws, int32_t *perm,
+                          cudaStream_t s) {
+    const int R = (Hq / Hkv) * last_block_rows(L, block);
+    const int nchunks = (L + kChunk - 1) / kChunk;
+    const float sl2 = scale * 1.4426950408889634f;
+    float *w = static_cast<float *>(ws);
+    const dim3 grid_c((unsigned)nchunks, (unsigned)(B * Hkv));
+    if (bf16) {
+        const auto *qq = static_cast<const __nv_bfloat16 *>(q);
+        const auto *kk = static_cast<const __nv_bfloat16 *>(k);
+        pbs_scores_bf16_kernel<D, false><<<grid_c, kThreads, 0, s>>>(qq, kk, Hq, Hkv, L, block, sl2, nchunks, w, perm);
+        pbs_lse_kernel<<<B * Hkv, kThreads, 0, s>>>(R, nchunks, w);
+        pbs_scores_bf16_kernel<D, true><<<grid_c, kThreads, 0, s>>>(qq, kk, Hq, Hkv, L, block, sl2, nchunks, w, perm);
+    } else {
+        const auto *qq = static_cast<const float *>(q);
+        const auto *kk = static_cast<const float *>(k);
+        pbs_scores_f32_kernel<D, false><<<grid_c, kThreads, 0, s>>>(qq, kk, Hq, Hkv, L, block, sl2, nchunks, w, perm);
+        pbs_lse_kernel<<<B * Hkv, kThreads, 0, s>>>(R, nchunks, w);
+        pbs_scores_f32_kernel<D, true><<<grid_c, kThreads, 0, s>>>(qq, kk, Hq, Hkv, L, block, sl2, nchunks, w, perm);
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
     const int seg_len = seg_blocks * block;
     int cap = 1;
     while (cap < seg_len) cap <<= 1;
     // the register sort pads to kRegSort keys and exchanges through two buffers
     const size_t smem = (size_t)(cap <= kRegSort ? 2 * kRegSort : cap) * 8;
-    auto kern = pbs_perm_kernel<T, D>;
     if (smem > 48 * 1024) {
-        const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                   (int)smem);
+        e = cudaFuncSetAttribute(pbs_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
     }
     dim3 grid((unsigned)((L + seg_len - 1) / seg_len), (unsigned)(B * Hkv));
-    kern<<<grid, kThreads, smem, s>>>(reinterpret_cast<const T *>(q), reinterpret_cast<const T *>(k),
-                                      Hq, Hkv, L, block, seg_len, cap, perm);
+    pbs_sort_kernel<<<grid, kThreads, smem, s>>>(L, seg_len, cap, perm);
     return cudaGetLastError();
 }
 
 }  // namespace
 
+size_t pbs_workspace_bytes(int B, int Hq, int Hkv, int L, int block) {
+    const int R = (Hq / Hkv) * last_block_rows(L, block);
+    const int nchunks = (L + kChunk - 1) / kChunk;
+    return (size_t)B * Hkv * ws_floats_per_group(R, nchunks) * sizeof(float);
+}
+
 cudaError_t launch_pbs_permutation(const void *q, const void *k, bool bf16, int B, int Hq, int Hkv,
-                                   int L, int d, int block, int seg_blocks, int32_t *perm,
-                                   cudaStream_t s) {
-    if (bf16)
-        return d == 128 ? launch_perm_t<__nv_bfloat16, 128>(q, k, B, Hq, Hkv, L, block, seg_blocks, perm, s)
-                        : launch_perm_t<__nv_bfloat16, 64>(q, k, B, Hq, Hkv, L, block, seg_blocks, perm, s);
-    return d == 128 ? launch_perm_t<float, 128>(q, k, B, Hq, Hkv, L, block, seg_blocks, perm, s)
-                    : launch_perm_t<float, 64>(q, k, B, Hq, Hkv, L, block, seg_blocks, perm, s);
+                                   int L, int d, int block, int seg_blocks, float scale,
+                                   void *workspace, int32_t *perm, cudaStream_t s) {
+    return d == 128 ? launch_perm_d<128>(q, k, bf16, B, Hq, Hkv, L, block, seg_blocks, scale, workspace, perm, s)
+                    : launch_perm_d<64>(q, k, bf16, B, Hq, Hkv, L, block, seg_blocks, scale, workspace, perm, s);
 }
 
 cudaError_t launch_gather_rows(const void *x, int B, int Hkv, int L, int row_bytes,

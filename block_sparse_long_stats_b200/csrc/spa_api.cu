@@ -12,7 +12,8 @@
 namespace spa {
 namespace {
 
-__device__ int g_device_error = 0;
+// [0]: error code; [2..3]: abort stamp of the last launch that timed out
+__device__ __align__(16) int g_device_error[4] = {0, 0, 0, 0};
 
 constexpr int kMaxDevices = 64;
 int *g_err_ptr[kMaxDevices] = {nullptr};
@@ -199,21 +200,31 @@ SPA_API spa_status spa_sparse_attn_prefill_early_stop(
     return e == cudaSuccess ? SPA_OK : cuda_fail(e, "prefill launch");
 }
 
+SPA_API size_t spa_pbs_workspace_bytes(int B, int Hq, int Hkv, int L, int block) {
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || L <= 0 || block <= 0 || Hq % Hkv) return 0;
+    return pbs_workspace_bytes(B, Hq, Hkv, L, block);
+}
+
 SPA_API spa_status spa_pbs_permutation(const void *q, const void *k, spa_dtype dt, int B, int Hq,
                                        int Hkv, int L, int d, int block, int seg_blocks,
+                                       float scale, void *workspace, size_t workspace_bytes,
                                        int32_t *perm, spa_stream stream) {
     t_last_error.clear();
-    if (!q || !k || !perm) return fail(SPA_ERR_INVALID, "null pointer");
+    if (!q || !k || !perm || !workspace) return fail(SPA_ERR_INVALID, "null pointer");
     if (B <= 0 || Hq <= 0 || Hkv <= 0 || L <= 0 || d <= 0 || block <= 0 || seg_blocks <= 0)
         return fail(SPA_ERR_INVALID, "sizes must be positive");
     if (Hq % Hkv) return fail(SPA_ERR_INVALID, "Hq must be a multiple of Hkv");
+    if (!(scale > 0.f)) return fail(SPA_ERR_INVALID, "scale must be positive");
     if (dt != SPA_F32 && dt != SPA_BF16) return fail(SPA_ERR_INVALID, "unknown dtype");
-    if (!aligned16(q) || !aligned16(k)) return fail(SPA_ERR_INVALID, "tensors must be 16-byte aligned");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(workspace))
+        return fail(SPA_ERR_INVALID, "tensors must be 16-byte aligned");
     if (d != 64 && d != 128) return fail(SPA_ERR_UNSUPPORTED, "d must be 64 or 128");
     if ((long)seg_blocks * block > 8192)
         return fail(SPA_ERR_UNSUPPORTED, "a segment holds at most 8192 tokens");
+    if (workspace_bytes < pbs_workspace_bytes(B, Hq, Hkv, L, block))
+        return fail(SPA_ERR_INVALID, "workspace smaller than spa_pbs_workspace_bytes");
     cudaError_t e = launch_pbs_permutation(q, k, dt == SPA_BF16, B, Hq, Hkv, L, d, block, seg_blocks,
-                                           perm, static_cast<cudaStream_t>(stream));
+                                           scale, workspace, perm, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? SPA_OK : cuda_fail(e, "permutation launch");
 }
 
@@ -545,8 +556,8 @@ SPA_API spa_status spa_get_device_error(int *code) {
     int v = 0;
     e = cudaMemcpy(&v, p, sizeof v, cudaMemcpyDeviceToHost);
     if (e != cudaSuccess) return cuda_fail(e, "read error word");
-    const int zero = 0;
-    e = cudaMemcpy(p, &zero, sizeof zero, cudaMemcpyHostToDevice);
+    const int zero[4] = {0, 0, 0, 0};
+    e = cudaMemcpy(p, zero, sizeof zero, cudaMemcpyHostToDevice);
     if (e != cudaSuccess) return cuda_fail(e, "clear error word");
     *code = v;
     return v ? SPA_ERR_DEVICE : SPA_OK;

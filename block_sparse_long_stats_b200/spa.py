@@ -71,7 +71,10 @@ def lib() -> ctypes.CDLL:
         L.spa_sparse_attn_prefill_early_stop.argtypes = [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I,
                                                          _P, _I, _P, _F, _I, _I, _F, _P, _P, _P,
                                                          _P]
-        L.spa_pbs_permutation.argtypes = [_P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P]
+        L.spa_pbs_workspace_bytes.argtypes = [_I, _I, _I, _I, _I]
+        L.spa_pbs_workspace_bytes.restype = ctypes.c_size_t
+        L.spa_pbs_permutation.argtypes = [_P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _P,
+                                          ctypes.c_size_t, _P, _P]
         L.spa_pbs_gather.argtypes = [_P, _I, _I, _I, _I, _I, _P, _P, _P]
         L.spa_select_segperm.argtypes = [_P, _I, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F,
                                          _F, _I, _I, _I, _P, _I, _P, _P]
@@ -296,16 +299,26 @@ def spa_prefill_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block: i
     return out
 
 
+def spa_pbs_workspace_bytes(B: int, Hq: int, Hkv: int, L: int, block: int) -> int:
+    return int(lib().spa_pbs_workspace_bytes(B, Hq, Hkv, L, block))
+
+
 def spa_pbs_permutation(q: torch.Tensor, k: torch.Tensor, block: int, seg_blocks: int,
-                        perm: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+                        scale: float, perm: torch.Tensor | None = None,
+                        workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """Segmented key permutation: perm [B, Hkv, L] int32 (original index per position)."""
     B, Hq, L, d = q.shape
     Hkv = k.shape[1]
     if perm is None:
         perm = torch.empty((B, Hkv, L), device=q.device, dtype=torch.int32)
+    need = spa_pbs_workspace_bytes(B, Hq, Hkv, L, block)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
     _check("spa_pbs_permutation",
            lib().spa_pbs_permutation(_ptr(q), _ptr(k), _dt(q), B, Hq, Hkv, L, d, block, seg_blocks,
-                                     _ptr(perm), _stream(stream)))
+                                     scale, _ptr(workspace),
+                                     workspace.numel() * workspace.element_size(), _ptr(perm),
+                                     _stream(stream)))
     return perm
 
 

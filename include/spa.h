@@ -28,7 +28,15 @@
  *     Faults the kernels detect themselves (a kept-list entry out of range or not
  *     ascending, a count outside [0, cap], a bounded wait that ran out) are
  *     recorded in a device error word, read with spa_get_device_error; the kernel
- *     skips the bad entry instead of touching memory out of bounds.
+ *     skips the bad entry instead of touching memory out of bounds. The code stays
+ *     set until it is read. A bounded wait that runs out ends only its own launch
+ *     (the launch's other waits give up at once); launches after it, on any
+ *     stream, wait normally and compute normally whether or not the word was read.
+ *   - The library looks up, once per device, the device addresses of its error
+ *     word and of the fixed scratch array of spa_sparse_attn_decode_noalloc, and
+ *     keeps them for the life of the process. After cudaDeviceReset on a device,
+ *     do not call the library on that device again in the same process: the
+ *     cached addresses may no longer be valid.
  *   - No C++ exception crosses this interface.
  */
 #ifndef SPA_H
@@ -210,14 +218,24 @@ spa_status spa_sparse_attn_prefill_early_stop(const void *q, const void *k, cons
  * seg_blocks * block tokens; inside each, keys (with their values) are sorted by a
  * global importance score, descending, so the keys many queries attend to gather
  * in the segment's first blocks; segments keep their order (causality between
- * segments holds); queries keep their order. Importance (the mean-pooled scores
- * of the last query block, taken on the logits): qbar . k_u, qbar the mean of the
- * last query block's rows over the query heads of the kv-group; equal scores keep
- * the smaller index first (fp32 scores).
+ * segments holds); queries keep their order. Importance (section 3, proxy
+ * scoring: the attention scores of the last query block, mean-pooled): for every
+ * row t of the last query block and every query head h of the kv-group, the
+ * causal softmax row a_{h,t}(u) = exp(scale q_{h,t}.k_u) / sum_{u'<=t} exp(...)
+ * (0 for u > t); importance(u) = the mean of a_{h,t}(u) over those G * n_r rows.
+ * Computed in fp32 (logits from exact bf16 products summed in fp32); equal
+ * importances keep the smaller index first.
  *
+ * spa_pbs_workspace_bytes: the device workspace spa_pbs_permutation needs (per
+ *   (b, kv-head): a (max, sum) pair per row and key chunk of 128, and a
+ *   log-sum-exp per row); 0 for invalid sizes.
  * spa_pbs_permutation: perm [B, Hkv, L] int32 output, perm[b,g,p] = the original
  *   index of the key at permuted position p. q [B, Hq, L, d], k [B, Hkv, L, d],
- *   dt, d = 64 or 128; a segment holds at most 8192 tokens.
+ *   dt, d = 64 or 128; scale > 0 (the attention's softmax scale); a segment holds
+ *   at most 8192 tokens. workspace: caller-owned device memory of at least
+ *   spa_pbs_workspace_bytes (16-byte aligned; contents on entry do not matter).
+ *   perm also holds the importances between the call's passes. Four launches on
+ *   the stream (row partials, log-sum-exp, importances, segment sort).
  * spa_pbs_gather: xp[b,g,p,:] = x[b,g,perm[b,g,p],:], for K and for V (rows of
  *   d elements of dt; the copies the two calls below read).
  * spa_select_segperm: spa_select for prefill on this layout: query block i scores
@@ -229,8 +247,10 @@ spa_status spa_sparse_attn_prefill_early_stop(const void *q, const void *k, cons
  *   past: no mask) and those of its own segment from k, v (the diagonal block
  *   masked token by token). bf16, d = 128, block 64 or 128.
  */
+size_t spa_pbs_workspace_bytes(int B, int Hq, int Hkv, int L, int block);
 spa_status spa_pbs_permutation(const void *q, const void *k, spa_dtype dt, int B, int Hq, int Hkv,
-                               int L, int d, int block, int seg_blocks, int32_t *perm,
+                               int L, int d, int block, int seg_blocks, float scale,
+                               void *workspace, size_t workspace_bytes, int32_t *perm,
                                spa_stream stream);
 spa_status spa_pbs_gather(const void *x, spa_dtype dt, int B, int Hkv, int L, int d,
                           const int32_t *perm, void *xp, spa_stream stream);

@@ -31,3 +31,9 @@ def test_reference_arm_prints_one_contract_line():
     assert "4 random query positions" in cb["sample"]
     assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}
+    assert d["extrapolated"] is True and cb["extrapolated"] is True
+    # the same config dict the CUDA arm prints for this workload
+    sys.path.insert(0, ROOT)
+    import bench
+    from workloads import WORKLOADS
+    assert d["config"] == bench.workload_config(WORKLOADS[1], 1)
