@@ -105,10 +105,26 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
     return t;
 }
 
+// Temporal launch number of this grid within the context (PTX %gridid).
+__device__ __forceinline__ uint64_t grid_launch_id() {
+    uint64_t g;
+    asm volatile("mov.u64 %0, %%gridid;" : "=l"(g));
+    return g;
+}
+
+// The device error word is four ints: [0] the error code (SPA_DEVERR_*), sticky
+// until spa_get_device_error reads it; [2..3] the abort stamp, the launch number +
+// 1 of the last launch whose bounded wait ran out. A wait gives up early only when
+// the stamp names its own launch, so one broken wait ends that launch quickly
+// while later launches (which have other numbers) wait normally.
+__device__ __forceinline__ unsigned long long *abort_stamp(int *err) {
+    return reinterpret_cast<unsigned long long *>(err + 2);
+}
+
 // Bounded wait for the phase with the given parity to complete. Gives up after
-// about `limit_ns` nanoseconds, records SPA_DEVERR_TIMEOUT and returns false. It
-// also gives up as soon as any CTA has recorded a timeout, so one broken wait ends
-// the whole launch quickly instead of every CTA waiting out its own limit.
+// about `limit_ns` nanoseconds, records SPA_DEVERR_TIMEOUT and this launch's abort
+// stamp, and returns false; gives up at once when another wait of the same launch
+// already ran out.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *err,
                                           uint64_t limit_ns = 1000000000ull) {
     const uint32_t a = smem_u32(bar);
@@ -117,13 +133,52 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *e
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(a, parity)) return true;
         if ((it & 255u) == 0) {
-            if (err && *reinterpret_cast<volatile int *>(err) == SPA_DEVERR_TIMEOUT) return false;
+            if (err && *reinterpret_cast<volatile unsigned long long *>(abort_stamp(err)) ==
+                           grid_launch_id() + 1ull)
+                return false;
             if (globaltimer_ns() - t0 > limit_ns) {
                 set_error(err, SPA_DEVERR_TIMEOUT);
+                if (err) atomicExch(abort_stamp(err), grid_launch_id() + 1ull);
                 return false;
             }
         }
     }
+}
+
+// Wait (bounded by limit_ns, never giving up early) for a copy this thread issued
+// to land, before the CTA leaves on a failure path: a bulk copy must not write
+// into shared memory the CTA no longer owns.
+__device__ __forceinline__ void mbar_drain(uint64_t *bar, uint32_t parity,
+                                           uint64_t limit_ns = 1000000000ull) {
+    const uint32_t a = smem_u32(bar);
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(a, parity))
+        if (globaltimer_ns() - t0 > limit_ns) return;
+}
+
+// After a producer issued n loads round-robin over the ST stages of a ring (load u
+// on stage u % ST, completing phase u / ST of full[u % ST]), wait for the last load
+// of every stage to land. On the normal path each of them was already consumed and
+// this returns at once; on a failure path it keeps the CTA until its copies land.
+template <int ST>
+__device__ __forceinline__ void drain_ring(uint64_t *full, int n) {
+#pragma unroll
+    for (int s = 0; s < ST; ++s) {
+        if (s >= n) break;
+        const int u = s + ((n - 1 - s) / ST) * ST;
+        mbar_drain(&full[s], (uint32_t)(u / ST) & 1u);
+    }
+}
+
+// Register reallocation between warpgroups (every warp of the warpgroup executes
+// it; the sum over the CTA must stay within the registers it was launched with).
+template <uint32_t N>
+__device__ __forceinline__ void regs_increase() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_decrease() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 // Named barrier over `nthreads` threads (a multiple of 32); id 0 is __syncthreads.

@@ -191,7 +191,8 @@ __global__ void __launch_bounds__((CONS + 1) * 32, BLOCK == 16 ? 3 : 1) decode_k
         if (lane == 0) {
             prefetch_tmap(&tk);
             prefetch_tmap(&tv);
-            for (int u = 0; u < nu; ++u) {
+            int u = 0;
+            for (; u < nu; ++u) {
                 const int s = u % STAGES;
                 if (!mbar_wait(&empty[s], ((u / STAGES) & 1) ^ 1, a.err)) break;
                 const int row = bg * a.T + (j_lo + ulist[u]) * BLOCK;
@@ -203,6 +204,7 @@ __global__ void __launch_bounds__((CONS + 1) * 32, BLOCK == 16 ? 3 : 1) decode_k
                 tma_load_2d(vt, &tv, &full[s], 0, row);
                 tma_load_2d(vt + TILE / 2, &tv, &full[s], 64, row);
             }
+            drain_ring<STAGES>(full, u);
         }
     } else {
         // ---------------- consumers

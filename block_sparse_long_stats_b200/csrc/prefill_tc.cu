@@ -323,6 +323,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                     tma_load_2d(dst + C::KV_HALF + 64 * 128, mb_, bar, 64, kv_row0 + jb * 64);
                 }
             };
+            int nk = 0, nv = 0;   // K and V tiles issued
             for (int n = 0; next_tile(j, mask, jb, mb, true); ++n) {
                 const int s = n % ST;
                 const uint32_t ph = (n / ST) & 1;
@@ -331,20 +332,23 @@ __global__ void __launch_bounds__(kThreads, 2)
                 if (!mbar_wait(&empty_k[s], ph ^ 1, a.err)) break;
                 mbar_arrive_expect_tx(&full_k[s], C::KV_BYTES);
                 load_tile(kt, &tk, &tkp, &full_k[s]);
+                ++nk;
                 if constexpr (ES) {
                     if (n > 0) {
                         if (!mbar_wait(&decided[(n - 1) & 1], ((n - 1) >> 1) & 1, a.err)) break;
-                        if (*reinterpret_cast<volatile int *>(&stop_at) <= n - 1) {
-                            mbar_wait(&full_k[s], ph, a.err);   // the copy already started
-                            break;
-                        }
+                        // stopped: the K copy already started lands in the drain below
+                        if (*reinterpret_cast<volatile int *>(&stop_at) <= n - 1) break;
                     }
                 }
                 if (!mbar_wait(&empty_v[s], ph ^ 1, a.err)) break;
                 mbar_arrive_expect_tx(&full_v[s], C::KV_BYTES);
                 load_tile(vt, &tv, &tvp, &full_v[s]);
+                ++nv;
             }
+            drain_ring<ST>(full_k, nk);
+            drain_ring<ST>(full_v, nv);
         }
+        if (lane == 0) mbar_drain(&bar_q, 0);
     } else if (warp == 5) {
         if (lane == 0) {
             cur.init(a, b, h0, i, false);

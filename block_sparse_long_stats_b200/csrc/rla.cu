@@ -119,7 +119,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             prefetch_tmap(&tk);
             prefetch_tmap(&tv);
-            for (int n = 0; n < nblk; ++n) {
+            int n = 0;
+            for (; n < nblk; ++n) {
                 const int s = n % ST;
                 if (!mbar_wait(&empty[s], ((n / ST) & 1) ^ 1, a.err)) break;
                 const int row = bg * a.T + (j0 + n) * BLK;
@@ -131,6 +132,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tma_load_2d(vt, &tv, &full[s], 0, row);
                 tma_load_2d(vt + C::HALF, &tv, &full[s], 64, row);
             }
+            drain_ring<ST>(full, n);
         }
     } else if (warp == kMmaWarp) {
         if (lane == 0) {
@@ -394,9 +396,11 @@ __global__ void __launch_bounds__(kThreads, 2)
                 tma_load_2d(wt, &tw, &full[s], 0, (wblk0 + j) * 128);
                 tma_load_2d(wt + 16384, &tw, &full[s], 64, (wblk0 + j) * 128);
             }
+            drain_ring<ST>(full, n);
+            int x = 0;
             if (ok && diag) {
                 const int kvrow = (b * a.Hkv + g) * a.L + i * BLK;
-                for (int x = 0; x < 2; ++x, ++n) {
+                for (; x < 2; ++x, ++n) {
                     const int s = n % ST;
                     if (!mbar_wait(&empty[s], ((n / ST) & 1) ^ 1, a.err)) break;
                     unsigned char *t = smem + C::OFF_W + s * C::W_BYTES;
@@ -407,6 +411,10 @@ __global__ void __launch_bounds__(kThreads, 2)
                     tma_load_2d(t + C::KV_HALF, m, fb, 64, kvrow);
                 }
             }
+            // the diagonal tiles' barriers are used once each
+            if (x > 0) mbar_drain(&full_kd, 0);
+            if (x > 1) mbar_drain(&full_vd, 0);
+            mbar_drain(&bar_q, 0);
         }
     } else if (warp == kMmaWarp) {
         if (lane == 0) {
@@ -593,7 +601,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             prefetch_tmap(&tk);
             prefetch_tmap(&tv);
-            for (int n = 0; n < nblk; ++n) {
+            int n = 0;
+            for (; n < nblk; ++n) {
                 const int s = n % ST;
                 if (!mbar_wait(&empty[s], ((n / ST) & 1) ^ 1, a.err)) break;
                 const int row = bg * a.T + a.tok_begin + (c0 + n) * 128;
@@ -605,6 +614,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tma_load_2d(vt, &tv, &full[s], 0, row);
                 tma_load_2d(vt + C::HALF, &tv, &full[s], 64, row);
             }
+            drain_ring<ST>(full, n);
         }
     } else if (warp == kMmaWarp) {
         if (lane == 0) {

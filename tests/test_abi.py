@@ -254,3 +254,13 @@ def test_binding_fails_loudly_without_cuda_tensors():
     k = torch.zeros((1, 1, 64, 128), dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         spa.spa_block_stats(k, 64)
+
+
+def test_decode_workload_fits_the_noalloc_scratch(lib):
+    # The allocation-free decode keeps its split-KV partials in a fixed 8 MiB
+    # device array; the decode workload (16 sequences, 32/8 heads, 131072 cached
+    # tokens, d = 128, block 16) must stay within it whatever the split heuristic.
+    f = lib.spa_decode_workspace_bytes
+    f.argtypes = [ctypes.c_int] * 6
+    f.restype = ctypes.c_size_t
+    assert 0 < f(16, 32, 8, 131072, 128, 16) <= 8 << 20

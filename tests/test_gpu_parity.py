@@ -257,10 +257,22 @@ def test_decode_random_lists_groupings_and_edges(Hq, Hkv, block, T):
     assert_no_device_error()
 
 
+def _prefill_matches_oracle(w, x, dev):
+    sel = oracle_select(w, x)
+    out, _ = spa.spa_sparse_attn_prefill(dev["q"], dev["k"], dev["v"], w.block,
+                                         torch.from_numpy(sel["idx"]).cuda(),
+                                         torch.from_numpy(sel["count"]).cuda(), w.scale)
+    torch.cuda.synchronize()
+    ref, _ = oracle.attention(x["q"], x["k"], x["v"], w.dtype, w.block, sel["idx"], sel["count"],
+                              w.scale)
+    assert float(np.abs(to_host(out) - ref).max()) <= TOL[w.dtype]
+
+
 def test_bounded_wait_runs_out_and_reports_timeout():
     # The failure path every kernel's waits share: a barrier that nothing completes.
     # The wait gives up after its limit, records the timeout in the device error
-    # word, and the context stays usable for the next launch.
+    # word, and the context stays usable for the next launch. The prefill kernel
+    # (whose waits are the same bounded waits) runs correctly after it.
     assert spa.spa_get_device_error() == 0
     spa.spa_selftest_wait_timeout(2000)
     assert spa.spa_get_device_error() == 3      # SPA_DEVERR_TIMEOUT
@@ -272,7 +284,21 @@ def test_bounded_wait_runs_out_and_reports_timeout():
     om, ov = oracle.block_stats(x["k"], w.dtype, w.block)
     np.testing.assert_allclose(mean.cpu().numpy(), om, rtol=1e-5, atol=1e-6)
     np.testing.assert_allclose(var.cpu().numpy(), ov, rtol=1e-5, atol=1e-6)
+    _prefill_matches_oracle(w, x, dev)
     assert_no_device_error()
+
+
+def test_timeout_ends_only_its_own_launch():
+    # A launch after a timed-out one, before anybody read the error word, still
+    # waits normally: giving up early is keyed to the launch that ran out. The code
+    # itself stays set until it is read.
+    assert spa.spa_get_device_error() == 0
+    w = PARITY_WORKLOADS["p_bf16_blk128"]
+    x, dev = inputs(w)
+    spa.spa_selftest_wait_timeout(2000)
+    _prefill_matches_oracle(w, x, dev)
+    assert spa.spa_get_device_error() == 3
+    assert spa.spa_get_device_error() == 0
 
 
 def test_corrupt_lists_are_reported_and_skipped():

@@ -3,9 +3,12 @@
 It serves callers that cannot allocate device memory for the call (a plugin
 interface that passes only input and output buffers, a hot loop that must not call
 cudaMalloc). These tests call it through the C-ABI and check that, on two calls in
-a row, it returns what the workspace-taking spa_sparse_attn_decode returns, and that
-sizes needing more scratch than the built-in 8 MiB are refused. This file is
-collected last, so a run that stops at its first failure has run everything else.
+a row, it returns bit for bit what the workspace-taking spa_sparse_attn_decode
+returns (the same kernels on the same inputs, only the partials live elsewhere),
+that both agree with the CPU oracle within the bf16 tolerance of the other parity
+tests, and that sizes needing more scratch than the built-in 8 MiB are refused.
+This file is collected last, so a run that stops at its first failure has run
+everything else.
 """
 import ctypes
 
@@ -14,6 +17,7 @@ import pytest
 import torch
 
 import block_sparse_long_stats_b200 as spa
+import oracle
 from workloads import PARITY_WORKLOADS, generate
 
 pytestmark = pytest.mark.gpu
@@ -42,6 +46,8 @@ def test_noalloc_decode_matches_workspace_decode_on_two_calls(key):
     idx, cnt = spa.spa_select(q, mean, var, w.T, w.block, w.scale, w.top_p)
     ref = spa.spa_sparse_attn_decode(q, k, v, w.block, idx, cnt, w.scale)
     torch.cuda.synchronize()
+    o_ref, _ = oracle.attention(x["q"], x["k"], x["v"], w.dtype, w.block, idx.cpu().numpy(),
+                                cnt.cpu().numpy(), w.scale)
     f = _noalloc()
     stream = P(torch.cuda.current_stream().cuda_stream)
     for call in range(2):
@@ -51,7 +57,8 @@ def test_noalloc_decode_matches_workspace_decode_on_two_calls(key):
                P(out.data_ptr()), stream)
         assert st == 0, spa.spa_last_error()
         torch.cuda.synchronize()
-        err = (out.float() - ref.float()).abs().max().item()
+        assert torch.equal(out.view(torch.int16), ref.view(torch.int16)), call
+        err = float(np.abs(out.float().cpu().numpy().reshape(o_ref.shape) - o_ref).max())
         assert err <= TOL, (call, err)
     assert spa.spa_get_device_error() == 0
 
