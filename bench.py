@@ -726,21 +726,26 @@ def main():
         torch.cuda.synchronize()
         assert spa.spa_get_device_error() == 0
         n_dec = max(10, args.steps // 2)
-        d_evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_dec)]
+        last = wd.nb - 1      # the block the new token lands in: its statistics are updated
+        # a decode step: statistics of the newest block, selection, attention
+        d_evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n_dec)]
         barrier()
         torch.cuda.synchronize()
         for s in range(n_dec):
             flush.zero_()
             d_evs[s][0].record(stream)
-            spa.spa_select(qd_, dm, dv, wd.T, wd.block, wd.scale, wd.top_p, idx=didx, count=dcnt)
+            spa.spa_block_stats(kc, wd.block, last, last + 1, mean=dm, var=dv)
             d_evs[s][1].record(stream)
+            spa.spa_select(qd_, dm, dv, wd.T, wd.block, wd.scale, wd.top_p, idx=didx, count=dcnt)
+            d_evs[s][2].record(stream)
             spa.spa_sparse_attn_decode(qd_, kc, vc, wd.block, didx, dcnt, wd.scale, workspace=ws,
                                        out=dout)
-            d_evs[s][2].record(stream)
+            d_evs[s][3].record(stream)
         torch.cuda.synchronize()
         barrier()
-        t_dsel = rank_max(statistics.mean(e[0].elapsed_time(e[1]) for e in d_evs))
-        t_dec = rank_max(statistics.mean(e[1].elapsed_time(e[2]) for e in d_evs))
+        t_dupd = rank_max(statistics.mean(e[0].elapsed_time(e[1]) for e in d_evs))
+        t_dsel = rank_max(statistics.mean(e[1].elapsed_time(e[2]) for e in d_evs))
+        t_dec = rank_max(statistics.mean(e[2].elapsed_time(e[3]) for e in d_evs))
         dbytes = kept_kv_bytes(dcnt.cpu().numpy(), didx.cpu().numpy(), wd.G, wd.T, wd.block, wd.d)
         gbs = dbytes / (t_dec / 1e3) / 1e9
         drla = None
@@ -805,32 +810,54 @@ def main():
                                          count=qc)
             torch.cuda.synchronize()
             assert spa.spa_get_device_error() == 0
-            qs_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                      for _ in range(n_dec)]
+            # the decode step on records: statistics and record of the newest block in
+            # one kernel, selection on the records, attention on its lists
+            qs_evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n_dec)]
+            qout = torch.empty_like(dout)
+            for _ in range(3):
+                spa.spa_block_stats_quantized(kc, wd.block, last, last + 1, dm, dv, qrec)
+                spa.spa_select_quantized(qd_, qrec, wd.T, wd.block, wd.scale, wd.top_p, idx=qi,
+                                         count=qc)
+                spa.spa_sparse_attn_decode(qd_, kc, vc, wd.block, qi, qc, wd.scale, workspace=ws,
+                                           out=qout)
+            torch.cuda.synchronize()
+            assert spa.spa_get_device_error() == 0
             barrier()
             torch.cuda.synchronize()
             for s in range(n_dec):
                 flush.zero_()
                 qs_evs[s][0].record(stream)
+                spa.spa_block_stats_quantized(kc, wd.block, last, last + 1, dm, dv, qrec)
+                qs_evs[s][1].record(stream)
                 spa.spa_select_quantized(qd_, qrec, wd.T, wd.block, wd.scale, wd.top_p, idx=qi,
                                          count=qc)
-                qs_evs[s][1].record(stream)
+                qs_evs[s][2].record(stream)
+                spa.spa_sparse_attn_decode(qd_, kc, vc, wd.block, qi, qc, wd.scale, workspace=ws,
+                                           out=qout)
+                qs_evs[s][3].record(stream)
             torch.cuda.synchronize()
             barrier()
-            t_qsel = rank_max(statistics.mean(a_.elapsed_time(b_) for a_, b_ in qs_evs))
+            t_qupd = rank_max(statistics.mean(e[0].elapsed_time(e[1]) for e in qs_evs))
+            t_qsel = rank_max(statistics.mean(e[1].elapsed_time(e[2]) for e in qs_evs))
+            t_qdec = rank_max(statistics.mean(e[2].elapsed_time(e[3]) for e in qs_evs))
+            qbytes = kept_kv_bytes(qc.cpu().numpy(), qi.cpu().numpy(), wd.G, wd.T, wd.block, wd.d)
             dq = {"stats_bytes_fp32": 2 * dm.numel() * 4, "stats_bytes_int4": qrec.numel(),
                   "quantize_full_cache_ms": statistics.median(q_ms[1:]),
-                  "select_ms": t_qsel,
+                  "update_newest_block_ms": t_qupd, "select_ms": t_qsel, "attn_ms": t_qdec,
+                  "kept_kv_bytes": qbytes, "GB/s": qbytes / (t_qdec / 1e3) / 1e9,
                   "kept_fraction": float(qc.float().mean().item()) / wd.nb,
-                  "tokens/s": world * wd.B / ((t_qsel + t_dec) / 1e3)}
+                  "tokens/s": world * wd.B / ((t_qupd + t_qsel + t_qdec) / 1e3)}
+            del qout
             del qrec, qi, qc
         decode = {"workload": wd.name, "kept_kv_bytes": dbytes, "attn_ms": t_dec,
-                  "select_ms": t_dsel,
+                  "update_newest_block_ms": t_dupd, "select_ms": t_dsel,
                   "select_GB/s": 2 * dm.numel() * 4 / (t_dsel / 1e3) / 1e9,
-                  "select_share_of_step": t_dsel / (t_dsel + t_dec),
+                  "select_share_of_step": t_dsel / (t_dupd + t_dsel + t_dec),
                   "GB/s": gbs, "peak_GB/s": peaks["hbm_gbs"],
                   "frac": gbs / peaks["hbm_gbs"], "peak_source": peak_src,
-                  "tokens/s": world * wd.B / ((t_dsel + t_dec) / 1e3),
+                  "tokens/s": world * wd.B / ((t_dupd + t_dsel + t_dec) / 1e3),
+                  "step": "statistics of the newest block, selection on fp32 statistics, "
+                          "attention; the step on INT4 records is quantized_stats",
                   "kept_fraction": float(dcnt.float().mean().item()) / wd.nb,
                   "kept_fraction_union": dbytes / float(2 * kc.numel() * kc.element_size()),
                   "block_stats_full_cache": stats_full, "rla": drla, "quantized_stats": dq}

@@ -8,7 +8,7 @@ from .spa import (SpaError, decode, lib, prefill, spa_block_stats, spa_decode_wo
                   spa_get_device_error, spa_last_error, spa_quantize_block_stats,
                   spa_quantized_stats_bytes, spa_rla_block_states, spa_rla_decode_state,
                   spa_rla_decode_workspace_bytes, spa_rla_prefill, spa_select_quantized,
-                  spa_select_score_order, spa_sparse_attn_prefill_early_stop,
+                  spa_select_score_order, spa_sparse_attn_prefill_early_stop, spa_block_stats_quantized,
                   spa_pbs_gather, spa_pbs_permutation, spa_pbs_workspace_bytes,
                   spa_select_segperm, spa_prefill_host, spa_prefill_host_workspace_bytes,
                   spa_selftest_wait_timeout, spa_sparse_attn_prefill_segperm,
@@ -18,7 +18,7 @@ from .spa import (SpaError, decode, lib, prefill, spa_block_stats, spa_decode_wo
 __all__ = ["SpaError", "decode", "lib", "prefill", "spa_block_stats",
            "spa_decode_workspace_bytes", "spa_get_device_error", "spa_last_error",
            "spa_quantize_block_stats", "spa_quantized_stats_bytes", "spa_select_quantized",
-           "spa_select_score_order", "spa_sparse_attn_prefill_early_stop",
+           "spa_select_score_order", "spa_sparse_attn_prefill_early_stop", "spa_block_stats_quantized",
            "spa_pbs_gather", "spa_pbs_permutation", "spa_pbs_workspace_bytes", "spa_select_segperm",
            "spa_prefill_host", "spa_prefill_host_workspace_bytes", "spa_selftest_wait_timeout",
            "spa_sparse_attn_prefill_segperm",

@@ -170,17 +170,6 @@ __device__ __forceinline__ void drain_ring(uint64_t *full, int n) {
     }
 }
 
-// Register reallocation between warpgroups (every warp of the warpgroup executes
-// it; the sum over the CTA must stay within the registers it was launched with).
-template <uint32_t N>
-__device__ __forceinline__ void regs_increase() {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
-}
-template <uint32_t N>
-__device__ __forceinline__ void regs_decrease() {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
-}
-
 // Named barrier over `nthreads` threads (a multiple of 32); id 0 is __syncthreads.
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");

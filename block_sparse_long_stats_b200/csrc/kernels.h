@@ -27,6 +27,10 @@ size_t quantized_stats_bytes(int B, int Hkv, int T, int d, int block);
 cudaError_t launch_quantize_stats(const float *mean, const float *var, int B, int Hkv, int T, int d,
                                   int block, int blk_begin, int blk_end, void *qstats,
                                   cudaStream_t s);
+// Statistics and records of blocks [blk_begin, blk_end) in one pass (few blocks).
+cudaError_t launch_stats_quantize(const void *k, bool bf16, int B, int Hkv, int T, int d,
+                                  int block, int blk_begin, int blk_end, float *mean, float *var,
+                                  void *qstats, cudaStream_t s);
 
 cudaError_t launch_prefill_f32(const float *q, const float *k, const float *v, int B, int Hq,
                                int Hkv, int L, int d, int block, const int32_t *idx, int cap,

@@ -39,31 +39,14 @@ __device__ __forceinline__ int group_exponent(float amax, float top) {
     return k;
 }
 
+// One lane's share of a record: features [lane * PL, lane * PL + PL) of the block's
+// mean m and variance v; the group maxima meet over the lanes of each 32-feature
+// group, then the lane writes its codes (and the group's first lane the exponents).
 template <int D>
-__global__ void __launch_bounds__(256) quantize_stats_kernel(const float *__restrict__ mean,
-                                                             const float *__restrict__ var, int nb,
-                                                             int blk_begin, int nblk, int units,
-                                                             uint8_t *__restrict__ qs) {
+__device__ __forceinline__ void quantize_lane(const float (&m)[D / 32], const float (&v)[D / 32],
+                                              int lane, uint8_t *rec) {
     constexpr int PL = D / 32;            // features per lane
     constexpr int LPG = 32 / PL;          // lanes per 32-feature group
-    constexpr int RB = D + D / 16;        // record bytes
-    const int lane = threadIdx.x & 31;
-    const int u = blockIdx.x * 8 + (threadIdx.x >> 5);
-    if (u >= units) return;               // warp-uniform
-    const int bg = u / nblk, j = blk_begin + u % nblk;
-    const size_t row = ((size_t)bg * nb + j) * D + lane * PL;
-    float m[PL], v[PL];
-    if constexpr (PL == 4) {
-        const float4 a = *reinterpret_cast<const float4 *>(mean + row);
-        const float4 b = *reinterpret_cast<const float4 *>(var + row);
-        m[0] = a.x; m[1] = a.y; m[2] = a.z; m[3] = a.w;
-        v[0] = b.x; v[1] = b.y; v[2] = b.z; v[3] = b.w;
-    } else {
-        const float2 a = *reinterpret_cast<const float2 *>(mean + row);
-        const float2 b = *reinterpret_cast<const float2 *>(var + row);
-        m[0] = a.x; m[1] = a.y;
-        v[0] = b.x; v[1] = b.y;
-    }
     float am = 0.f, av = 0.f;
 #pragma unroll
     for (int c = 0; c < PL; ++c) {
@@ -84,7 +67,6 @@ __global__ void __launch_bounds__(256) quantize_stats_kernel(const float *__rest
         pm |= (uint32_t)(qm & 15) << (4 * c);
         pv |= (uint32_t)qv << (4 * c);
     }
-    uint8_t *rec = qs + ((size_t)bg * nb + j) * RB;
     if constexpr (PL == 4) {
         reinterpret_cast<uint16_t *>(rec)[lane] = (uint16_t)pm;
         reinterpret_cast<uint16_t *>(rec + D / 2)[lane] = (uint16_t)pv;
@@ -96,6 +78,98 @@ __global__ void __launch_bounds__(256) quantize_stats_kernel(const float *__rest
         rec[D + lane / LPG] = (uint8_t)(int8_t)km;
         rec[D + D / 32 + lane / LPG] = (uint8_t)(int8_t)kv;
     }
+}
+
+template <int D>
+__global__ void __launch_bounds__(256) quantize_stats_kernel(const float *__restrict__ mean,
+                                                             const float *__restrict__ var, int nb,
+                                                             int blk_begin, int nblk, int units,
+                                                             uint8_t *__restrict__ qs) {
+    constexpr int PL = D / 32;            // features per lane
+    constexpr int RB = D + D / 16;        // record bytes
+    const int lane = threadIdx.x & 31;
+    const int u = blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (u >= units) return;               // warp-uniform
+    const int bg = u / nblk, j = blk_begin + u % nblk;
+    const size_t row = ((size_t)bg * nb + j) * D + lane * PL;
+    float m[PL], v[PL];
+    if constexpr (PL == 4) {
+        const float4 a = *reinterpret_cast<const float4 *>(mean + row);
+        const float4 b = *reinterpret_cast<const float4 *>(var + row);
+        m[0] = a.x; m[1] = a.y; m[2] = a.z; m[3] = a.w;
+        v[0] = b.x; v[1] = b.y; v[2] = b.z; v[3] = b.w;
+    } else {
+        const float2 a = *reinterpret_cast<const float2 *>(mean + row);
+        const float2 b = *reinterpret_cast<const float2 *>(var + row);
+        m[0] = a.x; m[1] = a.y;
+        v[0] = b.x; v[1] = b.y;
+    }
+    quantize_lane<D>(m, v, lane, qs + ((size_t)bg * nb + j) * RB);
+}
+
+// The statistics of a few blocks and their records in one pass (a decode step's
+// newest block): one warp per block, lane l holding features [l PL, l PL + PL);
+// mean, then the sum of squared deviations (a second read of the block's rows, from
+// L1), both over the block's rows in order, then the record of those fp32 values.
+template <typename T, int D>
+__global__ void __launch_bounds__(256) stats_quantize_kernel(const T *__restrict__ k, int T_len,
+                                                             int block, int nb, int blk_begin,
+                                                             int nblk, int units,
+                                                             float *__restrict__ mean,
+                                                             float *__restrict__ var,
+                                                             uint8_t *__restrict__ qs) {
+    constexpr int PL = D / 32;
+    constexpr int RB = D + D / 16;
+    const int lane = threadIdx.x & 31;
+    const int u = blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (u >= units) return;               // warp-uniform
+    const int bg = u / nblk, j = blk_begin + u % nblk;
+    const int t0 = j * block, n = min(block, T_len - t0);
+    const T *base = k + ((size_t)bg * T_len + t0) * D + lane * PL;
+    auto load = [&](int r, float (&x)[PL]) {
+        if constexpr (sizeof(T) == 2) {
+            if constexpr (PL == 4) {
+                const uint2 w = __ldg(reinterpret_cast<const uint2 *>(base + (size_t)r * D));
+                x[0] = bf16lo(w.x); x[1] = bf16hi(w.x); x[2] = bf16lo(w.y); x[3] = bf16hi(w.y);
+            } else {
+                const uint32_t w = __ldg(reinterpret_cast<const uint32_t *>(base + (size_t)r * D));
+                x[0] = bf16lo(w); x[1] = bf16hi(w);
+            }
+        } else {
+#pragma unroll
+            for (int c = 0; c < PL; ++c) x[c] = __ldg(reinterpret_cast<const float *>(base) + (size_t)r * D + c);
+        }
+    };
+    float m[PL], v[PL];
+#pragma unroll
+    for (int c = 0; c < PL; ++c) m[c] = v[c] = 0.f;
+    for (int r = 0; r < n; ++r) {
+        float x[PL];
+        load(r, x);
+#pragma unroll
+        for (int c = 0; c < PL; ++c) m[c] += x[c];
+    }
+    const float inv = 1.0f / (float)n;
+#pragma unroll
+    for (int c = 0; c < PL; ++c) m[c] *= inv;
+    for (int r = 0; r < n; ++r) {
+        float x[PL];
+        load(r, x);
+#pragma unroll
+        for (int c = 0; c < PL; ++c) {
+            const float dv = x[c] - m[c];
+            v[c] = fmaf(dv, dv, v[c]);
+        }
+    }
+#pragma unroll
+    for (int c = 0; c < PL; ++c) v[c] *= inv;
+    const size_t row = ((size_t)bg * nb + j) * D + lane * PL;
+#pragma unroll
+    for (int c = 0; c < PL; ++c) {
+        mean[row + c] = m[c];
+        var[row + c] = v[c];
+    }
+    quantize_lane<D>(m, v, lane, qs + ((size_t)bg * nb + j) * RB);
 }
 
 }  // namespace
@@ -116,6 +190,30 @@ cudaError_t launch_quantize_stats(const float *mean, const float *var, int B, in
         quantize_stats_kernel<128><<<grid, 256, 0, s>>>(mean, var, nb, blk_begin, nblk, units, q);
     else
         quantize_stats_kernel<64><<<grid, 256, 0, s>>>(mean, var, nb, blk_begin, nblk, units, q);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_stats_quantize(const void *k, bool bf16, int B, int Hkv, int T, int d,
+                                  int block, int blk_begin, int blk_end, float *mean, float *var,
+                                  void *qstats, cudaStream_t s) {
+    if (blk_end <= blk_begin) return cudaSuccess;
+    const int nb = (T + block - 1) / block, nblk = blk_end - blk_begin;
+    const int units = B * Hkv * nblk;
+    const unsigned grid = (unsigned)((units + 7) / 8);
+    uint8_t *q = reinterpret_cast<uint8_t *>(qstats);
+    if (bf16) {
+        const auto *kk = static_cast<const __nv_bfloat16 *>(k);
+        if (d == 128)
+            stats_quantize_kernel<__nv_bfloat16, 128><<<grid, 256, 0, s>>>(kk, T, block, nb, blk_begin, nblk, units, mean, var, q);
+        else
+            stats_quantize_kernel<__nv_bfloat16, 64><<<grid, 256, 0, s>>>(kk, T, block, nb, blk_begin, nblk, units, mean, var, q);
+    } else {
+        const auto *kk = static_cast<const float *>(k);
+        if (d == 128)
+            stats_quantize_kernel<float, 128><<<grid, 256, 0, s>>>(kk, T, block, nb, blk_begin, nblk, units, mean, var, q);
+        else
+            stats_quantize_kernel<float, 64><<<grid, 256, 0, s>>>(kk, T, block, nb, blk_begin, nblk, units, mean, var, q);
+    }
     return cudaGetLastError();
 }
 

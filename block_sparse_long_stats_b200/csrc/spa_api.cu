@@ -324,6 +324,26 @@ SPA_API spa_status spa_quantize_block_stats(const float *mean, const float *var,
     return e == cudaSuccess ? SPA_OK : cuda_fail(e, "quantize launch");
 }
 
+SPA_API spa_status spa_block_stats_quantized(const void *k, spa_dtype dt, int B, int Hkv, int T,
+                                             int d, int block, int blk_begin, int blk_end,
+                                             float *mean, float *var, void *qstats,
+                                             spa_stream stream) {
+    t_last_error.clear();
+    if (!k || !mean || !var || !qstats) return fail(SPA_ERR_INVALID, "null pointer");
+    if (B <= 0 || Hkv <= 0 || T <= 0 || d <= 0 || block <= 0)
+        return fail(SPA_ERR_INVALID, "sizes must be positive");
+    if (dt != SPA_F32 && dt != SPA_BF16) return fail(SPA_ERR_INVALID, "unknown dtype");
+    const int nb = ceil_div(T, block);
+    if (blk_begin < 0 || blk_end > nb || blk_begin > blk_end)
+        return fail(SPA_ERR_INVALID, "need 0 <= blk_begin <= blk_end <= nb");
+    if (!aligned16(k) || !aligned16(mean) || !aligned16(var) || !aligned16(qstats))
+        return fail(SPA_ERR_INVALID, "tensors must be 16-byte aligned");
+    if (d != 64 && d != 128) return fail(SPA_ERR_UNSUPPORTED, "d must be 64 or 128");
+    cudaError_t e = launch_stats_quantize(k, dt == SPA_BF16, B, Hkv, T, d, block, blk_begin, blk_end,
+                                          mean, var, qstats, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? SPA_OK : cuda_fail(e, "stats+quantize launch");
+}
+
 SPA_API spa_status spa_select_quantized(const void *q, spa_dtype dt, const void *qstats, int B,
                                         int Hq, int Hkv, int Lq, int T, int d, int block,
                                         float scale, float top_p, int n_sink, int n_local,

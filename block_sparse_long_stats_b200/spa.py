@@ -64,6 +64,7 @@ def lib() -> ctypes.CDLL:
         L.spa_quantized_stats_bytes.argtypes = [_I, _I, _I, _I, _I]
         L.spa_quantized_stats_bytes.restype = ctypes.c_size_t
         L.spa_quantize_block_stats.argtypes = [_P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P]
+        L.spa_block_stats_quantized.argtypes = [_P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P]
         L.spa_select_quantized.argtypes = [_P, _I, _P, _I, _I, _I, _I, _I, _I, _I, _F, _F, _I, _I,
                                            _I, _P, _I, _P, _P]
         L.spa_select_score_order.argtypes = [_P, _I, _P, _P, _I, _I, _I, _I, _I, _I, _F, _F, _I,
@@ -93,6 +94,7 @@ def lib() -> ctypes.CDLL:
                   "spa_sparse_attn_decode", "spa_get_device_error", "spa_rla_block_states",
                   "spa_rla_prefill", "spa_rla_decode_state", "spa_sparse_attn_decode_rla",
                   "spa_quantize_block_stats", "spa_select_quantized", "spa_select_score_order",
+                  "spa_block_stats_quantized",
                   "spa_sparse_attn_prefill_early_stop", "spa_pbs_permutation", "spa_pbs_gather",
                   "spa_select_segperm", "spa_sparse_attn_prefill_segperm", "spa_prefill_host",
                   "spa_selftest_wait_timeout"):
@@ -196,6 +198,17 @@ def spa_quantize_block_stats(mean: torch.Tensor, var: torch.Tensor, T: int, bloc
            lib().spa_quantize_block_stats(_ptr(mean), _ptr(var), B, Hkv, T, d, block, blk_begin,
                                           blk_end, _ptr(qstats), _stream(stream)))
     return qstats
+
+
+def spa_block_stats_quantized(k: torch.Tensor, block: int, blk_begin: int, blk_end: int,
+                              mean: torch.Tensor, var: torch.Tensor, qstats: torch.Tensor,
+                              stream=None) -> None:
+    """Statistics and INT4 records of blocks [blk_begin, blk_end) in one pass, into the
+    caller's mean, var [B, Hkv, nb, d] and qstats [B, Hkv, nb, d + d/16]."""
+    B, Hkv, T, d = k.shape
+    _check("spa_block_stats_quantized",
+           lib().spa_block_stats_quantized(_ptr(k), _dt(k), B, Hkv, T, d, block, blk_begin, blk_end,
+                                           _ptr(mean), _ptr(var), _ptr(qstats), _stream(stream)))
 
 
 def spa_select_quantized(q: torch.Tensor, qstats: torch.Tensor, T: int, block: int, scale: float,

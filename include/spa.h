@@ -139,6 +139,21 @@ spa_status spa_quantize_block_stats(const float *mean, const float *var, int B, 
                                     spa_stream stream);
 
 /*
+ * Block statistics and their INT4 records in one pass, for a few blocks (a decode
+ * step's newest block): for blocks [blk_begin, blk_end) of every (b, kv-head),
+ * mean and var exactly as spa_block_stats defines them (fp32, population variance,
+ * written into mean, var) and the record spa_quantize_block_stats makes of those
+ * fp32 values (written into qstats). One warp per block reads the block's keys
+ * twice (mean, then squared deviations); for a whole cache, spa_block_stats followed
+ * by spa_quantize_block_stats is faster.
+ *   k : [B, Hkv, T, d] (dt), d = 64 or 128; mean, var, qstats as in the two calls;
+ *   blocks outside the range are left untouched. Errors as spa_block_stats.
+ */
+spa_status spa_block_stats_quantized(const void *k, spa_dtype dt, int B, int Hkv, int T, int d,
+                                     int block, int blk_begin, int blk_end, float *mean,
+                                     float *var, void *qstats, spa_stream stream);
+
+/*
  * spa_select on quantised statistics: the same score, cut and output, with each
  * block's mean and variance read back from its record (code * 2^k) instead of
  * from fp32 arrays. Arguments as spa_select, with qstats in place of mean, var.

@@ -64,6 +64,30 @@ def test_quantizer_range_leaves_others_untouched():
     assert np.array_equal(r[:, :, w.nb - 3:], full[:, :, w.nb - 3:])
 
 
+@pytest.mark.parametrize("key", ["d_bf16_blk16", "d_bf16_blk64", "p_f32_d64", "p_bf16_blk128"])
+def test_fused_stats_and_records_of_a_block_range(key):
+    # spa_block_stats_quantized on the last blocks (a decode step's update): its
+    # statistics match the oracle's, its records are exactly the oracle's quantiser
+    # applied to those fp32 statistics, and blocks outside the range are untouched
+    w = PARITY_WORKLOADS[key]
+    x, dev = inputs(w)
+    nb = w.nb
+    lo = max(0, nb - 3)
+    mean = torch.full((w.B, w.Hkv, nb, w.d), 7.0, device="cuda")
+    var = torch.full_like(mean, 7.0)
+    rec = torch.full((w.B, w.Hkv, nb, w.d + w.d // 16), 0xAB, device="cuda", dtype=torch.uint8)
+    spa.spa_block_stats_quantized(dev["k"], w.block, lo, nb, mean, var, rec)
+    torch.cuda.synchronize()
+    om, ov = oracle.block_stats(x["k"], w.dtype, w.block)
+    m, v, r = mean.cpu().numpy(), var.cpu().numpy(), rec.cpu().numpy()
+    np.testing.assert_allclose(m[:, :, lo:], om[:, :, lo:], rtol=1e-5, atol=1e-6)
+    np.testing.assert_allclose(v[:, :, lo:], ov[:, :, lo:], rtol=1e-5, atol=1e-6)
+    assert np.all(m[:, :, :lo] == 7.0) and np.all(r[:, :, :lo] == 0xAB)
+    o = oracle.quantize_stats(m[:, :, lo:].astype(np.float64), v[:, :, lo:].astype(np.float64))
+    assert np.array_equal(r[:, :, lo:], pack_qstats(o))
+    assert spa.spa_get_device_error() == 0
+
+
 @pytest.mark.parametrize("key", list(PARITY_WORKLOADS))
 def test_select_quantized_on_oracle_records(key):
     w = PARITY_WORKLOADS[key]
