@@ -24,9 +24,12 @@ statistics -> Taylor-score top-p selection -> block-sparse causal attention
 reference arm of this comparison) and prints the same line with "impl":
 "reference".
 
-Multi-GPU: one process per GPU (torchrun); every rank runs its own replica of the
-workload (the units are independent, so the path needs no collective); the time
-is the max over ranks and the value counts the tokens of all ranks.
+Multi-GPU: one process per GPU (torchrun); each rank takes a contiguous share of
+the workload's (b, kv-head) units, its kv-heads with their query heads (the units
+are independent through every kernel, so the path needs no collective and the
+output stays head-sharded); the time is the max over ranks and the value counts
+every token of the job once (strong scaling). The legs beside the headline step
+run on one GPU only.
 """
 from __future__ import annotations
 
@@ -107,11 +110,22 @@ def kept_kv_bytes(count: np.ndarray, idx: np.ndarray, G: int, T: int, block: int
 def workload_config(w, n_gpus: int) -> dict:
     """The `config` of the JSON line, identical for the CUDA arm and the reference arm."""
     return {"workload": w.name, "B": w.B, "L": w.T, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d,
-            "block": w.block, "top_p": w.top_p, "parallelism": f"replicas x{n_gpus}",
+            "block": w.block, "top_p": w.top_p,
+            "parallelism": "one GPU" if n_gpus == 1 else f"(b, kv-head) units split over {n_gpus} GPUs",
             "l2": "flushed (256 MiB memset) between timed steps"}
 
 
 # ---------------------------------------------------------------- ranks
+
+def head_shard(B: int, Hkv: int, world: int, rank: int) -> tuple[int, int]:
+    """The (b, kv-head) units rank `rank` of `world` takes: a contiguous share
+    [u0, u1) of the B * Hkv units in (b, kv-head) order. Each unit is an independent
+    problem through every kernel (its kv-head's statistics, its query heads'
+    selection and attention), so a rank needs no other rank's data and the output
+    stays head-sharded, as tensor-parallel attention keeps it."""
+    U = B * Hkv
+    return rank * U // world, (rank + 1) * U // world
+
 
 def max_over_ranks(v: float, world: int, device) -> float:
     """Max of a per-rank device time over all ranks (all_reduce MAX; no-op on one rank)."""
@@ -222,7 +236,7 @@ def run_reference(args, rank: int):
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": w.B * w.Lq / value * 1e3, "higher_is_better": True, "scaling": "weak",
+        "ms_per_step": w.B * w.Lq / value * 1e3, "higher_is_better": True, "scaling": "strong",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(w, args.gpus),
         "extrapolated": True,
@@ -401,8 +415,24 @@ def main():
         return max_over_ranks(v, world, "cuda")
 
     peaks, peak_src = load_peaks()
-    w = WORKLOADS[args.workload]
-    x = generate(w)
+    w_full = WORKLOADS[args.workload]
+    # one GPU: the whole workload; N GPUs: each takes a contiguous share of the
+    # (b, kv-head) units (whole batch rows, kv-heads with their query heads), so the
+    # job processes every token once (strong scaling; no data-path collective)
+    u0, u1 = head_shard(w_full.B, w_full.Hkv, world, rank)
+    if world > 1 and not (w_full.B == 1 or (u1 - u0) % w_full.Hkv == 0):
+        raise SystemExit("head sharding needs whole batch rows or one batch row")
+    if w_full.B == 1:
+        g0, g1 = u0, u1
+        x = generate(w_full, heads=[(0, g) for g in range(g0, g1)])
+        G_ = w_full.G
+        x = {"q": x["q"][:, g0 * G_:g1 * G_], "k": x["k"][:, g0:g1], "v": x["v"][:, g0:g1]}
+        w = w_full.with_(Hq=(g1 - g0) * G_, Hkv=g1 - g0)
+    else:
+        b0, b1 = u0 // w_full.Hkv, u1 // w_full.Hkv
+        x = generate(w_full, heads=[(b, g) for b in range(b0, b1) for g in range(w_full.Hkv)])
+        x = {n: a[b0:b1] for n, a in x.items()}
+        w = w_full.with_(B=b1 - b0)
 
     def dev(a):
         if w.dtype == "bf16":
@@ -458,7 +488,8 @@ def main():
     t_step = [e[0].elapsed_time(e[3]) for e in evs]
     total_ms = rank_max(sum(t_step))
     ms_per_step = total_ms / args.steps
-    value = job_throughput(B * L, world, args.steps, total_ms)
+    # every token of the job once per step (the ranks hold disjoint head shares)
+    value = job_throughput(w_full.B * L, 1, args.steps, total_ms)
 
     count_h = cnt.cpu().numpy()
     idx_h = idx.cpu().numpy()
@@ -509,15 +540,17 @@ def main():
     torch.cuda.synchronize()
     barrier()
     e2e_ms = rank_max(sum(a.elapsed_time(b) for a, b in e_evs)) / args.e2e_steps
-    e2e = {"value": job_throughput(B * L, world, 1, e2e_ms), "unit": "tokens/s",
-           "h2d_bytes_per_step": int((qh.numel() + kh.numel() + vh.numel()) * 2),
-           "d2h_bytes_per_step": int(oh.numel() * 2), "ms_per_step": e2e_ms,
+    e2e = {"value": job_throughput(w_full.B * L, 1, 1, e2e_ms), "unit": "tokens/s",
+           "h2d_bytes_per_step": int((qh.numel() + kh.numel() + vh.numel()) * 2) * world,
+           "d2h_bytes_per_step": int(oh.numel() * 2) * world, "ms_per_step": e2e_ms,
            "api": "spa_prefill_host (pinned host buffers, copies pipelined with the kernels)"}
     del qh, kh, vh, oh, ws
 
     # ---- Residual Linear Attention leg (the branch over the blocks the lists leave out)
     rla = None
-    if not args.no_rla:
+    # the legs beside the headline step run on one GPU (the scaling run times the step)
+    legs = world == 1
+    if legs and not args.no_rla:
         states = torch.empty((B, Hkv, nb, d, d), device="cuda", dtype=torch.bfloat16)
         rout = torch.empty((B, Hq, L, d), device="cuda", dtype=torch.float32)
         for _ in range(3):
@@ -559,7 +592,7 @@ def main():
     # stays within 1.1 x the MSE of the top-p selection alone (the error budget)
     early = None
     taus = [float(t) for t in args.taus.split(",") if t.strip()]
-    if taus and w.block == 128 and w.dtype == "bf16":
+    if legs and taus and w.block == 128 and w.dtype == "bf16":
         oidx = torch.empty_like(idx)
         ocnt = torch.empty_like(cnt)
         proc = torch.empty_like(cnt)
@@ -632,7 +665,7 @@ def main():
 
     # ---- segmented key permutation (PBS, sections 2-3)
     pbs = None
-    if args.seg_blocks > 0 and w.dtype == "bf16" and args.seg_blocks * w.block <= 8192:
+    if legs and args.seg_blocks > 0 and w.dtype == "bf16" and args.seg_blocks * w.block <= 8192:
         perm = torch.empty((B, Hkv, L), device="cuda", dtype=torch.int32)
         pws = torch.empty(spa.spa_pbs_workspace_bytes(B, Hq, Hkv, L, w.block), dtype=torch.uint8,
                           device="cuda")
@@ -691,7 +724,7 @@ def main():
 
     # ---- decode leg
     decode = None
-    if not args.no_decode:
+    if legs and not args.no_decode:
         wd = WORKLOADS[args.decode_workload]
         if args.decode_batch:
             wd = wd.with_(B=args.decode_batch)
@@ -865,7 +898,7 @@ def main():
 
     # ---- the other prefill workloads, each timed like the headline step
     configs = {}
-    for cid in [int(c) for c in args.configs.split(",") if c.strip()]:
+    for cid in ([int(c) for c in args.configs.split(",") if c.strip()] if legs else []):
         if cid == args.workload or WORKLOADS[cid].mode != "prefill":
             continue
         n_st = {1: max(args.steps, 20), 4: min(args.steps, 8)}.get(cid, args.steps)
@@ -876,7 +909,7 @@ def main():
     # ---- selection diagnostics on the three prefill workloads (dense comparisons
     # on the 1K, 8K and 32K workloads only; the 128K one would need 140 TFLOP more)
     diag = None
-    if rank == 0 and not args.no_diagnostics:
+    if legs and not args.no_diagnostics:
         diag = {}
         for cid in (1, 2, args.workload):
             wl = WORKLOADS[cid]
@@ -910,9 +943,9 @@ def main():
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
-            "config": workload_config(w, world),
+            "config": workload_config(w_full, world),
             "kept_fraction": kept_frac,
             "roofline": {"bound": "tensor", "kernel": "sparse_attn_prefill", "achieved": achieved,
                          "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,

@@ -215,6 +215,88 @@ block_stats_kernel(const T *__restrict__ k, int T_len, int nb, int blk_begin, in
     }
 }
 
+// Blocks of 64 or more keys: one CTA per block, every load of the block issued at
+// once. Thread t owns 16-byte column chunk t % CPR of rows t / CPR, t / CPR + RG, ...
+// (RG = 256 / CPR row groups), so a block's bytes are all in flight before any is
+// reduced; the column sums meet in shared memory (mean), then the squared
+// deviations from the registers (variance). Several CTAs per SM keep enough bytes in
+// flight to cover the DRAM latency on short launches (the 32K workload's 66 MB).
+template <typename T, int D, int BLOCK>
+__global__ void __launch_bounds__(kThreads) block_stats_cta_kernel(const T *__restrict__ k, int T_len,
+                                                                   int nb, int blk_begin, int nblk,
+                                                                   float *__restrict__ mean,
+                                                                   float *__restrict__ var) {
+    constexpr int V = Elem<T>::kPerChunk;           // values per 16-byte chunk
+    constexpr int CPR = D / V;                      // chunks per row
+    constexpr int RG = kThreads / CPR;              // row groups
+    constexpr int RPT = BLOCK / RG;                 // rows per thread
+    static_assert(RPT * RG == BLOCK && RPT >= 1, "unsupported shape");
+    __shared__ float part[RG][D + 1];
+    __shared__ float colv[D];
+    const int u = blockIdx.x;
+    const int bg = u / nblk, j = blk_begin + u % nblk;
+    const int t0 = j * BLOCK, n = min(BLOCK, T_len - t0);
+    const int c = threadIdx.x % CPR, rg = threadIdx.x / CPR;
+    const uint4 *src = reinterpret_cast<const uint4 *>(k + ((size_t)bg * T_len + t0) * D) + c;
+    uint4 raw[RPT];
+#pragma unroll
+    for (int i = 0; i < RPT; ++i) {
+        const int r = rg + i * RG;
+        raw[i] = r < n ? __ldg(src + (size_t)r * CPR) : make_uint4(0, 0, 0, 0);
+    }
+    float s[V];
+#pragma unroll
+    for (int v = 0; v < V; ++v) s[v] = 0.f;
+#pragma unroll
+    for (int i = 0; i < RPT; ++i) {          // rows past the end were loaded as zeros
+        float x[V];
+        Elem<T>::unpack(raw[i], x);
+#pragma unroll
+        for (int v = 0; v < V; ++v) s[v] += x[v];
+    }
+#pragma unroll
+    for (int v = 0; v < V; ++v) part[rg][c * V + v] = s[v];
+    __syncthreads();
+    const float inv = 1.0f / (float)n;
+    for (int col = threadIdx.x; col < D; col += kThreads) {
+        float a = 0.f;
+#pragma unroll
+        for (int g = 0; g < RG; ++g) a += part[g][col];
+        colv[col] = a * inv;
+    }
+    __syncthreads();
+    float mu[V];
+#pragma unroll
+    for (int v = 0; v < V; ++v) {
+        mu[v] = colv[c * V + v];
+        s[v] = 0.f;
+    }
+#pragma unroll
+    for (int i = 0; i < RPT; ++i) {
+        if (rg + i * RG < n) {
+            float x[V];
+            Elem<T>::unpack(raw[i], x);
+#pragma unroll
+            for (int v = 0; v < V; ++v) {
+                const float dv = x[v] - mu[v];
+                s[v] = fmaf(dv, dv, s[v]);
+            }
+        }
+    }
+    __syncthreads();                         // every thread has read colv and part
+#pragma unroll
+    for (int v = 0; v < V; ++v) part[rg][c * V + v] = s[v];
+    __syncthreads();
+    const size_t o = ((size_t)bg * nb + j) * D;
+    for (int col = threadIdx.x; col < D; col += kThreads) {
+        float a = 0.f;
+#pragma unroll
+        for (int g = 0; g < RG; ++g) a += part[g][col];
+        mean[o + col] = colv[col];
+        var[o + col] = a * inv;
+    }
+}
+
 template <typename T, int D, int BLOCK>
 cudaError_t launch_t(const void *k, int B, int Hkv, int T_len, int blk_begin, int blk_end,
                      float *mean, float *var, cudaStream_t s) {
@@ -223,6 +305,11 @@ cudaError_t launch_t(const void *k, int B, int Hkv, int T_len, int blk_begin, in
     using S = StatsShape<T, D, BLOCK>;
     constexpr int SPW = S::NC > kThreads / 32 ? S::NC / (kThreads / 32) : 1;
     constexpr int BPT = (kThreads / 32) / (S::NC / SPW);   // blocks per tile
+    if constexpr (BLOCK >= 64) {
+        block_stats_cta_kernel<T, D, BLOCK><<<units, kThreads, 0, s>>>(
+            reinterpret_cast<const T *>(k), T_len, nb, blk_begin, nblk, mean, var);
+        return cudaGetLastError();
+    }
     const int tiles = (units + BPT - 1) / BPT;
     const unsigned grid = (unsigned)std::min(tiles, 148 * kCtasPerSm);
     block_stats_kernel<T, D, BLOCK><<<grid, kThreads, 0, s>>>(

@@ -24,7 +24,7 @@ def test_reference_arm_prints_one_contract_line():
     assert d["value"] > 0 and d["unit"] == "tokens/s" and d["higher_is_better"] is True
     assert d["n_gpus"] == 1 and d["steps"] == 1
     assert d["warmup"] >= 3                      # the timing rules' minimum is enforced
-    assert d["scaling"] == "weak" and d["data"] == "synthetic" and d["vs_baseline"] is None
+    assert d["scaling"] == "strong" and d["data"] == "synthetic" and d["vs_baseline"] is None
     assert d["config"]["workload"] == "prefill_f32_L1024_H1_d64_blk64"
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"]

@@ -1,6 +1,7 @@
 """The multi-rank logic of bench.py with two gloo ranks on the CPU: the device
 time is the max over ranks, the value counts the work of every rank, and the
-reference arm runs on rank 0 only. CPU only."""
+reference arm runs on rank 0 only; the ranks' head shares cover every (b,
+kv-head) unit once. CPU only."""
 import os
 import socket
 
@@ -58,3 +59,30 @@ def test_two_gloo_ranks_take_the_max_time_and_count_all_work():
 def test_single_rank_is_the_identity():
     assert bench.max_over_ranks(12.5, 1, "cpu") == 12.5
     assert bench.job_throughput(100, 1, 4, 200.0) == pytest.approx(2000.0)
+
+
+@pytest.mark.parametrize("B,Hkv,world", [(1, 8, 1), (1, 8, 2), (1, 8, 4), (1, 8, 8), (16, 8, 4),
+                                         (2, 8, 4), (1, 6, 4)])
+def test_head_shards_cover_every_unit_once(B, Hkv, world):
+    # the ranks' shares of the (b, kv-head) units are contiguous, disjoint, cover all
+    # units and differ in size by at most one
+    shards = [bench.head_shard(B, Hkv, world, r) for r in range(world)]
+    assert shards[0][0] == 0 and shards[-1][1] == B * Hkv
+    assert all(shards[r][1] == shards[r + 1][0] for r in range(world - 1))
+    sizes = [u1 - u0 for u0, u1 in shards]
+    assert max(sizes) - min(sizes) <= 1
+
+
+def test_head_shard_data_equals_the_full_draw():
+    # a rank draws only its kv-heads (with their query heads) and gets exactly the
+    # slices of the full workload
+    from workloads import PARITY_WORKLOADS, generate
+    w = PARITY_WORKLOADS["p_bf16_blk128"].with_(B=1)
+    full = generate(w)
+    G = w.Hq // w.Hkv
+    for r in range(2):
+        g0, g1 = bench.head_shard(1, w.Hkv, 2, r)
+        part = generate(w, heads=[(0, g) for g in range(g0, g1)])
+        assert (part["q"][:, g0 * G:g1 * G] == full["q"][:, g0 * G:g1 * G]).all()
+        assert (part["k"][:, g0:g1] == full["k"][:, g0:g1]).all()
+        assert (part["v"][:, g0:g1] == full["v"][:, g0:g1]).all()
