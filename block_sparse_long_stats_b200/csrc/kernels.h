@@ -46,8 +46,8 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, int B
                               int seg_blocks = 0);
 
 // Segmented key permutation: perm [B, Hkv, L] (original index per permuted
-// position; it holds the importances between the passes) from the workspace of
-// pbs_workspace_bytes, and the permuted copy of K or V (rows of row_bytes bytes).
+// position), with the workspace of pbs_workspace_bytes, and the permuted copy of K
+// or V (rows of row_bytes bytes).
 size_t pbs_workspace_bytes(int B, int Hq, int Hkv, int L, int block);
 cudaError_t launch_pbs_permutation(const void *q, const void *k, bool bf16, int B, int Hq, int Hkv,
                                    int L, int d, int block, int seg_blocks, float scale,

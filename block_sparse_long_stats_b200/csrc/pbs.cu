@@ -9,21 +9,22 @@
 // importance(u) = (1 / R) sum_rows a_{h,t}(u). Equal importances keep the smaller
 // index first.
 //
-// Three passes over the keys of each (b, kv-head), in chunks of kChunk keys:
-//   pbs_rowstats: per (chunk, row) the running maximum and sum of exp2 of the
-//     row's logits over the chunk's visible keys (log2 units) -> workspace;
-//   pbs_lse: per row, the chunks' partials merged into lse2 = m + log2(sum);
-//   pbs_importance: per key, sum over the rows of exp2(logit - lse2), / R, written
-//     as fp32 bits into perm (perm doubles as the importance buffer).
+// Three passes over each (b, kv-head), one CTA per (range of 1024 keys, block of 128
+// rows), a warp holding the A fragments of 16 rows while the range's keys pass
+// through shared memory 128 at a time (two buffers filled by cp.async):
+//   pbs_rowstats (IMP = false): per (range, row) the running maximum and sum of exp2
+//     of the row's logits over the range's visible keys (log2 units) -> workspace;
+//   pbs_lse: per row, the ranges' partials merged into lse2 = m + log2(sum);
+//   pbs_importance (IMP = true): per key, the sum over the block's rows of
+//     exp2(logit - lse2) -> workspace, one partial per row block.
 // For bf16 the logits are mma.sync m16n8k16 products (bf16 products are exact in
-// the fp32 accumulator): a warp holds the A fragments of 16 rows and walks the
-// chunk's keys, staged in padded shared memory, eight at a time. fp32 inputs take
-// plain per-thread dot products (the small fp32 workloads only).
-// pbs_sort_kernel: one CTA per (segment, b * Hkv + g) reads its segment's
-// importances, then a bitonic sort of 64-bit keys (order-flipped importance |
-// index): segments up to 2048 keys in registers (eight per thread; shuffles for
-// strides up to 128, shared memory for the six larger ones), longer ones in shared
-// memory; writes perm over the importances it read.
+// the fp32 accumulator). fp32 inputs take plain per-thread dot products (the small
+// fp32 workloads only).
+// pbs_sort_kernel: one CTA per (segment, b * Hkv + g) adds its segment's row-block
+// partials in order (/ R: the importance), then sorts 64-bit keys (order-flipped
+// importance | index) with a bitonic network: segments up to 2048 keys in registers
+// (eight per thread; shuffles for strides up to 128, shared memory for the six
+// larger ones), longer ones in shared memory; writes perm.
 // gather_rows_kernel: the permuted copy of K or V, 16 bytes per thread.
 #include <float.h>
 
@@ -44,17 +45,28 @@ __device__ __forceinline__ uint32_t order_desc(float f) {
     return ~ord;                                                        // descending with f
 }
 
-constexpr int kChunk = 128;              // keys per CTA in the importance passes
+constexpr int kKeyRange = 1024;          // keys per CTA in the importance passes
+constexpr int kChunkKeys = 128;          // keys staged in shared memory at a time
+constexpr int kRowBlock = 128;           // rows per CTA (eight warps of 16)
 
 __host__ __device__ __forceinline__ int last_block_rows(int L, int block) {
     const int nq = (L + block - 1) / block;
     return L - (nq - 1) * block;
 }
 
-// Workspace of one (b, kv-head): partials [nchunks][R] (m2, s) then lse2 [R].
-__host__ __device__ __forceinline__ size_t ws_floats_per_group(int R, int nchunks) {
-    return (size_t)nchunks * R * 2 + R;
-}
+// Workspace of one (b, kv-head), R rows, L keys:
+//   part [nkr][R]   (m2, s): each key range's maximum and sum of exp2 per row
+//   lse2 [R]        per row, over all keys (log2 units)
+//   imp  [nrb][L]   per row block of 128 rows, the sum of the rows' weights per key
+struct PbsLayout {
+    int R, nkr, nrb;
+    __host__ __device__ PbsLayout(int R_, int L) : R(R_), nkr((L + kKeyRange - 1) / kKeyRange),
+                                                   nrb((R_ + kRowBlock - 1) / kRowBlock) {}
+    __host__ __device__ size_t floats(int L) const { return (size_t)nkr * R * 2 + R + (size_t)nrb * L; }
+    __host__ __device__ float2 *part(float *g) const { return reinterpret_cast<float2 *>(g); }
+    __host__ __device__ float *lse2(float *g) const { return g + (size_t)nkr * R * 2; }
+    __host__ __device__ float *imp(float *g) const { return g + (size_t)nkr * R * 2 + R; }
+};
 
 __device__ __forceinline__ void mma_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
                                           uint32_t b1) {
@@ -64,6 +76,16 @@ __device__ __forceinline__ void mma_16816(float (&c)[4], const uint32_t (&a)[4],
         : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
+
+// 16-byte global -> shared copy that bypasses the registers; zero-filled when !valid.
+__device__ __forceinline__ void cp_async16(void *dst, const void *src, bool valid) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src),
+                 "r"(valid ? 16 : 0)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 // Merge a (maximum, sum of exp2 relative to it) pair into another.
 __device__ __forceinline__ void merge_ms(float &m, float &s, float m2, float s2) {
@@ -78,45 +100,51 @@ __device__ __forceinline__ void merge_ms(float &m, float &s, float m2, float s2)
     m = mn;
 }
 
-// bf16: one CTA per (key chunk, b * Hkv + g). IMP = false: row partials; true:
-// importances (needs lse2). Rows x in [0, R): head x / n_r, position r0 + x % n_r.
+// bf16: one CTA per (key range, row block, b * Hkv + g). IMP = false: row partials
+// over the key range; true: per key the sum over the row block's rows of
+// exp2(logit - lse2). Rows x in [0, R): head x / n_r, position r0 + x % n_r; a warp
+// holds the A fragments of its 16 rows for the whole key range, and the range's
+// keys pass through shared memory 128 at a time (two buffers, cp.async).
 template <int D, bool IMP>
 __global__ void __launch_bounds__(kThreads) pbs_scores_bf16_kernel(
     const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k, int Hq, int Hkv,
-    int L, int block, float scale_log2, int nchunks, float *__restrict__ ws,
-    int32_t *__restrict__ perm) {
+    int L, int block, float scale_log2, float *__restrict__ ws) {
     constexpr int KW = D / 2 + 4;                 // padded key row in 32-bit words
-    constexpr int NT = kChunk / 8;                // n-tiles of 8 keys
-    __shared__ __align__(16) uint32_t ks[kChunk * KW];
-    __shared__ float colsum[IMP ? kWarps : 1][IMP ? kChunk : 1];
+    constexpr int NT = kChunkKeys / 8;            // n-tiles of 8 keys per chunk
+    constexpr int CPR = D / 8;                    // 16-byte chunks per key row
+    extern __shared__ __align__(16) uint32_t ks[];   // [2][kChunkKeys * KW]
+    __shared__ float colsum[IMP ? kWarps : 1][IMP ? kChunkKeys : 1];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int gid = lane >> 2, tig = lane & 3;
-    const int bg = blockIdx.y, b = bg / Hkv, g = bg % Hkv, G = Hq / Hkv;
+    const int bg = blockIdx.z, b = bg / Hkv, g = bg % Hkv, G = Hq / Hkv;
     const int nr = last_block_rows(L, block), r0 = L - nr, R = G * nr;
-    const int u0 = blockIdx.x * kChunk, nk = min(kChunk, L - u0);
-    float *part = ws + (size_t)bg * ws_floats_per_group(R, nchunks);
-    const float *lse2 = part + (size_t)nchunks * R * 2;
+    const PbsLayout lay(R, L);
+    float *wsg = ws + (size_t)bg * lay.floats(L);
+    const int u_begin = blockIdx.x * kKeyRange, u_end = min(L, u_begin + kKeyRange);
+    const int nch = (u_end - u_begin + kChunkKeys - 1) / kChunkKeys;
+    const __nv_bfloat16 *kbase = k + (size_t)bg * L * D;
 
-    for (int x = tid; x < kChunk * (D / 8); x += kThreads) {
-        const int row = x / (D / 8), c = x % (D / 8);
-        const uint4 v = row < nk ? __ldg(reinterpret_cast<const uint4 *>(k + ((size_t)bg * L + u0 + row) * D) + c)
-                                 : make_uint4(0, 0, 0, 0);
-        *reinterpret_cast<uint4 *>(&ks[row * KW + c * 4]) = v;
-    }
-    __syncthreads();
+    auto load_chunk = [&](int c) {
+        uint32_t *dst = ks + (c & 1) * kChunkKeys * KW;
+        const int u0 = u_begin + c * kChunkKeys;
+        for (int x = tid; x < kChunkKeys * CPR; x += kThreads) {
+            const int row = x / CPR, cc = x % CPR;
+            const bool valid = u0 + row < u_end;
+            cp_async16(&dst[row * KW + cc * 4], kbase + (size_t)(valid ? u0 + row : u_begin) * D + cc * 8, valid);
+        }
+        cp_async_commit();
+    };
+    load_chunk(0);
 
-    float cs[NT][2];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) cs[nt][0] = cs[nt][1] = 0.f;
-    for (int rg = warp; rg * 16 < R; rg += kWarps) {
-        const int xa = rg * 16 + gid, xb = xa + 8;
-        const bool va = xa < R, vb = xb < R;
-        const int ta = va ? r0 + xa % nr : -1, tb = vb ? r0 + xb % nr : -1;
+    const int xa = blockIdx.y * kRowBlock + warp * 16 + gid, xb = xa + 8;
+    const bool va = xa < R, vb = xb < R;
+    const int ta = va ? r0 + xa % nr : -1, tb = vb ? r0 + xb % nr : -1;
+    uint32_t af[D / 16][4];
+    {
         const uint32_t *qa = reinterpret_cast<const uint32_t *>(
             q + (((size_t)b * Hq + g * G + (va ? xa / nr : 0)) * L + (va ? ta : r0)) * D);
         const uint32_t *qb = reinterpret_cast<const uint32_t *>(
             q + (((size_t)b * Hq + g * G + (vb ? xb / nr : 0)) * L + (vb ? tb : r0)) * D);
-        uint32_t af[D / 16][4];
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
             af[kk][0] = __ldg(qa + kk * 8 + tig);
@@ -124,19 +152,32 @@ __global__ void __launch_bounds__(kThreads) pbs_scores_bf16_kernel(
             af[kk][2] = __ldg(qa + kk * 8 + 4 + tig);
             af[kk][3] = __ldg(qb + kk * 8 + 4 + tig);
         }
-        float la = 0.f, lb = 0.f;
-        if constexpr (IMP) {
-            la = va ? lse2[xa] : 0.f;
-            lb = vb ? lse2[xb] : 0.f;
+    }
+    float la = 0.f, lb = 0.f;
+    if constexpr (IMP) {
+        const float *l2 = lay.lse2(wsg);
+        la = va ? l2[xa] : 0.f;
+        lb = vb ? l2[xb] : 0.f;
+    }
+    float ma = -INFINITY, sa = 0.f, mb = -INFINITY, sb = 0.f;
+    for (int c = 0; c < nch; ++c) {
+        if (c + 1 < nch) {
+            load_chunk(c + 1);
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
         }
-        float ma = -INFINITY, sa = 0.f, mb = -INFINITY, sb = 0.f;
+        __syncthreads();
+        const uint32_t *kc = ks + (c & 1) * kChunkKeys * KW;
+        const int u0 = u_begin + c * kChunkKeys;
+        float cs[NT][2];
 #pragma unroll
         for (int sub = 0; sub < NT / 8; ++sub) {
             float z[8][4];
 #pragma unroll
             for (int nt = 0; nt < 8; ++nt) {
                 z[nt][0] = z[nt][1] = z[nt][2] = z[nt][3] = 0.f;
-                const uint32_t *kr = &ks[(sub * 64 + nt * 8 + gid) * KW];
+                const uint32_t *kr = &kc[(sub * 64 + nt * 8 + gid) * KW];
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) mma_16816(z[nt], af[kk], kr[kk * 8 + tig], kr[kk * 8 + 4 + tig]);
             }
@@ -157,7 +198,7 @@ __global__ void __launch_bounds__(kThreads) pbs_scores_bf16_kernel(
                 for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
                     for (int e = 0; e < 2; ++e)
-                        cs[sub * 8 + nt][e] += fast_exp2(z[nt][e] - la) + fast_exp2(z[nt][2 + e] - lb);
+                        cs[sub * 8 + nt][e] = fast_exp2(z[nt][e] - la) + fast_exp2(z[nt][2 + e] - lb);
             } else {
                 float ta_ = 0.f, tb_ = 0.f;
                 if (mxa != -INFINITY) {
@@ -172,56 +213,59 @@ __global__ void __launch_bounds__(kThreads) pbs_scores_bf16_kernel(
                 merge_ms(mb, sb, mxb, tb_);
             }
         }
-        if constexpr (!IMP) {
-            // the four lanes of a row hold disjoint columns: merge them
+        if constexpr (IMP) {
+            // column sums over the warp's rows (lanes of equal tig), then over the warps
 #pragma unroll
-            for (int o = 1; o < 4; o <<= 1) {
-                const float m2a = __shfl_xor_sync(0xffffffffu, ma, o), s2a = __shfl_xor_sync(0xffffffffu, sa, o);
-                const float m2b = __shfl_xor_sync(0xffffffffu, mb, o), s2b = __shfl_xor_sync(0xffffffffu, sb, o);
-                merge_ms(ma, sa, m2a, s2a);
-                merge_ms(mb, sb, m2b, s2b);
-            }
-            if (tig == 0) {
-                float2 *pp = reinterpret_cast<float2 *>(part) + (size_t)blockIdx.x * R;
-                if (va) pp[xa] = make_float2(ma, sa);
-                if (vb) pp[xb] = make_float2(mb, sb);
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    float v = cs[nt][e];
+                    v += __shfl_xor_sync(0xffffffffu, v, 4);
+                    v += __shfl_xor_sync(0xffffffffu, v, 8);
+                    v += __shfl_xor_sync(0xffffffffu, v, 16);
+                    if (gid == 0) colsum[warp][nt * 8 + 2 * tig + e] = v;
+                }
+            __syncthreads();
+            float *imp = lay.imp(wsg) + (size_t)blockIdx.y * L;
+            for (int x = tid; x < kChunkKeys && u0 + x < u_end; x += kThreads) {
+                float v = 0.f;
+#pragma unroll
+                for (int w = 0; w < kWarps; ++w) v += colsum[w][x];
+                imp[u0 + x] = v;
             }
         }
+        __syncthreads();   // the buffer and colsum are reused two chunks on
     }
-    if constexpr (IMP) {
-        // column sums over the warp's rows (lanes of equal tig), then over the warps
+    if constexpr (!IMP) {
+        // the four lanes of a row hold disjoint columns: merge them
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                float v = cs[nt][e];
-                v += __shfl_xor_sync(0xffffffffu, v, 4);
-                v += __shfl_xor_sync(0xffffffffu, v, 8);
-                v += __shfl_xor_sync(0xffffffffu, v, 16);
-                if (gid == 0) colsum[warp][nt * 8 + 2 * tig + e] = v;
-            }
-        __syncthreads();
-        for (int x = tid; x < nk; x += kThreads) {
-            float v = 0.f;
-#pragma unroll
-            for (int w = 0; w < kWarps; ++w) v += colsum[w][x];
-            perm[(size_t)bg * L + u0 + x] = __float_as_int(v / (float)R);
+        for (int o = 1; o < 4; o <<= 1) {
+            const float m2a = __shfl_xor_sync(0xffffffffu, ma, o), s2a = __shfl_xor_sync(0xffffffffu, sa, o);
+            const float m2b = __shfl_xor_sync(0xffffffffu, mb, o), s2b = __shfl_xor_sync(0xffffffffu, sb, o);
+            merge_ms(ma, sa, m2a, s2a);
+            merge_ms(mb, sb, m2b, s2b);
+        }
+        if (tig == 0) {
+            float2 *pp = lay.part(wsg) + (size_t)blockIdx.x * R;
+            if (va) pp[xa] = make_float2(ma, sa);
+            if (vb) pp[xb] = make_float2(mb, sb);
         }
     }
 }
 
 // fp32 inputs: the same two passes with plain dot products (thread per row for the
-// partials, thread per key for the importances).
+// partials, thread per key for the sums over the row block).
 template <int D, bool IMP>
 __global__ void __launch_bounds__(kThreads) pbs_scores_f32_kernel(
     const float *__restrict__ q, const float *__restrict__ k, int Hq, int Hkv, int L, int block,
-    float scale_log2, int nchunks, float *__restrict__ ws, int32_t *__restrict__ perm) {
+    float scale_log2, float *__restrict__ ws) {
     const int tid = threadIdx.x;
-    const int bg = blockIdx.y, b = bg / Hkv, g = bg % Hkv, G = Hq / Hkv;
+    const int bg = blockIdx.z, b = bg / Hkv, g = bg % Hkv, G = Hq / Hkv;
     const int nr = last_block_rows(L, block), r0 = L - nr, R = G * nr;
-    const int u0 = blockIdx.x * kChunk, nk = min(kChunk, L - u0);
-    float *part = ws + (size_t)bg * ws_floats_per_group(R, nchunks);
-    const float *lse2 = part + (size_t)nchunks * R * 2;
+    const PbsLayout lay(R, L);
+    float *wsg = ws + (size_t)bg * lay.floats(L);
+    const int u_begin = blockIdx.x * kKeyRange, u_end = min(L, u_begin + kKeyRange);
+    const int x0 = blockIdx.y * kRowBlock, x1 = min(R, x0 + kRowBlock);
     auto logit = [&](int x, int u) {
         const float *qr = q + (((size_t)b * Hq + g * G + x / nr) * L + r0 + x % nr) * D;
         const float *kr = k + ((size_t)bg * L + u) * D;
@@ -231,31 +275,33 @@ __global__ void __launch_bounds__(kThreads) pbs_scores_f32_kernel(
         return s * scale_log2;
     };
     if constexpr (!IMP) {
-        for (int x = tid; x < R; x += kThreads) {
+        for (int x = x0 + tid; x < x1; x += kThreads) {
             const int t = r0 + x % nr;
             float m = -INFINITY, s = 0.f;
-            for (int u = u0; u < u0 + nk && u <= t; ++u) merge_ms(m, s, logit(x, u), 1.f);
-            reinterpret_cast<float2 *>(part)[(size_t)blockIdx.x * R + x] = make_float2(m, s);
+            for (int u = u_begin; u < u_end && u <= t; ++u) merge_ms(m, s, logit(x, u), 1.f);
+            lay.part(wsg)[(size_t)blockIdx.x * R + x] = make_float2(m, s);
         }
     } else {
-        for (int y = tid; y < nk; y += kThreads) {
-            const int u = u0 + y;
+        const float *l2 = lay.lse2(wsg);
+        float *imp = lay.imp(wsg) + (size_t)blockIdx.y * L;
+        for (int u = u_begin + tid; u < u_end; u += kThreads) {
             float v = 0.f;
-            for (int x = 0; x < R; ++x)
-                if (u <= r0 + x % nr) v += fast_exp2(logit(x, u) - lse2[x]);
-            perm[(size_t)bg * L + u] = __float_as_int(v / (float)R);
+            for (int x = x0; x < x1; ++x)
+                if (u <= r0 + x % nr) v += fast_exp2(logit(x, u) - l2[x]);
+            imp[u] = v;
         }
     }
 }
 
-// lse2 of every row: the chunks' partials merged in chunk order.
-__global__ void __launch_bounds__(kThreads) pbs_lse_kernel(int R, int nchunks, float *__restrict__ ws) {
-    float *part = ws + (size_t)blockIdx.x * ws_floats_per_group(R, nchunks);
-    float *lse2 = part + (size_t)nchunks * R * 2;
-    const float2 *pp = reinterpret_cast<const float2 *>(part);
+// lse2 of every row: the key ranges' partials merged in range order.
+__global__ void __launch_bounds__(kThreads) pbs_lse_kernel(int L, int R, float *__restrict__ ws) {
+    const PbsLayout lay(R, L);
+    float *wsg = ws + (size_t)blockIdx.x * lay.floats(L);
+    const float2 *pp = lay.part(wsg);
+    float *lse2 = lay.lse2(wsg);
     for (int x = threadIdx.x; x < R; x += kThreads) {
         float m = -INFINITY, s = 0.f;
-        for (int c = 0; c < nchunks; ++c) {
+        for (int c = 0; c < lay.nkr; ++c) {
             const float2 v = pp[(size_t)c * R + x];
             merge_ms(m, s, v.x, v.y);
         }
@@ -265,15 +311,22 @@ __global__ void __launch_bounds__(kThreads) pbs_lse_kernel(int R, int nchunks, f
 
 // One CTA per (segment, b * Hkv + g): the segment's importances (fp32 bits in
 // perm) sorted descending, equal values by ascending index; perm overwritten.
-__global__ void __launch_bounds__(kThreads) pbs_sort_kernel(int L, int seg_len, int sort_cap,
+__global__ void __launch_bounds__(kThreads) pbs_sort_kernel(int L, int R, int seg_len, int sort_cap,
+                                                            const float *__restrict__ ws,
                                                             int32_t *__restrict__ perm) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     uint64_t *keys = reinterpret_cast<uint64_t *>(smem_raw);     // [sort_cap]
     const int tid = threadIdx.x, lane = tid & 31;
     const int bg = blockIdx.y;
     const int s0 = blockIdx.x * seg_len, n = min(seg_len, L - s0);
-    for (int x = tid; x < n; x += kThreads)
-        keys[x] = ((uint64_t)order_desc(__int_as_float(perm[(size_t)bg * L + s0 + x])) << 32) | (uint32_t)x;
+    const PbsLayout lay(R, L);
+    const float *imp = lay.imp(const_cast<float *>(ws) + (size_t)bg * lay.floats(L));
+    const float inv_r = 1.0f / (float)R;
+    for (int x = tid; x < n; x += kThreads) {
+        float v = 0.f;   // the row blocks' sums, in order, over R rows
+        for (int rb = 0; rb < lay.nrb; ++rb) v += imp[(size_t)rb * L + s0 + x];
+        keys[x] = ((uint64_t)order_desc(v * inv_r) << 32) | (uint32_t)x;
+    }
     if (sort_cap <= kRegSort) {
         // up to 2048 keys: 8 per thread in registers, position x = 8 tid + e; strides
         // below 8 in registers, 8..128 by shuffles, 256 and up through shared memory
@@ -380,24 +433,31 @@ cudaError_t launch_perm_d(const void *q, const void *k, bool bf16, int B, int Hq
                           int block, int seg_blocks, float scale, void *ws, int32_t *perm,
                           cudaStream_t s) {
     const int R = (Hq / Hkv) * last_block_rows(L, block);
-    const int nchunks = (L + kChunk - 1) / kChunk;
+    const PbsLayout lay(R, L);
     const float sl2 = scale * 1.4426950408889634f;
     float *w = static_cast<float *>(ws);
-    const dim3 grid_c((unsigned)nchunks, (unsigned)(B * Hkv));
+    const dim3 grid_c((unsigned)lay.nkr, (unsigned)lay.nrb, (unsigned)(B * Hkv));
+    cudaError_t e;
     if (bf16) {
         const auto *qq = static_cast<const __nv_bfloat16 *>(q);
         const auto *kk = static_cast<const __nv_bfloat16 *>(k);
-        pbs_scores_bf16_kernel<D, false><<<grid_c, kThreads, 0, s>>>(qq, kk, Hq, Hkv, L, block, sl2, nchunks, w, perm);
-        pbs_lse_kernel<<<B * Hkv, kThreads, 0, s>>>(R, nchunks, w);
-        pbs_scores_bf16_kernel<D, true><<<grid_c, kThreads, 0, s>>>(qq, kk, Hq, Hkv, L, block, sl2, nchunks, w, perm);
+        const size_t smem = (size_t)2 * kChunkKeys * (D / 2 + 4) * 4;
+        auto k0 = pbs_scores_bf16_kernel<D, false>;
+        auto k1 = pbs_scores_bf16_kernel<D, true>;
+        if ((e = cudaFuncSetAttribute(k0, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess ||
+            (e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+            return e;
+        k0<<<grid_c, kThreads, smem, s>>>(qq, kk, Hq, Hkv, L, block, sl2, w);
+        pbs_lse_kernel<<<B * Hkv, kThreads, 0, s>>>(L, R, w);
+        k1<<<grid_c, kThreads, smem, s>>>(qq, kk, Hq, Hkv, L, block, sl2, w);
     } else {
         const auto *qq = static_cast<const float *>(q);
         const auto *kk = static_cast<const float *>(k);
-        pbs_scores_f32_kernel<D, false><<<grid_c, kThreads, 0, s>>>(qq, kk, Hq, Hkv, L, block, sl2, nchunks, w, perm);
-        pbs_lse_kernel<<<B * Hkv, kThreads, 0, s>>>(R, nchunks, w);
-        pbs_scores_f32_kernel<D, true><<<grid_c, kThreads, 0, s>>>(qq, kk, Hq, Hkv, L, block, sl2, nchunks, w, perm);
+        pbs_scores_f32_kernel<D, false><<<grid_c, kThreads, 0, s>>>(qq, kk, Hq, Hkv, L, block, sl2, w);
+        pbs_lse_kernel<<<B * Hkv, kThreads, 0, s>>>(L, R, w);
+        pbs_scores_f32_kernel<D, true><<<grid_c, kThreads, 0, s>>>(qq, kk, Hq, Hkv, L, block, sl2, w);
     }
-    cudaError_t e = cudaGetLastError();
+    e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const int seg_len = seg_blocks * block;
     int cap = 1;
@@ -409,7 +469,7 @@ cudaError_t launch_perm_d(const void *q, const void *k, bool bf16, int B, int Hq
         if (e != cudaSuccess) return e;
     }
     dim3 grid((unsigned)((L + seg_len - 1) / seg_len), (unsigned)(B * Hkv));
-    pbs_sort_kernel<<<grid, kThreads, smem, s>>>(L, seg_len, cap, perm);
+    pbs_sort_kernel<<<grid, kThreads, smem, s>>>(L, R, seg_len, cap, w, perm);
     return cudaGetLastError();
 }
 
@@ -417,8 +477,7 @@ cudaError_t launch_perm_d(const void *q, const void *k, bool bf16, int B, int Hq
 
 size_t pbs_workspace_bytes(int B, int Hq, int Hkv, int L, int block) {
     const int R = (Hq / Hkv) * last_block_rows(L, block);
-    const int nchunks = (L + kChunk - 1) / kChunk;
-    return (size_t)B * Hkv * ws_floats_per_group(R, nchunks) * sizeof(float);
+    return (size_t)B * Hkv * PbsLayout(R, L).floats(L) * sizeof(float);
 }
 
 cudaError_t launch_pbs_permutation(const void *q, const void *k, bool bf16, int B, int Hq, int Hkv,

@@ -242,15 +242,16 @@ spa_status spa_sparse_attn_prefill_early_stop(const void *q, const void *k, cons
  * importances keep the smaller index first.
  *
  * spa_pbs_workspace_bytes: the device workspace spa_pbs_permutation needs (per
- *   (b, kv-head): a (max, sum) pair per row and key chunk of 128, and a
- *   log-sum-exp per row); 0 for invalid sizes.
+ *   (b, kv-head): a (max, sum) pair per row and range of 1024 keys, a log-sum-exp
+ *   per row, and per block of 128 rows one partial importance per key); 0 for
+ *   invalid sizes.
  * spa_pbs_permutation: perm [B, Hkv, L] int32 output, perm[b,g,p] = the original
  *   index of the key at permuted position p. q [B, Hq, L, d], k [B, Hkv, L, d],
  *   dt, d = 64 or 128; scale > 0 (the attention's softmax scale); a segment holds
  *   at most 8192 tokens. workspace: caller-owned device memory of at least
  *   spa_pbs_workspace_bytes (16-byte aligned; contents on entry do not matter).
- *   perm also holds the importances between the call's passes. Four launches on
- *   the stream (row partials, log-sum-exp, importances, segment sort).
+ *   Four launches on the stream (row partials, log-sum-exp, importances, segment
+ *   sort).
  * spa_pbs_gather: xp[b,g,p,:] = x[b,g,perm[b,g,p],:], for K and for V (rows of
  *   d elements of dt; the copies the two calls below read).
  * spa_select_segperm: spa_select for prefill on this layout: query block i scores
