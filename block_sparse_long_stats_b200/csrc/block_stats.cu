@@ -215,85 +215,94 @@ block_stats_kernel(const T *__restrict__ k, int T_len, int nb, int blk_begin, in
     }
 }
 
-// Blocks of 64 or more keys: one CTA per block, every load of the block issued at
-// once. Thread t owns 16-byte column chunk t % CPR of rows t / CPR, t / CPR + RG, ...
-// (RG = 256 / CPR row groups), so a block's bytes are all in flight before any is
-// reduced; the column sums meet in shared memory (mean), then the squared
-// deviations from the registers (variance). Several CTAs per SM keep enough bytes in
-// flight to cover the DRAM latency on short launches (the 32K workload's 66 MB).
+// Blocks of 64 or more keys: one warp per block, no shared memory and no barriers.
+// Lane (rp, c) owns 16-byte column chunk c of rows rp, rp + RPL, ... (a warp load
+// covers RPL whole rows). Pass 1 streams the block from HBM, 16 loads in flight per
+// lane, and sums the columns; the sums meet over the rp lanes with xor shuffles (the
+// mean). Pass 2 reads the block again, from L2 where pass 1 left it, and sums the
+// squared deviations the same way (the population variance). At about 100
+// registers a thread an SM keeps 16 or more blocks' warps resident: on the 32K
+// prefill workload (2048 blocks) every block is requested at once.
+constexpr int kWarpBlockThreads = 128;
+
 template <typename T, int D, int BLOCK>
-__global__ void __launch_bounds__(kThreads) block_stats_cta_kernel(const T *__restrict__ k, int T_len,
-                                                                   int nb, int blk_begin, int nblk,
-                                                                   float *__restrict__ mean,
-                                                                   float *__restrict__ var) {
-    constexpr int V = Elem<T>::kPerChunk;           // values per 16-byte chunk
-    constexpr int CPR = D / V;                      // chunks per row
-    constexpr int RG = kThreads / CPR;              // row groups
-    constexpr int RPT = BLOCK / RG;                 // rows per thread
-    static_assert(RPT * RG == BLOCK && RPT >= 1, "unsupported shape");
-    __shared__ float part[RG][D + 1];
-    __shared__ float colv[D];
-    const int u = blockIdx.x;
-    const int bg = u / nblk, j = blk_begin + u % nblk;
-    const int t0 = j * BLOCK, n = min(BLOCK, T_len - t0);
-    const int c = threadIdx.x % CPR, rg = threadIdx.x / CPR;
-    const uint4 *src = reinterpret_cast<const uint4 *>(k + ((size_t)bg * T_len + t0) * D) + c;
-    uint4 raw[RPT];
-#pragma unroll
-    for (int i = 0; i < RPT; ++i) {
-        const int r = rg + i * RG;
-        raw[i] = r < n ? __ldg(src + (size_t)r * CPR) : make_uint4(0, 0, 0, 0);
-    }
+__global__ void __launch_bounds__(kWarpBlockThreads) block_stats_warp_kernel(
+    const T *__restrict__ k, int T_len, int nb, int blk_begin, int nblk, int units,
+    float *__restrict__ mean, float *__restrict__ var) {
+    constexpr int V = Elem<T>::kPerChunk;     // values per 16-byte chunk
+    constexpr int LPR = D / V;                // lanes per row
+    constexpr int RPL = 32 / LPR;             // rows per warp load
+    constexpr int RPT = BLOCK / RPL;          // loads per lane
+    constexpr int NB = RPT < 16 ? RPT : 16;   // loads in flight per lane
+    static_assert(LPR >= 4 && LPR <= 32 && RPT % NB == 0, "unsupported shape");
+    const int u = (int)blockIdx.x * (kWarpBlockThreads / 32) + (int)(threadIdx.x >> 5);
+    if (u >= units) return;                   // whole warps leave
+    const int lane = threadIdx.x & 31, rp = lane / LPR, c = lane % LPR;
+    const int j = blk_begin + u % nblk;
+    const int n = min(BLOCK, T_len - j * BLOCK);
+    const uint4 *src = reinterpret_cast<const uint4 *>(
+                           k + ((size_t)(u / nblk) * T_len + (size_t)j * BLOCK) * D) +
+                       (size_t)rp * LPR + c;
     float s[V];
 #pragma unroll
     for (int v = 0; v < V; ++v) s[v] = 0.f;
+#pragma unroll 1
+    for (int b0 = 0; b0 < RPT; b0 += NB) {
+        uint4 raw[NB];
 #pragma unroll
-    for (int i = 0; i < RPT; ++i) {          // rows past the end were loaded as zeros
-        float x[V];
-        Elem<T>::unpack(raw[i], x);
+        for (int i = 0; i < NB; ++i)
+            raw[i] = rp + (b0 + i) * RPL < n ? __ldg(src + (size_t)(b0 + i) * RPL * LPR)
+                                             : make_uint4(0, 0, 0, 0);
 #pragma unroll
-        for (int v = 0; v < V; ++v) s[v] += x[v];
-    }
-#pragma unroll
-    for (int v = 0; v < V; ++v) part[rg][c * V + v] = s[v];
-    __syncthreads();
-    const float inv = 1.0f / (float)n;
-    for (int col = threadIdx.x; col < D; col += kThreads) {
-        float a = 0.f;
-#pragma unroll
-        for (int g = 0; g < RG; ++g) a += part[g][col];
-        colv[col] = a * inv;
-    }
-    __syncthreads();
-    float mu[V];
-#pragma unroll
-    for (int v = 0; v < V; ++v) {
-        mu[v] = colv[c * V + v];
-        s[v] = 0.f;
-    }
-#pragma unroll
-    for (int i = 0; i < RPT; ++i) {
-        if (rg + i * RG < n) {
+        for (int i = 0; i < NB; ++i) {        // rows past the end were loaded as zeros
             float x[V];
             Elem<T>::unpack(raw[i], x);
 #pragma unroll
-            for (int v = 0; v < V; ++v) {
-                const float dv = x[v] - mu[v];
-                s[v] = fmaf(dv, dv, s[v]);
+            for (int v = 0; v < V; ++v) s[v] += x[v];
+        }
+    }
+#pragma unroll
+    for (int o = LPR; o < 32; o <<= 1)
+#pragma unroll
+        for (int v = 0; v < V; ++v) s[v] += __shfl_xor_sync(0xffffffffu, s[v], o);
+    const float inv = 1.0f / (float)n;
+    float mu[V], m2[V];
+#pragma unroll
+    for (int v = 0; v < V; ++v) {
+        mu[v] = s[v] * inv;
+        m2[v] = 0.f;
+    }
+#pragma unroll 1
+    for (int b0 = 0; b0 < RPT; b0 += NB) {
+        uint4 raw[NB];
+#pragma unroll
+        for (int i = 0; i < NB; ++i)
+            if (rp + (b0 + i) * RPL < n) raw[i] = __ldg(src + (size_t)(b0 + i) * RPL * LPR);
+#pragma unroll
+        for (int i = 0; i < NB; ++i) {
+            if (rp + (b0 + i) * RPL < n) {
+                float x[V];
+                Elem<T>::unpack(raw[i], x);
+#pragma unroll
+                for (int v = 0; v < V; ++v) {
+                    const float dv = x[v] - mu[v];
+                    m2[v] = fmaf(dv, dv, m2[v]);
+                }
             }
         }
     }
-    __syncthreads();                         // every thread has read colv and part
 #pragma unroll
-    for (int v = 0; v < V; ++v) part[rg][c * V + v] = s[v];
-    __syncthreads();
-    const size_t o = ((size_t)bg * nb + j) * D;
-    for (int col = threadIdx.x; col < D; col += kThreads) {
-        float a = 0.f;
+    for (int o = LPR; o < 32; o <<= 1)
 #pragma unroll
-        for (int g = 0; g < RG; ++g) a += part[g][col];
-        mean[o + col] = colv[col];
-        var[o + col] = a * inv;
+        for (int v = 0; v < V; ++v) m2[v] += __shfl_xor_sync(0xffffffffu, m2[v], o);
+    if (rp == 0) {
+        const size_t o = ((size_t)(u / nblk) * nb + j) * D + (size_t)c * V;
+#pragma unroll
+        for (int v = 0; v < V; v += 4) {
+            *reinterpret_cast<float4 *>(mean + o + v) = make_float4(mu[v], mu[v + 1], mu[v + 2], mu[v + 3]);
+            *reinterpret_cast<float4 *>(var + o + v) =
+                make_float4(m2[v] * inv, m2[v + 1] * inv, m2[v + 2] * inv, m2[v + 3] * inv);
+        }
     }
 }
 
@@ -302,14 +311,15 @@ cudaError_t launch_t(const void *k, int B, int Hkv, int T_len, int blk_begin, in
                      float *mean, float *var, cudaStream_t s) {
     const int nb = (T_len + BLOCK - 1) / BLOCK, nblk = blk_end - blk_begin;
     const int units = B * Hkv * nblk;
+    if constexpr (BLOCK >= 64) {
+        constexpr int wpc = kWarpBlockThreads / 32;
+        block_stats_warp_kernel<T, D, BLOCK><<<(unsigned)((units + wpc - 1) / wpc), kWarpBlockThreads, 0, s>>>(
+            reinterpret_cast<const T *>(k), T_len, nb, blk_begin, nblk, units, mean, var);
+        return cudaGetLastError();
+    }
     using S = StatsShape<T, D, BLOCK>;
     constexpr int SPW = S::NC > kThreads / 32 ? S::NC / (kThreads / 32) : 1;
     constexpr int BPT = (kThreads / 32) / (S::NC / SPW);   // blocks per tile
-    if constexpr (BLOCK >= 64) {
-        block_stats_cta_kernel<T, D, BLOCK><<<units, kThreads, 0, s>>>(
-            reinterpret_cast<const T *>(k), T_len, nb, blk_begin, nblk, mean, var);
-        return cudaGetLastError();
-    }
     const int tiles = (units + BPT - 1) / BPT;
     const unsigned grid = (unsigned)std::min(tiles, 148 * kCtasPerSm);
     block_stats_kernel<T, D, BLOCK><<<grid, kThreads, 0, s>>>(

@@ -75,6 +75,8 @@ __device__ V block_exclusive_scan(V x, V *warp_tot, V *total) {
 // query (qv, its squares q2) and of the block's mean and variance: per-lane fused
 // multiply-adds, then the xor-shuffle tree of reduce_transpose across the warp.
 // Prefill and decode scoring use this exact order, so their scores agree to the bit.
+// (Pairs of features in fma.rn.f32x2 need register pairs that the scoring loop,
+// at 80 registers, only finds by spilling.)
 template <int PL>
 __device__ __forceinline__ void lane_partials(const float (&qv)[PL], const float (&q2)[PL],
                                               const float (&mu)[PL], const float (&vr)[PL],
@@ -169,41 +171,52 @@ __device__ __forceinline__ float reduce_transpose(float (&v)[K], int lane) {
     return t;
 }
 
-// Sorts N = 32 KPL 64-bit keys ascending inside one warp, lane-major (lane l holds
-// positions KPL l .. KPL l + KPL - 1): a bitonic network whose strides below KPL
-// are compare-exchanges in registers and whose larger strides are xor shuffles.
-// No shared memory and no barriers.
+// One stage (block size kk, stride jj) of a bitonic network over N = 32 KPL 64-bit
+// keys held lane-major in one warp (lane l holds positions KPL l .. KPL l + KPL - 1):
+// strides below KPL are compare-exchanges in registers, larger ones xor shuffles.
+template <int KPL>
+__device__ __forceinline__ void warp_bitonic_stage(uint64_t (&k)[KPL], int lane, int kk, int jj) {
+    if (jj < KPL) {
+#pragma unroll
+        for (int e = 0; e < KPL; ++e) {
+            if ((e & jj) == 0) {
+                const bool up = ((lane * KPL + e) & kk) == 0;
+                const uint64_t x = k[e], y = k[e | jj];
+                const bool sw = (x > y) == up;
+                k[e] = sw ? y : x;
+                k[e | jj] = sw ? x : y;
+            }
+        }
+    } else {
+        const int lm = jj / KPL;                  // partner lane = lane ^ lm
+        const bool lower = (lane & lm) == 0;
+#pragma unroll
+        for (int e = 0; e < KPL; ++e) {
+            const bool up = ((lane * KPL + e) & kk) == 0;
+            const uint64_t o = __shfl_xor_sync(0xffffffffu, k[e], lm);
+            const uint64_t mn = k[e] < o ? k[e] : o, mx = k[e] < o ? o : k[e];
+            k[e] = lower == up ? mn : mx;
+        }
+    }
+}
+
+// Sorts the warp's N = 32 KPL keys ascending (a full bitonic network). No shared
+// memory and no barriers.
 template <int KPL>
 __device__ __forceinline__ void warp_bitonic_sort(uint64_t (&k)[KPL], int lane) {
     constexpr int N = 32 * KPL;
 #pragma unroll
-    for (int kk = 2; kk <= N; kk <<= 1) {
+    for (int kk = 2; kk <= N; kk <<= 1)
 #pragma unroll
-        for (int jj = kk >> 1; jj > 0; jj >>= 1) {
-            if (jj < KPL) {
+        for (int jj = kk >> 1; jj > 0; jj >>= 1) warp_bitonic_stage<KPL>(k, lane, kk, jj);
+}
+
+// Sorts a bitonic sequence of the warp's N keys ascending (the last merge phase).
+template <int KPL>
+__device__ __forceinline__ void warp_bitonic_merge(uint64_t (&k)[KPL], int lane) {
+    constexpr int N = 32 * KPL;
 #pragma unroll
-                for (int e = 0; e < KPL; ++e) {
-                    if ((e & jj) == 0) {
-                        const bool up = ((lane * KPL + e) & kk) == 0;
-                        const uint64_t x = k[e], y = k[e | jj];
-                        const bool sw = (x > y) == up;
-                        k[e] = sw ? y : x;
-                        k[e | jj] = sw ? x : y;
-                    }
-                }
-            } else {
-                const int lm = jj / KPL;                  // partner lane = lane ^ lm
-                const bool lower = (lane & lm) == 0;
-#pragma unroll
-                for (int e = 0; e < KPL; ++e) {
-                    const bool up = ((lane * KPL + e) & kk) == 0;
-                    const uint64_t o = __shfl_xor_sync(0xffffffffu, k[e], lm);
-                    const uint64_t mn = k[e] < o ? k[e] : o, mx = k[e] < o ? o : k[e];
-                    k[e] = lower == up ? mn : mx;
-                }
-            }
-        }
-    }
+    for (int jj = N >> 1; jj > 0; jj >>= 1) warp_bitonic_stage<KPL>(k, lane, 2 * N, jj);
 }
 
 struct SelectArgs {
@@ -264,11 +277,11 @@ __device__ __forceinline__ void warp_sort_cut(const uint64_t *keys, unsigned cha
         const double total = __shfl_sync(0xffffffffu, inc, 31);
         const double prev = __shfl_up_sync(0xffffffffu, inc, 1);
         double cum = lane == 0 ? 0.0 : prev;
-        const double p = (double)a.top_p;
+        const double thr = (double)a.top_p * total;   // cum / total < top_p
         int kept = 0;
 #pragma unroll
         for (int e = 0; e < KPL; ++e) {
-            if (lane * KPL + e < nres && cum / total < p) ++kept;
+            if (lane * KPL + e < nres && cum < thr) ++kept;
             cum += m[e];
         }
         nk = (int)__reduce_add_sync(0xffffffffu, (unsigned)kept);
@@ -289,6 +302,93 @@ __device__ __forceinline__ void warp_sort_cut(const uint64_t *keys, unsigned cha
 #pragma unroll
         for (int e = 0; e < KPL; ++e)
             if (lane * KPL + e < nk) flag[(int)(uint32_t)k[e]] = 1;
+    }
+}
+
+constexpr int kPairSortMax = 256;   // residuals up to this many: a pair of warps
+
+// 129 to 256 residual keys of one head (keys[0, nres) in shared memory) sorted by
+// a pair of warps, half = 0 and 1, each holding 128 positions (4 keys per lane):
+// each warp sorts its half ascending in registers and stores it back; after one
+// pair barrier, position x of the lower half meets position 127 - x of the upper
+// (the minima are the 128 smallest keys, the maxima the rest, each sequence
+// bitonic), and each warp merges its half in registers. The cut is the same as
+// warp_sort_cut's, with the upper warp's prefix starting at the lower warp's total
+// (both warps add the two totals in the same order). bar_id names the pair's
+// 64-thread barrier; xd, xi are two doubles and two ints of shared memory.
+__device__ __forceinline__ void pair_sort_cut(uint64_t *keys, double *xd, int *xi,
+                                              unsigned char *flag, const SelectArgs &a,
+                                              size_t unit, int nres, int r_lo, int r_hi, int jmax,
+                                              int half, int bar_id, int lane) {
+    constexpr int KPL = 4, NH = 32 * KPL;
+    const int base = half * NH;
+    uint64_t k[KPL];
+#pragma unroll
+    for (int e = 0; e < KPL; ++e) {
+        const int x = base + lane * KPL + e;
+        k[e] = x < nres ? keys[x] : ~0ull;
+    }
+    warp_bitonic_sort<KPL>(k, lane);
+#pragma unroll
+    for (int e = 0; e < KPL; ++e) keys[base + lane * KPL + e] = k[e];
+    named_bar_sync(bar_id, 64);
+    const uint64_t first = keys[0] < keys[NH] ? keys[0] : keys[NH];   // the largest score
+#pragma unroll
+    for (int e = 0; e < KPL; ++e) {
+        const uint64_t o = keys[(NH - base) + NH - 1 - (lane * KPL + e)];
+        k[e] = half == 0 ? (k[e] < o ? k[e] : o) : (k[e] < o ? o : k[e]);
+    }
+    warp_bitonic_merge<KPL>(k, lane);
+    int nk = nres;
+    if (a.top_p < 1.0f) {
+        const double mx = (double)key_score(first);
+        double m[KPL], local = 0.0;
+#pragma unroll
+        for (int e = 0; e < KPL; ++e) {
+            m[e] = base + lane * KPL + e < nres ? exp((double)key_score(k[e]) - mx) : 0.0;
+            local += m[e];
+        }
+        double inc = local;            // inclusive scan over lanes
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const double y = __shfl_up_sync(0xffffffffu, inc, o);
+            if (lane >= o) inc += y;
+        }
+        if (lane == 31) xd[half] = inc;
+        named_bar_sync(bar_id, 64);
+        const double total = xd[0] + xd[1];
+        const double prev = __shfl_up_sync(0xffffffffu, inc, 1);
+        double cum = (half == 0 ? 0.0 : xd[0]) + (lane == 0 ? 0.0 : prev);
+        const double thr = (double)a.top_p * total;   // cum / total < top_p
+        int kept = 0;
+#pragma unroll
+        for (int e = 0; e < KPL; ++e) {
+            if (base + lane * KPL + e < nres && cum < thr) ++kept;
+            cum += m[e];
+        }
+        kept = (int)__reduce_add_sync(0xffffffffu, (unsigned)kept);
+        if (lane == 0) xi[half] = kept;
+        named_bar_sync(bar_id, 64);
+        nk = xi[0] + xi[1];
+    }
+    nk = max(nk, min(a.k_min, nres));
+    if (a.score_order) {
+        int32_t *out = a.idx + unit * a.cap;
+        const int nloc = jmax + 1 - r_hi;
+        if (half == 0) {
+            for (int x = lane; x < nloc; x += 32) out[x] = jmax - x;
+            for (int x = lane; x < r_lo; x += 32) out[nloc + x] = x;
+            if (lane == 0) a.count[unit] = nloc + r_lo + nk;
+        }
+#pragma unroll
+        for (int e = 0; e < KPL; ++e) {
+            const int x = base + lane * KPL + e;
+            if (x < nk) out[nloc + r_lo + x] = (int)(uint32_t)k[e];
+        }
+    } else {
+#pragma unroll
+        for (int e = 0; e < KPL; ++e)
+            if (base + lane * KPL + e < nk) flag[(int)(uint32_t)k[e]] = 1;
     }
 }
 
@@ -489,12 +589,11 @@ __global__ void __launch_bounds__(kThreads) select_kernel(SelectArgs a) {
         double local = 0.0;
         for (int x = s0; x < s1; ++x) local += exp((double)key_score(keys[x]) - mx);
         const double before = block_exclusive_scan<double>(local, dtot, &dsum);
-        const double total = dsum;
-        const double p = (double)a.top_p;
+        const double thr = (double)a.top_p * dsum;    // cum / total < top_p
         int kept_here = 0;
         double cum = before;
         for (int x = s0; x < s1; ++x) {
-            if (cum / total < p) ++kept_here;
+            if (cum < thr) ++kept_here;
             cum += exp((double)key_score(keys[x]) - mx);
         }
         block_exclusive_scan<int>(kept_here, itot, &isum);
@@ -597,12 +696,11 @@ __device__ void cta_sort_cut(const uint64_t *keys, uint64_t *xbuf, unsigned char
             local += m[e];
         }
         double cum = block_exclusive_scan<double>(local, dtot, dsum);
-        const double total = *dsum;
-        const double p = (double)a.top_p;
+        const double thr = (double)a.top_p * *dsum;   // cum / total < top_p
         int kept = 0;
 #pragma unroll
         for (int e = 0; e < KPL; ++e) {
-            if (tid * KPL + e < nres && cum / total < p) ++kept;
+            if (tid * KPL + e < nres && cum < thr) ++kept;
             cum += m[e];
         }
         block_exclusive_scan<int>(kept, itot, isum);
@@ -652,6 +750,8 @@ __global__ void __launch_bounds__(kThreads, 3) select_group_kernel(SelectArgs a)
     __shared__ int itot[kWarps];
     __shared__ int isum;
     __shared__ uint64_t first_key;
+    __shared__ double pair_d[G][2];
+    __shared__ int pair_i[G][2];
     // dynamic: keys [G][kcap], then (more than kWarpSortMax residuals) the sort's two
     // exchange buffers [2][kcap], then flags [G][nb]
     extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -793,19 +893,28 @@ __global__ void __launch_bounds__(kThreads, 3) select_group_kernel(SelectArgs a)
         return;
     }
 
-    // ---- warp h: sort, cut and list of head h
-    if (warp < G) {
-        const int h = g * G + warp;
+    // ---- warp h: sort, cut and list of head h (129 to 256 residuals with 2G <=
+    // kWarps: warps h and h + G together)
+    const bool pair = 2 * G <= kWarps && nres > kPairSortMax / 2;
+    if (warp < (pair ? 2 * G : G)) {
+        const int hw = warp % G, half = warp / G;
+        const int h = g * G + hw;
         const size_t unit = ((size_t)b * a.Hq + h) * a.nq + i;
-        unsigned char *fl = flags + (size_t)warp * a.nb;
-        const int N = nres <= 32 ? 32 : nres <= 64 ? 64 : nres <= 128 ? 128 : 256;
-        const uint64_t *kw = keys + (size_t)warp * kcap;
-        if (N == 32) warp_sort_cut<1>(kw, fl, a, unit, nres, r_lo, r_hi, jmax, lane);
-        else if (N == 64) warp_sort_cut<2>(kw, fl, a, unit, nres, r_lo, r_hi, jmax, lane);
-        else if (N == 128) warp_sort_cut<4>(kw, fl, a, unit, nres, r_lo, r_hi, jmax, lane);
-        else warp_sort_cut<8>(kw, fl, a, unit, nres, r_lo, r_hi, jmax, lane);
-        if (!a.score_order) {
+        unsigned char *fl = flags + (size_t)hw * a.nb;
+        uint64_t *kw = keys + (size_t)hw * kcap;
+        if (pair) {
+            pair_sort_cut(kw, pair_d[hw], pair_i[hw], fl, a, unit, nres, r_lo, r_hi, jmax, half,
+                          1 + hw, lane);
+            if (!a.score_order) named_bar_sync(1 + hw, 64);   // both halves' flags are set
+        } else {
+            const int N = nres <= 32 ? 32 : nres <= 64 ? 64 : nres <= 128 ? 128 : 256;
+            if (N == 32) warp_sort_cut<1>(kw, fl, a, unit, nres, r_lo, r_hi, jmax, lane);
+            else if (N == 64) warp_sort_cut<2>(kw, fl, a, unit, nres, r_lo, r_hi, jmax, lane);
+            else if (N == 128) warp_sort_cut<4>(kw, fl, a, unit, nres, r_lo, r_hi, jmax, lane);
+            else warp_sort_cut<8>(kw, fl, a, unit, nres, r_lo, r_hi, jmax, lane);
             __syncwarp();
+        }
+        if (!a.score_order && half == 0) {
             // ascending list: lane l takes flags [l per, (l + 1) per), warp scan of counts
             const int n = jmax + 1, per = (n + 31) / 32;
             const int s0 = min(lane * per, n), s1 = min(s0 + per, n);

@@ -398,10 +398,14 @@ def test_decode_workload_full_size():
     assert_no_device_error()
 
 
-@pytest.mark.parametrize("T,Hq,Hkv", [(6000, 8, 2), (12000, 8, 2), (12000, 8, 1)])
+@pytest.mark.parametrize("T,Hq,Hkv", [(3000, 4, 1), (3000, 4, 2), (3000, 2, 2), (4000, 8, 1),
+                                     (6000, 8, 2), (12000, 8, 2), (12000, 8, 1)])
 def test_select_many_candidates(T, Hq, Hkv):
-    # 375 and 750 blocks of 16: more residual candidates than one warp sorts, so
-    # the grouped kernel sorts each head across the CTA (2 and 4 keys per thread)
+    # 188 and 250 blocks of 16: 129 to 256 residual candidates are sorted by a pair
+    # of warps per head where the CTA has two warps per head (G = 1, 2, 4), by one
+    # warp otherwise (G = 8); 375 and 750 blocks: more candidates than a warp pair
+    # sorts, so the grouped kernel sorts each head across the CTA (2 and 4 keys per
+    # thread)
     w = PARITY_WORKLOADS["p_bf16_blk128"].with_(T=T, B=1, Hq=Hq, Hkv=Hkv, block=16)
     x, dev = inputs(w)
     mean, var = spa.spa_block_stats(dev["k"], w.block)
