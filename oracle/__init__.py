@@ -62,9 +62,12 @@ def _bind(path: str):
                                              _I, _P, _D, _P, _I64, _P, _P]
     lib.oracle_quantize_stats.argtypes = [_P, _P, _I, _I, _I, _I, _P, _P, _P, _P]
     lib.oracle_dequantize_stats.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _P, _P]
+    lib.oracle_quantize_stats_fp4.argtypes = [_P, _P, _I, _I, _I, _I, _P, _P, _P, _P]
+    lib.oracle_dequantize_stats_fp4.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _P, _P]
     for f in ("oracle_block_stats", "oracle_scores", "oracle_select_from_scores",
               "oracle_attention", "oracle_rla", "oracle_rla_block_states",
-              "oracle_quantize_stats", "oracle_dequantize_stats", "oracle_early_stop",
+              "oracle_quantize_stats", "oracle_dequantize_stats", "oracle_quantize_stats_fp4",
+              "oracle_dequantize_stats_fp4", "oracle_early_stop",
               "oracle_pbs_permutation", "oracle_attention_segperm"):
         getattr(lib, f).restype = _I
     return lib
@@ -238,42 +241,54 @@ def rla_block_states(k, v, dtype: str, block: int) -> np.ndarray:
     return out
 
 
-def quantize_stats(mean: np.ndarray, var: np.ndarray) -> dict:
-    """INT4 microscale block statistics (SpotAttention, section 4; the format is
-    documented at oracle_quantize_stats). Returns codes cm (int8), cv (uint8) shaped
-    like mean, and per-32-feature exponents km, kv (int8) [B, Hkv, nb, d / 32]."""
+def quantize_stats(mean: np.ndarray, var: np.ndarray, fmt: str = "int4") -> dict:
+    """Microscale block statistics (SpotAttention, section 4): INT4 (fmt "int4", the
+    format documented at oracle_quantize_stats) or FP4 E2M1 (fmt "fp4", documented at
+    oracle_quantize_stats_fp4). Returns codes cm, cv shaped like mean (INT4: int8 and
+    uint8 values; FP4: uint8 4-bit patterns), per-32-feature exponents km, kv (int8)
+    [B, Hkv, nb, d / 32], and the format."""
     mean = np.ascontiguousarray(mean, np.float64)
     var = np.ascontiguousarray(var, np.float64)
     B, Hkv, nb, d = mean.shape
-    cm = np.empty(mean.shape, np.int8)
-    cv = np.empty(mean.shape, np.uint8)
     km = np.empty((B, Hkv, nb, d // 32), np.int8)
     kv = np.empty_like(km)
-    _check(_load().oracle_quantize_stats(_ptr(mean), _ptr(var), B, Hkv, nb, d, _ptr(cm), _ptr(cv),
-                                         _ptr(km), _ptr(kv)), "quantize_stats")
-    return {"cm": cm, "cv": cv, "km": km, "kv": kv}
+    cv = np.empty(mean.shape, np.uint8)
+    if fmt == "int4":
+        cm = np.empty(mean.shape, np.int8)
+        fn = _load().oracle_quantize_stats
+    elif fmt == "fp4":
+        cm = np.empty(mean.shape, np.uint8)
+        fn = _load().oracle_quantize_stats_fp4
+    else:
+        raise ValueError(f"unknown format {fmt!r}")
+    _check(fn(_ptr(mean), _ptr(var), B, Hkv, nb, d, _ptr(cm), _ptr(cv), _ptr(km), _ptr(kv)),
+           "quantize_stats")
+    return {"cm": cm, "cv": cv, "km": km, "kv": kv, "fmt": fmt}
 
 
 def dequantize_stats(qs: dict):
-    """(mean, var) fp64 from quantize_stats' codes: code * 2^k."""
-    cm = np.ascontiguousarray(qs["cm"], np.int8)
+    """(mean, var) fp64 from quantize_stats' codes: code * 2^k (INT4) or
+    E2M1(code) * 2^k (FP4)."""
+    fmt = qs.get("fmt", "int4")
+    cm = np.ascontiguousarray(qs["cm"], np.int8 if fmt == "int4" else np.uint8)
     cv = np.ascontiguousarray(qs["cv"], np.uint8)
     km = np.ascontiguousarray(qs["km"], np.int8)
     kv = np.ascontiguousarray(qs["kv"], np.int8)
     B, Hkv, nb, d = cm.shape
     mean = np.empty(cm.shape, np.float64)
     var = np.empty(cm.shape, np.float64)
-    _check(_load().oracle_dequantize_stats(_ptr(cm), _ptr(cv), _ptr(km), _ptr(kv), B, Hkv, nb, d,
-                                           _ptr(mean), _ptr(var)), "dequantize_stats")
+    fn = _load().oracle_dequantize_stats if fmt == "int4" else _load().oracle_dequantize_stats_fp4
+    _check(fn(_ptr(cm), _ptr(cv), _ptr(km), _ptr(kv), B, Hkv, nb, d, _ptr(mean), _ptr(var)),
+           "dequantize_stats")
     return mean, var
 
 
 def select_quantized(q, k, dtype: str, block: int, scale: float, top_p: float, n_sink: int = 1,
-                     n_local: int = 1, k_min: int = 0):
-    """The selection of `select` on quantised statistics: stats -> quantize ->
+                     n_local: int = 1, k_min: int = 0, fmt: str = "int4"):
+    """The selection of `select` on quantised statistics: stats -> quantize (fmt) ->
     dequantize -> scores -> cut."""
     mean, var = block_stats(k, dtype, block)
-    qs = quantize_stats(mean, var)
+    qs = quantize_stats(mean, var, fmt)
     dm, dv = dequantize_stats(qs)
     Lq, T = q.shape[2], k.shape[2]
     l = scores(q, dtype, dm, dv, T, block, scale)

@@ -574,6 +574,77 @@ int oracle_dequantize_stats(const int8_t *cm, const uint8_t *cv, const int8_t *k
 }
 
 /*
+ * FP4 microscale block statistics: the passage's other format. Reading: the element
+ * is the OCP microscaling FP4 type E2M1 (a sign bit, two exponent bits with bias 1,
+ * one mantissa bit: magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6), with the INT4 records'
+ * power-of-two scale per 32 features:
+ *   k    = the smallest k with max |x| <= 6 * 2^k over the group (no element is
+ *          clipped), clamped to [-126, 126] (a group of zeros gets k = -126);
+ *   code = the E2M1 value nearest x / 2^k, a tie going to the value whose mantissa
+ *          bit is 0; the sign bit is x's (a negative x that rounds to 0 gives -0).
+ * A code is the 4-bit pattern s e1 e0 m (sign in bit 3), for the mean and the
+ * variance alike (the variance's sign bit is 0). Dequantised: E2M1(code) * 2^k,
+ * exact. As for INT4, the decision is taken on the statistics rounded to fp32.
+ * mean, var: fp64 [B, Hkv, nb, d]; cm, cv: codes [B, Hkv, nb, d] (uint8, 0..15);
+ * km, kv: exponents [B, Hkv, nb, d / 32] (int8). d must be a multiple of 32.
+ */
+static const double kE2M1[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+
+static uint8_t e2m1_code(double y)
+{
+    const double a = fabs(y);
+    int best = 0;
+    for (int i = 1; i < 8; ++i) {
+        const double di = fabs(a - kE2M1[i]), db = fabs(a - kE2M1[best]);
+        if (di < db || (di == db && (i & 1) == 0)) best = i;   /* index bit 0 = mantissa */
+    }
+    return (uint8_t)(best | (signbit(y) ? 8 : 0));
+}
+
+int oracle_quantize_stats_fp4(const double *mean, const double *var, int B, int Hkv, int nb,
+                              int d, uint8_t *cm, uint8_t *cv, int8_t *km, int8_t *kv)
+{
+    if (B <= 0 || Hkv <= 0 || nb <= 0 || d <= 0 || d % 32) return ORACLE_EINVAL;
+    const int64_t groups = (int64_t)B * Hkv * nb * (d / 32);
+#pragma omp parallel for schedule(static)
+    for (int64_t gi = 0; gi < groups; ++gi) {
+        const size_t base = (size_t)gi * 32;
+        double am = 0.0, av = 0.0;
+        double xm[32], xv[32];
+        for (int c = 0; c < 32; ++c) {
+            xm[c] = (double)(float)mean[base + c];     /* the fp32 statistic */
+            xv[c] = (double)(float)var[base + c];
+            if (fabs(xm[c]) > am) am = fabs(xm[c]);
+            if (xv[c] > av) av = xv[c];
+        }
+        const int k1 = qexp(am, 6.0), k2 = qexp(av, 6.0);
+        km[gi] = (int8_t)k1;
+        kv[gi] = (int8_t)k2;
+        for (int c = 0; c < 32; ++c) {
+            cm[base + c] = e2m1_code(ldexp(xm[c], -k1));
+            cv[base + c] = e2m1_code(ldexp(xv[c], -k2));
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* Dequantised FP4 statistics: E2M1(code) * 2^k, exact. Layouts as above. */
+int oracle_dequantize_stats_fp4(const uint8_t *cm, const uint8_t *cv, const int8_t *km,
+                                const int8_t *kv, int B, int Hkv, int nb, int d, double *mean,
+                                double *var)
+{
+    if (B <= 0 || Hkv <= 0 || nb <= 0 || d <= 0 || d % 32) return ORACLE_EINVAL;
+    const int64_t n = (int64_t)B * Hkv * nb * d;
+    for (int64_t x = 0; x < n; ++x) {
+        const double m = kE2M1[cm[x] & 7] * ((cm[x] & 8) ? -1.0 : 1.0);
+        const double v = kE2M1[cv[x] & 7] * ((cv[x] & 8) ? -1.0 : 1.0);
+        mean[x] = ldexp(m, km[x / 32]);
+        var[x] = ldexp(v, kv[x / 32]);
+    }
+    return ORACLE_OK;
+}
+
+/*
  * Score-ordered traversal with a monotone-gain early stop ("S2O", section 2 and
  * section 3's second pass). The lists are in traversal order (the local blocks and
  * the sink first, then the kept residual blocks by descending score). For query

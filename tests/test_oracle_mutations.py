@@ -70,6 +70,28 @@ MUTATIONS = [
       pins.test_quantized_stats_on_the_grid_round_trip_exactly]),
     ("quant_variance_signed_range", "qexp(av, 15.0)", "qexp(av, 7.0)",
      [pins.test_quantized_stats_hand_worked_group, pins.test_quantized_stats_error_and_scale_bounds]),
+    ("fp4_ties_away_from_zero", "if (di < db || (di == db && (i & 1) == 0)) best = i;",
+     "if (di <= db) best = i;",
+     [pins.test_fp4_stats_hand_worked_group, pins.test_fp4_codes_are_the_nearest_e2m1_values]),
+    ("fp4_ties_toward_zero", "if (di < db || (di == db && (i & 1) == 0)) best = i;",
+     "if (di < db) best = i;",
+     [pins.test_fp4_stats_hand_worked_group, pins.test_fp4_codes_are_the_nearest_e2m1_values]),
+    ("fp4_sign_dropped", "return (uint8_t)(best | (signbit(y) ? 8 : 0));", "return (uint8_t)best;",
+     [pins.test_fp4_stats_hand_worked_group, pins.test_fp4_error_and_scale_bounds,
+      pins.test_fp4_on_the_grid_round_trip_exactly]),
+    ("fp4_scale_clips_like_a_floor_exponent", "const int k1 = qexp(am, 6.0), k2 = qexp(av, 6.0);",
+     "const int k1 = qexp(am, 4.0), k2 = qexp(av, 6.0);",
+     [pins.test_fp4_stats_hand_worked_group, pins.test_fp4_error_and_scale_bounds,
+      pins.test_fp4_on_the_grid_round_trip_exactly]),
+    ("fp4_variance_with_the_mean_scale", "cv[base + c] = e2m1_code(ldexp(xv[c], -k2));",
+     "cv[base + c] = e2m1_code(ldexp(xv[c], -k1));",
+     [pins.test_fp4_stats_hand_worked_group, pins.test_fp4_error_and_scale_bounds]),
+    ("fp4_table_three_as_two_and_a_half", "{0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0}",
+     "{0.0, 0.5, 1.0, 1.5, 2.0, 2.5, 4.0, 6.0}",
+     [pins.test_fp4_codes_decode_to_the_e2m1_values, pins.test_fp4_codes_are_the_nearest_e2m1_values]),
+    ("fp4_dequantised_without_sign", "const double m = kE2M1[cm[x] & 7] * ((cm[x] & 8) ? -1.0 : 1.0);",
+     "const double m = kE2M1[cm[x] & 7];",
+     [pins.test_fp4_codes_decode_to_the_e2m1_values, pins.test_fp4_on_the_grid_round_trip_exactly]),
     ("early_stop_on_reserved_blocks", "if (!reserved && R < tau) {", "if (R < tau) {",
      [pins.test_early_stop_limits_of_tau]),
     ("early_stop_drops_the_stopping_block", "done = n + 1;", "done = n;",

@@ -746,6 +746,128 @@ def test_quantized_selection_equals_plain_selection_on_grid_statistics():
     assert np.array_equal(a["scores"], b["scores"])
 
 
+# FP4 records: the same section's other format, read as the OCP microscaling
+# element E2M1 with the records' power-of-two scale per 32 features.
+
+E2M1_TABLE = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]   # the E2M1 magnitudes, codes 0..7
+
+
+def test_fp4_stats_hand_worked_group():
+    g = _golden()["quantized_stats_fp4"]
+    mean = np.array(g["mean_group"], np.float64).reshape(1, 1, 1, 32)
+    var = np.array(g["var_group"], np.float64).reshape(1, 1, 1, 32)
+    qs = oracle.quantize_stats(mean, var, "fp4")
+    assert int(qs["km"][0, 0, 0, 0]) == g["expected_km"]
+    assert int(qs["kv"][0, 0, 0, 0]) == g["expected_kv"]
+    assert qs["cm"].reshape(-1).tolist() == g["expected_cm"]
+    assert qs["cv"].reshape(-1).tolist() == g["expected_cv"]
+
+
+def test_fp4_codes_decode_to_the_e2m1_values():
+    # code s e1 e0 m: (-1)^s 2^(e - 1) (1 + m / 2) for e > 0, (-1)^s m / 2 for e = 0
+    codes = np.tile(np.arange(16, dtype=np.uint8), 2).reshape(1, 1, 1, 32)
+    k = np.zeros((1, 1, 1, 1), np.int8)
+    dm, dv = oracle.dequantize_stats({"cm": codes, "cv": codes, "km": k, "kv": k + 3, "fmt": "fp4"})
+    want = [sgn * v for sgn in (1.0, -1.0) for v in E2M1_TABLE]
+    assert dm.reshape(-1)[:16].tolist() == want
+    assert dv.reshape(-1)[:16].tolist() == [8.0 * x for x in want]
+    assert np.signbit(dm.reshape(-1)[8])                      # code 8 is -0
+
+
+def _fp4_inputs(seed):
+    rng = np.random.default_rng(seed)
+    mean = rng.standard_normal((2, 2, 5, 64)) * np.exp(rng.uniform(-6, 6, (2, 2, 5, 2))).repeat(32, -1)
+    var = rng.exponential(1.0, (2, 2, 5, 64)) * 10.0 ** rng.integers(-3, 3, (2, 2, 5, 1))
+    mean[0, 0, 1, :32] = 0.0                   # an all-zero group
+    var[1, 1, 2, 32:] = 0.0
+    return mean, var
+
+
+def test_fp4_error_and_scale_bounds():
+    mean, var = _fp4_inputs(80)
+    qs = oracle.quantize_stats(mean, var, "fp4")
+    dm, dv = oracle.dequantize_stats(qs)
+    for x, d, k in ((mean, dm, qs["km"]), (var, dv, qs["kv"])):
+        x32 = x.astype(np.float32).astype(np.float64)
+        sc = np.ldexp(1.0, k.astype(np.int64)).repeat(32, axis=-1)
+        a = np.abs(x32) / sc                    # in [0, 6]
+        half_gap = np.where(a < 2, 0.25, np.where(a < 4, 0.5, 1.0))
+        assert np.all(np.abs(d - x32) <= half_gap * sc)
+        assert np.all(np.sign(d) * np.sign(x32) >= 0)
+        gmax = np.abs(x32).reshape(2, 2, 5, 2, 32).max(-1)
+        kk = k.astype(np.int64)
+        nz = gmax > 0
+        # the smallest power of two whose 6 multiple holds the group maximum
+        assert np.all(gmax[nz] <= 6 * np.ldexp(1.0, kk[nz]))
+        assert np.all(gmax[nz] > 6 * np.ldexp(1.0, kk[nz] - 1))
+        assert np.all(kk[~nz] == -126)
+    assert np.all(dm[0, 0, 1, :32] == 0) and np.all(dv[1, 1, 2, 32:] == 0)
+    assert np.all(qs["cv"] < 8)                 # variances carry no sign
+
+
+def test_fp4_codes_are_the_nearest_e2m1_values():
+    # brute force: every scaled value against all 15 distinct values; at an exact
+    # midpoint the even mantissa (code bit 0 clear) wins
+    rng = np.random.default_rng(81)
+    mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+    y = np.concatenate([mids, -mids, rng.uniform(-6, 6, 2000)])
+    y = y[: (len(y) // 32) * 32].reshape(1, 1, -1, 32)
+    y[..., 0] = 6.0                             # every group's scale is 2^0
+    qs = oracle.quantize_stats(y, np.zeros_like(y), "fp4")
+    assert np.all(qs["km"] == 0)
+    vals = np.array(E2M1_TABLE)
+    for yy, c in zip(y.reshape(-1), qs["cm"].reshape(-1)):
+        yy32 = float(np.float32(yy))
+        dist = np.abs(abs(yy32) - vals)
+        best = np.flatnonzero(dist == dist.min())
+        want = best[0] if len(best) == 1 else best[best % 2 == 0][0]
+        assert int(c) & 7 == want and (int(c) >> 3) == int(np.signbit(yy32))
+
+
+def test_fp4_power_of_two_scaling_shifts_only_the_exponent():
+    mean, var = _fp4_inputs(82)
+    q0 = oracle.quantize_stats(mean, var, "fp4")
+    q1 = oracle.quantize_stats(mean * 2.0 ** 7, var * 2.0 ** -5, "fp4")
+    assert np.array_equal(q0["cm"], q1["cm"]) and np.array_equal(q0["cv"], q1["cv"])
+    nzm = np.abs(mean).reshape(2, 2, 5, 2, 32).max(-1) > 0
+    nzv = var.reshape(2, 2, 5, 2, 32).max(-1) > 0
+    assert np.all(q1["km"][nzm].astype(int) == q0["km"][nzm].astype(int) + 7)
+    assert np.all(q1["kv"][nzv].astype(int) == q0["kv"][nzv].astype(int) - 5)
+
+
+def test_fp4_on_the_grid_round_trip_exactly():
+    rng = np.random.default_rng(83)
+    vals = np.array(E2M1_TABLE)
+    m = vals[rng.integers(0, 8, (1, 2, 3, 64))] * rng.choice([-1.0, 1.0], (1, 2, 3, 64))
+    m[..., 0] = 6.0                             # every group reaches the top value
+    m[..., 32] = -6.0
+    v = vals[rng.integers(0, 8, (1, 2, 3, 64))]
+    v[..., 0] = 6.0
+    v[..., 32] = 6.0
+    mean, var = m * 2.0 ** -4, v * 2.0 ** 3
+    qs = oracle.quantize_stats(mean, var, "fp4")
+    dm, dv = oracle.dequantize_stats(qs)
+    assert np.array_equal(dm, mean) and np.array_equal(dv, var)
+    assert np.all(qs["km"] == -4) and np.all(qs["kv"] == 3)
+
+
+def test_fp4_selection_equals_plain_selection_on_grid_statistics():
+    # keys constant within a block, on the E2M1 grid: the mean is exactly
+    # representable, the variance 0, so the selection is that of fp32 statistics
+    rng = np.random.default_rng(84)
+    B, Hq, Hkv, T, d, blk = 1, 4, 2, 256, 64, 32
+    grid = np.array(E2M1_TABLE, np.float32) * np.float32(0.125)
+    vals = grid[rng.integers(0, 8, (B, Hkv, T // blk, d))] * rng.choice([-1, 1], (B, Hkv, T // blk, d)).astype(np.float32)
+    vals[..., 0] = 6 * 0.125
+    vals[..., 32] = -6 * 0.125
+    k = np.repeat(vals, blk, axis=2)
+    q = _rand((B, Hq, T, d), 85)
+    a = oracle.select(q, k, "f32", blk, 0.125, 0.6)
+    b = oracle.select_quantized(q, k, "f32", blk, 0.125, 0.6, fmt="fp4")
+    assert np.array_equal(a["count"], b["count"]) and np.array_equal(a["idx"], b["idx"])
+    assert np.array_equal(a["scores"], b["scores"])
+
+
 # ---------------------------------------------------------------- score-ordered early stop
 # S2O, sections 2-3: blocks in descending estimated importance after the dense pass
 # over the own block; stop once a block's marginal gain in attention mass falls
