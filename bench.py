@@ -839,10 +839,9 @@ def main():
                     "GB/s": (dbytes + dstate.numel() * 4) / (t_drla / 1e3) / 1e9,
                     "tokens/s": world * wd.B / ((t_dsel + t_drla) / 1e3)}
             del dstate, ws_r, orla
-        # selection on INT4 microscale statistics (SpotAttention, section 4)
-        dq = None
-        if not args.no_quant:
-            qrec = spa.spa_quantize_block_stats(dm, dv, wd.T, wd.block)
+        # selection on INT4 or FP4 microscale statistics (SpotAttention, section 4)
+        def quant_step(fmt):
+            qrec = spa.spa_quantize_block_stats(dm, dv, wd.T, wd.block, fmt=fmt)
             qi = torch.empty_like(didx)
             qc = torch.empty_like(dcnt)
             q_ms = []
@@ -850,13 +849,13 @@ def main():
                 flush.zero_()
                 e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 e0.record(stream)
-                spa.spa_quantize_block_stats(dm, dv, wd.T, wd.block, qstats=qrec)
+                spa.spa_quantize_block_stats(dm, dv, wd.T, wd.block, qstats=qrec, fmt=fmt)
                 e1.record(stream)
                 torch.cuda.synchronize()
                 q_ms.append(e0.elapsed_time(e1))
             for _ in range(3):
                 spa.spa_select_quantized(qd_, qrec, wd.T, wd.block, wd.scale, wd.top_p, idx=qi,
-                                         count=qc)
+                                         count=qc, fmt=fmt)
             torch.cuda.synchronize()
             assert spa.spa_get_device_error() == 0
             # the decode step on records: statistics and record of the newest block in
@@ -864,9 +863,9 @@ def main():
             qs_evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n_dec)]
             qout = torch.empty_like(dout)
             for _ in range(3):
-                spa.spa_block_stats_quantized(kc, wd.block, last, last + 1, dm, dv, qrec)
+                spa.spa_block_stats_quantized(kc, wd.block, last, last + 1, dm, dv, qrec, fmt=fmt)
                 spa.spa_select_quantized(qd_, qrec, wd.T, wd.block, wd.scale, wd.top_p, idx=qi,
-                                         count=qc)
+                                         count=qc, fmt=fmt)
                 spa.spa_sparse_attn_decode(qd_, kc, vc, wd.block, qi, qc, wd.scale, workspace=ws,
                                            out=qout)
             torch.cuda.synchronize()
@@ -876,10 +875,10 @@ def main():
             for s in range(n_dec):
                 flush.zero_()
                 qs_evs[s][0].record(stream)
-                spa.spa_block_stats_quantized(kc, wd.block, last, last + 1, dm, dv, qrec)
+                spa.spa_block_stats_quantized(kc, wd.block, last, last + 1, dm, dv, qrec, fmt=fmt)
                 qs_evs[s][1].record(stream)
                 spa.spa_select_quantized(qd_, qrec, wd.T, wd.block, wd.scale, wd.top_p, idx=qi,
-                                         count=qc)
+                                         count=qc, fmt=fmt)
                 qs_evs[s][2].record(stream)
                 spa.spa_sparse_attn_decode(qd_, kc, vc, wd.block, qi, qc, wd.scale, workspace=ws,
                                            out=qout)
@@ -890,7 +889,7 @@ def main():
             t_qsel = rank_max(statistics.mean(e[1].elapsed_time(e[2]) for e in qs_evs))
             t_qdec = rank_max(statistics.mean(e[2].elapsed_time(e[3]) for e in qs_evs))
             qbytes = kept_kv_bytes(qc.cpu().numpy(), qi.cpu().numpy(), wd.G, wd.T, wd.block, wd.d)
-            dq = {"stats_bytes_fp32": 2 * dm.numel() * 4, "stats_bytes_int4": qrec.numel(),
+            res = {"format": fmt, "stats_bytes_fp32": 2 * dm.numel() * 4, "stats_bytes_records": qrec.numel(),
                   "quantize_full_cache_ms": statistics.median(q_ms[1:]),
                   "update_newest_block_ms": t_qupd, "select_ms": t_qsel, "attn_ms": t_qdec,
                   "kept_kv_bytes": qbytes, "GB/s": qbytes / (t_qdec / 1e3) / 1e9,
@@ -898,6 +897,12 @@ def main():
                   "tokens/s": world * wd.B / ((t_qupd + t_qsel + t_qdec) / 1e3)}
             del qout
             del qrec, qi, qc
+            return res
+
+        dq = None
+        if not args.no_quant:
+            dq = quant_step("int4")
+            dq["fp4"] = quant_step("fp4")
         decode = {"workload": wd.name, "kept_kv_bytes": dbytes, "attn_ms": t_dec,
                   "update_newest_block_ms": t_dupd, "select_ms": t_dsel,
                   "select_GB/s": 2 * dm.numel() * 4 / (t_dsel / 1e3) / 1e9,

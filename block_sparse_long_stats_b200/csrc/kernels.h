@@ -19,18 +19,19 @@ cudaError_t launch_select(const void *q, bool bf16, const float *mean, const flo
                           float top_p, int n_sink, int n_local, int k_min, int32_t *idx, int cap,
                           int32_t *count, int *err, cudaStream_t s, const void *qstats = nullptr,
                           bool score_order = false, const float *mean_p = nullptr,
-                          const float *var_p = nullptr, int seg_blocks = 0);
+                          const float *var_p = nullptr, int seg_blocks = 0, int qfmt = 0);
 
-// Quantised block statistics (INT4 microscale records of d + d/16 bytes per block;
-// format in qstats.cu). launch_select reads them instead of mean/var when qstats is set.
+// Quantised block statistics (microscale records of d + d/16 bytes per block, 4-bit
+// codes: qfmt 0 INT4, 1 FP4 E2M1; format in qstats.cu). launch_select reads them
+// instead of mean/var when qstats is set.
 size_t quantized_stats_bytes(int B, int Hkv, int T, int d, int block);
 cudaError_t launch_quantize_stats(const float *mean, const float *var, int B, int Hkv, int T, int d,
-                                  int block, int blk_begin, int blk_end, void *qstats,
+                                  int block, int blk_begin, int blk_end, void *qstats, int qfmt,
                                   cudaStream_t s);
 // Statistics and records of blocks [blk_begin, blk_end) in one pass (few blocks).
 cudaError_t launch_stats_quantize(const void *k, bool bf16, int B, int Hkv, int T, int d,
                                   int block, int blk_begin, int blk_end, float *mean, float *var,
-                                  void *qstats, cudaStream_t s);
+                                  void *qstats, int qfmt, cudaStream_t s);
 
 cudaError_t launch_prefill_f32(const float *q, const float *k, const float *v, int B, int Hq,
                                int Hkv, int L, int d, int block, const int32_t *idx, int cap,

@@ -109,16 +109,23 @@ __device__ __forceinline__ void load_stats(const float *mb, const float *vb, flo
     }
 }
 
-// The same PL components from a quantised record (INT4 codes, a power-of-two scale
-// per 32 features; layout in qstats.cu): the codes as floats in mu, vr and the
-// lane's two group scales 2^k in sm, sv (a lane's PL features lie in one group).
+// The same PL components from a quantised record (4-bit codes, a power-of-two scale
+// per 32 features; layout in qstats.cu): the codes' values as floats in mu, vr and
+// the lane's two group scales 2^k in sm, sv (a lane's PL features lie in one group).
 // The callers scale the lane's dot and variance sums by sm, sv instead of each
 // component: scaling by a power of two commutes with every rounding of the FMA
-// chain (in the normal range), so the sums equal those over code * 2^k exactly.
-// A 4-bit code n becomes a float without a conversion instruction: 2^23 + n has n
-// in its low mantissa bits, so subtracting 2^23 (plus the signed codes' bias of 8,
-// n ^ 8 = code + 8 for two's-complement nibbles) is exact.
-template <int D>
+// chain (in the normal range), so the sums equal those over value * 2^k exactly.
+// QS = 1, INT4: a code n becomes a float without a conversion instruction: 2^23 + n
+// has n in its low mantissa bits, so subtracting 2^23 (plus the signed codes' bias
+// of 8, n ^ 8 = code + 8 for two's-complement nibbles) is exact. QS = 2, FP4 (E2M1):
+// twice the magnitude is an integer (0, 1, 2, 3, 4, 6, 8, 12), read from a nibble
+// table in one word, made a float the same way and halved; the sign bit is bit 3.
+__device__ __forceinline__ float e2m1_value(uint32_t n) {
+    const uint32_t twice = (0xC8643210u >> (4 * (n & 7u))) & 15u;
+    const float a = (__uint_as_float(0x4B000000u | twice) - 8388608.0f) * 0.5f;
+    return __uint_as_float(__float_as_uint(a) | ((n & 8u) << 28));
+}
+template <int D, int QS>
 __device__ __forceinline__ void load_stats_q(const uint8_t *rec, int lane, float (&mu)[D / 32],
                                              float (&vr)[D / 32], float &sm, float &sv) {
     constexpr int PL = D / 32, LPG = 32 / PL;
@@ -136,8 +143,13 @@ __device__ __forceinline__ void load_stats_q(const uint8_t *rec, int lane, float
     sv = __int_as_float((kv + 127) << 23);
 #pragma unroll
     for (int c = 0; c < PL; ++c) {
-        mu[c] = __uint_as_float(0x4B000000u | (((cm >> (4 * c)) & 15u) ^ 8u)) - 8388616.0f;
-        vr[c] = __uint_as_float(0x4B000000u | ((cv >> (4 * c)) & 15u)) - 8388608.0f;
+        if constexpr (QS == 2) {
+            mu[c] = e2m1_value(cm >> (4 * c));
+            vr[c] = e2m1_value(cv >> (4 * c));
+        } else {
+            mu[c] = __uint_as_float(0x4B000000u | (((cm >> (4 * c)) & 15u) ^ 8u)) - 8388616.0f;
+            vr[c] = __uint_as_float(0x4B000000u | ((cv >> (4 * c)) & 15u)) - 8388608.0f;
+        }
     }
 }
 
@@ -234,6 +246,7 @@ struct SelectArgs {
     int sort_cap;   // power of two >= the largest residual of any unit
     bool prescored; // decode: the fp32 scores are already in the unit's row of idx
     const uint8_t *qstats;  // quantised statistics (records of d + d/16 bytes) or null
+    int qfmt;               // their codes: 0 INT4, 1 FP4 (E2M1)
     bool score_order;       // prefill: lists in traversal order instead of ascending
     // segment-permuted layout: blocks before the query's own segment are scored on
     // the permuted keys' statistics (seg_blocks = 0: off)
@@ -408,7 +421,7 @@ __device__ __forceinline__ void write_ascending(const unsigned char *flag, const
     if (tid == 0) a.count[unit] = *isum;
 }
 
-template <typename T, int D, bool QS>
+template <typename T, int D, int QS>
 __global__ void __launch_bounds__(kThreads) select_kernel(SelectArgs a) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     uint64_t *keys = reinterpret_cast<uint64_t *>(smem_raw);               // [sort_cap]
@@ -498,7 +511,7 @@ __global__ void __launch_bounds__(kThreads) select_kernel(SelectArgs a) {
             for (int u = 0; u < U; ++u) {
                 const int j = r_lo + min(r0 + u, nres - 1);   // past the end: a repeat, unused
                 if constexpr (QS)
-                    load_stats_q<D>(qb + (size_t)j * (D + D / 16), lane, mu[u], vr[u], sm[u], sv[u]);
+                    load_stats_q<D, QS>(qb + (size_t)j * (D + D / 16), lane, mu[u], vr[u], sm[u], sv[u]);
                 else if (j < seg0)
                     load_stats<PL>(mbp + (size_t)j * D, vbp + (size_t)j * D, mu[u], vr[u]);
                 else
@@ -732,7 +745,7 @@ __device__ void cta_sort_cut(const uint64_t *keys, uint64_t *xbuf, unsigned char
 // the scores from lane_partials + reduce_transpose (U candidates x G heads per
 // reduction, as in decode scoring), then warp h sorts and cuts head h's keys in
 // registers and writes head h's list, with no block-wide barrier after the scoring.
-template <typename T, int D, int G, bool QS>
+template <typename T, int D, int G, int QS>
 __global__ void __launch_bounds__(kThreads, 3) select_group_kernel(SelectArgs a) {
     constexpr int PL = D / 32;
     constexpr int U = G >= 8 ? 2 : (G == 4 ? 4 : 8);
@@ -845,7 +858,7 @@ __global__ void __launch_bounds__(kThreads, 3) select_group_kernel(SelectArgs a)
             for (int u = 0; u < U; ++u) {
                 const int j = r_lo + min(r0 + u, nres - 1);   // past the end: a repeat, unused
                 if constexpr (QS)
-                    load_stats_q<D>(qb + (size_t)j * (D + D / 16), lane, mu[u], vr[u], sm[u], sv[u]);
+                    load_stats_q<D, QS>(qb + (size_t)j * (D + D / 16), lane, mu[u], vr[u], sm[u], sv[u]);
                 else if (j < seg0)
                     load_stats<PL>(mbp + (size_t)j * D, vbp + (size_t)j * D, mu[u], vr[u]);
                 else
@@ -945,7 +958,7 @@ __global__ void __launch_bounds__(kThreads, 3) select_group_kernel(SelectArgs a)
 // the cut kernel replaces it with the kept list.
 constexpr int kDecTile = 256;
 
-template <typename T, int D, int G, bool QS>
+template <typename T, int D, int G, int QS>
 __global__ void __launch_bounds__(kThreads, 2) decode_score_kernel(SelectArgs a) {
     constexpr int PL = D / 32;
     // U candidates per warp step, so that the 2G partial sums of all of them fill
@@ -991,7 +1004,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_score_kernel(SelectArgs a)
         for (int u = 0; u < U; ++u) {
             const int j = min(j0 + r + u, a.nb - 1);
             if constexpr (QS)
-                load_stats_q<D>(qb + (size_t)j * (D + D / 16), lane, m[u], w[u], cs[u], ws[u]);
+                load_stats_q<D, QS>(qb + (size_t)j * (D + D / 16), lane, m[u], w[u], cs[u], ws[u]);
             else
                 load_stats<PL>(mb + (size_t)j * D, vb + (size_t)j * D, m[u], w[u]);
         }
@@ -1059,7 +1072,25 @@ __device__ __forceinline__ uint32_t codes_bf16x2(uint32_t w, int t, bool is_sign
     return r;
 }
 
-template <int G>
+// Byte t of w: two FP4 (E2M1) codes as exact bf16 values: the magnitudes' low and
+// high bf16 bytes from two byte tables (prmt), the sign bits from the codes.
+__device__ __forceinline__ uint32_t fp4_bf16x2(uint32_t w, int t) {
+    const uint32_t b = (w >> (8 * t)) & 0xFFu;
+    const uint32_t c0 = b & 7u, c1 = (b >> 4) & 7u;
+    uint32_t lo, hi;
+    // low bytes of the bf16 magnitudes 0, .5, 1, 1.5, 2, 3, 4, 6: 00 00 80 C0 00 40 80 C0
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(lo) : "r"(0xC0800000u), "r"(0xC0804000u), "r"(c0 | (c1 << 8)));
+    // high bytes: 00 3F 3F 3F 40 40 40 40
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(hi) : "r"(0x3F3F3F00u), "r"(0x40404040u), "r"((c0 << 4) | (c1 << 12)));
+    return lo | hi | ((b & 0x08u) << 12) | ((b & 0x80u) << 24);
+}
+template <int QS>
+__device__ __forceinline__ uint32_t codes_bf16(uint32_t w, int t, bool is_signed) {
+    if constexpr (QS == 2) return fp4_bf16x2(w, t);
+    else return codes_bf16x2(w, t, is_signed);
+}
+
+template <int G, int QS>
 __global__ void __launch_bounds__(kThreads, 2) decode_score_q_mma_kernel(SelectArgs a) {
     constexpr int D = 128, RB = D + D / 16;   // record bytes
     static_assert(G >= 1 && G <= 8, "the heads are the 8 MMA columns");
@@ -1115,16 +1146,16 @@ __global__ void __launch_bounds__(kThreads, 2) decode_score_q_mma_kernel(SelectA
             const uint4 va = ld16(ra + D / 2 + 16 * gr), vb = ld16(rb + D / 2 + 16 * gr);
             float pd[4] = {0.f, 0.f, 0.f, 0.f}, pq[4] = {0.f, 0.f, 0.f, 0.f};
             // k-step 2 gr: features 0..15 of the group (words x, y); 2 gr + 1: 16..31 (z, w)
-            mma16816(pd, codes_bf16x2(ma.x, t, true), codes_bf16x2(mb.x, t, true),
-                     codes_bf16x2(ma.y, t, true), codes_bf16x2(mb.y, t, true), bq[2 * gr][0],
+            mma16816(pd, codes_bf16<QS>(ma.x, t, true), codes_bf16<QS>(mb.x, t, true),
+                     codes_bf16<QS>(ma.y, t, true), codes_bf16<QS>(mb.y, t, true), bq[2 * gr][0],
                      bq[2 * gr][1]);
-            mma16816(pd, codes_bf16x2(ma.z, t, true), codes_bf16x2(mb.z, t, true),
-                     codes_bf16x2(ma.w, t, true), codes_bf16x2(mb.w, t, true), bq[2 * gr + 1][0],
+            mma16816(pd, codes_bf16<QS>(ma.z, t, true), codes_bf16<QS>(mb.z, t, true),
+                     codes_bf16<QS>(ma.w, t, true), codes_bf16<QS>(mb.w, t, true), bq[2 * gr + 1][0],
                      bq[2 * gr + 1][1]);
-            const uint32_t v0 = codes_bf16x2(va.x, t, false), v1 = codes_bf16x2(vb.x, t, false);
-            const uint32_t v2 = codes_bf16x2(va.y, t, false), v3 = codes_bf16x2(vb.y, t, false);
-            const uint32_t v4 = codes_bf16x2(va.z, t, false), v5 = codes_bf16x2(vb.z, t, false);
-            const uint32_t v6 = codes_bf16x2(va.w, t, false), v7 = codes_bf16x2(vb.w, t, false);
+            const uint32_t v0 = codes_bf16<QS>(va.x, t, false), v1 = codes_bf16<QS>(vb.x, t, false);
+            const uint32_t v2 = codes_bf16<QS>(va.y, t, false), v3 = codes_bf16<QS>(vb.y, t, false);
+            const uint32_t v4 = codes_bf16<QS>(va.z, t, false), v5 = codes_bf16<QS>(vb.z, t, false);
+            const uint32_t v6 = codes_bf16<QS>(va.w, t, false), v7 = codes_bf16<QS>(vb.w, t, false);
             mma16816(pq, v0, v1, v2, v3, bh[2 * gr][0], bh[2 * gr][1]);
             mma16816(pq, v0, v1, v2, v3, bl[2 * gr][0], bl[2 * gr][1]);
             mma16816(pq, v4, v5, v6, v7, bh[2 * gr + 1][0], bh[2 * gr + 1][1]);
@@ -1154,16 +1185,16 @@ __global__ void __launch_bounds__(kThreads, 2) decode_score_q_mma_kernel(SelectA
     }
 }
 
-template <typename T, int D, bool QS>
+template <typename T, int D, int QS>
 cudaError_t launch_decode_scores(const SelectArgs &a, cudaStream_t s) {
     dim3 grid((unsigned)((a.nb + kDecTile - 1) / kDecTile), (unsigned)(a.B * a.Hkv));
     if constexpr (QS && D == 128 && sizeof(T) == 2) {
-        // INT4 records with bf16 queries: the tensor-core form
+        // records with bf16 queries: the tensor-core form
         switch (a.G) {
-            case 1: decode_score_q_mma_kernel<1><<<grid, kThreads, 0, s>>>(a); break;
-            case 2: decode_score_q_mma_kernel<2><<<grid, kThreads, 0, s>>>(a); break;
-            case 4: decode_score_q_mma_kernel<4><<<grid, kThreads, 0, s>>>(a); break;
-            default: decode_score_q_mma_kernel<8><<<grid, kThreads, 0, s>>>(a); break;
+            case 1: decode_score_q_mma_kernel<1, QS><<<grid, kThreads, 0, s>>>(a); break;
+            case 2: decode_score_q_mma_kernel<2, QS><<<grid, kThreads, 0, s>>>(a); break;
+            case 4: decode_score_q_mma_kernel<4, QS><<<grid, kThreads, 0, s>>>(a); break;
+            default: decode_score_q_mma_kernel<8, QS><<<grid, kThreads, 0, s>>>(a); break;
         }
         return cudaGetLastError();
     }
@@ -1437,7 +1468,7 @@ cudaError_t allow_smem(K kern, size_t dyn) {
     return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
 }
 
-template <typename T, int D, int G, bool QS>
+template <typename T, int D, int G, int QS>
 cudaError_t launch_group(const SelectArgs &a, cudaStream_t s) {
     const size_t kcap = a.sort_cap <= kWarpSortMax ? kWarpSortMax : a.sort_cap;
     const size_t smem = (size_t)G * kcap * 8 + (a.sort_cap <= kWarpSortMax ? 0 : 2 * kcap * 8) +
@@ -1449,7 +1480,7 @@ cudaError_t launch_group(const SelectArgs &a, cudaStream_t s) {
     return cudaGetLastError();
 }
 
-template <typename T, int D, bool QS>
+template <typename T, int D, int QS>
 cudaError_t launch_tq(const SelectArgs &a, cudaStream_t s) {
     // prefill, up to kCtaSortMax residual candidates, a head grouping the grouped
     // kernel has: one CTA per kv-head and query block
@@ -1482,7 +1513,8 @@ cudaError_t launch_tq(const SelectArgs &a, cudaStream_t s) {
 
 template <typename T, int D>
 cudaError_t launch_t(const SelectArgs &a, cudaStream_t s) {
-    return a.qstats ? launch_tq<T, D, true>(a, s) : launch_tq<T, D, false>(a, s);
+    if (!a.qstats) return launch_tq<T, D, 0>(a, s);
+    return a.qfmt == 1 ? launch_tq<T, D, 2>(a, s) : launch_tq<T, D, 1>(a, s);
 }
 
 }  // namespace
@@ -1492,8 +1524,9 @@ cudaError_t launch_select(const void *q, bool bf16, const float *mean, const flo
                           float top_p, int n_sink, int n_local, int k_min, int32_t *idx, int cap,
                           int32_t *count, int *err, cudaStream_t s, const void *qstats,
                           bool score_order, const float *mean_p, const float *var_p,
-                          int seg_blocks) {
+                          int seg_blocks, int qfmt) {
     SelectArgs a;
+    a.qfmt = qfmt;
     a.score_order = score_order;
     a.mean_p = mean_p;
     a.var_p = var_p;

@@ -308,9 +308,10 @@ SPA_API size_t spa_quantized_stats_bytes(int B, int Hkv, int T, int d, int block
 
 SPA_API spa_status spa_quantize_block_stats(const float *mean, const float *var, int B, int Hkv,
                                             int T, int d, int block, int blk_begin, int blk_end,
-                                            void *qstats, spa_stream stream) {
+                                            void *qstats, spa_qformat fmt, spa_stream stream) {
     t_last_error.clear();
     if (!mean || !var || !qstats) return fail(SPA_ERR_INVALID, "null pointer");
+    if (fmt != SPA_QFMT_INT4 && fmt != SPA_QFMT_FP4) return fail(SPA_ERR_INVALID, "unknown record format");
     if (B <= 0 || Hkv <= 0 || T <= 0 || d <= 0 || block <= 0)
         return fail(SPA_ERR_INVALID, "sizes must be positive");
     const int nb = ceil_div(T, block);
@@ -320,16 +321,17 @@ SPA_API spa_status spa_quantize_block_stats(const float *mean, const float *var,
         return fail(SPA_ERR_INVALID, "tensors must be 16-byte aligned");
     if (d != 64 && d != 128) return fail(SPA_ERR_UNSUPPORTED, "d must be 64 or 128");
     cudaError_t e = launch_quantize_stats(mean, var, B, Hkv, T, d, block, blk_begin, blk_end, qstats,
-                                          static_cast<cudaStream_t>(stream));
+                                          (int)fmt, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? SPA_OK : cuda_fail(e, "quantize launch");
 }
 
 SPA_API spa_status spa_block_stats_quantized(const void *k, spa_dtype dt, int B, int Hkv, int T,
                                              int d, int block, int blk_begin, int blk_end,
                                              float *mean, float *var, void *qstats,
-                                             spa_stream stream) {
+                                             spa_qformat fmt, spa_stream stream) {
     t_last_error.clear();
     if (!k || !mean || !var || !qstats) return fail(SPA_ERR_INVALID, "null pointer");
+    if (fmt != SPA_QFMT_INT4 && fmt != SPA_QFMT_FP4) return fail(SPA_ERR_INVALID, "unknown record format");
     if (B <= 0 || Hkv <= 0 || T <= 0 || d <= 0 || block <= 0)
         return fail(SPA_ERR_INVALID, "sizes must be positive");
     if (dt != SPA_F32 && dt != SPA_BF16) return fail(SPA_ERR_INVALID, "unknown dtype");
@@ -340,17 +342,18 @@ SPA_API spa_status spa_block_stats_quantized(const void *k, spa_dtype dt, int B,
         return fail(SPA_ERR_INVALID, "tensors must be 16-byte aligned");
     if (d != 64 && d != 128) return fail(SPA_ERR_UNSUPPORTED, "d must be 64 or 128");
     cudaError_t e = launch_stats_quantize(k, dt == SPA_BF16, B, Hkv, T, d, block, blk_begin, blk_end,
-                                          mean, var, qstats, static_cast<cudaStream_t>(stream));
+                                          mean, var, qstats, (int)fmt, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? SPA_OK : cuda_fail(e, "stats+quantize launch");
 }
 
-SPA_API spa_status spa_select_quantized(const void *q, spa_dtype dt, const void *qstats, int B,
-                                        int Hq, int Hkv, int Lq, int T, int d, int block,
-                                        float scale, float top_p, int n_sink, int n_local,
-                                        int k_min, int32_t *idx, int cap, int32_t *count,
-                                        spa_stream stream) {
+SPA_API spa_status spa_select_quantized(const void *q, spa_dtype dt, const void *qstats,
+                                        spa_qformat fmt, int B, int Hq, int Hkv, int Lq, int T,
+                                        int d, int block, float scale, float top_p, int n_sink,
+                                        int n_local, int k_min, int32_t *idx, int cap,
+                                        int32_t *count, spa_stream stream) {
     t_last_error.clear();
     if (!q || !qstats || !idx || !count) return fail(SPA_ERR_INVALID, "null pointer");
+    if (fmt != SPA_QFMT_INT4 && fmt != SPA_QFMT_FP4) return fail(SPA_ERR_INVALID, "unknown record format");
     if (B <= 0 || Hq <= 0 || Hkv <= 0 || Lq <= 0 || T <= 0 || d <= 0 || block <= 0)
         return fail(SPA_ERR_INVALID, "sizes must be positive");
     if (Hq % Hkv) return fail(SPA_ERR_INVALID, "Hq must be a multiple of Hkv");
@@ -369,7 +372,8 @@ SPA_API spa_status spa_select_quantized(const void *q, spa_dtype dt, const void 
     if (!err) return fail(SPA_ERR_CUDA, "device error word unavailable");
     cudaError_t e = launch_select(q, dt == SPA_BF16, nullptr, nullptr, B, Hq, Hkv, Lq, T, d, block,
                                   scale, top_p, n_sink, n_local, k_min, idx, cap, count, err,
-                                  static_cast<cudaStream_t>(stream), qstats);
+                                  static_cast<cudaStream_t>(stream), qstats, false, nullptr, nullptr,
+                                  0, (int)fmt);
     return e == cudaSuccess ? SPA_OK : cuda_fail(e, "select launch");
 }
 

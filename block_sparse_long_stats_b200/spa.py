@@ -63,9 +63,9 @@ def lib() -> ctypes.CDLL:
                                                  _I, _P, _F, _P, _P, _P, _P]
         L.spa_quantized_stats_bytes.argtypes = [_I, _I, _I, _I, _I]
         L.spa_quantized_stats_bytes.restype = ctypes.c_size_t
-        L.spa_quantize_block_stats.argtypes = [_P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P]
-        L.spa_block_stats_quantized.argtypes = [_P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P]
-        L.spa_select_quantized.argtypes = [_P, _I, _P, _I, _I, _I, _I, _I, _I, _I, _F, _F, _I, _I,
+        L.spa_quantize_block_stats.argtypes = [_P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _I, _P]
+        L.spa_block_stats_quantized.argtypes = [_P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _I, _P]
+        L.spa_select_quantized.argtypes = [_P, _I, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _F, _I, _I,
                                            _I, _P, _I, _P, _P]
         L.spa_select_score_order.argtypes = [_P, _I, _P, _P, _I, _I, _I, _I, _I, _I, _F, _F, _I,
                                              _I, _I, _P, _I, _P, _P]
@@ -130,6 +130,15 @@ def _ptr(t: torch.Tensor | None):
     return ctypes.c_void_p(t.data_ptr())
 
 
+_QFMT = {"int4": 0, "fp4": 1}
+
+
+def _qfmt(fmt: str) -> int:
+    if fmt not in _QFMT:
+        raise ValueError(f"unknown record format {fmt!r} (int4 or fp4)")
+    return _QFMT[fmt]
+
+
 def _dt(t: torch.Tensor) -> int:
     if t.dtype == torch.bfloat16:
         return SPA_BF16
@@ -187,8 +196,10 @@ def spa_quantized_stats_bytes(B: int, Hkv: int, T: int, d: int, block: int) -> i
 
 def spa_quantize_block_stats(mean: torch.Tensor, var: torch.Tensor, T: int, block: int,
                              blk_begin: int = 0, blk_end: int | None = None,
-                             qstats: torch.Tensor | None = None, stream=None) -> torch.Tensor:
-    """INT4 microscale records [B, Hkv, nb, d + d/16] uint8 from fp32 block statistics."""
+                             qstats: torch.Tensor | None = None, fmt: str = "int4",
+                             stream=None) -> torch.Tensor:
+    """Microscale records [B, Hkv, nb, d + d/16] uint8 (fmt "int4" or "fp4") from fp32
+    block statistics."""
     B, Hkv, nb, d = mean.shape
     if blk_end is None:
         blk_end = nb
@@ -196,26 +207,28 @@ def spa_quantize_block_stats(mean: torch.Tensor, var: torch.Tensor, T: int, bloc
         qstats = torch.empty((B, Hkv, nb, d + d // 16), device=mean.device, dtype=torch.uint8)
     _check("spa_quantize_block_stats",
            lib().spa_quantize_block_stats(_ptr(mean), _ptr(var), B, Hkv, T, d, block, blk_begin,
-                                          blk_end, _ptr(qstats), _stream(stream)))
+                                          blk_end, _ptr(qstats), _qfmt(fmt), _stream(stream)))
     return qstats
 
 
 def spa_block_stats_quantized(k: torch.Tensor, block: int, blk_begin: int, blk_end: int,
                               mean: torch.Tensor, var: torch.Tensor, qstats: torch.Tensor,
-                              stream=None) -> None:
-    """Statistics and INT4 records of blocks [blk_begin, blk_end) in one pass, into the
-    caller's mean, var [B, Hkv, nb, d] and qstats [B, Hkv, nb, d + d/16]."""
+                              fmt: str = "int4", stream=None) -> None:
+    """Statistics and records (fmt "int4" or "fp4") of blocks [blk_begin, blk_end) in
+    one pass, into the caller's mean, var [B, Hkv, nb, d] and qstats [B, Hkv, nb,
+    d + d/16]."""
     B, Hkv, T, d = k.shape
     _check("spa_block_stats_quantized",
            lib().spa_block_stats_quantized(_ptr(k), _dt(k), B, Hkv, T, d, block, blk_begin, blk_end,
-                                           _ptr(mean), _ptr(var), _ptr(qstats), _stream(stream)))
+                                           _ptr(mean), _ptr(var), _ptr(qstats), _qfmt(fmt),
+                                           _stream(stream)))
 
 
 def spa_select_quantized(q: torch.Tensor, qstats: torch.Tensor, T: int, block: int, scale: float,
                          top_p: float, n_sink: int = 1, n_local: int = 1, k_min: int = 0,
                          idx: torch.Tensor | None = None, count: torch.Tensor | None = None,
-                         stream=None):
-    """spa_select on quantised statistics. Returns (idx, count)."""
+                         fmt: str = "int4", stream=None):
+    """spa_select on quantised statistics (records in format fmt). Returns (idx, count)."""
     B, Hq, Lq, d = q.shape
     Hkv = qstats.shape[1]
     nb = -(-T // block)
@@ -225,8 +238,8 @@ def spa_select_quantized(q: torch.Tensor, qstats: torch.Tensor, T: int, block: i
     if count is None:
         count = torch.empty((B, Hq, nq), device=q.device, dtype=torch.int32)
     _check("spa_select_quantized",
-           lib().spa_select_quantized(_ptr(q), _dt(q), _ptr(qstats), B, Hq, Hkv, Lq, T, d, block,
-                                      scale, top_p, n_sink, n_local, k_min, _ptr(idx),
+           lib().spa_select_quantized(_ptr(q), _dt(q), _ptr(qstats), _qfmt(fmt), B, Hq, Hkv, Lq,
+                                      T, d, block, scale, top_p, n_sink, n_local, k_min, _ptr(idx),
                                       idx.shape[-1], _ptr(count), _stream(stream)))
     return idx, count
 

@@ -58,6 +58,8 @@ typedef enum {
 } spa_status;
 
 typedef enum { SPA_F32 = 0, SPA_BF16 = 1 } spa_dtype;
+/* The 4-bit code of a quantised-statistics record (spa_quantize_block_stats). */
+typedef enum { SPA_QFMT_INT4 = 0, SPA_QFMT_FP4 = 1 } spa_qformat;
 
 /* Device-side error codes reported by spa_get_device_error. */
 #define SPA_DEVERR_NONE 0
@@ -115,53 +117,61 @@ spa_status spa_select(const void *q, spa_dtype dt, const float *mean, const floa
 
 /*
  * Quantised block statistics. Follows "SpotAttention", section 4: the selector's
- * cache may be held in INT4 / FP4 microscale (about 3.5x smaller than bf16) without
+ * cache may be held in INT4 or FP4 microscale (about 3.5x smaller than bf16) without
  * touching the backbone's KV cache. Here the selector's cache is the block
  * statistics; the format read from that passage: per (b, g, block) one record of
  * d + d/16 bytes,
- *   [0, d/2)        mean codes, two per byte (feature 2c in the low nibble),
- *                   signed 4-bit in [-7, 7]
- *   [d/2, d)        variance codes, unsigned 4-bit in [0, 15]
+ *   [0, d/2)        mean codes, two per byte (feature 2c in the low nibble)
+ *   [d/2, d)        variance codes
  *   [d, d + d/32)   mean scale exponents k, int8, one per 32 features
  *   [d + d/32, d + d/16)  variance scale exponents
- * where 2^k is the smallest power of two with max |mean| <= 7 * 2^k over the 32
- * features (variance: max var <= 15 * 2^k), k clamped to [-126, 126], and
- * code = round-half-even(x / 2^k); the value read back is code * 2^k, exactly.
- * 136 bytes per block at d = 128, against 1024 in fp32.
+ * fmt = SPA_QFMT_INT4: mean codes signed 4-bit in [-7, 7], variance codes unsigned
+ *   in [0, 15]; 2^k is the smallest power of two with max |mean| <= 7 * 2^k over the
+ *   32 features (variance: max var <= 15 * 2^k); code = round-half-even(x / 2^k);
+ *   the value read back is code * 2^k, exactly.
+ * fmt = SPA_QFMT_FP4: codes are FP4 E2M1 (the OCP microscaling element: bits
+ *   s e1 e0 m, magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6) for mean and variance; 2^k is
+ *   the smallest power of two with max |x| <= 6 * 2^k (no element saturates); code =
+ *   the E2M1 value nearest x / 2^k, ties to the even mantissa bit, with x's sign bit
+ *   (a negative value rounding to zero gives -0); read back as E2M1(code) * 2^k.
+ * Both: k clamped to [-126, 126]; decided on the fp32 statistics. 136 bytes per
+ * block at d = 128, against 1024 in fp32.
  *   mean, var : spa_block_stats output [B, Hkv, nb, d] fp32; d = 64 or 128
  *   blk_begin, blk_end : records [blk_begin, blk_end) are written (others untouched)
  *   qstats : [B, Hkv, nb] records, spa_quantized_stats_bytes(...) bytes, 16-byte aligned
  *            (that call returns 0 for sizes it does not support)
+ *   fmt    : the code format; any other value is SPA_ERR_INVALID
  */
 size_t spa_quantized_stats_bytes(int B, int Hkv, int T, int d, int block);
 spa_status spa_quantize_block_stats(const float *mean, const float *var, int B, int Hkv, int T,
                                     int d, int block, int blk_begin, int blk_end, void *qstats,
-                                    spa_stream stream);
+                                    spa_qformat fmt, spa_stream stream);
 
 /*
- * Block statistics and their INT4 records in one pass, for a few blocks (a decode
+ * Block statistics and their records in one pass, for a few blocks (a decode
  * step's newest block): for blocks [blk_begin, blk_end) of every (b, kv-head),
  * mean and var exactly as spa_block_stats defines them (fp32, population variance,
  * written into mean, var) and the record spa_quantize_block_stats makes of those
- * fp32 values (written into qstats). One warp per block reads the block's keys
- * twice (mean, then squared deviations); for a whole cache, spa_block_stats followed
- * by spa_quantize_block_stats is faster.
- *   k : [B, Hkv, T, d] (dt), d = 64 or 128; mean, var, qstats as in the two calls;
- *   blocks outside the range are left untouched. Errors as spa_block_stats.
+ * fp32 values in format fmt (written into qstats). One warp per block reads the
+ * block's keys twice (mean, then squared deviations); for a whole cache,
+ * spa_block_stats followed by spa_quantize_block_stats is faster.
+ *   k : [B, Hkv, T, d] (dt), d = 64 or 128; mean, var, qstats, fmt as in the two
+ *   calls; blocks outside the range are left untouched. Errors as spa_block_stats.
  */
 spa_status spa_block_stats_quantized(const void *k, spa_dtype dt, int B, int Hkv, int T, int d,
                                      int block, int blk_begin, int blk_end, float *mean,
-                                     float *var, void *qstats, spa_stream stream);
+                                     float *var, void *qstats, spa_qformat fmt, spa_stream stream);
 
 /*
  * spa_select on quantised statistics: the same score, cut and output, with each
- * block's mean and variance read back from its record (code * 2^k) instead of
- * from fp32 arrays. Arguments as spa_select, with qstats in place of mean, var.
+ * block's mean and variance read back from its record (the value of its code times
+ * 2^k, exactly) instead of from fp32 arrays. Arguments as spa_select, with qstats
+ * (records in format fmt) in place of mean, var.
  */
-spa_status spa_select_quantized(const void *q, spa_dtype dt, const void *qstats, int B, int Hq,
-                                int Hkv, int Lq, int T, int d, int block, float scale,
-                                float top_p, int n_sink, int n_local, int k_min, int32_t *idx,
-                                int cap, int32_t *count, spa_stream stream);
+spa_status spa_select_quantized(const void *q, spa_dtype dt, const void *qstats, spa_qformat fmt,
+                                int B, int Hq, int Hkv, int Lq, int T, int d, int block,
+                                float scale, float top_p, int n_sink, int n_local, int k_min,
+                                int32_t *idx, int cap, int32_t *count, spa_stream stream);
 
 /*
  * Block-sparse causal prefill attention. Follows "S2O", sections 1 and 3 (index-

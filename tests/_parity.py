@@ -104,32 +104,43 @@ def pack_qstats(qs: dict) -> np.ndarray:
     return rec
 
 
-def unpack_qstats(rec: np.ndarray, d: int) -> dict:
+def unpack_qstats(rec: np.ndarray, d: int, fmt: str = "int4") -> dict:
     rec = np.asarray(rec, np.uint8)
     lo_m, hi_m = rec[..., :d // 2] & 15, rec[..., :d // 2] >> 4
     lo_v, hi_v = rec[..., d // 2:d] & 15, rec[..., d // 2:d] >> 4
     cm = np.empty(rec.shape[:-1] + (d,), np.int16)
     cm[..., 0::2], cm[..., 1::2] = lo_m, hi_m
-    cm = np.where(cm >= 8, cm - 16, cm).astype(np.int8)
+    # INT4 mean codes are two's-complement nibbles; FP4 codes stay 4-bit patterns
+    cm = np.where(cm >= 8, cm - 16, cm).astype(np.int8) if fmt == "int4" else cm.astype(np.uint8)
     cv = np.empty(rec.shape[:-1] + (d,), np.uint8)
     cv[..., 0::2], cv[..., 1::2] = lo_v, hi_v
     return {"cm": cm, "cv": cv, "km": rec[..., d:d + d // 32].view(np.int8),
             "kv": rec[..., d + d // 32:].view(np.int8)}
 
 
+E2M1_MIDPOINTS = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+
+
 def quant_ambiguous(mean: np.ndarray, var: np.ndarray, qs: dict, rel: float = 1e-5) -> np.ndarray:
     """Per 32-feature group: True where the oracle's quantisation decision is a near
     tie for fp32 statistics that differ in rounding order: a value within `rel` of a
-    rounding boundary (a half step), or the group maximum within `rel` of a scale
+    rounding boundary (INT4: a half step; FP4: a midpoint of the E2M1 grid, or zero,
+    where the sign bit decides), or the group maximum within `rel` of a scale
     boundary. [B, Hkv, nb, d / 32], for mean or variance."""
+    fmt = qs.get("fmt", "int4")
+    tops = (7.0, 15.0) if fmt == "int4" else (6.0, 6.0)
     out = []
-    for x, k, top in ((np.abs(mean.astype(np.float32).astype(np.float64)), qs["km"], 7.0),
-                      (var.astype(np.float32).astype(np.float64), qs["kv"], 15.0)):
+    for x, k, top in ((np.abs(mean.astype(np.float32).astype(np.float64)), qs["km"], tops[0]),
+                      (var.astype(np.float32).astype(np.float64), qs["kv"], tops[1])):
         B, Hkv, nb, d = x.shape
         step = np.ldexp(1.0, k.astype(np.int64)).repeat(32, axis=-1)
         t = x / step
-        frac = np.abs(t - np.floor(t) - 0.5)
-        near_code = (frac <= rel * np.maximum(1.0, t)).reshape(B, Hkv, nb, d // 32, 32).any(-1)
+        tol = rel * np.maximum(1.0, t)
+        if fmt == "int4":
+            near = np.abs(t - np.floor(t) - 0.5) <= tol
+        else:
+            near = (np.abs(t[..., None] - E2M1_MIDPOINTS).min(-1) <= tol) | (t <= rel)
+        near_code = near.reshape(B, Hkv, nb, d // 32, 32).any(-1)
         amax = x.reshape(B, Hkv, nb, d // 32, 32).max(-1)
         kk = k.astype(np.int64)
         near_scale = ((np.abs(amax / (top * np.ldexp(1.0, kk)) - 1) <= rel) |

@@ -173,15 +173,21 @@ def test_quantized_stats_host_checks(lib):
     assert n(16, 8, 131072, 128, 16) == 16 * 8 * 8192 * 136
     assert n(1, 1, 100, 96, 16) == 0                                     # d % 32
     f = lib.spa_quantize_block_stats
-    f.argtypes = [P, P, I, I, I, I, I, I, I, P, P]
-    assert f(FAKE, FAKE, 1, 2, 256, 96, 16, 0, 16, FAKE, None) == 2       # d = 96
-    assert f(FAKE, FAKE, 1, 2, 256, 128, 16, 0, 17, FAKE, None) == 1      # beyond nb
-    assert f(FAKE, None, 1, 2, 256, 128, 16, 0, 16, FAKE, None) == 1
+    f.argtypes = [P, P, I, I, I, I, I, I, I, P, I, P]
+    assert f(FAKE, FAKE, 1, 2, 256, 96, 16, 0, 16, FAKE, 0, None) == 2    # d = 96
+    assert f(FAKE, FAKE, 1, 2, 256, 128, 16, 0, 17, FAKE, 1, None) == 1   # beyond nb
+    assert f(FAKE, None, 1, 2, 256, 128, 16, 0, 16, FAKE, 0, None) == 1
+    assert f(FAKE, FAKE, 1, 2, 256, 128, 16, 0, 16, FAKE, 2, None) == 1   # unknown format
+    h = lib.spa_block_stats_quantized
+    h.argtypes = [P, I, I, I, I, I, I, I, I, P, P, P, I, P]
+    assert h(FAKE, 1, 1, 2, 256, 128, 16, 0, 16, FAKE, FAKE, FAKE, 3, None) == 1   # unknown format
+    assert h(FAKE, 1, 1, 2, 256, 96, 16, 0, 16, FAKE, FAKE, FAKE, 1, None) == 2    # d = 96
     g = lib.spa_select_quantized
-    g.argtypes = [P, I, P, I, I, I, I, I, I, I, F, F, I, I, I, P, I, P, P]
-    assert g(FAKE, 1, FAKE, 1, 4, 2, 1, 256, 128, 16, 0.1, 0.9, 1, 1, 0, FAKE, 15, FAKE, None) == 1
-    assert g(FAKE, 1, FAKE, 1, 4, 2, 1, 256, 96, 16, 0.1, 0.9, 1, 1, 0, FAKE, 16, FAKE, None) == 2
-    assert g(FAKE, 1, None, 1, 4, 2, 1, 256, 128, 16, 0.1, 0.9, 1, 1, 0, FAKE, 16, FAKE, None) == 1
+    g.argtypes = [P, I, P, I, I, I, I, I, I, I, I, F, F, I, I, I, P, I, P, P]
+    assert g(FAKE, 1, FAKE, 0, 1, 4, 2, 1, 256, 128, 16, 0.1, 0.9, 1, 1, 0, FAKE, 15, FAKE, None) == 1
+    assert g(FAKE, 1, FAKE, 1, 1, 4, 2, 1, 256, 96, 16, 0.1, 0.9, 1, 1, 0, FAKE, 16, FAKE, None) == 2
+    assert g(FAKE, 1, None, 0, 1, 4, 2, 1, 256, 128, 16, 0.1, 0.9, 1, 1, 0, FAKE, 16, FAKE, None) == 1
+    assert g(FAKE, 1, FAKE, -1, 1, 4, 2, 1, 256, 128, 16, 0.1, 0.9, 1, 1, 0, FAKE, 16, FAKE, None) == 1
 
 
 def test_early_stop_host_checks(lib):

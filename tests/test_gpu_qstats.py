@@ -1,5 +1,5 @@
-"""Parity of the quantised block statistics ("SpotAttention", section 4; INT4
-microscale as read, format in include/spa.h) with the CPU oracle.
+"""Parity of the quantised block statistics ("SpotAttention", section 4; INT4 and
+FP4 (E2M1) microscale as read, format in include/spa.h) with the CPU oracle.
 
 The quantiser is checked against the oracle's codes: they must be equal except in
 groups where the oracle flags its own decision as a near tie (a value within 1e-5
@@ -31,41 +31,47 @@ def inputs(w):
     return _cache[key]
 
 
+FMTS = ["int4", "fp4"]
+
+
+@pytest.mark.parametrize("fmt", FMTS)
 @pytest.mark.parametrize("key", list(PARITY_WORKLOADS))
-def test_quantizer_matches_oracle_codes(key):
+def test_quantizer_matches_oracle_codes(key, fmt):
     w = PARITY_WORKLOADS[key]
     x, dev = inputs(w)
     mean, var = spa.spa_block_stats(dev["k"], w.block)
-    rec = spa.spa_quantize_block_stats(mean, var, w.T, w.block)
+    rec = spa.spa_quantize_block_stats(mean, var, w.T, w.block, fmt=fmt)
     torch.cuda.synchronize()
-    g = unpack_qstats(rec.cpu().numpy(), w.d)
+    g = unpack_qstats(rec.cpu().numpy(), w.d, fmt)
     om, ov = oracle.block_stats(x["k"], w.dtype, w.block)
-    o = oracle.quantize_stats(om, ov)
+    o = oracle.quantize_stats(om, ov, fmt)
     amb = quant_ambiguous(om, ov, o)
     grp = lambda a: a.reshape(a.shape[:-1] + (w.d // 32, 32))
     diff = ((grp(g["cm"]) != grp(o["cm"])).any(-1) | (grp(g["cv"]) != grp(o["cv"])).any(-1) |
             (g["km"] != o["km"]) | (g["kv"] != o["kv"]))
-    print(f"\n{w.name}: {int(diff.sum())} of {diff.size} groups differ, "
+    print(f"\n{w.name} {fmt}: {int(diff.sum())} of {diff.size} groups differ, "
           f"{int(amb.sum())} near ties flagged")
     assert not (diff & ~amb).any()
     assert rec.numel() == spa.spa_quantized_stats_bytes(w.B, w.Hkv, w.T, w.d, w.block)
 
 
-def test_quantizer_range_leaves_others_untouched():
+@pytest.mark.parametrize("fmt", FMTS)
+def test_quantizer_range_leaves_others_untouched(fmt):
     w = PARITY_WORKLOADS["d_bf16_blk16"]
     x, dev = inputs(w)
     mean, var = spa.spa_block_stats(dev["k"], w.block)
     rec = torch.full((w.B, w.Hkv, w.nb, w.d + w.d // 16), 0xAB, device="cuda", dtype=torch.uint8)
-    spa.spa_quantize_block_stats(mean, var, w.T, w.block, w.nb - 3, w.nb, qstats=rec)
+    spa.spa_quantize_block_stats(mean, var, w.T, w.block, w.nb - 3, w.nb, qstats=rec, fmt=fmt)
     torch.cuda.synchronize()
     r = rec.cpu().numpy()
     assert np.all(r[:, :, :w.nb - 3] == 0xAB)
-    full = spa.spa_quantize_block_stats(mean, var, w.T, w.block).cpu().numpy()
+    full = spa.spa_quantize_block_stats(mean, var, w.T, w.block, fmt=fmt).cpu().numpy()
     assert np.array_equal(r[:, :, w.nb - 3:], full[:, :, w.nb - 3:])
 
 
+@pytest.mark.parametrize("fmt", FMTS)
 @pytest.mark.parametrize("key", ["d_bf16_blk16", "d_bf16_blk64", "p_f32_d64", "p_bf16_blk128"])
-def test_fused_stats_and_records_of_a_block_range(key):
+def test_fused_stats_and_records_of_a_block_range(key, fmt):
     # spa_block_stats_quantized on the last blocks (a decode step's update): its
     # statistics match the oracle's, its records are exactly the oracle's quantiser
     # applied to those fp32 statistics, and blocks outside the range are untouched
@@ -76,27 +82,28 @@ def test_fused_stats_and_records_of_a_block_range(key):
     mean = torch.full((w.B, w.Hkv, nb, w.d), 7.0, device="cuda")
     var = torch.full_like(mean, 7.0)
     rec = torch.full((w.B, w.Hkv, nb, w.d + w.d // 16), 0xAB, device="cuda", dtype=torch.uint8)
-    spa.spa_block_stats_quantized(dev["k"], w.block, lo, nb, mean, var, rec)
+    spa.spa_block_stats_quantized(dev["k"], w.block, lo, nb, mean, var, rec, fmt=fmt)
     torch.cuda.synchronize()
     om, ov = oracle.block_stats(x["k"], w.dtype, w.block)
     m, v, r = mean.cpu().numpy(), var.cpu().numpy(), rec.cpu().numpy()
     np.testing.assert_allclose(m[:, :, lo:], om[:, :, lo:], rtol=1e-5, atol=1e-6)
     np.testing.assert_allclose(v[:, :, lo:], ov[:, :, lo:], rtol=1e-5, atol=1e-6)
     assert np.all(m[:, :, :lo] == 7.0) and np.all(r[:, :, :lo] == 0xAB)
-    o = oracle.quantize_stats(m[:, :, lo:].astype(np.float64), v[:, :, lo:].astype(np.float64))
+    o = oracle.quantize_stats(m[:, :, lo:].astype(np.float64), v[:, :, lo:].astype(np.float64), fmt)
     assert np.array_equal(r[:, :, lo:], pack_qstats(o))
     assert spa.spa_get_device_error() == 0
 
 
+@pytest.mark.parametrize("fmt", FMTS)
 @pytest.mark.parametrize("key", list(PARITY_WORKLOADS))
-def test_select_quantized_on_oracle_records(key):
+def test_select_quantized_on_oracle_records(key, fmt):
     w = PARITY_WORKLOADS[key]
     x, dev = inputs(w)
     sel = oracle.select_quantized(x["q"], x["k"], w.dtype, w.block, w.scale, w.top_p, w.n_sink,
-                                  w.n_local, w.k_min)
+                                  w.n_local, w.k_min, fmt)
     rec = torch.from_numpy(pack_qstats(sel["q"])).cuda()
     idx, cnt = spa.spa_select_quantized(dev["q"], rec, w.T, w.block, w.scale, w.top_p, w.n_sink,
-                                        w.n_local, w.k_min)
+                                        w.n_local, w.k_min, fmt=fmt)
     torch.cuda.synchronize()
     r = compare_lists(idx.cpu().numpy(), cnt.cpu().numpy(), sel["idx"], sel["count"],
                       sel["scores"], w.top_p, w.n_sink, w.n_local, w.Lq, w.T, w.block)
@@ -105,18 +112,19 @@ def test_select_quantized_on_oracle_records(key):
     assert spa.spa_get_device_error() == 0
 
 
+@pytest.mark.parametrize("fmt", FMTS)
 @pytest.mark.parametrize("Hq,Hkv", [(2, 2), (4, 2), (8, 1), (16, 2)])
-def test_select_quantized_decode_head_groupings(Hq, Hkv):
+def test_select_quantized_decode_head_groupings(Hq, Hkv, fmt):
     # decode scoring on records runs on the tensor cores with the group's heads as
     # the MMA columns: one, two, eight (all columns) and eight heads per kv-head
     # (the four-head case is the parity workload above); a ragged candidate tile
     w = PARITY_WORKLOADS["d_bf16_blk16"].with_(Hq=Hq, Hkv=Hkv, T=16 * 300 + 5)
     x, dev = inputs(w)
     sel = oracle.select_quantized(x["q"], x["k"], w.dtype, w.block, w.scale, w.top_p, w.n_sink,
-                                  w.n_local, w.k_min)
+                                  w.n_local, w.k_min, fmt)
     rec = torch.from_numpy(pack_qstats(sel["q"])).cuda()
     idx, cnt = spa.spa_select_quantized(dev["q"], rec, w.T, w.block, w.scale, w.top_p, w.n_sink,
-                                        w.n_local, w.k_min)
+                                        w.n_local, w.k_min, fmt=fmt)
     torch.cuda.synchronize()
     r = compare_lists(idx.cpu().numpy(), cnt.cpu().numpy(), sel["idx"], sel["count"],
                       sel["scores"], w.top_p, w.n_sink, w.n_local, w.Lq, w.T, w.block)
@@ -125,15 +133,16 @@ def test_select_quantized_decode_head_groupings(Hq, Hkv):
     assert spa.spa_get_device_error() == 0
 
 
-def test_select_quantized_rule_variants():
+@pytest.mark.parametrize("fmt", FMTS)
+def test_select_quantized_rule_variants(fmt):
     w = PARITY_WORKLOADS["d_bf16_blk16"]
     x, dev = inputs(w)
     for top_p, k_min in ((0.3, 0), (0.5, 20), (1.0, 0)):
         sel = oracle.select_quantized(x["q"], x["k"], w.dtype, w.block, w.scale, top_p, w.n_sink,
-                                      w.n_local, k_min)
+                                      w.n_local, k_min, fmt)
         rec = torch.from_numpy(pack_qstats(sel["q"])).cuda()
         idx, cnt = spa.spa_select_quantized(dev["q"], rec, w.T, w.block, w.scale, top_p,
-                                            w.n_sink, w.n_local, k_min)
+                                            w.n_sink, w.n_local, k_min, fmt=fmt)
         torch.cuda.synchronize()
         r = compare_lists(idx.cpu().numpy(), cnt.cpu().numpy(), sel["idx"], sel["count"],
                           sel["scores"], top_p, w.n_sink, w.n_local, 1, w.T, w.block)
@@ -141,13 +150,14 @@ def test_select_quantized_rule_variants():
 
 
 @pytest.mark.slow
-def test_select_quantized_decode_workload_full_size():
+@pytest.mark.parametrize("fmt", FMTS)
+def test_select_quantized_decode_workload_full_size(fmt):
     w = WORKLOADS[5]
     x = generate(w)
     q = to_dev(x["q"], w.dtype)
-    sel = oracle.select_quantized(x["q"], x["k"], w.dtype, w.block, w.scale, w.top_p)
+    sel = oracle.select_quantized(x["q"], x["k"], w.dtype, w.block, w.scale, w.top_p, fmt=fmt)
     rec = torch.from_numpy(pack_qstats(sel["q"])).cuda()
-    idx, cnt = spa.spa_select_quantized(q, rec, w.T, w.block, w.scale, w.top_p)
+    idx, cnt = spa.spa_select_quantized(q, rec, w.T, w.block, w.scale, w.top_p, fmt=fmt)
     torch.cuda.synchronize()
     r = compare_lists(idx.cpu().numpy(), cnt.cpu().numpy(), sel["idx"], sel["count"],
                       sel["scores"], w.top_p, w.n_sink, w.n_local, 1, w.T, w.block)
@@ -156,7 +166,7 @@ def test_select_quantized_decode_workload_full_size():
     for u, c in np.ndenumerate(plain["count"]):
         a_, b_ = set(plain["idx"][u][:c].tolist()), set(sel["idx"][u][:sel["count"][u]].tolist())
         overlap.append(len(a_ & b_) / len(a_ | b_))
-    print(f"\n{w.name}: {r['units']} lists, {r['equal']} equal, {r['excused']} excused; "
+    print(f"\n{w.name} {fmt}: {r['units']} lists, {r['equal']} equal, {r['excused']} excused; "
           f"kept fraction {sel['count'].mean() / w.nb:.3f} (fp32 statistics "
           f"{plain['count'].mean() / w.nb:.3f}); mean Jaccard overlap with the fp32 "
           f"selection {np.mean(overlap):.4f}")
