@@ -8,7 +8,12 @@
 // Three streams per device carry the work: h2d copies a chunk's q, k, v into a
 // workspace slot, comp runs the three kernels of the chunk in that slot, d2h copies
 // the slot's output back. With three slots, chunk c+1 arrives, chunk c computes and
-// chunk c-1 leaves at the same time; events order each slot's reuse.
+// chunk c-1 leaves at the same time; events order each slot's reuse. The last chunk
+// is what the pipeline drains on: when it is one pair whose query heads split into
+// two halves the attention kernel takes as they are, its attention runs as two
+// launches (one per half) and the first half's output is copied back while the
+// second half computes. The selection still runs once over all the pair's heads,
+// so every kernel sees exactly what it sees on the device-resident path.
 #include <stdio.h>
 
 #include <mutex>
@@ -103,7 +108,7 @@ Layout layout(spa_dtype dt, int B, int Hq, int Hkv, int L, int d, int block) {
 struct Pipe {
     cudaStream_t h2d = nullptr, comp = nullptr, d2h = nullptr;
     cudaEvent_t start = nullptr, join[3] = {}, in[kSlots] = {}, done[kSlots] = {},
-                freed[kSlots] = {};
+                freed[kSlots] = {}, half = nullptr;
 };
 
 std::mutex g_pipe_mu;
@@ -112,9 +117,9 @@ Pipe *g_pipe[64];
 void destroy_pipe(Pipe *p) {
     for (cudaStream_t st : {p->h2d, p->comp, p->d2h})
         if (st) cudaStreamDestroy(st);
-    cudaEvent_t *groups[] = {&p->start, p->join, p->in, p->done, p->freed};
-    const int sizes[] = {1, 3, kSlots, kSlots, kSlots};
-    for (int g = 0; g < 5; ++g)
+    cudaEvent_t *groups[] = {&p->start, p->join, p->in, p->done, p->freed, &p->half};
+    const int sizes[] = {1, 3, kSlots, kSlots, kSlots, 1};
+    for (int g = 0; g < 6; ++g)
         for (int i = 0; i < sizes[g]; ++i)
             if (groups[g][i]) cudaEventDestroy(groups[g][i]);
     delete p;
@@ -134,6 +139,7 @@ cudaError_t get_pipe(Pipe **out) {
         if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&p->comp, sf);
         if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&p->d2h, sf);
         if (e == cudaSuccess) e = cudaEventCreateWithFlags(&p->start, ef);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&p->half, ef);
         for (int i = 0; i < 3 && e == cudaSuccess; ++i) e = cudaEventCreateWithFlags(&p->join[i], ef);
         for (int s = 0; s < kSlots && e == cudaSuccess; ++s) {
             e = cudaEventCreateWithFlags(&p->in[s], ef);
@@ -232,16 +238,35 @@ SPA_API spa_status spa_prefill_host(const void *q, const void *k, const void *v,
         if (st == SPA_OK)
             st = spa_select(qd, dt, mean, var, n, y.G, 1, L, L, d, block, scale, top_p, n_sink,
                             n_local, k_min, idx, cap, cnt, p.comp);
-        if (st == SPA_OK)
+        // the last chunk: one pair whose heads halve into whole attention tiles
+        const int hpt = dt == SPA_BF16 ? 128 / block : 1;   // heads per attention tile
+        const bool halves = c == y.chunks - 1 && n == 1 && y.G % (2 * hpt) == 0;
+        const size_t hq = halves ? (size_t)(y.G / 2) * L * d * y.es : 0;   // bytes of half the heads
+        if (st == SPA_OK && halves) {
+            const size_t hl = (size_t)(y.G / 2) * y.nq;                       // lists per half
+            st = spa_sparse_attn_prefill(qd, kd, vd, dt, 1, y.G / 2, 1, L, d, block, idx, cap,
+                                         cnt, scale, od, nullptr, p.comp);
+            if (st == SPA_OK &&
+                ((e = cudaEventRecord(p.half, p.comp)) != cudaSuccess ||
+                 (e = cudaStreamWaitEvent(p.d2h, p.half, 0)) != cudaSuccess ||
+                 (e = cudaMemcpyAsync(oh + (size_t)u0 * y.q_unit, od, hq, cudaMemcpyDeviceToHost,
+                                      p.d2h)) != cudaSuccess))
+                break;
+            if (st == SPA_OK)
+                st = spa_sparse_attn_prefill(qd + hq, kd, vd, dt, 1, y.G / 2, 1, L, d, block,
+                                             idx + hl * cap, cap, cnt + hl, scale, od + hq,
+                                             nullptr, p.comp);
+        } else if (st == SPA_OK) {
             st = spa_sparse_attn_prefill(qd, kd, vd, dt, n, y.G, 1, L, d, block, idx, cap, cnt,
                                          scale, od, nullptr, p.comp);
+        }
         if (st != SPA_OK) {
             join(p, caller);
             return st;
         }
         if ((e = cudaEventRecord(p.done[s], p.comp)) != cudaSuccess ||
             (e = cudaStreamWaitEvent(p.d2h, p.done[s], 0)) != cudaSuccess ||
-            (e = cudaMemcpyAsync(oh + (size_t)u0 * y.q_unit, od, (size_t)n * y.q_unit,
+            (e = cudaMemcpyAsync(oh + (size_t)u0 * y.q_unit + hq, od + hq, (size_t)n * y.q_unit - hq,
                                  cudaMemcpyDeviceToHost, p.d2h)) != cudaSuccess ||
             (e = cudaEventRecord(p.freed[s], p.d2h)) != cudaSuccess)
             break;
