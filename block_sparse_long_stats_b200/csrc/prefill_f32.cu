@@ -3,12 +3,18 @@
 // index ("coordinate-scheduled loading", section 1) and folded into an online
 // softmax state (m, l, acc) per query row.
 //
-// One warp per query row: the row's query sits in every lane's registers; the
-// kept blocks are walked 32 keys at a time, lane l scoring key l of the chunk with
-// a full dot product (16-byte loads of its key row); the warp takes the chunk's
-// maximum and sum with shuffles, then folds the 32 values into the output, lane l
-// owning d/32 output columns (the values' rows read 16 or 8 bytes per lane,
-// coalesced across the warp). Eight warps (rows) per CTA.
+// One CTA of eight warps per query row (rows in reverse order, so the rows with the
+// most kept blocks start first). Warp 0 first validates the row's kept list into
+// shared memory (entries outside [0, i] or not ascending are dropped and reported;
+// an entry is valid when it lies in range and exceeds every earlier in-range entry,
+// so a warp prefix maximum decides 32 entries at once). The warps then take the
+// valid blocks round robin, each keeping its own online-softmax state: the row's
+// query pre-scaled in every lane's registers, 32 keys at a time (lane per key, a
+// full dot product from 16-byte loads of its key row), the chunk's maximum and sum
+// by shuffles, then the 32 value rows folded into the output (lane l owning d/32
+// output columns). The eight states (m, l, acc) merge in shared memory at the end.
+// A single warp per row left the short launch bound by one row's chain of dependent
+// L2 round trips; eight split it eightfold.
 #include <math.h>
 
 #include "kernels.h"
@@ -16,7 +22,7 @@
 namespace spa {
 namespace {
 
-constexpr int kWarpsF32 = 8;
+constexpr int kWarpsF32 = 8;   // warps per row
 
 template <int D>
 __global__ void __launch_bounds__(32 * kWarpsF32) prefill_f32_kernel(
@@ -25,13 +31,49 @@ __global__ void __launch_bounds__(32 * kWarpsF32) prefill_f32_kernel(
     const int32_t *__restrict__ count, float scale, float *__restrict__ out,
     float *__restrict__ lse, int *err) {
     constexpr int DL = D / 32;                 // output columns per lane
+    extern __shared__ int32_t valid_list[];    // the row's valid kept blocks, ascending
+    __shared__ float sm_m[kWarpsF32], sm_l[kWarpsF32];
+    __shared__ float sm_acc[kWarpsF32][D];
+    __shared__ int n_valid;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    // rows in reverse order, so the longest rows (the most kept blocks) start first
-    const int t = L - 1 - ((int)blockIdx.x * kWarpsF32 + warp);
-    if (t < 0) return;
+    const int t = L - 1 - (int)blockIdx.x;
     const int bh = blockIdx.y;
     const int b = bh / Hq, h = bh % Hq, g = h / (Hq / Hkv);
     const int i = t / block;
+    const size_t unit = (size_t)bh * nq + i;
+
+    if (warp == 0) {
+        int cnt = __ldg(count + unit);
+        if (cnt < 0 || cnt > cap) {
+            if (lane == 0) set_error(err, SPA_DEVERR_BAD_COUNT);
+            cnt = cnt < 0 ? 0 : cap;
+        }
+        const int32_t *list = idx + unit * cap;
+        int carry = -1, nv = 0;                // largest in-range entry so far
+        bool bad = false;
+        for (int base = 0; base < cnt; base += 32) {
+            const int e = base + lane;
+            const int j = e < cnt ? __ldg(list + e) : -1;
+            const bool in_range = e < cnt && j >= 0 && j <= i;
+            // largest in-range entry among the earlier lanes of this chunk
+            int pm = in_range ? j : -1;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, pm, o);
+                if (lane >= o) pm = max(pm, y);
+            }
+            int before = __shfl_up_sync(0xffffffffu, pm, 1);
+            before = max(carry, lane == 0 ? -1 : before);
+            const bool ok = in_range && j > before;
+            if (e < cnt && !ok) bad = true;
+            const unsigned bal = __ballot_sync(0xffffffffu, ok);
+            if (ok) valid_list[nv + __popc(bal & ((1u << lane) - 1u))] = j;
+            nv += __popc(bal);
+            carry = max(carry, __shfl_sync(0xffffffffu, pm, 31));
+        }
+        if (__any_sync(0xffffffffu, bad) && lane == 0) set_error(err, SPA_DEVERR_BAD_INDEX);
+        if (lane == 0) n_valid = nv;
+    }
 
     float qr[D];
     const float4 *q4 = reinterpret_cast<const float4 *>(q + ((size_t)bh * L + t) * D);
@@ -47,24 +89,12 @@ __global__ void __launch_bounds__(32 * kWarpsF32) prefill_f32_kernel(
     float acc[DL];
 #pragma unroll
     for (int c = 0; c < DL; ++c) acc[c] = 0.f;
-
-    const size_t unit = (size_t)bh * nq + i;
-    int cnt = __ldg(count + unit);
-    if (cnt < 0 || cnt > cap) {
-        if (lane == 0) set_error(err, SPA_DEVERR_BAD_COUNT);
-        cnt = cnt < 0 ? 0 : cap;
-    }
-    const int32_t *list = idx + unit * cap;
+    __syncthreads();
+    const int nv = n_valid;
     const float *kb = k + ((size_t)b * Hkv + g) * L * D;
     const float *vb = v + ((size_t)b * Hkv + g) * L * D;
-    int last = -1;
-    for (int n = 0; n < cnt; ++n) {
-        const int j = __ldg(list + n);
-        if (j <= last || j > i) {          // out of range or not ascending: skip
-            if (lane == 0) set_error(err, SPA_DEVERR_BAD_INDEX);
-            continue;
-        }
-        last = j;
+    for (int n = warp; n < nv; n += kWarpsF32) {
+        const int j = valid_list[n];
         const int kend = min(min((j + 1) * block, L), t + 1);   // keys [j block, kend)
         for (int key0 = j * block; key0 < kend; key0 += 32) {
             const int u = key0 + lane;
@@ -86,7 +116,7 @@ __global__ void __launch_bounds__(32 * kWarpsF32) prefill_f32_kernel(
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
             const float m_new = fmaxf(m, mx);           // finite: key j * block <= t is in the chunk
-            const float alpha = expf(m - m_new);        // 0 on the row's first chunk
+            const float alpha = expf(m - m_new);        // 0 on the warp's first chunk
             const float p = expf(s - m_new);            // 0 for the masked lanes
             float ps = p;
 #pragma unroll
@@ -118,11 +148,32 @@ __global__ void __launch_bounds__(32 * kWarpsF32) prefill_f32_kernel(
             }
         }
     }
-    const float inv = l > 0.f ? 1.f / l : 0.f;
-    float *o = out + ((size_t)bh * L + t) * D + lane * DL;
+    // merge the warps' states: M = max m_w, l = sum l_w e^(m_w - M), acc likewise
+    if (lane == 0) {
+        sm_m[warp] = m;
+        sm_l[warp] = l;
+    }
 #pragma unroll
-    for (int c = 0; c < DL; ++c) o[c] = acc[c] * inv;
-    if (lse && lane == 0) lse[(size_t)bh * L + t] = l > 0.f ? m + logf(l) : -INFINITY;
+    for (int c = 0; c < DL; ++c) sm_acc[warp][lane * DL + c] = acc[c];
+    __syncthreads();
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kWarpsF32; ++w) M = fmaxf(M, sm_m[w]);
+    float wgt[kWarpsF32], ls = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWarpsF32; ++w) {
+        wgt[w] = sm_l[w] > 0.f ? expf(sm_m[w] - M) : 0.f;   // a warp with no keys adds 0
+        ls = fmaf(sm_l[w], wgt[w], ls);
+    }
+    const float inv = ls > 0.f ? 1.f / ls : 0.f;
+    float *o = out + ((size_t)bh * L + t) * D;
+    for (int col = threadIdx.x; col < D; col += 32 * kWarpsF32) {
+        float a = 0.f;
+#pragma unroll
+        for (int w = 0; w < kWarpsF32; ++w) a = fmaf(sm_acc[w][col], wgt[w], a);
+        o[col] = a * inv;
+    }
+    if (lse && threadIdx.x == 0) lse[(size_t)bh * L + t] = ls > 0.f ? M + logf(ls) : -INFINITY;
 }
 
 }  // namespace
@@ -132,13 +183,22 @@ cudaError_t launch_prefill_f32(const float *q, const float *k, const float *v, i
                                const int32_t *count, float scale, float *out, float *lse,
                                int *err, cudaStream_t s) {
     const int nq = (L + block - 1) / block;
-    dim3 grid((unsigned)((L + kWarpsF32 - 1) / kWarpsF32), (unsigned)(B * Hq));
-    if (d == 64)
-        prefill_f32_kernel<64><<<grid, 32 * kWarpsF32, 0, s>>>(q, k, v, Hq, Hkv, L, block, nq, idx,
-                                                               cap, count, scale, out, lse, err);
-    else
-        prefill_f32_kernel<128><<<grid, 32 * kWarpsF32, 0, s>>>(q, k, v, Hq, Hkv, L, block, nq, idx,
-                                                                cap, count, scale, out, lse, err);
+    const size_t smem = (size_t)nq * sizeof(int32_t);   // the validated list (at most i + 1 <= nq)
+    dim3 grid((unsigned)L, (unsigned)(B * Hq));
+    cudaError_t e;
+    if (d == 64) {
+        if ((e = cudaFuncSetAttribute(prefill_f32_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)smem)) != cudaSuccess)
+            return e;
+        prefill_f32_kernel<64><<<grid, 32 * kWarpsF32, smem, s>>>(q, k, v, Hq, Hkv, L, block, nq, idx,
+                                                                  cap, count, scale, out, lse, err);
+    } else {
+        if ((e = cudaFuncSetAttribute(prefill_f32_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)smem)) != cudaSuccess)
+            return e;
+        prefill_f32_kernel<128><<<grid, 32 * kWarpsF32, smem, s>>>(q, k, v, Hq, Hkv, L, block, nq, idx,
+                                                                   cap, count, scale, out, lse, err);
+    }
     return cudaGetLastError();
 }
 
