@@ -9,7 +9,8 @@
 // an entry is valid when it lies in range and exceeds every earlier in-range entry,
 // so a warp prefix maximum decides 32 entries at once). The warps then take the
 // valid blocks round robin, each keeping its own online-softmax state: the row's
-// query pre-scaled in every lane's registers, 32 keys at a time (lane per key, a
+// query pre-scaled in shared memory (read as broadcasts, which keeps a thread at
+// 64 registers and four CTAs on an SM at d = 64), 32 keys at a time (lane per key, a
 // full dot product from 16-byte loads of its key row), the chunk's maximum and sum
 // by shuffles, then the 32 value rows folded into the output (lane l owning d/32
 // output columns). The eight states (m, l, acc) merge in shared memory at the end.
@@ -25,7 +26,7 @@ namespace {
 constexpr int kWarpsF32 = 8;   // warps per row
 
 template <int D>
-__global__ void __launch_bounds__(32 * kWarpsF32) prefill_f32_kernel(
+__global__ void __launch_bounds__(32 * kWarpsF32, D == 64 ? 4 : 2) prefill_f32_kernel(
     const float *__restrict__ q, const float *__restrict__ k, const float *__restrict__ v, int Hq,
     int Hkv, int L, int block, int nq, const int32_t *__restrict__ idx, int cap,
     const int32_t *__restrict__ count, float scale, float *__restrict__ out,
@@ -34,6 +35,7 @@ __global__ void __launch_bounds__(32 * kWarpsF32) prefill_f32_kernel(
     extern __shared__ int32_t valid_list[];    // the row's valid kept blocks, ascending
     __shared__ float sm_m[kWarpsF32], sm_l[kWarpsF32];
     __shared__ float sm_acc[kWarpsF32][D];
+    __shared__ __align__(16) float qs[D];      // the row's query, pre-scaled
     __shared__ int n_valid;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int t = L - 1 - (int)blockIdx.x;
@@ -75,16 +77,8 @@ __global__ void __launch_bounds__(32 * kWarpsF32) prefill_f32_kernel(
         if (lane == 0) n_valid = nv;
     }
 
-    float qr[D];
-    const float4 *q4 = reinterpret_cast<const float4 *>(q + ((size_t)bh * L + t) * D);
-#pragma unroll
-    for (int c = 0; c < D / 4; ++c) {
-        const float4 x = __ldg(q4 + c);
-        qr[4 * c] = x.x * scale;
-        qr[4 * c + 1] = x.y * scale;
-        qr[4 * c + 2] = x.z * scale;
-        qr[4 * c + 3] = x.w * scale;
-    }
+    if (threadIdx.x < D) qs[threadIdx.x] = __ldg(q + ((size_t)bh * L + t) * D + threadIdx.x) * scale;
+    const float4 *qs4 = reinterpret_cast<const float4 *>(qs);
     float m = -INFINITY, l = 0.f;
     float acc[DL];
 #pragma unroll
@@ -105,10 +99,11 @@ __global__ void __launch_bounds__(32 * kWarpsF32) prefill_f32_kernel(
 #pragma unroll
                 for (int c = 0; c < D / 4; ++c) {
                     const float4 x = __ldg(k4 + c);
-                    d0 = fmaf(qr[4 * c], x.x, d0);
-                    d1 = fmaf(qr[4 * c + 1], x.y, d1);
-                    d2 = fmaf(qr[4 * c + 2], x.z, d2);
-                    d3 = fmaf(qr[4 * c + 3], x.w, d3);
+                    const float4 y = qs4[c];           // the same address in every lane
+                    d0 = fmaf(y.x, x.x, d0);
+                    d1 = fmaf(y.y, x.y, d1);
+                    d2 = fmaf(y.z, x.z, d2);
+                    d3 = fmaf(y.w, x.w, d3);
                 }
                 s = (d0 + d1) + (d2 + d3);
             }
