@@ -301,20 +301,35 @@ def test_timeout_ends_only_its_own_launch():
     assert spa.spa_get_device_error() == 0
 
 
-def test_corrupt_lists_are_reported_and_skipped():
-    w = PARITY_WORKLOADS["p_bf16_blk128"]
+def _valid_entries(lst, i):
+    """The list as the kernels walk it: an entry is kept when it lies in [0, i] and
+    exceeds the last kept entry; the rest are skipped (and reported)."""
+    out, last = [], -1
+    for j in lst:
+        if 0 <= j <= i and j > last:
+            out.append(j)
+            last = j
+    return out
+
+
+@pytest.mark.parametrize("key", ["p_bf16_blk128", "p_f32_d64"])
+def test_corrupt_lists_are_reported_and_skipped(key):
+    w = PARITY_WORKLOADS[key]
     x, dev = inputs(w)
     sel = oracle_select(w, x)
     idx = sel["idx"].copy()
     cnt = sel["count"].copy()
     idx[0, 0, 5, 1] = 7          # beyond the causal limit of query block 5: skipped
     idx[0, 1, 6, 2] = 0          # not ascending: skipped
-    ref_idx, ref_cnt = sel["idx"].copy(), sel["count"].copy()
-    for (b, h, i, p) in [(0, 0, 5, 1), (0, 1, 6, 2)]:
-        keep = [j for j in ref_idx[b, h, i, :ref_cnt[b, h, i]].tolist()
-                if j != sel["idx"][b, h, i, p]]
-        ref_idx[b, h, i, :len(keep)] = keep
-        ref_cnt[b, h, i] = len(keep)
+    # a longer mix on the last query block: out of range, repeats, a step back
+    last_i = w.nq - 1
+    idx[0, 0, last_i, :8] = [0, 3, last_i + 40, 5, 5, 4, -3, 6]
+    cnt[0, 0, last_i] = 8
+    ref_idx, ref_cnt = np.full_like(idx, -1), cnt.copy()
+    for u, c in np.ndenumerate(cnt):
+        keep = _valid_entries(idx[u][:c].tolist(), u[2])
+        ref_idx[u][:len(keep)] = keep
+        ref_cnt[u] = len(keep)
     out, _ = spa.spa_sparse_attn_prefill(dev["q"], dev["k"], dev["v"], w.block,
                                          torch.from_numpy(idx).cuda(),
                                          torch.from_numpy(cnt).cuda(), w.scale)
@@ -323,12 +338,31 @@ def test_corrupt_lists_are_reported_and_skipped():
                                 w.scale)
     assert np.abs(to_host(out) - o_out).max() <= TOL[w.dtype]
     cnt2 = sel["count"].copy()
-    cnt2[1, 3, 2] = w.nb + 5     # count beyond cap: clamped
+    cnt2[w.B - 1, w.Hq - 1, 2] = w.nb + 5       # count beyond cap: clamped
     spa.spa_sparse_attn_prefill(dev["q"], dev["k"], dev["v"], w.block,
                                 torch.from_numpy(sel["idx"]).cuda(),
                                 torch.from_numpy(cnt2).cuda(), w.scale)
     assert spa.spa_get_device_error() == 2      # SPA_DEVERR_BAD_COUNT
     assert spa.spa_get_device_error() == 0      # reading clears it
+
+
+@pytest.mark.parametrize("block", [64, 128])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_block_stats_of_a_block_range_equal_the_full_launch(block, dtype):
+    # a sub-range [blk_begin, blk_end) of blocks of 64+ keys (the one-warp-per-block
+    # kernel) writes exactly what the full launch writes there, and nothing else
+    rng = np.random.default_rng(block + (dtype == "bf16"))
+    T = 9 * block + 17
+    k = rng.standard_normal((2, 3, T, 128)) * 1.5 + 0.25
+    kd = to_dev(bf16_bits(k) if dtype == "bf16" else k.astype(np.float32), dtype)
+    full_m, full_v = spa.spa_block_stats(kd, block)
+    nb = full_m.shape[2]
+    m = torch.full_like(full_m, 7.0)
+    v = torch.full_like(full_v, 7.0)
+    spa.spa_block_stats(kd, block, 3, nb, mean=m, var=v)
+    torch.cuda.synchronize()
+    assert torch.equal(m[:, :, 3:], full_m[:, :, 3:]) and torch.equal(v[:, :, 3:], full_v[:, :, 3:])
+    assert torch.all(m[:, :, :3] == 7.0) and torch.all(v[:, :, :3] == 7.0)
 
 
 # ------------------------------------------------------------------ headline workloads
