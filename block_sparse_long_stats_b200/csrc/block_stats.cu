@@ -3,16 +3,20 @@
 // Modeling", section 2.1: first- and second-order block statistics, covariance
 // approximated as diagonal).
 //
-// HBM-bound: every key is read once with 16-byte loads. A warp load covers
-// RPL = 512 / row_bytes consecutive rows (lane = (row rp, 16-byte column chunk cl));
-// a chunk of R such loads (16 rows for bf16 d = 128) sits in registers, its mean
-// and sum of squared deviations are taken two-pass there and reduced over the rp
-// lanes with xor shuffles. Chunks are combined by exact moment merging of
-// (n, mean, M2): inside a warp in registers (Chan et al.'s pairwise update), across
-// the warps that share a block through shared memory (total mean first, then
-// M2 = sum of M2_p + n_p (mean_p - mean)^2). CTAs are persistent and walk tiles of 8 warps'
-// worth of chunks; every warp issues the loads of its next chunk before it reduces
-// the current one, so two chunks per warp are in flight.
+// HBM-bound: every key is read from HBM once with 16-byte loads. Two kernels:
+//  - blocks of 64 keys or more (prefill): block_stats_warp_kernel, one warp per
+//    block, two passes (the second from L2), described at the kernel;
+//  - blocks of 16 or 32 keys (a decode cache of many small blocks):
+//    block_stats_kernel, persistent. A warp load covers RPL = 512 / row_bytes
+//    consecutive rows (lane = (row rp, 16-byte column chunk cl)); a chunk of R such
+//    loads (16 rows for bf16 d = 128) sits in registers, its mean and sum of
+//    squared deviations are taken two-pass there and reduced over the rp lanes with
+//    xor shuffles. Chunks are combined by exact moment merging of (n, mean, M2):
+//    inside a warp in registers (Chan et al.'s pairwise update), across the warps
+//    that share a block through shared memory (total mean first, then M2 = sum of
+//    M2_p + n_p (mean_p - mean)^2). CTAs walk tiles of 8 warps' worth of chunks;
+//    every warp issues the loads of its next chunk before it reduces the current
+//    one, so two chunks per warp are in flight.
 #include <algorithm>
 
 #include "kernels.h"
