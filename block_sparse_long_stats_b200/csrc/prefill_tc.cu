@@ -147,12 +147,16 @@ struct Cfg {
 
 // ES: score-ordered traversal with S2O's monotone-gain early stop (sections 2-3).
 // The unit's list (in traversal order) is validated into shared memory first:
-// entries outside [0, i] and repeats are dropped (and reported). After each ranked
-// block the softmax warps take, over the tile's rows, the largest ratio of the
-// block's mass to the accumulated mass (both in the running normalisation); below
-// tau, the tile stops after that block. The MMA thread learns it at p_ready and
-// issues that block's P V as the last product; the producer learns it from
-// decided[] before loading the next V, and waits for the K copy it already started.
+// entries outside [0, i] and repeats are dropped (and reported). After each block
+// every softmax warp posts, by one vote, whether all its rows have the block's mass
+// below tau times the accumulated mass (both in the running normalisation; the
+// largest ratio is below tau exactly when every row's is) before it arrives at
+// p_ready. The MMA thread issues that block's P V and the next S, then takes the
+// maximum of the four: for a ranked block below tau the walk stops (that P V was
+// the last product; the next S is computed and unused), which the softmax warps
+// and the producer learn from decided[] (the producer before loading the next V,
+// waiting for the K copy it already started). The decision stays off the MMA chain
+// and the softmax warps need no barrier of their own per block.
 template <int BLK, bool ES>
 __global__ void __launch_bounds__(kThreads, 2)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
@@ -174,7 +178,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     __shared__ uint64_t info_full[2];
     __shared__ int4 tinfo[2];
     __shared__ int n_list, stop_at;
-    __shared__ float es_max[2][4];
+    __shared__ unsigned es_below[2][4];
     int32_t *list_s = reinterpret_cast<int32_t *>(smem + C::SMEM);          // ES: [nq]
     uint32_t *bits = reinterpret_cast<uint32_t *>(list_s + (ES ? a.nq : 0)); // ES: [nwords]
 
@@ -372,6 +376,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 return true;
             };
             bool stopped = false;
+            int j_prev = -1;                  // ES: the block of tile n - 1
             while (ok) {
                 const bool more = next_tile(j, mask, jb, mb, false);
                 if constexpr (!ES) {
@@ -381,10 +386,6 @@ __global__ void __launch_bounds__(kThreads, 2)
                 }
                 if (!more) break;
                 if (n > 0 && !issue_pv(n - 1)) { ok = false; break; }
-                if (ES && *reinterpret_cast<volatile int *>(&stop_at) <= n - 1) {
-                    stopped = true;   // P(n - 1) V was the last product
-                    break;
-                }
                 const int s = n % ST;
                 if (!mbar_wait(&full_k[s], (n / ST) & 1, a.err)) break;
                 tc_fence_after();
@@ -397,6 +398,24 @@ __global__ void __launch_bounds__(kThreads, 2)
                 }
                 tc_commit(&s_full);
                 tc_commit(&empty_k[s]);
+                if constexpr (ES) {
+                    // S(n) is issued ahead of the decision on tile n - 1, which so stays
+                    // off the MMA chain; if the walk stops, S(n) is computed and unused.
+                    // The softmax warps posted tile n - 1's ratios before p_ready.
+                    if (n > 0) {
+                        const unsigned below = es_below[(n - 1) & 1][0] & es_below[(n - 1) & 1][1] &
+                                               es_below[(n - 1) & 1][2] & es_below[(n - 1) & 1][3];
+                        const bool ranked = !(j_prev < a.n_sink || j_prev > i - a.n_local);
+                        const bool stop = ranked && below != 0u;
+                        if (stop) stop_at = n - 1;
+                        mbar_arrive(&decided[(n - 1) & 1]);
+                        if (stop) {
+                            stopped = true;   // P(n - 1) V was the last product
+                            break;
+                        }
+                    }
+                    j_prev = j;
+                }
                 ++n;
             }
             if (ok && n > 0 && (stopped || issue_pv(n - 1))) tc_commit(&o_done);
@@ -426,6 +445,11 @@ __global__ void __launch_bounds__(kThreads, 2)
                 mb = (uint32_t)ti.w;
             }
             if (!mbar_wait(&s_full, n & 1, a.err)) { ok = false; break; }
+            if constexpr (ES) {
+                // the MMA thread's decision on tile n - 1 (taken after it issued S(n))
+                if (n > 0 && !mbar_wait(&decided[(n - 1) & 1], ((n - 1) >> 1) & 1, a.err)) { ok = false; break; }
+                if (*reinterpret_cast<volatile int *>(&stop_at) <= n - 1) break;   // stopped after n - 1
+            }
             tc_fence_after();
             float x[TK];
 #pragma unroll
@@ -505,27 +529,20 @@ __global__ void __launch_bounds__(kThreads, 2)
             f32x2_split(add_f32x2(add_f32x2(sp[0], sp[1]), add_f32x2(sp[2], sp[3])), rs0, rs1);
             const float rs = rs0 + rs1;
             l = l * alpha + rs;
-            bool stop = false;
             if constexpr (ES) {
-                // largest ratio of this block's mass to the accumulated mass over the
-                // tile's rows; reserved blocks (sink, local) never stop the walk
-                float ratio = (t < a.L && l > 0.f) ? rs / l : 0.f;
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) ratio = fmaxf(ratio, __shfl_xor_sync(0xffffffffu, ratio, o));
-                if (lane == 0) es_max[n & 1][warp] = ratio;
-                named_bar_sync(1, 128);
-                const float rmax = fmaxf(fmaxf(es_max[n & 1][0], es_max[n & 1][1]),
-                                         fmaxf(es_max[n & 1][2], es_max[n & 1][3]));
-                const bool ranked = !(j < a.n_sink || j > i - a.n_local);
-                stop = ranked && rmax < a.tau;
-                if (tid == 0 && stop) stop_at = n;
+                // whether every row of the warp has this block's mass below tau times
+                // the accumulated mass (rs < tau l, the ratio test without a division;
+                // a row past the sequence or with no mass counts as a ratio of 0), for
+                // the MMA thread's decision (reserved blocks, sink and local, never stop
+                // the walk: it checks that)
+                const bool below = (t < a.L && l > 0.f) ? rs < a.tau * l : 0.f < a.tau;
+                const unsigned all_below = __all_sync(0xffffffffu, below) ? 1u : 0u;
+                if (lane == 0) es_below[n & 1][warp] = all_below;
             }
             tc_wait_st();
             tc_fence_before();
             mbar_arrive(&p_ready);
-            if (ES && tid == 0) mbar_arrive(&decided[n & 1]);
             ++n;
-            if (stop) break;
         }
         if (ES && tid == 0) a.processed[((size_t)b * a.Hq + h0) * a.nq + i] = n;
         if (ok && n > 0) ok = mbar_wait(&o_done, 0, a.err);
